@@ -1,0 +1,143 @@
+"""CPU oracle for paged decode -- TEST INFRASTRUCTURE ONLY.
+
+Plain, slow and obviously correct.  Only ``tests/``, ``__graft_entry__.smoke()``
+and ``bench.py``'s CPU-baseline leg may import this package; the product path
+(the ``paged_kv_cache_405_b200`` package and its CUDA library) never does, and
+nothing here imports the product.
+
+Contents
+--------
+* ``paged_attention`` -- fp64 decode attention over the paged pool (C, see
+  ``oracle.c`` for the definition and its citations).
+* ``slot`` -- block-table translation of one token.
+* ``kv_append`` / ``block_copy`` -- the two byte-moving operations, on CPU
+  tensors, as plain indexing.
+* ``Allocator`` (``allocator.py``) -- free pool, refcounts, block tables,
+  sharing and copy-on-write.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import numpy as np
+import torch
+
+from . import build as _build
+from .allocator import INVALID, NO_FREE_BLOCK, OK, Allocator  # noqa: F401
+
+_DT = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(_build.build())
+        lib.oracle_paged_attention.restype = ctypes.c_int
+        lib.oracle_paged_attention.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int]
+        lib.oracle_slot.restype = ctypes.c_int64
+        lib.oracle_slot.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64]
+        lib.oracle_max_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def max_threads() -> int:
+    return _load().oracle_max_threads()
+
+
+def _cpu(t):
+    if isinstance(t, np.ndarray):
+        return torch.from_numpy(np.ascontiguousarray(t))
+    return t.detach().to("cpu").contiguous()
+
+
+def slot(bt_row, block_size: int, t: int) -> int:
+    """Physical slot of token ``t`` given one block-table row."""
+    row = np.ascontiguousarray(np.asarray(bt_row, dtype=np.int32))
+    return int(_load().oracle_slot(row.ctypes.data, block_size, t))
+
+
+def paged_attention(q, k_pool, v_pool, block_tables, context_lens, scale=None,
+                    items=None, threads: int = 1) -> np.ndarray:
+    """fp64 decode attention.
+
+    q ``[S, Hq, D]``; pools ``[NB, Hkv, bs, D]`` (fp32/bf16/f16, same dtype);
+    block_tables int32 ``[S, maxB]``; context_lens ``[S]``.  ``scale`` defaults
+    to 1/sqrt(D).  ``items`` is an optional list of (s, h) pairs; the result is
+    then ``[len(items), D]``, else ``[S, Hq, D]``.
+    """
+    q, k_pool, v_pool = _cpu(q), _cpu(k_pool), _cpu(v_pool)
+    if not (q.dtype == k_pool.dtype == v_pool.dtype) or q.dtype not in _DT:
+        raise TypeError("q and pools must share one of fp32/bf16/f16")
+    S, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if D2 != D or tuple(v_pool.shape) != tuple(k_pool.shape):
+        raise ValueError("shape mismatch")
+    bt = np.ascontiguousarray(np.asarray(block_tables, dtype=np.int32))
+    cl = np.ascontiguousarray(np.asarray(context_lens, dtype=np.int32))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if items is None:
+        ss, hh = np.meshgrid(np.arange(S), np.arange(Hq), indexing="ij")
+        its = np.stack([ss.ravel(), hh.ravel()], 1).astype(np.int32)
+    else:
+        its = np.asarray(items, dtype=np.int32).reshape(-1, 2)
+    its_s = np.ascontiguousarray(its[:, 0])
+    its_h = np.ascontiguousarray(its[:, 1])
+    out = np.zeros((len(its), D), dtype=np.float64)
+    rc = _load().oracle_paged_attention(
+        out.ctypes.data, q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(),
+        bt.ctypes.data, bt.shape[1], cl.ctypes.data, S, Hq, Hkv, D, bs, NB,
+        float(scale), _DT[q.dtype], its_s.ctypes.data, its_h.ctypes.data, len(its), threads)
+    if rc != 0:
+        raise ValueError("oracle_paged_attention: invalid indices (status %d)" % rc)
+    if items is None:
+        return out.reshape(S, Hq, D)
+    return out
+
+
+def kv_append(k_pool: torch.Tensor, v_pool: torch.Tensor, k_new, v_new, slot_mapping) -> None:
+    """Write each new token's K and V (all kv heads) into its slot, in place.
+
+    Token i goes to block ``slot // bs`` at offset ``slot % bs``; a negative
+    slot means "no write" (aiknowledge.cn 2.2.3: the new token lands in the
+    sequence's last block; openeuler.csdn.net explainer 2.2: each step caches
+    one new K/V).  Slots must be distinct.
+    """
+    bs = k_pool.shape[2]
+    sm = np.asarray(slot_mapping, dtype=np.int64)
+    valid = sm[sm >= 0]
+    if len(np.unique(valid)) != len(valid):
+        raise ValueError("duplicate slots")
+    k_new, v_new = _cpu(k_new), _cpu(v_new)
+    for i, sl in enumerate(sm.tolist()):
+        if sl < 0:
+            continue
+        blk, off = divmod(sl, bs)
+        k_pool[blk, :, off, :] = k_new[i]
+        v_pool[blk, :, off, :] = v_new[i]
+
+
+def block_copy(k_pool: torch.Tensor, v_pool: torch.Tensor, pairs) -> None:
+    """Copy whole blocks (all kv heads, all offsets) src -> dst, as if at once.
+
+    Copy-on-write copies only the block being written (openeuler.csdn.net
+    explainer 6.2).  No destination may also be a source.
+    """
+    pr = np.asarray(pairs, dtype=np.int64).reshape(-1, 2)
+    if len(pr) == 0:
+        return
+    src, dst = pr[:, 0].tolist(), pr[:, 1].tolist()
+    if set(src) & set(dst) or len(set(dst)) != len(dst):
+        raise ValueError("overlapping copy pairs")
+    ks = k_pool[src].clone()
+    vs = v_pool[src].clone()
+    k_pool[dst] = ks
+    v_pool[dst] = vs
