@@ -1,0 +1,227 @@
+/*
+ * pagedkv -- paged KV cache decode on B200 (sm_100a): C ABI.
+ *
+ * The KV cache of every running sequence lives in fixed-size blocks of
+ * `block_size` tokens drawn from one shared physical pool; a per-sequence block
+ * table maps logical block j (tokens j*block_size .. (j+1)*block_size-1) to a
+ * physical block.  Sources (web pages, cited by site, title and section):
+ *   [E]  openeuler.csdn.net, PagedAttention explainer: 4.1 fixed-size blocks,
+ *        4.2 block table (logical -> physical), 4.3 on-demand growth,
+ *        6.1 shared prefix, 6.2 copy-on-write.
+ *   [B]  agent.csdn.net, PagedAttention blog: 2.1 blocks of 16 tokens, only the
+ *        last block partly filled; 2.2 copy-on-write for parallel samples and
+ *        beams; 3.1 block-manager sketch (allocate a free block on demand).
+ *   [T]  aiknowledge.cn, "2.2 PagedAttention 与 KV Cache 分页管理": 2.2.2 free
+ *        pool, blocks freed on finish or preemption; 2.2.3 worked example
+ *        (35 tokens -> physical blocks 7, 3, 9) and prefix sharing; 2.2.4 a
+ *        kernel fused over non-contiguous blocks; 2.2.13 pool monitoring.
+ *
+ * Conventions for every call
+ *   - Device pointers are caller-owned device memory, 16-byte aligned; the
+ *     library never allocates device memory (the split-K workspace is passed
+ *     in; query its size first).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Device calls are asynchronous on that stream.
+ *   - Host-side validation happens before any launch; a rejected call returns
+ *     PKV_ERR_INVALID / PKV_ERR_UNSUPPORTED and launches nothing.  A failed
+ *     launch returns PKV_ERR_CUDA.  pkv_last_error() gives a message.
+ *   - Kernels check every index they read from device memory (block ids,
+ *     slots, context lengths).  A bad one is not dereferenced: the kernel
+ *     records a bit in a device error word and carries on with a safe value,
+ *     so the output is then meaningless but no fault occurs.  Read and clear
+ *     the word with pkv_device_error().
+ *   - No C++ exception crosses this boundary.
+ *
+ * Pool layout (K and V pools alike, one array each):
+ *     pool[num_blocks][num_kv_heads][block_size][head_dim], row-major,
+ * so the `block_size x head_dim` tile of one (block, kv head) is contiguous.
+ * Element types: PKV_F32, PKV_BF16, PKV_F16; q, new K/V, pools and the output
+ * of one call share one type.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PKV_OK = 0,
+    PKV_ERR_INVALID = 1,        /* bad argument; nothing was done */
+    PKV_ERR_NO_FREE_BLOCK = 2,  /* allocator: pool exhausted; nothing changed */
+    PKV_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed */
+    PKV_ERR_UNSUPPORTED = 4,    /* valid but not built (e.g. head_dim 96) */
+    PKV_ERR_DEVICE_CHECK = 5    /* pkv_device_error found a recorded bad index */
+} pkv_status;
+
+typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_F16 = 2 } pkv_dtype;
+
+/* Bits of the device error word. */
+#define PKV_DEVERR_BLOCK_ID   1u  /* block id outside [0, num_blocks) */
+#define PKV_DEVERR_SLOT       2u  /* slot outside [0, num_blocks*block_size) */
+#define PKV_DEVERR_CONTEXT    4u  /* context length < 0 or > max_blocks_per_seq*block_size */
+#define PKV_DEVERR_TIMEOUT    8u  /* a bounded wait on an async copy gave up */
+
+/* ------------------------------------------------------------------ device */
+
+/*
+ * pkv_kv_append -- write each new token's K and V into its slot.
+ * [E] 2.2 (each step caches one new K/V), [T] 2.2.3 (the token lands in the
+ * sequence's last block), [E] 4.3 (growth by whole blocks).
+ *   k_new, v_new   [T][num_kv_heads][head_dim]
+ *   k_pool, v_pool [num_blocks][num_kv_heads][block_size][head_dim]
+ *   slot_mapping   int64 [T]; token i goes to block slot/block_size at offset
+ *                  slot%block_size.  slot < 0 = skip the token.  Slots must be
+ *                  distinct (duplicates: unspecified which token wins).
+ * Bit-exact byte copy.  Supported head_dim*elem_size multiple of 16 bytes.
+ */
+pkv_status pkv_kv_append(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                         const int64_t* slot_mapping, int num_tokens, int num_blocks,
+                         int num_kv_heads, int head_dim, int block_size, pkv_dtype dtype,
+                         void* stream);
+
+/*
+ * Bytes of split-K workspace pkv_paged_attention_decode needs.
+ *   max_context_len  upper bound on any context length of the call; the decode
+ *                    call uses max_blocks_per_seq*block_size as that bound.
+ *   partition_size   as in the decode call (0 = library's choice; the size
+ *                    returned then covers whatever the library picks).
+ * Returns 0 when no workspace is needed (every context fits one partition).
+ */
+size_t pkv_attention_workspace_bytes(int num_seqs, int num_q_heads, int head_dim,
+                                     int max_context_len, int partition_size);
+
+/* The partition size (tokens) the decode call will use for these arguments. */
+int pkv_attention_partition_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                 int max_context_len, int partition_size);
+
+/*
+ * pkv_paged_attention_decode -- one query token per sequence attends to its
+ * cached tokens, read block by block through its block table
+ * ([E] 4.2 "the kernel reads KV at block granularity via the block table";
+ *  [T] 2.2.4 fused over non-contiguous blocks).  For sequence s, query head h:
+ *     g   = h / (num_q_heads / num_kv_heads)   (grouped-query attention)
+ *     x_t = scale * q[s,h,:] . K[slot(s,t), g, :],  t < context_lens[s]
+ *     out[s,h,:] = sum_t softmax(x)_t V[slot(s,t), g, :]
+ *     slot(s,t) = block_tables[s][t / block_size] * block_size + t % block_size
+ * No mask; context_lens[s] = 0 gives zeros.  Accumulation is fp32 (online
+ * softmax); the result is rounded once to the element type.
+ *   out, q          [num_seqs][num_q_heads][head_dim]
+ *   block_tables    int32 [num_seqs][max_blocks_per_seq]; entries past a
+ *                   sequence's last block are never read.
+ *   context_lens    int32 [num_seqs], 0 <= len <= max_blocks_per_seq*block_size
+ *   scale           0 -> 1/sqrt(head_dim)
+ *   partition_size  0 -> library's choice; > 0 (multiple of 16) splits every
+ *                   context into partitions of that many tokens that run in
+ *                   parallel, then a reduce kernel merges them.
+ *   workspace       >= pkv_attention_workspace_bytes(...) bytes of device
+ *                   memory, 256-byte aligned; contents need no initialisation.
+ * Supported: head_dim 64 or 128; block_size 16, 32, 64, 128 or 256;
+ * num_blocks*num_kv_heads*block_size < 2^31.  16-bit types with a query group
+ * of 2..16 heads run on tensor cores; other cases on CUDA cores.
+ * Deterministic: the same inputs give bit-identical outputs.
+ */
+pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_pool, const void* v_pool,
+                                      const int32_t* block_tables, int max_blocks_per_seq,
+                                      const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                      int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                      float scale, int partition_size, void* workspace,
+                                      size_t workspace_bytes, pkv_dtype dtype, void* stream);
+
+/*
+ * pkv_block_copy -- copy-on-write support: copy whole blocks (every kv head,
+ * every offset, K and V) from src to dst ([E] 6.2: only the block being
+ * written is copied; the original keeps serving its other users; [B] 2.2).
+ *   pairs  int32 [num_pairs][2] = (src, dst) in device memory.  Destinations
+ *          must be distinct and none may also be a source.
+ * Bit-exact.
+ */
+pkv_status pkv_block_copy(void* k_pool, void* v_pool, const int32_t* pairs, int num_pairs,
+                          int num_blocks, int num_kv_heads, int head_dim, int block_size,
+                          pkv_dtype dtype, void* stream);
+
+/*
+ * Wait for `stream`, then return the device error word (PKV_DEVERR_* bits)
+ * in *code and clear it.  Returns PKV_ERR_DEVICE_CHECK when a bit was set.
+ */
+pkv_status pkv_device_error(void* stream, uint32_t* code);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t pkv_launch_count(void);
+
+/* --------------------------------------------------------- host allocator */
+
+/*
+ * Host block allocator: free pool, per-block reference counts, per-sequence
+ * block tables, shared prefixes, forks and the copy-on-write trigger
+ * ([E] 4.1-4.3, 6.1-6.2; [B] 2.1-2.2, 3.1; [T] 2.2.2-2.2.3, 2.2.13).
+ * The handle is owned by the library; one handle must not be used from two
+ * threads at once.  Every call is all-or-nothing: on any error the state is
+ * unchanged.  Policy: the free pool is a FIFO queue; a new block is taken
+ * from its front only when a sequence's last block is full; freed blocks go
+ * to its back in block-table order.
+ */
+typedef struct pkv_alloc pkv_alloc;
+
+/* free_order: a permutation of 0..num_blocks-1 giving the initial queue, or NULL for 0,1,2,... */
+pkv_alloc* pkv_alloc_create(int num_blocks, int block_size, const int32_t* free_order);
+void pkv_alloc_destroy(pkv_alloc* a);
+
+/* Register an empty sequence. */
+pkv_status pkv_seq_add(pkv_alloc* a, int64_t seq_id);
+
+/*
+ * Point an empty, registered sequence at existing blocks holding its first
+ * `num_tokens` tokens (a shared system prompt: [E] 6.1, [T] 2.2.3).
+ * nblocks must equal ceil(num_tokens/block_size); blocks must be distinct and
+ * currently in use.  Each block's reference count goes up by one.
+ */
+pkv_status pkv_seq_share_prefix(pkv_alloc* a, int64_t seq_id, const int32_t* blocks, int nblocks,
+                                int num_tokens);
+
+/* New sequence `child` sharing every block of `parent` ([B] 2.2). */
+pkv_status pkv_seq_fork(pkv_alloc* a, int64_t parent, int64_t child);
+
+/*
+ * Reserve slots for `ntok` new tokens of a sequence.
+ *   slots_out  int64 [ntok]: the slot of each new token, in order.
+ *   cow_out    int32 [cow_cap][2]: (src, dst) block pairs the caller must copy
+ *              (pkv_block_copy) before writing the new tokens; at most one
+ *              per call, so cow_cap >= 1 suffices.  *n_cow = pairs written.
+ * A fresh block is taken when the last block is full; if the token lands in a
+ * block whose reference count is above one, that block alone is copied to a
+ * fresh block and replaced in this sequence's table ([E] 6.2).
+ * PKV_ERR_NO_FREE_BLOCK if the pool runs out (counted in alloc_failures).
+ */
+pkv_status pkv_seq_append_slots(pkv_alloc* a, int64_t seq_id, int ntok, int64_t* slots_out,
+                                int32_t* cow_out, int cow_cap, int* n_cow);
+
+/* Drop a sequence; blocks whose count reaches zero return to the free pool ([T] 2.2.2). */
+pkv_status pkv_seq_free(pkv_alloc* a, int64_t seq_id);
+
+/*
+ * Copy a sequence's block table into out[cap]; *n = its number of blocks
+ * (PKV_ERR_INVALID if cap < *n, with *n still set), *len_tokens = its length.
+ */
+pkv_status pkv_seq_block_table(const pkv_alloc* a, int64_t seq_id, int32_t* out, int cap, int* n,
+                               int64_t* len_tokens);
+
+/* Pool occupancy and counters for monitoring ([T] 2.2.13). Any pointer may be NULL. */
+pkv_status pkv_alloc_stats(const pkv_alloc* a, int* free_blocks, int* used_blocks,
+                           int64_t* alloc_failures, int64_t* cow_copies);
+
+/* Reference count of a block, or -1 if the id is out of range. */
+int pkv_block_refcount(const pkv_alloc* a, int block);
+
+/* ------------------------------------------------------------------ misc */
+const char* pkv_status_str(pkv_status s);
+/* Message describing the last failed call on this thread ("" if none). */
+const char* pkv_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PAGEDKV_H */

@@ -1,0 +1,10 @@
+"""pagedkv -- paged KV cache decode on B200 (sm_100a).
+
+A thin Python face over ``libpagedkv.so`` (C ABI in ``include/pagedkv.h``):
+``kv_append``, ``paged_attention_decode``, ``block_copy``, the host
+``BlockAllocator``, and ``DecodeSession`` which strings one decode step
+together.  PyTorch supplies device memory and streams only.
+"""
+from .binding import (BlockAllocator, PagedKVError, attention_partition_size,  # noqa: F401
+                      attention_workspace_bytes, block_copy, device_error, kv_append, launch_count,
+                      paged_attention_decode, workspace_for)

@@ -1,0 +1,256 @@
+"""ctypes binding for ``libpagedkv.so`` -- argument marshalling only.
+
+Every function here forwards to the C call of the same name (``pkv_`` prefix
+dropped) declared in ``include/pagedkv.h``; shapes are read off the torch
+tensors, pointers passed as integers, and a non-OK status raises
+``PagedKVError``.  All computation happens in the library's CUDA kernels and
+its C++ allocator.  There is no fallback: if the library is missing, importing
+this module fails; device calls demand CUDA tensors.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
+
+OK, INVALID, NO_FREE_BLOCK, CUDA_ERROR, UNSUPPORTED, DEVICE_CHECK = range(6)
+DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_CONTEXT, DEVERR_TIMEOUT = 1, 2, 4, 8
+_DTYPE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+
+# Every symbol include/pagedkv.h declares.
+EXPORTS = [
+    "pkv_kv_append", "pkv_attention_workspace_bytes", "pkv_attention_partition_size",
+    "pkv_paged_attention_decode", "pkv_block_copy", "pkv_device_error", "pkv_launch_count",
+    "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_add", "pkv_seq_share_prefix", "pkv_seq_fork",
+    "pkv_seq_append_slots", "pkv_seq_free", "pkv_seq_block_table", "pkv_alloc_stats",
+    "pkv_block_refcount", "pkv_status_str", "pkv_last_error",
+]
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__("%s (status %d)" % (msg, status))
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("libpagedkv.so is not built; run `python -m paged_kv_cache_405_b200.build` "
+                          "or __graft_entry__.build()")
+    lib = ctypes.CDLL(LIB_PATH)
+    c_int, c_i64, c_vp, c_sz = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t
+    sig = {
+        "pkv_kv_append": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int, c_vp]),
+        "pkv_attention_workspace_bytes": (c_sz, [c_int, c_int, c_int, c_int, c_int]),
+        "pkv_attention_partition_size": (c_int, [c_int, c_int, c_int, c_int, c_int, c_int]),
+        "pkv_paged_attention_decode": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_vp, c_int, c_int, c_int,
+                                               c_int, c_int, c_int, ctypes.c_float, c_int, c_vp, c_sz, c_int,
+                                               c_vp]),
+        "pkv_block_copy": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int, c_vp]),
+        "pkv_device_error": (c_int, [c_vp, ctypes.POINTER(ctypes.c_uint32)]),
+        "pkv_launch_count": (ctypes.c_uint64, []),
+        "pkv_alloc_create": (c_vp, [c_int, c_int, c_vp]),
+        "pkv_alloc_destroy": (None, [c_vp]),
+        "pkv_seq_add": (c_int, [c_vp, c_i64]),
+        "pkv_seq_share_prefix": (c_int, [c_vp, c_i64, c_vp, c_int, c_int]),
+        "pkv_seq_fork": (c_int, [c_vp, c_i64, c_i64]),
+        "pkv_seq_append_slots": (c_int, [c_vp, c_i64, c_int, c_vp, c_vp, c_int, ctypes.POINTER(c_int)]),
+        "pkv_seq_free": (c_int, [c_vp, c_i64]),
+        "pkv_seq_block_table": (c_int, [c_vp, c_i64, c_vp, c_int, ctypes.POINTER(c_int),
+                                        ctypes.POINTER(c_i64)]),
+        "pkv_alloc_stats": (c_int, [c_vp, ctypes.POINTER(c_int), ctypes.POINTER(c_int),
+                                    ctypes.POINTER(c_i64), ctypes.POINTER(c_i64)]),
+        "pkv_block_refcount": (c_int, [c_vp, c_int]),
+        "pkv_status_str": (ctypes.c_char_p, [c_int]),
+        "pkv_last_error": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+lib = _load()
+
+
+def _check(status: int):
+    if status != OK:
+        raise PagedKVError(status, lib.pkv_last_error().decode() or lib.pkv_status_str(status).decode())
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    return t.data_ptr()
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype not in _DTYPE:
+        raise TypeError("element type must be float32, bfloat16 or float16")
+    return _DTYPE[t.dtype]
+
+
+# ------------------------------------------------------------------ device calls
+def kv_append(k_new, v_new, k_pool, v_pool, slot_mapping, stream=None) -> None:
+    """Write token i's K/V ``[T, Hkv, D]`` into pool slot ``slot_mapping[i]`` (int64; < 0 skips)."""
+    NB, Hkv, bs, D = k_pool.shape
+    T = k_new.shape[0]
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    _check(lib.pkv_kv_append(_dev(k_new, "k_new"), _dev(v_new, "v_new"), _dev(k_pool, "k_pool"),
+                             _dev(v_pool, "v_pool"), _dev(slot_mapping, "slot_mapping"), T, NB, Hkv, D, bs,
+                             _dt(k_pool), _stream(stream)))
+
+
+def attention_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int,
+                              partition_size: int = 0) -> int:
+    return int(lib.pkv_attention_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len,
+                                                 partition_size))
+
+
+def attention_partition_size(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                             partition_size=0) -> int:
+    return int(lib.pkv_attention_partition_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                                max_context_len, partition_size))
+
+
+def workspace_for(q, block_tables, block_size, partition_size=0) -> torch.Tensor:
+    """Allocate (via torch) a workspace big enough for a decode call with these inputs."""
+    S, Hq, D = q.shape
+    n = attention_workspace_bytes(S, Hq, D, block_tables.shape[1] * block_size, partition_size)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+
+
+def paged_attention_decode(out, q, k_pool, v_pool, block_tables, context_lens, scale: float = 0.0,
+                           partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
+                           stream=None) -> torch.Tensor:
+    """Decode attention: ``out[s, h] = softmax(scale q K^T) V`` over ``context_lens[s]`` cached tokens."""
+    S, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    maxB = block_tables.shape[1]
+    if workspace is None:
+        workspace = workspace_for(q, block_tables, bs, partition_size)
+    ws_ptr = _dev(workspace, "workspace")
+    _check(lib.pkv_paged_attention_decode(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
+        _dev(block_tables, "block_tables"), maxB, _dev(context_lens, "context_lens"), S, Hq, Hkv, D, bs, NB,
+        float(scale), int(partition_size), ws_ptr, workspace.numel() * workspace.element_size(), _dt(q),
+        _stream(stream)))
+    return out
+
+
+def block_copy(k_pool, v_pool, pairs, stream=None) -> None:
+    """Copy whole blocks ``pairs[i] = (src, dst)`` (int32 ``[n, 2]`` on the device), K and V."""
+    NB, Hkv, bs, D = k_pool.shape
+    if pairs.dtype != torch.int32:
+        raise TypeError("pairs must be int32")
+    n = pairs.shape[0] if pairs.numel() else 0
+    _check(lib.pkv_block_copy(_dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
+                              _dev(pairs, "pairs") if n else None, n, NB, Hkv, D, bs, _dt(k_pool),
+                              _stream(stream)))
+
+
+def device_error(stream=None) -> int:
+    """Wait for the stream; return and clear the device error word (0 = clean)."""
+    code = ctypes.c_uint32(0)
+    st = lib.pkv_device_error(_stream(stream), ctypes.byref(code))
+    if st not in (OK, DEVICE_CHECK):
+        _check(st)
+    return int(code.value)
+
+
+def launch_count() -> int:
+    return int(lib.pkv_launch_count())
+
+
+# -------------------------------------------------------------- host allocator
+class BlockAllocator:
+    """The library's host block allocator (free pool, refcounts, block tables, COW)."""
+
+    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+        fo = None
+        if free_order is not None:
+            self._fo = np.ascontiguousarray(np.asarray(free_order, dtype=np.int32))
+            fo = self._fo.ctypes.data
+        h = lib.pkv_alloc_create(num_blocks, block_size, fo)
+        if not h:
+            raise PagedKVError(INVALID, lib.pkv_last_error().decode())
+        self._h = ctypes.c_void_p(h)
+        self._slots = np.zeros(64, dtype=np.int64)
+        self._cow = np.zeros(2, dtype=np.int32)
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            lib.pkv_alloc_destroy(h)
+            self._h = None
+
+    def seq_add(self, sid: int) -> int:
+        return lib.pkv_seq_add(self._h, sid)
+
+    def seq_share_prefix(self, sid: int, blocks, ntok: int) -> int:
+        b = np.ascontiguousarray(np.asarray(blocks, dtype=np.int32))
+        return lib.pkv_seq_share_prefix(self._h, sid, b.ctypes.data if len(b) else None, len(b), ntok)
+
+    def seq_fork(self, parent: int, child: int) -> int:
+        return lib.pkv_seq_fork(self._h, parent, child)
+
+    def seq_append_slots(self, sid: int, n: int):
+        """Returns (status, slots list, [(src, dst)] copy-on-write pairs)."""
+        if n > len(self._slots):
+            self._slots = np.zeros(max(n, 2 * len(self._slots)), dtype=np.int64)
+        ncow = ctypes.c_int(0)
+        st = lib.pkv_seq_append_slots(self._h, sid, n, self._slots.ctypes.data, self._cow.ctypes.data, 1,
+                                      ctypes.byref(ncow))
+        if st != OK:
+            return st, [], []
+        pairs = [(int(self._cow[0]), int(self._cow[1]))] if ncow.value else []
+        return st, self._slots[:n].tolist(), pairs
+
+    def seq_free(self, sid: int) -> int:
+        return lib.pkv_seq_free(self._h, sid)
+
+    def seq_block_table(self, sid: int):
+        """Returns (status, block table list, length in tokens)."""
+        n = ctypes.c_int(-1)
+        ln = ctypes.c_int64(0)
+        st = lib.pkv_seq_block_table(self._h, sid, None, 0, ctypes.byref(n), ctypes.byref(ln))
+        if n.value < 0:          # unknown sequence
+            return st, [], 0
+        if n.value == 0:
+            return OK, [], int(ln.value)
+        buf = np.zeros(n.value, dtype=np.int32)
+        st = lib.pkv_seq_block_table(self._h, sid, buf.ctypes.data, n.value, ctypes.byref(n), ctypes.byref(ln))
+        if st != OK:
+            return st, [], 0
+        return st, buf.tolist(), int(ln.value)
+
+    def stats(self) -> dict:
+        f, u = ctypes.c_int(0), ctypes.c_int(0)
+        af, cc = ctypes.c_int64(0), ctypes.c_int64(0)
+        _check(lib.pkv_alloc_stats(self._h, ctypes.byref(f), ctypes.byref(u), ctypes.byref(af), ctypes.byref(cc)))
+        return dict(free_blocks=f.value, used_blocks=u.value, alloc_failures=af.value, cow_copies=cc.value)
+
+    def refcount(self, block: int) -> int:
+        return lib.pkv_block_refcount(self._h, block)

@@ -1,0 +1,45 @@
+"""Build ``libpagedkv.so`` in-tree with nvcc for sm_100a (B200).
+
+The CUDA kernels and the C ABI (``csrc/pagedkv.cu``) and the host allocator
+(``csrc/allocator.cpp``) go into one shared library next to this file, so the
+binary travels with the source tree.
+"""
+import os
+import subprocess
+import sys
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+CSRC = os.path.join(HERE, "csrc")
+LIB = os.path.join(HERE, "libpagedkv.so")
+INCLUDE = os.path.join(os.path.dirname(HERE), "include")
+NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
+
+SOURCES = ["pagedkv.cu", "allocator.cpp"]
+DEPS = SOURCES + ["common.cuh", "attention_common.cuh", "attention_simt.cuh", "attention_mma.cuh",
+                  "kv_append.cuh", "block_copy.cuh", "reduce.cuh"]
+
+FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
+         "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr", "-I", INCLUDE]
+
+
+def _stale() -> bool:
+    if not os.path.exists(LIB):
+        return True
+    t = os.path.getmtime(LIB)
+    srcs = [os.path.join(CSRC, f) for f in DEPS] + [os.path.join(INCLUDE, "pagedkv.h"), __file__]
+    return any(os.path.getmtime(f) > t for f in srcs)
+
+
+def build(force: bool = False, verbose: bool = False) -> str:
+    if not force and not _stale():
+        return LIB
+    tmp = LIB + ".tmp%d" % os.getpid()
+    cmd = [NVCC] + FLAGS + (["-Xptxas", "-v"] if verbose else []) + \
+        [os.path.join(CSRC, f) for f in SOURCES] + ["-o", tmp]
+    subprocess.check_call(cmd)
+    os.replace(tmp, LIB)
+    return LIB
+
+
+if __name__ == "__main__":
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))

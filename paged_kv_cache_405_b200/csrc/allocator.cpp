@@ -1,0 +1,234 @@
+// Host block allocator for the paged KV pool (C ABI in include/pagedkv.h).
+//
+// Free pool, per-block reference counts, per-sequence block tables, shared
+// prefixes, forks and the copy-on-write trigger:
+//   openeuler.csdn.net PagedAttention explainer 4.1-4.3 (fixed blocks, block
+//   table, growth only when the last block is full), 6.1 (shared prefix),
+//   6.2 (copy only the block being written);
+//   agent.csdn.net PagedAttention blog 2.2 (forked samples/beams share blocks),
+//   3.1 (allocate a free block on demand);
+//   aiknowledge.cn "2.2 PagedAttention 与 KV Cache 分页管理" 2.2.2 (free on
+//   finish/preemption), 2.2.3 (worked example), 2.2.13 (monitoring counters).
+//
+// Every call checks all preconditions and counts the blocks it needs before it
+// changes anything, so a failing call leaves the state untouched.
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+#include <deque>
+#include <string>
+#include <unordered_map>
+#include <vector>
+
+#include "../../include/pagedkv.h"
+
+namespace pkv_host {
+void set_error(const std::string& msg);
+}
+
+struct pkv_alloc {
+    struct Seq {
+        std::vector<int32_t> table;  // logical block -> physical block
+        int64_t len = 0;             // tokens cached
+    };
+    int num_blocks = 0;
+    int block_size = 0;
+    std::deque<int32_t> free_q;
+    std::vector<int32_t> ref;
+    std::unordered_map<int64_t, Seq> seqs;
+    int64_t alloc_failures = 0;
+    int64_t cow_copies = 0;
+
+    int32_t pop_free() {
+        int32_t b = free_q.front();
+        free_q.pop_front();
+        return b;
+    }
+};
+
+using pkv_host::set_error;
+
+static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+extern "C" {
+
+pkv_alloc* pkv_alloc_create(int num_blocks, int block_size, const int32_t* free_order) {
+    if (num_blocks <= 0 || block_size <= 0) {
+        set_error("pkv_alloc_create: num_blocks and block_size must be positive");
+        return nullptr;
+    }
+    pkv_alloc* a = new (std::nothrow) pkv_alloc();
+    if (!a) return nullptr;
+    a->num_blocks = num_blocks;
+    a->block_size = block_size;
+    a->ref.assign(num_blocks, 0);
+    if (free_order) {
+        std::vector<char> seen(num_blocks, 0);
+        for (int i = 0; i < num_blocks; ++i) {
+            int32_t b = free_order[i];
+            if (b < 0 || b >= num_blocks || seen[b]) {
+                set_error("pkv_alloc_create: free_order is not a permutation of the pool");
+                delete a;
+                return nullptr;
+            }
+            seen[b] = 1;
+            a->free_q.push_back(b);
+        }
+    } else {
+        for (int i = 0; i < num_blocks; ++i) a->free_q.push_back(i);
+    }
+    return a;
+}
+
+void pkv_alloc_destroy(pkv_alloc* a) { delete a; }
+
+pkv_status pkv_seq_add(pkv_alloc* a, int64_t seq_id) {
+    if (!a) return PKV_ERR_INVALID;
+    if (a->seqs.count(seq_id)) {
+        set_error("pkv_seq_add: sequence already registered");
+        return PKV_ERR_INVALID;
+    }
+    a->seqs.emplace(seq_id, pkv_alloc::Seq());
+    return PKV_OK;
+}
+
+pkv_status pkv_seq_share_prefix(pkv_alloc* a, int64_t seq_id, const int32_t* blocks, int nblocks,
+                                int num_tokens) {
+    if (!a) return PKV_ERR_INVALID;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end() || it->second.len != 0 || !it->second.table.empty()) {
+        set_error("pkv_seq_share_prefix: sequence must be registered and empty");
+        return PKV_ERR_INVALID;
+    }
+    if (num_tokens < 0 || nblocks != ceil_div(num_tokens, a->block_size) || (nblocks > 0 && !blocks)) {
+        set_error("pkv_seq_share_prefix: nblocks must equal ceil(num_tokens / block_size)");
+        return PKV_ERR_INVALID;
+    }
+    std::vector<int32_t> sorted(blocks, blocks + nblocks);
+    std::sort(sorted.begin(), sorted.end());
+    for (int i = 0; i < nblocks; ++i) {
+        int32_t b = sorted[i];
+        if (b < 0 || b >= a->num_blocks || a->ref[b] == 0 || (i > 0 && sorted[i - 1] == b)) {
+            set_error("pkv_seq_share_prefix: blocks must be distinct and in use");
+            return PKV_ERR_INVALID;
+        }
+    }
+    for (int i = 0; i < nblocks; ++i) a->ref[blocks[i]] += 1;
+    it->second.table.assign(blocks, blocks + nblocks);
+    it->second.len = num_tokens;
+    return PKV_OK;
+}
+
+pkv_status pkv_seq_fork(pkv_alloc* a, int64_t parent, int64_t child) {
+    if (!a) return PKV_ERR_INVALID;
+    auto p = a->seqs.find(parent);
+    if (p == a->seqs.end() || a->seqs.count(child)) {
+        set_error("pkv_seq_fork: parent must exist and child must not");
+        return PKV_ERR_INVALID;
+    }
+    pkv_alloc::Seq c = p->second;
+    for (int32_t b : c.table) a->ref[b] += 1;
+    a->seqs.emplace(child, std::move(c));
+    return PKV_OK;
+}
+
+pkv_status pkv_seq_append_slots(pkv_alloc* a, int64_t seq_id, int ntok, int64_t* slots_out,
+                                int32_t* cow_out, int cow_cap, int* n_cow) {
+    if (!a) return PKV_ERR_INVALID;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end() || ntok < 0 || (ntok > 0 && !slots_out)) {
+        set_error("pkv_seq_append_slots: unknown sequence or bad arguments");
+        return PKV_ERR_INVALID;
+    }
+    pkv_alloc::Seq& s = it->second;
+    const int64_t bs = a->block_size;
+    const int64_t L = s.len;
+    // Only the first new token can land in an existing block (the partly
+    // filled last one); it needs a private copy if that block is shared.
+    bool cow = ntok > 0 && (L % bs) != 0 && a->ref[s.table[L / bs]] > 1;
+    int64_t fresh = ceil_div(L + ntok, bs) - (int64_t)s.table.size();
+    int64_t need = fresh + (cow ? 1 : 0);
+    if (cow && (cow_cap < 1 || !cow_out)) {
+        set_error("pkv_seq_append_slots: a copy-on-write pair is due but cow_cap < 1");
+        return PKV_ERR_INVALID;
+    }
+    if (need > (int64_t)a->free_q.size()) {
+        a->alloc_failures += 1;
+        set_error("pkv_seq_append_slots: free pool exhausted");
+        return PKV_ERR_NO_FREE_BLOCK;
+    }
+    int ncow = 0;
+    for (int64_t t = L; t < L + ntok; ++t) {
+        int64_t j = t / bs;
+        if (j == (int64_t)s.table.size()) {
+            int32_t b = a->pop_free();
+            a->ref[b] = 1;
+            s.table.push_back(b);
+        } else if (a->ref[s.table[j]] > 1) {
+            int32_t src = s.table[j];
+            int32_t dst = a->pop_free();
+            cow_out[2 * ncow] = src;
+            cow_out[2 * ncow + 1] = dst;
+            ++ncow;
+            a->ref[src] -= 1;
+            a->ref[dst] = 1;
+            s.table[j] = dst;
+            a->cow_copies += 1;
+        }
+        slots_out[t - L] = (int64_t)s.table[j] * bs + t % bs;
+    }
+    s.len = L + ntok;
+    if (n_cow) *n_cow = ncow;
+    return PKV_OK;
+}
+
+pkv_status pkv_seq_free(pkv_alloc* a, int64_t seq_id) {
+    if (!a) return PKV_ERR_INVALID;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) {
+        set_error("pkv_seq_free: unknown sequence");
+        return PKV_ERR_INVALID;
+    }
+    for (int32_t b : it->second.table) {
+        if (--a->ref[b] == 0) a->free_q.push_back(b);
+    }
+    a->seqs.erase(it);
+    return PKV_OK;
+}
+
+pkv_status pkv_seq_block_table(const pkv_alloc* a, int64_t seq_id, int32_t* out, int cap, int* n,
+                               int64_t* len_tokens) {
+    if (!a) return PKV_ERR_INVALID;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end()) {
+        set_error("pkv_seq_block_table: unknown sequence");
+        return PKV_ERR_INVALID;
+    }
+    int nb = (int)it->second.table.size();
+    if (n) *n = nb;
+    if (len_tokens) *len_tokens = it->second.len;
+    if (cap < nb || (nb > 0 && !out)) {
+        set_error("pkv_seq_block_table: output capacity too small");
+        return PKV_ERR_INVALID;
+    }
+    if (nb > 0) std::memcpy(out, it->second.table.data(), sizeof(int32_t) * nb);
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_stats(const pkv_alloc* a, int* free_blocks, int* used_blocks,
+                           int64_t* alloc_failures, int64_t* cow_copies) {
+    if (!a) return PKV_ERR_INVALID;
+    int nfree = (int)a->free_q.size();
+    if (free_blocks) *free_blocks = nfree;
+    if (used_blocks) *used_blocks = a->num_blocks - nfree;
+    if (alloc_failures) *alloc_failures = a->alloc_failures;
+    if (cow_copies) *cow_copies = a->cow_copies;
+    return PKV_OK;
+}
+
+int pkv_block_refcount(const pkv_alloc* a, int block) {
+    if (!a || block < 0 || block >= a->num_blocks) return -1;
+    return a->ref[block];
+}
+
+}  // extern "C"

@@ -1,0 +1,368 @@
+// pagedkv C ABI: argument checking, launch configuration and dispatch for the
+// device calls declared in include/pagedkv.h.  One translation unit holds all
+// kernels so that they share the device error word.
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include <cudaTypedefs.h>
+
+#include "../../include/pagedkv.h"
+#include "attention_mma.cuh"
+#include "attention_simt.cuh"
+#include "block_copy.cuh"
+#include "kv_append.cuh"
+#include "reduce.cuh"
+
+namespace pkv_host {
+
+thread_local std::string g_msg;
+std::atomic<uint64_t> g_launches{0};
+
+void set_error(const std::string& msg) { g_msg = msg; }
+
+static pkv_status invalid(const char* msg) {
+    g_msg = msg;
+    return PKV_ERR_INVALID;
+}
+
+static pkv_status cuda_fail(const char* where, cudaError_t e) {
+    g_msg = std::string(where) + ": " + cudaGetErrorString(e);
+    return PKV_ERR_CUDA;
+}
+
+static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+
+static int elem_size(pkv_dtype dt) { return dt == PKV_F32 ? 4 : 2; }
+
+static bool valid_dtype(int dt) { return dt == PKV_F32 || dt == PKV_BF16 || dt == PKV_F16; }
+
+static bool valid_block_size(int bs) { return bs == 16 || bs == 32 || bs == 64 || bs == 128 || bs == 256; }
+
+static int num_sms() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            n = 148;
+    }
+    return n;
+}
+
+// Partition size in tokens.  Explicit sizes are used as given.  The library's
+// own choice splits a context only when it is long: units of at most 512
+// tokens keep per-warp work short enough for the CTA scheduler to balance
+// ragged lengths, and never go below kMinAutoPartition.
+constexpr int kMinAutoPartition = 256;
+
+static int choose_partition(int max_len, int requested) {
+    if (requested > 0) return requested;
+    const int whole = std::max(16, (max_len + 15) / 16 * 16);
+    if (max_len <= 512) return whole;
+    return 512;
+}
+
+static size_t workspace_for(int S, int Hq, int D, int max_len, int P) {
+    const int64_t maxP = (max_len + P - 1) / P;
+    if (maxP <= 1) return 0;
+    return (size_t)S * Hq * maxP * (size_t)(D + 2) * sizeof(float);
+}
+
+// --------------------------------------------------------------- tensor maps
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void* f = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// A pool as a (rows x D) matrix of 16-bit elements; box = 64 elements x 16 rows,
+// 128-byte swizzle.
+static bool make_pool_map(CUtensorMap* map, const void* pool, int64_t rows, int D, pkv_dtype dt) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)pkv::kTileTok};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, dt == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
+                    const_cast<void*>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------ launch helpers
+template <typename Kern>
+static cudaError_t set_smem(Kern k, int bytes) {
+    return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+constexpr int kSimtWarps = 4, kSimtStages = 3;
+constexpr int kMmaWarps = 4, kMmaStages = 3;
+
+template <typename T, int D>
+static cudaError_t launch_simt(const pkv::AttnParams& p, dim3 grid, cudaStream_t st) {
+    using C = pkv::SimtCfg<T, D, kSimtWarps, kSimtStages>;
+    auto k = pkv::paged_attn_simt_kernel<T, D, kSimtWarps, kSimtStages>;
+    static cudaError_t attr = set_smem(k, C::kSmemBytes);
+    if (attr != cudaSuccess) return attr;
+    k<<<grid, kSimtWarps * 32, C::kSmemBytes, st>>>(p);
+    g_launches++;
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+static cudaError_t launch_mma(const pkv::AttnParams& p, dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv,
+                              cudaStream_t st) {
+    using C = pkv::MmaCfg<T, D, kMmaWarps, kMmaStages>;
+    auto k = pkv::paged_attn_mma_kernel<T, D, kMmaWarps, kMmaStages>;
+    static cudaError_t attr = set_smem(k, C::kSmemBytes);
+    if (attr != cudaSuccess) return attr;
+    k<<<grid, kMmaWarps * 32, C::kSmemBytes, st>>>(p, mk, mv);
+    g_launches++;
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+static cudaError_t launch_reduce(const pkv::ReduceParams& r, cudaStream_t st) {
+    const int warps = r.S * r.Hq;
+    const int blocks = (warps + 7) / 8;
+    pkv::splitk_reduce_kernel<T, D><<<blocks, 256, 0, st>>>(r);
+    g_launches++;
+    return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, bool use_mma, const CUtensorMap* mk,
+                                      const CUtensorMap* mv, cudaStream_t st) {
+    cudaError_t e;
+    if (use_mma) {
+        if constexpr (std::is_same<T, float>::value) {
+            return cudaErrorInvalidValue;
+        } else {
+            dim3 grid((p.Hkv + kMmaWarps - 1) / kMmaWarps, p.maxP, p.S);
+            e = D == 64 ? launch_mma<T, 64>(p, grid, *mk, *mv, st) : launch_mma<T, 128>(p, grid, *mk, *mv, st);
+        }
+    } else {
+        dim3 grid((p.Hq + kSimtWarps - 1) / kSimtWarps, p.maxP, p.S);
+        e = D == 64 ? launch_simt<T, 64>(p, grid, st) : launch_simt<T, 128>(p, grid, st);
+    }
+    if (e != cudaSuccess || p.maxP <= 1) return e;
+    pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len};
+    return D == 64 ? launch_reduce<T, 64>(r, st) : launch_reduce<T, 128>(r, st);
+}
+
+}  // namespace pkv_host
+
+using namespace pkv_host;
+
+extern "C" {
+
+const char* pkv_status_str(pkv_status s) {
+    switch (s) {
+        case PKV_OK: return "ok";
+        case PKV_ERR_INVALID: return "invalid argument";
+        case PKV_ERR_NO_FREE_BLOCK: return "no free block";
+        case PKV_ERR_CUDA: return "CUDA error";
+        case PKV_ERR_UNSUPPORTED: return "unsupported configuration";
+        case PKV_ERR_DEVICE_CHECK: return "device-side index check failed";
+    }
+    return "unknown status";
+}
+
+const char* pkv_last_error(void) { return g_msg.c_str(); }
+
+uint64_t pkv_launch_count(void) { return g_launches.load(); }
+
+pkv_status pkv_kv_append(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                         const int64_t* slot_mapping, int num_tokens, int num_blocks, int num_kv_heads,
+                         int head_dim, int block_size, pkv_dtype dtype, void* stream) {
+    if (!valid_dtype(dtype)) return invalid("pkv_kv_append: bad dtype");
+    if (num_tokens < 0 || num_blocks <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
+        return invalid("pkv_kv_append: sizes must be positive");
+    const int row_bytes = head_dim * elem_size(dtype);
+    if (row_bytes % 16 != 0) return invalid("pkv_kv_append: head_dim * element size must be a multiple of 16 bytes");
+    if (num_tokens == 0) return PKV_OK;
+    if (!k_new || !v_new || !k_pool || !v_pool || !slot_mapping)
+        return invalid("pkv_kv_append: null pointer");
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+        return invalid("pkv_kv_append: pointers must be 16-byte aligned (slot_mapping 8-byte)");
+    pkv::AppendParams p;
+    p.k_new = static_cast<const uint4*>(k_new);
+    p.v_new = static_cast<const uint4*>(v_new);
+    p.k_pool = static_cast<uint4*>(k_pool);
+    p.v_pool = static_cast<uint4*>(v_pool);
+    p.slot_mapping = slot_mapping;
+    p.vecs_per_row = row_bytes / 16;
+    p.Hkv = num_kv_heads;
+    p.bs = block_size;
+    p.num_slots = (int64_t)num_blocks * block_size;
+    p.total_vecs = (int64_t)num_tokens * num_kv_heads * p.vecs_per_row;
+    int64_t blocks = (p.total_vecs + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 16;
+    if (blocks > cap) blocks = cap;
+    pkv::kv_append_kernel<<<(unsigned)blocks, 256, 0, (cudaStream_t)stream>>>(p);
+    g_launches++;
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PKV_OK : cuda_fail("pkv_kv_append", e);
+}
+
+size_t pkv_attention_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
+                                     int partition_size) {
+    if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0 || partition_size < 0) return 0;
+    int P = partition_size > 0 ? partition_size : choose_partition(max_context_len, 0);
+    if (partition_size == 0 && P < max_context_len) P = std::min(P, kMinAutoPartition);
+    return workspace_for(num_seqs, num_q_heads, head_dim, max_context_len, P);
+}
+
+int pkv_attention_partition_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
+                                 int partition_size) {
+    (void)num_seqs;
+    (void)num_q_heads;
+    (void)num_kv_heads;
+    (void)head_dim;
+    return choose_partition(max_context_len, partition_size);
+}
+
+pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_pool, const void* v_pool,
+                                      const int32_t* block_tables, int max_blocks_per_seq,
+                                      const int32_t* context_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+                                      int head_dim, int block_size, int num_blocks, float scale, int partition_size,
+                                      void* workspace, size_t workspace_bytes, pkv_dtype dtype, void* stream) {
+    if (!valid_dtype(dtype)) return invalid("pkv_paged_attention_decode: bad dtype");
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+        return invalid("pkv_paged_attention_decode: sizes must be positive");
+    if (num_q_heads % num_kv_heads != 0)
+        return invalid("pkv_paged_attention_decode: num_q_heads must be a multiple of num_kv_heads");
+    if (!valid_block_size(block_size))
+        return invalid("pkv_paged_attention_decode: block_size must be 16, 32, 64, 128 or 256");
+    if (head_dim != 64 && head_dim != 128) {
+        g_msg = "pkv_paged_attention_decode: head_dim must be 64 or 128";
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (partition_size < 0 || partition_size % 16 != 0)
+        return invalid("pkv_paged_attention_decode: partition_size must be 0 or a positive multiple of 16");
+    if (!(std::isfinite(scale)) || scale < 0.f) return invalid("pkv_paged_attention_decode: scale must be >= 0");
+    const int64_t max_len64 = (int64_t)max_blocks_per_seq * block_size;
+    if (max_len64 > (int64_t)1 << 30) return invalid("pkv_paged_attention_decode: max_blocks_per_seq*block_size too large");
+    if ((int64_t)num_blocks * num_kv_heads * block_size >= ((int64_t)1 << 31))
+        return invalid("pkv_paged_attention_decode: pool has 2^31 or more rows");
+    if (num_seqs == 0) return PKV_OK;
+    if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens)
+        return invalid("pkv_paged_attention_decode: null pointer");
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+        return invalid("pkv_paged_attention_decode: pointers must be 16-byte aligned (tables 4-byte)");
+    if (num_seqs > 65535) return invalid("pkv_paged_attention_decode: at most 65535 sequences per call");
+
+    const int max_len = (int)max_len64;
+    const int P = choose_partition(max_len, partition_size);
+    const int64_t maxP = (max_len + P - 1) / P;
+    if (maxP > 65535) return invalid("pkv_paged_attention_decode: too many partitions; raise partition_size");
+    const size_t need = workspace_for(num_seqs, num_q_heads, head_dim, max_len, P);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need) return invalid("pkv_paged_attention_decode: workspace too small");
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+            return invalid("pkv_paged_attention_decode: workspace must be 256-byte aligned");
+    }
+
+    pkv::AttnParams p;
+    p.out = out;
+    p.q = q;
+    p.k_pool = k_pool;
+    p.v_pool = v_pool;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    const size_t n_part = (size_t)num_seqs * num_q_heads * maxP;
+    p.ws_o = need ? static_cast<float*>(workspace) : nullptr;
+    p.ws_ml = need ? static_cast<float*>(workspace) + n_part * head_dim : nullptr;
+    p.S = num_seqs;
+    p.Hq = num_q_heads;
+    p.Hkv = num_kv_heads;
+    p.G = num_q_heads / num_kv_heads;
+    p.bs = block_size;
+    p.NB = num_blocks;
+    p.maxB = max_blocks_per_seq;
+    p.P = P;
+    p.maxP = (int)maxP;
+    p.max_len = max_len;
+    const float sc = scale > 0.f ? scale : 1.f / std::sqrt((float)head_dim);
+    p.scale_log2 = sc * 1.4426950408889634f;
+
+    const bool use_mma = dtype != PKV_F32 && p.G >= 2 && p.G <= 16;
+    CUtensorMap mk, mv;
+    if (use_mma) {
+        const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
+        if (!make_pool_map(&mk, k_pool, rows, head_dim, dtype) || !make_pool_map(&mv, v_pool, rows, head_dim, dtype)) {
+            g_msg = "pkv_paged_attention_decode: cuTensorMapEncodeTiled failed";
+            return PKV_ERR_CUDA;
+        }
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e;
+    switch (dtype) {
+        case PKV_F32: e = dispatch_attention<float>(p, head_dim, false, nullptr, nullptr, st); break;
+        case PKV_BF16: e = dispatch_attention<__nv_bfloat16>(p, head_dim, use_mma, &mk, &mv, st); break;
+        default: e = dispatch_attention<__half>(p, head_dim, use_mma, &mk, &mv, st); break;
+    }
+    return e == cudaSuccess ? PKV_OK : cuda_fail("pkv_paged_attention_decode", e);
+}
+
+pkv_status pkv_block_copy(void* k_pool, void* v_pool, const int32_t* pairs, int num_pairs, int num_blocks,
+                          int num_kv_heads, int head_dim, int block_size, pkv_dtype dtype, void* stream) {
+    if (!valid_dtype(dtype)) return invalid("pkv_block_copy: bad dtype");
+    if (num_pairs < 0 || num_blocks <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
+        return invalid("pkv_block_copy: sizes must be positive");
+    const int64_t block_bytes = (int64_t)num_kv_heads * block_size * head_dim * elem_size(dtype);
+    if (block_bytes % 16 != 0) return invalid("pkv_block_copy: block bytes must be a multiple of 16");
+    if (num_pairs == 0) return PKV_OK;
+    if (!k_pool || !v_pool || !pairs) return invalid("pkv_block_copy: null pointer");
+    if (!aligned16(k_pool) || !aligned16(v_pool) || (reinterpret_cast<uintptr_t>(pairs) & 3u))
+        return invalid("pkv_block_copy: pools must be 16-byte aligned");
+    pkv::CopyParams p;
+    p.k_pool = static_cast<uint4*>(k_pool);
+    p.v_pool = static_cast<uint4*>(v_pool);
+    p.pairs = pairs;
+    p.block_vecs = block_bytes / 16;
+    p.num_blocks = num_blocks;
+    // ~4 vectors of K and of V per thread, at most 64 slices per block.
+    int64_t slices = (p.block_vecs + 1023) / 1024;
+    if (slices > 64) slices = 64;
+    if (num_pairs > 2147483647) return invalid("pkv_block_copy: too many pairs");
+    pkv::block_copy_kernel<<<dim3((unsigned)num_pairs, (unsigned)slices), 256, 0, (cudaStream_t)stream>>>(p);
+    g_launches++;
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PKV_OK : cuda_fail("pkv_block_copy", e);
+}
+
+pkv_status pkv_device_error(void* stream, uint32_t* code) {
+    cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
+    if (e != cudaSuccess) return cuda_fail("pkv_device_error: stream", e);
+    unsigned int v = 0;
+    e = cudaMemcpyFromSymbol(&v, pkv::g_device_error, sizeof v);
+    if (e != cudaSuccess) return cuda_fail("pkv_device_error: read", e);
+    if (v) {
+        unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(pkv::g_device_error, &zero, sizeof zero);
+        if (e != cudaSuccess) return cuda_fail("pkv_device_error: clear", e);
+    }
+    if (code) *code = v;
+    if (v) {
+        g_msg = "device-side index check recorded bits " + std::to_string(v);
+        return PKV_ERR_DEVICE_CHECK;
+    }
+    return PKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+"""The C-ABI library loads and exports every symbol include/pagedkv.h declares;
+host-side validation rejects bad arguments before any launch (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_405_b200 as pkv
+from paged_kv_cache_405_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names |= set(re.findall(r"\b(pkv_\w+)\s*\(", src))
+    return names
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_symbols() == set(binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(binding.LIB_PATH)
+    missing = [n for n in declared_symbols() if not hasattr(lib, n)]
+    assert not missing
+
+
+def test_status_strings():
+    assert binding.lib.pkv_status_str(0) == b"ok"
+    assert binding.lib.pkv_status_str(2) == b"no free block"
+
+
+def test_workspace_size_rules():
+    # fits one partition: no workspace
+    assert pkv.attention_workspace_bytes(4, 4, 64, 512, 0) == 0
+    # forced 512-token partitions of a 100k context (8 seqs x 64 heads x 196 parts x (128+2) floats)
+    assert pkv.attention_workspace_bytes(8, 64, 128, 100_160, 512) == 8 * 64 * 196 * 130 * 4
+    # the library's own choice is covered by the size it reports
+    auto = pkv.attention_partition_size(64, 32, 32, 128, 2048, 0)
+    assert pkv.attention_workspace_bytes(64, 32, 128, 2048, 0) >= \
+        pkv.attention_workspace_bytes(64, 32, 128, 2048, auto)
+
+
+def call_decode(**over):
+    a = dict(out=16, q=16, k=16, v=16, bt=16, maxB=4, cl=16, S=1, Hq=4, Hkv=4, D=64, bs=16, NB=8,
+             scale=0.0, P=0, ws=None, wsb=0, dt=1, stream=None)
+    a.update(over)
+    return binding.lib.pkv_paged_attention_decode(a["out"], a["q"], a["k"], a["v"], a["bt"], a["maxB"],
+                                                  a["cl"], a["S"], a["Hq"], a["Hkv"], a["D"], a["bs"],
+                                                  a["NB"], a["scale"], a["P"], a["ws"], a["wsb"], a["dt"],
+                                                  a["stream"])
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(Hq=6, Hkv=4), binding.INVALID),          # group not integral
+    (dict(bs=24), binding.INVALID),                # unsupported block size
+    (dict(D=96), binding.UNSUPPORTED),
+    (dict(dt=7), binding.INVALID),
+    (dict(P=24), binding.INVALID),                 # not a multiple of 16
+    (dict(q=8), binding.INVALID),                  # misaligned pointer
+    (dict(out=None), binding.INVALID),
+    (dict(maxB=64, P=16), binding.INVALID),        # split needs a workspace
+    (dict(scale=-1.0), binding.INVALID),
+    (dict(S=0, out=None), binding.OK),             # empty batch: nothing to do
+])
+def test_decode_validation(over, status):
+    assert call_decode(**over) == status
+
+
+def test_append_and_copy_validation():
+    lib = binding.lib
+    # head_dim*elem not a multiple of 16 bytes
+    assert lib.pkv_kv_append(16, 16, 16, 16, 16, 1, 4, 1, 6, 16, 1, None) == binding.INVALID
+    assert lib.pkv_kv_append(None, None, None, None, None, 0, 4, 1, 64, 16, 1, None) == binding.OK
+    assert lib.pkv_block_copy(16, 16, 16, -1, 4, 1, 64, 16, 1, None) == binding.INVALID
+    assert lib.pkv_block_copy(None, None, None, 0, 4, 1, 64, 16, 1, None) == binding.OK
+
+
+def test_device_calls_demand_cuda_tensors():
+    import torch
+    k = torch.zeros(4, 1, 16, 64)
+    with pytest.raises(TypeError):
+        pkv.kv_append(k[0], k[0], k, k, torch.zeros(1, dtype=torch.int64))

@@ -1,0 +1,136 @@
+"""Product allocator (C++ in libpagedkv) vs the oracle allocator: bit-exact.
+
+Both get the same seeded operation sequences; statuses, slots, copy-on-write
+pairs, block tables, reference counts and counters must match after every op.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from paged_kv_cache_405_b200 import BlockAllocator
+from oracle.allocator import OK, INVALID, NO_FREE_BLOCK
+
+
+def compare(prod: BlockAllocator, orc: oracle.Allocator, sids):
+    assert prod.stats() == orc.stats()
+    for b in range(orc.num_blocks):
+        assert prod.refcount(b) == orc.refcount(b)
+    for sid in sids:
+        assert prod.seq_block_table(sid) == orc.seq_block_table(sid)
+
+
+def apply(a, op, bs):
+    kind = op[0]
+    if kind == "add":
+        return a.seq_add(op[1])
+    if kind == "append":
+        return a.seq_append_slots(op[1], op[2])
+    if kind == "fork":
+        return a.seq_fork(op[1], op[2])
+    if kind == "share":
+        sid, donor, ntok = op[1], op[2], op[3]
+        st, bt, n = a.seq_block_table(donor)
+        blocks = bt[: -(-ntok // bs)] if st == OK and ntok <= n else [0] * (-(-ntok // bs))
+        return a.seq_share_prefix(sid, blocks, ntok)
+    return a.seq_free(op[1])
+
+
+@pytest.mark.parametrize("seed0", [0, 1000, 2000])
+def test_random_ops_bit_exact(seed0):
+    for seed in range(seed0, seed0 + 700):
+        nb = 4 + seed % 5
+        bs = (1, 2, 4)[seed % 3]
+        order = np.random.default_rng(seed).permutation(nb)
+        prod = BlockAllocator(nb, bs, order)
+        orc = oracle.Allocator(nb, bs, order)
+        for op in synth.random_ops(seed, 10, max_seqs=4, max_append=6):
+            r1 = apply(prod, op, bs)
+            r2 = apply(orc, op, bs)
+            assert r1 == r2, (seed, op, r1, r2)
+            compare(prod, orc, range(4))
+
+
+def test_worked_example_table():
+    order = [7, 3, 9, 12] + [b for b in range(16) if b not in (7, 3, 9, 12)]
+    a = BlockAllocator(16, 16, order)
+    assert a.seq_add(0) == OK
+    st, slots, pairs = a.seq_append_slots(0, 35)
+    assert st == OK and pairs == [] and slots[0] == 112 and slots[34] == 146
+    assert a.seq_block_table(0) == (OK, [7, 3, 9], 35)
+    assert a.seq_append_slots(0, 13)[0] == OK
+    assert a.seq_block_table(0)[1] == [7, 3, 9]
+    st, slots, _ = a.seq_append_slots(0, 1)
+    assert a.seq_block_table(0)[1] == [7, 3, 9, 12] and slots == [12 * 16]
+
+
+def test_exhaustion_leaves_state_unchanged():
+    a = BlockAllocator(3, 4)
+    a.seq_add(1)
+    assert a.seq_append_slots(1, 9)[0] == OK
+    before = (a.stats(), a.seq_block_table(1))
+    st, slots, pairs = a.seq_append_slots(1, 4)
+    assert st == NO_FREE_BLOCK and slots == []
+    after = (a.stats(), a.seq_block_table(1))
+    assert after[1] == before[1]
+    assert after[0]["alloc_failures"] == 1 and after[0]["free_blocks"] == 0
+
+
+def test_invalid_calls():
+    a = BlockAllocator(8, 4)
+    assert a.seq_append_slots(5, 1)[0] == INVALID
+    assert a.seq_free(5) == INVALID
+    assert a.seq_add(1) == OK and a.seq_add(1) == INVALID
+    assert a.seq_fork(1, 1) == INVALID and a.seq_fork(2, 3) == INVALID
+    assert a.seq_share_prefix(1, [0], 2) == INVALID          # block 0 not in use
+    assert a.refcount(-1) == -1 and a.refcount(8) == -1
+    with pytest.raises(Exception):
+        BlockAllocator(4, 4, [0, 1, 1, 2])
+
+
+def test_shared_prefix_refcount():
+    """A 512-token system prompt (32 blocks of 16) shared by 256 sequences."""
+    b = synth.make_batch(synth.shrink(synth.CONFIGS["llama13b_prefix"], D=64, Hq=1, Hkv=1))
+    a = BlockAllocator(b.num_blocks, 16, b.free_order)
+    a.seq_add(-1)
+    a.seq_append_slots(-1, 512)                              # the prompt, written once
+    prefix = a.seq_block_table(-1)[1]
+    assert prefix == b.prefix_blocks.tolist()
+    for s in range(256):
+        a.seq_add(s)
+        assert a.seq_share_prefix(s, prefix, 512) == OK
+    a.seq_free(-1)
+    assert all(a.refcount(x) == 256 for x in prefix)
+    for s in range(256):
+        st, slots, pairs = a.seq_append_slots(s, int(b.lens[s]) - 512)
+        assert st == OK and pairs == []                        # prefix ends on a block boundary
+    for s in range(256):
+        assert a.seq_block_table(s)[1] == b.block_tables[s][b.block_tables[s] >= 0].tolist()
+
+
+def test_generator_handout_matches_allocator():
+    b = synth.make_batch(synth.shrink(synth.CONFIGS["llama7b"], D=64, Hq=1, Hkv=1))
+    a = BlockAllocator(b.num_blocks, b.shape.bs, b.free_order)
+    for s in range(b.shape.S):
+        a.seq_add(s)
+        assert a.seq_append_slots(s, int(b.lens[s]))[0] == OK
+        assert a.seq_block_table(s)[1] == b.block_tables[s][b.block_tables[s] >= 0].tolist()
+
+
+def test_beam_fork_copy_on_write():
+    """Four beams share a 100k-token parent (bs 64, last block holds 32 tokens)."""
+    bs = 64
+    nb = 1563 * 2 + 8
+    a = BlockAllocator(nb, bs)
+    o = oracle.Allocator(nb, bs)
+    for x in (a, o):
+        x.seq_add(0)
+        assert x.seq_append_slots(0, 100_000)[0] == OK
+        for c in (1, 2, 3):
+            x.seq_fork(0, c)
+    res = [[x.seq_append_slots(beam, 1) for beam in (1, 2, 3, 0)] for x in (a, o)]
+    assert res[0] == res[1]
+    assert [len(r[2]) for r in res[0]] == [1, 1, 1, 0]
+    last = a.seq_block_table(0)[1][-1]
+    assert all(r[2][0][0] == last for r in res[0][:3])
+    assert a.stats() == o.stats() and a.stats()["cow_copies"] == 3
