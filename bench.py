@@ -1,0 +1,554 @@
+#!/usr/bin/env python
+"""Paged KV cache decode benchmark (one JSON line on rank 0).
+
+A step is one decode step of one layer for a whole batch: every sequence gets
+the slot of its next token from the block allocator (copy-on-write pairs
+where a shared, partly filled block is written), the copies are made
+(block_copy), the new K/V are written (kv_append) and every query attends to
+its cached tokens through its block table (paged_attention_decode).  Lengths
+grow by one token per step.
+
+value  -- algorithmic bytes of the step (unique K/V bytes the attention must
+          read, shared blocks counted once, plus q, out, tables, split-K
+          workspace, appended and copied bytes) / device time, inputs already
+          resident in HBM (the step's plan is made on the host beforehand).
+e2e    -- the same metric through DecodeSession.step: allocator on the host,
+          step inputs copied in from pinned host memory, output copied back.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+       [--impl ours|reference].  Under torchrun each rank runs its own
+replica (own pool, own sequences; no collective on the data path): weak
+scaling.  ``--impl reference`` times the CPU oracle instead (rank 0 only).
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "paged decode attention HBM GB/s (% of B200 peak) and seq-steps/s per layer"
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------- accounting
+def attention_bytes(bt: np.ndarray, lens: np.ndarray, Hq: int, Hkv: int, D: int, bs: int, elt: int,
+                    P: int) -> dict:
+    """Algorithmic bytes of one decode-attention call.
+
+    K/V: every physical (block, kv head) tile covered by some context counts
+    once, with the number of tokens covered (a shared prefix is read once by
+    the algorithm's definition of "unique"); plus q and out, the block-table
+    entries and context lengths read, and the split-K partials written and
+    read back.
+    """
+    S = len(lens)
+    covered = {}
+    for s in range(S):
+        L = int(lens[s])
+        nb = -(-L // bs)
+        row = bt[s, :nb]
+        for j in range(nb):
+            c = min(bs, L - j * bs)
+            b = int(row[j])
+            if covered.get(b, 0) < c:
+                covered[b] = c
+    tok = sum(covered.values())
+    kv = 2 * Hkv * D * elt * tok
+    logical = 2 * Hkv * D * elt * int(lens.sum())
+    qo = 2 * S * Hq * D * elt
+    tables = 4 * int(sum(-(-int(L) // bs) for L in lens)) + 4 * S
+    nparts = [-(-int(L) // P) for L in lens]
+    ws = sum(2 * n * Hq * (D + 2) * 4 for n in nparts if n > 1)
+    return dict(kv=kv, logical_kv=logical, total=kv + qo + tables + ws, ws=ws)
+
+
+def append_bytes(T, Hkv, D, elt):
+    return 2 * 2 * T * Hkv * D * elt + 8 * T
+
+
+def copy_bytes(n_pairs, Hkv, bs, D, elt):
+    return 2 * 2 * n_pairs * Hkv * bs * D * elt
+
+
+# ------------------------------------------------------------------- workload
+class Workload:
+    """A batch laid out in the pool plus the session that drives its steps."""
+
+    def __init__(self, shape, seed, device, partition_size):
+        import paged_kv_cache_405_b200 as pkv
+        self.shape = shape
+        self.batch = synth.make_batch(shape, device=device, seed=seed)
+        b = self.batch
+        self.P = partition_size or shape.partition_size
+        self.session = pkv.DecodeSession(b.k_pool, b.v_pool, shape.Hq, b.max_blocks, free_order=b.free_order,
+                                         partition_size=self.P, max_batch=shape.S)
+        ss = self.session
+        if shape.prefix:
+            ss.add(-1, shape.prefix)                       # the prompt, stored once
+            prefix, _ = ss.table(-1)
+        for s in range(shape.S):
+            if shape.prefix:
+                ss.add(s, int(b.lens[s]) - shape.prefix, shared_prefix=prefix, prefix_tokens=shape.prefix)
+            else:
+                ss.add(s, int(b.lens[s]))
+            t, _ = ss.table(s)
+            exp = b.block_tables[s][b.block_tables[s] >= 0].tolist()
+            if t != exp:
+                raise RuntimeError("allocator disagrees with the batch layout for seq %d" % s)
+        if shape.prefix:
+            ss.free(-1)
+        self.parents = list(range(shape.S))
+        self.elt = b.k_pool.element_size()
+        self.eff_P = pkv.attention_partition_size(shape.S, shape.Hq, shape.Hkv, shape.D,
+                                                  b.max_blocks * shape.bs, self.P)
+        self.next_child = shape.S
+
+    def plan(self):
+        """Host work of one step; returns (plan, children written)."""
+        sh, ss = self.shape, self.session
+        children = []
+        if sh.beams:
+            for p in self.parents:
+                for _ in range(sh.beams - 1):
+                    ss.fork(p, self.next_child)
+                    children.append(self.next_child)
+                    self.next_child += 1
+        # children write first (each copies the shared last block); the parent
+        # is then the block's only user and writes in place.
+        write = []
+        for i, p in enumerate(self.parents):
+            write += children[i * (sh.beams - 1):(i + 1) * (sh.beams - 1)] if sh.beams else []
+            write.append(p)
+        plan = ss.plan(self.parents, write)
+        for c in children:
+            ss.free(c)
+        return plan
+
+    def step_bytes(self, plan):
+        sh = self.shape
+        a = attention_bytes(plan.block_tables, plan.lens, sh.Hq, sh.Hkv, sh.D, sh.bs, self.elt, self.eff_P)
+        total = a["total"] + append_bytes(len(plan.slot_mapping), sh.Hkv, sh.D, self.elt) + \
+            copy_bytes(len(plan.cow_pairs), sh.Hkv, sh.bs, sh.D, self.elt)
+        return total, a
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ------------------------------------------------------------- profiles data
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "paged_kv_cache_405_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(open(os.path.join(csrc, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(config):
+    """DRAM bytes per decode call from the committed ncu summary, if it was
+    taken on the current kernel sources."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = kernel_source_hash()
+    for line in open(path):
+        f = line.split()
+        if len(f) >= 3 and not line.startswith("#") and f[0] == config and f[1] == src:
+            return float(f[2])
+    return None
+
+
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        return float(json.load(open(path))["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------- CPU oracle leg
+def oracle_sample(batch, budget_s, threads):
+    """Time the CPU oracle on whole sequences of the batch until ~budget_s of
+    work; returns (KV GB/s, seq-steps/s, description)."""
+    import oracle
+    S, Hq = batch.shape.S, batch.shape.Hq
+    q = batch.q.cpu()
+    k = batch.k_pool.cpu()
+    v = batch.v_pool.cpu()
+    elt = k.element_size()
+    bytes_done, secs, seqs, heads = 0, 0.0, 0, 0
+    order = np.random.default_rng(0).permutation(S)
+    for s in order:
+        L = int(batch.lens[s])
+        items = [(int(s), h) for h in range(Hq)]
+        t0 = time.perf_counter()
+        oracle.paged_attention(q, k, v, batch.block_tables, batch.lens, items=items, threads=threads)
+        secs += time.perf_counter() - t0
+        bytes_done += 2 * L * batch.shape.D * elt * Hq
+        seqs += 1
+        heads += Hq
+        if secs >= budget_s:
+            break
+    desc = "%d of %d sequences (all %d query heads each, %.2f GB of K/V reads), fp64 oracle" % (
+        seqs, S, Hq, bytes_done / 1e9)
+    return bytes_done / secs / 1e9, seqs / secs, desc, secs
+
+
+# ------------------------------------------------------------------- runners
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=300))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def run_ours(args, world, rank, local):
+    import paged_kv_cache_405_b200 as pkv
+    shape = synth.CONFIGS[args.config]
+    dev = torch.device("cuda", local)
+    wl = Workload(shape, shape.seed + rank, dev, args.partition_size)
+    ss = wl.session
+    K, W = args.steps, args.warmup
+    dt = synth.DTYPES[shape.dtype]
+
+    # ---- plan every step on the host first (device-resident inputs)
+    plans, step_bytes, attn_bytes = [], [], []
+    for i in range(W + K):
+        p = wl.plan()
+        plans.append(ss.to_device(p))
+        tb, a = wl.step_bytes(p)
+        step_bytes.append(tb)
+        attn_bytes.append(a)
+    T = len(plans[0].slot_mapping)
+    inputs = []
+    for i in range(W + K):
+        q, _, _ = synth.step_inputs(shape, i, device=dev, seed=shape.seed + rank)
+        kn = synth.randn((T, shape.Hkv, shape.D), torch.Generator(device=dev).manual_seed(7919 * i + rank), dt, dev)
+        vn = synth.randn((T, shape.Hkv, shape.D), torch.Generator(device=dev).manual_seed(7919 * i + rank + 1),
+                         dt, dev)
+        inputs.append((q, kn, vn))
+    out = torch.empty_like(inputs[0][0])
+    stream = torch.cuda.current_stream()
+
+    def run_step(i, ev=None):
+        d = plans[i]
+        q, kn, vn = inputs[i]
+        if d.n_cow:
+            pkv.block_copy(ss.k_pool, ss.v_pool, d.cow_pairs)
+        pkv.kv_append(kn, vn, ss.k_pool, ss.v_pool, d.slot_mapping)
+        if ev is not None:
+            ev[0].record(stream)
+        pkv.paged_attention_decode(out, q, ss.k_pool, ss.v_pool, d.block_tables, d.lens,
+                                   partition_size=wl.P, workspace=ss.workspace)
+        if ev is not None:
+            ev[1].record(stream)
+
+    for i in range(W):
+        run_step(i)
+    torch.cuda.synchronize()
+    if pkv.device_error() != 0:
+        raise RuntimeError("device-side check failed during warm-up")
+    attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    # Clocks are sampled while the GPU is busy: repeat the last warm-up step
+    # (its writes are idempotent) for ~0.5 s right before the timed region.
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run_step(W - 1)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    n_busy = int(min(20000, max(1, args.clock_warm_s * 1e3 / max(e0.elapsed_time(e1), 1e-3))))
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.15)
+    for _ in range(n_busy):
+        run_step(W - 1)
+    launches0 = pkv.launch_count()
+    t0.record(stream)
+    for j in range(K):
+        run_step(W + j, attn_ev[j])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    launches = pkv.launch_count() - launches0
+    clk = clocks.stop()
+    barrier(world)
+    if pkv.device_error() != 0:
+        raise RuntimeError("device-side check failed during the timed steps")
+    ms = t0.elapsed_time(t1)
+    attn_ms = [a.elapsed_time(b) for a, b in attn_ev]
+    ms_max = max_over_ranks(ms, world)
+    timed_bytes = float(sum(step_bytes[W:]))
+    total_bytes = sum_over_ranks(timed_bytes, world)
+    value = total_bytes / (ms_max * 1e-3) / 1e9
+    seq_steps = sum_over_ranks(float(shape.S * K), world) / (ms_max * 1e-3)
+
+    # ---- roofline of the decode-attention call (attention kernel + its split-K reduce)
+    peak, peak_kind = measured_hbm_peak()
+    a_bytes = float(np.mean([a["total"] for a in attn_bytes[W:]]))
+    a_s = float(np.mean(attn_ms)) * 1e-3
+    achieved = a_bytes / a_s / 1e9
+    traffic = recorded_traffic(args.config)
+
+    # ---- end to end through DecodeSession.step (host buffers)
+    e2e = None
+    if not args.no_e2e:
+        wl2 = Workload(shape, shape.seed + rank, dev, args.partition_size)
+        del wl
+        torch.cuda.empty_cache()
+        e2e = run_e2e(args, wl2, world, rank, dev)
+
+    line = None
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": round(ms_max / K, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic (seeded N(0,1) K/V/q; pages' workload shapes)",
+            "config": {"workload": args.config, "description": shape.description, "batch": shape.S,
+                       "q_heads": shape.Hq, "kv_heads": shape.Hkv, "head_dim": shape.D, "block_size": shape.bs,
+                       "partition_size": wl_P(shape, args), "effective_partition_size": eff_P_of(shape, args, plans),
+                       "mean_context": round(float(plans[W].lens.float().mean().item()), 1),
+                       "l2": "inputs larger than L2 (K/V pool %.2f GB per rank)" % (
+                           2 * ss.k_pool.numel() * ss.k_pool.element_size() / 1e9),
+                       "parallelism": "replica per GPU" if world > 1 else "1 GPU"},
+            "pct_of_peak": round(100 * value / peak, 1),
+            "seq_steps_per_s": round(seq_steps, 1),
+            "attention_us": round(a_s * 1e6, 2),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
+                         "kernel": "paged_attention_decode (attention + split-K reduce)",
+                         "algorithmic_bytes": round(a_bytes)},
+            "e2e": e2e,
+            "gpu_launches": int(launches),
+            "clocks": clk,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            v, sps, desc, secs = oracle_sample(host_batch(shape, shape.seed + rank), args.cpu_seconds,
+                                               threads=os.cpu_count())
+            line["cpu_baseline"] = {"value": round(v, 3), "unit": "GB/s", "cores": os.cpu_count(),
+                                    "kind": "oracle", "sample": desc, "seq_steps_per_s": round(sps, 3),
+                                    "seconds": round(secs, 1)}
+    return line
+
+
+def wl_P(shape, args):
+    return args.partition_size or shape.partition_size
+
+
+def eff_P_of(shape, args, plans):
+    import paged_kv_cache_405_b200 as pkv
+    return pkv.attention_partition_size(shape.S, shape.Hq, shape.Hkv, shape.D,
+                                        plans[0].block_tables.shape[1] * shape.bs, wl_P(shape, args))
+
+
+def host_batch(shape, seed):
+    """The same workload generated on the host for the CPU oracle."""
+    return synth.make_batch(shape, device="cpu", seed=seed)
+
+
+def run_e2e(args, wl, world, rank, dev):
+    import paged_kv_cache_405_b200 as pkv
+    shape = wl.shape
+    ss = wl.session
+    K, W = args.steps, args.warmup
+    dt = synth.DTYPES[shape.dtype]
+    T = shape.S * max(1, shape.beams)
+    host_inputs = []
+    for i in range(W + K):
+        g = torch.Generator().manual_seed(104729 * (i + 1) + rank)
+        q = synth.randn((shape.S, shape.Hq, shape.D), g, dt, "cpu").pin_memory()
+        kn = synth.randn((T, shape.Hkv, shape.D), g, dt, "cpu").pin_memory()
+        vn = synth.randn((T, shape.Hkv, shape.D), g, dt, "cpu").pin_memory()
+        host_inputs.append((q, kn, vn))
+    out_host = torch.empty((shape.S, shape.Hq, shape.D), dtype=dt, pin_memory=True)
+    stream = torch.cuda.current_stream()
+    h2d = d2h = 0
+    nbytes = []
+
+    def one(i):
+        nonlocal h2d, d2h
+        q, kn, vn = host_inputs[i]
+        p = wl.plan()
+        tb, _ = wl.step_bytes(p)
+        d = pkv.session.DevicePlan(*(ss._h2d(n, a) for n, a in (("slots", p.slot_mapping), ("cow", p.cow_pairs),
+                                                                 ("lens", p.lens), ("bt", p.block_tables))),
+                                   len(p.cow_pairs))
+        qd = q.to(dev, non_blocking=True)
+        kd = kn.to(dev, non_blocking=True)
+        vd = vn.to(dev, non_blocking=True)
+        out = torch.empty_like(qd)
+        ss.launch(d, qd, kd, vd, out)
+        out_host.copy_(out, non_blocking=True)
+        stream.synchronize()
+        h2d = sum(x.numel() * x.element_size() for x in (q, kn, vn)) + \
+            sum(a.nbytes for a in (p.slot_mapping, p.cow_pairs, p.lens, p.block_tables))
+        d2h = out_host.numel() * out_host.element_size()
+        return tb
+
+    for i in range(W):
+        one(i)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for j in range(K):
+        nbytes.append(one(W + j))
+    t1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), world)
+    tot = sum_over_ranks(float(sum(nbytes)), world)
+    if pkv.device_error() != 0:
+        raise RuntimeError("device-side check failed during the end-to-end steps")
+    return {"value": round(tot / (ms * 1e-3) / 1e9, 1), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms / K, 4),
+            "api": "DecodeSession allocator plan + pinned H2D + block_copy/kv_append/paged_attention_decode + D2H"}
+
+
+def run_reference(args, world, rank):
+    """The CPU oracle as the reference arm: each step is a bounded sample of the workload."""
+    if rank != 0:
+        return None
+    shape = synth.CONFIGS[args.config]
+    batch = synth.make_batch(shape, device="cpu")
+    per = max(0.5, args.reference_step_seconds)
+    for _ in range(args.warmup):
+        oracle_sample(batch, per / 4, threads=os.cpu_count())
+    vals, secs = [], []
+    desc = ""
+    for _ in range(args.steps):
+        v, sps, desc, s = oracle_sample(batch, per, threads=os.cpu_count())
+        vals.append(v)
+        secs.append(s)
+    value = float(np.mean(vals))
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * float(np.mean(secs)), 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (same seeded workload, host copy)",
+        "config": {"workload": args.config, "description": shape.description},
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", default="llama7b", choices=sorted(synth.CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--partition-size", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--reference-step-seconds", type=float, default=3.0)
+    ap.add_argument("--clock-warm-s", type=float, default=0.5,
+                    help="seconds of untimed repeats before the timed region, while clocks are sampled")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, rank, local = dist_setup()
+    if world != args.gpus and rank == 0:
+        print("warning: --gpus %d but WORLD_SIZE %d" % (args.gpus, world), file=sys.stderr)
+    if args.impl == "reference":
+        line = run_reference(args, world, rank)
+    else:
+        line = run_ours(args, world, rank, local)
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -199,6 +199,27 @@ pkv_status pkv_seq_fork(pkv_alloc* a, int64_t parent, int64_t child);
 pkv_status pkv_seq_append_slots(pkv_alloc* a, int64_t seq_id, int ntok, int64_t* slots_out,
                                 int32_t* cow_out, int cow_cap, int* n_cow);
 
+/*
+ * One decode step's host work for many sequences in one call: reserve one
+ * slot for each of seq_ids[0..n-1], in that order, exactly as n calls of
+ * pkv_seq_append_slots(a, seq_ids[i], 1, ...) would.
+ *   slots_out  int64 [n]
+ *   cow_out    int32 [cow_cap][2]; *n_cow = pairs written (at most n).
+ * All-or-nothing: if any sequence fails (unknown id, pool exhausted, cow_cap
+ * too small), nothing changes and *n_cow = 0.
+ */
+pkv_status pkv_seq_append_slots_batch(pkv_alloc* a, const int64_t* seq_ids, int n, int64_t* slots_out,
+                                      int32_t* cow_out, int cow_cap, int* n_cow);
+
+/*
+ * Block tables and lengths of many sequences: row i of out (int32 [n][max_blocks])
+ * gets seq_ids[i]'s table padded with -1, lens_out[i] its length in tokens.
+ * PKV_ERR_INVALID (nothing written) if a sequence is unknown or longer than
+ * max_blocks blocks.
+ */
+pkv_status pkv_seq_block_tables_batch(const pkv_alloc* a, const int64_t* seq_ids, int n, int32_t* out,
+                                      int max_blocks, int32_t* lens_out);
+
 /* Drop a sequence; blocks whose count reaches zero return to the free pool ([T] 2.2.2). */
 pkv_status pkv_seq_free(pkv_alloc* a, int64_t seq_id);
 

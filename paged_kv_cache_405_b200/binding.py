@@ -28,7 +28,7 @@ EXPORTS = [
     "pkv_kv_append", "pkv_attention_workspace_bytes", "pkv_attention_partition_size",
     "pkv_paged_attention_decode", "pkv_block_copy", "pkv_device_error", "pkv_launch_count",
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_add", "pkv_seq_share_prefix", "pkv_seq_fork",
-    "pkv_seq_append_slots", "pkv_seq_free", "pkv_seq_block_table", "pkv_alloc_stats",
+    "pkv_seq_append_slots", "pkv_seq_append_slots_batch", "pkv_seq_block_tables_batch", "pkv_seq_free", "pkv_seq_block_table", "pkv_alloc_stats",
     "pkv_block_refcount", "pkv_status_str", "pkv_last_error",
 ]
 
@@ -61,6 +61,8 @@ def _load():
         "pkv_seq_share_prefix": (c_int, [c_vp, c_i64, c_vp, c_int, c_int]),
         "pkv_seq_fork": (c_int, [c_vp, c_i64, c_i64]),
         "pkv_seq_append_slots": (c_int, [c_vp, c_i64, c_int, c_vp, c_vp, c_int, ctypes.POINTER(c_int)]),
+        "pkv_seq_append_slots_batch": (c_int, [c_vp, c_vp, c_int, c_vp, c_vp, c_int, ctypes.POINTER(c_int)]),
+        "pkv_seq_block_tables_batch": (c_int, [c_vp, c_vp, c_int, c_vp, c_int, c_vp]),
         "pkv_seq_free": (c_int, [c_vp, c_i64]),
         "pkv_seq_block_table": (c_int, [c_vp, c_i64, c_vp, c_int, ctypes.POINTER(c_int),
                                         ctypes.POINTER(c_i64)]),
@@ -227,6 +229,30 @@ class BlockAllocator:
             return st, [], []
         pairs = [(int(self._cow[0]), int(self._cow[1]))] if ncow.value else []
         return st, self._slots[:n].tolist(), pairs
+
+    def seq_append_slots_batch(self, sids):
+        """One slot for each sequence id, in order.  Returns (status, slots int64 array,
+        cow pairs int32 [n, 2] array)."""
+        ids = np.ascontiguousarray(np.asarray(sids, dtype=np.int64))
+        n = len(ids)
+        slots = np.zeros(n, dtype=np.int64)
+        cow = np.zeros((max(n, 1), 2), dtype=np.int32)
+        ncow = ctypes.c_int(0)
+        st = lib.pkv_seq_append_slots_batch(self._h, ids.ctypes.data, n, slots.ctypes.data, cow.ctypes.data,
+                                            max(n, 1), ctypes.byref(ncow))
+        if st != OK:
+            return st, slots[:0], cow[:0]
+        return st, slots, cow[:ncow.value]
+
+    def seq_block_tables_batch(self, sids, max_blocks: int, out=None, lens_out=None):
+        """Block tables (int32 [n, max_blocks], -1 padded) and lengths (int32 [n])."""
+        ids = np.ascontiguousarray(np.asarray(sids, dtype=np.int64))
+        n = len(ids)
+        out = np.empty((n, max_blocks), dtype=np.int32) if out is None else out
+        lens_out = np.empty(n, dtype=np.int32) if lens_out is None else lens_out
+        st = lib.pkv_seq_block_tables_batch(self._h, ids.ctypes.data, n, out.ctypes.data, max_blocks,
+                                            lens_out.ctypes.data)
+        return st, out, lens_out
 
     def seq_free(self, sid: int) -> int:
         return lib.pkv_seq_free(self._h, sid)

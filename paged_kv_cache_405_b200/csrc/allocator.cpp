@@ -13,6 +13,7 @@
 // Every call checks all preconditions and counts the blocks it needs before it
 // changes anything, so a failing call leaves the state untouched.
 #include <algorithm>
+#include <climits>
 #include <cstdint>
 #include <cstring>
 #include <deque>
@@ -179,6 +180,87 @@ pkv_status pkv_seq_append_slots(pkv_alloc* a, int64_t seq_id, int ntok, int64_t*
     }
     s.len = L + ntok;
     if (n_cow) *n_cow = ncow;
+    return PKV_OK;
+}
+
+pkv_status pkv_seq_append_slots_batch(pkv_alloc* a, const int64_t* seq_ids, int n, int64_t* slots_out,
+                                      int32_t* cow_out, int cow_cap, int* n_cow) {
+    if (n_cow) *n_cow = 0;
+    if (!a || n < 0 || (n > 0 && (!seq_ids || !slots_out))) {
+        set_error("pkv_seq_append_slots_batch: bad arguments");
+        return PKV_ERR_INVALID;
+    }
+    // Dry run: count the blocks and copy pairs the whole batch needs.  A
+    // sequence listed twice sees its own first reservation (its length grows).
+    std::unordered_map<int64_t, int64_t> extra;      // tokens already reserved in this call
+    std::unordered_map<int32_t, int32_t> ref_drop;   // copies already made of a shared block
+    int64_t need = 0, ncow = 0;
+    for (int i = 0; i < n; ++i) {
+        auto it = a->seqs.find(seq_ids[i]);
+        if (it == a->seqs.end()) {
+            set_error("pkv_seq_append_slots_batch: unknown sequence");
+            return PKV_ERR_INVALID;
+        }
+        const pkv_alloc::Seq& s = it->second;
+        const int64_t bs = a->block_size;
+        int64_t& k = extra[seq_ids[i]];
+        const int64_t L = s.len + k;
+        if (L % bs == 0) {
+            need += 1;
+        } else if (k == 0) {
+            const int32_t b = s.table[L / bs];
+            int32_t& drop = ref_drop[b];
+            if (a->ref[b] - drop > 1) {  // still shared when this sequence writes
+                need += 1;
+                ncow += 1;
+                drop += 1;
+            }
+        }
+        k += 1;
+    }
+    if (ncow > 0 && (!cow_out || cow_cap < ncow)) {
+        set_error("pkv_seq_append_slots_batch: cow_cap too small");
+        return PKV_ERR_INVALID;
+    }
+    if (need > (int64_t)a->free_q.size()) {
+        a->alloc_failures += 1;
+        set_error("pkv_seq_append_slots_batch: free pool exhausted");
+        return PKV_ERR_NO_FREE_BLOCK;
+    }
+    int done = 0;
+    for (int i = 0; i < n; ++i) {
+        int c = 0;
+        pkv_status st = pkv_seq_append_slots(a, seq_ids[i], 1, slots_out + i, cow_out ? cow_out + 2 * done : nullptr,
+                                             cow_cap - done, &c);
+        if (st != PKV_OK) return st;  // unreachable: the dry run checked every condition
+        done += c;
+    }
+    if (n_cow) *n_cow = done;
+    return PKV_OK;
+}
+
+pkv_status pkv_seq_block_tables_batch(const pkv_alloc* a, const int64_t* seq_ids, int n, int32_t* out,
+                                      int max_blocks, int32_t* lens_out) {
+    if (!a || n < 0 || max_blocks < 0 || (n > 0 && (!seq_ids || !out || !lens_out))) {
+        set_error("pkv_seq_block_tables_batch: bad arguments");
+        return PKV_ERR_INVALID;
+    }
+    std::vector<const pkv_alloc::Seq*> rows(n);
+    for (int i = 0; i < n; ++i) {
+        auto it = a->seqs.find(seq_ids[i]);
+        if (it == a->seqs.end() || (int64_t)it->second.table.size() > max_blocks || it->second.len > INT32_MAX) {
+            set_error("pkv_seq_block_tables_batch: unknown sequence or table longer than max_blocks");
+            return PKV_ERR_INVALID;
+        }
+        rows[i] = &it->second;
+    }
+    for (int i = 0; i < n; ++i) {
+        int32_t* row = out + (int64_t)i * max_blocks;
+        const auto& t = rows[i]->table;
+        std::copy(t.begin(), t.end(), row);
+        std::fill(row + t.size(), row + max_blocks, -1);
+        lens_out[i] = (int32_t)rows[i]->len;
+    }
     return PKV_OK;
 }
 

@@ -1,0 +1,158 @@
+"""One decode step over a batch of sequences, end to end.
+
+A step, per the pages' description of paged decoding: each running sequence
+asks the block allocator for the slot of its next token (a fresh block only
+when its last block is full; a private copy of a shared, partly filled last
+block first -- openeuler.csdn.net PagedAttention explainer 4.3 and 6.2;
+aiknowledge.cn "2.2 PagedAttention 与 KV Cache 分页管理" 2.2.3); the copies
+are made (``block_copy``); the new K/V are written (``kv_append``); and every
+sequence's query attends to its cached tokens through its block table
+(``paged_attention_decode``).
+
+``DecodeSession`` keeps the host side (allocator, block tables as a pinned
+host array) and issues the three device calls on one stream.  ``plan`` does
+the host work of a step and returns its device inputs; ``launch`` issues the
+kernels for a planned step; ``step`` does both, with the host<->device copies a
+serving loop makes every step (inputs in, attention output out).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import binding as B
+
+
+@dataclass
+class StepPlan:
+    seq_ids: list              # sequences whose query attends this step (rows of q/out)
+    slot_mapping: np.ndarray   # int64 [T] slots of the tokens written this step
+    cow_pairs: np.ndarray      # int32 [n, 2] blocks to copy before writing
+    lens: np.ndarray           # int32 [len(seq_ids)] context after the write
+    block_tables: np.ndarray   # int32 [len(seq_ids), max_blocks]
+
+
+@dataclass
+class DevicePlan:
+    slot_mapping: torch.Tensor
+    cow_pairs: torch.Tensor
+    lens: torch.Tensor
+    block_tables: torch.Tensor
+    n_cow: int
+
+
+class DecodeSession:
+    def __init__(self, k_pool: torch.Tensor, v_pool: torch.Tensor, num_q_heads: int, max_blocks_per_seq: int,
+                 free_order=None, partition_size: int = 0, max_batch: int = 0):
+        self.k_pool, self.v_pool = k_pool, v_pool
+        self.num_blocks, self.num_kv_heads, self.block_size, self.head_dim = k_pool.shape
+        self.num_q_heads = num_q_heads
+        self.max_blocks = max_blocks_per_seq
+        self.partition_size = partition_size
+        self.alloc = B.BlockAllocator(self.num_blocks, self.block_size, free_order)
+        self.device = k_pool.device
+        n = max(max_batch, 1)
+        self.workspace = torch.empty(
+            max(256, B.attention_workspace_bytes(n, num_q_heads, self.head_dim,
+                                                 max_blocks_per_seq * self.block_size, partition_size)),
+            dtype=torch.uint8, device=self.device)
+        self._pinned = {}
+
+    # ------------------------------------------------------------ host side
+    def add(self, sid: int, num_tokens: int = 0, shared_prefix: Optional[Sequence[int]] = None,
+            prefix_tokens: int = 0) -> list:
+        """Register a sequence; map a shared prefix onto existing blocks, then
+        reserve slots for ``num_tokens`` more tokens.  Returns their slots."""
+        self._ok(self.alloc.seq_add(sid))
+        if shared_prefix is not None:
+            self._ok(self.alloc.seq_share_prefix(sid, shared_prefix, prefix_tokens))
+        if num_tokens:
+            st, slots, cow = self.alloc.seq_append_slots(sid, num_tokens)
+            self._ok(st)
+            assert not cow
+            return slots
+        return []
+
+    def fork(self, parent: int, child: int):
+        self._ok(self.alloc.seq_fork(parent, child))
+
+    def free(self, sid: int):
+        self._ok(self.alloc.seq_free(sid))
+
+    def table(self, sid: int):
+        st, bt, n = self.alloc.seq_block_table(sid)
+        self._ok(st)
+        return bt, n
+
+    @staticmethod
+    def _ok(st):
+        if st != B.OK:
+            raise B.PagedKVError(st, B.lib.pkv_last_error().decode())
+
+    def plan(self, attend: Sequence[int], write: Optional[Sequence[int]] = None) -> StepPlan:
+        """Reserve one new slot for every sequence in ``write`` (default: ``attend``),
+        collect copy-on-write pairs, and snapshot the tables of ``attend``."""
+        write = list(attend if write is None else write)
+        st, slots, pairs = self.alloc.seq_append_slots_batch(write)
+        self._ok(st)
+        st, bt, lens = self.alloc.seq_block_tables_batch(list(attend), self.max_blocks)
+        self._ok(st)
+        return StepPlan(list(attend), slots, pairs.reshape(-1, 2), lens, bt)
+
+    def to_device(self, p: StepPlan, non_blocking: bool = False) -> DevicePlan:
+        dev = self.device
+
+        def up(a):
+            return torch.from_numpy(np.ascontiguousarray(a)).to(dev, non_blocking=non_blocking)
+        return DevicePlan(up(p.slot_mapping), up(p.cow_pairs) if len(p.cow_pairs) else
+                          torch.zeros((0, 2), dtype=torch.int32, device=dev),
+                          up(p.lens), up(p.block_tables), len(p.cow_pairs))
+
+    # ---------------------------------------------------------- device side
+    def launch(self, d: DevicePlan, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+               out: torch.Tensor, stream=None):
+        """block_copy (if any pair) -> kv_append -> paged_attention_decode."""
+        if d.n_cow:
+            B.block_copy(self.k_pool, self.v_pool, d.cow_pairs, stream=stream)
+        B.kv_append(k_new, v_new, self.k_pool, self.v_pool, d.slot_mapping, stream=stream)
+        B.paged_attention_decode(out, q, self.k_pool, self.v_pool, d.block_tables, d.lens,
+                                 partition_size=self.partition_size, workspace=self.workspace, stream=stream)
+        return out
+
+    def _pin(self, name, like: torch.Tensor):
+        t = self._pinned.get(name)
+        if t is None or t.shape != like.shape or t.dtype != like.dtype:
+            t = torch.empty(like.shape, dtype=like.dtype, pin_memory=True)
+            self._pinned[name] = t
+        return t
+
+    def step(self, q_host: torch.Tensor, k_new_host: torch.Tensor, v_new_host: torch.Tensor,
+             attend: Sequence[int], out_host: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """A full step from host buffers: plan, copy inputs in, run, copy the output back."""
+        p = self.plan(attend)
+        s = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(s):
+            d = DevicePlan(*(self._h2d(n, a) for n, a in (("slots", p.slot_mapping), ("cow", p.cow_pairs),
+                                                          ("lens", p.lens), ("bt", p.block_tables))),
+                           len(p.cow_pairs))
+            q = q_host.to(self.device, non_blocking=True)
+            kn = k_new_host.to(self.device, non_blocking=True)
+            vn = v_new_host.to(self.device, non_blocking=True)
+            out = torch.empty_like(q)
+            self.launch(d, q, kn, vn, out, stream=s)
+            if out_host is None:
+                out_host = self._pin("out", out)
+            out_host.copy_(out, non_blocking=True)
+        s.synchronize()
+        return out_host
+
+    def _h2d(self, name, a: np.ndarray) -> torch.Tensor:
+        src = torch.from_numpy(np.ascontiguousarray(a))
+        if src.numel() == 0:
+            return torch.zeros(a.shape, dtype=src.dtype, device=self.device)
+        pin = self._pin(name, src)
+        pin.copy_(src)
+        return pin.to(self.device, non_blocking=True)

@@ -134,3 +134,36 @@ def test_beam_fork_copy_on_write():
     last = a.seq_block_table(0)[1][-1]
     assert all(r[2][0][0] == last for r in res[0][:3])
     assert a.stats() == o.stats() and a.stats()["cow_copies"] == 3
+
+
+def test_batch_calls_equal_sequential_calls():
+    """The batched step call equals one append call per sequence, in order,
+    including several beams copying one shared partial block."""
+    for seed in range(300):
+        rng = np.random.default_rng(seed)
+        nb, bs = 12 + seed % 7, (2, 4)[seed % 2]
+        a1, a2 = BlockAllocator(nb, bs), BlockAllocator(nb, bs)
+        o = oracle.Allocator(nb, bs)
+        n0 = int(rng.integers(1, 7))
+        for a in (a1, a2, o):
+            a.seq_add(0)
+            a.seq_append_slots(0, n0)
+            for c in (1, 2, 3):
+                a.seq_fork(0, c)
+        ids = [int(x) for x in rng.integers(0, 4, size=int(rng.integers(1, 9)))]
+        st, slots, pairs = a1.seq_append_slots_batch(ids)
+        seq = [a2.seq_append_slots(i, 1) for i in ids]
+        oseq = [o.seq_append_slots(i, 1) for i in ids]
+        assert seq == oseq
+        if all(r[0] == OK for r in seq):
+            assert st == OK
+            assert slots.tolist() == [r[1][0] for r in seq]
+            assert [tuple(p) for p in pairs.tolist()] == [p for r in seq for p in r[2]]
+        else:   # the batch fails as a whole with the first failing status, changing nothing
+            assert st == next(r[0] for r in seq if r[0] != OK)
+            assert slots.size == 0 and pairs.size == 0
+        st, bt, lens = a1.seq_block_tables_batch([0, 1, 2, 3], 64)
+        if all(r[0] == OK for r in seq):
+            for i in range(4):
+                t = a2.seq_block_table(i)
+                assert bt[i][bt[i] >= 0].tolist() == t[1] and lens[i] == t[2]

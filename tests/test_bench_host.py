@@ -1,0 +1,71 @@
+"""Host-side logic of bench.py on CPU tensors: allocator replay of each
+workload's layout, step planning (beams, copy-on-write), byte accounting, and
+the multi-rank reductions over a 2-rank gloo group."""
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+import oracle
+import synth
+
+
+@pytest.mark.parametrize("cfg,over", [
+    ("tiny", {}),
+    ("llama7b", dict(S=6, Hq=2, Hkv=2, D=64)),
+    ("llama13b_prefix", dict(S=5, Hq=1, Hkv=1, D=64)),
+    ("llama3_gqa_bs32", dict(S=3, Hq=4, Hkv=1, D=64, len_fixed=300)),
+    ("longctx_beam", dict(S=2, Hq=2, Hkv=1, D=64, len_fixed=1000)),
+])
+def test_workload_steps_on_cpu(cfg, over):
+    sh = synth.shrink(synth.CONFIGS[cfg], **over)
+    wl = bench.Workload(sh, sh.seed, "cpu", 0)
+    orc = oracle.Allocator(wl.batch.num_blocks, sh.bs, wl.batch.free_order)
+    lens0 = wl.batch.lens.copy()
+    for i in range(3):
+        p = wl.plan()
+        assert p.lens.tolist() == (lens0 + i + 1).tolist()
+        T = sh.S * max(1, sh.beams)
+        assert len(p.slot_mapping) == T and len(set(p.slot_mapping.tolist())) == T
+        if sh.beams:
+            assert len(p.cow_pairs) == sh.S * (sh.beams - 1) or i > 0
+        else:
+            assert len(p.cow_pairs) == 0
+        total, a = wl.step_bytes(p)
+        assert a["kv"] <= a["logical_kv"] and total > a["kv"]
+    del orc
+
+
+def test_attention_bytes_counts_shared_blocks_once():
+    bt = np.array([[5, 6, 1], [5, 6, 2]], np.int32)
+    lens = np.array([40, 35])
+    a = bench.attention_bytes(bt, lens, Hq=1, Hkv=1, D=8, bs=16, elt=2, P=512)
+    # blocks 5, 6 once (32 tokens) + block 1 (8 tokens) + block 2 (3 tokens)
+    assert a["kv"] == 2 * 8 * 2 * (32 + 8 + 3)
+    assert a["logical_kv"] == 2 * 8 * 2 * 75 and a["ws"] == 0
+
+
+def _ranks(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    torch.distributed.init_process_group("gloo", rank=rank, world_size=world)
+    mx = bench.max_over_ranks(float(rank + 1), world)
+    sm = bench.sum_over_ranks(float(rank + 1), world)
+    bench.barrier(world)
+    q.put((rank, mx, sm))
+    torch.distributed.destroy_process_group()
+
+
+def test_rank_reductions_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + os.getpid() % 1000
+    ps = [ctx.Process(target=_ranks, args=(r, 2, port, q)) for r in range(2)]
+    for p in ps:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in ps)
+    for p in ps:
+        p.join(timeout=60)
+    assert res == [(0, 2.0, 3.0), (1, 2.0, 3.0)]
