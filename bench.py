@@ -53,23 +53,21 @@ def attention_bytes(bt: np.ndarray, lens: np.ndarray, Hq: int, Hkv: int, D: int,
     read back.
     """
     S = len(lens)
-    covered = {}
-    for s in range(S):
-        L = int(lens[s])
-        nb = -(-L // bs)
-        row = bt[s, :nb]
-        for j in range(nb):
-            c = min(bs, L - j * bs)
-            b = int(row[j])
-            if covered.get(b, 0) < c:
-                covered[b] = c
-    tok = sum(covered.values())
+    lens = np.asarray(lens, dtype=np.int64)
+    nb = -(-lens // bs)
+    j = np.arange(bt.shape[1])[None, :]
+    used = j < nb[:, None]
+    cov = np.clip(lens[:, None] - j * bs, 0, bs)[used]       # tokens covered in each used entry
+    blk = bt[used].astype(np.int64)
+    best = np.zeros(int(blk.max()) + 1 if blk.size else 1, dtype=np.int64)
+    np.maximum.at(best, blk, cov)                            # a block shared by several contexts counts once
+    tok = int(best.sum())
     kv = 2 * Hkv * D * elt * tok
     logical = 2 * Hkv * D * elt * int(lens.sum())
     qo = 2 * S * Hq * D * elt
-    tables = 4 * int(sum(-(-int(L) // bs) for L in lens)) + 4 * S
-    nparts = [-(-int(L) // P) for L in lens]
-    ws = sum(2 * n * Hq * (D + 2) * 4 for n in nparts if n > 1)
+    tables = 4 * int(nb.sum()) + 4 * S
+    nparts = -(-lens // P)
+    ws = int((2 * nparts * Hq * (D + 2) * 4)[nparts > 1].sum())
     return dict(kv=kv, logical_kv=logical, total=kv + qo + tables + ws, ws=ws)
 
 
@@ -232,21 +230,22 @@ def oracle_sample(batch, budget_s, threads):
     k = batch.k_pool.cpu()
     v = batch.v_pool.cpu()
     elt = k.element_size()
-    bytes_done, secs, seqs, heads = 0, 0.0, 0, 0
+    bytes_done, secs, seqs, passes = 0, 0.0, 0, 0
     order = np.random.default_rng(0).permutation(S)
-    for s in order:
-        L = int(batch.lens[s])
-        items = [(int(s), h) for h in range(Hq)]
-        t0 = time.perf_counter()
-        oracle.paged_attention(q, k, v, batch.block_tables, batch.lens, items=items, threads=threads)
-        secs += time.perf_counter() - t0
-        bytes_done += 2 * L * batch.shape.D * elt * Hq
-        seqs += 1
-        heads += Hq
-        if secs >= budget_s:
-            break
-    desc = "%d of %d sequences (all %d query heads each, %.2f GB of K/V reads), fp64 oracle" % (
-        seqs, S, Hq, bytes_done / 1e9)
+    while secs < budget_s:
+        for s in order:
+            L = int(batch.lens[s])
+            items = [(int(s), h) for h in range(Hq)]
+            t0 = time.perf_counter()
+            oracle.paged_attention(q, k, v, batch.block_tables, batch.lens, items=items, threads=threads)
+            secs += time.perf_counter() - t0
+            bytes_done += 2 * L * batch.shape.D * elt * Hq
+            seqs += 1
+            if secs >= budget_s:
+                break
+        passes += 1
+    desc = "%d sequence-steps over %d pass(es) of the %d-sequence batch (every query head; %.2f GB of K/V " \
+        "reads), fp64 oracle, %d threads" % (seqs, passes, S, bytes_done / 1e9, threads)
     return bytes_done / secs / 1e9, seqs / secs, desc, secs
 
 
@@ -451,13 +450,14 @@ def run_e2e(args, wl, world, rank, dev):
     out_host = torch.empty((shape.S, shape.Hq, shape.D), dtype=dt, pin_memory=True)
     stream = torch.cuda.current_stream()
     h2d = d2h = 0
-    nbytes = []
+
+    plans = []
 
     def one(i):
         nonlocal h2d, d2h
         q, kn, vn = host_inputs[i]
         p = wl.plan()
-        tb, _ = wl.step_bytes(p)
+        plans.append(p)
         d = pkv.session.DevicePlan(*(ss._h2d(n, a) for n, a in (("slots", p.slot_mapping), ("cow", p.cow_pairs),
                                                                  ("lens", p.lens), ("bt", p.block_tables))),
                                    len(p.cow_pairs))
@@ -471,7 +471,6 @@ def run_e2e(args, wl, world, rank, dev):
         h2d = sum(x.numel() * x.element_size() for x in (q, kn, vn)) + \
             sum(a.nbytes for a in (p.slot_mapping, p.cow_pairs, p.lens, p.block_tables))
         d2h = out_host.numel() * out_host.element_size()
-        return tb
 
     for i in range(W):
         one(i)
@@ -480,10 +479,11 @@ def run_e2e(args, wl, world, rank, dev):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
     for j in range(K):
-        nbytes.append(one(W + j))
+        one(W + j)
     t1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1), world)
+    nbytes = [wl.step_bytes(p)[0] for p in plans[W:]]
     tot = sum_over_ranks(float(sum(nbytes)), world)
     if pkv.device_error() != 0:
         raise RuntimeError("device-side check failed during the end-to-end steps")
