@@ -132,6 +132,40 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_po
                                       size_t workspace_bytes, pkv_dtype dtype, void* stream);
 
 /*
+ * pkv_paged_attention_decode_static -- the same decode attention, for callers
+ * that cannot allocate device memory.  The pages have no counterpart to this
+ * call; it exists for integration only.
+ *
+ * Some callers cannot call cudaMalloc or hand in a workspace: a host process
+ * whose memory allocator owns all device memory and forbids side
+ * allocations, a plug-in limited to the buffers it is given, or a step loop
+ * that must not hit a synchronising allocation.  This call takes its split-K
+ * scratch from a buffer built into the library instead: 64 MiB of device
+ * memory, one per GPU that loads the library, held until the process exits.
+ * Arguments and results are those of pkv_paged_attention_decode without the
+ * workspace pair; the caller still passes every input and output.
+ *   - Size limit: a call whose split-K partials would need more than 64 MiB
+ *     (num_seqs * num_q_heads * ceil(max_blocks_per_seq*block_size /
+ *     partition) * (head_dim + 2) * 4 bytes) is rejected with
+ *     PKV_ERR_INVALID and a message; nothing is launched.
+ *   - Set-up: the first call on each device looks up the buffer's device
+ *     address (a CUDA runtime query made with that device current).  Make
+ *     that first call before any stream capture.  Calls run on the device
+ *     that is current when they are made.
+ *   - Sharing: every call on a device uses the same buffer, and it keeps
+ *     whatever the last call left in it.  Nothing in it needs to start at
+ *     zero.  Calls that overlap on the GPU (different streams, no ordering
+ *     between them) race on the buffer and their results are undefined;
+ *     order them on one stream or with events.
+ *   - The call itself allocates nothing.
+ */
+pkv_status pkv_paged_attention_decode_static(void* out, const void* q, const void* k_pool, const void* v_pool,
+                                             const int32_t* block_tables, int max_blocks_per_seq,
+                                             const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                             int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                             float scale, int partition_size, pkv_dtype dtype, void* stream);
+
+/*
  * pkv_block_copy -- copy-on-write support: copy whole blocks (every kv head,
  * every offset, K and V) from src to dst ([E] 6.2: only the block being
  * written is copied; the original keeps serving its other users; [B] 2.2).

@@ -7,5 +7,5 @@ together.  PyTorch supplies device memory and streams only.
 """
 from .binding import (BlockAllocator, PagedKVError, attention_partition_size,  # noqa: F401
                       attention_workspace_bytes, block_copy, device_error, kv_append, launch_count,
-                      paged_attention_decode, workspace_for)
+                      paged_attention_decode, paged_attention_decode_static, workspace_for)
 from .session import DecodeSession, DevicePlan, StepPlan  # noqa: F401,E402

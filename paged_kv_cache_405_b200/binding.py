@@ -26,7 +26,7 @@ _DTYPE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 # Every symbol include/pagedkv.h declares.
 EXPORTS = [
     "pkv_kv_append", "pkv_attention_workspace_bytes", "pkv_attention_partition_size",
-    "pkv_paged_attention_decode", "pkv_block_copy", "pkv_device_error", "pkv_launch_count",
+    "pkv_paged_attention_decode", "pkv_paged_attention_decode_static", "pkv_block_copy", "pkv_device_error", "pkv_launch_count",
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_add", "pkv_seq_share_prefix", "pkv_seq_fork",
     "pkv_seq_append_slots", "pkv_seq_append_slots_batch", "pkv_seq_block_tables_batch", "pkv_seq_free", "pkv_seq_block_table", "pkv_alloc_stats",
     "pkv_block_refcount", "pkv_status_str", "pkv_last_error",
@@ -52,6 +52,9 @@ def _load():
         "pkv_paged_attention_decode": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_vp, c_int, c_int, c_int,
                                                c_int, c_int, c_int, ctypes.c_float, c_int, c_vp, c_sz, c_int,
                                                c_vp]),
+        "pkv_paged_attention_decode_static": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_vp, c_int, c_int,
+                                                      c_int, c_int, c_int, c_int, ctypes.c_float, c_int, c_int,
+                                                      c_vp]),
         "pkv_block_copy": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int, c_vp]),
         "pkv_device_error": (c_int, [c_vp, ctypes.POINTER(ctypes.c_uint32)]),
         "pkv_launch_count": (ctypes.c_uint64, []),
@@ -157,6 +160,23 @@ def paged_attention_decode(out, q, k_pool, v_pool, block_tables, context_lens, s
         _dev(block_tables, "block_tables"), maxB, _dev(context_lens, "context_lens"), S, Hq, Hkv, D, bs, NB,
         float(scale), int(partition_size), ws_ptr, workspace.numel() * workspace.element_size(), _dt(q),
         _stream(stream)))
+    return out
+
+
+def paged_attention_decode_static(out, q, k_pool, v_pool, block_tables, context_lens, scale: float = 0.0,
+                                  partition_size: int = 0, stream=None) -> torch.Tensor:
+    """Decode attention that allocates nothing: the split-K scratch is a fixed
+    64 MiB buffer inside the library (one per GPU), for callers that cannot
+    allocate device memory.  Calls on one device share that buffer, so calls
+    that overlap on the GPU must not be issued; oversized calls raise."""
+    S, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    _check(lib.pkv_paged_attention_decode_static(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
+        _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"), S, Hq, Hkv,
+        D, bs, NB, float(scale), int(partition_size), _dt(q), _stream(stream)))
     return out
 
 

@@ -366,3 +366,75 @@ pkv_status pkv_device_error(void* stream, uint32_t* code) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode attention with built-in scratch, for callers that cannot allocate.
+//
+// Some callers have no way to hand us device memory for the split-K
+// workspace: code that runs where cudaMalloc is off limits (a host process
+// whose allocator owns all device memory and forbids side allocations, a
+// plug-in that may only use what it is given, code that must not reach a
+// synchronising allocation in the middle of a step).  For them this entry
+// point takes the partials from a fixed buffer compiled into this library.
+//
+// The buffer is one file-scope device array of kStaticScratchBytes per GPU,
+// held by every GPU that loads this library until the process exits.  Its
+// device address is looked up once per device (cudaGetSymbolAddress, with
+// that device current) on the first call made on that device; the host-side
+// name of the array is not a device address and is never handed to a kernel.
+// ---------------------------------------------------------------------------
+namespace pkv_host {
+
+constexpr size_t kStaticScratchBytes = size_t(64) << 20;  // 64 MiB per GPU
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+static void* g_static_scratch_ptr[kMaxDevices];
+static std::mutex g_static_scratch_mu;
+
+static cudaError_t static_scratch(void** ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_static_scratch_mu);
+    if (!g_static_scratch_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess) return e;
+        g_static_scratch_ptr[dev] = p;
+    }
+    *ptr = g_static_scratch_ptr[dev];
+    return cudaSuccess;
+}
+
+}  // namespace pkv_host
+
+extern "C" pkv_status pkv_paged_attention_decode_static(void* out, const void* q, const void* k_pool,
+                                                        const void* v_pool, const int32_t* block_tables,
+                                                        int max_blocks_per_seq, const int32_t* context_lens,
+                                                        int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                                        int block_size, int num_blocks, float scale,
+                                                        int partition_size, pkv_dtype dtype, void* stream) {
+    using namespace pkv_host;
+    if (max_blocks_per_seq > 0 && block_size > 0 && num_seqs > 0 && num_q_heads > 0 && head_dim > 0 &&
+        partition_size >= 0 && (int64_t)max_blocks_per_seq * block_size <= ((int64_t)1 << 30)) {
+        const int max_len = max_blocks_per_seq * block_size;
+        const int P = choose_partition(max_len, partition_size);
+        const size_t need = P > 0 ? workspace_for(num_seqs, num_q_heads, head_dim, max_len, P) : 0;
+        if (need > kStaticScratchBytes) {
+            g_msg = "pkv_paged_attention_decode_static: this call needs " + std::to_string(need) +
+                    " bytes of split-K scratch but the built-in buffer holds " +
+                    std::to_string(kStaticScratchBytes) +
+                    "; use a larger partition_size, fewer sequences, or pkv_paged_attention_decode with a "
+                    "caller-provided workspace";
+            return PKV_ERR_INVALID;
+        }
+    }
+    void* scratch = nullptr;
+    cudaError_t e = static_scratch(&scratch);
+    if (e != cudaSuccess) return cuda_fail("pkv_paged_attention_decode_static: scratch address", e);
+    return pkv_paged_attention_decode(out, q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens,
+                                      num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
+                                      partition_size, scratch, kStaticScratchBytes, dtype, stream);
+}

@@ -88,3 +88,11 @@ def test_device_calls_demand_cuda_tensors():
     k = torch.zeros(4, 1, 16, 64)
     with pytest.raises(TypeError):
         pkv.kv_append(k[0], k[0], k, k, torch.zeros(1, dtype=torch.int64))
+
+
+def test_package_exposes_every_binding_call():
+    import inspect
+    public = [n for n, f in inspect.getmembers(binding, inspect.isfunction)
+              if not n.startswith("_") and f.__module__ == binding.__name__]
+    missing = [n for n in public if not hasattr(pkv, n)]
+    assert not missing
