@@ -43,7 +43,7 @@ FALLBACK_HBM_GBS = 6650.0
 
 # ----------------------------------------------------------------- accounting
 def attention_bytes(bt: np.ndarray, lens: np.ndarray, Hq: int, Hkv: int, D: int, bs: int, elt: int,
-                    P: int) -> dict:
+                    P: int, shared=None) -> dict:
     """Algorithmic bytes of one decode-attention call.
 
     K/V: every physical (block, kv head) tile covered by some context counts
@@ -66,8 +66,10 @@ def attention_bytes(bt: np.ndarray, lens: np.ndarray, Hq: int, Hkv: int, D: int,
     logical = 2 * Hkv * D * elt * int(lens.sum())
     qo = 2 * S * Hq * D * elt
     tables = 4 * int(nb.sum()) + 4 * S
-    nparts = -(-lens // P)
-    ws = int((2 * nparts * Hq * (D + 2) * 4)[nparts > 1].sum())
+    sh = np.zeros(S, dtype=np.int64) if shared is None else np.asarray(shared, dtype=np.int64)
+    nparts = -(-sh // P) + -(-(lens - sh) // P)
+    merged = (nparts > 1) | (sh > 0)
+    ws = int((2 * nparts * Hq * (D + 2) * 4)[merged].sum())
     return dict(kv=kv, logical_kv=logical, total=kv + qo + tables + ws, ws=ws)
 
 
@@ -135,7 +137,11 @@ class Workload:
 
     def step_bytes(self, plan):
         sh = self.shape
-        a = attention_bytes(plan.block_tables, plan.lens, sh.Hq, sh.Hkv, sh.D, sh.bs, self.elt, self.eff_P)
+        shared = None
+        if plan.has_groups:   # per-sequence shared length of its group
+            shared = np.repeat(plan.group_shared, np.diff(plan.group_first))
+        a = attention_bytes(plan.block_tables, plan.lens, sh.Hq, sh.Hkv, sh.D, sh.bs, self.elt, self.eff_P,
+                            shared=shared)
         total = a["total"] + append_bytes(len(plan.slot_mapping), sh.Hkv, sh.D, self.elt) + \
             copy_bytes(len(plan.cow_pairs), sh.Hkv, sh.bs, sh.D, self.elt)
         return total, a
@@ -324,8 +330,7 @@ def run_ours(args, world, rank, local):
         pkv.kv_append(kn, vn, ss.k_pool, ss.v_pool, d.slot_mapping)
         if ev is not None:
             ev[0].record(stream)
-        pkv.paged_attention_decode(out, q, ss.k_pool, ss.v_pool, d.block_tables, d.lens,
-                                   partition_size=wl.P, workspace=ss.workspace)
+        ss.attend(d, q, out)
         if ev is not None:
             ev[1].record(stream)
 
@@ -397,7 +402,9 @@ def run_ours(args, world, rank, local):
                        "mean_context": round(float(plans[W].lens.float().mean().item()), 1),
                        "l2": "inputs larger than L2 (K/V pool %.2f GB per rank)" % (
                            2 * ss.k_pool.numel() * ss.k_pool.element_size() / 1e9),
-                       "parallelism": "replica per GPU" if world > 1 else "1 GPU"},
+                       "parallelism": "replica per GPU" if world > 1 else "1 GPU",
+                       "shared_prefix_groups": int((plans[W].group_shared > 0).sum().item())
+                       if plans[W].group_shared is not None else 0},
             "pct_of_peak": round(100 * value / peak, 1),
             "seq_steps_per_s": round(seq_steps, 1),
             "attention_us": round(a_s * 1e6, 2),
@@ -458,9 +465,7 @@ def run_e2e(args, wl, world, rank, dev):
         q, kn, vn = host_inputs[i]
         p = wl.plan()
         plans.append(p)
-        d = pkv.session.DevicePlan(*(ss._h2d(n, a) for n, a in (("slots", p.slot_mapping), ("cow", p.cow_pairs),
-                                                                 ("lens", p.lens), ("bt", p.block_tables))),
-                                   len(p.cow_pairs))
+        d = ss.upload(p)
         qd = q.to(dev, non_blocking=True)
         kd = kn.to(dev, non_blocking=True)
         vd = vn.to(dev, non_blocking=True)
@@ -469,7 +474,8 @@ def run_e2e(args, wl, world, rank, dev):
         out_host.copy_(out, non_blocking=True)
         stream.synchronize()
         h2d = sum(x.numel() * x.element_size() for x in (q, kn, vn)) + \
-            sum(a.nbytes for a in (p.slot_mapping, p.cow_pairs, p.lens, p.block_tables))
+            sum(a.nbytes for a in (p.slot_mapping, p.cow_pairs, p.lens, p.block_tables)) + \
+            (p.group_first.nbytes + p.group_shared.nbytes if p.has_groups else 0)
         d2h = out_host.numel() * out_host.element_size()
 
     for i in range(W):

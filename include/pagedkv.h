@@ -64,6 +64,7 @@ typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_F16 = 2 } pkv_dtype;
 #define PKV_DEVERR_SLOT       2u  /* slot outside [0, num_blocks*block_size) */
 #define PKV_DEVERR_CONTEXT    4u  /* context length < 0 or > max_blocks_per_seq*block_size */
 #define PKV_DEVERR_TIMEOUT    8u  /* a bounded wait on an async copy gave up */
+#define PKV_DEVERR_GROUP     16u  /* a shared-prefix group has more members than max_group_size */
 
 /* ------------------------------------------------------------------ device */
 
@@ -130,6 +131,67 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_po
                                       int num_kv_heads, int head_dim, int block_size, int num_blocks,
                                       float scale, int partition_size, void* workspace,
                                       size_t workspace_bytes, pkv_dtype dtype, void* stream);
+
+/*
+ * pkv_paged_attention_decode_shared -- the same decode attention for a batch
+ * in which runs of consecutive sequences share their first tokens in the same
+ * physical blocks (one system prompt stored once and referenced by every
+ * sequence: [E] 6.1, [T] 2.2.3).  The result equals pkv_paged_attention_decode
+ * on the same inputs (up to fp32 rounding order).  The shared tokens are
+ * attended once per group by a prefix pass in which every warp multiplies 16
+ * queries of the group (sequence x head pairs) by each shared K/V tile on
+ * tensor cores, so a shared tile is read once per 16 queries instead of once
+ * per query; each sequence's own tokens go through the usual split-K pass and
+ * one reduce merges both.
+ *   group_first   device int32 [num_groups + 1], non-decreasing, within
+ *                 [0, num_seqs]: group g is sequences group_first[g] ..
+ *                 group_first[g+1]-1.  Sequences outside every group are
+ *                 handled as in pkv_paged_attention_decode.
+ *   group_shared  device int32 [num_groups]: number of leading tokens the
+ *                 members of group g share, a multiple of block_size, at most
+ *                 every member's context length.  The first
+ *                 group_shared[g]/block_size block-table entries of every
+ *                 member must be those of the group's first sequence (the
+ *                 prefix pass reads the first sequence's).  A value breaking
+ *                 these rules is recorded (PKV_DEVERR_CONTEXT) and the group's
+ *                 members are then handled as non-members.
+ *   max_group_size  host bound on members per group (PKV_DEVERR_GROUP if a
+ *                 group is larger; its extra members get no prefix result).
+ *   workspace     >= pkv_attention_shared_workspace_bytes(...) bytes.
+ * 16-bit element types only (PKV_ERR_UNSUPPORTED for fp32).
+ */
+pkv_status pkv_paged_attention_decode_shared(void* out, const void* q, const void* k_pool, const void* v_pool,
+                                             const int32_t* block_tables, int max_blocks_per_seq,
+                                             const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                             int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                             float scale, int partition_size, const int32_t* group_first,
+                                             const int32_t* group_shared, int num_groups, int max_group_size,
+                                             void* workspace, size_t workspace_bytes, pkv_dtype dtype,
+                                             void* stream);
+
+/* Workspace bytes for pkv_paged_attention_decode_shared (arguments as in
+ * pkv_attention_workspace_bytes; never 0 for num_seqs > 0). */
+size_t pkv_attention_shared_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
+                                            int partition_size);
+
+/*
+ * Host helper: find runs of consecutive sequences whose block tables start
+ * with the same physical blocks (what pkv_paged_attention_decode_shared
+ * needs).  block_tables / context_lens are HOST arrays ([n][max_blocks],
+ * [n]).  A run of at least min_group_size sequences whose tables agree on
+ * their first k >= 1 entries, all full blocks of every member, becomes a
+ * group sharing k*block_size tokens (the greedy run from its first member;
+ * k is the smallest agreement inside the run).  The output partitions
+ * 0..n-1 into runs -- the groups and the gaps between them, the latter with
+ * group_shared = 0 -- in the format pkv_paged_attention_decode_shared takes:
+ * group_first[0..n_groups] (group_first[n_groups] = n) and
+ * group_shared[0..n_groups-1].  max_groups must be >= n (group_first then
+ * needs n + 1 entries).
+ */
+pkv_status pkv_find_shared_prefix_groups(const int32_t* block_tables, const int32_t* context_lens, int n,
+                                         int max_blocks, int block_size, int min_group_size,
+                                         int32_t* group_first, int32_t* group_shared, int max_groups,
+                                         int* n_groups);
 
 /*
  * pkv_paged_attention_decode_static -- the same decode attention, for callers

@@ -26,7 +26,8 @@ _DTYPE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 # Every symbol include/pagedkv.h declares.
 EXPORTS = [
     "pkv_kv_append", "pkv_attention_workspace_bytes", "pkv_attention_partition_size",
-    "pkv_paged_attention_decode", "pkv_paged_attention_decode_static", "pkv_block_copy", "pkv_device_error", "pkv_launch_count",
+    "pkv_paged_attention_decode", "pkv_paged_attention_decode_static", "pkv_paged_attention_decode_shared",
+    "pkv_attention_shared_workspace_bytes", "pkv_find_shared_prefix_groups", "pkv_block_copy", "pkv_device_error", "pkv_launch_count",
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_add", "pkv_seq_share_prefix", "pkv_seq_fork",
     "pkv_seq_append_slots", "pkv_seq_append_slots_batch", "pkv_seq_block_tables_batch", "pkv_seq_free", "pkv_seq_block_table", "pkv_alloc_stats",
     "pkv_block_refcount", "pkv_status_str", "pkv_last_error",
@@ -55,6 +56,12 @@ def _load():
         "pkv_paged_attention_decode_static": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_vp, c_int, c_int,
                                                       c_int, c_int, c_int, c_int, ctypes.c_float, c_int, c_int,
                                                       c_vp]),
+        "pkv_paged_attention_decode_shared": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_vp, c_int, c_int,
+                                                      c_int, c_int, c_int, c_int, ctypes.c_float, c_int, c_vp,
+                                                      c_vp, c_int, c_int, c_vp, c_sz, c_int, c_vp]),
+        "pkv_attention_shared_workspace_bytes": (c_sz, [c_int, c_int, c_int, c_int, c_int]),
+        "pkv_find_shared_prefix_groups": (c_int, [c_vp, c_vp, c_int, c_int, c_int, c_int, c_vp, c_vp, c_int,
+                                                  ctypes.POINTER(c_int)]),
         "pkv_block_copy": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int, c_vp]),
         "pkv_device_error": (c_int, [c_vp, ctypes.POINTER(ctypes.c_uint32)]),
         "pkv_launch_count": (ctypes.c_uint64, []),
@@ -177,6 +184,52 @@ def paged_attention_decode_static(out, q, k_pool, v_pool, block_tables, context_
         _dev(out, "out"), _dev(q, "q"), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
         _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"), S, Hq, Hkv,
         D, bs, NB, float(scale), int(partition_size), _dt(q), _stream(stream)))
+    return out
+
+
+def attention_shared_workspace_bytes(num_seqs: int, num_q_heads: int, head_dim: int, max_context_len: int,
+                                     partition_size: int = 0) -> int:
+    return int(lib.pkv_attention_shared_workspace_bytes(num_seqs, num_q_heads, head_dim, max_context_len,
+                                                        partition_size))
+
+
+def find_shared_prefix_groups(block_tables: np.ndarray, context_lens: np.ndarray, block_size: int,
+                              min_group_size: int = 4):
+    """Runs of consecutive sequences whose tables start with the same blocks.
+    Returns (group_first int32 [n+1], group_shared int32 [n]) -- n runs, gaps
+    between groups included with shared length 0."""
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    lens = np.ascontiguousarray(context_lens, dtype=np.int32)
+    S = bt.shape[0]
+    first = np.zeros(S + 1, dtype=np.int32)
+    shared = np.zeros(max(S, 1), dtype=np.int32)
+    ng = ctypes.c_int(0)
+    _check(lib.pkv_find_shared_prefix_groups(bt.ctypes.data, lens.ctypes.data, S, bt.shape[1], block_size,
+                                             min_group_size, first.ctypes.data, shared.ctypes.data, S,
+                                             ctypes.byref(ng)))
+    n = ng.value
+    return first[:n + 1] if n else first[:0], shared[:n]
+
+
+def paged_attention_decode_shared(out, q, k_pool, v_pool, block_tables, context_lens, group_first, group_shared,
+                                  max_group_size: int, scale: float = 0.0, partition_size: int = 0,
+                                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Decode attention with shared-prefix groups (device int32 group_first [n+1], group_shared [n])."""
+    S, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    n = group_shared.numel()
+    maxB = block_tables.shape[1]
+    if workspace is None:
+        nb = attention_shared_workspace_bytes(S, Hq, D, maxB * bs, partition_size)
+        workspace = torch.empty(max(nb, 256), dtype=torch.uint8, device=q.device)
+    _check(lib.pkv_paged_attention_decode_shared(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
+        _dev(block_tables, "block_tables"), maxB, _dev(context_lens, "context_lens"), S, Hq, Hkv, D, bs, NB,
+        float(scale), int(partition_size), _dev(group_first, "group_first") if n else None,
+        _dev(group_shared, "group_shared") if n else None, n, int(max_group_size), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _dt(q), _stream(stream)))
     return out
 
 

@@ -313,4 +313,60 @@ int pkv_block_refcount(const pkv_alloc* a, int block) {
     return a->ref[block];
 }
 
+pkv_status pkv_find_shared_prefix_groups(const int32_t* block_tables, const int32_t* context_lens, int n,
+                                         int max_blocks, int block_size, int min_group_size,
+                                         int32_t* group_first, int32_t* group_shared, int max_groups,
+                                         int* n_groups) {
+    if (n_groups) *n_groups = 0;
+    if (n < 0 || max_blocks < 0 || block_size <= 0 || !n_groups || max_groups < n ||
+        (n > 0 && (!block_tables || !context_lens || !group_first || !group_shared))) {
+        set_error("pkv_find_shared_prefix_groups: bad arguments (max_groups must be >= n)");
+        return PKV_ERR_INVALID;
+    }
+    if (min_group_size < 2) min_group_size = 2;
+    // The output partitions [0, n) into runs: groups (shared > 0) and the gaps
+    // between them (shared = 0); there are at most n runs.
+    int ng = 0;
+    auto full_blocks = [&](int i) {
+        const int L = context_lens[i] < 0 ? 0 : context_lens[i];
+        return std::min(L / block_size, max_blocks);
+    };
+    int gap_begin = -1;
+    int i = 0;
+    while (i < n) {
+        int k = full_blocks(i);
+        int j = i + 1;
+        const int32_t* lead = block_tables + (int64_t)i * max_blocks;
+        while (j < n && k >= 1) {
+            const int32_t* row = block_tables + (int64_t)j * max_blocks;
+            const int lim = std::min(k, full_blocks(j));
+            int c = 0;
+            while (c < lim && row[c] == lead[c]) ++c;
+            if (c < 1) break;
+            k = c;
+            ++j;
+        }
+        if (j - i >= min_group_size && k >= 1) {
+            if (gap_begin >= 0) {
+                group_first[ng] = gap_begin;
+                group_shared[ng++] = 0;
+                gap_begin = -1;
+            }
+            group_first[ng] = i;
+            group_shared[ng++] = k * block_size;
+            i = j;
+        } else {
+            if (gap_begin < 0) gap_begin = i;
+            ++i;
+        }
+    }
+    if (gap_begin >= 0) {
+        group_first[ng] = gap_begin;
+        group_shared[ng++] = 0;
+    }
+    if (ng > 0) group_first[ng] = n;  // group_first holds max_groups + 1 entries
+    *n_groups = ng;
+    return PKV_OK;
+}
+
 }  // extern "C"

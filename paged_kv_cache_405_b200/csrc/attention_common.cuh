@@ -17,7 +17,50 @@ struct AttnParams {
     float* ws_ml;              // [S][Hq][maxP][2]   (m, l) per partial
     int S, Hq, Hkv, G, bs, NB, maxB, P, maxP, max_len;
     float scale_log2;          // softmax scale * log2(e)
+    // Shared-prefix groups (num_groups = 0: none).  Group i is the sequences
+    // group_first[i] .. group_first[i+1]-1; the first group_shared[i] tokens
+    // of each of them sit in the same physical blocks (those of the group's
+    // first sequence).  The prefix pass covers those tokens once per group.
+    const int32_t* group_first;   // [num_groups + 1]
+    const int32_t* group_shared;  // [num_groups]
+    int num_groups;
+    int max_group_size;           // prefix-pass grid covers groups up to this many sequences
 };
+
+// Which tokens one (sequence, partition) unit covers and where its result goes.
+//   member  -- the sequence belongs to a valid shared-prefix group; its first
+//              `shared` tokens are done by the prefix pass in npre partials
+//              (slots 0..npre-1), its own partitions follow from slot npre.
+//   direct  -- a lone partition of a non-member: write the output itself.
+struct Unit {
+    int L, shared, npre, nsuf, t_begin, t_end, slot;
+    bool member, direct;
+};
+
+__device__ __forceinline__ int find_group(const AttnParams& p, int s) {
+    if (p.num_groups <= 0) return -1;
+    if (s < p.group_first[0] || s >= p.group_first[p.num_groups]) return -1;
+    int lo = 0, hi = p.num_groups;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (p.group_first[mid] <= s) lo = mid;
+        else hi = mid;
+    }
+    return lo;
+}
+
+// Shared length of group gi for a member whose context is L tokens, or -1 if
+// the group's description is unusable for it (then it is treated as a
+// non-member and the bad value recorded).
+__device__ __forceinline__ int group_shared_len(const AttnParams& p, int gi, int L, bool report) {
+    const int sh = p.group_shared[gi];
+    if (sh < 0 || sh % p.bs != 0 || sh > L) {
+        if (report) flag_error(4u /* PKV_DEVERR_CONTEXT */);
+        return -1;
+    }
+    return sh;
+}
+
 
 // Context length of sequence s, clamped into [0, max_len]; an out-of-range
 // value is recorded once per sequence (by the unit that owns partition 0).
@@ -28,6 +71,28 @@ __device__ __forceinline__ int load_context_len(const AttnParams& p, int s, bool
         L = L < 0 ? 0 : p.max_len;
     }
     return L;
+}
+
+__device__ __forceinline__ Unit resolve_unit(const AttnParams& p, int s, int part, bool report) {
+    Unit u;
+    u.L = load_context_len(p, s, report);
+    u.shared = 0;
+    u.member = false;
+    const int gi = find_group(p, s);
+    if (gi >= 0) {
+        const int sh = group_shared_len(p, gi, u.L, report);
+        if (sh > 0) {
+            u.shared = sh;
+            u.member = true;
+        }
+    }
+    u.npre = (u.shared + p.P - 1) / p.P;
+    u.nsuf = (u.L - u.shared + p.P - 1) / p.P;
+    u.t_begin = u.shared + part * p.P;
+    u.t_end = min(u.L, u.t_begin + p.P);
+    u.slot = u.npre + part;
+    u.direct = !u.member && u.nsuf == 1;
+    return u;
 }
 
 // Block-table window held in registers: lane l holds entry (first + base + l)

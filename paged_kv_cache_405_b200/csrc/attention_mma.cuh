@@ -1,24 +1,36 @@
-// Paged decode attention for grouped-query attention on tensor cores: one
-// warp per (sequence, kv head, partition) serves all G query heads of the
-// group (2 <= G <= 16), so each K/V byte is read once for G queries and the
-// work is a real (G x D) . (D x tokens) contraction.
+// Paged decode attention on tensor cores (mma.sync m16n8k16, fp32 accumulate).
 //
-// Per 16-token tile (tokens of one block, via the block table; openeuler.csdn.net
-// PagedAttention explainer 4.2, aiknowledge.cn "2.2 PagedAttention 与 KV
-// Cache 分页管理" 2.2.3-2.2.4):
-//   S = Q K^T   : m16n8k16 MMAs, A = Q (the G heads padded to 16 rows, held in
-//                 registers for the whole unit), B = K^T straight from the
-//                 shared-memory tile (ldmatrix; a K row is a "column" of B).
-//   online softmax on the accumulator fragments (rows = heads; each row is
-//                 spread over the 4 lanes of a quad), log2 domain.
-//   O += P V    : P re-packed from the S accumulators into A fragments without
-//                 touching memory; B = V via ldmatrix.trans.
+// Two kernels share one per-warp core that streams a token range of one kv
+// head through a shared-memory ring and attends 16 query rows to it:
 //
-// Data movement: each stage is one 16-token tile of K and one of V, brought in
-// by 2-D tensor TMA (box 64 elements x 16 rows) with 128-byte swizzle, so the
-// 8 rows an ldmatrix reads fall in 8 different bank groups.  The tensor maps
-// view a pool as a matrix of (num_blocks*Hkv*block_size) rows of D elements;
-// row (block*Hkv + g)*block_size + offset is the token's K (or V) row.
+//  * paged_attn_mma_kernel -- grouped-query attention: one warp per
+//    (sequence, kv head, partition); its 16 rows are the G query heads of the
+//    group (2 <= G <= 16, padded with zero rows), so every K/V byte serves G
+//    queries.
+//  * prefix_attn_mma_kernel -- sequences that share their first tokens (a
+//    system prompt stored once: openeuler.csdn.net PagedAttention explainer
+//    6.1; aiknowledge.cn "2.2 PagedAttention 与 KV Cache 分页管理" 2.2.3):
+//    one warp per (group, 16 query rows, kv head, partition of the shared
+//    tokens); its rows are (sequence, head) pairs of 16 different queries of
+//    the group, all attending to the same shared blocks, so each shared K/V
+//    tile is read once per 16 queries instead of once per query.  Results are
+//    split-K partials merged with each sequence's own partitions by the
+//    reduce kernel.
+//
+// Per 16-token tile (tokens of one block, found through the block table;
+// explainer 4.2, aiknowledge.cn 2.2.3-2.2.4):
+//   S = Q K^T   A = Q rows (registers, loaded once per unit), B = K^T from the
+//               shared-memory tile via ldmatrix (a K row is a column of B).
+//   online softmax on the accumulator fragments (each row is spread over the
+//               4 lanes of a quad), log2 domain.
+//   O += P V    P re-packed from the S accumulators into A fragments in
+//               registers; B = V via ldmatrix.trans.
+//
+// Data movement: each stage is one 16-token tile of K and one of V, loaded by
+// 2-D tensor TMA (box 64 elements x 16 rows) with 128-byte swizzle, so the 8
+// rows one ldmatrix phase reads fall in 8 different bank groups.  The tensor
+// maps view a pool as a (num_blocks*Hkv*block_size) x D matrix; row
+// (block*Hkv + g)*block_size + offset holds a token's K (or V) for kv head g.
 #pragma once
 #include "attention_common.cuh"
 
@@ -34,70 +46,50 @@ struct MmaCfg {
     static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
 };
 
-template <typename T, int D, int WARPS, int STAGES>
-__global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnParams p,
-                                                                    const __grid_constant__ CUtensorMap tmK,
-                                                                    const __grid_constant__ CUtensorMap tmV) {
-    using C = MmaCfg<T, D, WARPS, STAGES>;
-    constexpr int KSTEPS = D / 16;  // MMA k-steps over head_dim
-    constexpr int NT_O = D / 8;     // output n-tiles
-    extern __shared__ __align__(1024) uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+// Attention state of one warp over 16 query rows.  Accumulator element e of
+// output n-tile j is row gid (e < 2) or gid + 8 (e >= 2), column j*8 + 2*tig + (e & 1).
+template <typename T, int D>
+struct MmaAcc {
+    static constexpr int KSTEPS = D / 16;
+    static constexpr int NT_O = D / 8;
+    uint32_t qa[KSTEPS][4];  // Q as A fragments
+    float o[NT_O][4];
+    float m_lo, m_hi, l_lo, l_hi;
 
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const int g = blockIdx.x * WARPS + warp;  // kv head
-    const int part = blockIdx.y;
-    const int s = blockIdx.z;
-    if (g >= p.Hkv) return;
-
-    const int gid = lane >> 2;  // accumulator row (query head within the group) and row+8
-    const int tig = lane & 3;
-    const int G = p.G;
-    const int h0 = g * G;
-
-    const int L = load_context_len(p, s, part == 0 && g == 0 && lane == 0);
-    const int nP = (L + p.P - 1) / p.P;
-    const int t_begin = part * p.P;
-    if (t_begin >= L) {
-        if (part == 0) {  // empty context: zeros for the group's heads
-            T* o = reinterpret_cast<T*>(p.out) + ((int64_t)s * p.Hq + h0) * D;
-            for (int i = lane; i < G * D; i += 32) o[i] = T(0.f);
-        }
-        return;
-    }
-    const int t_end = min(L, t_begin + p.P);
-    const int ntiles = (t_end - t_begin + kTileTok - 1) / kTileTok;
-
-    uint8_t* ring = smem + warp * STAGES * C::kStageBytes;
-    const uint32_t ring_s = smem_u32(ring);
-    const uint32_t bar0 = smem_u32(smem + C::kDataBytes + warp * STAGES * 8);
-    if (lane == 0) {
-        prefetch_tensor_map(&tmK);
-        prefetch_tensor_map(&tmV);
-        for (int i = 0; i < STAGES; ++i) mbar_init(bar0 + 8 * i, 1);
-        fence_barrier_init();
-    }
-    __syncwarp();
-
-    // Q fragments (A operand, rows = heads of the group, zero past G).
-    uint32_t qa[KSTEPS][4];
-    {
-        const T* qb = reinterpret_cast<const T*>(p.q) + ((int64_t)s * p.Hq + h0) * D;
-        const bool r0 = gid < G, r1 = gid + 8 < G;
+    // Row pointers (nullptr = zero row).
+    __device__ __forceinline__ void load_q(const T* row_lo, const T* row_hi, int tig) {
 #pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
             const int c0 = kk * 16 + 2 * tig;
-            qa[kk][0] = r0 ? *reinterpret_cast<const uint32_t*>(qb + gid * D + c0) : 0u;
-            qa[kk][1] = r1 ? *reinterpret_cast<const uint32_t*>(qb + (gid + 8) * D + c0) : 0u;
-            qa[kk][2] = r0 ? *reinterpret_cast<const uint32_t*>(qb + gid * D + c0 + 8) : 0u;
-            qa[kk][3] = r1 ? *reinterpret_cast<const uint32_t*>(qb + (gid + 8) * D + c0 + 8) : 0u;
+            qa[kk][0] = row_lo ? *reinterpret_cast<const uint32_t*>(row_lo + c0) : 0u;
+            qa[kk][1] = row_hi ? *reinterpret_cast<const uint32_t*>(row_hi + c0) : 0u;
+            qa[kk][2] = row_lo ? *reinterpret_cast<const uint32_t*>(row_lo + c0 + 8) : 0u;
+            qa[kk][3] = row_hi ? *reinterpret_cast<const uint32_t*>(row_hi + c0 + 8) : 0u;
         }
+#pragma unroll
+        for (int j = 0; j < NT_O; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+        m_lo = m_hi = -INFINITY;
+        l_lo = l_hi = 0.f;
     }
+};
+
+// Stream tokens [t_begin, t_end) of kv head g (block ids from bt_row) through
+// this warp's ring and accumulate into acc.  Returns false if a wait on a copy
+// timed out (the unit is then abandoned after draining its copies).
+template <typename T, int D, int WARPS, int STAGES>
+__device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                           uint8_t* ring, uint32_t bar0, const int32_t* bt_row, int t_begin,
+                                           int t_end, int g, int lane, MmaAcc<T, D>& acc) {
+    using C = MmaCfg<T, D, WARPS, STAGES>;
+    constexpr int KSTEPS = D / 16;
+    constexpr int NT_O = D / 8;
+    const int tig = lane & 3;
+    const int ntiles = (t_end - t_begin + kTileTok - 1) / kTileTok;
+    const uint32_t ring_s = smem_u32(ring);
 
     const int jb0 = t_begin / p.bs;
     BlockWindow win;
-    win.init(p.block_tables + (int64_t)s * p.maxB, jb0, (t_end - 1) / p.bs - jb0 + 1, lane);
+    win.init(bt_row, jb0, (t_end - 1) / p.bs - jb0 + 1, lane);
 
     auto issue = [&](int i) {
         const int t0 = t_begin + i * kTileTok;
@@ -111,8 +103,8 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnPa
             mbar_arrive_expect_tx(bar, C::kStageBytes);
 #pragma unroll
             for (int hx = 0; hx < D / 64; ++hx) {
-                tma_load_2d(dst + hx * C::kHalfTile, &tmK, hx * 64, row, bar);
-                tma_load_2d(dst + C::kTileBytes + hx * C::kHalfTile, &tmV, hx * 64, row, bar);
+                tma_load_2d(dst + hx * C::kHalfTile, tmK, hx * 64, row, bar);
+                tma_load_2d(dst + C::kTileBytes + hx * C::kHalfTile, tmV, hx * 64, row, bar);
             }
         }
     };
@@ -120,30 +112,25 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnPa
     const int npre = ntiles < STAGES ? ntiles : STAGES;
     for (int i = 0; i < npre; ++i) issue(i);
 
-    // Per-lane ldmatrix row addresses (byte offsets inside a tile).
+    // Per-lane ldmatrix row addresses.
     const int mi = lane >> 3, ri = lane & 7;
     const int k_tok = (mi >> 1) * 8 + ri;  // K: matrices (tok 0-7|8-15) x (d lo|hi)
     const int k_hi = mi & 1;
     const int v_tok = (mi & 1) * 8 + ri;   // V (trans): (tok lo|hi) x (d lo|hi)
     const int v_hi = mi >> 1;
 
-    float oacc[NT_O][4];
-#pragma unroll
-    for (int j = 0; j < NT_O; ++j) oacc[j][0] = oacc[j][1] = oacc[j][2] = oacc[j][3] = 0.f;
-    float m_lo = -INFINITY, m_hi = -INFINITY, l_lo = 0.f, l_hi = 0.f;
-
     for (int i = 0; i < ntiles; ++i) {
         const int st = i % STAGES;
         const bool ok = mbar_wait(bar0 + 8 * st, (i / STAGES) & 1);
         if (!__all_sync(0xffffffffu, ok)) {
             for (int k = i + 1; k < ntiles && k < i + STAGES; ++k) mbar_wait(bar0 + 8 * (k % STAGES), (k / STAGES) & 1);
-            return;
+            return false;
         }
         const int valid = min(kTileTok, t_end - (t_begin + i * kTileTok));
         const uint32_t Ks = ring_s + st * C::kStageBytes;
         const uint32_t Vs = Ks + C::kTileBytes;
 
-        // S = Q K^T  (16 heads x 16 tokens as two n-tiles of 8 tokens)
+        // S = Q K^T  (16 rows x 16 tokens as two n-tiles of 8 tokens)
         float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
@@ -151,12 +138,11 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnPa
             const uint32_t addr = Ks + (chunk >> 3) * C::kHalfTile + k_tok * 128 + (((chunk & 7) ^ (k_tok & 7)) << 4);
             uint32_t b0, b1, b2, b3;
             ldmatrix_x4(addr, b0, b1, b2, b3);
-            mma_16816<T>(sacc[0], qa[kk], b0, b1);
-            mma_16816<T>(sacc[1], qa[kk], b2, b3);
+            mma_16816<T>(sacc[0], acc.qa[kk], b0, b1);
+            mma_16816<T>(sacc[1], acc.qa[kk], b2, b3);
         }
 
-        // Online softmax.  Element e of n-tile nt is token nt*8 + 2*tig + (e&1),
-        // head row gid (e<2) or gid+8 (e>=2).
+        // Online softmax.  Element e of n-tile nt is token nt*8 + 2*tig + (e&1).
         float mx_lo = -INFINITY, mx_hi = -INFINITY;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
@@ -174,10 +160,10 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnPa
             mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, off));
             mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, off));
         }
-        const float mn_lo = fmaxf(m_lo, mx_lo), mn_hi = fmaxf(m_hi, mx_hi);
-        const float a_lo = ex2(m_lo - mn_lo), a_hi = ex2(m_hi - mn_hi);
-        m_lo = mn_lo;
-        m_hi = mn_hi;
+        const float mn_lo = fmaxf(acc.m_lo, mx_lo), mn_hi = fmaxf(acc.m_hi, mx_hi);
+        const float a_lo = ex2(acc.m_lo - mn_lo), a_hi = ex2(acc.m_hi - mn_hi);
+        acc.m_lo = mn_lo;
+        acc.m_hi = mn_hi;
         float ps_lo = 0.f, ps_hi = 0.f;
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
@@ -189,14 +175,14 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnPa
                 else ps_hi += pr;
             }
         }
-        l_lo = l_lo * a_lo + ps_lo;
-        l_hi = l_hi * a_hi + ps_hi;
+        acc.l_lo = acc.l_lo * a_lo + ps_lo;
+        acc.l_hi = acc.l_hi * a_hi + ps_hi;
 #pragma unroll
         for (int j = 0; j < NT_O; ++j) {
-            oacc[j][0] *= a_lo;
-            oacc[j][1] *= a_lo;
-            oacc[j][2] *= a_hi;
-            oacc[j][3] *= a_hi;
+            acc.o[j][0] *= a_lo;
+            acc.o[j][1] *= a_lo;
+            acc.o[j][2] *= a_hi;
+            acc.o[j][3] *= a_hi;
         }
         uint32_t pa[4];
         pa[0] = Elt<T>::pack2(sacc[0][0], sacc[0][1]);
@@ -225,42 +211,166 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnPa
             const uint32_t addr = Vs + (chunk >> 3) * C::kHalfTile + v_tok * 128 + (((chunk & 7) ^ (v_tok & 7)) << 4);
             uint32_t b0, b1, b2, b3;
             ldmatrix_x4_trans(addr, b0, b1, b2, b3);
-            mma_16816<T>(oacc[2 * jj], pa, b0, b1);
-            mma_16816<T>(oacc[2 * jj + 1], pa, b2, b3);
+            mma_16816<T>(acc.o[2 * jj], pa, b0, b1);
+            mma_16816<T>(acc.o[2 * jj + 1], pa, b2, b3);
         }
         __syncwarp();
         if (i + STAGES < ntiles) issue(i + STAGES);
     }
-
 #pragma unroll
     for (int off = 1; off < 4; off <<= 1) {
-        l_lo += __shfl_xor_sync(0xffffffffu, l_lo, off);
-        l_hi += __shfl_xor_sync(0xffffffffu, l_hi, off);
+        acc.l_lo += __shfl_xor_sync(0xffffffffu, acc.l_lo, off);
+        acc.l_hi += __shfl_xor_sync(0xffffffffu, acc.l_hi, off);
     }
-    const bool w_lo = gid < G, w_hi = gid + 8 < G;
-    if (nP == 1) {
-        const float i_lo = 1.f / l_lo, i_hi = 1.f / l_hi;
-        T* ob = reinterpret_cast<T*>(p.out) + ((int64_t)s * p.Hq + h0) * D;
+    return true;
+}
+
+// Write one accumulator row: the normalised output (out_row != nullptr) or a
+// split-K partial (o_row, ml).  hi selects rows gid+8.
+template <typename T, int D>
+__device__ __forceinline__ void mma_store_row(const MmaAcc<T, D>& acc, bool hi, int tig, T* out_row, float* o_row,
+                                              float* ml) {
+    constexpr int NT_O = D / 8;
+    const int e0 = hi ? 2 : 0;
+    const float l = hi ? acc.l_hi : acc.l_lo;
+    if (out_row) {
+        const float inv = 1.f / l;
 #pragma unroll
-        for (int j = 0; j < NT_O; ++j) {
-            const int d = j * 8 + 2 * tig;
-            if (w_lo) *reinterpret_cast<uint32_t*>(ob + gid * D + d) = Elt<T>::pack2(oacc[j][0] * i_lo, oacc[j][1] * i_lo);
-            if (w_hi)
-                *reinterpret_cast<uint32_t*>(ob + (gid + 8) * D + d) = Elt<T>::pack2(oacc[j][2] * i_hi, oacc[j][3] * i_hi);
-        }
+        for (int j = 0; j < NT_O; ++j)
+            *reinterpret_cast<uint32_t*>(out_row + j * 8 + 2 * tig) =
+                Elt<T>::pack2(acc.o[j][e0] * inv, acc.o[j][e0 + 1] * inv);
     } else {
-        const int64_t i_lo = ((int64_t)s * p.Hq + h0 + gid) * p.maxP + part;
-        const int64_t i_hi = ((int64_t)s * p.Hq + h0 + gid + 8) * p.maxP + part;
 #pragma unroll
-        for (int j = 0; j < NT_O; ++j) {
-            const int d = j * 8 + 2 * tig;
-            if (w_lo) *reinterpret_cast<float2*>(p.ws_o + i_lo * D + d) = make_float2(oacc[j][0], oacc[j][1]);
-            if (w_hi) *reinterpret_cast<float2*>(p.ws_o + i_hi * D + d) = make_float2(oacc[j][2], oacc[j][3]);
+        for (int j = 0; j < NT_O; ++j)
+            *reinterpret_cast<float2*>(o_row + j * 8 + 2 * tig) = make_float2(acc.o[j][e0], acc.o[j][e0 + 1]);
+        if (tig == 0) *reinterpret_cast<float2*>(ml) = make_float2(hi ? acc.m_hi : acc.m_lo, l);
+    }
+}
+
+template <typename T, int D, int WARPS, int STAGES>
+__device__ __forceinline__ uint8_t* mma_setup_ring(uint8_t* smem_raw, int warp, int lane, uint32_t& bar0,
+                                                   const CUtensorMap* tmK, const CUtensorMap* tmV) {
+    using C = MmaCfg<T, D, WARPS, STAGES>;
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    bar0 = smem_u32(smem + C::kDataBytes + warp * STAGES * 8);
+    if (lane == 0) {
+        prefetch_tensor_map(tmK);
+        prefetch_tensor_map(tmV);
+        for (int i = 0; i < STAGES; ++i) mbar_init(bar0 + 8 * i, 1);
+        fence_barrier_init();
+    }
+    __syncwarp();
+    return smem + warp * STAGES * C::kStageBytes;
+}
+
+// Grouped-query decode: grid (ceil(Hkv / WARPS), partitions, S).
+template <typename T, int D, int WARPS, int STAGES>
+__global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnParams p,
+                                                                    const __grid_constant__ CUtensorMap tmK,
+                                                                    const __grid_constant__ CUtensorMap tmV) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = blockIdx.x * WARPS + warp;  // kv head
+    const int part = blockIdx.y;
+    const int s = blockIdx.z;
+    if (g >= p.Hkv) return;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int G = p.G;
+    const int h0 = g * G;
+
+    const Unit u = resolve_unit(p, s, part, part == 0 && g == 0 && lane == 0);
+    if (u.t_begin >= u.L) {
+        if (part == 0 && u.L == 0) {  // empty context: zeros for the group's heads
+            T* o = reinterpret_cast<T*>(p.out) + ((int64_t)s * p.Hq + h0) * D;
+            for (int i = lane; i < G * D; i += 32) o[i] = T(0.f);
         }
-        if (tig == 0) {
-            if (w_lo) *reinterpret_cast<float2*>(p.ws_ml + i_lo * 2) = make_float2(m_lo, l_lo);
-            if (w_hi) *reinterpret_cast<float2*>(p.ws_ml + i_hi * 2) = make_float2(m_hi, l_hi);
+        return;
+    }
+    uint32_t bar0;
+    uint8_t* ring = mma_setup_ring<T, D, WARPS, STAGES>(smem_raw, warp, lane, bar0, &tmK, &tmV);
+
+    const T* qb = reinterpret_cast<const T*>(p.q) + ((int64_t)s * p.Hq + h0) * D;
+    MmaAcc<T, D> acc;
+    acc.load_q(gid < G ? qb + gid * D : nullptr, gid + 8 < G ? qb + (gid + 8) * D : nullptr, tig);
+    if (!mma_attend<T, D, WARPS, STAGES>(p, &tmK, &tmV, ring, bar0, p.block_tables + (int64_t)s * p.maxB,
+                                         u.t_begin, u.t_end, g, lane, acc))
+        return;
+
+#pragma unroll
+    for (int hi = 0; hi < 2; ++hi) {
+        const int r = gid + 8 * hi;
+        if (r >= G) continue;
+        const int64_t row = (int64_t)s * p.Hq + h0 + r;
+        if (u.direct) {
+            mma_store_row<T, D>(acc, hi, tig, reinterpret_cast<T*>(p.out) + row * D, nullptr, nullptr);
+        } else {
+            const int64_t idx = row * p.maxP + u.slot;
+            mma_store_row<T, D>(acc, hi, tig, nullptr, p.ws_o + idx * D, p.ws_ml + idx * 2);
         }
+    }
+}
+
+// Shared-prefix pass: grid (row-tile blocks, prefix partitions, groups * Hkv).
+// Row r of group i is (sequence group_first[i] + r / G, query head g*G + r % G).
+template <typename T, int D, int WARPS, int STAGES>
+__global__ void __launch_bounds__(WARPS * 32) prefix_attn_mma_kernel(const AttnParams p,
+                                                                     const __grid_constant__ CUtensorMap tmK,
+                                                                     const __grid_constant__ CUtensorMap tmV) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int tile = blockIdx.x * WARPS + warp;
+    const int pp = blockIdx.y;  // partition of the shared tokens
+    const int gi = blockIdx.z / p.Hkv;
+    const int g = blockIdx.z - gi * p.Hkv;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int G = p.G;
+
+    int first = p.group_first[gi], last = p.group_first[gi + 1];
+    first = max(0, min(first, p.S));
+    last = max(first, min(last, p.S));
+    if (last - first > p.max_group_size) {
+        if (tile == 0 && pp == 0 && g == 0 && lane == 0) flag_error(16u /* PKV_DEVERR_GROUP */);
+        last = first + p.max_group_size;  // members past the grid get no prefix partials
+    }
+    const int rows = (last - first) * G;
+    if (tile * 16 >= rows) return;
+    const int shared = p.group_shared[gi];
+    if (shared <= 0 || shared % p.bs != 0 || shared > p.max_len) return;  // reported by the decode kernels
+    const int t_begin = pp * p.P;
+    if (t_begin >= shared) return;
+    const int t_end = min(shared, t_begin + p.P);
+
+    // Query rows of this lane (gid, gid+8); a member whose context is shorter
+    // than the shared run is not a member (the decode kernels report it).
+    int rs[2], rh[2];
+    bool use[2];
+#pragma unroll
+    for (int hi = 0; hi < 2; ++hi) {
+        const int r = tile * 16 + gid + 8 * hi;
+        use[hi] = r < rows;
+        rs[hi] = first + (use[hi] ? r / G : 0);
+        rh[hi] = g * G + (use[hi] ? r % G : 0);
+        if (use[hi]) {  // same clamp as the decode kernels
+            const int L = min(max(p.context_lens[rs[hi]], 0), p.max_len);
+            if (L < shared) use[hi] = false;
+        }
+    }
+    uint32_t bar0;
+    uint8_t* ring = mma_setup_ring<T, D, WARPS, STAGES>(smem_raw, warp, lane, bar0, &tmK, &tmV);
+    const T* q = reinterpret_cast<const T*>(p.q);
+    MmaAcc<T, D> acc;
+    acc.load_q(use[0] ? q + ((int64_t)rs[0] * p.Hq + rh[0]) * D : nullptr,
+               use[1] ? q + ((int64_t)rs[1] * p.Hq + rh[1]) * D : nullptr, tig);
+    if (!mma_attend<T, D, WARPS, STAGES>(p, &tmK, &tmV, ring, bar0, p.block_tables + (int64_t)first * p.maxB,
+                                         t_begin, t_end, g, lane, acc))
+        return;
+#pragma unroll
+    for (int hi = 0; hi < 2; ++hi) {
+        if (!use[hi]) continue;
+        const int64_t idx = ((int64_t)rs[hi] * p.Hq + rh[hi]) * p.maxP + pp;
+        mma_store_row<T, D>(acc, hi, tig, nullptr, p.ws_o + idx * D, p.ws_ml + idx * 2);
     }
 }
 

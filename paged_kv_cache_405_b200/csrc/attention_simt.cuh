@@ -55,20 +55,18 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_simt_kernel(const AttnP
     const int s = blockIdx.z;
     if (h >= p.Hq) return;
 
-    const int L = load_context_len(p, s, part == 0 && h == 0 && lane == 0);
-    const int nP = (L + p.P - 1) / p.P;
-    const int t_begin = part * p.P;
+    const Unit u = resolve_unit(p, s, part, part == 0 && h == 0 && lane == 0);
     const int sub = lane / LPT;  // which token of a pass
     const int c = lane % LPT;    // which 16-byte slice of the row
-    if (t_begin >= L) {
-        if (part == 0 && sub == 0) {  // empty context: zeros
+    if (u.t_begin >= u.L) {
+        if (part == 0 && u.L == 0 && sub == 0) {  // empty context: zeros
             float z[EPL > 4 ? EPL : 4] = {};
             uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) + ((int64_t)s * p.Hq + h) * D) + c;
             *o = Elt<T>::narrow(z);
         }
         return;
     }
-    const int t_end = min(L, t_begin + p.P);
+    const int t_begin = u.t_begin, t_end = u.t_end;
     const int g = h / p.G;
     const int ntiles = (t_end - t_begin + kTileTok - 1) / kTileTok;
 
@@ -183,7 +181,7 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_simt_kernel(const AttnP
         for (int e = 0; e < EPL; ++e) o[e] += __shfl_xor_sync(0xffffffffu, o[e], off);
     }
     if (sub != 0) return;
-    if (nP == 1) {
+    if (u.direct) {
         const float inv = 1.f / l;
         float r[EPL];
 #pragma unroll
@@ -191,7 +189,7 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_simt_kernel(const AttnP
         uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.out) + ((int64_t)s * p.Hq + h) * D) + c;
         *dst = Elt<T>::narrow(r);
     } else {
-        const int64_t idx = ((int64_t)s * p.Hq + h) * p.maxP + part;
+        const int64_t idx = ((int64_t)s * p.Hq + h) * p.maxP + u.slot;
         float4* dst = reinterpret_cast<float4*>(p.ws_o + idx * D + c * EPL);
 #pragma unroll
         for (int e = 0; e < EPL; e += 4) dst[e / 4] = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);

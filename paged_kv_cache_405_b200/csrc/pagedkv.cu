@@ -72,6 +72,22 @@ static size_t workspace_for(int S, int Hq, int D, int max_len, int P) {
     return (size_t)S * Hq * maxP * (size_t)(D + 2) * sizeof(float);
 }
 
+// Shared-prefix mode: one more partial slot per (sequence, head) than
+// partitions, since a member's prefix and suffix partitions can each end
+// part-way through a partition.
+static size_t shared_workspace_for(int S, int Hq, int D, int max_len, int P) {
+    const int64_t slots = (max_len + P - 1) / P + 1;
+    return (size_t)S * Hq * slots * (size_t)(D + 2) * sizeof(float);
+}
+
+// Smallest partition the library's own choice can produce for max_len: the
+// workspace queries size for it, so the buffer fits whatever is chosen.
+static int partition_bound(int max_len, int requested) {
+    const int P = choose_partition(max_len, requested);
+    if (requested == 0 && P < max_len) return std::min(P, kMinAutoPartition);
+    return P;
+}
+
 // --------------------------------------------------------------- tensor maps
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -134,6 +150,18 @@ static cudaError_t launch_mma(const pkv::AttnParams& p, dim3 grid, const CUtenso
 }
 
 template <typename T, int D>
+static cudaError_t launch_prefix(const pkv::AttnParams& p, dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv,
+                                 cudaStream_t st) {
+    using C = pkv::MmaCfg<T, D, kMmaWarps, kMmaStages>;
+    auto k = pkv::prefix_attn_mma_kernel<T, D, kMmaWarps, kMmaStages>;
+    static cudaError_t attr = set_smem(k, C::kSmemBytes);
+    if (attr != cudaSuccess) return attr;
+    k<<<grid, kMmaWarps * 32, C::kSmemBytes, st>>>(p, mk, mv);
+    g_launches++;
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
 static cudaError_t launch_reduce(const pkv::ReduceParams& r, cudaStream_t st) {
     const int warps = r.S * r.Hq;
     const int blocks = (warps + 7) / 8;
@@ -143,23 +171,147 @@ static cudaError_t launch_reduce(const pkv::ReduceParams& r, cudaStream_t st) {
 }
 
 template <typename T>
-static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, bool use_mma, const CUtensorMap* mk,
-                                      const CUtensorMap* mv, cudaStream_t st) {
-    cudaError_t e;
-    if (use_mma) {
-        if constexpr (std::is_same<T, float>::value) {
-            return cudaErrorInvalidValue;
-        } else {
-            dim3 grid((p.Hkv + kMmaWarps - 1) / kMmaWarps, p.maxP, p.S);
+static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int nparts, bool use_mma, bool shared_mode,
+                                      const CUtensorMap* mk, const CUtensorMap* mv, cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
+    if constexpr (std::is_same<T, float>::value) {
+        if (use_mma || shared_mode) return cudaErrorInvalidValue;
+    } else {
+        if (shared_mode && p.num_groups > 0) {
+            const int tiles = (p.max_group_size * p.G + 15) / 16;
+            dim3 grid((tiles + kMmaWarps - 1) / kMmaWarps, nparts, p.num_groups * p.Hkv);
+            e = D == 64 ? launch_prefix<T, 64>(p, grid, *mk, *mv, st) : launch_prefix<T, 128>(p, grid, *mk, *mv, st);
+            if (e != cudaSuccess) return e;
+        }
+        if (use_mma) {
+            dim3 grid((p.Hkv + kMmaWarps - 1) / kMmaWarps, nparts, p.S);
             e = D == 64 ? launch_mma<T, 64>(p, grid, *mk, *mv, st) : launch_mma<T, 128>(p, grid, *mk, *mv, st);
         }
-    } else {
-        dim3 grid((p.Hq + kSimtWarps - 1) / kSimtWarps, p.maxP, p.S);
+    }
+    if (!use_mma) {
+        dim3 grid((p.Hq + kSimtWarps - 1) / kSimtWarps, nparts, p.S);
         e = D == 64 ? launch_simt<T, 64>(p, grid, st) : launch_simt<T, 128>(p, grid, st);
     }
     if (e != cudaSuccess || p.maxP <= 1) return e;
-    pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len};
+    pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
+                        p.group_first, p.group_shared, p.num_groups};
     return D == 64 ? launch_reduce<T, 64>(r, st) : launch_reduce<T, 128>(r, st);
+}
+
+struct GroupArgs {
+    const int32_t* first = nullptr;
+    const int32_t* shared = nullptr;
+    int num = 0;
+    int max_size = 0;
+    bool mode = false;  // called through the shared-prefix entry point
+};
+
+static pkv_status decode_impl(void* out, const void* q, const void* k_pool, const void* v_pool,
+                              const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
+                              int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                              int num_blocks, float scale, int partition_size, const GroupArgs& grp, void* workspace,
+                              size_t workspace_bytes, pkv_dtype dtype, void* stream) {
+    if (!valid_dtype(dtype)) return invalid("pkv_paged_attention_decode: bad dtype");
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
+        return invalid("pkv_paged_attention_decode: sizes must be positive");
+    if (num_q_heads % num_kv_heads != 0)
+        return invalid("pkv_paged_attention_decode: num_q_heads must be a multiple of num_kv_heads");
+    if (!valid_block_size(block_size))
+        return invalid("pkv_paged_attention_decode: block_size must be 16, 32, 64, 128 or 256");
+    if (head_dim != 64 && head_dim != 128) {
+        g_msg = "pkv_paged_attention_decode: head_dim must be 64 or 128";
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (grp.mode && dtype == PKV_F32) {
+        g_msg = "pkv_paged_attention_decode_shared: fp32 is not supported (tensor-core prefix pass)";
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (partition_size < 0 || partition_size % 16 != 0)
+        return invalid("pkv_paged_attention_decode: partition_size must be 0 or a positive multiple of 16");
+    if (!(std::isfinite(scale)) || scale < 0.f) return invalid("pkv_paged_attention_decode: scale must be >= 0");
+    const int64_t max_len64 = (int64_t)max_blocks_per_seq * block_size;
+    if (max_len64 > (int64_t)1 << 30) return invalid("pkv_paged_attention_decode: max_blocks_per_seq*block_size too large");
+    if ((int64_t)num_blocks * num_kv_heads * block_size >= ((int64_t)1 << 31))
+        return invalid("pkv_paged_attention_decode: pool has 2^31 or more rows");
+    if (grp.mode) {
+        if (grp.num < 0) return invalid("pkv_paged_attention_decode_shared: num_groups must be >= 0");
+        if (grp.num > 0 && (!grp.first || !grp.shared || (reinterpret_cast<uintptr_t>(grp.first) & 3u) ||
+                            (reinterpret_cast<uintptr_t>(grp.shared) & 3u)))
+            return invalid("pkv_paged_attention_decode_shared: group arrays must be 4-byte aligned device pointers");
+        if (grp.num > 0 && grp.max_size < 1)
+            return invalid("pkv_paged_attention_decode_shared: max_group_size must be >= 1");
+        if ((int64_t)grp.num * num_kv_heads > 65535)
+            return invalid("pkv_paged_attention_decode_shared: num_groups * num_kv_heads must be <= 65535");
+        if ((int64_t)grp.max_size * (num_q_heads / num_kv_heads) > ((int64_t)1 << 24))
+            return invalid("pkv_paged_attention_decode_shared: max_group_size too large");
+    }
+    if (num_seqs == 0) return PKV_OK;
+    if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens)
+        return invalid("pkv_paged_attention_decode: null pointer");
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
+        return invalid("pkv_paged_attention_decode: pointers must be 16-byte aligned (tables 4-byte)");
+    if (num_seqs > 65535) return invalid("pkv_paged_attention_decode: at most 65535 sequences per call");
+
+    const int max_len = (int)max_len64;
+    const int P = choose_partition(max_len, partition_size);
+    const int64_t nparts = (max_len + P - 1) / P;
+    if (nparts > 65535) return invalid("pkv_paged_attention_decode: too many partitions; raise partition_size");
+    const int64_t slots = nparts + (grp.mode ? 1 : 0);
+    const size_t need = grp.mode ? shared_workspace_for(num_seqs, num_q_heads, head_dim, max_len, P)
+                                 : workspace_for(num_seqs, num_q_heads, head_dim, max_len, P);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need) return invalid("pkv_paged_attention_decode: workspace too small");
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+            return invalid("pkv_paged_attention_decode: workspace must be 256-byte aligned");
+    }
+
+    pkv::AttnParams p;
+    p.out = out;
+    p.q = q;
+    p.k_pool = k_pool;
+    p.v_pool = v_pool;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    const size_t n_part = (size_t)num_seqs * num_q_heads * slots;
+    p.ws_o = need ? static_cast<float*>(workspace) : nullptr;
+    p.ws_ml = need ? static_cast<float*>(workspace) + n_part * head_dim : nullptr;
+    p.S = num_seqs;
+    p.Hq = num_q_heads;
+    p.Hkv = num_kv_heads;
+    p.G = num_q_heads / num_kv_heads;
+    p.bs = block_size;
+    p.NB = num_blocks;
+    p.maxB = max_blocks_per_seq;
+    p.P = P;
+    p.maxP = (int)slots;
+    p.max_len = max_len;
+    const float sc = scale > 0.f ? scale : 1.f / std::sqrt((float)head_dim);
+    p.scale_log2 = sc * 1.4426950408889634f;
+    p.group_first = grp.num > 0 ? grp.first : nullptr;
+    p.group_shared = grp.num > 0 ? grp.shared : nullptr;
+    p.num_groups = grp.num;
+    p.max_group_size = grp.max_size;
+
+    const bool use_mma = dtype != PKV_F32 && p.G >= 2 && p.G <= 16;
+    CUtensorMap mk, mv;
+    if (use_mma || (grp.mode && grp.num > 0)) {
+        const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
+        if (!make_pool_map(&mk, k_pool, rows, head_dim, dtype) || !make_pool_map(&mv, v_pool, rows, head_dim, dtype)) {
+            g_msg = "pkv_paged_attention_decode: cuTensorMapEncodeTiled failed";
+            return PKV_ERR_CUDA;
+        }
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e;
+    switch (dtype) {
+        case PKV_F32: e = dispatch_attention<float>(p, head_dim, (int)nparts, false, false, nullptr, nullptr, st); break;
+        case PKV_BF16:
+            e = dispatch_attention<__nv_bfloat16>(p, head_dim, (int)nparts, use_mma, grp.mode, &mk, &mv, st);
+            break;
+        default: e = dispatch_attention<__half>(p, head_dim, (int)nparts, use_mma, grp.mode, &mk, &mv, st); break;
+    }
+    return e == cudaSuccess ? PKV_OK : cuda_fail("pkv_paged_attention_decode", e);
 }
 
 }  // namespace pkv_host
@@ -221,9 +373,8 @@ pkv_status pkv_kv_append(const void* k_new, const void* v_new, void* k_pool, voi
 size_t pkv_attention_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
                                      int partition_size) {
     if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0 || partition_size < 0) return 0;
-    int P = partition_size > 0 ? partition_size : choose_partition(max_context_len, 0);
-    if (partition_size == 0 && P < max_context_len) P = std::min(P, kMinAutoPartition);
-    return workspace_for(num_seqs, num_q_heads, head_dim, max_context_len, P);
+    return workspace_for(num_seqs, num_q_heads, head_dim, max_context_len,
+                         partition_bound(max_context_len, partition_size));
 }
 
 int pkv_attention_partition_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
@@ -240,83 +391,35 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_po
                                       const int32_t* context_lens, int num_seqs, int num_q_heads, int num_kv_heads,
                                       int head_dim, int block_size, int num_blocks, float scale, int partition_size,
                                       void* workspace, size_t workspace_bytes, pkv_dtype dtype, void* stream) {
-    if (!valid_dtype(dtype)) return invalid("pkv_paged_attention_decode: bad dtype");
-    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
-        return invalid("pkv_paged_attention_decode: sizes must be positive");
-    if (num_q_heads % num_kv_heads != 0)
-        return invalid("pkv_paged_attention_decode: num_q_heads must be a multiple of num_kv_heads");
-    if (!valid_block_size(block_size))
-        return invalid("pkv_paged_attention_decode: block_size must be 16, 32, 64, 128 or 256");
-    if (head_dim != 64 && head_dim != 128) {
-        g_msg = "pkv_paged_attention_decode: head_dim must be 64 or 128";
-        return PKV_ERR_UNSUPPORTED;
-    }
-    if (partition_size < 0 || partition_size % 16 != 0)
-        return invalid("pkv_paged_attention_decode: partition_size must be 0 or a positive multiple of 16");
-    if (!(std::isfinite(scale)) || scale < 0.f) return invalid("pkv_paged_attention_decode: scale must be >= 0");
-    const int64_t max_len64 = (int64_t)max_blocks_per_seq * block_size;
-    if (max_len64 > (int64_t)1 << 30) return invalid("pkv_paged_attention_decode: max_blocks_per_seq*block_size too large");
-    if ((int64_t)num_blocks * num_kv_heads * block_size >= ((int64_t)1 << 31))
-        return invalid("pkv_paged_attention_decode: pool has 2^31 or more rows");
-    if (num_seqs == 0) return PKV_OK;
-    if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens)
-        return invalid("pkv_paged_attention_decode: null pointer");
-    if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) ||
-        (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u))
-        return invalid("pkv_paged_attention_decode: pointers must be 16-byte aligned (tables 4-byte)");
-    if (num_seqs > 65535) return invalid("pkv_paged_attention_decode: at most 65535 sequences per call");
+    return decode_impl(out, q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads,
+                       num_kv_heads, head_dim, block_size, num_blocks, scale, partition_size, GroupArgs(), workspace,
+                       workspace_bytes, dtype, stream);
+}
 
-    const int max_len = (int)max_len64;
-    const int P = choose_partition(max_len, partition_size);
-    const int64_t maxP = (max_len + P - 1) / P;
-    if (maxP > 65535) return invalid("pkv_paged_attention_decode: too many partitions; raise partition_size");
-    const size_t need = workspace_for(num_seqs, num_q_heads, head_dim, max_len, P);
-    if (need > 0) {
-        if (!workspace || workspace_bytes < need) return invalid("pkv_paged_attention_decode: workspace too small");
-        if (reinterpret_cast<uintptr_t>(workspace) & 255u)
-            return invalid("pkv_paged_attention_decode: workspace must be 256-byte aligned");
-    }
+pkv_status pkv_paged_attention_decode_shared(void* out, const void* q, const void* k_pool, const void* v_pool,
+                                             const int32_t* block_tables, int max_blocks_per_seq,
+                                             const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                             int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                             float scale, int partition_size, const int32_t* group_first,
+                                             const int32_t* group_shared, int num_groups, int max_group_size,
+                                             void* workspace, size_t workspace_bytes, pkv_dtype dtype,
+                                             void* stream) {
+    GroupArgs g;
+    g.first = group_first;
+    g.shared = group_shared;
+    g.num = num_groups;
+    g.max_size = max_group_size;
+    g.mode = true;
+    return decode_impl(out, q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads,
+                       num_kv_heads, head_dim, block_size, num_blocks, scale, partition_size, g, workspace,
+                       workspace_bytes, dtype, stream);
+}
 
-    pkv::AttnParams p;
-    p.out = out;
-    p.q = q;
-    p.k_pool = k_pool;
-    p.v_pool = v_pool;
-    p.block_tables = block_tables;
-    p.context_lens = context_lens;
-    const size_t n_part = (size_t)num_seqs * num_q_heads * maxP;
-    p.ws_o = need ? static_cast<float*>(workspace) : nullptr;
-    p.ws_ml = need ? static_cast<float*>(workspace) + n_part * head_dim : nullptr;
-    p.S = num_seqs;
-    p.Hq = num_q_heads;
-    p.Hkv = num_kv_heads;
-    p.G = num_q_heads / num_kv_heads;
-    p.bs = block_size;
-    p.NB = num_blocks;
-    p.maxB = max_blocks_per_seq;
-    p.P = P;
-    p.maxP = (int)maxP;
-    p.max_len = max_len;
-    const float sc = scale > 0.f ? scale : 1.f / std::sqrt((float)head_dim);
-    p.scale_log2 = sc * 1.4426950408889634f;
-
-    const bool use_mma = dtype != PKV_F32 && p.G >= 2 && p.G <= 16;
-    CUtensorMap mk, mv;
-    if (use_mma) {
-        const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
-        if (!make_pool_map(&mk, k_pool, rows, head_dim, dtype) || !make_pool_map(&mv, v_pool, rows, head_dim, dtype)) {
-            g_msg = "pkv_paged_attention_decode: cuTensorMapEncodeTiled failed";
-            return PKV_ERR_CUDA;
-        }
-    }
-    cudaStream_t st = (cudaStream_t)stream;
-    cudaError_t e;
-    switch (dtype) {
-        case PKV_F32: e = dispatch_attention<float>(p, head_dim, false, nullptr, nullptr, st); break;
-        case PKV_BF16: e = dispatch_attention<__nv_bfloat16>(p, head_dim, use_mma, &mk, &mv, st); break;
-        default: e = dispatch_attention<__half>(p, head_dim, use_mma, &mk, &mv, st); break;
-    }
-    return e == cudaSuccess ? PKV_OK : cuda_fail("pkv_paged_attention_decode", e);
+size_t pkv_attention_shared_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
+                                            int partition_size) {
+    if (num_seqs <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0 || partition_size < 0) return 0;
+    return shared_workspace_for(num_seqs, num_q_heads, head_dim, max_context_len,
+                                partition_bound(max_context_len, partition_size));
 }
 
 pkv_status pkv_block_copy(void* k_pool, void* v_pool, const int32_t* pairs, int num_pairs, int num_blocks,

@@ -17,7 +17,10 @@ struct ReduceParams {
     const float* ws_o;          // [S][Hq][maxP][D]
     const float* ws_ml;         // [S][Hq][maxP][2]
     const int32_t* context_lens;
-    int S, Hq, D, P, maxP, max_len;
+    int S, Hq, D, P, maxP, max_len, bs;
+    const int32_t* group_first;   // shared-prefix groups, as in AttnParams
+    const int32_t* group_shared;
+    int num_groups;
 };
 
 template <typename T, int D>
@@ -30,8 +33,22 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const ReduceParams p
     int L = p.context_lens[s];
     if (L < 0) L = 0;
     if (L > p.max_len) L = p.max_len;
-    const int nP = (L + p.P - 1) / p.P;
-    if (nP <= 1) return;  // written directly by the attention kernel
+    // Same rule as the attention kernels: a member of a valid shared-prefix
+    // group has ceil(shared/P) prefix partials followed by its own ones.
+    int shared = 0;
+    if (p.num_groups > 0 && s >= p.group_first[0] && s < p.group_first[p.num_groups]) {
+        int lo = 0, hi = p.num_groups;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (p.group_first[mid] <= s) lo = mid;
+            else hi = mid;
+        }
+        const int sh = p.group_shared[lo];
+        if (sh > 0 && sh % p.bs == 0 && sh <= L) shared = sh;
+    }
+    const int nsuf = (L - shared + p.P - 1) / p.P;
+    const int nP = (shared + p.P - 1) / p.P + nsuf;
+    if (shared == 0 && nP <= 1) return;  // written directly by the attention kernel
     const int64_t base = (int64_t)warp * p.maxP;
     const float* ml = p.ws_ml + base * 2;
     float M = -INFINITY;

@@ -33,6 +33,13 @@ class StepPlan:
     cow_pairs: np.ndarray      # int32 [n, 2] blocks to copy before writing
     lens: np.ndarray           # int32 [len(seq_ids)] context after the write
     block_tables: np.ndarray   # int32 [len(seq_ids), max_blocks]
+    group_first: np.ndarray = None   # int32 [g + 1] shared-prefix runs (see find_shared_prefix_groups)
+    group_shared: np.ndarray = None  # int32 [g]
+    max_group_size: int = 0
+
+    @property
+    def has_groups(self) -> bool:
+        return self.group_shared is not None and bool((self.group_shared > 0).any())
 
 
 @dataclass
@@ -42,11 +49,15 @@ class DevicePlan:
     lens: torch.Tensor
     block_tables: torch.Tensor
     n_cow: int
+    group_first: Optional[torch.Tensor] = None
+    group_shared: Optional[torch.Tensor] = None
+    max_group_size: int = 0
 
 
 class DecodeSession:
     def __init__(self, k_pool: torch.Tensor, v_pool: torch.Tensor, num_q_heads: int, max_blocks_per_seq: int,
-                 free_order=None, partition_size: int = 0, max_batch: int = 0):
+                 free_order=None, partition_size: int = 0, max_batch: int = 0, share_prefixes: bool = True,
+                 min_group_size: int = 4):
         self.k_pool, self.v_pool = k_pool, v_pool
         self.num_blocks, self.num_kv_heads, self.block_size, self.head_dim = k_pool.shape
         self.num_q_heads = num_q_heads
@@ -54,11 +65,16 @@ class DecodeSession:
         self.partition_size = partition_size
         self.alloc = B.BlockAllocator(self.num_blocks, self.block_size, free_order)
         self.device = k_pool.device
+        # Runs of sequences sharing leading blocks go through the shared-prefix
+        # pass (16-bit pools only: it runs on tensor cores).
+        self.share_prefixes = share_prefixes and k_pool.dtype != torch.float32
+        self.min_group_size = min_group_size
         n = max(max_batch, 1)
-        self.workspace = torch.empty(
-            max(256, B.attention_workspace_bytes(n, num_q_heads, self.head_dim,
-                                                 max_blocks_per_seq * self.block_size, partition_size)),
-            dtype=torch.uint8, device=self.device)
+        max_len = max_blocks_per_seq * self.block_size
+        ws = B.attention_workspace_bytes(n, num_q_heads, self.head_dim, max_len, partition_size)
+        if self.share_prefixes:
+            ws = max(ws, B.attention_shared_workspace_bytes(n, num_q_heads, self.head_dim, max_len, partition_size))
+        self.workspace = torch.empty(max(256, ws), dtype=torch.uint8, device=self.device)
         self._pinned = {}
 
     # ------------------------------------------------------------ host side
@@ -100,16 +116,25 @@ class DecodeSession:
         self._ok(st)
         st, bt, lens = self.alloc.seq_block_tables_batch(list(attend), self.max_blocks)
         self._ok(st)
-        return StepPlan(list(attend), slots, pairs.reshape(-1, 2), lens, bt)
+        plan = StepPlan(list(attend), slots, pairs.reshape(-1, 2), lens, bt)
+        if self.share_prefixes and len(attend) >= self.min_group_size:
+            gf, gs = B.find_shared_prefix_groups(bt, lens, self.block_size, self.min_group_size)
+            if (gs > 0).any():
+                plan.group_first, plan.group_shared = gf, gs
+                plan.max_group_size = int(np.diff(gf).max())
+        return plan
 
     def to_device(self, p: StepPlan, non_blocking: bool = False) -> DevicePlan:
         dev = self.device
 
         def up(a):
             return torch.from_numpy(np.ascontiguousarray(a)).to(dev, non_blocking=non_blocking)
-        return DevicePlan(up(p.slot_mapping), up(p.cow_pairs) if len(p.cow_pairs) else
-                          torch.zeros((0, 2), dtype=torch.int32, device=dev),
-                          up(p.lens), up(p.block_tables), len(p.cow_pairs))
+        d = DevicePlan(up(p.slot_mapping), up(p.cow_pairs) if len(p.cow_pairs) else
+                       torch.zeros((0, 2), dtype=torch.int32, device=dev),
+                       up(p.lens), up(p.block_tables), len(p.cow_pairs))
+        if p.has_groups:
+            d.group_first, d.group_shared, d.max_group_size = up(p.group_first), up(p.group_shared), p.max_group_size
+        return d
 
     # ---------------------------------------------------------- device side
     def launch(self, d: DevicePlan, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
@@ -118,8 +143,18 @@ class DecodeSession:
         if d.n_cow:
             B.block_copy(self.k_pool, self.v_pool, d.cow_pairs, stream=stream)
         B.kv_append(k_new, v_new, self.k_pool, self.v_pool, d.slot_mapping, stream=stream)
-        B.paged_attention_decode(out, q, self.k_pool, self.v_pool, d.block_tables, d.lens,
-                                 partition_size=self.partition_size, workspace=self.workspace, stream=stream)
+        return self.attend(d, q, out, stream=stream)
+
+    def attend(self, d: DevicePlan, q: torch.Tensor, out: torch.Tensor, stream=None):
+        """The step's attention: the shared-prefix call when the plan found groups."""
+        if d.group_shared is not None:
+            B.paged_attention_decode_shared(out, q, self.k_pool, self.v_pool, d.block_tables, d.lens,
+                                            d.group_first, d.group_shared, d.max_group_size,
+                                            partition_size=self.partition_size, workspace=self.workspace,
+                                            stream=stream)
+        else:
+            B.paged_attention_decode(out, q, self.k_pool, self.v_pool, d.block_tables, d.lens,
+                                     partition_size=self.partition_size, workspace=self.workspace, stream=stream)
         return out
 
     def _pin(self, name, like: torch.Tensor):
@@ -135,9 +170,7 @@ class DecodeSession:
         p = self.plan(attend)
         s = torch.cuda.current_stream() if stream is None else stream
         with torch.cuda.stream(s):
-            d = DevicePlan(*(self._h2d(n, a) for n, a in (("slots", p.slot_mapping), ("cow", p.cow_pairs),
-                                                          ("lens", p.lens), ("bt", p.block_tables))),
-                           len(p.cow_pairs))
+            d = self.upload(p)
             q = q_host.to(self.device, non_blocking=True)
             kn = k_new_host.to(self.device, non_blocking=True)
             vn = v_new_host.to(self.device, non_blocking=True)
@@ -148,6 +181,17 @@ class DecodeSession:
             out_host.copy_(out, non_blocking=True)
         s.synchronize()
         return out_host
+
+    def upload(self, p: StepPlan) -> DevicePlan:
+        """Copy a plan to the device through pinned staging buffers (asynchronous)."""
+        d = DevicePlan(*(self._h2d(n, a) for n, a in (("slots", p.slot_mapping), ("cow", p.cow_pairs),
+                                                      ("lens", p.lens), ("bt", p.block_tables))),
+                       len(p.cow_pairs))
+        if p.has_groups:
+            d.group_first = self._h2d("gfirst", p.group_first)
+            d.group_shared = self._h2d("gshared", p.group_shared)
+            d.max_group_size = p.max_group_size
+        return d
 
     def _h2d(self, name, a: np.ndarray) -> torch.Tensor:
         src = torch.from_numpy(np.ascontiguousarray(a))

@@ -167,3 +167,51 @@ def test_batch_calls_equal_sequential_calls():
             for i in range(4):
                 t = a2.seq_block_table(i)
                 assert bt[i][bt[i] >= 0].tolist() == t[1] and lens[i] == t[2]
+
+
+def reference_groups(bt, lens, bs, min_size):
+    """Plain restatement of the documented grouping rule."""
+    n = len(lens)
+    full = [min(max(int(L), 0) // bs, bt.shape[1]) for L in lens]
+    runs, gap, i = [], None, 0
+    while i < n:
+        k, j = full[i], i + 1
+        while j < n and k >= 1:
+            c = 0
+            while c < min(k, full[j]) and bt[j, c] == bt[i, c]:
+                c += 1
+            if c < 1:
+                break
+            k, j = c, j + 1
+        if j - i >= min_size and k >= 1:
+            if gap is not None:
+                runs.append((gap, 0))
+                gap = None
+            runs.append((i, k * bs))
+            i = j
+        else:
+            gap = i if gap is None else gap
+            i += 1
+    if gap is not None:
+        runs.append((gap, 0))
+    return [r[0] for r in runs] + ([n] if runs else []), [r[1] for r in runs]
+
+
+def test_find_shared_prefix_groups_matches_rule():
+    import paged_kv_cache_405_b200 as pkv
+    for seed in range(400):
+        rng = np.random.default_rng(seed)
+        n, mb, bs = int(rng.integers(0, 14)), int(rng.integers(1, 7)), int(rng.choice([2, 4, 16]))
+        bt = rng.integers(0, 4, size=(n, mb)).astype(np.int32)   # few ids: many coincidences
+        lens = rng.integers(0, mb * bs + 1, size=n).astype(np.int32)
+        ms = int(rng.integers(2, 5))
+        gf, gs = pkv.find_shared_prefix_groups(bt, lens, bs, ms)
+        rf, rs = reference_groups(bt, lens, bs, ms)
+        assert gf.tolist() == rf and gs.tolist() == rs, seed
+
+
+def test_shared_prefix_layout_is_one_group():
+    import paged_kv_cache_405_b200 as pkv
+    b = synth.make_batch(synth.shrink(synth.CONFIGS["llama13b_prefix"], D=64, Hq=1, Hkv=1))
+    gf, gs = pkv.find_shared_prefix_groups(b.block_tables, b.lens, 16, 4)
+    assert gf.tolist() == [0, 256] and gs.tolist() == [512]
