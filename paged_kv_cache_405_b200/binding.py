@@ -17,7 +17,8 @@ import numpy as np
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
+# PKV_LIBRARY may name another build of the same library (e.g. other launch shapes).
+LIB_PATH = os.environ.get("PKV_LIBRARY") or os.path.join(_HERE, "libpagedkv.so")
 
 OK, INVALID, NO_FREE_BLOCK, CUDA_ERROR, UNSUPPORTED, DEVICE_CHECK = range(6)
 DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_CONTEXT, DEVERR_TIMEOUT = 1, 2, 4, 8

@@ -102,18 +102,24 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// A pool as a (rows x D) matrix of 16-bit elements; box = 64 elements x 16 rows,
-// 128-byte swizzle.
-static bool make_pool_map(CUtensorMap* map, const void* pool, int64_t rows, int D, pkv_dtype dt) {
+// A pool as a (rows x D) matrix.  swizzled: 16-bit elements, box = 64 elements
+// x 16 rows, 128-byte swizzle (tensor-core kernels).  Otherwise: box = D
+// elements x tile rows, no swizzle (a plain row-major copy of the tile).
+static bool make_pool_map(CUtensorMap* map, const void* pool, int64_t rows, int D, pkv_dtype dt, bool swizzled,
+                          int tile_rows = pkv::kTileTok) {
     auto fn = encode_fn();
     if (!fn) return false;
+    const int esz = elem_size(dt);
     cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    cuuint32_t box[2] = {64, (cuuint32_t)pkv::kTileTok};
+    cuuint64_t strides[1] = {(cuuint64_t)D * esz};
+    cuuint32_t box[2] = {swizzled ? 64u : (cuuint32_t)D, (cuuint32_t)(swizzled ? pkv::kTileTok : tile_rows)};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, dt == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2,
-                    const_cast<void*>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUtensorMapDataType ty = dt == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                   : dt == PKV_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
+                                                   : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    CUresult r = fn(map, ty, 2, const_cast<void*>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzled ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
@@ -123,16 +129,48 @@ static cudaError_t set_smem(Kern k, int bytes) {
     return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
 }
 
-constexpr int kSimtWarps = 4, kSimtStages = 3;
-constexpr int kMmaWarps = 4, kMmaStages = 3;
+// Launch shapes (warps per CTA, pipeline stages per warp); build-time tunables.
+#ifndef PKV_SIMT_WARPS
+#define PKV_SIMT_WARPS 4
+#endif
+#ifndef PKV_SIMT_STAGES
+#define PKV_SIMT_STAGES 2
+#endif
+#ifndef PKV_SIMT_TILE
+#define PKV_SIMT_TILE 16
+#endif
+#ifndef PKV_SIMT_TENSOR
+#define PKV_SIMT_TENSOR 0
+#endif
+#ifndef PKV_MMA_WARPS
+#define PKV_MMA_WARPS 4
+#endif
+#ifndef PKV_MMA_STAGES
+#define PKV_MMA_STAGES 2
+#endif
+constexpr int kSimtWarps = PKV_SIMT_WARPS, kSimtStages = PKV_SIMT_STAGES, kSimtTile = PKV_SIMT_TILE;
+constexpr int kMmaWarps = PKV_MMA_WARPS, kMmaStages = PKV_MMA_STAGES;
 
 template <typename T, int D>
 static cudaError_t launch_simt(const pkv::AttnParams& p, dim3 grid, cudaStream_t st) {
-    using C = pkv::SimtCfg<T, D, kSimtWarps, kSimtStages>;
-    auto k = pkv::paged_attn_simt_kernel<T, D, kSimtWarps, kSimtStages>;
+    using C = pkv::SimtCfg<T, D, kSimtWarps, kSimtStages, kSimtTile>;
+    constexpr bool kTensor = PKV_SIMT_TENSOR != 0;
+    auto k = pkv::paged_attn_simt_kernel<T, D, kSimtWarps, kSimtStages, kSimtTile, kTensor>;
     static cudaError_t attr = set_smem(k, C::kSmemBytes);
     if (attr != cudaSuccess) return attr;
-    k<<<grid, kSimtWarps * 32, C::kSmemBytes, st>>>(p);
+    CUtensorMap mk, mv;
+    if (kTensor) {
+        const pkv_dtype dt = std::is_same<T, float>::value ? PKV_F32
+                             : std::is_same<T, __half>::value ? PKV_F16 : PKV_BF16;
+        const int64_t rows = (int64_t)p.NB * p.Hkv * p.bs;
+        if (!make_pool_map(&mk, p.k_pool, rows, D, dt, false, kSimtTile) ||
+            !make_pool_map(&mv, p.v_pool, rows, D, dt, false, kSimtTile))
+            return cudaErrorInvalidValue;
+    } else {
+        std::memset(&mk, 0, sizeof mk);
+        std::memset(&mv, 0, sizeof mv);
+    }
+    k<<<grid, kSimtWarps * 32, C::kSmemBytes, st>>>(p, mk, mv);
     g_launches++;
     return cudaGetLastError();
 }
@@ -161,11 +199,13 @@ static cudaError_t launch_prefix(const pkv::AttnParams& p, dim3 grid, const CUte
     return cudaGetLastError();
 }
 
+// One CTA per (sequence, head); more warps when there are many partitions.
 template <typename T, int D>
 static cudaError_t launch_reduce(const pkv::ReduceParams& r, cudaStream_t st) {
-    const int warps = r.S * r.Hq;
-    const int blocks = (warps + 7) / 8;
-    pkv::splitk_reduce_kernel<T, D><<<blocks, 256, 0, st>>>(r);
+    const unsigned rows = (unsigned)(r.S * r.Hq);
+    if (r.maxP > 32) pkv::splitk_reduce_kernel<T, D, 8><<<rows, 256, 0, st>>>(r);
+    else if (r.maxP > 8) pkv::splitk_reduce_kernel<T, D, 4><<<rows, 128, 0, st>>>(r);
+    else pkv::splitk_reduce_kernel<T, D, 1><<<rows, 32, 0, st>>>(r);
     g_launches++;
     return cudaGetLastError();
 }
@@ -297,7 +337,7 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
     CUtensorMap mk, mv;
     if (use_mma || (grp.mode && grp.num > 0)) {
         const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
-        if (!make_pool_map(&mk, k_pool, rows, head_dim, dtype) || !make_pool_map(&mv, v_pool, rows, head_dim, dtype)) {
+        if (!make_pool_map(&mk, k_pool, rows, head_dim, dtype, true) || !make_pool_map(&mv, v_pool, rows, head_dim, dtype, true)) {
             g_msg = "pkv_paged_attention_decode: cuTensorMapEncodeTiled failed";
             return PKV_ERR_CUDA;
         }

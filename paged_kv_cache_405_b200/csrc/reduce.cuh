@@ -23,13 +23,22 @@ struct ReduceParams {
     int num_groups;
 };
 
-template <typename T, int D>
-__global__ void __launch_bounds__(256) splitk_reduce_kernel(const ReduceParams p) {
+// One CTA of W warps per (sequence, query head).  The partitions' maxima are
+// reduced first (M); then warp w sums the partitions w, w+W, ... scaled by
+// 2^(m_p - M), each lane owning D/32 columns, with several partitions' loads
+// in flight; the W partial sums are added in warp order through shared
+// memory, so the result does not depend on timing.
+template <typename T, int D, int W>
+__global__ void __launch_bounds__(W * 32) splitk_reduce_kernel(const ReduceParams p) {
     constexpr int kPerLane = D / 32;  // 2 or 4 floats
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    __shared__ float s_acc[W][D];
+    __shared__ float s_den[W];
+    __shared__ float s_max[W];
+    const int row = blockIdx.x;       // s * Hq + h
+    const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    if (warp >= p.S * p.Hq) return;
-    const int s = warp / p.Hq;
+    if (row >= p.S * p.Hq) return;
+    const int s = row / p.Hq;
     int L = p.context_lens[s];
     if (L < 0) L = 0;
     if (L > p.max_len) L = p.max_len;
@@ -49,36 +58,73 @@ __global__ void __launch_bounds__(256) splitk_reduce_kernel(const ReduceParams p
     const int nsuf = (L - shared + p.P - 1) / p.P;
     const int nP = (shared + p.P - 1) / p.P + nsuf;
     if (shared == 0 && nP <= 1) return;  // written directly by the attention kernel
-    const int64_t base = (int64_t)warp * p.maxP;
+    const int64_t base = (int64_t)row * p.maxP;
     const float* ml = p.ws_ml + base * 2;
+
     float M = -INFINITY;
-    for (int i = lane; i < nP; i += 32) M = fmaxf(M, ml[2 * i]);
+    for (int i = threadIdx.x; i < nP; i += W * 32) M = fmaxf(M, ml[2 * i]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    if (lane == 0) s_max[warp] = M;
+    __syncthreads();
+    M = s_max[0];
+#pragma unroll
+    for (int w = 1; w < W; ++w) M = fmaxf(M, s_max[w]);
+
     float acc[kPerLane];
 #pragma unroll
     for (int k = 0; k < kPerLane; ++k) acc[k] = 0.f;
     float den = 0.f;
     const float* o = p.ws_o + base * D + lane * kPerLane;
-    for (int i = 0; i < nP; ++i) {
-        const float w = ex2(ml[2 * i] - M);
-        den += w * ml[2 * i + 1];
-        if constexpr (kPerLane == 4) {
-            float4 v = *reinterpret_cast<const float4*>(o + (int64_t)i * D);
-            acc[0] += w * v.x;
-            acc[1] += w * v.y;
-            acc[2] += w * v.z;
-            acc[3] += w * v.w;
-        } else {
-            float2 v = *reinterpret_cast<const float2*>(o + (int64_t)i * D);
-            acc[0] += w * v.x;
-            acc[1] += w * v.y;
+    constexpr int U = 4;  // partitions per batch of loads
+    for (int i0 = warp; i0 < nP; i0 += W * U) {
+        float wt[U], lp[U], v[U][kPerLane];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = i0 + u * W;
+            if (i < nP) {
+                const float2 m_l = *reinterpret_cast<const float2*>(ml + 2 * i);
+                wt[u] = m_l.x;
+                lp[u] = m_l.y;
+                if constexpr (kPerLane == 4) {
+                    const float4 x = *reinterpret_cast<const float4*>(o + (int64_t)i * D);
+                    v[u][0] = x.x; v[u][1] = x.y; v[u][2] = x.z; v[u][3] = x.w;
+                } else {
+                    const float2 x = *reinterpret_cast<const float2*>(o + (int64_t)i * D);
+                    v[u][0] = x.x; v[u][1] = x.y;
+                }
+            } else {
+                wt[u] = -INFINITY;
+                lp[u] = 0.f;
+#pragma unroll
+                for (int k = 0; k < kPerLane; ++k) v[u][k] = 0.f;
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const float w = ex2(wt[u] - M);
+            den += w * lp[u];
+#pragma unroll
+            for (int k = 0; k < kPerLane; ++k) acc[k] += w * v[u][k];
         }
     }
-    const float inv = 1.f / den;
-    T* dst = reinterpret_cast<T*>(p.out) + (int64_t)warp * D + lane * kPerLane;
 #pragma unroll
-    for (int k = 0; k < kPerLane; ++k) dst[k] = static_cast<T>(acc[k] * inv);
+    for (int k = 0; k < kPerLane; ++k) s_acc[warp][lane * kPerLane + k] = acc[k];
+    if (lane == 0) s_den[warp] = den;
+    __syncthreads();
+    if (warp != 0) return;
+    float tot = s_den[0];
+#pragma unroll
+    for (int w = 1; w < W; ++w) tot += s_den[w];
+    const float inv = 1.f / tot;
+    T* dst = reinterpret_cast<T*>(p.out) + (int64_t)row * D + lane * kPerLane;
+#pragma unroll
+    for (int k = 0; k < kPerLane; ++k) {
+        float a = s_acc[0][lane * kPerLane + k];
+#pragma unroll
+        for (int w = 1; w < W; ++w) a += s_acc[w][lane * kPerLane + k];
+        dst[k] = static_cast<T>(a * inv);
+    }
 }
 
 }  // namespace pkv
