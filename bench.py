@@ -294,9 +294,16 @@ def barrier(world):
         torch.distributed.barrier()
 
 
+def workload_shape(args):
+    shape = synth.CONFIGS[args.config]
+    if args.batch:
+        shape = synth.shrink(shape, S=args.batch)
+    return shape
+
+
 def run_ours(args, world, rank, local):
     import paged_kv_cache_405_b200 as pkv
-    shape = synth.CONFIGS[args.config]
+    shape = workload_shape(args)
     dev = torch.device("cuda", local)
     wl = Workload(shape, shape.seed + rank, dev, args.partition_size)
     ss = wl.session
@@ -396,7 +403,8 @@ def run_ours(args, world, rank, local):
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": round(ms_max / K, 4), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic (seeded N(0,1) K/V/q; pages' workload shapes)",
-            "config": {"workload": args.config, "description": shape.description, "batch": shape.S,
+            "config": {"workload": args.config + ("" if not args.batch else "@batch%d" % args.batch),
+                       "description": shape.description, "batch": shape.S,
                        "q_heads": shape.Hq, "kv_heads": shape.Hkv, "head_dim": shape.D, "block_size": shape.bs,
                        "partition_size": wl_P(shape, args), "effective_partition_size": eff_P_of(shape, args, plans),
                        "mean_context": round(float(plans[W].lens.float().mean().item()), 1),
@@ -502,7 +510,7 @@ def run_reference(args, world, rank):
     """The CPU oracle as the reference arm: each step is a bounded sample of the workload."""
     if rank != 0:
         return None
-    shape = synth.CONFIGS[args.config]
+    shape = workload_shape(args)
     batch = synth.make_batch(shape, device="cpu")
     per = max(0.5, args.reference_step_seconds)
     for _ in range(args.warmup):
@@ -534,6 +542,8 @@ def main(argv=None):
     ap.add_argument("--config", default="llama7b", choices=sorted(synth.CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--partition-size", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch size (small cases for profiling)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

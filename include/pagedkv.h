@@ -157,6 +157,9 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_po
  *                 members are then handled as non-members.
  *   max_group_size  host bound on members per group (PKV_DEVERR_GROUP if a
  *                 group is larger; its extra members get no prefix result).
+ *   max_shared_len  host bound on every group_shared[g] (it sizes the prefix
+ *                 pass; a larger group_shared is recorded as PKV_DEVERR_GROUP
+ *                 and its tokens past the bound get no prefix result).
  *   workspace     >= pkv_attention_shared_workspace_bytes(...) bytes.
  * 16-bit element types only (PKV_ERR_UNSUPPORTED for fp32).
  */
@@ -166,8 +169,8 @@ pkv_status pkv_paged_attention_decode_shared(void* out, const void* q, const voi
                                              int num_kv_heads, int head_dim, int block_size, int num_blocks,
                                              float scale, int partition_size, const int32_t* group_first,
                                              const int32_t* group_shared, int num_groups, int max_group_size,
-                                             void* workspace, size_t workspace_bytes, pkv_dtype dtype,
-                                             void* stream);
+                                             int max_shared_len, void* workspace, size_t workspace_bytes,
+                                             pkv_dtype dtype, void* stream);
 
 /* Workspace bytes for pkv_paged_attention_decode_shared (arguments as in
  * pkv_attention_workspace_bytes; never 0 for num_seqs > 0). */

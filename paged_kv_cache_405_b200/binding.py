@@ -59,7 +59,7 @@ def _load():
                                                       c_vp]),
         "pkv_paged_attention_decode_shared": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_vp, c_int, c_int,
                                                       c_int, c_int, c_int, c_int, ctypes.c_float, c_int, c_vp,
-                                                      c_vp, c_int, c_int, c_vp, c_sz, c_int, c_vp]),
+                                                      c_vp, c_int, c_int, c_int, c_vp, c_sz, c_int, c_vp]),
         "pkv_attention_shared_workspace_bytes": (c_sz, [c_int, c_int, c_int, c_int, c_int]),
         "pkv_find_shared_prefix_groups": (c_int, [c_vp, c_vp, c_int, c_int, c_int, c_int, c_vp, c_vp, c_int,
                                                   ctypes.POINTER(c_int)]),
@@ -213,9 +213,11 @@ def find_shared_prefix_groups(block_tables: np.ndarray, context_lens: np.ndarray
 
 
 def paged_attention_decode_shared(out, q, k_pool, v_pool, block_tables, context_lens, group_first, group_shared,
-                                  max_group_size: int, scale: float = 0.0, partition_size: int = 0,
-                                  workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """Decode attention with shared-prefix groups (device int32 group_first [n+1], group_shared [n])."""
+                                  max_group_size: int, max_shared_len: int, scale: float = 0.0,
+                                  partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
+                                  stream=None) -> torch.Tensor:
+    """Decode attention with shared-prefix groups (device int32 group_first [n+1], group_shared [n];
+    host bounds max_group_size and max_shared_len)."""
     S, Hq, D = q.shape
     NB, Hkv, bs, D2 = k_pool.shape
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
@@ -229,7 +231,8 @@ def paged_attention_decode_shared(out, q, k_pool, v_pool, block_tables, context_
         _dev(out, "out"), _dev(q, "q"), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
         _dev(block_tables, "block_tables"), maxB, _dev(context_lens, "context_lens"), S, Hq, Hkv, D, bs, NB,
         float(scale), int(partition_size), _dev(group_first, "group_first") if n else None,
-        _dev(group_shared, "group_shared") if n else None, n, int(max_group_size), _dev(workspace, "workspace"),
+        _dev(group_shared, "group_shared") if n else None, n, int(max_group_size), int(max_shared_len),
+        _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _dt(q), _stream(stream)))
     return out
 

@@ -25,6 +25,7 @@ struct AttnParams {
     const int32_t* group_shared;  // [num_groups]
     int num_groups;
     int max_group_size;           // prefix-pass grid covers groups up to this many sequences
+    int max_shared;               // ... and shared runs up to this many tokens
 };
 
 // Which tokens one (sequence, partition) unit covers and where its result goes.
@@ -56,6 +57,10 @@ __device__ __forceinline__ int group_shared_len(const AttnParams& p, int gi, int
     const int sh = p.group_shared[gi];
     if (sh < 0 || sh % p.bs != 0 || sh > L) {
         if (report) flag_error(4u /* PKV_DEVERR_CONTEXT */);
+        return -1;
+    }
+    if (sh > p.max_shared) {
+        if (report) flag_error(16u /* PKV_DEVERR_GROUP */);
         return -1;
     }
     return sh;

@@ -311,16 +311,22 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnPa
     }
 }
 
-// Shared-prefix pass: grid (row-tile blocks, prefix partitions, groups * Hkv).
-// Row r of group i is (sequence group_first[i] + r / G, query head g*G + r % G).
+// Shared-prefix pass: grid (row tiles, prefix partitions, groups * Hkv).  Row r
+// of group i is (sequence group_first[i] + r / G, query head g*G + r % G).
+// The WARPS warps of a CTA split the partition's tokens of one 16-row tile
+// (so each warp's chain of dependent tile loads is short), then merge their
+// (m, l, o) in shared memory into the single partial of that partition.
 template <typename T, int D, int WARPS, int STAGES>
 __global__ void __launch_bounds__(WARPS * 32) prefix_attn_mma_kernel(const AttnParams p,
                                                                      const __grid_constant__ CUtensorMap tmK,
                                                                      const __grid_constant__ CUtensorMap tmV) {
+    using C = MmaCfg<T, D, WARPS, STAGES>;
+    constexpr int NT_O = D / 8;
+    static_assert(WARPS * 16 * (D + 2) * 4 <= C::kDataBytes, "merge buffer must fit in the ring");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int tile = blockIdx.x * WARPS + warp;
+    const int tile = blockIdx.x;
     const int pp = blockIdx.y;  // partition of the shared tokens
     const int gi = blockIdx.z / p.Hkv;
     const int g = blockIdx.z - gi * p.Hkv;
@@ -331,16 +337,20 @@ __global__ void __launch_bounds__(WARPS * 32) prefix_attn_mma_kernel(const AttnP
     first = max(0, min(first, p.S));
     last = max(first, min(last, p.S));
     if (last - first > p.max_group_size) {
-        if (tile == 0 && pp == 0 && g == 0 && lane == 0) flag_error(16u /* PKV_DEVERR_GROUP */);
+        if (tile == 0 && pp == 0 && g == 0 && threadIdx.x == 0) flag_error(16u /* PKV_DEVERR_GROUP */);
         last = first + p.max_group_size;  // members past the grid get no prefix partials
     }
     const int rows = (last - first) * G;
     if (tile * 16 >= rows) return;
     const int shared = p.group_shared[gi];
-    if (shared <= 0 || shared % p.bs != 0 || shared > p.max_len) return;  // reported by the decode kernels
-    const int t_begin = pp * p.P;
-    if (t_begin >= shared) return;
-    const int t_end = min(shared, t_begin + p.P);
+    if (shared <= 0 || shared % p.bs != 0 || shared > p.max_len || shared > p.max_shared)
+        return;  // reported by the decode kernels
+    const int t0 = pp * p.P;
+    if (t0 >= shared) return;
+    const int t1 = min(shared, t0 + p.P);
+    // This warp's share of [t0, t1), in whole 16-token tiles.
+    const int per = ((t1 - t0 + WARPS * kTileTok - 1) / (WARPS * kTileTok)) * kTileTok;
+    const int w0 = min(t1, t0 + warp * per), w1 = min(t1, w0 + per);
 
     // Query rows of this lane (gid, gid+8); a member whose context is shorter
     // than the shared run is not a member (the decode kernels report it).
@@ -363,15 +373,70 @@ __global__ void __launch_bounds__(WARPS * 32) prefix_attn_mma_kernel(const AttnP
     MmaAcc<T, D> acc;
     acc.load_q(use[0] ? q + ((int64_t)rs[0] * p.Hq + rh[0]) * D : nullptr,
                use[1] ? q + ((int64_t)rs[1] * p.Hq + rh[1]) * D : nullptr, tig);
-    if (!mma_attend<T, D, WARPS, STAGES>(p, &tmK, &tmV, ring, bar0, p.block_tables + (int64_t)first * p.maxB,
-                                         t_begin, t_end, g, lane, acc))
-        return;
+    bool ok = true;
+    if (w0 < w1)
+        ok = mma_attend<T, D, WARPS, STAGES>(p, &tmK, &tmV, ring, bar0, p.block_tables + (int64_t)first * p.maxB,
+                                             w0, w1, g, lane, acc);
+    const int all_ok = __syncthreads_and(ok ? 1 : 0);  // every warp is done with its ring
+
+    // Merge buffer (reuses the rings): o [WARPS][16][D], then m, l [WARPS][16].
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    float* so = reinterpret_cast<float*>(base);
+    float* sm = so + WARPS * 16 * D;
+    float* sl = sm + WARPS * 16;
 #pragma unroll
-    for (int hi = 0; hi < 2; ++hi) {
-        if (!use[hi]) continue;
-        const int64_t idx = ((int64_t)rs[hi] * p.Hq + rh[hi]) * p.maxP + pp;
-        mma_store_row<T, D>(acc, hi, tig, nullptr, p.ws_o + idx * D, p.ws_ml + idx * 2);
+    for (int j = 0; j < NT_O; ++j) {
+        const int col = j * 8 + 2 * tig;
+        *reinterpret_cast<float2*>(so + (warp * 16 + gid) * D + col) = make_float2(acc.o[j][0], acc.o[j][1]);
+        *reinterpret_cast<float2*>(so + (warp * 16 + gid + 8) * D + col) = make_float2(acc.o[j][2], acc.o[j][3]);
     }
+    if (tig == 0) {
+        sm[warp * 16 + gid] = acc.m_lo;
+        sm[warp * 16 + gid + 8] = acc.m_hi;
+        sl[warp * 16 + gid] = acc.l_lo;
+        sl[warp * 16 + gid + 8] = acc.l_hi;
+    }
+    __syncthreads();
+    if (!all_ok) return;
+    // Thread t merges row t / (WARPS*2) ... : 16 rows x D columns over the CTA.
+    constexpr int kThreads = WARPS * 32;
+    constexpr int kPerRow = kThreads / 16;   // threads per row
+    constexpr int kCols = D / kPerRow;       // columns per thread
+    static_assert(kCols % 4 == 0, "float4 columns");
+    const int r = threadIdx.x / kPerRow;
+    const int c0 = (threadIdx.x % kPerRow) * kCols;
+    const int rr = tile * 16 + r;
+    if (rr >= rows) return;
+    const int s_r = first + rr / G, h_r = g * G + rr % G;
+    {
+        const int L = min(max(p.context_lens[s_r], 0), p.max_len);
+        if (L < shared) return;
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) M = fmaxf(M, sm[w * 16 + r]);
+    float f[WARPS], lsum = 0.f;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) {
+        f[w] = ex2(sm[w * 16 + r] - M);  // 0 for a warp that saw no token
+        lsum += f[w] * sl[w * 16 + r];
+    }
+    const int64_t idx = ((int64_t)s_r * p.Hq + h_r) * p.maxP + pp;
+    float* dst = p.ws_o + idx * D + c0;
+#pragma unroll
+    for (int cc = 0; cc < kCols; cc += 4) {
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < WARPS; ++w) {
+            const float4 v = *reinterpret_cast<const float4*>(so + (w * 16 + r) * D + c0 + cc);
+            a.x += f[w] * v.x;
+            a.y += f[w] * v.y;
+            a.z += f[w] * v.z;
+            a.w += f[w] * v.w;
+        }
+        *reinterpret_cast<float4*>(dst + cc) = a;
+    }
+    if (c0 == 0) *reinterpret_cast<float2*>(p.ws_ml + idx * 2) = make_float2(M, lsum);
 }
 
 }  // namespace pkv

@@ -150,6 +150,11 @@ static cudaError_t set_smem(Kern k, int bytes) {
 #endif
 constexpr int kSimtWarps = PKV_SIMT_WARPS, kSimtStages = PKV_SIMT_STAGES, kSimtTile = PKV_SIMT_TILE;
 constexpr int kMmaWarps = PKV_MMA_WARPS, kMmaStages = PKV_MMA_STAGES;
+// Ring depth of the shared-prefix pass.
+#ifndef PKV_PREFIX_STAGES
+#define PKV_PREFIX_STAGES 2
+#endif
+constexpr int kPrefixStages = PKV_PREFIX_STAGES;
 
 template <typename T, int D>
 static cudaError_t launch_simt(const pkv::AttnParams& p, dim3 grid, cudaStream_t st) {
@@ -190,8 +195,8 @@ static cudaError_t launch_mma(const pkv::AttnParams& p, dim3 grid, const CUtenso
 template <typename T, int D>
 static cudaError_t launch_prefix(const pkv::AttnParams& p, dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv,
                                  cudaStream_t st) {
-    using C = pkv::MmaCfg<T, D, kMmaWarps, kMmaStages>;
-    auto k = pkv::prefix_attn_mma_kernel<T, D, kMmaWarps, kMmaStages>;
+    using C = pkv::MmaCfg<T, D, kMmaWarps, kPrefixStages>;
+    auto k = pkv::prefix_attn_mma_kernel<T, D, kMmaWarps, kPrefixStages>;
     static cudaError_t attr = set_smem(k, C::kSmemBytes);
     if (attr != cudaSuccess) return attr;
     k<<<grid, kMmaWarps * 32, C::kSmemBytes, st>>>(p, mk, mv);
@@ -199,27 +204,28 @@ static cudaError_t launch_prefix(const pkv::AttnParams& p, dim3 grid, const CUte
     return cudaGetLastError();
 }
 
-// One CTA per (sequence, head); more warps when there are many partitions.
+// Many partitions: 8 warps on each (sequence, head); few: 8 rows per CTA,
+// one warp each.
 template <typename T, int D>
 static cudaError_t launch_reduce(const pkv::ReduceParams& r, cudaStream_t st) {
     const unsigned rows = (unsigned)(r.S * r.Hq);
-    if (r.maxP > 32) pkv::splitk_reduce_kernel<T, D, 8><<<rows, 256, 0, st>>>(r);
-    else if (r.maxP > 8) pkv::splitk_reduce_kernel<T, D, 4><<<rows, 128, 0, st>>>(r);
-    else pkv::splitk_reduce_kernel<T, D, 1><<<rows, 32, 0, st>>>(r);
+    if (r.maxP > 32) pkv::splitk_reduce_kernel<T, D, 8, 1><<<rows, 256, 0, st>>>(r);
+    else pkv::splitk_reduce_kernel<T, D, 1, 8><<<(rows + 7) / 8, 256, 0, st>>>(r);
     g_launches++;
     return cudaGetLastError();
 }
 
 template <typename T>
-static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int nparts, bool use_mma, bool shared_mode,
-                                      const CUtensorMap* mk, const CUtensorMap* mv, cudaStream_t st) {
+static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int nparts, int npre, bool use_mma,
+                                      bool shared_mode, const CUtensorMap* mk, const CUtensorMap* mv,
+                                      cudaStream_t st) {
     cudaError_t e = cudaSuccess;
     if constexpr (std::is_same<T, float>::value) {
         if (use_mma || shared_mode) return cudaErrorInvalidValue;
     } else {
-        if (shared_mode && p.num_groups > 0) {
+        if (shared_mode && p.num_groups > 0 && npre > 0) {
             const int tiles = (p.max_group_size * p.G + 15) / 16;
-            dim3 grid((tiles + kMmaWarps - 1) / kMmaWarps, nparts, p.num_groups * p.Hkv);
+            dim3 grid(tiles, npre, p.num_groups * p.Hkv);
             e = D == 64 ? launch_prefix<T, 64>(p, grid, *mk, *mv, st) : launch_prefix<T, 128>(p, grid, *mk, *mv, st);
             if (e != cudaSuccess) return e;
         }
@@ -234,7 +240,7 @@ static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int npart
     }
     if (e != cudaSuccess || p.maxP <= 1) return e;
     pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
-                        p.group_first, p.group_shared, p.num_groups};
+                        p.group_first, p.group_shared, p.num_groups, p.max_shared};
     return D == 64 ? launch_reduce<T, 64>(r, st) : launch_reduce<T, 128>(r, st);
 }
 
@@ -243,7 +249,8 @@ struct GroupArgs {
     const int32_t* shared = nullptr;
     int num = 0;
     int max_size = 0;
-    bool mode = false;  // called through the shared-prefix entry point
+    int max_shared = 0;  // host bound on group_shared (sizes the prefix grid)
+    bool mode = false;   // called through the shared-prefix entry point
 };
 
 static pkv_status decode_impl(void* out, const void* q, const void* k_pool, const void* v_pool,
@@ -284,6 +291,8 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
             return invalid("pkv_paged_attention_decode_shared: num_groups * num_kv_heads must be <= 65535");
         if ((int64_t)grp.max_size * (num_q_heads / num_kv_heads) > ((int64_t)1 << 24))
             return invalid("pkv_paged_attention_decode_shared: max_group_size too large");
+        if (grp.num > 0 && (grp.max_shared < 0 || grp.max_shared > max_len64))
+            return invalid("pkv_paged_attention_decode_shared: max_shared_len must be in [0, max_blocks_per_seq*block_size]");
     }
     if (num_seqs == 0) return PKV_OK;
     if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens)
@@ -332,6 +341,7 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
     p.group_shared = grp.num > 0 ? grp.shared : nullptr;
     p.num_groups = grp.num;
     p.max_group_size = grp.max_size;
+    p.max_shared = grp.max_shared;
 
     const bool use_mma = dtype != PKV_F32 && p.G >= 2 && p.G <= 16;
     CUtensorMap mk, mv;
@@ -343,13 +353,18 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
         }
     }
     cudaStream_t st = (cudaStream_t)stream;
+    const int npre = (grp.max_shared + P - 1) / P;  // partitions of the longest shared run
     cudaError_t e;
     switch (dtype) {
-        case PKV_F32: e = dispatch_attention<float>(p, head_dim, (int)nparts, false, false, nullptr, nullptr, st); break;
-        case PKV_BF16:
-            e = dispatch_attention<__nv_bfloat16>(p, head_dim, (int)nparts, use_mma, grp.mode, &mk, &mv, st);
+        case PKV_F32:
+            e = dispatch_attention<float>(p, head_dim, (int)nparts, 0, false, false, nullptr, nullptr, st);
             break;
-        default: e = dispatch_attention<__half>(p, head_dim, (int)nparts, use_mma, grp.mode, &mk, &mv, st); break;
+        case PKV_BF16:
+            e = dispatch_attention<__nv_bfloat16>(p, head_dim, (int)nparts, npre, use_mma, grp.mode, &mk, &mv, st);
+            break;
+        default:
+            e = dispatch_attention<__half>(p, head_dim, (int)nparts, npre, use_mma, grp.mode, &mk, &mv, st);
+            break;
     }
     return e == cudaSuccess ? PKV_OK : cuda_fail("pkv_paged_attention_decode", e);
 }
@@ -442,13 +457,14 @@ pkv_status pkv_paged_attention_decode_shared(void* out, const void* q, const voi
                                              int num_kv_heads, int head_dim, int block_size, int num_blocks,
                                              float scale, int partition_size, const int32_t* group_first,
                                              const int32_t* group_shared, int num_groups, int max_group_size,
-                                             void* workspace, size_t workspace_bytes, pkv_dtype dtype,
-                                             void* stream) {
+                                             int max_shared_len, void* workspace, size_t workspace_bytes,
+                                             pkv_dtype dtype, void* stream) {
     GroupArgs g;
     g.first = group_first;
     g.shared = group_shared;
     g.num = num_groups;
     g.max_size = max_group_size;
+    g.max_shared = max_shared_len;
     g.mode = true;
     return decode_impl(out, q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads,
                        num_kv_heads, head_dim, block_size, num_blocks, scale, partition_size, g, workspace,

@@ -20,24 +20,35 @@ struct ReduceParams {
     int S, Hq, D, P, maxP, max_len, bs;
     const int32_t* group_first;   // shared-prefix groups, as in AttnParams
     const int32_t* group_shared;
-    int num_groups;
+    int num_groups, max_shared;
 };
 
-// One CTA of W warps per (sequence, query head).  The partitions' maxima are
-// reduced first (M); then warp w sums the partitions w, w+W, ... scaled by
-// 2^(m_p - M), each lane owning D/32 columns, with several partitions' loads
-// in flight; the W partial sums are added in warp order through shared
-// memory, so the result does not depend on timing.
-template <typename T, int D, int W>
-__global__ void __launch_bounds__(W * 32) splitk_reduce_kernel(const ReduceParams p) {
+// A CTA handles ROWS (sequence, query head) rows with W warps each.  The
+// partitions' maxima are reduced first (M); then warp w of a row sums the
+// partitions w, w+W, ... scaled by 2^(m_p - M), each lane owning D/32
+// columns, with several partitions' loads in flight; the W partial sums are
+// added in warp order through shared memory, so the result does not depend
+// on timing.
+// Barrier over the W warps of one row (named barrier 1 + row; W > 1 only).
+template <int W>
+__device__ __forceinline__ void row_sync(int row_in_cta) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + row_in_cta), "r"(W * 32) : "memory");
+}
+
+template <typename T, int D, int W, int ROWS>
+__global__ void __launch_bounds__(W * ROWS * 32) splitk_reduce_kernel(const ReduceParams p) {
     constexpr int kPerLane = D / 32;  // 2 or 4 floats
-    __shared__ float s_acc[W][D];
-    __shared__ float s_den[W];
-    __shared__ float s_max[W];
-    const int row = blockIdx.x;       // s * Hq + h
-    const int warp = threadIdx.x >> 5;
+    __shared__ float s_acc_all[ROWS][W][D];
+    __shared__ float s_den_all[ROWS][W];
+    __shared__ float s_max_all[ROWS][W];
+    const int sub = threadIdx.x / (W * 32);  // row of this CTA
+    const int row = blockIdx.x * ROWS + sub;  // s * Hq + h
+    const int warp = (threadIdx.x >> 5) % W;
     const int lane = threadIdx.x & 31;
-    if (row >= p.S * p.Hq) return;
+    float (&s_acc)[W][D] = s_acc_all[sub];
+    float (&s_den)[W] = s_den_all[sub];
+    float (&s_max)[W] = s_max_all[sub];
+    if (row >= p.S * p.Hq) return;  // whole rows return together (W warps of a row)
     const int s = row / p.Hq;
     int L = p.context_lens[s];
     if (L < 0) L = 0;
@@ -53,7 +64,7 @@ __global__ void __launch_bounds__(W * 32) splitk_reduce_kernel(const ReduceParam
             else hi = mid;
         }
         const int sh = p.group_shared[lo];
-        if (sh > 0 && sh % p.bs == 0 && sh <= L) shared = sh;
+        if (sh > 0 && sh % p.bs == 0 && sh <= L && sh <= p.max_shared) shared = sh;
     }
     const int nsuf = (L - shared + p.P - 1) / p.P;
     const int nP = (shared + p.P - 1) / p.P + nsuf;
@@ -62,14 +73,16 @@ __global__ void __launch_bounds__(W * 32) splitk_reduce_kernel(const ReduceParam
     const float* ml = p.ws_ml + base * 2;
 
     float M = -INFINITY;
-    for (int i = threadIdx.x; i < nP; i += W * 32) M = fmaxf(M, ml[2 * i]);
+    for (int i = warp * 32 + lane; i < nP; i += W * 32) M = fmaxf(M, ml[2 * i]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    if (lane == 0) s_max[warp] = M;
-    __syncthreads();
-    M = s_max[0];
+    if (W > 1) {
+        if (lane == 0) s_max[warp] = M;
+        row_sync<W>(sub);
+        M = s_max[0];
 #pragma unroll
-    for (int w = 1; w < W; ++w) M = fmaxf(M, s_max[w]);
+        for (int w = 1; w < W; ++w) M = fmaxf(M, s_max[w]);
+    }
 
     float acc[kPerLane];
 #pragma unroll
@@ -108,11 +121,18 @@ __global__ void __launch_bounds__(W * 32) splitk_reduce_kernel(const ReduceParam
             for (int k = 0; k < kPerLane; ++k) acc[k] += w * v[u][k];
         }
     }
+    if (W > 1) {
 #pragma unroll
-    for (int k = 0; k < kPerLane; ++k) s_acc[warp][lane * kPerLane + k] = acc[k];
-    if (lane == 0) s_den[warp] = den;
-    __syncthreads();
-    if (warp != 0) return;
+        for (int k = 0; k < kPerLane; ++k) s_acc[warp][lane * kPerLane + k] = acc[k];
+        if (lane == 0) s_den[warp] = den;
+        row_sync<W>(sub);
+        if (warp != 0) return;
+    } else {
+#pragma unroll
+        for (int k = 0; k < kPerLane; ++k) s_acc[0][lane * kPerLane + k] = acc[k];
+        if (lane == 0) s_den[0] = den;
+        __syncwarp();
+    }
     float tot = s_den[0];
 #pragma unroll
     for (int w = 1; w < W; ++w) tot += s_den[w];

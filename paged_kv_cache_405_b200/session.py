@@ -36,6 +36,7 @@ class StepPlan:
     group_first: np.ndarray = None   # int32 [g + 1] shared-prefix runs (see find_shared_prefix_groups)
     group_shared: np.ndarray = None  # int32 [g]
     max_group_size: int = 0
+    max_shared_len: int = 0
 
     @property
     def has_groups(self) -> bool:
@@ -52,6 +53,7 @@ class DevicePlan:
     group_first: Optional[torch.Tensor] = None
     group_shared: Optional[torch.Tensor] = None
     max_group_size: int = 0
+    max_shared_len: int = 0
 
 
 class DecodeSession:
@@ -122,6 +124,7 @@ class DecodeSession:
             if (gs > 0).any():
                 plan.group_first, plan.group_shared = gf, gs
                 plan.max_group_size = int(np.diff(gf).max())
+                plan.max_shared_len = int(gs.max())
         return plan
 
     def to_device(self, p: StepPlan, non_blocking: bool = False) -> DevicePlan:
@@ -133,7 +136,8 @@ class DecodeSession:
                        torch.zeros((0, 2), dtype=torch.int32, device=dev),
                        up(p.lens), up(p.block_tables), len(p.cow_pairs))
         if p.has_groups:
-            d.group_first, d.group_shared, d.max_group_size = up(p.group_first), up(p.group_shared), p.max_group_size
+            d.group_first, d.group_shared = up(p.group_first), up(p.group_shared)
+            d.max_group_size, d.max_shared_len = p.max_group_size, p.max_shared_len
         return d
 
     # ---------------------------------------------------------- device side
@@ -149,7 +153,7 @@ class DecodeSession:
         """The step's attention: the shared-prefix call when the plan found groups."""
         if d.group_shared is not None:
             B.paged_attention_decode_shared(out, q, self.k_pool, self.v_pool, d.block_tables, d.lens,
-                                            d.group_first, d.group_shared, d.max_group_size,
+                                            d.group_first, d.group_shared, d.max_group_size, d.max_shared_len,
                                             partition_size=self.partition_size, workspace=self.workspace,
                                             stream=stream)
         else:
@@ -190,7 +194,7 @@ class DecodeSession:
         if p.has_groups:
             d.group_first = self._h2d("gfirst", p.group_first)
             d.group_shared = self._h2d("gshared", p.group_shared)
-            d.max_group_size = p.max_group_size
+            d.max_group_size, d.max_shared_len = p.max_group_size, p.max_shared_len
         return d
 
     def _h2d(self, name, a: np.ndarray) -> torch.Tensor:

@@ -21,13 +21,14 @@ def pkv():
     return m
 
 
-def run_shared(batch, gf, gs, P=0, max_group=None):
+def run_shared(batch, gf, gs, P=0, max_group=None, max_shared=None):
     d = to_dev(batch)
     out = torch.full_like(d["q"], float("nan"))
     gft = torch.as_tensor(np.asarray(gf, np.int32)).cuda()
     gst = torch.as_tensor(np.asarray(gs, np.int32)).cuda()
     mg = int(np.diff(gf).max()) if max_group is None else max_group
-    pkv().paged_attention_decode_shared(out, d["q"], d["k"], d["v"], d["bt"], d["cl"], gft, gst, mg,
+    ms = int(np.max(gs)) if max_shared is None else max_shared
+    pkv().paged_attention_decode_shared(out, d["q"], d["k"], d["v"], d["bt"], d["cl"], gft, gst, mg, ms,
                                         partition_size=P)
     return out
 
@@ -137,3 +138,11 @@ def test_session_uses_groups_for_the_prefix_workload():
     ref = oracle.paged_attention(b.q, kc, vc, plan.block_tables, plan.lens)
     assert m.device_error() == 0
     assert max_err(out, ref) <= TOL[out.dtype]
+
+
+def test_shared_run_longer_than_declared_is_reported():
+    b = mixed_batch(seed=8)
+    out = run_shared(b, [0, 6, 9, 16], [256, 0, 128], 0, max_shared=128)
+    assert pkv().device_error() & 16
+    # the group over the bound is handled without the prefix pass: still right
+    assert max_err(out, oracle_attention(b)) <= TOL[out.dtype]
