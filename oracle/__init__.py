@@ -44,6 +44,13 @@ def _load():
         lib.oracle_slot.restype = ctypes.c_int64
         lib.oracle_slot.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64]
         lib.oracle_max_threads.restype = ctypes.c_int
+        lib.oracle_paged_attention_chunk.restype = ctypes.c_int
+        lib.oracle_paged_attention_chunk.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_double, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int]
         _lib = lib
     return _lib
 
@@ -101,6 +108,43 @@ def paged_attention(q, k_pool, v_pool, block_tables, context_lens, scale=None,
     if items is None:
         return out.reshape(S, Hq, D)
     return out
+
+
+def paged_attention_chunk(q, k_pool, v_pool, block_tables, context_lens, query_start, scale=None,
+                          items=None, threads: int = 1) -> np.ndarray:
+    """fp64 causal attention of a chunk of new tokens per sequence.
+
+    q ``[T, Hq, D]``: rows ``query_start[s] .. query_start[s+1]-1`` are the
+    last tokens of sequence s's ``context_lens[s]`` cached tokens; each attends
+    to the cache up to and including its own position.  Returns ``[T, Hq, D]``
+    or ``[len(items), D]`` for (row, head) ``items``.
+    """
+    q, k_pool, v_pool = _cpu(q), _cpu(k_pool), _cpu(v_pool)
+    if not (q.dtype == k_pool.dtype == v_pool.dtype) or q.dtype not in _DT:
+        raise TypeError("q and pools must share one of fp32/bf16/f16")
+    T, Hq, D = q.shape
+    NB, Hkv, bs, _ = k_pool.shape
+    bt = np.ascontiguousarray(np.asarray(block_tables, dtype=np.int32))
+    cl = np.ascontiguousarray(np.asarray(context_lens, dtype=np.int32))
+    qs = np.ascontiguousarray(np.asarray(query_start, dtype=np.int32))
+    S = len(cl)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if items is None:
+        tt, hh = np.meshgrid(np.arange(T), np.arange(Hq), indexing="ij")
+        its = np.stack([tt.ravel(), hh.ravel()], 1).astype(np.int32)
+    else:
+        its = np.asarray(items, dtype=np.int32).reshape(-1, 2)
+    it_t = np.ascontiguousarray(its[:, 0])
+    it_h = np.ascontiguousarray(its[:, 1])
+    out = np.zeros((len(its), D), dtype=np.float64)
+    rc = _load().oracle_paged_attention_chunk(
+        out.ctypes.data, q.data_ptr(), k_pool.data_ptr(), v_pool.data_ptr(), bt.ctypes.data, bt.shape[1],
+        cl.ctypes.data, qs.ctypes.data, S, T, Hq, Hkv, D, bs, NB, float(scale), _DT[q.dtype],
+        it_t.ctypes.data, it_h.ctypes.data, len(its), threads)
+    if rc != 0:
+        raise ValueError("oracle_paged_attention_chunk: invalid indices (status %d)" % rc)
+    return out.reshape(T, Hq, D) if items is None else out
 
 
 def kv_append(k_pool: torch.Tensor, v_pool: torch.Tensor, k_new, v_new, slot_mapping) -> None:

@@ -24,6 +24,13 @@
  *   tokens, the plainest reading of "attention over the KV cache"
  *   (openeuler.csdn.net explainer, section 2.2).
  *
+ * A chunk of new tokens per sequence (oracle_paged_attention_chunk): sequence s
+ * owns query rows query_start[s] .. query_start[s+1]-1, which are the last
+ * n_s tokens of its L_s cached tokens; row i (0-based) sits at position
+ * L_s - n_s + i and attends causally to tokens 0 .. L_s - n_s + i -- each
+ * token sees itself and what precedes it, as in autoregressive generation
+ * (openeuler.csdn.net explainer, sections 2.1-2.2).  n_s = 1 is decode.
+ *
  * Storage types are widened exactly to double: fp32 directly, bf16 by placing
  * its 16 bits on top of a float, fp16 by decoding sign/exponent/mantissa.
  */
@@ -117,6 +124,67 @@ int oracle_paged_attention(double *out, const void *q, const void *k_pool, const
             double w = exp(x[t] - mx);
             den += w;
             int64_t slot = oracle_slot(bt, block_size, t);
+            int64_t blk = slot / block_size, off = slot % block_size;
+            int64_t vbase = ((blk * Hkv + g) * block_size + off) * D;
+            for (int d = 0; d < D; ++d) o[d] += w * widen(v_pool, vbase + d, dtype);
+        }
+        for (int d = 0; d < D; ++d) o[d] /= den;
+        free(x);
+    }
+    return status;
+}
+
+/*
+ * Causal attention of a chunk of query tokens per sequence (see the header).
+ * out[i, :] (fp64, [n_items, D]) for (query row items_t[i], head items_h[i]).
+ * Returns 0, -1 on an index outside the arrays, -2 on bad shapes.
+ */
+int oracle_paged_attention_chunk(double *out, const void *q, const void *k_pool, const void *v_pool,
+                                 const int32_t *block_tables, int max_blocks, const int32_t *context_lens,
+                                 const int32_t *query_start, int S, int T, int Hq, int Hkv, int D,
+                                 int block_size, int num_blocks, double scale, int dtype,
+                                 const int32_t *items_t, const int32_t *items_h, int n_items, int num_threads) {
+    if (Hkv <= 0 || Hq % Hkv != 0 || D <= 0 || block_size <= 0) return -2;
+    int G = Hq / Hkv;
+    int status = 0;
+    if (num_threads <= 0) num_threads = 1;
+#pragma omp parallel for schedule(dynamic, 1) num_threads(num_threads) reduction(min : status)
+    for (int it = 0; it < n_items; ++it) {
+        int t = items_t[it], h = items_h[it];
+        double *o = out + (int64_t)it * D;
+        for (int d = 0; d < D; ++d) o[d] = 0.0;
+        if (t < 0 || t >= T || h < 0 || h >= Hq) { status = -1; continue; }
+        int s = -1;
+        for (int j = 0; j < S; ++j)
+            if (query_start[j] <= t && t < query_start[j + 1]) s = j;
+        if (s < 0) { status = -1; continue; }
+        int64_t n = query_start[s + 1] - query_start[s];
+        int64_t L = context_lens[s];
+        if (n > L || L > (int64_t)max_blocks * block_size) { status = -1; continue; }
+        int64_t upto = L - n + (t - query_start[s]) + 1; /* tokens this row sees */
+        int g = h / G;
+        const int32_t *bt = block_tables + (int64_t)s * max_blocks;
+        int bad = 0;
+        for (int64_t j = 0; j < (upto + block_size - 1) / block_size; ++j)
+            if (bt[j] < 0 || bt[j] >= num_blocks) bad = 1;
+        if (bad) { status = -1; continue; }
+        double *x = (double *)malloc(sizeof(double) * (size_t)upto);
+        int64_t qbase = ((int64_t)t * Hq + h) * D;
+        double mx = -INFINITY;
+        for (int64_t u = 0; u < upto; ++u) {
+            int64_t slot = oracle_slot(bt, block_size, u);
+            int64_t blk = slot / block_size, off = slot % block_size;
+            int64_t kbase = ((blk * Hkv + g) * block_size + off) * D;
+            double acc = 0.0;
+            for (int d = 0; d < D; ++d) acc += widen(q, qbase + d, dtype) * widen(k_pool, kbase + d, dtype);
+            x[u] = scale * acc;
+            if (x[u] > mx) mx = x[u];
+        }
+        double den = 0.0;
+        for (int64_t u = 0; u < upto; ++u) {
+            double w = exp(x[u] - mx);
+            den += w;
+            int64_t slot = oracle_slot(bt, block_size, u);
             int64_t blk = slot / block_size, off = slot % block_size;
             int64_t vbase = ((blk * Hkv + g) * block_size + off) * D;
             for (int d = 0; d < D; ++d) o[d] += w * widen(v_pool, vbase + d, dtype);

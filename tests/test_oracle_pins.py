@@ -399,3 +399,58 @@ def test_fork_then_append_copies_partial_block_once_per_writer():
     assert all(p[0][0] == last for p in copies[:3])
     assert a.refcount(last) == 1 and a.seqs[0][0][1] == last
     assert a.refcount(a.seqs[0][0][0]) == 4                # full blocks stay shared
+
+
+# ------------------------------------------------ chunks of new tokens (causal)
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("Hq,Hkv,D,bs", [(4, 4, 64, 16), (8, 2, 128, 32)])
+def test_chunk_equals_sdpa_with_causal_mask(dtype, Hq, Hkv, D, bs):
+    """n new tokens at the end of a context of L: row i attends to tokens
+    0 .. L-n+i -- torch SDPA on the contiguous layout with that mask."""
+    rng = np.random.default_rng(D + bs)
+    lens, ns = [40, 7, 100], [5, 7, 1]        # the second chunk is a whole prompt
+    T = sum(ns)
+    qs = np.concatenate([[0], np.cumsum(ns)]).astype(np.int32)
+    q = torch.randn(T, Hq, D).to(dtype)
+    NB = sum(-(-L // bs) for L in lens) + 4
+    kp = torch.randn(NB, Hkv, bs, D).to(dtype)
+    vp = torch.randn(NB, Hkv, bs, D).to(dtype)
+    maxb = max(-(-L // bs) for L in lens)
+    bt = np.full((3, maxb), -1, np.int32)
+    perm = rng.permutation(NB)
+    cur = 0
+    ref = torch.zeros(T, Hq, D, dtype=torch.float64)
+    for s, L in enumerate(lens):
+        nb = -(-L // bs)
+        bt[s, :nb] = perm[cur:cur + nb]
+        cur += nb
+        Kc = torch.cat([kp[bt[s, j]] for j in range(nb)], dim=1)[:, :L].double()   # [Hkv, L, D]
+        Vc = torch.cat([vp[bt[s, j]] for j in range(nb)], dim=1)[:, :L].double()
+        n = ns[s]
+        mask = torch.arange(L)[None, :] <= (L - n + torch.arange(n))[:, None]       # [n, L]
+        qq = q[qs[s]:qs[s + 1]].double().transpose(0, 1)[None]                     # [1, Hq, n, D]
+        o = F.scaled_dot_product_attention(qq, Kc[None], Vc[None], attn_mask=mask, enable_gqa=(Hq != Hkv))
+        ref[qs[s]:qs[s + 1]] = o[0].transpose(0, 1)
+    got = oracle.paged_attention_chunk(q, kp, vp, bt, lens, qs)
+    assert np.abs(got - ref.numpy()).max() < 1e-12
+
+
+def test_chunk_of_one_token_is_decode():
+    b = synth.make_batch(synth.shrink(synth.CONFIGS["llama3_gqa_bs16"], S=3, Hq=8, Hkv=2, D=64,
+                                      len_fixed=None, len_uniform=(1, 90)))
+    qs = np.arange(4, dtype=np.int32)
+    a = oracle.paged_attention_chunk(b.q, b.k_pool, b.v_pool, b.block_tables, b.lens, qs)
+    d = oracle.paged_attention(b.q, b.k_pool, b.v_pool, b.block_tables, b.lens)
+    assert np.array_equal(a, d)
+
+
+def test_chunk_last_row_sees_whole_context_first_row_sees_its_prefix():
+    b = synth.make_batch(synth.shrink(synth.CONFIGS["llama7b"], S=1, Hq=2, Hkv=2, D=64, lens=[50], len_uniform=None))
+    n = 6
+    q = torch.randn(n, 2, 64)
+    qs = np.array([0, n], np.int32)
+    got = oracle.paged_attention_chunk(q, b.k_pool.float(), b.v_pool.float(), b.block_tables, b.lens, qs)
+    for i in range(n):
+        one = oracle.paged_attention(q[i:i + 1], b.k_pool.float(), b.v_pool.float(), b.block_tables[:1],
+                                     [50 - n + i + 1])
+        assert np.array_equal(got[i], one[0])
