@@ -197,6 +197,38 @@ pkv_status pkv_find_shared_prefix_groups(const int32_t* block_tables, const int3
                                          int* n_groups);
 
 /*
+ * pkv_paged_attention_chunk -- causal attention for a chunk of new tokens per
+ * sequence (speculative verification of draft tokens, or a short chunk of a
+ * prompt), read through the block tables like decode.  Sequence s owns query
+ * rows query_start[s] .. query_start[s+1]-1 (n_s rows), which are the last
+ * n_s of its context_lens[s] cached tokens (their K/V already appended);
+ * row i sits at position context_lens[s] - n_s + i and attends to tokens
+ * 0 .. context_lens[s] - n_s + i: itself and everything before it
+ * ([E] 2.1-2.2: each new token attends to all earlier ones).  n_s = 1 is
+ * decode.
+ *   out, q        [num_tokens][num_q_heads][head_dim]
+ *   query_start   device int32 [num_seqs + 1], non-decreasing, within
+ *                 [0, num_tokens]; n_s <= context_lens[s] and <= max_query_len
+ *                 (a violation is recorded as PKV_DEVERR_CONTEXT and that
+ *                 sequence's rows are left untouched).
+ *   max_query_len host bound on n_s.
+ *   workspace     >= pkv_attention_chunk_workspace_bytes(...) bytes.
+ * 16-bit element types, query groups of 1..16 heads (tensor cores: the 16
+ * rows of an MMA are (new token, head) pairs).
+ */
+pkv_status pkv_paged_attention_chunk(void* out, const void* q, const void* k_pool, const void* v_pool,
+                                     const int32_t* block_tables, int max_blocks_per_seq,
+                                     const int32_t* context_lens, const int32_t* query_start, int num_seqs,
+                                     int num_tokens, int max_query_len, int num_q_heads, int num_kv_heads,
+                                     int head_dim, int block_size, int num_blocks, float scale,
+                                     int partition_size, void* workspace, size_t workspace_bytes,
+                                     pkv_dtype dtype, void* stream);
+
+/* Workspace bytes for pkv_paged_attention_chunk (0 if no context needs splitting). */
+size_t pkv_attention_chunk_workspace_bytes(int num_tokens, int num_q_heads, int head_dim, int max_context_len,
+                                           int partition_size);
+
+/*
  * pkv_paged_attention_decode_static -- the same decode attention, for callers
  * that cannot allocate device memory.  The pages have no counterpart to this
  * call; it exists for integration only.

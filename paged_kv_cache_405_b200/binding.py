@@ -28,7 +28,8 @@ _DTYPE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 EXPORTS = [
     "pkv_kv_append", "pkv_attention_workspace_bytes", "pkv_attention_partition_size",
     "pkv_paged_attention_decode", "pkv_paged_attention_decode_static", "pkv_paged_attention_decode_shared",
-    "pkv_attention_shared_workspace_bytes", "pkv_find_shared_prefix_groups", "pkv_block_copy", "pkv_device_error", "pkv_launch_count",
+    "pkv_attention_shared_workspace_bytes", "pkv_find_shared_prefix_groups", "pkv_paged_attention_chunk",
+    "pkv_attention_chunk_workspace_bytes", "pkv_block_copy", "pkv_device_error", "pkv_launch_count",
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_add", "pkv_seq_share_prefix", "pkv_seq_fork",
     "pkv_seq_append_slots", "pkv_seq_append_slots_batch", "pkv_seq_block_tables_batch", "pkv_seq_free", "pkv_seq_block_table", "pkv_alloc_stats",
     "pkv_block_refcount", "pkv_status_str", "pkv_last_error",
@@ -61,6 +62,10 @@ def _load():
                                                       c_int, c_int, c_int, c_int, ctypes.c_float, c_int, c_vp,
                                                       c_vp, c_int, c_int, c_int, c_vp, c_sz, c_int, c_vp]),
         "pkv_attention_shared_workspace_bytes": (c_sz, [c_int, c_int, c_int, c_int, c_int]),
+        "pkv_paged_attention_chunk": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_vp, c_vp, c_int, c_int, c_int,
+                                              c_int, c_int, c_int, c_int, c_int, ctypes.c_float, c_int, c_vp, c_sz,
+                                              c_int, c_vp]),
+        "pkv_attention_chunk_workspace_bytes": (c_sz, [c_int, c_int, c_int, c_int, c_int]),
         "pkv_find_shared_prefix_groups": (c_int, [c_vp, c_vp, c_int, c_int, c_int, c_int, c_vp, c_vp, c_int,
                                                   ctypes.POINTER(c_int)]),
         "pkv_block_copy": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int, c_vp]),
@@ -234,6 +239,35 @@ def paged_attention_decode_shared(out, q, k_pool, v_pool, block_tables, context_
         _dev(group_shared, "group_shared") if n else None, n, int(max_group_size), int(max_shared_len),
         _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _dt(q), _stream(stream)))
+    return out
+
+
+def attention_chunk_workspace_bytes(num_tokens: int, num_q_heads: int, head_dim: int, max_context_len: int,
+                                    partition_size: int = 0) -> int:
+    return int(lib.pkv_attention_chunk_workspace_bytes(num_tokens, num_q_heads, head_dim, max_context_len,
+                                                       partition_size))
+
+
+def paged_attention_chunk(out, q, k_pool, v_pool, block_tables, context_lens, query_start, max_query_len: int,
+                          scale: float = 0.0, partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
+                          stream=None) -> torch.Tensor:
+    """Causal attention of the last ``query_start[s+1]-query_start[s]`` tokens of each sequence."""
+    T, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    for t, nm in ((block_tables, "block_tables"), (context_lens, "context_lens"), (query_start, "query_start")):
+        if t.dtype != torch.int32:
+            raise TypeError("%s must be int32" % nm)
+    S = context_lens.numel()
+    maxB = block_tables.shape[1]
+    if workspace is None:
+        nb = attention_chunk_workspace_bytes(T, Hq, D, maxB * bs, partition_size)
+        workspace = torch.empty(max(nb, 256), dtype=torch.uint8, device=q.device)
+    _check(lib.pkv_paged_attention_chunk(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
+        _dev(block_tables, "block_tables"), maxB, _dev(context_lens, "context_lens"),
+        _dev(query_start, "query_start"), S, T, int(max_query_len), Hq, Hkv, D, bs, NB, float(scale),
+        int(partition_size), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _dt(q),
+        _stream(stream)))
     return out
 
 

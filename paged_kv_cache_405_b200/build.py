@@ -18,7 +18,7 @@ SOURCES = ["pagedkv.cu", "allocator.cpp"]
 DEPS = SOURCES + ["common.cuh", "attention_common.cuh", "attention_simt.cuh", "attention_mma.cuh",
                   "kv_append.cuh", "block_copy.cuh", "reduce.cuh"]
 
-FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
+FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-Werror", "all-warnings",
          "-Xcompiler", "-fPIC", "-shared", "--expt-relaxed-constexpr", "-I", INCLUDE]
 
 

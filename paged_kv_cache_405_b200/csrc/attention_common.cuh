@@ -28,6 +28,15 @@ struct AttnParams {
     int max_shared;               // ... and shared runs up to this many tokens
 };
 
+// A chunk of new tokens per sequence (causal): sequence s owns query rows
+// query_start[s] .. query_start[s+1]-1, the last tokens of its context.
+struct ChunkParams {
+    const int32_t* query_start;  // [S + 1]
+    int T;                       // query rows in q / out
+    int max_query_len;           // host bound on query_start[s+1] - query_start[s]
+    int nparts;                  // partitions of the longest context
+};
+
 // Which tokens one (sequence, partition) unit covers and where its result goes.
 //   member  -- the sequence belongs to a valid shared-prefix group; its first
 //              `shared` tokens are done by the prefix pass in npre partials

@@ -74,12 +74,15 @@ struct MmaAcc {
 };
 
 // Stream tokens [t_begin, t_end) of kv head g (block ids from bt_row) through
-// this warp's ring and accumulate into acc.  Returns false if a wait on a copy
-// timed out (the unit is then abandoned after draining its copies).
+// this warp's ring and accumulate into acc.  Row gid sees only tokens below
+// lim_lo, row gid+8 only tokens below lim_hi (causal chunks; pass t_end when
+// every row sees the whole range).  Returns false if a wait on a copy timed
+// out (the unit is then abandoned after draining its copies).
 template <typename T, int D, int WARPS, int STAGES>
 __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                            uint8_t* ring, uint32_t bar0, const int32_t* bt_row, int t_begin,
-                                           int t_end, int g, int lane, MmaAcc<T, D>& acc) {
+                                           int t_end, int g, int lane, MmaAcc<T, D>& acc, int lim_lo,
+                                           int lim_hi) {
     using C = MmaCfg<T, D, WARPS, STAGES>;
     constexpr int KSTEPS = D / 16;
     constexpr int NT_O = D / 8;
@@ -127,6 +130,8 @@ __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMa
             return false;
         }
         const int valid = min(kTileTok, t_end - (t_begin + i * kTileTok));
+        const int seen_lo = min(valid, lim_lo - (t_begin + i * kTileTok));  // tokens row gid sees
+        const int seen_hi = min(valid, lim_hi - (t_begin + i * kTileTok));  // ... and row gid+8
         const uint32_t Ks = ring_s + st * C::kStageBytes;
         const uint32_t Vs = Ks + C::kTileBytes;
 
@@ -149,7 +154,7 @@ __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMa
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int tok = nt * 8 + 2 * tig + (e & 1);
-                const float x = tok < valid ? sacc[nt][e] * p.scale_log2 : -INFINITY;
+                const float x = tok < (e < 2 ? seen_lo : seen_hi) ? sacc[nt][e] * p.scale_log2 : -INFINITY;
                 sacc[nt][e] = x;
                 if (e < 2) mx_lo = fmaxf(mx_lo, x);
                 else mx_hi = fmaxf(mx_hi, x);
@@ -161,7 +166,10 @@ __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMa
             mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, off));
         }
         const float mn_lo = fmaxf(acc.m_lo, mx_lo), mn_hi = fmaxf(acc.m_hi, mx_hi);
-        const float a_lo = ex2(acc.m_lo - mn_lo), a_hi = ex2(acc.m_hi - mn_hi);
+        // A row that has seen no token yet keeps m = -inf; exponentiate
+        // against 0 then, so that no -inf - -inf appears.
+        const float b_lo = mn_lo == -INFINITY ? 0.f : mn_lo, b_hi = mn_hi == -INFINITY ? 0.f : mn_hi;
+        const float a_lo = ex2(acc.m_lo - b_lo), a_hi = ex2(acc.m_hi - b_hi);
         acc.m_lo = mn_lo;
         acc.m_hi = mn_hi;
         float ps_lo = 0.f, ps_hi = 0.f;
@@ -169,7 +177,7 @@ __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMa
         for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float pr = ex2(sacc[nt][e] - (e < 2 ? mn_lo : mn_hi));
+                const float pr = ex2(sacc[nt][e] - (e < 2 ? b_lo : b_hi));
                 sacc[nt][e] = pr;
                 if (e < 2) ps_lo += pr;
                 else ps_hi += pr;
@@ -294,7 +302,7 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnPa
     MmaAcc<T, D> acc;
     acc.load_q(gid < G ? qb + gid * D : nullptr, gid + 8 < G ? qb + (gid + 8) * D : nullptr, tig);
     if (!mma_attend<T, D, WARPS, STAGES>(p, &tmK, &tmV, ring, bar0, p.block_tables + (int64_t)s * p.maxB,
-                                         u.t_begin, u.t_end, g, lane, acc))
+                                         u.t_begin, u.t_end, g, lane, acc, u.t_end, u.t_end))
         return;
 
 #pragma unroll
@@ -376,7 +384,7 @@ __global__ void __launch_bounds__(WARPS * 32) prefix_attn_mma_kernel(const AttnP
     bool ok = true;
     if (w0 < w1)
         ok = mma_attend<T, D, WARPS, STAGES>(p, &tmK, &tmV, ring, bar0, p.block_tables + (int64_t)first * p.maxB,
-                                             w0, w1, g, lane, acc);
+                                             w0, w1, g, lane, acc, w1, w1);
     const int all_ok = __syncthreads_and(ok ? 1 : 0);  // every warp is done with its ring
 
     // Merge buffer (reuses the rings): o [WARPS][16][D], then m, l [WARPS][16].
@@ -437,6 +445,76 @@ __global__ void __launch_bounds__(WARPS * 32) prefix_attn_mma_kernel(const AttnP
         *reinterpret_cast<float4*>(dst + cc) = a;
     }
     if (c0 == 0) *reinterpret_cast<float2*>(p.ws_ml + idx * 2) = make_float2(M, lsum);
+}
+
+// Causal chunk of new tokens per sequence (speculative verification, chunked
+// prefill): grid (ceil(Hkv / WARPS), row tiles * partitions, S).  The rows of
+// sequence s for kv head g are (new token i, query head g*G + r) flattened as
+// i*G + r; row i sits at position L - n + i and sees tokens 0 .. L - n + i
+// (each token attends to itself and what precedes it: openeuler.csdn.net
+// PagedAttention explainer 2.1-2.2).  16 rows per warp -- for multi-head
+// attention 16 new tokens of one head, a real contraction over shared K/V.
+template <typename T, int D, int WARPS, int STAGES>
+__global__ void __launch_bounds__(WARPS * 32, 3) chunk_attn_mma_kernel(const AttnParams p, const ChunkParams c,
+                                                                    const __grid_constant__ CUtensorMap tmK,
+                                                                    const __grid_constant__ CUtensorMap tmV) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = blockIdx.x * WARPS + warp;  // kv head
+    const int part = blockIdx.y % c.nparts;
+    const int tile = blockIdx.y / c.nparts;
+    const int s = blockIdx.z;
+    if (g >= p.Hkv) return;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int G = p.G;
+    const bool report = part == 0 && tile == 0 && g == 0 && lane == 0;
+
+    const int L = load_context_len(p, s, report);
+    const int q0 = c.query_start[s], q1 = c.query_start[s + 1];
+    if (q0 < 0 || q1 < q0 || q1 > c.T || q1 - q0 > L || q1 - q0 > c.max_query_len) {
+        if (report) flag_error(4u /* PKV_DEVERR_CONTEXT */);
+        return;
+    }
+    const int n = q1 - q0;
+    const int rows = n * G;
+    if (tile * 16 >= rows) return;
+    const int last_row = min(rows - 1, tile * 16 + 15);
+    const int t_begin = part * p.P;
+    const int t_end = min(min(L, t_begin + p.P), L - n + last_row / G + 1);
+    if (t_begin >= t_end) return;
+
+    int ri[2], rh[2], lim[2];
+    bool use[2];
+#pragma unroll
+    for (int hi = 0; hi < 2; ++hi) {
+        const int r = tile * 16 + gid + 8 * hi;
+        use[hi] = r < rows;
+        ri[hi] = use[hi] ? r / G : 0;
+        rh[hi] = g * G + (use[hi] ? r % G : 0);
+        lim[hi] = use[hi] ? L - n + ri[hi] + 1 : 0;  // tokens this row sees
+    }
+    uint32_t bar0;
+    uint8_t* ring = mma_setup_ring<T, D, WARPS, STAGES>(smem_raw, warp, lane, bar0, &tmK, &tmV);
+    const T* q = reinterpret_cast<const T*>(p.q);
+    MmaAcc<T, D> acc;
+    acc.load_q(use[0] ? q + ((int64_t)(q0 + ri[0]) * p.Hq + rh[0]) * D : nullptr,
+               use[1] ? q + ((int64_t)(q0 + ri[1]) * p.Hq + rh[1]) * D : nullptr, tig);
+    if (!mma_attend<T, D, WARPS, STAGES>(p, &tmK, &tmV, ring, bar0, p.block_tables + (int64_t)s * p.maxB, t_begin,
+                                         t_end, g, lane, acc, lim[0], lim[1]))
+        return;
+    const bool direct = (L + p.P - 1) / p.P == 1;  // every row of the sequence has one partition
+#pragma unroll
+    for (int hi = 0; hi < 2; ++hi) {
+        if (!use[hi] || lim[hi] <= t_begin) continue;  // no token of this row in the partition
+        const int64_t row = (int64_t)(q0 + ri[hi]) * p.Hq + rh[hi];
+        if (direct) {
+            mma_store_row<T, D>(acc, hi, tig, reinterpret_cast<T*>(p.out) + row * D, nullptr, nullptr);
+        } else {
+            const int64_t idx = row * p.maxP + part;
+            mma_store_row<T, D>(acc, hi, tig, nullptr, p.ws_o + idx * D, p.ws_ml + idx * 2);
+        }
+    }
 }
 
 }  // namespace pkv

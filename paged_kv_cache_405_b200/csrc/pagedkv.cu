@@ -3,6 +3,7 @@
 // kernels so that they share the device error word.
 #include <algorithm>
 #include <atomic>
+#include <climits>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -207,8 +208,20 @@ static cudaError_t launch_prefix(const pkv::AttnParams& p, dim3 grid, const CUte
 // Many partitions: 8 warps on each (sequence, head); few: 8 rows per CTA,
 // one warp each.
 template <typename T, int D>
+static cudaError_t launch_chunk(const pkv::AttnParams& p, const pkv::ChunkParams& c, dim3 grid,
+                                const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t st) {
+    using C = pkv::MmaCfg<T, D, kMmaWarps, kMmaStages>;
+    auto k = pkv::chunk_attn_mma_kernel<T, D, kMmaWarps, kMmaStages>;
+    static cudaError_t attr = set_smem(k, C::kSmemBytes);
+    if (attr != cudaSuccess) return attr;
+    k<<<grid, kMmaWarps * 32, C::kSmemBytes, st>>>(p, c, mk, mv);
+    g_launches++;
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
 static cudaError_t launch_reduce(const pkv::ReduceParams& r, cudaStream_t st) {
-    const unsigned rows = (unsigned)(r.S * r.Hq);
+    const unsigned rows = (unsigned)((r.query_start ? r.T : r.S) * r.Hq);
     if (r.maxP > 32) pkv::splitk_reduce_kernel<T, D, 8, 1><<<rows, 256, 0, st>>>(r);
     else pkv::splitk_reduce_kernel<T, D, 1, 8><<<(rows + 7) / 8, 256, 0, st>>>(r);
     g_launches++;
@@ -240,7 +253,7 @@ static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int npart
     }
     if (e != cudaSuccess || p.maxP <= 1) return e;
     pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
-                        p.group_first, p.group_shared, p.num_groups, p.max_shared};
+                        p.group_first, p.group_shared, p.num_groups, p.max_shared, nullptr, 0};
     return D == 64 ? launch_reduce<T, 64>(r, st) : launch_reduce<T, 128>(r, st);
 }
 
@@ -525,6 +538,130 @@ pkv_status pkv_device_error(void* stream, uint32_t* code) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Causal attention for a chunk of new tokens per sequence.
+// ---------------------------------------------------------------------------
+namespace pkv_host {
+
+static size_t chunk_workspace_for(int T, int Hq, int D, int max_len, int P) {
+    const int64_t nparts = (max_len + P - 1) / P;
+    if (nparts <= 1) return 0;
+    return (size_t)T * Hq * nparts * (size_t)(D + 2) * sizeof(float);
+}
+
+template <typename T>
+static cudaError_t dispatch_chunk(const pkv::AttnParams& p, const pkv::ChunkParams& c, int D, int tiles,
+                                  const CUtensorMap& mk, const CUtensorMap& mv, cudaStream_t st) {
+    if constexpr (std::is_same<T, float>::value) {
+        return cudaErrorInvalidValue;
+    } else {
+        dim3 grid((p.Hkv + kMmaWarps - 1) / kMmaWarps, tiles * c.nparts, p.S);
+        cudaError_t e = D == 64 ? launch_chunk<T, 64>(p, c, grid, mk, mv, st) : launch_chunk<T, 128>(p, c, grid, mk, mv, st);
+        if (e != cudaSuccess || c.nparts <= 1) return e;
+        pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
+                            nullptr, nullptr, 0, 0, c.query_start, c.T};
+        return D == 64 ? launch_reduce<T, 64>(r, st) : launch_reduce<T, 128>(r, st);
+    }
+}
+
+}  // namespace pkv_host
+
+extern "C" size_t pkv_attention_chunk_workspace_bytes(int num_tokens, int num_q_heads, int head_dim,
+                                                      int max_context_len, int partition_size) {
+    using namespace pkv_host;
+    if (num_tokens <= 0 || num_q_heads <= 0 || head_dim <= 0 || max_context_len <= 0 || partition_size < 0) return 0;
+    return chunk_workspace_for(num_tokens, num_q_heads, head_dim, max_context_len,
+                               partition_bound(max_context_len, partition_size));
+}
+
+extern "C" pkv_status pkv_paged_attention_chunk(void* out, const void* q, const void* k_pool, const void* v_pool,
+                                                const int32_t* block_tables, int max_blocks_per_seq,
+                                                const int32_t* context_lens, const int32_t* query_start,
+                                                int num_seqs, int num_tokens, int max_query_len, int num_q_heads,
+                                                int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                                float scale, int partition_size, void* workspace,
+                                                size_t workspace_bytes, pkv_dtype dtype, void* stream) {
+    using namespace pkv_host;
+    const char* fn = "pkv_paged_attention_chunk";
+    if (dtype != PKV_BF16 && dtype != PKV_F16) {
+        g_msg = std::string(fn) + ": 16-bit element types only (tensor-core kernel)";
+        return valid_dtype(dtype) ? PKV_ERR_UNSUPPORTED : PKV_ERR_INVALID;
+    }
+    if (num_seqs < 0 || num_tokens < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
+        max_blocks_per_seq <= 0 || max_query_len < 1)
+        return invalid("pkv_paged_attention_chunk: sizes must be positive");
+    if (num_q_heads % num_kv_heads != 0 || num_q_heads / num_kv_heads > 16)
+        return invalid("pkv_paged_attention_chunk: num_q_heads must be 1..16 times num_kv_heads");
+    if (!valid_block_size(block_size))
+        return invalid("pkv_paged_attention_chunk: block_size must be 16, 32, 64, 128 or 256");
+    if (head_dim != 64 && head_dim != 128) {
+        g_msg = std::string(fn) + ": head_dim must be 64 or 128";
+        return PKV_ERR_UNSUPPORTED;
+    }
+    if (partition_size < 0 || partition_size % 16 != 0)
+        return invalid("pkv_paged_attention_chunk: partition_size must be 0 or a positive multiple of 16");
+    if (!(std::isfinite(scale)) || scale < 0.f) return invalid("pkv_paged_attention_chunk: scale must be >= 0");
+    const int64_t max_len64 = (int64_t)max_blocks_per_seq * block_size;
+    if (max_len64 > (int64_t)1 << 30) return invalid("pkv_paged_attention_chunk: max_blocks_per_seq*block_size too large");
+    if ((int64_t)num_blocks * num_kv_heads * block_size >= ((int64_t)1 << 31))
+        return invalid("pkv_paged_attention_chunk: pool has 2^31 or more rows");
+    if (num_seqs == 0 || num_tokens == 0) return PKV_OK;
+    if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !query_start)
+        return invalid("pkv_paged_attention_chunk: null pointer");
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) || (reinterpret_cast<uintptr_t>(context_lens) & 3u) ||
+        (reinterpret_cast<uintptr_t>(query_start) & 3u))
+        return invalid("pkv_paged_attention_chunk: pointers must be 16-byte aligned (int arrays 4-byte)");
+    if (num_seqs > 65535) return invalid("pkv_paged_attention_chunk: at most 65535 sequences per call");
+    const int max_len = (int)max_len64;
+    const int G = num_q_heads / num_kv_heads;
+    const int P = choose_partition(max_len, partition_size);
+    const int64_t nparts = (max_len + P - 1) / P;
+    const int64_t tiles = ((int64_t)max_query_len * G + 15) / 16;
+    if (tiles * nparts > 65535) return invalid("pkv_paged_attention_chunk: too many row tiles x partitions");
+    if ((int64_t)num_tokens * num_q_heads > INT32_MAX) return invalid("pkv_paged_attention_chunk: too many rows");
+    const size_t need = chunk_workspace_for(num_tokens, num_q_heads, head_dim, max_len, P);
+    if (need > 0) {
+        if (!workspace || workspace_bytes < need) return invalid("pkv_paged_attention_chunk: workspace too small");
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+            return invalid("pkv_paged_attention_chunk: workspace must be 256-byte aligned");
+    }
+    pkv::AttnParams p;
+    std::memset(&p, 0, sizeof p);
+    p.out = out;
+    p.q = q;
+    p.k_pool = k_pool;
+    p.v_pool = v_pool;
+    p.block_tables = block_tables;
+    p.context_lens = context_lens;
+    const size_t n_part = (size_t)num_tokens * num_q_heads * nparts;
+    p.ws_o = need ? static_cast<float*>(workspace) : nullptr;
+    p.ws_ml = need ? static_cast<float*>(workspace) + n_part * head_dim : nullptr;
+    p.S = num_seqs;
+    p.Hq = num_q_heads;
+    p.Hkv = num_kv_heads;
+    p.G = G;
+    p.bs = block_size;
+    p.NB = num_blocks;
+    p.maxB = max_blocks_per_seq;
+    p.P = P;
+    p.maxP = (int)nparts;
+    p.max_len = max_len;
+    const float sc = scale > 0.f ? scale : 1.f / std::sqrt((float)head_dim);
+    p.scale_log2 = sc * 1.4426950408889634f;
+    pkv::ChunkParams c{query_start, num_tokens, max_query_len, (int)nparts};
+    CUtensorMap mk, mv;
+    const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
+    if (!make_pool_map(&mk, k_pool, rows, head_dim, dtype, true) || !make_pool_map(&mv, v_pool, rows, head_dim, dtype, true)) {
+        g_msg = std::string(fn) + ": cuTensorMapEncodeTiled failed";
+        return PKV_ERR_CUDA;
+    }
+    cudaStream_t st = (cudaStream_t)stream;
+    cudaError_t e = dtype == PKV_BF16 ? dispatch_chunk<__nv_bfloat16>(p, c, head_dim, (int)tiles, mk, mv, st)
+                                      : dispatch_chunk<__half>(p, c, head_dim, (int)tiles, mk, mv, st);
+    return e == cudaSuccess ? PKV_OK : cuda_fail(fn, e);
+}
 
 // ---------------------------------------------------------------------------
 // Decode attention with built-in scratch, for callers that cannot allocate.

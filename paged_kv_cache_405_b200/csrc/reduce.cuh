@@ -21,7 +21,52 @@ struct ReduceParams {
     const int32_t* group_first;   // shared-prefix groups, as in AttnParams
     const int32_t* group_shared;
     int num_groups, max_shared;
+    const int32_t* query_start;   // chunk mode (non-null): rows are (query row, head), [S + 1]
+    int T;
 };
+
+// Partials to merge for one output row (0 = the attention kernel wrote it).
+__device__ __forceinline__ int reduce_count(const ReduceParams& p, int row) {
+    const int h_rows = p.Hq;
+    if (p.query_start) {  // causal chunk: row = t * Hq + h
+        const int t = row / h_rows;
+        if (t < p.query_start[0] || t >= p.query_start[p.S]) return 0;
+        int lo = 0, hi = p.S;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (p.query_start[mid] <= t) lo = mid;
+            else hi = mid;
+        }
+        int L = p.context_lens[lo];
+        L = L < 0 ? 0 : (L > p.max_len ? p.max_len : L);
+        const int n = p.query_start[lo + 1] - p.query_start[lo];
+        if (n > L) return 0;  // reported by the attention kernel
+        if ((L + p.P - 1) / p.P <= 1) return 0;
+        const int pos = L - n + (t - p.query_start[lo]);
+        return pos / p.P + 1;
+    }
+    const int s = row / h_rows;
+    int L = p.context_lens[s];
+    if (L < 0) L = 0;
+    if (L > p.max_len) L = p.max_len;
+    // A member of a valid shared-prefix group has ceil(shared/P) prefix
+    // partials followed by its own ones (same rule as the attention kernels).
+    int shared = 0;
+    if (p.num_groups > 0 && s >= p.group_first[0] && s < p.group_first[p.num_groups]) {
+        int lo = 0, hi = p.num_groups;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (p.group_first[mid] <= s) lo = mid;
+            else hi = mid;
+        }
+        const int sh = p.group_shared[lo];
+        if (sh > 0 && sh % p.bs == 0 && sh <= L && sh <= p.max_shared) shared = sh;
+    }
+    const int nsuf = (L - shared + p.P - 1) / p.P;
+    const int nP = (shared + p.P - 1) / p.P + nsuf;
+    if (shared == 0 && nP <= 1) return 0;  // written directly by the attention kernel
+    return nP;
+}
 
 // A CTA handles ROWS (sequence, query head) rows with W warps each.  The
 // partitions' maxima are reduced first (M); then warp w of a row sums the
@@ -48,27 +93,10 @@ __global__ void __launch_bounds__(W * ROWS * 32) splitk_reduce_kernel(const Redu
     float (&s_acc)[W][D] = s_acc_all[sub];
     float (&s_den)[W] = s_den_all[sub];
     float (&s_max)[W] = s_max_all[sub];
-    if (row >= p.S * p.Hq) return;  // whole rows return together (W warps of a row)
-    const int s = row / p.Hq;
-    int L = p.context_lens[s];
-    if (L < 0) L = 0;
-    if (L > p.max_len) L = p.max_len;
-    // Same rule as the attention kernels: a member of a valid shared-prefix
-    // group has ceil(shared/P) prefix partials followed by its own ones.
-    int shared = 0;
-    if (p.num_groups > 0 && s >= p.group_first[0] && s < p.group_first[p.num_groups]) {
-        int lo = 0, hi = p.num_groups;
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (p.group_first[mid] <= s) lo = mid;
-            else hi = mid;
-        }
-        const int sh = p.group_shared[lo];
-        if (sh > 0 && sh % p.bs == 0 && sh <= L && sh <= p.max_shared) shared = sh;
-    }
-    const int nsuf = (L - shared + p.P - 1) / p.P;
-    const int nP = (shared + p.P - 1) / p.P + nsuf;
-    if (shared == 0 && nP <= 1) return;  // written directly by the attention kernel
+    const int nrows = p.query_start ? p.T * p.Hq : p.S * p.Hq;
+    if (row >= nrows) return;  // whole rows return together (W warps of a row)
+    const int nP = reduce_count(p, row);
+    if (nP == 0) return;
     const int64_t base = (int64_t)row * p.maxP;
     const float* ml = p.ws_ml + base * 2;
 
