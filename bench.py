@@ -42,8 +42,20 @@ FALLBACK_HBM_GBS = 6650.0
 
 
 # ----------------------------------------------------------------- accounting
+def chunk_ws_bytes(lens, query_start, Hq: int, D: int, P: int) -> int:
+    """Split-K partials written and read back by a causal chunk call."""
+    total = 0
+    for s in range(len(lens)):
+        L, n = int(lens[s]), int(query_start[s + 1] - query_start[s])
+        if -(-L // P) <= 1:
+            continue
+        pos = L - n + np.arange(n)
+        total += int((pos // P + 1).sum()) * Hq * (D + 2) * 4 * 2
+    return total
+
+
 def attention_bytes(bt: np.ndarray, lens: np.ndarray, Hq: int, Hkv: int, D: int, bs: int, elt: int,
-                    P: int, shared=None) -> dict:
+                    P: int, shared=None, q_rows=None) -> dict:
     """Algorithmic bytes of one decode-attention call.
 
     K/V: every physical (block, kv head) tile covered by some context counts
@@ -64,7 +76,7 @@ def attention_bytes(bt: np.ndarray, lens: np.ndarray, Hq: int, Hkv: int, D: int,
     tok = int(best.sum())
     kv = 2 * Hkv * D * elt * tok
     logical = 2 * Hkv * D * elt * int(lens.sum())
-    qo = 2 * S * Hq * D * elt
+    qo = 2 * (S if q_rows is None else q_rows) * Hq * D * elt
     tables = 4 * int(nb.sum()) + 4 * S
     sh = np.zeros(S, dtype=np.int64) if shared is None else np.asarray(shared, dtype=np.int64)
     nparts = -(-sh // P) + -(-(lens - sh) // P)
@@ -109,14 +121,18 @@ class Workload:
         if shape.prefix:
             ss.free(-1)
         self.parents = list(range(shape.S))
+        if shape.chunk:
+            ss.reserve_chunk_workspace(shape.S * shape.chunk)
         self.elt = b.k_pool.element_size()
         self.eff_P = pkv.attention_partition_size(shape.S, shape.Hq, shape.Hkv, shape.D,
                                                   b.max_blocks * shape.bs, self.P)
         self.next_child = shape.S
 
     def plan(self):
-        """Host work of one step; returns (plan, children written)."""
+        """Host work of one step: a StepPlan, or a ChunkPlan for chunk workloads."""
         sh, ss = self.shape, self.session
+        if sh.chunk:
+            return ss.plan_chunk(self.parents, [sh.chunk] * len(self.parents))
         children = []
         if sh.beams:
             for p in self.parents:
@@ -135,8 +151,28 @@ class Workload:
             ss.free(c)
         return plan
 
+    def to_device(self, plan):
+        return self.session.chunk_to_device(plan) if self.shape.chunk else self.session.to_device(plan)
+
+    def upload(self, plan):
+        return self.session.chunk_to_device(plan) if self.shape.chunk else self.session.upload(plan)
+
+    def launch(self, d, q, kn, vn, out):
+        if self.shape.chunk:
+            return self.session.launch_chunk(d, q, kn, vn, out)
+        return self.session.launch(d, q, kn, vn, out)
+
     def step_bytes(self, plan):
         sh = self.shape
+        if sh.chunk:
+            a = attention_bytes(plan.block_tables, plan.lens, sh.Hq, sh.Hkv, sh.D, sh.bs, self.elt, self.eff_P,
+                                q_rows=len(plan.slot_mapping))
+            a["ws"] = chunk_ws_bytes(plan.lens, plan.query_start, sh.Hq, sh.D, self.eff_P)
+            a["total"] = a["kv"] + 2 * len(plan.slot_mapping) * sh.Hq * sh.D * self.elt + a["ws"] + \
+                4 * int(sum(-(-int(L) // sh.bs) for L in plan.lens)) + 8 * len(plan.lens)
+            total = a["total"] + append_bytes(len(plan.slot_mapping), sh.Hkv, sh.D, self.elt) + \
+                copy_bytes(len(plan.cow_pairs), sh.Hkv, sh.bs, sh.D, self.elt)
+            return total, a
         shared = None
         if plan.has_groups:   # per-sequence shared length of its group
             shared = np.repeat(plan.group_shared, np.diff(plan.group_first))
@@ -298,6 +334,10 @@ def workload_shape(args):
     shape = synth.CONFIGS[args.config]
     if args.batch:
         shape = synth.shrink(shape, S=args.batch)
+    # room in every table and in the pool for the tokens the run appends
+    grow = (args.warmup + args.steps + 8) * max(1, shape.chunk)
+    if grow > shape.reserve_tokens:
+        shape = synth.shrink(shape, reserve_tokens=grow)
     return shape
 
 
@@ -314,14 +354,15 @@ def run_ours(args, world, rank, local):
     plans, step_bytes, attn_bytes = [], [], []
     for i in range(W + K):
         p = wl.plan()
-        plans.append(ss.to_device(p))
+        plans.append(wl.to_device(p))
         tb, a = wl.step_bytes(p)
         step_bytes.append(tb)
         attn_bytes.append(a)
-    T = len(plans[0].slot_mapping)
+    T = len(plans[0]["slot_mapping"] if shape.chunk else plans[0].slot_mapping)
+    Tq = shape.S * max(1, shape.chunk)
     inputs = []
     for i in range(W + K):
-        q, _, _ = synth.step_inputs(shape, i, device=dev, seed=shape.seed + rank)
+        q = synth.randn((Tq, shape.Hq, shape.D), torch.Generator(device=dev).manual_seed(7907 * i + rank), dt, dev)
         kn = synth.randn((T, shape.Hkv, shape.D), torch.Generator(device=dev).manual_seed(7919 * i + rank), dt, dev)
         vn = synth.randn((T, shape.Hkv, shape.D), torch.Generator(device=dev).manual_seed(7919 * i + rank + 1),
                          dt, dev)
@@ -332,12 +373,22 @@ def run_ours(args, world, rank, local):
     def run_step(i, ev=None):
         d = plans[i]
         q, kn, vn = inputs[i]
-        if d.n_cow:
-            pkv.block_copy(ss.k_pool, ss.v_pool, d.cow_pairs)
-        pkv.kv_append(kn, vn, ss.k_pool, ss.v_pool, d.slot_mapping)
-        if ev is not None:
-            ev[0].record(stream)
-        ss.attend(d, q, out)
+        if shape.chunk:
+            if d["n_cow"]:
+                pkv.block_copy(ss.k_pool, ss.v_pool, d["cow_pairs"])
+            pkv.kv_append(kn, vn, ss.k_pool, ss.v_pool, d["slot_mapping"])
+            if ev is not None:
+                ev[0].record(stream)
+            pkv.paged_attention_chunk(out, q, ss.k_pool, ss.v_pool, d["block_tables"], d["lens"],
+                                      d["query_start"], d["max_query_len"], partition_size=wl.P,
+                                      workspace=ss.workspace)
+        else:
+            if d.n_cow:
+                pkv.block_copy(ss.k_pool, ss.v_pool, d.cow_pairs)
+            pkv.kv_append(kn, vn, ss.k_pool, ss.v_pool, d.slot_mapping)
+            if ev is not None:
+                ev[0].record(stream)
+            ss.attend(d, q, out)
         if ev is not None:
             ev[1].record(stream)
 
@@ -407,12 +458,14 @@ def run_ours(args, world, rank, local):
                        "description": shape.description, "batch": shape.S,
                        "q_heads": shape.Hq, "kv_heads": shape.Hkv, "head_dim": shape.D, "block_size": shape.bs,
                        "partition_size": wl_P(shape, args), "effective_partition_size": eff_P_of(shape, args, plans),
-                       "mean_context": round(float(plans[W].lens.float().mean().item()), 1),
+                       "mean_context": round(float((plans[W]["lens"] if shape.chunk else plans[W].lens)
+                                                   .float().mean().item()), 1),
+                       "new_tokens_per_seq": max(1, shape.chunk),
                        "l2": "inputs larger than L2 (K/V pool %.2f GB per rank)" % (
                            2 * ss.k_pool.numel() * ss.k_pool.element_size() / 1e9),
                        "parallelism": "replica per GPU" if world > 1 else "1 GPU",
                        "shared_prefix_groups": int((plans[W].group_shared > 0).sum().item())
-                       if plans[W].group_shared is not None else 0},
+                       if not shape.chunk and plans[W].group_shared is not None else 0},
             "pct_of_peak": round(100 * value / peak, 1),
             "seq_steps_per_s": round(seq_steps, 1),
             "attention_us": round(a_s * 1e6, 2),
@@ -439,8 +492,9 @@ def wl_P(shape, args):
 
 def eff_P_of(shape, args, plans):
     import paged_kv_cache_405_b200 as pkv
-    return pkv.attention_partition_size(shape.S, shape.Hq, shape.Hkv, shape.D,
-                                        plans[0].block_tables.shape[1] * shape.bs, wl_P(shape, args))
+    bt = plans[0]["block_tables"] if shape.chunk else plans[0].block_tables
+    return pkv.attention_partition_size(shape.S, shape.Hq, shape.Hkv, shape.D, bt.shape[1] * shape.bs,
+                                        wl_P(shape, args))
 
 
 def host_batch(shape, seed):
@@ -454,15 +508,16 @@ def run_e2e(args, wl, world, rank, dev):
     ss = wl.session
     K, W = args.steps, args.warmup
     dt = synth.DTYPES[shape.dtype]
-    T = shape.S * max(1, shape.beams)
+    T = shape.S * max(1, shape.beams, shape.chunk)
+    Tq = shape.S * max(1, shape.chunk)
     host_inputs = []
     for i in range(W + K):
         g = torch.Generator().manual_seed(104729 * (i + 1) + rank)
-        q = synth.randn((shape.S, shape.Hq, shape.D), g, dt, "cpu").pin_memory()
+        q = synth.randn((Tq, shape.Hq, shape.D), g, dt, "cpu").pin_memory()
         kn = synth.randn((T, shape.Hkv, shape.D), g, dt, "cpu").pin_memory()
         vn = synth.randn((T, shape.Hkv, shape.D), g, dt, "cpu").pin_memory()
         host_inputs.append((q, kn, vn))
-    out_host = torch.empty((shape.S, shape.Hq, shape.D), dtype=dt, pin_memory=True)
+    out_host = torch.empty((Tq, shape.Hq, shape.D), dtype=dt, pin_memory=True)
     stream = torch.cuda.current_stream()
     h2d = d2h = 0
 
@@ -473,17 +528,20 @@ def run_e2e(args, wl, world, rank, dev):
         q, kn, vn = host_inputs[i]
         p = wl.plan()
         plans.append(p)
-        d = ss.upload(p)
+        d = wl.upload(p)
         qd = q.to(dev, non_blocking=True)
         kd = kn.to(dev, non_blocking=True)
         vd = vn.to(dev, non_blocking=True)
         out = torch.empty_like(qd)
-        ss.launch(d, qd, kd, vd, out)
+        wl.launch(d, qd, kd, vd, out)
         out_host.copy_(out, non_blocking=True)
         stream.synchronize()
         h2d = sum(x.numel() * x.element_size() for x in (q, kn, vn)) + \
-            sum(a.nbytes for a in (p.slot_mapping, p.cow_pairs, p.lens, p.block_tables)) + \
-            (p.group_first.nbytes + p.group_shared.nbytes if p.has_groups else 0)
+            sum(a.nbytes for a in (p.slot_mapping, p.cow_pairs, p.lens, p.block_tables))
+        if shape.chunk:
+            h2d += p.query_start.nbytes
+        elif p.has_groups:
+            h2d += p.group_first.nbytes + p.group_shared.nbytes
         d2h = out_host.numel() * out_host.element_size()
 
     for i in range(W):

@@ -310,13 +310,14 @@ class BlockAllocator:
         if not h:
             raise PagedKVError(INVALID, lib.pkv_last_error().decode())
         self._h = ctypes.c_void_p(h)
+        self._destroy = lib.pkv_alloc_destroy  # kept: module globals may be gone at interpreter exit
         self._slots = np.zeros(64, dtype=np.int64)
         self._cow = np.zeros(2, dtype=np.int32)
 
     def __del__(self):
         h = getattr(self, "_h", None)
         if h is not None and h.value:
-            lib.pkv_alloc_destroy(h)
+            self._destroy(h)
             self._h = None
 
     def seq_add(self, sid: int) -> int:

@@ -44,6 +44,17 @@ class StepPlan:
 
 
 @dataclass
+class ChunkPlan:
+    seq_ids: list
+    slot_mapping: np.ndarray   # int64 [T] slots of the new tokens, sequence by sequence
+    cow_pairs: np.ndarray      # int32 [n, 2]
+    lens: np.ndarray           # int32 [S] context after the write
+    block_tables: np.ndarray   # int32 [S, max_blocks]
+    query_start: np.ndarray    # int32 [S + 1]
+    max_query_len: int
+
+
+@dataclass
 class DevicePlan:
     slot_mapping: torch.Tensor
     cow_pairs: torch.Tensor
@@ -126,6 +137,44 @@ class DecodeSession:
                 plan.max_group_size = int(np.diff(gf).max())
                 plan.max_shared_len = int(gs.max())
         return plan
+
+    def plan_chunk(self, seq_ids: Sequence[int], n_new: Sequence[int]) -> ChunkPlan:
+        """Reserve slots for n_new[i] new tokens of seq_ids[i] (a causal chunk:
+        draft tokens to verify, or part of a prompt)."""
+        ids = np.repeat(np.asarray(seq_ids, dtype=np.int64), np.asarray(n_new, dtype=np.int64))
+        st, slots, pairs = self.alloc.seq_append_slots_batch(ids)
+        self._ok(st)
+        st, bt, lens = self.alloc.seq_block_tables_batch(list(seq_ids), self.max_blocks)
+        self._ok(st)
+        qs = np.concatenate([[0], np.cumsum(n_new)]).astype(np.int32)
+        return ChunkPlan(list(seq_ids), slots, pairs.reshape(-1, 2), lens, bt, qs, int(max(n_new)))
+
+    def launch_chunk(self, d: dict, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor, out: torch.Tensor,
+                     stream=None):
+        """block_copy -> kv_append (all new tokens) -> causal chunk attention."""
+        if d["n_cow"]:
+            B.block_copy(self.k_pool, self.v_pool, d["cow_pairs"], stream=stream)
+        B.kv_append(k_new, v_new, self.k_pool, self.v_pool, d["slot_mapping"], stream=stream)
+        B.paged_attention_chunk(out, q, self.k_pool, self.v_pool, d["block_tables"], d["lens"], d["query_start"],
+                                d["max_query_len"], partition_size=self.partition_size, workspace=self.workspace,
+                                stream=stream)
+        return out
+
+    def chunk_to_device(self, p: ChunkPlan) -> dict:
+        dev = self.device
+
+        def up(a):
+            return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
+        return dict(slot_mapping=up(p.slot_mapping), n_cow=len(p.cow_pairs),
+                    cow_pairs=up(p.cow_pairs) if len(p.cow_pairs) else None, lens=up(p.lens),
+                    block_tables=up(p.block_tables), query_start=up(p.query_start), max_query_len=p.max_query_len)
+
+    def reserve_chunk_workspace(self, num_tokens: int):
+        """Grow the workspace for chunk calls of up to num_tokens query rows."""
+        need = B.attention_chunk_workspace_bytes(num_tokens, self.num_q_heads, self.head_dim,
+                                                 self.max_blocks * self.block_size, self.partition_size)
+        if need > self.workspace.numel():
+            self.workspace = torch.empty(need, dtype=torch.uint8, device=self.device)
 
     def to_device(self, p: StepPlan, non_blocking: bool = False) -> DevicePlan:
         dev = self.device

@@ -51,6 +51,7 @@ class Shape:
     partition_size: int = 0             # 0 = library's choice
     beams: int = 0                      # beams forked per sequence
     pinned_seq0: Optional[list] = None  # explicit physical blocks of seq 0
+    chunk: int = 0                      # new tokens per sequence per step (causal chunk); 0 = decode
     description: str = ""
 
 
@@ -77,6 +78,12 @@ CONFIGS = {
     "llama3_gqa_bs32": Shape("llama3_gqa_bs32", S=128, Hq=32, Hkv=8, D=128, bs=32, dtype="bf16",
                              seed=5, len_fixed=8192, pool_factor=1.0,
                              description="Llama-3-8B-shaped GQA decode: batch 128, 32q/8kv x 128, bf16, ctx 8192, bs 32"),
+    # Speculative verification (an extension beyond the five decode
+    # workloads): Llama-3-8B-shaped GQA, batch 64, 4 draft tokens per
+    # sequence attending causally to contexts of U[1024, 8192].
+    "spec_verify": Shape("spec_verify", S=64, Hq=32, Hkv=8, D=128, bs=16, dtype="bf16", seed=7,
+                         len_uniform=(1024, 8192), chunk=4,
+                         description="speculative verification: batch 64 x 4 draft tokens, 32q/8kv x 128, bf16, bs 16, ctx U[1024,8192]"),
     # Long context + beams: 8 x 100k tokens, 64 q / 8 kv heads, bs 64,
     # split over 512-token partitions; 4 beams fork each sequence.
     "longctx_beam": Shape("longctx_beam", S=8, Hq=64, Hkv=8, D=128, bs=64, dtype="bf16", seed=6,

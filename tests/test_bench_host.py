@@ -19,6 +19,7 @@ import synth
     ("llama13b_prefix", dict(S=5, Hq=1, Hkv=1, D=64)),
     ("llama3_gqa_bs32", dict(S=3, Hq=4, Hkv=1, D=64, len_fixed=300)),
     ("longctx_beam", dict(S=2, Hq=2, Hkv=1, D=64, len_fixed=1000)),
+    ("spec_verify", dict(S=3, Hq=4, Hkv=1, D=64, len_uniform=(20, 300))),
 ])
 def test_workload_steps_on_cpu(cfg, over):
     sh = synth.shrink(synth.CONFIGS[cfg], **over)
@@ -27,8 +28,9 @@ def test_workload_steps_on_cpu(cfg, over):
     lens0 = wl.batch.lens.copy()
     for i in range(3):
         p = wl.plan()
-        assert p.lens.tolist() == (lens0 + i + 1).tolist()
-        T = sh.S * max(1, sh.beams)
+        step = max(1, sh.chunk)
+        assert p.lens.tolist() == (lens0 + step * (i + 1)).tolist()
+        T = sh.S * max(1, sh.beams, sh.chunk)
         assert len(p.slot_mapping) == T and len(set(p.slot_mapping.tolist())) == T
         if sh.beams:
             assert len(p.cow_pairs) == sh.S * (sh.beams - 1) or i > 0

@@ -86,3 +86,32 @@ def test_bad_query_start_is_reported():
     out = run_chunk(b, q, bad, max_n, 0)
     assert pkv.device_error() & pkv.binding.DEVERR_CONTEXT
     del out
+
+
+def test_session_chunk_step_matches_oracle():
+    """DecodeSession: reserve 3 draft tokens per sequence, write their K/V,
+    attend causally; the oracle replays the same writes on the CPU."""
+    import paged_kv_cache_405_b200 as m
+    sh = synth.shrink(synth.CONFIGS["spec_verify"], S=5, len_uniform=(20, 700), chunk=3)
+    b = synth.make_batch(sh)
+    dev = torch.device("cuda")
+    k, v = b.k_pool.to(dev), b.v_pool.to(dev)
+    ss = m.DecodeSession(k, v, sh.Hq, b.max_blocks, free_order=b.free_order, max_batch=sh.S)
+    for s in range(sh.S):
+        ss.add(s, int(b.lens[s]))
+    ss.reserve_chunk_workspace(sh.S * sh.chunk)
+    plan = ss.plan_chunk(list(range(sh.S)), [sh.chunk] * sh.S)
+    T = sh.S * sh.chunk
+    g = torch.Generator().manual_seed(11)
+    q = synth.randn((T, sh.Hq, sh.D), g, torch.bfloat16, "cpu")
+    kn = synth.randn((T, sh.Hkv, sh.D), g, torch.bfloat16, "cpu")
+    vn = synth.randn((T, sh.Hkv, sh.D), g, torch.bfloat16, "cpu")
+    out = torch.empty((T, sh.Hq, sh.D), dtype=torch.bfloat16, device=dev)
+    ss.launch_chunk(ss.chunk_to_device(plan), q.to(dev), kn.to(dev), vn.to(dev), out)
+    kc, vc = b.k_pool.clone(), b.v_pool.clone()
+    oracle.kv_append(kc, vc, kn, vn, plan.slot_mapping)
+    ref = oracle.paged_attention_chunk(q, kc, vc, plan.block_tables, plan.lens, plan.query_start,
+                                       threads=oracle.max_threads())
+    assert m.device_error() == 0
+    assert torch.equal(k.cpu(), kc) and torch.equal(v.cpu(), vc)
+    assert max_err(out, ref) <= TOL[out.dtype]
