@@ -1,0 +1,139 @@
+"""Automatic prefix caching: the oracle's caching allocator pinned by a token
+payload model, and the product's allocator bit-exact against it."""
+import numpy as np
+import pytest
+
+from oracle.allocator import OK, INVALID, NO_FREE_BLOCK, CachingAllocator
+
+
+def caching_ops(seed, n_ops, max_seqs=5, vocab=3):
+    """Prompts drawn from a few shared stems so that prefixes repeat."""
+    rng = np.random.default_rng(seed)
+    stems = [list(rng.integers(0, vocab, size=int(rng.integers(0, 9)))) for _ in range(3)]
+    ops = []
+    for _ in range(n_ops):
+        k = rng.choice(["prompt", "prompt", "tokens", "tokens", "slots", "fork", "free", "free"])
+        a = int(rng.integers(0, max_seqs))
+        if k == "prompt":
+            toks = list(stems[int(rng.integers(0, 3))]) + list(rng.integers(0, vocab, size=int(rng.integers(0, 4))))
+            ops.append(("prompt", a, [int(x) for x in toks]))
+        elif k == "tokens":
+            ops.append(("tokens", a, [int(x) for x in rng.integers(0, vocab, size=int(rng.integers(1, 5)))]))
+        elif k == "slots":
+            ops.append(("slots", a, int(rng.integers(1, 3))))
+        elif k == "fork":
+            ops.append(("fork", a, int(rng.integers(0, max_seqs))))
+        else:
+            ops.append(("free", a))
+    return ops
+
+
+def apply(a, op):
+    k = op[0]
+    if k == "prompt":
+        return a.seq_add_with_prompt(op[1], op[2])
+    if k == "tokens":
+        return a.seq_append_tokens(op[1], op[2])
+    if k == "slots":
+        return a.seq_append_slots(op[1], op[2])
+    if k == "fork":
+        return a.seq_fork(op[1], op[2])
+    return a.seq_free(op[1])
+
+
+def check(a: CachingAllocator, model, data):
+    bs = a.block_size
+    refs = [0] * a.num_blocks
+    for sid, (bt, n) in a.seqs.items():
+        assert len(bt) == -(-n // bs) and len(model[sid]) == n
+        for t in range(n):   # every sequence reads back its own tokens
+            assert data.get(bt[t // bs] * bs + t % bs) == model[sid][t]
+        for b in bt:
+            refs[b] += 1
+    assert refs == a.ref
+    assert all(a.ref[b] == 0 and b in a.key_of for b in a.lru)
+    used = {b for b in range(a.num_blocks) if a.ref[b] > 0}
+    assert len(a.free) + len(a.lru) + len(used) == a.num_blocks
+    assert not (set(a.free) & set(a.lru)) and not (set(a.free) & used)
+    for key, b in a.cache.items():     # a cached block holds exactly its key's tokens
+        assert a.key_of[b] == key
+        assert [data.get(b * bs + o) for o in range(bs)] == list(key[1])
+
+
+def run(a, ops):
+    model, data = {}, {}
+    for op in ops:
+        r = apply(a, op)
+        k = op[0]
+        if k == "prompt" and r[0] == OK:
+            sid, toks = op[1], op[2]
+            n_cached, slots = r[1], r[2]
+            assert n_cached % a.block_size == 0 and len(slots) == len(toks) - n_cached
+            for sl, tok in zip(slots, toks[n_cached:]):
+                data[sl] = tok
+            model[sid] = list(toks)
+        elif k in ("tokens", "slots") and r[0] == OK:
+            st, slots, pairs = r
+            for src, dst in pairs:
+                for o in range(a.block_size):
+                    if src * a.block_size + o in data:
+                        data[dst * a.block_size + o] = data[src * a.block_size + o]
+            toks = op[2] if k == "tokens" else [None] * op[2]
+            for sl, tok in zip(slots, toks):
+                data[sl] = tok
+            model[op[1]] = model[op[1]] + list(toks)
+        elif k == "fork" and r == OK:
+            model[op[2]] = list(model[op[1]])
+        elif k == "free" and r == OK:
+            del model[op[1]]
+        check(a, model, data)
+    return model
+
+
+def test_caching_oracle_payload_model():
+    hits = 0
+    for seed in range(1500):
+        nb = 6 + seed % 5
+        a = CachingAllocator(nb, 2)
+        run(a, caching_ops(seed, 12))
+        hits += a.hits
+    assert hits > 100     # the shared stems were found again
+
+
+def test_hit_counts_closed_form():
+    bs, m = 4, 5
+    prompt = list(range(m * bs + 2))          # 5 full blocks + 2 tokens
+    a = CachingAllocator(64, bs)
+    for k in range(4):
+        st, n_cached, slots = a.seq_add_with_prompt(k, prompt)
+        assert st == OK and n_cached == (0 if k == 0 else m * bs) and len(slots) == len(prompt) - n_cached
+    assert a.cache_stats()["lookups"] == 4 * m and a.cache_stats()["hits"] == 3 * m
+    assert all(a.refcount(b) == 4 for b in a.seq_block_table(0)[1][:m])
+
+
+def test_freed_cached_blocks_are_evicted_oldest_first():
+    bs = 2
+    a = CachingAllocator(6, bs)
+    a.seq_add_with_prompt(0, [1, 2, 3, 4])       # blocks x0, x1 cached
+    a.seq_add_with_prompt(1, [5, 6, 7, 8])       # blocks y0, y1 cached
+    x, y = a.seq_block_table(0)[1], a.seq_block_table(1)[1]
+    a.seq_free(1)                                # y released first ...
+    a.seq_free(0)                                # ... then x
+    assert a.lru == y + x and a.stats()["free_blocks"] == 6
+    st, n_cached, slots = a.seq_add_with_prompt(2, [9, 9, 9, 9, 9, 9])   # 2 free + 1 evicted
+    assert st == OK and n_cached == 0 and a.cache_stats()["evictions"] == 1
+    assert (CachingAllocator.ROOT, (5, 6)) not in a.cache          # y0 (released first) was evicted
+    assert a.cache[(CachingAllocator.ROOT, (1, 2))] == x[0]         # x0 is still cached
+    assert y[0] in a.seq_block_table(2)[1]                           # and its block was reused
+    # the evicted block's key is gone: [5, 6, 7, 8] no longer hits
+    st, n_cached, _ = a.seq_add_with_prompt(3, [5, 6, 7, 8])
+    assert st == NO_FREE_BLOCK or n_cached == 0
+
+
+def test_prompt_that_does_not_fit_changes_nothing():
+    a = CachingAllocator(3, 2)
+    a.seq_add_with_prompt(0, [1, 2, 3, 4])
+    before = (list(a.free), list(a.lru), dict(a.cache), a.cache_stats())
+    st, n_cached, slots = a.seq_add_with_prompt(1, [1, 2, 5, 6, 7, 8, 9])
+    assert st == NO_FREE_BLOCK and 1 not in a.seqs
+    assert before == (list(a.free), list(a.lru), dict(a.cache), a.cache_stats())
