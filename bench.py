@@ -592,6 +592,76 @@ def run_reference(args, world, rank):
     }
 
 
+def run_allocator_bench(args):
+    """Host-only serving simulation of the block allocator with automatic
+    prefix caching: requests whose prompts start with one of a few system
+    prompts (512 tokens, skewed popularity) plus a private suffix, served 64
+    at a time, each then decoding 64 tokens.  Reports the prefix-cache hit
+    rate, the fraction of prompt tokens whose prefill is skipped and the host
+    cost per allocator call, for the product allocator and the oracle."""
+    from paged_kv_cache_405_b200 import BlockAllocator
+    n_req, conc, decode, bs, NB = args.requests, 64, 64, 16, 16384
+
+    def workload():
+        rng = np.random.default_rng(1234)
+        prompts = [rng.integers(0, 32000, size=512).tolist() for _ in range(8)]
+        w = 1.0 / np.arange(1, 9)
+        reqs = []
+        for _ in range(n_req):
+            sys_p = prompts[int(rng.choice(8, p=w / w.sum()))]
+            reqs.append(sys_p + rng.integers(0, 32000, size=int(rng.integers(16, 257))).tolist())
+        return reqs, rng
+
+    def simulate(alloc, limit=None):
+        reqs, rng = workload()
+        if limit is not None:
+            reqs = reqs[:limit]
+        live, nxt, calls, skipped, total = {}, 0, 0, 0, 0
+        t0 = time.perf_counter()
+        nr = len(reqs)
+        while nxt < nr or live:
+            while nxt < nr and len(live) < conc:
+                st, nc, _ = alloc.seq_add_with_prompt(nxt, reqs[nxt])
+                if st != 0:
+                    raise RuntimeError("pool exhausted in the allocator benchmark")
+                calls += 1
+                skipped += nc
+                total += len(reqs[nxt])
+                live[nxt] = decode
+                nxt += 1
+            for sid in list(live):
+                alloc.seq_append_tokens(sid, [int(rng.integers(0, 32000))])
+                calls += 1
+                live[sid] -= 1
+                if live[sid] == 0:
+                    alloc.seq_free(sid)
+                    calls += 1
+                    del live[sid]
+        return time.perf_counter() - t0, calls, skipped, total
+
+    prod = BlockAllocator(NB, bs, prefix_caching=True)
+    t, calls, skipped, total = simulate(prod)
+    cs = prod.cache_stats()
+    # the oracle (snapshots its whole state per call) on a bounded sample,
+    # with the product on the same sample for an exact counter comparison
+    from oracle.allocator import CachingAllocator
+    sample = min(n_req, 20)
+    orc = CachingAllocator(NB, bs)
+    t_o, calls_o, skipped_o, _ = simulate(orc, sample)
+    prod2 = BlockAllocator(NB, bs, prefix_caching=True)
+    _, _, skipped_p2, _ = simulate(prod2, sample)
+    oc = orc.cache_stats()
+    return {
+        "metric": "prefix-cache hit rate and allocator host cost", "mode": "allocator-bench",
+        "requests": n_req, "concurrency": conc, "decode_tokens": decode, "block_size": bs, "num_blocks": NB,
+        "hit_rate": round(cs["hits"] / max(1, cs["lookups"]), 4),
+        "prefill_tokens_skipped_frac": round(skipped / total, 4),
+        "host_us_per_call": round(1e6 * t / calls, 3), "calls": calls, "evictions": cs["evictions"],
+        "oracle": {"host_us_per_call": round(1e6 * t_o / calls_o, 3), "sample_requests": sample,
+                   "same_counters_on_sample": (oc == prod2.cache_stats() and skipped_o == skipped_p2)},
+    }
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -606,11 +676,17 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-step-seconds", type=float, default=3.0)
+    ap.add_argument("--allocator-bench", action="store_true",
+                    help="host-only prefix-caching allocator simulation (prints its own JSON line)")
+    ap.add_argument("--requests", type=int, default=2000)
     ap.add_argument("--clock-warm-s", type=float, default=0.5,
                     help="seconds of untimed repeats before the timed region, while clocks are sampled")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
+    if args.allocator_bench:
+        print(json.dumps(run_allocator_bench(args)), flush=True)
+        return
     world, rank, local = dist_setup()
     if world != args.gpus and rank == 0:
         print("warning: --gpus %d but WORLD_SIZE %d" % (args.gpus, world), file=sys.stderr)

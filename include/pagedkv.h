@@ -351,6 +351,41 @@ pkv_status pkv_seq_append_slots_batch(pkv_alloc* a, const int64_t* seq_ids, int 
 pkv_status pkv_seq_block_tables_batch(const pkv_alloc* a, const int64_t* seq_ids, int n, int32_t* out,
                                       int max_blocks, int32_t* lens_out);
 
+/*
+ * Automatic prefix caching ([E] 7.4: a prompt prefix computed once is reused
+ * by later requests, which skip that part of the prefill; [T] 2.2.3 shared
+ * blocks, 2.2.8 only byte-identical prefixes may share, 2.2.13 hit rate).
+ * Off by default; switch it on before any sequence is registered.  With it
+ * on: every full block filled through pkv_seq_append_tokens or
+ * pkv_seq_add_with_prompt is keyed by its block_size token ids plus the key
+ * of the block before it (exact equality, no hashing of content), so a key
+ * match means an identical whole prefix; a block whose count drops to zero
+ * stays cached (evictable, least recently released first) and counts as
+ * free; a fresh block comes from the free queue first, then by evicting the
+ * oldest evictable block.  Appending without token ids (pkv_seq_append_slots,
+ * _batch) or sharing by block list stops a sequence from registering blocks.
+ */
+pkv_status pkv_alloc_set_prefix_caching(pkv_alloc* a, int enable);
+
+/*
+ * Register a new sequence with its prompt tokens[0..ntok-1]: the longest run
+ * of cached full blocks matching the prompt's leading blocks is reused (their
+ * K/V need not be computed), the rest get fresh slots.  *n_cached = tokens
+ * reused (a multiple of block_size); slots_out[0 .. ntok-*n_cached-1] = slots
+ * of the remaining tokens, for pkv_kv_append.  All-or-nothing.
+ */
+pkv_status pkv_seq_add_with_prompt(pkv_alloc* a, int64_t seq_id, const int32_t* tokens, int ntok,
+                                   int64_t* slots_out, int* n_cached);
+
+/* pkv_seq_append_slots with the new tokens' ids, so that blocks they fill get cached. */
+pkv_status pkv_seq_append_tokens(pkv_alloc* a, int64_t seq_id, const int32_t* tokens, int ntok,
+                                 int64_t* slots_out, int32_t* cow_out, int cow_cap, int* n_cow);
+
+/* Prefix-cache counters: full prompt blocks looked up, found, cached now,
+ * evictable now, evicted so far.  Any pointer may be NULL. */
+pkv_status pkv_prefix_cache_stats(const pkv_alloc* a, int64_t* lookups, int64_t* hits, int* cached_blocks,
+                                  int* evictable_blocks, int64_t* evictions);
+
 /* Drop a sequence; blocks whose count reaches zero return to the free pool ([T] 2.2.2). */
 pkv_status pkv_seq_free(pkv_alloc* a, int64_t seq_id);
 

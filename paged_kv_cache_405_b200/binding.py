@@ -31,6 +31,7 @@ EXPORTS = [
     "pkv_attention_shared_workspace_bytes", "pkv_find_shared_prefix_groups", "pkv_paged_attention_chunk",
     "pkv_attention_chunk_workspace_bytes", "pkv_block_copy", "pkv_device_error", "pkv_launch_count",
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_add", "pkv_seq_share_prefix", "pkv_seq_fork",
+    "pkv_alloc_set_prefix_caching", "pkv_seq_add_with_prompt", "pkv_seq_append_tokens", "pkv_prefix_cache_stats",
     "pkv_seq_append_slots", "pkv_seq_append_slots_batch", "pkv_seq_block_tables_batch", "pkv_seq_free", "pkv_seq_block_table", "pkv_alloc_stats",
     "pkv_block_refcount", "pkv_status_str", "pkv_last_error",
 ]
@@ -80,6 +81,11 @@ def _load():
         "pkv_seq_append_slots_batch": (c_int, [c_vp, c_vp, c_int, c_vp, c_vp, c_int, ctypes.POINTER(c_int)]),
         "pkv_seq_block_tables_batch": (c_int, [c_vp, c_vp, c_int, c_vp, c_int, c_vp]),
         "pkv_seq_free": (c_int, [c_vp, c_i64]),
+        "pkv_alloc_set_prefix_caching": (c_int, [c_vp, c_int]),
+        "pkv_seq_add_with_prompt": (c_int, [c_vp, c_i64, c_vp, c_int, c_vp, ctypes.POINTER(c_int)]),
+        "pkv_seq_append_tokens": (c_int, [c_vp, c_i64, c_vp, c_int, c_vp, c_vp, c_int, ctypes.POINTER(c_int)]),
+        "pkv_prefix_cache_stats": (c_int, [c_vp, ctypes.POINTER(c_i64), ctypes.POINTER(c_i64),
+                                           ctypes.POINTER(c_int), ctypes.POINTER(c_int), ctypes.POINTER(c_i64)]),
         "pkv_seq_block_table": (c_int, [c_vp, c_i64, c_vp, c_int, ctypes.POINTER(c_int),
                                         ctypes.POINTER(c_i64)]),
         "pkv_alloc_stats": (c_int, [c_vp, ctypes.POINTER(c_int), ctypes.POINTER(c_int),
@@ -299,7 +305,7 @@ def launch_count() -> int:
 class BlockAllocator:
     """The library's host block allocator (free pool, refcounts, block tables, COW)."""
 
-    def __init__(self, num_blocks: int, block_size: int, free_order=None):
+    def __init__(self, num_blocks: int, block_size: int, free_order=None, prefix_caching: bool = False):
         self.num_blocks = num_blocks
         self.block_size = block_size
         fo = None
@@ -311,6 +317,8 @@ class BlockAllocator:
             raise PagedKVError(INVALID, lib.pkv_last_error().decode())
         self._h = ctypes.c_void_p(h)
         self._destroy = lib.pkv_alloc_destroy  # kept: module globals may be gone at interpreter exit
+        if prefix_caching:
+            _check(lib.pkv_alloc_set_prefix_caching(self._h, 1))
         self._slots = np.zeros(64, dtype=np.int64)
         self._cow = np.zeros(2, dtype=np.int32)
 
@@ -365,6 +373,38 @@ class BlockAllocator:
         st = lib.pkv_seq_block_tables_batch(self._h, ids.ctypes.data, n, out.ctypes.data, max_blocks,
                                             lens_out.ctypes.data)
         return st, out, lens_out
+
+    def seq_add_with_prompt(self, sid: int, tokens):
+        """Returns (status, cached tokens, slots of the remaining tokens)."""
+        t = np.ascontiguousarray(np.asarray(tokens, dtype=np.int32))
+        slots = np.zeros(max(len(t), 1), dtype=np.int64)
+        nc = ctypes.c_int(0)
+        st = lib.pkv_seq_add_with_prompt(self._h, sid, t.ctypes.data if len(t) else None, len(t),
+                                         slots.ctypes.data, ctypes.byref(nc))
+        if st != OK:
+            return st, 0, []
+        return st, nc.value, slots[:len(t) - nc.value].tolist()
+
+    def seq_append_tokens(self, sid: int, tokens):
+        """Returns (status, slots, [(src, dst)] copy-on-write pairs)."""
+        t = np.ascontiguousarray(np.asarray(tokens, dtype=np.int32))
+        n = len(t)
+        slots = np.zeros(max(n, 1), dtype=np.int64)
+        ncow = ctypes.c_int(0)
+        st = lib.pkv_seq_append_tokens(self._h, sid, t.ctypes.data if n else None, n, slots.ctypes.data,
+                                       self._cow.ctypes.data, 1, ctypes.byref(ncow))
+        if st != OK:
+            return st, [], []
+        pairs = [(int(self._cow[0]), int(self._cow[1]))] if ncow.value else []
+        return st, slots[:n].tolist(), pairs
+
+    def cache_stats(self) -> dict:
+        lk, ht, ev = ctypes.c_int64(0), ctypes.c_int64(0), ctypes.c_int64(0)
+        cb, eb = ctypes.c_int(0), ctypes.c_int(0)
+        _check(lib.pkv_prefix_cache_stats(self._h, ctypes.byref(lk), ctypes.byref(ht), ctypes.byref(cb),
+                                          ctypes.byref(eb), ctypes.byref(ev)))
+        return dict(lookups=lk.value, hits=ht.value, cached_blocks=cb.value, evictable_blocks=eb.value,
+                    evictions=ev.value)
 
     def seq_free(self, sid: int) -> int:
         return lib.pkv_seq_free(self._h, sid)

@@ -17,6 +17,8 @@
 #include <cstdint>
 #include <cstring>
 #include <deque>
+#include <iterator>
+#include <list>
 #include <string>
 #include <unordered_map>
 #include <vector>
@@ -27,10 +29,37 @@ namespace pkv_host {
 void set_error(const std::string& msg);
 }
 
+// Automatic prefix caching (openeuler.csdn.net explainer 7.4: a prompt
+// prefix computed once is reused and its prefill skipped; aiknowledge.cn
+// 2.2.3 shared blocks, 2.2.8 only byte-identical prefixes share, 2.2.13 hit
+// rate).  Only full blocks are cached.  A block's key is (node id of the
+// cached block before it on its sequence -- kRoot for the first block --,
+// its block_size token ids), so equal keys mean identical whole prefixes.
+// Each registration gets a fresh node id.  Cached blocks whose count drops
+// to zero stay cached at the back of an LRU list; fresh blocks come from the
+// free queue first, then by evicting the LRU front (its key is dropped).
+constexpr int64_t kRoot = -1;
+constexpr int64_t kBroken = -2;  // chain unknown: this sequence registers nothing
+
+struct CacheKey {
+    int64_t parent;
+    std::vector<int32_t> toks;
+    bool operator==(const CacheKey& o) const { return parent == o.parent && toks == o.toks; }
+};
+struct CacheKeyHash {
+    size_t operator()(const CacheKey& k) const {
+        uint64_t h = 1469598103934665603ull ^ (uint64_t)k.parent;
+        for (int32_t t : k.toks) h = (h ^ (uint32_t)t) * 1099511628211ull;
+        return (size_t)h;
+    }
+};
+
 struct pkv_alloc {
     struct Seq {
         std::vector<int32_t> table;  // logical block -> physical block
         int64_t len = 0;             // tokens cached
+        int64_t chain = kRoot;       // node of its last cached block (prefix caching)
+        std::vector<int32_t> tail;   // token ids of its partly filled last block
     };
     int num_blocks = 0;
     int block_size = 0;
@@ -40,10 +69,66 @@ struct pkv_alloc {
     int64_t alloc_failures = 0;
     int64_t cow_copies = 0;
 
-    int32_t pop_free() {
-        int32_t b = free_q.front();
-        free_q.pop_front();
+    bool caching = false;
+    std::unordered_map<CacheKey, int32_t, CacheKeyHash> cache;
+    std::vector<CacheKey> key_of;  // per block, valid while node_of >= 0
+    std::vector<int64_t> node_of;  // per block, -1 if not cached
+    std::list<int32_t> lru;        // cached blocks with count 0, oldest first
+    std::vector<std::list<int32_t>::iterator> lru_it;
+    std::vector<char> in_lru;
+    int64_t next_node = 0, lookups = 0, hits = 0, evictions = 0;
+
+    int64_t available() const { return (int64_t)free_q.size() + (int64_t)lru.size(); }
+
+    // A fresh block: the free queue's front, else the least recently released
+    // cached block (its key is dropped).  Callers check available() first.
+    int32_t take() {
+        if (!free_q.empty()) {
+            int32_t b = free_q.front();
+            free_q.pop_front();
+            return b;
+        }
+        int32_t b = lru.front();
+        lru.pop_front();
+        in_lru[b] = 0;
+        cache.erase(key_of[b]);
+        key_of[b].toks.clear();
+        node_of[b] = -1;
+        evictions += 1;
         return b;
+    }
+
+    void release(int32_t b) {
+        if (--ref[b] != 0) return;
+        if (caching && node_of[b] >= 0) {
+            lru.push_back(b);
+            lru_it[b] = std::prev(lru.end());
+            in_lru[b] = 1;
+        } else {
+            free_q.push_back(b);
+        }
+    }
+
+    void revive(int32_t b) {  // a cached block with count 0 found by a lookup
+        if (in_lru[b]) {
+            lru.erase(lru_it[b]);
+            in_lru[b] = 0;
+        }
+        ref[b] += 1;
+    }
+
+    void register_block(Seq& s, int32_t b) {
+        if (s.chain == kBroken) return;
+        CacheKey k{s.chain, s.tail};
+        if (cache.count(k)) {  // this prefix was computed elsewhere: stop this chain
+            s.chain = kBroken;
+            return;
+        }
+        const int64_t node = next_node++;
+        cache.emplace(k, b);
+        key_of[b] = std::move(k);
+        node_of[b] = node;
+        s.chain = node;
     }
 };
 
@@ -63,6 +148,10 @@ pkv_alloc* pkv_alloc_create(int num_blocks, int block_size, const int32_t* free_
     a->num_blocks = num_blocks;
     a->block_size = block_size;
     a->ref.assign(num_blocks, 0);
+    a->key_of.resize(num_blocks);
+    a->node_of.assign(num_blocks, -1);
+    a->lru_it.resize(num_blocks);
+    a->in_lru.assign(num_blocks, 0);
     if (free_order) {
         std::vector<char> seen(num_blocks, 0);
         for (int i = 0; i < num_blocks; ++i) {
@@ -117,6 +206,8 @@ pkv_status pkv_seq_share_prefix(pkv_alloc* a, int64_t seq_id, const int32_t* blo
     for (int i = 0; i < nblocks; ++i) a->ref[blocks[i]] += 1;
     it->second.table.assign(blocks, blocks + nblocks);
     it->second.len = num_tokens;
+    it->second.chain = kBroken;  // token ids unknown
+    it->second.tail.clear();
     return PKV_OK;
 }
 
@@ -133,15 +224,12 @@ pkv_status pkv_seq_fork(pkv_alloc* a, int64_t parent, int64_t child) {
     return PKV_OK;
 }
 
-pkv_status pkv_seq_append_slots(pkv_alloc* a, int64_t seq_id, int ntok, int64_t* slots_out,
-                                int32_t* cow_out, int cow_cap, int* n_cow) {
-    if (!a) return PKV_ERR_INVALID;
-    auto it = a->seqs.find(seq_id);
-    if (it == a->seqs.end() || ntok < 0 || (ntok > 0 && !slots_out)) {
-        set_error("pkv_seq_append_slots: unknown sequence or bad arguments");
-        return PKV_ERR_INVALID;
-    }
-    pkv_alloc::Seq& s = it->second;
+}  // extern "C"
+
+// Reserve slots for ntok tokens of s (tokens: their ids, or nullptr if
+// unknown -- then the sequence registers no more blocks).
+static pkv_status append_impl(pkv_alloc* a, pkv_alloc::Seq& s, int ntok, const int32_t* tokens, int64_t* slots_out,
+                              int32_t* cow_out, int cow_cap, int* n_cow) {
     const int64_t bs = a->block_size;
     const int64_t L = s.len;
     // Only the first new token can land in an existing block (the partly
@@ -153,7 +241,7 @@ pkv_status pkv_seq_append_slots(pkv_alloc* a, int64_t seq_id, int ntok, int64_t*
         set_error("pkv_seq_append_slots: a copy-on-write pair is due but cow_cap < 1");
         return PKV_ERR_INVALID;
     }
-    if (need > (int64_t)a->free_q.size()) {
+    if (need > a->available()) {
         a->alloc_failures += 1;
         set_error("pkv_seq_append_slots: free pool exhausted");
         return PKV_ERR_NO_FREE_BLOCK;
@@ -162,24 +250,126 @@ pkv_status pkv_seq_append_slots(pkv_alloc* a, int64_t seq_id, int ntok, int64_t*
     for (int64_t t = L; t < L + ntok; ++t) {
         int64_t j = t / bs;
         if (j == (int64_t)s.table.size()) {
-            int32_t b = a->pop_free();
+            int32_t b = a->take();
             a->ref[b] = 1;
             s.table.push_back(b);
         } else if (a->ref[s.table[j]] > 1) {
             int32_t src = s.table[j];
-            int32_t dst = a->pop_free();
+            int32_t dst = a->take();
             cow_out[2 * ncow] = src;
             cow_out[2 * ncow + 1] = dst;
             ++ncow;
-            a->ref[src] -= 1;
+            a->release(src);
             a->ref[dst] = 1;
             s.table[j] = dst;
             a->cow_copies += 1;
         }
         slots_out[t - L] = (int64_t)s.table[j] * bs + t % bs;
+        if (a->caching) {
+            if (!tokens) {
+                s.chain = kBroken;
+                s.tail.clear();
+            } else if (s.chain != kBroken) {
+                s.tail.push_back(tokens[t - L]);
+                if (t % bs == bs - 1) {  // block j just filled
+                    a->register_block(s, s.table[j]);
+                    s.tail.clear();
+                }
+            }
+        }
     }
     s.len = L + ntok;
     if (n_cow) *n_cow = ncow;
+    return PKV_OK;
+}
+
+extern "C" {
+
+pkv_status pkv_seq_append_slots(pkv_alloc* a, int64_t seq_id, int ntok, int64_t* slots_out,
+                                int32_t* cow_out, int cow_cap, int* n_cow) {
+    if (!a) return PKV_ERR_INVALID;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end() || ntok < 0 || (ntok > 0 && !slots_out)) {
+        set_error("pkv_seq_append_slots: unknown sequence or bad arguments");
+        return PKV_ERR_INVALID;
+    }
+    return append_impl(a, it->second, ntok, nullptr, slots_out, cow_out, cow_cap, n_cow);
+}
+
+pkv_status pkv_seq_append_tokens(pkv_alloc* a, int64_t seq_id, const int32_t* tokens, int ntok,
+                                 int64_t* slots_out, int32_t* cow_out, int cow_cap, int* n_cow) {
+    if (!a) return PKV_ERR_INVALID;
+    auto it = a->seqs.find(seq_id);
+    if (it == a->seqs.end() || ntok < 0 || (ntok > 0 && (!slots_out || !tokens))) {
+        set_error("pkv_seq_append_tokens: unknown sequence or bad arguments");
+        return PKV_ERR_INVALID;
+    }
+    return append_impl(a, it->second, ntok, tokens, slots_out, cow_out, cow_cap, n_cow);
+}
+
+pkv_status pkv_seq_add_with_prompt(pkv_alloc* a, int64_t seq_id, const int32_t* tokens, int ntok,
+                                   int64_t* slots_out, int* n_cached) {
+    if (n_cached) *n_cached = 0;
+    if (!a || ntok < 0 || (ntok > 0 && (!tokens || !slots_out)) || a->seqs.count(seq_id)) {
+        set_error("pkv_seq_add_with_prompt: sequence exists or bad arguments");
+        return PKV_ERR_INVALID;
+    }
+    const int bs = a->block_size;
+    const int nfull = ntok / bs;
+    std::vector<int32_t> hit;
+    int64_t node = kRoot;
+    if (a->caching) {
+        CacheKey k{kRoot, {}};
+        for (int j = 0; j < nfull; ++j) {
+            k.parent = node;
+            k.toks.assign(tokens + (int64_t)j * bs, tokens + (int64_t)(j + 1) * bs);
+            auto f = a->cache.find(k);
+            if (f == a->cache.end()) break;
+            hit.push_back(f->second);
+            node = a->node_of[f->second];
+        }
+    }
+    int64_t revived = 0;
+    for (int32_t b : hit) revived += a->ref[b] == 0 ? 1 : 0;
+    const int64_t cached = (int64_t)hit.size() * bs;
+    if (ceil_div(ntok - cached, bs) > a->available() - revived) {
+        a->alloc_failures += 1;
+        set_error("pkv_seq_add_with_prompt: free pool exhausted");
+        return PKV_ERR_NO_FREE_BLOCK;
+    }
+    for (int32_t b : hit) a->revive(b);
+    pkv_alloc::Seq s;
+    s.table = hit;
+    s.len = cached;
+    s.chain = node;
+    auto ins = a->seqs.emplace(seq_id, std::move(s));
+    int dummy = 0;
+    append_impl(a, ins.first->second, (int)(ntok - cached), tokens + cached, slots_out, nullptr, 0, &dummy);
+    if (a->caching) {
+        a->lookups += nfull;
+        a->hits += (int64_t)hit.size();
+    }
+    if (n_cached) *n_cached = (int)cached;
+    return PKV_OK;
+}
+
+pkv_status pkv_alloc_set_prefix_caching(pkv_alloc* a, int enable) {
+    if (!a || !a->seqs.empty()) {
+        set_error("pkv_alloc_set_prefix_caching: only before any sequence is registered");
+        return PKV_ERR_INVALID;
+    }
+    a->caching = enable != 0;
+    return PKV_OK;
+}
+
+pkv_status pkv_prefix_cache_stats(const pkv_alloc* a, int64_t* lookups, int64_t* hits, int* cached_blocks,
+                                  int* evictable_blocks, int64_t* evictions) {
+    if (!a) return PKV_ERR_INVALID;
+    if (lookups) *lookups = a->lookups;
+    if (hits) *hits = a->hits;
+    if (cached_blocks) *cached_blocks = (int)a->cache.size();
+    if (evictable_blocks) *evictable_blocks = (int)a->lru.size();
+    if (evictions) *evictions = a->evictions;
     return PKV_OK;
 }
 
@@ -222,7 +412,7 @@ pkv_status pkv_seq_append_slots_batch(pkv_alloc* a, const int64_t* seq_ids, int 
         set_error("pkv_seq_append_slots_batch: cow_cap too small");
         return PKV_ERR_INVALID;
     }
-    if (need > (int64_t)a->free_q.size()) {
+    if (need > a->available()) {
         a->alloc_failures += 1;
         set_error("pkv_seq_append_slots_batch: free pool exhausted");
         return PKV_ERR_NO_FREE_BLOCK;
@@ -271,9 +461,7 @@ pkv_status pkv_seq_free(pkv_alloc* a, int64_t seq_id) {
         set_error("pkv_seq_free: unknown sequence");
         return PKV_ERR_INVALID;
     }
-    for (int32_t b : it->second.table) {
-        if (--a->ref[b] == 0) a->free_q.push_back(b);
-    }
+    for (int32_t b : it->second.table) a->release(b);
     a->seqs.erase(it);
     return PKV_OK;
 }
@@ -300,7 +488,7 @@ pkv_status pkv_seq_block_table(const pkv_alloc* a, int64_t seq_id, int32_t* out,
 pkv_status pkv_alloc_stats(const pkv_alloc* a, int* free_blocks, int* used_blocks,
                            int64_t* alloc_failures, int64_t* cow_copies) {
     if (!a) return PKV_ERR_INVALID;
-    int nfree = (int)a->free_q.size();
+    int nfree = (int)a->available();  // evictable cached blocks are free to reuse
     if (free_blocks) *free_blocks = nfree;
     if (used_blocks) *used_blocks = a->num_blocks - nfree;
     if (alloc_failures) *alloc_failures = a->alloc_failures;

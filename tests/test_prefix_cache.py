@@ -137,3 +137,36 @@ def test_prompt_that_does_not_fit_changes_nothing():
     st, n_cached, slots = a.seq_add_with_prompt(1, [1, 2, 5, 6, 7, 8, 9])
     assert st == NO_FREE_BLOCK and 1 not in a.seqs
     assert before == (list(a.free), list(a.lru), dict(a.cache), a.cache_stats())
+
+
+def test_product_allocator_matches_caching_oracle():
+    from paged_kv_cache_405_b200 import BlockAllocator
+    for seed in range(1500):
+        nb, bs = 6 + seed % 5, (2, 3)[seed % 2]
+        order = np.random.default_rng(seed).permutation(nb)
+        prod = BlockAllocator(nb, bs, order, prefix_caching=True)
+        orc = CachingAllocator(nb, bs, order)
+        for op in caching_ops(seed, 12):
+            r1 = apply(prod, op)
+            r2 = apply(orc, op)
+            assert r1 == r2, (seed, op, r1, r2)
+            assert prod.stats() == orc.stats()
+            assert prod.cache_stats() == orc.cache_stats()
+            for sid in range(5):
+                assert prod.seq_block_table(sid) == orc.seq_block_table(sid)
+            assert [prod.refcount(b) for b in range(nb)] == orc.ref
+
+
+def test_caching_off_behaves_like_plain_allocator():
+    from paged_kv_cache_405_b200 import BlockAllocator
+    from oracle.allocator import Allocator
+    a = BlockAllocator(8, 4)
+    o = Allocator(8, 4)
+    st, n_cached, slots = a.seq_add_with_prompt(0, list(range(10)))
+    o.seq_add(0)
+    assert (st, n_cached) == (OK, 0) and slots == o.seq_append_slots(0, 10)[1]
+    a.seq_free(0)
+    o.seq_free(0)
+    assert a.stats() == o.stats() and a.cache_stats()["cached_blocks"] == 0
+    st, n_cached, _ = a.seq_add_with_prompt(1, list(range(10)))
+    assert n_cached == 0
