@@ -44,6 +44,14 @@ def _load():
         lib.oracle_slot.restype = ctypes.c_int64
         lib.oracle_slot.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int64]
         lib.oracle_max_threads.restype = ctypes.c_int
+        lib.oracle_paged_attention_kv.restype = ctypes.c_int
+        lib.oracle_paged_attention_kv.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+            ctypes.c_double, ctypes.c_double, ctypes.c_void_p, ctypes.c_int, ctypes.c_void_p,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_double,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int]
+        lib.oracle_e4m3_table.restype = None
+        lib.oracle_e4m3_table.argtypes = [ctypes.c_void_p]
         lib.oracle_paged_attention_chunk.restype = ctypes.c_int
         lib.oracle_paged_attention_chunk.argtypes = [
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -145,6 +153,89 @@ def paged_attention_chunk(q, k_pool, v_pool, block_tables, context_lens, query_s
     if rc != 0:
         raise ValueError("oracle_paged_attention_chunk: invalid indices (status %d)" % rc)
     return out.reshape(T, Hq, D) if items is None else out
+
+
+# ----------------------------------------------------------------- FP8 E4M3 KV
+E4M3_MAX = 448.0
+
+
+def e4m3_table() -> np.ndarray:
+    """Value of each of the 256 E4M3 codes (NaN for the two NaN codes)."""
+    out = np.zeros(256, dtype=np.float64)
+    _load().oracle_e4m3_table(out.ctypes.data)
+    return out
+
+
+def quantize_e4m3(x, scale: float) -> np.ndarray:
+    """FP8 E4M3 codes of x / scale, computed as x * (1/scale) in fp32 (the
+    inverse itself rounded to fp32), rounded to nearest (ties to even) and
+    saturated to +-448; NaN stays NaN.  Returns uint8 codes."""
+    xf = np.asarray(_cpu(x).float().numpy(), dtype=np.float32)
+    inv = np.float32(1.0) / np.float32(scale)
+    y = (xf * inv).astype(np.float32).astype(np.float64).ravel()
+    table = e4m3_table()
+    finite = np.arange(256)[np.isfinite(table) & (table >= 0)]           # non-negative codes, ascending
+    vals = table[finite]
+    order = np.argsort(vals, kind="stable")
+    finite, vals = finite[order], vals[order]
+    keep = np.concatenate([[True], np.diff(vals) > 0])                    # +0 only (drop duplicates)
+    finite, vals = finite[keep], vals[keep]
+    a = np.minimum(np.abs(y), E4M3_MAX)
+    hi = np.searchsorted(vals, a, side="left").clip(0, len(vals) - 1)
+    lo = (hi - 1).clip(0, len(vals) - 1)
+    dl, dh = np.abs(a - vals[lo]), np.abs(vals[hi] - a)
+    even_hi = (finite[hi] & 1) == 0
+    pick = np.where(dl < dh, lo, np.where(dh < dl, hi, np.where(even_hi, hi, lo)))
+    code = finite[pick].astype(np.uint8)
+    code = np.where(np.signbit(y), code | 0x80, code).astype(np.uint8)   # rounding keeps the sign (-0 too)
+    code = np.where(np.isnan(y), np.uint8(0x7F), code)
+    return code.reshape(np.shape(xf))
+
+
+def paged_attention_kv(q, k_codes, v_codes, k_scale: float, v_scale: float, block_tables, context_lens,
+                       scale=None, items=None, threads: int = 1) -> np.ndarray:
+    """fp64 decode attention over FP8 E4M3 pools (uint8 codes, values = code
+    value x k_scale / v_scale); q in fp32/bf16/f16."""
+    q = _cpu(q)
+    kc = np.ascontiguousarray(np.asarray(k_codes.cpu() if isinstance(k_codes, torch.Tensor) else k_codes,
+                                         dtype=np.uint8))
+    vc = np.ascontiguousarray(np.asarray(v_codes.cpu() if isinstance(v_codes, torch.Tensor) else v_codes,
+                                         dtype=np.uint8))
+    S, Hq, D = q.shape
+    NB, Hkv, bs, _ = kc.shape
+    bt = np.ascontiguousarray(np.asarray(block_tables, dtype=np.int32))
+    cl = np.ascontiguousarray(np.asarray(context_lens, dtype=np.int32))
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if items is None:
+        ss, hh = np.meshgrid(np.arange(S), np.arange(Hq), indexing="ij")
+        its = np.stack([ss.ravel(), hh.ravel()], 1).astype(np.int32)
+    else:
+        its = np.asarray(items, dtype=np.int32).reshape(-1, 2)
+    its_s, its_h = np.ascontiguousarray(its[:, 0]), np.ascontiguousarray(its[:, 1])
+    out = np.zeros((len(its), D), dtype=np.float64)
+    rc = _load().oracle_paged_attention_kv(
+        out.ctypes.data, q.data_ptr(), _DT[q.dtype], kc.ctypes.data, vc.ctypes.data, 3, float(np.float32(k_scale)),
+        float(np.float32(v_scale)), bt.ctypes.data, bt.shape[1], cl.ctypes.data, S, Hq, Hkv, D, bs, NB,
+        float(scale), its_s.ctypes.data, its_h.ctypes.data, len(its), threads)
+    if rc != 0:
+        raise ValueError("oracle_paged_attention_kv: invalid indices (status %d)" % rc)
+    return out.reshape(S, Hq, D) if items is None else out
+
+
+def kv_append_fp8(k_codes: np.ndarray, v_codes: np.ndarray, k_new, v_new, k_scale: float, v_scale: float,
+                  slot_mapping) -> None:
+    """Quantize each new token's K and V (quantize_e4m3) into its slot of the
+    uint8 code pools, in place; a negative slot means no write."""
+    bs = k_codes.shape[2]
+    kq = quantize_e4m3(k_new, k_scale)
+    vq = quantize_e4m3(v_new, v_scale)
+    for i, sl in enumerate(np.asarray(slot_mapping, dtype=np.int64).tolist()):
+        if sl < 0:
+            continue
+        blk, off = divmod(sl, bs)
+        k_codes[blk, :, off, :] = kq[i]
+        v_codes[blk, :, off, :] = vq[i]
 
 
 def kv_append(k_pool: torch.Tensor, v_pool: torch.Tensor, k_new, v_new, slot_mapping) -> None:

@@ -42,10 +42,22 @@
 #include <omp.h>
 #endif
 
-enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_F16 = 2 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_F16 = 2, ORC_E4M3 = 3 };
+
+/* FP8 E4M3 (sign, 4 exponent bits with bias 7, 3 mantissa bits; no
+ * infinities; exponent 15 with mantissa 7 is NaN; largest finite 448). */
+static double e4m3_value(uint8_t c) {
+    int sign = c >> 7, e = (c >> 3) & 15, m = c & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp((double)(8 + m), e - 10);
+    return sign ? -v : v;
+}
 
 static double widen(const void *base, int64_t i, int dtype) {
     if (dtype == ORC_F32) return (double)((const float *)base)[i];
+    if (dtype == ORC_E4M3) return e4m3_value(((const uint8_t *)base)[i]);
     uint16_t h = ((const uint16_t *)base)[i];
     if (dtype == ORC_BF16) {
         uint32_t u = (uint32_t)h << 16;
@@ -81,12 +93,39 @@ int oracle_max_threads(void) {
  * Returns 0, or -1 on an index outside the given arrays (nothing written for
  * that item then), or -2 on bad shapes.
  */
+/* Decode value of entry i of a K/V pool: code (or element) times its scale. */
+static double pool_value(const void *pool, int64_t i, int kv_dtype, double kv_scale) {
+    return widen(pool, i, kv_dtype) * kv_scale;
+}
+
+/*
+ * Decode attention with K/V pools of their own element type: kv_dtype
+ * ORC_E4M3 means FP8 codes, whose values are code value x k_scale (x
+ * v_scale); for the other types the scales are 1.  q and out as in
+ * oracle_paged_attention.
+ */
+int oracle_paged_attention_kv(double *out, const void *q, int q_dtype, const void *k_pool, const void *v_pool,
+                              int kv_dtype, double k_scale, double v_scale, const int32_t *block_tables,
+                              int max_blocks, const int32_t *context_lens, int S, int Hq, int Hkv, int D,
+                              int block_size, int num_blocks, double scale, const int32_t *items_s,
+                              const int32_t *items_h, int n_items, int num_threads);
+
 int oracle_paged_attention(double *out, const void *q, const void *k_pool, const void *v_pool,
                            const int32_t *block_tables, int max_blocks,
                            const int32_t *context_lens, int S, int Hq, int Hkv, int D,
                            int block_size, int num_blocks, double scale, int dtype,
                            const int32_t *items_s, const int32_t *items_h, int n_items,
                            int num_threads) {
+    return oracle_paged_attention_kv(out, q, dtype, k_pool, v_pool, dtype, 1.0, 1.0, block_tables, max_blocks,
+                                     context_lens, S, Hq, Hkv, D, block_size, num_blocks, scale, items_s,
+                                     items_h, n_items, num_threads);
+}
+
+int oracle_paged_attention_kv(double *out, const void *q, int q_dtype, const void *k_pool, const void *v_pool,
+                              int kv_dtype, double k_scale, double v_scale, const int32_t *block_tables,
+                              int max_blocks, const int32_t *context_lens, int S, int Hq, int Hkv, int D,
+                              int block_size, int num_blocks, double scale, const int32_t *items_s,
+                              const int32_t *items_h, int n_items, int num_threads) {
     if (Hkv <= 0 || Hq % Hkv != 0 || D <= 0 || block_size <= 0) return -2;
     int G = Hq / Hkv;
     int status = 0;
@@ -115,7 +154,8 @@ int oracle_paged_attention(double *out, const void *q, const void *k_pool, const
             int64_t blk = slot / block_size, off = slot % block_size;
             int64_t kbase = ((blk * Hkv + g) * block_size + off) * D;
             double acc = 0.0;
-            for (int d = 0; d < D; ++d) acc += widen(q, qbase + d, dtype) * widen(k_pool, kbase + d, dtype);
+            for (int d = 0; d < D; ++d)
+                acc += widen(q, qbase + d, q_dtype) * pool_value(k_pool, kbase + d, kv_dtype, k_scale);
             x[t] = scale * acc;
             if (x[t] > mx) mx = x[t];
         }
@@ -126,7 +166,7 @@ int oracle_paged_attention(double *out, const void *q, const void *k_pool, const
             int64_t slot = oracle_slot(bt, block_size, t);
             int64_t blk = slot / block_size, off = slot % block_size;
             int64_t vbase = ((blk * Hkv + g) * block_size + off) * D;
-            for (int d = 0; d < D; ++d) o[d] += w * widen(v_pool, vbase + d, dtype);
+            for (int d = 0; d < D; ++d) o[d] += w * pool_value(v_pool, vbase + d, kv_dtype, v_scale);
         }
         for (int d = 0; d < D; ++d) o[d] /= den;
         free(x);
@@ -193,4 +233,9 @@ int oracle_paged_attention_chunk(double *out, const void *q, const void *k_pool,
         free(x);
     }
     return status;
+}
+
+/* Value of every E4M3 code (out[256]), for pinning against other decoders. */
+void oracle_e4m3_table(double *out) {
+    for (int c = 0; c < 256; ++c) out[c] = e4m3_value((uint8_t)c);
 }

@@ -454,3 +454,42 @@ def test_chunk_last_row_sees_whole_context_first_row_sees_its_prefix():
         one = oracle.paged_attention(q[i:i + 1], b.k_pool.float(), b.v_pool.float(), b.block_tables[:1],
                                      [50 - n + i + 1])
         assert np.array_equal(got[i], one[0])
+
+
+# ------------------------------------------------------------- FP8 E4M3 pools
+def test_e4m3_table_matches_torch_float8():
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    got = oracle.e4m3_table()
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    assert np.array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
+
+
+@pytest.mark.parametrize("scale", [1.0, 0.125, 0.37])
+def test_e4m3_quantize_matches_torch_cast_and_saturates(scale):
+    g = torch.Generator().manual_seed(3)
+    x = torch.cat([torch.randn(200000, generator=g) * 60, torch.tensor([0.0, -0.0, 1e-30, -1e-30, 447.9, 448.0,
+                                                                         449.0, 463.9, 1e6, -1e6])])
+    codes = oracle.quantize_e4m3(x, scale)
+    y = (x.float() * (torch.tensor(1.0, dtype=torch.float32) / torch.tensor(scale, dtype=torch.float32)))
+    inside = y.abs() < 448
+    ref = y.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes[inside.numpy()], ref[inside.numpy()])
+    table = oracle.e4m3_table()
+    out = ~inside.numpy()
+    assert np.all(np.abs(table[codes[out]]) == 448.0)                    # saturated, sign kept
+    assert np.array_equal(np.sign(table[codes[out]]), np.sign(y.numpy()[out]))
+
+
+def test_fp8_attention_equals_attention_on_dequantized_values():
+    """Pools of codes with power-of-two scales == the same values held as fp32."""
+    b = synth.make_batch(synth.shrink(synth.CONFIGS["llama3_gqa_bs16"], S=3, Hq=8, Hkv=2, D=64,
+                                      len_fixed=None, len_uniform=(1, 120)))
+    ks, vs = 0.25, 2.0
+    kc = oracle.quantize_e4m3(b.k_pool, ks)
+    vc = oracle.quantize_e4m3(b.v_pool, vs)
+    table = oracle.e4m3_table()
+    kf = torch.from_numpy(table[kc] * ks).float()
+    vf = torch.from_numpy(table[vc] * vs).float()
+    a = oracle.paged_attention_kv(b.q, kc, vc, ks, vs, b.block_tables, b.lens)
+    r = oracle.paged_attention(b.q.float(), kf, vf, b.block_tables, b.lens)
+    assert np.array_equal(a, r)
