@@ -57,7 +57,7 @@ typedef enum {
     PKV_ERR_DEVICE_CHECK = 5    /* pkv_device_error found a recorded bad index */
 } pkv_status;
 
-typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_F16 = 2 } pkv_dtype;
+typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_F16 = 2, PKV_FP8_E4M3 = 3 /* pools of the _fp8 calls only */ } pkv_dtype;
 
 /* Bits of the device error word. */
 #define PKV_DEVERR_BLOCK_ID   1u  /* block id outside [0, num_blocks) */
@@ -227,6 +227,38 @@ pkv_status pkv_paged_attention_chunk(void* out, const void* q, const void* k_poo
 /* Workspace bytes for pkv_paged_attention_chunk (0 if no context needs splitting). */
 size_t pkv_attention_chunk_workspace_bytes(int num_tokens, int num_q_heads, int head_dim, int max_context_len,
                                            int partition_size);
+
+/*
+ * Quantized KV pools: FP8 E4M3 codes (1 byte per element, same layout as the
+ * other pools).  The pages only say that bandwidth decides which precision
+ * serves fastest ([B] 4.2); the scheme here: one scale per pool, a stored
+ * code c stands for e4m3(c) * k_scale (K) or * v_scale (V), halving the bytes
+ * decode attention streams.  E4M3: sign, 4 exponent bits (bias 7), 3 mantissa
+ * bits, largest finite 448, no infinities.
+ *
+ * pkv_kv_append_fp8 -- as pkv_kv_append, but the new K/V (src_dtype: f32,
+ * bf16 or f16) are quantized: code = e4m3(x * (1/scale)), the inverse scale
+ * rounded to fp32 once, the product computed in fp32, rounded to nearest
+ * (ties to even) and saturated to +-448.  head_dim a multiple of 16.
+ */
+pkv_status pkv_kv_append_fp8(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                             const int64_t* slot_mapping, int num_tokens, int num_blocks, int num_kv_heads,
+                             int head_dim, int block_size, pkv_dtype src_dtype, float k_scale, float v_scale,
+                             void* stream);
+
+/*
+ * pkv_paged_attention_decode_fp8 -- pkv_paged_attention_decode over FP8
+ * pools: q and out of type dtype (bf16 or f16), K/V values = code x k_scale /
+ * x v_scale.  Same workspace as pkv_attention_workspace_bytes.  Query groups
+ * of 2..16 heads run on tensor cores in FP16 (codes convert exactly; q is
+ * rounded to FP16 once), others on CUDA cores.
+ */
+pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* k_pool, const void* v_pool,
+                                          const int32_t* block_tables, int max_blocks_per_seq,
+                                          const int32_t* context_lens, int num_seqs, int num_q_heads,
+                                          int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                          float scale, float k_scale, float v_scale, int partition_size,
+                                          void* workspace, size_t workspace_bytes, pkv_dtype dtype, void* stream);
 
 /*
  * pkv_paged_attention_decode_static -- the same decode attention, for callers

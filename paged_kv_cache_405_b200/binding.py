@@ -23,13 +23,14 @@ LIB_PATH = os.environ.get("PKV_LIBRARY") or os.path.join(_HERE, "libpagedkv.so")
 OK, INVALID, NO_FREE_BLOCK, CUDA_ERROR, UNSUPPORTED, DEVICE_CHECK = range(6)
 DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_CONTEXT, DEVERR_TIMEOUT = 1, 2, 4, 8
 _DTYPE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+FP8_E4M3 = 3  # pool element type of the _fp8 calls (uint8 tensors of E4M3 codes)
 
 # Every symbol include/pagedkv.h declares.
 EXPORTS = [
     "pkv_kv_append", "pkv_attention_workspace_bytes", "pkv_attention_partition_size",
     "pkv_paged_attention_decode", "pkv_paged_attention_decode_static", "pkv_paged_attention_decode_shared",
     "pkv_attention_shared_workspace_bytes", "pkv_find_shared_prefix_groups", "pkv_paged_attention_chunk",
-    "pkv_attention_chunk_workspace_bytes", "pkv_block_copy", "pkv_device_error", "pkv_launch_count",
+    "pkv_attention_chunk_workspace_bytes", "pkv_kv_append_fp8", "pkv_paged_attention_decode_fp8", "pkv_block_copy", "pkv_device_error", "pkv_launch_count",
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_add", "pkv_seq_share_prefix", "pkv_seq_fork",
     "pkv_alloc_set_prefix_caching", "pkv_seq_add_with_prompt", "pkv_seq_append_tokens", "pkv_prefix_cache_stats",
     "pkv_seq_append_slots", "pkv_seq_append_slots_batch", "pkv_seq_block_tables_batch", "pkv_seq_free", "pkv_seq_block_table", "pkv_alloc_stats",
@@ -67,6 +68,11 @@ def _load():
                                               c_int, c_int, c_int, c_int, c_int, ctypes.c_float, c_int, c_vp, c_sz,
                                               c_int, c_vp]),
         "pkv_attention_chunk_workspace_bytes": (c_sz, [c_int, c_int, c_int, c_int, c_int]),
+        "pkv_kv_append_fp8": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int,
+                                      ctypes.c_float, ctypes.c_float, c_vp]),
+        "pkv_paged_attention_decode_fp8": (c_int, [c_vp, c_vp, c_vp, c_vp, c_vp, c_int, c_vp, c_int, c_int, c_int,
+                                                   c_int, c_int, c_int, ctypes.c_float, ctypes.c_float,
+                                                   ctypes.c_float, c_int, c_vp, c_sz, c_int, c_vp]),
         "pkv_find_shared_prefix_groups": (c_int, [c_vp, c_vp, c_int, c_int, c_int, c_int, c_vp, c_vp, c_int,
                                                   ctypes.POINTER(c_int)]),
         "pkv_block_copy": (c_int, [c_vp, c_vp, c_vp, c_int, c_int, c_int, c_int, c_int, c_int, c_vp]),
@@ -277,15 +283,49 @@ def paged_attention_chunk(out, q, k_pool, v_pool, block_tables, context_lens, qu
     return out
 
 
+def kv_append_fp8(k_new, v_new, k_pool, v_pool, slot_mapping, k_scale: float, v_scale: float,
+                  stream=None) -> None:
+    """Quantize new K/V ([T, Hkv, D], f32/bf16/f16) into FP8 E4M3 pools (uint8 [NB, Hkv, bs, D])."""
+    NB, Hkv, bs, D = k_pool.shape
+    if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
+        raise TypeError("FP8 pools are uint8 tensors of E4M3 codes")
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    _check(lib.pkv_kv_append_fp8(_dev(k_new, "k_new"), _dev(v_new, "v_new"), _dev(k_pool, "k_pool"),
+                                 _dev(v_pool, "v_pool"), _dev(slot_mapping, "slot_mapping"), k_new.shape[0], NB,
+                                 Hkv, D, bs, _dt(k_new), float(k_scale), float(v_scale), _stream(stream)))
+
+
+def paged_attention_decode_fp8(out, q, k_pool, v_pool, block_tables, context_lens, k_scale: float,
+                               v_scale: float, scale: float = 0.0, partition_size: int = 0,
+                               workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Decode attention over FP8 E4M3 pools (values = code x k_scale / x v_scale); q/out bf16 or f16."""
+    S, Hq, D = q.shape
+    NB, Hkv, bs, D2 = k_pool.shape
+    if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
+        raise TypeError("FP8 pools are uint8 tensors of E4M3 codes")
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    maxB = block_tables.shape[1]
+    if workspace is None:
+        workspace = workspace_for(q, block_tables, bs, partition_size)
+    _check(lib.pkv_paged_attention_decode_fp8(
+        _dev(out, "out"), _dev(q, "q"), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
+        _dev(block_tables, "block_tables"), maxB, _dev(context_lens, "context_lens"), S, Hq, Hkv, D, bs, NB,
+        float(scale), float(k_scale), float(v_scale), int(partition_size), _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _dt(q), _stream(stream)))
+    return out
+
+
 def block_copy(k_pool, v_pool, pairs, stream=None) -> None:
     """Copy whole blocks ``pairs[i] = (src, dst)`` (int32 ``[n, 2]`` on the device), K and V."""
     NB, Hkv, bs, D = k_pool.shape
     if pairs.dtype != torch.int32:
         raise TypeError("pairs must be int32")
     n = pairs.shape[0] if pairs.numel() else 0
+    dt = FP8_E4M3 if k_pool.dtype == torch.uint8 else _dt(k_pool)
     _check(lib.pkv_block_copy(_dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
-                              _dev(pairs, "pairs") if n else None, n, NB, Hkv, D, bs, _dt(k_pool),
-                              _stream(stream)))
+                              _dev(pairs, "pairs") if n else None, n, NB, Hkv, D, bs, dt, _stream(stream)))
 
 
 def device_error(stream=None) -> int:

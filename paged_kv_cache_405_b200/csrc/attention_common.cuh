@@ -16,7 +16,8 @@ struct AttnParams {
     float* ws_o;               // [S][Hq][maxP][D]   (split-K partials)
     float* ws_ml;              // [S][Hq][maxP][2]   (m, l) per partial
     int S, Hq, Hkv, G, bs, NB, maxB, P, maxP, max_len;
-    float scale_log2;          // softmax scale * log2(e)
+    float scale_log2;          // softmax scale * log2(e) (* k_scale for FP8 pools)
+    float v_scale;             // V code scale for FP8 pools (1 otherwise), applied to outputs
     // Shared-prefix groups (num_groups = 0: none).  Group i is the sequences
     // group_first[i] .. group_first[i+1]-1; the first group_shared[i] tokens
     // of each of them sit in the same physical blocks (those of the group's

@@ -32,16 +32,24 @@
 // maps view a pool as a (num_blocks*Hkv*block_size) x D matrix; row
 // (block*Hkv + g)*block_size + offset holds a token's K (or V) for kv head g.
 #pragma once
+#include <type_traits>
+
 #include "attention_common.cuh"
 
 namespace pkv {
 
-template <typename T, int D, int WARPS, int STAGES>
+// Shared memory of one warp: [FP8 only: K and V tiles converted to 16-bit,
+// swizzled] then STAGES stages of (K tile, V tile) as loaded by TMA (16-bit
+// swizzled tiles, or FP8 codes row-major).
+template <typename T, int D, int WARPS, int STAGES, bool FP8 = false>
 struct MmaCfg {
-    static constexpr int kHalfTile = kTileTok * 128;        // 16 rows x 64 elements (bytes)
-    static constexpr int kTileBytes = kTileTok * D * 2;     // one K (or V) tile
-    static constexpr int kStageBytes = 2 * kTileBytes;
-    static constexpr int kDataBytes = WARPS * STAGES * kStageBytes;
+    static constexpr int kHalfTile = kTileTok * 128;                 // 16 rows x 64 16-bit elements (bytes)
+    static constexpr int kTileBytes = kTileTok * D * 2;              // one 16-bit K (or V) tile
+    static constexpr int kStageTile = FP8 ? kTileTok * D : kTileBytes;  // one tile as loaded
+    static constexpr int kStageBytes = 2 * kStageTile;
+    static constexpr int kConvBytes = FP8 ? 2 * kTileBytes : 0;
+    static constexpr int kWarpBytes = (kConvBytes + STAGES * kStageBytes + 1023) / 1024 * 1024;
+    static constexpr int kDataBytes = WARPS * kWarpBytes;
     static constexpr int kSmemBytes = 1024 + kDataBytes + WARPS * STAGES * 8;  // + alignment slack
     static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
 };
@@ -56,15 +64,29 @@ struct MmaAcc {
     float o[NT_O][4];
     float m_lo, m_hi, l_lo, l_hi;
 
+    // Two Tq elements -> a T pair (converted through fp32 when the types differ).
+    template <typename Tq>
+    __device__ __forceinline__ static uint32_t pair(const Tq* p) {
+        const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+        if constexpr (std::is_same<Tq, T>::value) {
+            return w;
+        } else {
+            float f[2];
+            Elt<Tq>::widen2(w, f);
+            return Elt<T>::pack2(f[0], f[1]);
+        }
+    }
+
     // Row pointers (nullptr = zero row).
-    __device__ __forceinline__ void load_q(const T* row_lo, const T* row_hi, int tig) {
+    template <typename Tq>
+    __device__ __forceinline__ void load_q(const Tq* row_lo, const Tq* row_hi, int tig) {
 #pragma unroll
         for (int kk = 0; kk < KSTEPS; ++kk) {
             const int c0 = kk * 16 + 2 * tig;
-            qa[kk][0] = row_lo ? *reinterpret_cast<const uint32_t*>(row_lo + c0) : 0u;
-            qa[kk][1] = row_hi ? *reinterpret_cast<const uint32_t*>(row_hi + c0) : 0u;
-            qa[kk][2] = row_lo ? *reinterpret_cast<const uint32_t*>(row_lo + c0 + 8) : 0u;
-            qa[kk][3] = row_hi ? *reinterpret_cast<const uint32_t*>(row_hi + c0 + 8) : 0u;
+            qa[kk][0] = row_lo ? pair(row_lo + c0) : 0u;
+            qa[kk][1] = row_hi ? pair(row_hi + c0) : 0u;
+            qa[kk][2] = row_lo ? pair(row_lo + c0 + 8) : 0u;
+            qa[kk][3] = row_hi ? pair(row_hi + c0 + 8) : 0u;
         }
 #pragma unroll
         for (int j = 0; j < NT_O; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
@@ -78,17 +100,24 @@ struct MmaAcc {
 // lim_lo, row gid+8 only tokens below lim_hi (causal chunks; pass t_end when
 // every row sees the whole range).  Returns false if a wait on a copy timed
 // out (the unit is then abandoned after draining its copies).
-template <typename T, int D, int WARPS, int STAGES>
+//
+// FP8 mode: TMA brings tiles of E4M3 codes (row-major, one box per tile);
+// after a stage arrives the warp converts its K and V tiles to 16-bit (exact:
+// every E4M3 value is an FP16 value) into the swizzled layout the tensor-core
+// code reads, and the stage is refilled at once.
+template <typename T, int D, int WARPS, int STAGES, bool FP8 = false>
 __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                            uint8_t* ring, uint32_t bar0, const int32_t* bt_row, int t_begin,
                                            int t_end, int g, int lane, MmaAcc<T, D>& acc, int lim_lo,
                                            int lim_hi) {
-    using C = MmaCfg<T, D, WARPS, STAGES>;
+    using C = MmaCfg<T, D, WARPS, STAGES, FP8>;
     constexpr int KSTEPS = D / 16;
     constexpr int NT_O = D / 8;
     const int tig = lane & 3;
     const int ntiles = (t_end - t_begin + kTileTok - 1) / kTileTok;
-    const uint32_t ring_s = smem_u32(ring);
+    const uint32_t conv_s = smem_u32(ring);
+    uint8_t* stages = ring + C::kConvBytes;
+    const uint32_t ring_s = smem_u32(stages);
 
     const int jb0 = t_begin / p.bs;
     BlockWindow win;
@@ -104,10 +133,15 @@ __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMa
             const uint32_t dst = ring_s + st * C::kStageBytes;
             fence_proxy_async();
             mbar_arrive_expect_tx(bar, C::kStageBytes);
+            if constexpr (FP8) {
+                tma_load_2d(dst, tmK, 0, row, bar);
+                tma_load_2d(dst + C::kStageTile, tmV, 0, row, bar);
+            } else {
 #pragma unroll
-            for (int hx = 0; hx < D / 64; ++hx) {
-                tma_load_2d(dst + hx * C::kHalfTile, tmK, hx * 64, row, bar);
-                tma_load_2d(dst + C::kTileBytes + hx * C::kHalfTile, tmV, hx * 64, row, bar);
+                for (int hx = 0; hx < D / 64; ++hx) {
+                    tma_load_2d(dst + hx * C::kHalfTile, tmK, hx * 64, row, bar);
+                    tma_load_2d(dst + C::kTileBytes + hx * C::kHalfTile, tmV, hx * 64, row, bar);
+                }
             }
         }
     };
@@ -132,7 +166,39 @@ __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMa
         const int valid = min(kTileTok, t_end - (t_begin + i * kTileTok));
         const int seen_lo = min(valid, lim_lo - (t_begin + i * kTileTok));  // tokens row gid sees
         const int seen_hi = min(valid, lim_hi - (t_begin + i * kTileTok));  // ... and row gid+8
-        const uint32_t Ks = ring_s + st * C::kStageBytes;
+        uint32_t Ks = ring_s + st * C::kStageBytes;
+        uint8_t* vtile = stages + st * C::kStageBytes + C::kTileBytes;
+        if constexpr (FP8) {
+            // E4M3 codes (row-major, D bytes per token) -> 16-bit swizzled tiles.
+            const uint8_t* src = stages + st * C::kStageBytes;
+#pragma unroll
+            for (int kv = 0; kv < 2; ++kv) {
+#pragma unroll
+                for (int k = 0; k < D / 32; ++k) {
+                    const int q16 = k * 32 + lane;       // 16-code piece of the tile
+                    const int r = q16 / (D / 16), c16 = q16 % (D / 16);
+                    const uint4 w = *reinterpret_cast<const uint4*>(src + kv * C::kStageTile + r * D + c16 * 16);
+                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+                    uint32_t h[8];
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        h[2 * j] = e4m3x2_to_f16x2((uint16_t)(ww[j] & 0xffffu));
+                        h[2 * j + 1] = e4m3x2_to_f16x2((uint16_t)(ww[j] >> 16));
+                    }
+#pragma unroll
+                    for (int hc = 0; hc < 2; ++hc) {   // two 8-element (16-byte) chunks
+                        const int ch = c16 * 2 + hc;
+                        uint8_t* dst = ring + kv * C::kTileBytes + (ch >> 3) * C::kHalfTile + r * 128 +
+                                       (((ch & 7) ^ (r & 7)) << 4);
+                        *reinterpret_cast<uint4*>(dst) = make_uint4(h[4 * hc], h[4 * hc + 1], h[4 * hc + 2], h[4 * hc + 3]);
+                    }
+                }
+            }
+            __syncwarp();
+            if (i + STAGES < ntiles) issue(i + STAGES);  // the stage is free again
+            Ks = conv_s;
+            vtile = ring + C::kTileBytes;
+        }
         const uint32_t Vs = Ks + C::kTileBytes;
 
         // S = Q K^T  (16 rows x 16 tokens as two n-tiles of 8 tokens)
@@ -201,7 +267,7 @@ __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMa
         // Rows past the context may hold anything (even NaN): zero them in V so
         // that 0-weights cannot turn into NaN inside the MMA.
         if (valid < kTileTok) {
-            uint8_t* vrow = ring + st * C::kStageBytes + C::kTileBytes;
+            uint8_t* vrow = vtile;
             for (int idx = lane; idx < (kTileTok - valid) * (D / 8); idx += 32) {
                 const int r = valid + idx / (D / 8);
                 const int q16 = idx % (D / 8);  // 16-byte unit in the row (any order)
@@ -223,7 +289,7 @@ __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMa
             mma_16816<T>(acc.o[2 * jj + 1], pa, b2, b3);
         }
         __syncwarp();
-        if (i + STAGES < ntiles) issue(i + STAGES);
+        if (!FP8 && i + STAGES < ntiles) issue(i + STAGES);
     }
 #pragma unroll
     for (int off = 1; off < 4; off <<= 1) {
@@ -233,32 +299,34 @@ __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMa
     return true;
 }
 
-// Write one accumulator row: the normalised output (out_row != nullptr) or a
-// split-K partial (o_row, ml).  hi selects rows gid+8.
-template <typename T, int D>
-__device__ __forceinline__ void mma_store_row(const MmaAcc<T, D>& acc, bool hi, int tig, T* out_row, float* o_row,
-                                              float* ml) {
+// Write one accumulator row, scaled by vs (the V code scale, 1 for 16-bit
+// pools): the normalised output of type To (out_row != nullptr) or a split-K
+// partial (o_row, ml).  hi selects rows gid+8.
+template <typename To, typename T, int D>
+__device__ __forceinline__ void mma_store_row(const MmaAcc<T, D>& acc, bool hi, int tig, To* out_row, float* o_row,
+                                              float* ml, float vs) {
     constexpr int NT_O = D / 8;
     const int e0 = hi ? 2 : 0;
     const float l = hi ? acc.l_hi : acc.l_lo;
     if (out_row) {
-        const float inv = 1.f / l;
+        const float inv = vs / l;
 #pragma unroll
         for (int j = 0; j < NT_O; ++j)
             *reinterpret_cast<uint32_t*>(out_row + j * 8 + 2 * tig) =
-                Elt<T>::pack2(acc.o[j][e0] * inv, acc.o[j][e0 + 1] * inv);
+                Elt<To>::pack2(acc.o[j][e0] * inv, acc.o[j][e0 + 1] * inv);
     } else {
 #pragma unroll
         for (int j = 0; j < NT_O; ++j)
-            *reinterpret_cast<float2*>(o_row + j * 8 + 2 * tig) = make_float2(acc.o[j][e0], acc.o[j][e0 + 1]);
+            *reinterpret_cast<float2*>(o_row + j * 8 + 2 * tig) =
+                make_float2(acc.o[j][e0] * vs, acc.o[j][e0 + 1] * vs);
         if (tig == 0) *reinterpret_cast<float2*>(ml) = make_float2(hi ? acc.m_hi : acc.m_lo, l);
     }
 }
 
-template <typename T, int D, int WARPS, int STAGES>
+template <typename T, int D, int WARPS, int STAGES, bool FP8 = false>
 __device__ __forceinline__ uint8_t* mma_setup_ring(uint8_t* smem_raw, int warp, int lane, uint32_t& bar0,
                                                    const CUtensorMap* tmK, const CUtensorMap* tmV) {
-    using C = MmaCfg<T, D, WARPS, STAGES>;
+    using C = MmaCfg<T, D, WARPS, STAGES, FP8>;
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     bar0 = smem_u32(smem + C::kDataBytes + warp * STAGES * 8);
     if (lane == 0) {
@@ -268,11 +336,13 @@ __device__ __forceinline__ uint8_t* mma_setup_ring(uint8_t* smem_raw, int warp, 
         fence_barrier_init();
     }
     __syncwarp();
-    return smem + warp * STAGES * C::kStageBytes;
+    return smem + warp * C::kWarpBytes;
 }
 
-// Grouped-query decode: grid (ceil(Hkv / WARPS), partitions, S).
-template <typename T, int D, int WARPS, int STAGES>
+// Grouped-query decode: grid (ceil(Hkv / WARPS), partitions, S).  T is the
+// MMA type; To the type of q and out (T itself, or bf16 q/out with FP8 pools
+// computed in FP16).
+template <typename T, int D, int WARPS, int STAGES, bool FP8 = false, typename To = T>
 __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnParams p,
                                                                     const __grid_constant__ CUtensorMap tmK,
                                                                     const __grid_constant__ CUtensorMap tmV) {
@@ -290,19 +360,19 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnPa
     const Unit u = resolve_unit(p, s, part, part == 0 && g == 0 && lane == 0);
     if (u.t_begin >= u.L) {
         if (part == 0 && u.L == 0) {  // empty context: zeros for the group's heads
-            T* o = reinterpret_cast<T*>(p.out) + ((int64_t)s * p.Hq + h0) * D;
-            for (int i = lane; i < G * D; i += 32) o[i] = T(0.f);
+            To* o = reinterpret_cast<To*>(p.out) + ((int64_t)s * p.Hq + h0) * D;
+            for (int i = lane; i < G * D; i += 32) o[i] = To(0.f);
         }
         return;
     }
     uint32_t bar0;
-    uint8_t* ring = mma_setup_ring<T, D, WARPS, STAGES>(smem_raw, warp, lane, bar0, &tmK, &tmV);
+    uint8_t* ring = mma_setup_ring<T, D, WARPS, STAGES, FP8>(smem_raw, warp, lane, bar0, &tmK, &tmV);
 
-    const T* qb = reinterpret_cast<const T*>(p.q) + ((int64_t)s * p.Hq + h0) * D;
+    const To* qb = reinterpret_cast<const To*>(p.q) + ((int64_t)s * p.Hq + h0) * D;
     MmaAcc<T, D> acc;
     acc.load_q(gid < G ? qb + gid * D : nullptr, gid + 8 < G ? qb + (gid + 8) * D : nullptr, tig);
-    if (!mma_attend<T, D, WARPS, STAGES>(p, &tmK, &tmV, ring, bar0, p.block_tables + (int64_t)s * p.maxB,
-                                         u.t_begin, u.t_end, g, lane, acc, u.t_end, u.t_end))
+    if (!mma_attend<T, D, WARPS, STAGES, FP8>(p, &tmK, &tmV, ring, bar0, p.block_tables + (int64_t)s * p.maxB,
+                                              u.t_begin, u.t_end, g, lane, acc, u.t_end, u.t_end))
         return;
 
 #pragma unroll
@@ -311,10 +381,10 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnPa
         if (r >= G) continue;
         const int64_t row = (int64_t)s * p.Hq + h0 + r;
         if (u.direct) {
-            mma_store_row<T, D>(acc, hi, tig, reinterpret_cast<T*>(p.out) + row * D, nullptr, nullptr);
+            mma_store_row<To, T, D>(acc, hi, tig, reinterpret_cast<To*>(p.out) + row * D, nullptr, nullptr, p.v_scale);
         } else {
             const int64_t idx = row * p.maxP + u.slot;
-            mma_store_row<T, D>(acc, hi, tig, nullptr, p.ws_o + idx * D, p.ws_ml + idx * 2);
+            mma_store_row<To, T, D>(acc, hi, tig, (To*)nullptr, p.ws_o + idx * D, p.ws_ml + idx * 2, p.v_scale);
         }
     }
 }
@@ -509,10 +579,10 @@ __global__ void __launch_bounds__(WARPS * 32, 3) chunk_attn_mma_kernel(const Att
         if (!use[hi] || lim[hi] <= t_begin) continue;  // no token of this row in the partition
         const int64_t row = (int64_t)(q0 + ri[hi]) * p.Hq + rh[hi];
         if (direct) {
-            mma_store_row<T, D>(acc, hi, tig, reinterpret_cast<T*>(p.out) + row * D, nullptr, nullptr);
+            mma_store_row<T, T, D>(acc, hi, tig, reinterpret_cast<T*>(p.out) + row * D, nullptr, nullptr, p.v_scale);
         } else {
             const int64_t idx = row * p.maxP + part;
-            mma_store_row<T, D>(acc, hi, tig, nullptr, p.ws_o + idx * D, p.ws_ml + idx * 2);
+            mma_store_row<T, T, D>(acc, hi, tig, (T*)nullptr, p.ws_o + idx * D, p.ws_ml + idx * 2, p.v_scale);
         }
     }
 }

@@ -38,7 +38,7 @@ static pkv_status cuda_fail(const char* where, cudaError_t e) {
 
 static bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
-static int elem_size(pkv_dtype dt) { return dt == PKV_F32 ? 4 : 2; }
+static int elem_size(pkv_dtype dt) { return dt == PKV_F32 ? 4 : dt == PKV_FP8_E4M3 ? 1 : 2; }
 
 static bool valid_dtype(int dt) { return dt == PKV_F32 || dt == PKV_BF16 || dt == PKV_F16; }
 
@@ -117,7 +117,8 @@ static bool make_pool_map(CUtensorMap* map, const void* pool, int64_t rows, int 
     cuuint32_t estr[2] = {1, 1};
     const CUtensorMapDataType ty = dt == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                    : dt == PKV_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
-                                                   : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+                                   : dt == PKV_FP8_E4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
     CUresult r = fn(map, ty, 2, const_cast<void*>(pool), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                     swizzled ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -219,6 +220,37 @@ static cudaError_t launch_chunk(const pkv::AttnParams& p, const pkv::ChunkParams
     return cudaGetLastError();
 }
 
+// FP8 pools: stages of E4M3 tiles converted to FP16 per warp.
+#ifndef PKV_FP8_STAGES
+#define PKV_FP8_STAGES 4
+#endif
+constexpr int kFp8Stages = PKV_FP8_STAGES;
+
+template <typename To, int D>
+static cudaError_t launch_mma_fp8(const pkv::AttnParams& p, dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv,
+                                  cudaStream_t st) {
+    using C = pkv::MmaCfg<__half, D, kMmaWarps, kFp8Stages, true>;
+    auto k = pkv::paged_attn_mma_kernel<__half, D, kMmaWarps, kFp8Stages, true, To>;
+    static cudaError_t attr = set_smem(k, C::kSmemBytes);
+    if (attr != cudaSuccess) return attr;
+    k<<<grid, kMmaWarps * 32, C::kSmemBytes, st>>>(p, mk, mv);
+    g_launches++;
+    return cudaGetLastError();
+}
+
+template <typename To, int D>
+static cudaError_t launch_simt_fp8(const pkv::AttnParams& p, dim3 grid, cudaStream_t st) {
+    using C = pkv::SimtCfg<To, D, kSimtWarps, kSimtStages, kSimtTile, pkv::fp8e4m3>;
+    auto k = pkv::paged_attn_simt_kernel<To, D, kSimtWarps, kSimtStages, kSimtTile, false, pkv::fp8e4m3>;
+    static cudaError_t attr = set_smem(k, C::kSmemBytes);
+    if (attr != cudaSuccess) return attr;
+    CUtensorMap none;
+    std::memset(&none, 0, sizeof none);
+    k<<<grid, kSimtWarps * 32, C::kSmemBytes, st>>>(p, none, none);
+    g_launches++;
+    return cudaGetLastError();
+}
+
 template <typename T, int D>
 static cudaError_t launch_reduce(const pkv::ReduceParams& r, cudaStream_t st) {
     const unsigned rows = (unsigned)((r.query_start ? r.T : r.S) * r.Hq);
@@ -257,6 +289,29 @@ static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int npart
     return D == 64 ? launch_reduce<T, 64>(r, st) : launch_reduce<T, 128>(r, st);
 }
 
+template <typename To>
+static cudaError_t dispatch_attention_fp8(const pkv::AttnParams& p, int D, int nparts, bool use_mma,
+                                          const CUtensorMap* mk, const CUtensorMap* mv, cudaStream_t st) {
+    cudaError_t e;
+    if (use_mma) {
+        dim3 grid((p.Hkv + kMmaWarps - 1) / kMmaWarps, nparts, p.S);
+        e = D == 64 ? launch_mma_fp8<To, 64>(p, grid, *mk, *mv, st) : launch_mma_fp8<To, 128>(p, grid, *mk, *mv, st);
+    } else {
+        dim3 grid((p.Hq + kSimtWarps - 1) / kSimtWarps, nparts, p.S);
+        e = D == 64 ? launch_simt_fp8<To, 64>(p, grid, st) : launch_simt_fp8<To, 128>(p, grid, st);
+    }
+    if (e != cudaSuccess || p.maxP <= 1) return e;
+    pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
+                        nullptr, nullptr, 0, 0, nullptr, 0};
+    return D == 64 ? launch_reduce<To, 64>(r, st) : launch_reduce<To, 128>(r, st);
+}
+
+struct KvArgs {
+    pkv_dtype dtype = PKV_BF16;  // pool element type (the call's type unless FP8)
+    bool fp8 = false;
+    float k_scale = 1.f, v_scale = 1.f;
+};
+
 struct GroupArgs {
     const int32_t* first = nullptr;
     const int32_t* shared = nullptr;
@@ -270,8 +325,20 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
                               const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
                               int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                               int num_blocks, float scale, int partition_size, const GroupArgs& grp, void* workspace,
-                              size_t workspace_bytes, pkv_dtype dtype, void* stream) {
+                              size_t workspace_bytes, pkv_dtype dtype, void* stream, const KvArgs& kv = KvArgs()) {
     if (!valid_dtype(dtype)) return invalid("pkv_paged_attention_decode: bad dtype");
+    if (kv.fp8) {
+        if (dtype == PKV_F32) {
+            g_msg = "pkv_paged_attention_decode_fp8: q/out must be bf16 or f16";
+            return PKV_ERR_UNSUPPORTED;
+        }
+        if (!(std::isfinite(kv.k_scale) && std::isfinite(kv.v_scale)) || kv.k_scale <= 0.f || kv.v_scale <= 0.f)
+            return invalid("pkv_paged_attention_decode_fp8: k_scale and v_scale must be positive and finite");
+        if (grp.mode) {
+            g_msg = "pkv_paged_attention_decode_fp8: no shared-prefix mode for FP8 pools";
+            return PKV_ERR_UNSUPPORTED;
+        }
+    }
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
         return invalid("pkv_paged_attention_decode: sizes must be positive");
     if (num_q_heads % num_kv_heads != 0)
@@ -329,6 +396,7 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
     }
 
     pkv::AttnParams p;
+    std::memset(&p, 0, sizeof p);
     p.out = out;
     p.q = q;
     p.k_pool = k_pool;
@@ -349,7 +417,8 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
     p.maxP = (int)slots;
     p.max_len = max_len;
     const float sc = scale > 0.f ? scale : 1.f / std::sqrt((float)head_dim);
-    p.scale_log2 = sc * 1.4426950408889634f;
+    p.scale_log2 = sc * 1.4426950408889634f * (kv.fp8 ? kv.k_scale : 1.f);
+    p.v_scale = kv.fp8 ? kv.v_scale : 1.f;
     p.group_first = grp.num > 0 ? grp.first : nullptr;
     p.group_shared = grp.num > 0 ? grp.shared : nullptr;
     p.num_groups = grp.num;
@@ -358,6 +427,20 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
 
     const bool use_mma = dtype != PKV_F32 && p.G >= 2 && p.G <= 16;
     CUtensorMap mk, mv;
+    if (kv.fp8) {
+        const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
+        if (use_mma && (!make_pool_map(&mk, k_pool, rows, head_dim, PKV_FP8_E4M3, false) ||
+                        !make_pool_map(&mv, v_pool, rows, head_dim, PKV_FP8_E4M3, false))) {
+            g_msg = "pkv_paged_attention_decode_fp8: cuTensorMapEncodeTiled failed";
+            return PKV_ERR_CUDA;
+        }
+        cudaError_t e = dtype == PKV_BF16
+                            ? dispatch_attention_fp8<__nv_bfloat16>(p, head_dim, (int)nparts, use_mma, &mk, &mv,
+                                                                    (cudaStream_t)stream)
+                            : dispatch_attention_fp8<__half>(p, head_dim, (int)nparts, use_mma, &mk, &mv,
+                                                             (cudaStream_t)stream);
+        return e == cudaSuccess ? PKV_OK : cuda_fail("pkv_paged_attention_decode_fp8", e);
+    }
     if (use_mma || (grp.mode && grp.num > 0)) {
         const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
         if (!make_pool_map(&mk, k_pool, rows, head_dim, dtype, true) || !make_pool_map(&mv, v_pool, rows, head_dim, dtype, true)) {
@@ -493,7 +576,7 @@ size_t pkv_attention_shared_workspace_bytes(int num_seqs, int num_q_heads, int h
 
 pkv_status pkv_block_copy(void* k_pool, void* v_pool, const int32_t* pairs, int num_pairs, int num_blocks,
                           int num_kv_heads, int head_dim, int block_size, pkv_dtype dtype, void* stream) {
-    if (!valid_dtype(dtype)) return invalid("pkv_block_copy: bad dtype");
+    if (!valid_dtype(dtype) && dtype != PKV_FP8_E4M3) return invalid("pkv_block_copy: bad dtype");
     if (num_pairs < 0 || num_blocks <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
         return invalid("pkv_block_copy: sizes must be positive");
     const int64_t block_bytes = (int64_t)num_kv_heads * block_size * head_dim * elem_size(dtype);
@@ -538,6 +621,71 @@ pkv_status pkv_device_error(void* stream, uint32_t* code) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// FP8 E4M3 pools.
+// ---------------------------------------------------------------------------
+extern "C" pkv_status pkv_kv_append_fp8(const void* k_new, const void* v_new, void* k_pool, void* v_pool,
+                                        const int64_t* slot_mapping, int num_tokens, int num_blocks,
+                                        int num_kv_heads, int head_dim, int block_size, pkv_dtype src_dtype,
+                                        float k_scale, float v_scale, void* stream) {
+    using namespace pkv_host;
+    if (src_dtype != PKV_F32 && src_dtype != PKV_BF16 && src_dtype != PKV_F16)
+        return invalid("pkv_kv_append_fp8: new K/V must be f32, bf16 or f16");
+    if (num_tokens < 0 || num_blocks <= 0 || num_kv_heads <= 0 || head_dim <= 0 || block_size <= 0)
+        return invalid("pkv_kv_append_fp8: sizes must be positive");
+    if (head_dim % 16 != 0) return invalid("pkv_kv_append_fp8: head_dim must be a multiple of 16");
+    if (!(std::isfinite(k_scale) && std::isfinite(v_scale)) || k_scale <= 0.f || v_scale <= 0.f)
+        return invalid("pkv_kv_append_fp8: k_scale and v_scale must be positive and finite");
+    if (num_tokens == 0) return PKV_OK;
+    if (!k_new || !v_new || !k_pool || !v_pool || !slot_mapping) return invalid("pkv_kv_append_fp8: null pointer");
+    if (!aligned16(k_new) || !aligned16(v_new) || !aligned16(k_pool) || !aligned16(v_pool) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+        return invalid("pkv_kv_append_fp8: pointers must be 16-byte aligned (slot_mapping 8-byte)");
+    pkv::AppendFp8Params p;
+    p.k_new = k_new;
+    p.v_new = v_new;
+    p.k_pool = static_cast<uint4*>(k_pool);
+    p.v_pool = static_cast<uint4*>(v_pool);
+    p.slot_mapping = slot_mapping;
+    p.vecs_per_row = head_dim / 16;
+    p.Hkv = num_kv_heads;
+    p.bs = block_size;
+    p.num_slots = (int64_t)num_blocks * block_size;
+    p.total_vecs = (int64_t)num_tokens * num_kv_heads * p.vecs_per_row;
+    p.k_inv = 1.0f / k_scale;  // the inverse is rounded to fp32 once, on the host
+    p.v_inv = 1.0f / v_scale;
+    int64_t blocks = (p.total_vecs + 255) / 256;
+    const int64_t cap = (int64_t)num_sms() * 16;
+    if (blocks > cap) blocks = cap;
+    cudaStream_t st = (cudaStream_t)stream;
+    switch (src_dtype) {
+        case PKV_F32: pkv::kv_append_fp8_kernel<float><<<(unsigned)blocks, 256, 0, st>>>(p); break;
+        case PKV_BF16: pkv::kv_append_fp8_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(p); break;
+        default: pkv::kv_append_fp8_kernel<__half><<<(unsigned)blocks, 256, 0, st>>>(p); break;
+    }
+    g_launches++;
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? PKV_OK : cuda_fail("pkv_kv_append_fp8", e);
+}
+
+extern "C" pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* k_pool,
+                                                     const void* v_pool, const int32_t* block_tables,
+                                                     int max_blocks_per_seq, const int32_t* context_lens,
+                                                     int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                                     int block_size, int num_blocks, float scale, float k_scale,
+                                                     float v_scale, int partition_size, void* workspace,
+                                                     size_t workspace_bytes, pkv_dtype dtype, void* stream) {
+    using namespace pkv_host;
+    KvArgs kv;
+    kv.dtype = PKV_FP8_E4M3;
+    kv.fp8 = true;
+    kv.k_scale = k_scale;
+    kv.v_scale = v_scale;
+    return decode_impl(out, q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads,
+                       num_kv_heads, head_dim, block_size, num_blocks, scale, partition_size, GroupArgs(), workspace,
+                       workspace_bytes, dtype, stream, kv);
+}
 
 // ---------------------------------------------------------------------------
 // Causal attention for a chunk of new tokens per sequence.
@@ -650,6 +798,7 @@ extern "C" pkv_status pkv_paged_attention_chunk(void* out, const void* q, const 
     p.max_len = max_len;
     const float sc = scale > 0.f ? scale : 1.f / std::sqrt((float)head_dim);
     p.scale_log2 = sc * 1.4426950408889634f;
+    p.v_scale = 1.f;
     pkv::ChunkParams c{query_start, num_tokens, max_query_len, (int)nparts};
     CUtensorMap mk, mv;
     const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;

@@ -1,0 +1,96 @@
+"""GPU parity of the FP8 E4M3 pools: quantizing append byte for byte, decode
+attention element by element, against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_helpers import TOL, max_err
+
+pytestmark = pytest.mark.gpu
+
+
+def fp8_pools(b, seed, k_scale, v_scale):
+    """E4M3 code pools: N(0,1) values / scale cast by torch's float8_e4m3fn;
+    rows no context covers hold the NaN code."""
+    g = torch.Generator().manual_seed(seed)
+    shape = tuple(b.k_pool.shape)
+    kc = (torch.randn(shape, generator=g) / k_scale).to(torch.float8_e4m3fn).view(torch.uint8)
+    vc = (torch.randn(shape, generator=g) / v_scale).to(torch.float8_e4m3fn).view(torch.uint8)
+    covered = torch.zeros(shape[0], shape[2], dtype=torch.bool)
+    bs = shape[2]
+    for s in range(b.shape.S):
+        L = int(b.lens[s])
+        for j in range(-(-L // bs)):
+            covered[int(b.block_tables[s, j]), : min(bs, L - j * bs)] = True
+    mask = ~covered[:, None, :, None].expand(shape)
+    kc[mask] = 0x7F
+    vc[mask] = 0x7F
+    return kc.contiguous(), vc.contiguous()
+
+
+@pytest.mark.parametrize("src", [torch.bfloat16, torch.float16, torch.float32])
+@pytest.mark.parametrize("scales", [(1.0, 1.0), (0.37, 2.5), (1 / 64, 1 / 16)])
+def test_kv_append_fp8_bit_exact(src, scales):
+    import paged_kv_cache_405_b200 as pkv
+    ks, vs = scales
+    NB, Hkv, bs, D, T = 40, 4, 16, 128, 23
+    g = torch.Generator().manual_seed(7)
+    kn = (torch.randn(T, Hkv, D, generator=g) * 30).to(src)     # some values saturate
+    vn = (torch.randn(T, Hkv, D, generator=g) * 3).to(src)
+    kn[0, 0, :4] = torch.tensor([0.0, -0.0, 1e-7, -1e-7]).to(src)
+    slots = np.random.default_rng(1).choice(NB * bs, size=T, replace=False).astype(np.int64)
+    slots[::6] = -1
+    kc = np.zeros((NB, Hkv, bs, D), np.uint8)
+    vc = np.zeros((NB, Hkv, bs, D), np.uint8)
+    oracle.kv_append_fp8(kc, vc, kn, vn, ks, vs, slots)
+    kd = torch.zeros((NB, Hkv, bs, D), dtype=torch.uint8, device="cuda")
+    vd = torch.zeros_like(kd)
+    pkv.kv_append_fp8(kn.cuda(), vn.cuda(), kd, vd, torch.from_numpy(slots).cuda(), ks, vs)
+    assert pkv.device_error() == 0
+    assert np.array_equal(kd.cpu().numpy(), kc) and np.array_equal(vd.cpu().numpy(), vc)
+
+
+@pytest.mark.parametrize("qdt", ["bf16", "f16"])
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 2), (8, 1), (32, 2)])
+@pytest.mark.parametrize("bs,D", [(16, 128), (64, 128), (32, 64)])
+@pytest.mark.parametrize("P", [0, 32, 512])
+def test_decode_fp8_matches_oracle(qdt, Hq, Hkv, bs, D, P):
+    import paged_kv_cache_405_b200 as pkv
+    sh = synth.shrink(synth.CONFIGS["llama7b"], S=6, Hq=Hq, Hkv=Hkv, bs=bs, D=D, dtype=qdt,
+                      len_uniform=(1, 900), seed=Hq + bs + D + P)
+    b = synth.make_batch(sh)
+    ks, vs = 1 / 32, 1 / 8
+    kc, vc = fp8_pools(b, 5, ks, vs)
+    ref = oracle.paged_attention_kv(b.q, kc, vc, ks, vs, b.block_tables, b.lens, threads=oracle.max_threads())
+    out = torch.full_like(b.q, float("nan"), device="cuda")
+    pkv.paged_attention_decode_fp8(out, b.q.cuda(), kc.cuda(), vc.cuda(), torch.from_numpy(b.block_tables).cuda(),
+                                   torch.from_numpy(b.lens.astype(np.int32)).cuda(), ks, vs, partition_size=P)
+    assert pkv.device_error() == 0
+    assert max_err(out, ref) <= TOL[out.dtype]
+
+
+def test_fp8_decode_step_end_to_end():
+    """Quantized append of one new token per sequence, then attention over
+    L+1 tokens, against the oracle's quantizer and attention."""
+    import paged_kv_cache_405_b200 as pkv
+    sh = synth.shrink(synth.CONFIGS["llama3_gqa_bs16"], S=5, len_fixed=None, len_uniform=(1, 600))
+    b = synth.make_batch(sh)
+    ks, vs = 0.05, 0.2
+    kc, vc = fp8_pools(b, 9, ks, vs)
+    slots = np.array([int(b.block_tables[s, int(b.lens[s]) // sh.bs]) * sh.bs + int(b.lens[s]) % sh.bs
+                      if int(b.lens[s]) // sh.bs < b.max_blocks and b.block_tables[s, int(b.lens[s]) // sh.bs] >= 0
+                      else -1 for s in range(sh.S)], np.int64)
+    lens = b.lens + (slots >= 0)
+    kcn, vcn = kc.numpy().copy(), vc.numpy().copy()
+    oracle.kv_append_fp8(kcn, vcn, b.k_new, b.v_new, ks, vs, slots)
+    ref = oracle.paged_attention_kv(b.q, kcn, vcn, ks, vs, b.block_tables, lens, threads=oracle.max_threads())
+    kd, vd = kc.cuda(), vc.cuda()
+    pkv.kv_append_fp8(b.k_new.cuda(), b.v_new.cuda(), kd, vd, torch.from_numpy(slots).cuda(), ks, vs)
+    out = torch.empty_like(b.q, device="cuda")
+    pkv.paged_attention_decode_fp8(out, b.q.cuda(), kd, vd, torch.from_numpy(b.block_tables).cuda(),
+                                   torch.from_numpy(lens.astype(np.int32)).cuda(), ks, vs)
+    assert pkv.device_error() == 0
+    assert np.array_equal(kd.cpu().numpy(), kcn) and np.array_equal(vd.cpu().numpy(), vcn)
+    assert max_err(out, ref) <= TOL[out.dtype]
