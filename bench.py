@@ -55,7 +55,7 @@ def chunk_ws_bytes(lens, query_start, Hq: int, D: int, P: int) -> int:
 
 
 def attention_bytes(bt: np.ndarray, lens: np.ndarray, Hq: int, Hkv: int, D: int, bs: int, elt: int,
-                    P: int, shared=None, q_rows=None) -> dict:
+                    P: int, shared=None, q_rows=None, q_elt=None) -> dict:
     """Algorithmic bytes of one decode-attention call.
 
     K/V: every physical (block, kv head) tile covered by some context counts
@@ -76,7 +76,7 @@ def attention_bytes(bt: np.ndarray, lens: np.ndarray, Hq: int, Hkv: int, D: int,
     tok = int(best.sum())
     kv = 2 * Hkv * D * elt * tok
     logical = 2 * Hkv * D * elt * int(lens.sum())
-    qo = 2 * (S if q_rows is None else q_rows) * Hq * D * elt
+    qo = 2 * (S if q_rows is None else q_rows) * Hq * D * (elt if q_elt is None else q_elt)
     tables = 4 * int(nb.sum()) + 4 * S
     sh = np.zeros(S, dtype=np.int64) if shared is None else np.asarray(shared, dtype=np.int64)
     nparts = -(-sh // P) + -(-(lens - sh) // P)
@@ -104,7 +104,8 @@ class Workload:
         b = self.batch
         self.P = partition_size or shape.partition_size
         self.session = pkv.DecodeSession(b.k_pool, b.v_pool, shape.Hq, b.max_blocks, free_order=b.free_order,
-                                         partition_size=self.P, max_batch=shape.S)
+                                         partition_size=self.P, max_batch=shape.S,
+                                         kv_scales=(shape.kv_scale, shape.kv_scale) if shape.kv_fp8 else None)
         ss = self.session
         if shape.prefix:
             ss.add(-1, shape.prefix)                       # the prompt, stored once
@@ -123,7 +124,8 @@ class Workload:
         self.parents = list(range(shape.S))
         if shape.chunk:
             ss.reserve_chunk_workspace(shape.S * shape.chunk)
-        self.elt = b.k_pool.element_size()
+        self.elt = b.k_pool.element_size()     # pool element (1 byte for FP8 codes)
+        self.q_elt = b.q.element_size()
         self.eff_P = pkv.attention_partition_size(shape.S, shape.Hq, shape.Hkv, shape.D,
                                                   b.max_blocks * shape.bs, self.P)
         self.next_child = shape.S
@@ -177,8 +179,10 @@ class Workload:
         if plan.has_groups:   # per-sequence shared length of its group
             shared = np.repeat(plan.group_shared, np.diff(plan.group_first))
         a = attention_bytes(plan.block_tables, plan.lens, sh.Hq, sh.Hkv, sh.D, sh.bs, self.elt, self.eff_P,
-                            shared=shared)
-        total = a["total"] + append_bytes(len(plan.slot_mapping), sh.Hkv, sh.D, self.elt) + \
+                            shared=shared, q_elt=self.q_elt)
+        # append: new K/V read in the q/out type, written as pool elements
+        total = a["total"] + append_bytes(len(plan.slot_mapping), sh.Hkv, sh.D, self.elt) // 2 + \
+            append_bytes(len(plan.slot_mapping), sh.Hkv, sh.D, self.q_elt) // 2 + \
             copy_bytes(len(plan.cow_pairs), sh.Hkv, sh.bs, sh.D, self.elt)
         return total, a
 
@@ -279,7 +283,11 @@ def oracle_sample(batch, budget_s, threads):
             L = int(batch.lens[s])
             items = [(int(s), h) for h in range(Hq)]
             t0 = time.perf_counter()
-            oracle.paged_attention(q, k, v, batch.block_tables, batch.lens, items=items, threads=threads)
+            if batch.shape.kv_fp8:
+                oracle.paged_attention_kv(q, k, v, batch.shape.kv_scale, batch.shape.kv_scale, batch.block_tables,
+                                          batch.lens, items=items, threads=threads)
+            else:
+                oracle.paged_attention(q, k, v, batch.block_tables, batch.lens, items=items, threads=threads)
             secs += time.perf_counter() - t0
             bytes_done += 2 * L * batch.shape.D * elt * Hq
             seqs += 1
@@ -385,7 +393,10 @@ def run_ours(args, world, rank, local):
         else:
             if d.n_cow:
                 pkv.block_copy(ss.k_pool, ss.v_pool, d.cow_pairs)
-            pkv.kv_append(kn, vn, ss.k_pool, ss.v_pool, d.slot_mapping)
+            if ss.fp8:
+                pkv.kv_append_fp8(kn, vn, ss.k_pool, ss.v_pool, d.slot_mapping, *ss.kv_scales)
+            else:
+                pkv.kv_append(kn, vn, ss.k_pool, ss.v_pool, d.slot_mapping)
             if ev is not None:
                 ev[0].record(stream)
             ss.attend(d, q, out)
@@ -453,7 +464,8 @@ def run_ours(args, world, rank, local):
         line = {
             "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": round(ms_max / K, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": shape.dtype, "data": "synthetic (seeded N(0,1) K/V/q; pages' workload shapes)",
+            "vs_baseline": None, "dtype": shape.dtype + ("+e4m3-kv" if shape.kv_fp8 else ""),
+            "data": "synthetic (seeded N(0,1) K/V/q; pages' workload shapes)",
             "config": {"workload": args.config + ("" if not args.batch else "@batch%d" % args.batch),
                        "description": shape.description, "batch": shape.S,
                        "q_heads": shape.Hq, "kv_heads": shape.Hkv, "head_dim": shape.D, "block_size": shape.bs,

@@ -222,7 +222,7 @@ static cudaError_t launch_chunk(const pkv::AttnParams& p, const pkv::ChunkParams
 
 // FP8 pools: stages of E4M3 tiles converted to FP16 per warp.
 #ifndef PKV_FP8_STAGES
-#define PKV_FP8_STAGES 4
+#define PKV_FP8_STAGES 2
 #endif
 constexpr int kFp8Stages = PKV_FP8_STAGES;
 

@@ -70,8 +70,13 @@ class DevicePlan:
 class DecodeSession:
     def __init__(self, k_pool: torch.Tensor, v_pool: torch.Tensor, num_q_heads: int, max_blocks_per_seq: int,
                  free_order=None, partition_size: int = 0, max_batch: int = 0, share_prefixes: bool = True,
-                 min_group_size: int = 4):
+                 min_group_size: int = 4, kv_scales=None):
+        """Pools of a 16-bit/fp32 type, or uint8 FP8 E4M3 codes with kv_scales = (k_scale, v_scale)."""
         self.k_pool, self.v_pool = k_pool, v_pool
+        self.fp8 = k_pool.dtype == torch.uint8
+        if self.fp8 and kv_scales is None:
+            raise ValueError("FP8 pools need kv_scales")
+        self.kv_scales = kv_scales
         self.num_blocks, self.num_kv_heads, self.block_size, self.head_dim = k_pool.shape
         self.num_q_heads = num_q_heads
         self.max_blocks = max_blocks_per_seq
@@ -80,7 +85,7 @@ class DecodeSession:
         self.device = k_pool.device
         # Runs of sequences sharing leading blocks go through the shared-prefix
         # pass (16-bit pools only: it runs on tensor cores).
-        self.share_prefixes = share_prefixes and k_pool.dtype != torch.float32
+        self.share_prefixes = share_prefixes and k_pool.dtype not in (torch.float32, torch.uint8)
         self.min_group_size = min_group_size
         n = max(max_batch, 1)
         max_len = max_blocks_per_seq * self.block_size
@@ -195,12 +200,19 @@ class DecodeSession:
         """block_copy (if any pair) -> kv_append -> paged_attention_decode."""
         if d.n_cow:
             B.block_copy(self.k_pool, self.v_pool, d.cow_pairs, stream=stream)
-        B.kv_append(k_new, v_new, self.k_pool, self.v_pool, d.slot_mapping, stream=stream)
+        if self.fp8:
+            B.kv_append_fp8(k_new, v_new, self.k_pool, self.v_pool, d.slot_mapping, *self.kv_scales, stream=stream)
+        else:
+            B.kv_append(k_new, v_new, self.k_pool, self.v_pool, d.slot_mapping, stream=stream)
         return self.attend(d, q, out, stream=stream)
 
     def attend(self, d: DevicePlan, q: torch.Tensor, out: torch.Tensor, stream=None):
         """The step's attention: the shared-prefix call when the plan found groups."""
-        if d.group_shared is not None:
+        if self.fp8:
+            B.paged_attention_decode_fp8(out, q, self.k_pool, self.v_pool, d.block_tables, d.lens, *self.kv_scales,
+                                         partition_size=self.partition_size, workspace=self.workspace,
+                                         stream=stream)
+        elif d.group_shared is not None:
             B.paged_attention_decode_shared(out, q, self.k_pool, self.v_pool, d.block_tables, d.lens,
                                             d.group_first, d.group_shared, d.max_group_size, d.max_shared_len,
                                             partition_size=self.partition_size, workspace=self.workspace,

@@ -52,6 +52,8 @@ class Shape:
     beams: int = 0                      # beams forked per sequence
     pinned_seq0: Optional[list] = None  # explicit physical blocks of seq 0
     chunk: int = 0                      # new tokens per sequence per step (causal chunk); 0 = decode
+    kv_fp8: bool = False                # pools of FP8 E4M3 codes (values = code x kv_scale)
+    kv_scale: float = 1.0 / 32          # k_scale = v_scale for FP8 pools
     description: str = ""
 
 
@@ -84,6 +86,14 @@ CONFIGS = {
     "spec_verify": Shape("spec_verify", S=64, Hq=32, Hkv=8, D=128, bs=16, dtype="bf16", seed=7,
                          len_uniform=(1024, 8192), chunk=4,
                          description="speculative verification: batch 64 x 4 draft tokens, 32q/8kv x 128, bf16, bs 16, ctx U[1024,8192]"),
+    # FP8 E4M3 pools (extensions): the Llama-2-7B and Llama-3-8B decode
+    # workloads with K/V stored as 1-byte codes.
+    "llama7b_fp8": Shape("llama7b_fp8", S=64, Hq=32, Hkv=32, D=128, bs=16, dtype="bf16", seed=1,
+                         len_uniform=(128, 2048), kv_fp8=True,
+                         description="Llama-2-7B-shaped decode over FP8 E4M3 pools: batch 64, MHA 32x128, bf16 q/out, bs 16"),
+    "llama3_gqa_fp8": Shape("llama3_gqa_fp8", S=128, Hq=32, Hkv=8, D=128, bs=16, dtype="bf16", seed=5,
+                            len_fixed=8192, pool_factor=1.0, kv_fp8=True,
+                            description="Llama-3-8B-shaped GQA decode over FP8 E4M3 pools: batch 128, 32q/8kv x 128, ctx 8192"),
     # Long context + beams: 8 x 100k tokens, 64 q / 8 kv heads, bs 64,
     # split over 512-token partitions; 4 beams fork each sequence.
     "longctx_beam": Shape("longctx_beam", S=8, Hq=64, Hkv=8, D=128, bs=64, dtype="bf16", seed=6,
@@ -147,6 +157,17 @@ def randn(shape, gen: torch.Generator, dtype: torch.dtype, device, chunk: int = 
     return out.view(*shape)
 
 
+def fp8_codes(shape, gen: torch.Generator, scale: float, device, chunk: int = 1 << 27) -> torch.Tensor:
+    """uint8 E4M3 codes of N(0,1) samples divided by ``scale`` (torch cast)."""
+    n = int(np.prod(shape))
+    out = torch.empty(n, dtype=torch.uint8, device=device)
+    for s in range(0, n, chunk):
+        e = min(n, s + chunk)
+        x = torch.randn(e - s, generator=gen, dtype=torch.float32, device=device) / scale
+        out[s:e] = x.to(torch.float8_e4m3fn).view(torch.uint8)
+    return out.view(*shape)
+
+
 def make_batch(shape: Shape, device="cpu", seed: Optional[int] = None,
                value_scale: float = 1.0, fill_unused=None) -> Batch:
     """Build the batch for ``shape``.
@@ -198,13 +219,17 @@ def make_batch(shape: Shape, device="cpu", seed: Optional[int] = None,
     gen.manual_seed(seed)
     dt = DTYPES[shape.dtype]
     pshape = (NB, shape.Hkv, bs, shape.D)
-    k_pool = randn(pshape, gen, dt, device)
-    v_pool = randn(pshape, gen, dt, device)
+    if shape.kv_fp8:   # codes of N(0,1) values / kv_scale, cast by torch's float8_e4m3fn
+        k_pool = fp8_codes(pshape, gen, shape.kv_scale, device)
+        v_pool = fp8_codes(pshape, gen, shape.kv_scale, device)
+    else:
+        k_pool = randn(pshape, gen, dt, device)
+        v_pool = randn(pshape, gen, dt, device)
     q = randn((shape.S, shape.Hq, shape.D), gen, dt, device)
     k_new = randn((shape.S, shape.Hkv, shape.D), gen, dt, device)
     v_new = randn((shape.S, shape.Hkv, shape.D), gen, dt, device)
     if value_scale != 1.0:
-        for t in (k_pool, v_pool, q, k_new, v_new):
+        for t in ((q, k_new, v_new) if shape.kv_fp8 else (k_pool, v_pool, q, k_new, v_new)):
             t.copy_((t.float() * value_scale).to(dt))
     if fill_unused is not None:
         covered = torch.zeros((NB, bs), dtype=torch.bool)

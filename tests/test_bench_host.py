@@ -20,6 +20,7 @@ import synth
     ("llama3_gqa_bs32", dict(S=3, Hq=4, Hkv=1, D=64, len_fixed=300)),
     ("longctx_beam", dict(S=2, Hq=2, Hkv=1, D=64, len_fixed=1000)),
     ("spec_verify", dict(S=3, Hq=4, Hkv=1, D=64, len_uniform=(20, 300))),
+    ("llama7b_fp8", dict(S=4, Hq=2, Hkv=2, D=64)),
 ])
 def test_workload_steps_on_cpu(cfg, over):
     sh = synth.shrink(synth.CONFIGS[cfg], **over)

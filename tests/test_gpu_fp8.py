@@ -94,3 +94,25 @@ def test_fp8_decode_step_end_to_end():
     assert pkv.device_error() == 0
     assert np.array_equal(kd.cpu().numpy(), kcn) and np.array_equal(vd.cpu().numpy(), vcn)
     assert max_err(out, ref) <= TOL[out.dtype]
+
+
+def test_session_fp8_step_matches_oracle():
+    import paged_kv_cache_405_b200 as m
+    sh = synth.shrink(synth.CONFIGS["llama7b_fp8"], S=5, Hq=8, Hkv=8, len_uniform=(1, 500))
+    b = synth.make_batch(sh)
+    dev = torch.device("cuda")
+    k, v = b.k_pool.to(dev), b.v_pool.to(dev)
+    ss = m.DecodeSession(k, v, sh.Hq, b.max_blocks, free_order=b.free_order, max_batch=sh.S,
+                         kv_scales=(sh.kv_scale, sh.kv_scale))
+    for s in range(sh.S):
+        ss.add(s, int(b.lens[s]))
+    plan = ss.plan(list(range(sh.S)))
+    out = torch.empty_like(b.q, device=dev)
+    ss.launch(ss.to_device(plan), b.q.to(dev), b.k_new.to(dev), b.v_new.to(dev), out)
+    kc, vc = b.k_pool.numpy().copy(), b.v_pool.numpy().copy()
+    oracle.kv_append_fp8(kc, vc, b.k_new, b.v_new, sh.kv_scale, sh.kv_scale, plan.slot_mapping)
+    ref = oracle.paged_attention_kv(b.q, kc, vc, sh.kv_scale, sh.kv_scale, plan.block_tables, plan.lens,
+                                    threads=oracle.max_threads())
+    assert m.device_error() == 0
+    assert np.array_equal(k.cpu().numpy(), kc) and np.array_equal(v.cpu().numpy(), vc)
+    assert max_err(out, ref) <= TOL[out.dtype]
