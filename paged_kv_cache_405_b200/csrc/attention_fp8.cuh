@@ -1,0 +1,254 @@
+// Grouped-query paged decode over FP8 E4M3 pools on the tensor cores.
+//
+// Same unit of work as paged_attn_mma_kernel: one warp per (sequence, kv
+// head, partition), the G query heads of the group being the 16 MMA rows
+// (padded with zero rows), tokens found through the block table
+// (openeuler.csdn.net PagedAttention explainer 4.2; aiknowledge.cn "2.2
+// PagedAttention 与 KV Cache 分页管理" 2.2.3-2.2.4).  The K and V tiles stay in
+// shared memory as E4M3 codes; each lane widens only the codes its own MMA
+// fragments need, straight into registers.  Every E4M3 value is an FP16
+// value, so the widening is exact and the MMA runs in FP16 with fp32
+// accumulation; the per-pool scales fold into the softmax scale (K) and the
+// final normalisation (V).
+//
+// Fragment layouts (mma.m16n8k16; lane = 4 * gid + tig).  A dot product may
+// take its terms in any order, so each product's contraction index is
+// permuted to make every lane's codes contiguous in the tile:
+//  * S = Q K^T.  K-step kk, lane tig: the logical k indices {2tig, 2tig+1,
+//    2tig+8, 2tig+9} are head-dim elements tig*D/4 + 4kk + {0, 1, 2, 3}.  A
+//    lane reads D/4 consecutive codes of token nt*8 + gid (n-tile nt), and
+//    the Q fragments follow the same map.
+//  * O += P V.  The contraction runs over the tokens in the order of the S
+//    columns (lane tig holds tokens 2tig, 2tig+1, 8+2tig, 9+2tig).  Output
+//    n-tile j, column n is head-dim element n*D/8 + j, so a lane reads D/8
+//    consecutive codes of each of its four tokens and pairs the codes of two
+//    tokens with one byte permute per four columns.
+//
+// Tiles arrive by 2-D tensor TMA as 16 tokens x D codes.  D = 128: 128-byte
+// rows with the 128-byte swizzle (16-byte chunk c of row r lands at chunk
+// c ^ (r & 7)), under which the K reads (two chunks per lane: 2tig, 2tig+1)
+// and the V reads (one chunk per lane: gid) of each quarter warp hit eight
+// different chunk positions.  D = 64: 64-byte rows, no swizzle.
+#pragma once
+#include "attention_mma.cuh"
+
+namespace pkv {
+
+template <int D, int WARPS, int STAGES>
+struct Fp8Cfg {
+    static constexpr int kTileBytes = kTileTok * D;  // one K (or V) tile of codes
+    static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kWarpBytes = STAGES * kStageBytes;
+    static constexpr int kDataBytes = WARPS * kWarpBytes;
+    static constexpr int kSmemBytes = 1024 + kDataBytes + WARPS * STAGES * 8;  // + alignment slack
+    static constexpr bool kSwizzle = D == 128;
+    static_assert(D == 64 || D == 128, "head_dim must be 64 or 128");
+    static_assert(kTileBytes % 1024 == 0, "swizzled tiles must start on 1024-byte boundaries");
+};
+
+// Byte offset of the 16-byte chunk c of tile row r.
+template <int D>
+__device__ __forceinline__ int fp8_chunk(int r, int c) {
+    if constexpr (D == 128) return r * 128 + ((c ^ (r & 7)) << 4);
+    else return r * D + (c << 4);
+}
+
+template <int D, int WARPS, int STAGES, typename To>
+__global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_fp8_kernel(const AttnParams p,
+                                                                       const __grid_constant__ CUtensorMap tmK,
+                                                                       const __grid_constant__ CUtensorMap tmV) {
+    using C = Fp8Cfg<D, WARPS, STAGES>;
+    constexpr int KSTEPS = D / 16;
+    constexpr int NT_O = D / 8;
+    constexpr int KW = KSTEPS;  // 32-bit words of K codes per lane and n-tile (D/4 codes)
+    constexpr int VW = NT_O / 4;  // 32-bit words of V codes per lane and token (D/8 codes)
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int g = blockIdx.x * WARPS + warp;  // kv head
+    const int part = blockIdx.y;
+    const int s = blockIdx.z;
+    if (g >= p.Hkv) return;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int G = p.G;
+    const int h0 = g * G;
+
+    const Unit u = resolve_unit(p, s, part, part == 0 && g == 0 && lane == 0);
+    if (u.t_begin >= u.L) {
+        if (part == 0 && u.L == 0) {  // empty context: zeros for the group's heads
+            To* o = reinterpret_cast<To*>(p.out) + ((int64_t)s * p.Hq + h0) * D;
+            for (int i = lane; i < G * D; i += 32) o[i] = To(0.f);
+        }
+        return;
+    }
+    uint32_t bar0;
+    uint8_t* ring = ring_setup<C::kWarpBytes, C::kDataBytes, STAGES>(smem_raw, warp, lane, bar0, &tmK, &tmV);
+    const uint32_t ring_s = smem_u32(ring);
+
+    // Q rows gid and gid + 8 as A fragments under the permuted contraction.
+    MmaAcc<__half, D> acc;
+    {
+        const To* qb = reinterpret_cast<const To*>(p.q) + ((int64_t)s * p.Hq + h0) * D;
+        const To* row_lo = gid < G ? qb + gid * D + tig * (D / 4) : nullptr;
+        const To* row_hi = gid + 8 < G ? qb + (gid + 8) * D + tig * (D / 4) : nullptr;
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+            acc.qa[kk][0] = row_lo ? MmaAcc<__half, D>::pair(row_lo + 4 * kk) : 0u;
+            acc.qa[kk][1] = row_hi ? MmaAcc<__half, D>::pair(row_hi + 4 * kk) : 0u;
+            acc.qa[kk][2] = row_lo ? MmaAcc<__half, D>::pair(row_lo + 4 * kk + 2) : 0u;
+            acc.qa[kk][3] = row_hi ? MmaAcc<__half, D>::pair(row_hi + 4 * kk + 2) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < NT_O; ++j) acc.o[j][0] = acc.o[j][1] = acc.o[j][2] = acc.o[j][3] = 0.f;
+        acc.m_lo = acc.m_hi = -INFINITY;
+        acc.l_lo = acc.l_hi = 0.f;
+    }
+
+    const int t_begin = u.t_begin, t_end = u.t_end;
+    const int ntiles = (t_end - t_begin + kTileTok - 1) / kTileTok;
+    const int32_t* bt_row = p.block_tables + (int64_t)s * p.maxB;
+    const int jb0 = t_begin / p.bs;
+    BlockWindow win;
+    win.init(bt_row, jb0, (t_end - 1) / p.bs - jb0 + 1, lane);
+
+    auto issue = [&](int i) {
+        const int t0 = t_begin + i * kTileTok;
+        const int blk = win.get(t0 / p.bs - jb0, lane, p.NB);
+        if (lane == 0) {
+            const int row = (blk * p.Hkv + g) * p.bs + (t0 % p.bs);
+            const int st = i % STAGES;
+            const uint32_t bar = bar0 + 8 * st;
+            const uint32_t dst = ring_s + st * C::kStageBytes;
+            fence_proxy_async();
+            mbar_arrive_expect_tx(bar, C::kStageBytes);
+            tma_load_2d(dst, &tmK, 0, row, bar);
+            tma_load_2d(dst + C::kTileBytes, &tmV, 0, row, bar);
+        }
+    };
+    const int npre = ntiles < STAGES ? ntiles : STAGES;
+    for (int i = 0; i < npre; ++i) issue(i);
+
+    // This lane's tokens for the P V contraction, in S-column order.
+    const int vtok[4] = {2 * tig, 2 * tig + 1, 8 + 2 * tig, 9 + 2 * tig};
+
+    for (int i = 0; i < ntiles; ++i) {
+        const int st = i % STAGES;
+        if (!ring_wait<STAGES>(bar0, i, ntiles)) return;
+        const int valid = min(kTileTok, t_end - (t_begin + i * kTileTok));
+        const uint8_t* kt = ring + st * C::kStageBytes;
+        const uint8_t* vt = kt + C::kTileBytes;
+
+        // Codes of this lane's fragments, then the stage goes back to TMA.
+        uint32_t kw[2][KW];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int c = 0; c < KW / 4; ++c) {
+                const uint4 w = *reinterpret_cast<const uint4*>(kt + fp8_chunk<D>(nt * 8 + gid, tig * (KW / 4) + c));
+                kw[nt][4 * c] = w.x;
+                kw[nt][4 * c + 1] = w.y;
+                kw[nt][4 * c + 2] = w.z;
+                kw[nt][4 * c + 3] = w.w;
+            }
+        }
+        uint32_t vw[4][VW];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            if constexpr (VW == 4) {
+                const uint4 w = *reinterpret_cast<const uint4*>(vt + fp8_chunk<D>(vtok[t], gid));
+                vw[t][0] = w.x;
+                vw[t][1] = w.y;
+                vw[t][2] = w.z;
+                vw[t][3] = w.w;
+            } else {
+                const uint2 w = *reinterpret_cast<const uint2*>(vt + vtok[t] * D + gid * 8);
+                vw[t][0] = w.x;
+                vw[t][1] = w.y;
+            }
+            // Rows past the context may hold any code (NaN included): a zero
+            // weight times NaN would poison the sum, so drop them here.
+            if (vtok[t] >= valid) {
+#pragma unroll
+                for (int w = 0; w < VW; ++w) vw[t][w] = 0u;
+            }
+        }
+        __syncwarp();
+        if (i + STAGES < ntiles) issue(i + STAGES);
+
+        // S = Q K^T
+        float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                const uint32_t b0 = e4m3x2_to_f16x2((uint16_t)(kw[nt][kk] & 0xffffu));
+                const uint32_t b1 = e4m3x2_to_f16x2((uint16_t)(kw[nt][kk] >> 16));
+                mma_16816<__half>(sacc[nt], acc.qa[kk], b0, b1);
+            }
+        }
+        uint32_t pa[4];
+        mma_softmax(acc, sacc, tig, valid, valid, p.scale_log2, pa);
+
+        // O += P V
+#pragma unroll
+        for (int w = 0; w < VW; ++w) {
+            // Bytes [x0, y0, x1, y1] and [x2, y2, x3, y3] of tokens x, y.
+            const uint32_t lo0 = __byte_perm(vw[0][w], vw[1][w], 0x5140);
+            const uint32_t hi0 = __byte_perm(vw[0][w], vw[1][w], 0x7362);
+            const uint32_t lo1 = __byte_perm(vw[2][w], vw[3][w], 0x5140);
+            const uint32_t hi1 = __byte_perm(vw[2][w], vw[3][w], 0x7362);
+            mma_16816<__half>(acc.o[4 * w], pa, e4m3x2_to_f16x2((uint16_t)(lo0 & 0xffffu)),
+                              e4m3x2_to_f16x2((uint16_t)(lo1 & 0xffffu)));
+            mma_16816<__half>(acc.o[4 * w + 1], pa, e4m3x2_to_f16x2((uint16_t)(lo0 >> 16)),
+                              e4m3x2_to_f16x2((uint16_t)(lo1 >> 16)));
+            mma_16816<__half>(acc.o[4 * w + 2], pa, e4m3x2_to_f16x2((uint16_t)(hi0 & 0xffffu)),
+                              e4m3x2_to_f16x2((uint16_t)(hi1 & 0xffffu)));
+            mma_16816<__half>(acc.o[4 * w + 3], pa, e4m3x2_to_f16x2((uint16_t)(hi0 >> 16)),
+                              e4m3x2_to_f16x2((uint16_t)(hi1 >> 16)));
+        }
+    }
+#pragma unroll
+    for (int off = 1; off < 4; off <<= 1) {
+        acc.l_lo += __shfl_xor_sync(0xffffffffu, acc.l_lo, off);
+        acc.l_hi += __shfl_xor_sync(0xffffffffu, acc.l_hi, off);
+    }
+
+    // Lane (gid, tig) holds, for row gid (+8), the columns (2tig + e) * D/8 + j
+    // (e = 0, 1; j = 0 .. D/8-1): two runs of D/8 consecutive elements.
+#pragma unroll
+    for (int hi = 0; hi < 2; ++hi) {
+        const int r = gid + 8 * hi;
+        if (r >= G) continue;
+        const int64_t row = (int64_t)s * p.Hq + h0 + r;
+        const int e0 = hi ? 2 : 0;
+        const float l = hi ? acc.l_hi : acc.l_lo;
+        if (u.direct) {
+            const float inv = p.v_scale / l;
+            To* out = reinterpret_cast<To*>(p.out) + row * D;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                uint32_t h[NT_O / 2];
+#pragma unroll
+                for (int j = 0; j < NT_O; j += 2)
+                    h[j / 2] = Elt<To>::pack2(acc.o[j][e0 + e] * inv, acc.o[j + 1][e0 + e] * inv);
+                uint4* dst = reinterpret_cast<uint4*>(out + (2 * tig + e) * NT_O);
+#pragma unroll
+                for (int v = 0; v < NT_O / 8; ++v) dst[v] = make_uint4(h[4 * v], h[4 * v + 1], h[4 * v + 2], h[4 * v + 3]);
+            }
+        } else {
+            const int64_t idx = row * p.maxP + u.slot;
+            float* o_row = p.ws_o + idx * D;
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float4* dst = reinterpret_cast<float4*>(o_row + (2 * tig + e) * NT_O);
+#pragma unroll
+                for (int v = 0; v < NT_O / 4; ++v)
+                    dst[v] = make_float4(acc.o[4 * v][e0 + e] * p.v_scale, acc.o[4 * v + 1][e0 + e] * p.v_scale,
+                                         acc.o[4 * v + 2][e0 + e] * p.v_scale, acc.o[4 * v + 3][e0 + e] * p.v_scale);
+            }
+            if (tig == 0) *reinterpret_cast<float2*>(p.ws_ml + idx * 2) = make_float2(hi ? acc.m_hi : acc.m_lo, l);
+        }
+    }
+}
+
+}  // namespace pkv

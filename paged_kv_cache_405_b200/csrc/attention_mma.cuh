@@ -38,17 +38,14 @@
 
 namespace pkv {
 
-// Shared memory of one warp: [FP8 only: K and V tiles converted to 16-bit,
-// swizzled] then STAGES stages of (K tile, V tile) as loaded by TMA (16-bit
-// swizzled tiles, or FP8 codes row-major).
-template <typename T, int D, int WARPS, int STAGES, bool FP8 = false>
+// Shared memory of one warp: STAGES stages of (K tile, V tile), 16-bit
+// swizzled tiles as loaded by TMA.
+template <typename T, int D, int WARPS, int STAGES>
 struct MmaCfg {
-    static constexpr int kHalfTile = kTileTok * 128;                 // 16 rows x 64 16-bit elements (bytes)
-    static constexpr int kTileBytes = kTileTok * D * 2;              // one 16-bit K (or V) tile
-    static constexpr int kStageTile = FP8 ? kTileTok * D : kTileBytes;  // one tile as loaded
-    static constexpr int kStageBytes = 2 * kStageTile;
-    static constexpr int kConvBytes = FP8 ? 2 * kTileBytes : 0;
-    static constexpr int kWarpBytes = (kConvBytes + STAGES * kStageBytes + 1023) / 1024 * 1024;
+    static constexpr int kHalfTile = kTileTok * 128;     // 16 rows x 64 16-bit elements (bytes)
+    static constexpr int kTileBytes = kTileTok * D * 2;  // one K (or V) tile
+    static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kWarpBytes = STAGES * kStageBytes;
     static constexpr int kDataBytes = WARPS * kWarpBytes;
     static constexpr int kSmemBytes = 1024 + kDataBytes + WARPS * STAGES * 8;  // + alignment slack
     static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
@@ -95,29 +92,95 @@ struct MmaAcc {
     }
 };
 
+// Online-softmax step for one 16 x 16 score tile (log2 domain).  sacc holds
+// the raw scores, element e of n-tile nt being token nt*8 + 2*tig + (e & 1) of
+// row gid (e < 2) or gid + 8 (e >= 2); row gid sees the first seen_lo tokens,
+// row gid + 8 the first seen_hi.  Updates the running max and sum, rescales
+// the output accumulators and returns the probabilities packed as the A
+// fragments of the P V product.
+template <typename T, int D>
+__device__ __forceinline__ void mma_softmax(MmaAcc<T, D>& acc, float (&sacc)[2][4], int tig, int seen_lo,
+                                            int seen_hi, float scale_log2, uint32_t (&pa)[4]) {
+    constexpr int NT_O = D / 8;
+    float mx_lo = -INFINITY, mx_hi = -INFINITY;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int tok = nt * 8 + 2 * tig + (e & 1);
+            const float x = tok < (e < 2 ? seen_lo : seen_hi) ? sacc[nt][e] * scale_log2 : -INFINITY;
+            sacc[nt][e] = x;
+            if (e < 2) mx_lo = fmaxf(mx_lo, x);
+            else mx_hi = fmaxf(mx_hi, x);
+        }
+    }
+#pragma unroll
+    for (int off = 1; off < 4; off <<= 1) {
+        mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, off));
+        mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, off));
+    }
+    const float mn_lo = fmaxf(acc.m_lo, mx_lo), mn_hi = fmaxf(acc.m_hi, mx_hi);
+    // A row that has seen no token yet keeps m = -inf; exponentiate against 0
+    // then, so that no -inf - -inf appears.
+    const float b_lo = mn_lo == -INFINITY ? 0.f : mn_lo, b_hi = mn_hi == -INFINITY ? 0.f : mn_hi;
+    const float a_lo = ex2(acc.m_lo - b_lo), a_hi = ex2(acc.m_hi - b_hi);
+    acc.m_lo = mn_lo;
+    acc.m_hi = mn_hi;
+    float ps_lo = 0.f, ps_hi = 0.f;
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float pr = ex2(sacc[nt][e] - (e < 2 ? b_lo : b_hi));
+            sacc[nt][e] = pr;
+            if (e < 2) ps_lo += pr;
+            else ps_hi += pr;
+        }
+    }
+    acc.l_lo = acc.l_lo * a_lo + ps_lo;
+    acc.l_hi = acc.l_hi * a_hi + ps_hi;
+    // Once the running maxima settle, every factor is exactly 1 and the
+    // multiplications change nothing: skip them when that holds warp-wide.
+    if (!__all_sync(0xffffffffu, a_lo == 1.f && a_hi == 1.f)) {
+#pragma unroll
+        for (int j = 0; j < NT_O; ++j) {
+            acc.o[j][0] *= a_lo;
+            acc.o[j][1] *= a_lo;
+            acc.o[j][2] *= a_hi;
+            acc.o[j][3] *= a_hi;
+        }
+    }
+    pa[0] = Elt<T>::pack2(sacc[0][0], sacc[0][1]);
+    pa[1] = Elt<T>::pack2(sacc[0][2], sacc[0][3]);
+    pa[2] = Elt<T>::pack2(sacc[1][0], sacc[1][1]);
+    pa[3] = Elt<T>::pack2(sacc[1][2], sacc[1][3]);
+}
+
+// Per-lane wait for stage st of tile i; on a timeout anywhere in the warp,
+// drain the copies still in flight (tiles i+1 .. i+STAGES-1) and report false.
+template <int STAGES>
+__device__ __forceinline__ bool ring_wait(uint32_t bar0, int i, int ntiles) {
+    const bool ok = mbar_wait(bar0 + 8 * (i % STAGES), (i / STAGES) & 1);
+    if (__all_sync(0xffffffffu, ok)) return true;
+    for (int k = i + 1; k < ntiles && k < i + STAGES; ++k) mbar_wait(bar0 + 8 * (k % STAGES), (k / STAGES) & 1);
+    return false;
+}
+
 // Stream tokens [t_begin, t_end) of kv head g (block ids from bt_row) through
 // this warp's ring and accumulate into acc.  Row gid sees only tokens below
 // lim_lo, row gid+8 only tokens below lim_hi (causal chunks; pass t_end when
 // every row sees the whole range).  Returns false if a wait on a copy timed
 // out (the unit is then abandoned after draining its copies).
-//
-// FP8 mode: TMA brings tiles of E4M3 codes (row-major, one box per tile);
-// after a stage arrives the warp converts its K and V tiles to 16-bit (exact:
-// every E4M3 value is an FP16 value) into the swizzled layout the tensor-core
-// code reads, and the stage is refilled at once.
-template <typename T, int D, int WARPS, int STAGES, bool FP8 = false>
+template <typename T, int D, int WARPS, int STAGES>
 __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMap* tmK, const CUtensorMap* tmV,
                                            uint8_t* ring, uint32_t bar0, const int32_t* bt_row, int t_begin,
                                            int t_end, int g, int lane, MmaAcc<T, D>& acc, int lim_lo,
                                            int lim_hi) {
-    using C = MmaCfg<T, D, WARPS, STAGES, FP8>;
+    using C = MmaCfg<T, D, WARPS, STAGES>;
     constexpr int KSTEPS = D / 16;
-    constexpr int NT_O = D / 8;
     const int tig = lane & 3;
     const int ntiles = (t_end - t_begin + kTileTok - 1) / kTileTok;
-    const uint32_t conv_s = smem_u32(ring);
-    uint8_t* stages = ring + C::kConvBytes;
-    const uint32_t ring_s = smem_u32(stages);
+    const uint32_t ring_s = smem_u32(ring);
 
     const int jb0 = t_begin / p.bs;
     BlockWindow win;
@@ -133,15 +196,10 @@ __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMa
             const uint32_t dst = ring_s + st * C::kStageBytes;
             fence_proxy_async();
             mbar_arrive_expect_tx(bar, C::kStageBytes);
-            if constexpr (FP8) {
-                tma_load_2d(dst, tmK, 0, row, bar);
-                tma_load_2d(dst + C::kStageTile, tmV, 0, row, bar);
-            } else {
 #pragma unroll
-                for (int hx = 0; hx < D / 64; ++hx) {
-                    tma_load_2d(dst + hx * C::kHalfTile, tmK, hx * 64, row, bar);
-                    tma_load_2d(dst + C::kTileBytes + hx * C::kHalfTile, tmV, hx * 64, row, bar);
-                }
+            for (int hx = 0; hx < D / 64; ++hx) {
+                tma_load_2d(dst + hx * C::kHalfTile, tmK, hx * 64, row, bar);
+                tma_load_2d(dst + C::kTileBytes + hx * C::kHalfTile, tmV, hx * 64, row, bar);
             }
         }
     };
@@ -158,48 +216,13 @@ __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMa
 
     for (int i = 0; i < ntiles; ++i) {
         const int st = i % STAGES;
-        const bool ok = mbar_wait(bar0 + 8 * st, (i / STAGES) & 1);
-        if (!__all_sync(0xffffffffu, ok)) {
-            for (int k = i + 1; k < ntiles && k < i + STAGES; ++k) mbar_wait(bar0 + 8 * (k % STAGES), (k / STAGES) & 1);
-            return false;
-        }
+        if (!ring_wait<STAGES>(bar0, i, ntiles)) return false;
         const int valid = min(kTileTok, t_end - (t_begin + i * kTileTok));
         const int seen_lo = min(valid, lim_lo - (t_begin + i * kTileTok));  // tokens row gid sees
         const int seen_hi = min(valid, lim_hi - (t_begin + i * kTileTok));  // ... and row gid+8
-        uint32_t Ks = ring_s + st * C::kStageBytes;
-        uint8_t* vtile = stages + st * C::kStageBytes + C::kTileBytes;
-        if constexpr (FP8) {
-            // E4M3 codes (row-major, D bytes per token) -> 16-bit swizzled tiles.
-            const uint8_t* src = stages + st * C::kStageBytes;
-#pragma unroll
-            for (int kv = 0; kv < 2; ++kv) {
-#pragma unroll
-                for (int k = 0; k < D / 32; ++k) {
-                    const int q16 = k * 32 + lane;       // 16-code piece of the tile
-                    const int r = q16 / (D / 16), c16 = q16 % (D / 16);
-                    const uint4 w = *reinterpret_cast<const uint4*>(src + kv * C::kStageTile + r * D + c16 * 16);
-                    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-                    uint32_t h[8];
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        h[2 * j] = e4m3x2_to_f16x2((uint16_t)(ww[j] & 0xffffu));
-                        h[2 * j + 1] = e4m3x2_to_f16x2((uint16_t)(ww[j] >> 16));
-                    }
-#pragma unroll
-                    for (int hc = 0; hc < 2; ++hc) {   // two 8-element (16-byte) chunks
-                        const int ch = c16 * 2 + hc;
-                        uint8_t* dst = ring + kv * C::kTileBytes + (ch >> 3) * C::kHalfTile + r * 128 +
-                                       (((ch & 7) ^ (r & 7)) << 4);
-                        *reinterpret_cast<uint4*>(dst) = make_uint4(h[4 * hc], h[4 * hc + 1], h[4 * hc + 2], h[4 * hc + 3]);
-                    }
-                }
-            }
-            __syncwarp();
-            if (i + STAGES < ntiles) issue(i + STAGES);  // the stage is free again
-            Ks = conv_s;
-            vtile = ring + C::kTileBytes;
-        }
+        const uint32_t Ks = ring_s + st * C::kStageBytes;
         const uint32_t Vs = Ks + C::kTileBytes;
+        uint8_t* vtile = ring + st * C::kStageBytes + C::kTileBytes;
 
         // S = Q K^T  (16 rows x 16 tokens as two n-tiles of 8 tokens)
         float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
@@ -212,66 +235,16 @@ __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMa
             mma_16816<T>(sacc[0], acc.qa[kk], b0, b1);
             mma_16816<T>(sacc[1], acc.qa[kk], b2, b3);
         }
-
-        // Online softmax.  Element e of n-tile nt is token nt*8 + 2*tig + (e&1).
-        float mx_lo = -INFINITY, mx_hi = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int tok = nt * 8 + 2 * tig + (e & 1);
-                const float x = tok < (e < 2 ? seen_lo : seen_hi) ? sacc[nt][e] * p.scale_log2 : -INFINITY;
-                sacc[nt][e] = x;
-                if (e < 2) mx_lo = fmaxf(mx_lo, x);
-                else mx_hi = fmaxf(mx_hi, x);
-            }
-        }
-#pragma unroll
-        for (int off = 1; off < 4; off <<= 1) {
-            mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, off));
-            mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, off));
-        }
-        const float mn_lo = fmaxf(acc.m_lo, mx_lo), mn_hi = fmaxf(acc.m_hi, mx_hi);
-        // A row that has seen no token yet keeps m = -inf; exponentiate
-        // against 0 then, so that no -inf - -inf appears.
-        const float b_lo = mn_lo == -INFINITY ? 0.f : mn_lo, b_hi = mn_hi == -INFINITY ? 0.f : mn_hi;
-        const float a_lo = ex2(acc.m_lo - b_lo), a_hi = ex2(acc.m_hi - b_hi);
-        acc.m_lo = mn_lo;
-        acc.m_hi = mn_hi;
-        float ps_lo = 0.f, ps_hi = 0.f;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float pr = ex2(sacc[nt][e] - (e < 2 ? b_lo : b_hi));
-                sacc[nt][e] = pr;
-                if (e < 2) ps_lo += pr;
-                else ps_hi += pr;
-            }
-        }
-        acc.l_lo = acc.l_lo * a_lo + ps_lo;
-        acc.l_hi = acc.l_hi * a_hi + ps_hi;
-#pragma unroll
-        for (int j = 0; j < NT_O; ++j) {
-            acc.o[j][0] *= a_lo;
-            acc.o[j][1] *= a_lo;
-            acc.o[j][2] *= a_hi;
-            acc.o[j][3] *= a_hi;
-        }
         uint32_t pa[4];
-        pa[0] = Elt<T>::pack2(sacc[0][0], sacc[0][1]);
-        pa[1] = Elt<T>::pack2(sacc[0][2], sacc[0][3]);
-        pa[2] = Elt<T>::pack2(sacc[1][0], sacc[1][1]);
-        pa[3] = Elt<T>::pack2(sacc[1][2], sacc[1][3]);
+        mma_softmax(acc, sacc, tig, seen_lo, seen_hi, p.scale_log2, pa);
 
         // Rows past the context may hold anything (even NaN): zero them in V so
         // that 0-weights cannot turn into NaN inside the MMA.
         if (valid < kTileTok) {
-            uint8_t* vrow = vtile;
             for (int idx = lane; idx < (kTileTok - valid) * (D / 8); idx += 32) {
                 const int r = valid + idx / (D / 8);
                 const int q16 = idx % (D / 8);  // 16-byte unit in the row (any order)
-                *reinterpret_cast<uint4*>(vrow + (q16 >> 3) * C::kHalfTile + r * 128 + (q16 & 7) * 16) =
+                *reinterpret_cast<uint4*>(vtile + (q16 >> 3) * C::kHalfTile + r * 128 + (q16 & 7) * 16) =
                     make_uint4(0u, 0u, 0u, 0u);
             }
             fence_proxy_async();  // these generic writes precede a later TMA refill
@@ -289,7 +262,7 @@ __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMa
             mma_16816<T>(acc.o[2 * jj + 1], pa, b2, b3);
         }
         __syncwarp();
-        if (!FP8 && i + STAGES < ntiles) issue(i + STAGES);
+        if (i + STAGES < ntiles) issue(i + STAGES);
     }
 #pragma unroll
     for (int off = 1; off < 4; off <<= 1) {
@@ -323,12 +296,13 @@ __device__ __forceinline__ void mma_store_row(const MmaAcc<T, D>& acc, bool hi, 
     }
 }
 
-template <typename T, int D, int WARPS, int STAGES, bool FP8 = false>
-__device__ __forceinline__ uint8_t* mma_setup_ring(uint8_t* smem_raw, int warp, int lane, uint32_t& bar0,
-                                                   const CUtensorMap* tmK, const CUtensorMap* tmV) {
-    using C = MmaCfg<T, D, WARPS, STAGES, FP8>;
+// One warp's ring: WARP_BYTES of stages at smem + warp * WARP_BYTES (smem
+// 1024-byte aligned), its STAGES mbarriers after all warps' data.
+template <int WARP_BYTES, int DATA_BYTES, int STAGES>
+__device__ __forceinline__ uint8_t* ring_setup(uint8_t* smem_raw, int warp, int lane, uint32_t& bar0,
+                                               const CUtensorMap* tmK, const CUtensorMap* tmV) {
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    bar0 = smem_u32(smem + C::kDataBytes + warp * STAGES * 8);
+    bar0 = smem_u32(smem + DATA_BYTES + warp * STAGES * 8);
     if (lane == 0) {
         prefetch_tensor_map(tmK);
         prefetch_tensor_map(tmV);
@@ -336,13 +310,18 @@ __device__ __forceinline__ uint8_t* mma_setup_ring(uint8_t* smem_raw, int warp, 
         fence_barrier_init();
     }
     __syncwarp();
-    return smem + warp * C::kWarpBytes;
+    return smem + warp * WARP_BYTES;
 }
 
-// Grouped-query decode: grid (ceil(Hkv / WARPS), partitions, S).  T is the
-// MMA type; To the type of q and out (T itself, or bf16 q/out with FP8 pools
-// computed in FP16).
-template <typename T, int D, int WARPS, int STAGES, bool FP8 = false, typename To = T>
+template <typename T, int D, int WARPS, int STAGES>
+__device__ __forceinline__ uint8_t* mma_setup_ring(uint8_t* smem_raw, int warp, int lane, uint32_t& bar0,
+                                                   const CUtensorMap* tmK, const CUtensorMap* tmV) {
+    using C = MmaCfg<T, D, WARPS, STAGES>;
+    return ring_setup<C::kWarpBytes, C::kDataBytes, STAGES>(smem_raw, warp, lane, bar0, tmK, tmV);
+}
+
+// Grouped-query decode: grid (ceil(Hkv / WARPS), partitions, S).
+template <typename T, int D, int WARPS, int STAGES>
 __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnParams p,
                                                                     const __grid_constant__ CUtensorMap tmK,
                                                                     const __grid_constant__ CUtensorMap tmV) {
@@ -360,19 +339,19 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnPa
     const Unit u = resolve_unit(p, s, part, part == 0 && g == 0 && lane == 0);
     if (u.t_begin >= u.L) {
         if (part == 0 && u.L == 0) {  // empty context: zeros for the group's heads
-            To* o = reinterpret_cast<To*>(p.out) + ((int64_t)s * p.Hq + h0) * D;
-            for (int i = lane; i < G * D; i += 32) o[i] = To(0.f);
+            T* o = reinterpret_cast<T*>(p.out) + ((int64_t)s * p.Hq + h0) * D;
+            for (int i = lane; i < G * D; i += 32) o[i] = T(0.f);
         }
         return;
     }
     uint32_t bar0;
-    uint8_t* ring = mma_setup_ring<T, D, WARPS, STAGES, FP8>(smem_raw, warp, lane, bar0, &tmK, &tmV);
+    uint8_t* ring = mma_setup_ring<T, D, WARPS, STAGES>(smem_raw, warp, lane, bar0, &tmK, &tmV);
 
-    const To* qb = reinterpret_cast<const To*>(p.q) + ((int64_t)s * p.Hq + h0) * D;
+    const T* qb = reinterpret_cast<const T*>(p.q) + ((int64_t)s * p.Hq + h0) * D;
     MmaAcc<T, D> acc;
     acc.load_q(gid < G ? qb + gid * D : nullptr, gid + 8 < G ? qb + (gid + 8) * D : nullptr, tig);
-    if (!mma_attend<T, D, WARPS, STAGES, FP8>(p, &tmK, &tmV, ring, bar0, p.block_tables + (int64_t)s * p.maxB,
-                                              u.t_begin, u.t_end, g, lane, acc, u.t_end, u.t_end))
+    if (!mma_attend<T, D, WARPS, STAGES>(p, &tmK, &tmV, ring, bar0, p.block_tables + (int64_t)s * p.maxB,
+                                         u.t_begin, u.t_end, g, lane, acc, u.t_end, u.t_end))
         return;
 
 #pragma unroll
@@ -381,10 +360,10 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnPa
         if (r >= G) continue;
         const int64_t row = (int64_t)s * p.Hq + h0 + r;
         if (u.direct) {
-            mma_store_row<To, T, D>(acc, hi, tig, reinterpret_cast<To*>(p.out) + row * D, nullptr, nullptr, p.v_scale);
+            mma_store_row<T, T, D>(acc, hi, tig, reinterpret_cast<T*>(p.out) + row * D, nullptr, nullptr, 1.f);
         } else {
             const int64_t idx = row * p.maxP + u.slot;
-            mma_store_row<To, T, D>(acc, hi, tig, (To*)nullptr, p.ws_o + idx * D, p.ws_ml + idx * 2, p.v_scale);
+            mma_store_row<T, T, D>(acc, hi, tig, (T*)nullptr, p.ws_o + idx * D, p.ws_ml + idx * 2, 1.f);
         }
     }
 }

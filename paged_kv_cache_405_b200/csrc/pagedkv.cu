@@ -13,6 +13,7 @@
 #include <cudaTypedefs.h>
 
 #include "../../include/pagedkv.h"
+#include "attention_fp8.cuh"
 #include "attention_mma.cuh"
 #include "attention_simt.cuh"
 #include "block_copy.cuh"
@@ -103,9 +104,10 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
-// A pool as a (rows x D) matrix.  swizzled: 16-bit elements, box = 64 elements
-// x 16 rows, 128-byte swizzle (tensor-core kernels).  Otherwise: box = D
-// elements x tile rows, no swizzle (a plain row-major copy of the tile).
+// A pool as a (rows x D) matrix.  swizzled: box = 128 bytes of a row (64
+// 16-bit elements or 128 FP8 codes) x 16 rows, 128-byte swizzle (tensor-core
+// kernels).  Otherwise: box = D elements x tile rows, no swizzle (a plain
+// row-major copy of the tile).
 static bool make_pool_map(CUtensorMap* map, const void* pool, int64_t rows, int D, pkv_dtype dt, bool swizzled,
                           int tile_rows = pkv::kTileTok) {
     auto fn = encode_fn();
@@ -113,7 +115,8 @@ static bool make_pool_map(CUtensorMap* map, const void* pool, int64_t rows, int 
     const int esz = elem_size(dt);
     cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
     cuuint64_t strides[1] = {(cuuint64_t)D * esz};
-    cuuint32_t box[2] = {swizzled ? 64u : (cuuint32_t)D, (cuuint32_t)(swizzled ? pkv::kTileTok : tile_rows)};
+    cuuint32_t box[2] = {swizzled ? (cuuint32_t)(128 / esz) : (cuuint32_t)D,
+                         (cuuint32_t)(swizzled ? pkv::kTileTok : tile_rows)};
     cuuint32_t estr[2] = {1, 1};
     const CUtensorMapDataType ty = dt == PKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                    : dt == PKV_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
@@ -220,17 +223,22 @@ static cudaError_t launch_chunk(const pkv::AttnParams& p, const pkv::ChunkParams
     return cudaGetLastError();
 }
 
-// FP8 pools: stages of E4M3 tiles converted to FP16 per warp.
+// FP8 pools: stages of E4M3 tiles per warp, widened to FP16 in registers.
 #ifndef PKV_FP8_STAGES
 #define PKV_FP8_STAGES 2
 #endif
 constexpr int kFp8Stages = PKV_FP8_STAGES;
+// Smallest query group that FP8 pools send to the tensor-core kernel.
+#ifndef PKV_FP8_MMA_MIN_GROUP
+#define PKV_FP8_MMA_MIN_GROUP 2
+#endif
+constexpr int kFp8MmaMinGroup = PKV_FP8_MMA_MIN_GROUP;
 
 template <typename To, int D>
 static cudaError_t launch_mma_fp8(const pkv::AttnParams& p, dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv,
                                   cudaStream_t st) {
-    using C = pkv::MmaCfg<__half, D, kMmaWarps, kFp8Stages, true>;
-    auto k = pkv::paged_attn_mma_kernel<__half, D, kMmaWarps, kFp8Stages, true, To>;
+    using C = pkv::Fp8Cfg<D, kMmaWarps, kFp8Stages>;
+    auto k = pkv::paged_attn_fp8_kernel<D, kMmaWarps, kFp8Stages, To>;
     static cudaError_t attr = set_smem(k, C::kSmemBytes);
     if (attr != cudaSuccess) return attr;
     k<<<grid, kMmaWarps * 32, C::kSmemBytes, st>>>(p, mk, mv);
@@ -425,12 +433,12 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
     p.max_group_size = grp.max_size;
     p.max_shared = grp.max_shared;
 
-    const bool use_mma = dtype != PKV_F32 && p.G >= 2 && p.G <= 16;
+    const bool use_mma = dtype != PKV_F32 && p.G >= (kv.fp8 ? kFp8MmaMinGroup : 2) && p.G <= 16;
     CUtensorMap mk, mv;
     if (kv.fp8) {
         const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
-        if (use_mma && (!make_pool_map(&mk, k_pool, rows, head_dim, PKV_FP8_E4M3, false) ||
-                        !make_pool_map(&mv, v_pool, rows, head_dim, PKV_FP8_E4M3, false))) {
+        if (use_mma && (!make_pool_map(&mk, k_pool, rows, head_dim, PKV_FP8_E4M3, head_dim == 128) ||
+                        !make_pool_map(&mv, v_pool, rows, head_dim, PKV_FP8_E4M3, head_dim == 128))) {
             g_msg = "pkv_paged_attention_decode_fp8: cuTensorMapEncodeTiled failed";
             return PKV_ERR_CUDA;
         }
