@@ -249,9 +249,10 @@ pkv_status pkv_kv_append_fp8(const void* k_new, const void* v_new, void* k_pool,
 /*
  * pkv_paged_attention_decode_fp8 -- pkv_paged_attention_decode over FP8
  * pools: q and out of type dtype (bf16 or f16), K/V values = code x k_scale /
- * x v_scale.  Same workspace as pkv_attention_workspace_bytes.  Query groups
- * of 2..16 heads run on tensor cores in FP16 (codes convert exactly; q is
- * rounded to FP16 once), others on CUDA cores.
+ * x v_scale.  Same workspace as pkv_attention_workspace_bytes.  Runs on
+ * tensor cores in FP16 with fp32 accumulation (every code converts exactly;
+ * q and the softmax weights are rounded to FP16 once): query groups of 2..16
+ * heads share each K/V tile, other group sizes go one query head per warp.
  */
 pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* k_pool, const void* v_pool,
                                           const int32_t* block_tables, int max_blocks_per_seq,

@@ -251,4 +251,212 @@ __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_fp8_kernel(const Att
     }
 }
 
+// Per-head decode over FP8 pools (multi-head attention: one query head per
+// kv head, so no two queries share a K/V byte).  One warp per (sequence,
+// query head, partition).  The tokens are the MMA rows and the query is the
+// single live column of an n8 operand:
+//  * S^T = K q^T.  A = the K tile (16 tokens x 16 head-dim elements per
+//    k-step, rows gid and gid+8 per lane, the same permuted contraction as
+//    above); B column 0 = q, held by the lanes with gid = 0, other columns 0.
+//    The score of token gid (gid + 8) lands in the lane (gid, tig = 0).
+//  * O^T += V^T p^T.  A = V^T: m-tile mt, row r is head-dim element
+//    gid*D/8 + 2mt (r = gid) or gid*D/8 + 2mt + 1 (r = gid + 8), contraction
+//    over the tokens in S-column order (2tig, 2tig+1, 8+2tig, 9+2tig); the
+//    lane reads D/8 consecutive codes of each of its four tokens, as in the
+//    grouped kernel.  B column 0 = p, gathered into the gid = 0 lanes with
+//    four shuffles.  The lane (gid, tig = 0) ends with output elements
+//    gid*D/8 .. gid*D/8 + D/8 - 1.
+// Half the MMAs of the grouped layout (8 + 8 per tile at D = 128) and a
+// quarter of the CUDA-core instructions of widening every code to fp32.
+template <int D, int WARPS, int STAGES, typename To>
+__global__ void __launch_bounds__(WARPS * 32, 4) paged_attn_fp8_head_kernel(const AttnParams p,
+                                                                            const __grid_constant__ CUtensorMap tmK,
+                                                                            const __grid_constant__ CUtensorMap tmV) {
+    using C = Fp8Cfg<D, WARPS, STAGES>;
+    using H = MmaAcc<__half, D>;
+    constexpr int KSTEPS = D / 16;  // S^T k-steps; also 32-bit words of K codes per lane and row
+    constexpr int NMT = D / 16;     // O^T m-tiles
+    constexpr int VW = D / 32;      // 32-bit words of V codes per lane and token (D/8 codes)
+    constexpr int SPAN = D / 8;     // output elements per lane with tig = 0
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int h = blockIdx.x * WARPS + warp;  // query head
+    const int part = blockIdx.y;
+    const int s = blockIdx.z;
+    if (h >= p.Hq) return;
+    const int gid = lane >> 2, tig = lane & 3;
+    const int g = h / p.G;
+
+    const Unit u = resolve_unit(p, s, part, part == 0 && h == 0 && lane == 0);
+    if (u.t_begin >= u.L) {
+        if (part == 0 && u.L == 0) {  // empty context: zeros
+            To* o = reinterpret_cast<To*>(p.out) + ((int64_t)s * p.Hq + h) * D;
+            for (int i = lane; i < D; i += 32) o[i] = To(0.f);
+        }
+        return;
+    }
+    uint32_t bar0;
+    uint8_t* ring = ring_setup<C::kWarpBytes, C::kDataBytes, STAGES>(smem_raw, warp, lane, bar0, &tmK, &tmV);
+    const uint32_t ring_s = smem_u32(ring);
+
+    // q as column 0 of the B operand of S^T (lanes gid = 0).
+    uint32_t qb[KSTEPS][2];
+    {
+        const To* qr = reinterpret_cast<const To*>(p.q) + ((int64_t)s * p.Hq + h) * D + tig * (D / 4);
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+            qb[kk][0] = gid == 0 ? H::pair(qr + 4 * kk) : 0u;
+            qb[kk][1] = gid == 0 ? H::pair(qr + 4 * kk + 2) : 0u;
+        }
+    }
+    float o[NMT][4];
+#pragma unroll
+    for (int j = 0; j < NMT; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+    float m = -INFINITY, l = 0.f;  // m warp-uniform; l a per-lane share
+
+    const int t_begin = u.t_begin, t_end = u.t_end;
+    const int ntiles = (t_end - t_begin + kTileTok - 1) / kTileTok;
+    const int jb0 = t_begin / p.bs;
+    BlockWindow win;
+    win.init(p.block_tables + (int64_t)s * p.maxB, jb0, (t_end - 1) / p.bs - jb0 + 1, lane);
+
+    auto issue = [&](int i) {
+        const int t0 = t_begin + i * kTileTok;
+        const int blk = win.get(t0 / p.bs - jb0, lane, p.NB);
+        if (lane == 0) {
+            const int row = (blk * p.Hkv + g) * p.bs + (t0 % p.bs);
+            const int st = i % STAGES;
+            const uint32_t bar = bar0 + 8 * st;
+            const uint32_t dst = ring_s + st * C::kStageBytes;
+            fence_proxy_async();
+            mbar_arrive_expect_tx(bar, C::kStageBytes);
+            tma_load_2d(dst, &tmK, 0, row, bar);
+            tma_load_2d(dst + C::kTileBytes, &tmV, 0, row, bar);
+        }
+    };
+    const int npre = ntiles < STAGES ? ntiles : STAGES;
+    for (int i = 0; i < npre; ++i) issue(i);
+
+    const int vtok[4] = {2 * tig, 2 * tig + 1, 8 + 2 * tig, 9 + 2 * tig};
+
+    for (int i = 0; i < ntiles; ++i) {
+        const int st = i % STAGES;
+        if (!ring_wait<STAGES>(bar0, i, ntiles)) return;
+        const int valid = min(kTileTok, t_end - (t_begin + i * kTileTok));
+        const uint8_t* kt = ring + st * C::kStageBytes;
+        const uint8_t* vt = kt + C::kTileBytes;
+
+        uint32_t kw[2][KSTEPS];  // codes of rows gid and gid + 8
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+#pragma unroll
+            for (int c = 0; c < KSTEPS / 4; ++c) {
+                const uint4 w = *reinterpret_cast<const uint4*>(kt + fp8_chunk<D>(hh * 8 + gid, tig * (KSTEPS / 4) + c));
+                kw[hh][4 * c] = w.x;
+                kw[hh][4 * c + 1] = w.y;
+                kw[hh][4 * c + 2] = w.z;
+                kw[hh][4 * c + 3] = w.w;
+            }
+        }
+        uint32_t vw[4][VW];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            if constexpr (VW == 4) {
+                const uint4 w = *reinterpret_cast<const uint4*>(vt + fp8_chunk<D>(vtok[t], gid));
+                vw[t][0] = w.x;
+                vw[t][1] = w.y;
+                vw[t][2] = w.z;
+                vw[t][3] = w.w;
+            } else {
+                const uint2 w = *reinterpret_cast<const uint2*>(vt + vtok[t] * D + gid * 8);
+                vw[t][0] = w.x;
+                vw[t][1] = w.y;
+            }
+            if (vtok[t] >= valid) {  // rows past the context may hold NaN codes
+#pragma unroll
+                for (int w = 0; w < VW; ++w) vw[t][w] = 0u;
+            }
+        }
+        __syncwarp();
+        if (i + STAGES < ntiles) issue(i + STAGES);
+
+        // S^T: two accumulator chains (even / odd k-steps) halve the MMA
+        // dependency depth.
+        float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int kk = 0; kk < KSTEPS; ++kk) {
+            const uint32_t a[4] = {e4m3x2_to_f16x2((uint16_t)(kw[0][kk] & 0xffffu)),
+                                   e4m3x2_to_f16x2((uint16_t)(kw[1][kk] & 0xffffu)),
+                                   e4m3x2_to_f16x2((uint16_t)(kw[0][kk] >> 16)),
+                                   e4m3x2_to_f16x2((uint16_t)(kw[1][kk] >> 16))};
+            mma_16816<__half>(sa[kk & 1], a, qb[kk][0], qb[kk][1]);
+        }
+        const bool live = tig == 0;
+        const float x_lo = live && gid < valid ? (sa[0][0] + sa[1][0]) * p.scale_log2 : -INFINITY;
+        const float x_hi = live && gid + 8 < valid ? (sa[0][2] + sa[1][2]) * p.scale_log2 : -INFINITY;
+        float mt = fmaxf(x_lo, x_hi);
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
+        const float mn = fmaxf(m, mt);
+        const float b = mn == -INFINITY ? 0.f : mn;  // no -inf - -inf
+        const float alpha = ex2(m - b);
+        const float p_lo = ex2(x_lo - b), p_hi = ex2(x_hi - b);
+        l = l * alpha + p_lo + p_hi;
+        m = mn;
+        if (alpha != 1.f) {  // warp-uniform; exactly 1 once the maximum settles
+#pragma unroll
+            for (int j = 0; j < NMT; ++j) {
+                o[j][0] *= alpha;
+                o[j][2] *= alpha;
+            }
+        }
+        // p^T column 0: tokens 2tig, 2tig+1 (b0) and 8+2tig, 9+2tig (b1).
+        const float p0 = __shfl_sync(0xffffffffu, p_lo, 8 * tig);
+        const float p1 = __shfl_sync(0xffffffffu, p_lo, 8 * tig + 4);
+        const float p2 = __shfl_sync(0xffffffffu, p_hi, 8 * tig);
+        const float p3 = __shfl_sync(0xffffffffu, p_hi, 8 * tig + 4);
+        const uint32_t pb0 = gid == 0 ? Elt<__half>::pack2(p0, p1) : 0u;
+        const uint32_t pb1 = gid == 0 ? Elt<__half>::pack2(p2, p3) : 0u;
+
+        // O^T += V^T p^T
+#pragma unroll
+        for (int w = 0; w < VW; ++w) {
+            const uint32_t lo0 = __byte_perm(vw[0][w], vw[1][w], 0x5140);
+            const uint32_t hi0 = __byte_perm(vw[0][w], vw[1][w], 0x7362);
+            const uint32_t lo1 = __byte_perm(vw[2][w], vw[3][w], 0x5140);
+            const uint32_t hi1 = __byte_perm(vw[2][w], vw[3][w], 0x7362);
+            const uint32_t a0[4] = {e4m3x2_to_f16x2((uint16_t)(lo0 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(lo0 >> 16)),
+                                    e4m3x2_to_f16x2((uint16_t)(lo1 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(lo1 >> 16))};
+            mma_16816<__half>(o[2 * w], a0, pb0, pb1);
+            const uint32_t a1[4] = {e4m3x2_to_f16x2((uint16_t)(hi0 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(hi0 >> 16)),
+                                    e4m3x2_to_f16x2((uint16_t)(hi1 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(hi1 >> 16))};
+            mma_16816<__half>(o[2 * w + 1], a1, pb0, pb1);
+        }
+    }
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
+    if (tig != 0) return;
+
+    // Lane (gid, 0): elements gid*SPAN + 2mt (o[mt][0]) and + 2mt + 1 (o[mt][2]).
+    const int64_t row = (int64_t)s * p.Hq + h;
+    if (u.direct) {
+        const float inv = p.v_scale / l;
+        uint32_t hw[NMT];
+#pragma unroll
+        for (int j = 0; j < NMT; ++j) hw[j] = Elt<To>::pack2(o[j][0] * inv, o[j][2] * inv);
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<To*>(p.out) + row * D + gid * SPAN);
+#pragma unroll
+        for (int v = 0; v < NMT / 4; ++v) dst[v] = make_uint4(hw[4 * v], hw[4 * v + 1], hw[4 * v + 2], hw[4 * v + 3]);
+    } else {
+        const int64_t idx = row * p.maxP + u.slot;
+        float4* dst = reinterpret_cast<float4*>(p.ws_o + idx * D + gid * SPAN);
+#pragma unroll
+        for (int v = 0; v < NMT / 2; ++v)
+            dst[v] = make_float4(o[2 * v][0] * p.v_scale, o[2 * v][2] * p.v_scale, o[2 * v + 1][0] * p.v_scale,
+                                 o[2 * v + 1][2] * p.v_scale);
+        if (gid == 0) *reinterpret_cast<float2*>(p.ws_ml + idx * 2) = make_float2(m, l);
+    }
+}
+
 }  // namespace pkv

@@ -228,11 +228,7 @@ static cudaError_t launch_chunk(const pkv::AttnParams& p, const pkv::ChunkParams
 #define PKV_FP8_STAGES 2
 #endif
 constexpr int kFp8Stages = PKV_FP8_STAGES;
-// Smallest query group that FP8 pools send to the tensor-core kernel.
-#ifndef PKV_FP8_MMA_MIN_GROUP
-#define PKV_FP8_MMA_MIN_GROUP 2
-#endif
-constexpr int kFp8MmaMinGroup = PKV_FP8_MMA_MIN_GROUP;
+
 
 template <typename To, int D>
 static cudaError_t launch_mma_fp8(const pkv::AttnParams& p, dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv,
@@ -247,14 +243,13 @@ static cudaError_t launch_mma_fp8(const pkv::AttnParams& p, dim3 grid, const CUt
 }
 
 template <typename To, int D>
-static cudaError_t launch_simt_fp8(const pkv::AttnParams& p, dim3 grid, cudaStream_t st) {
-    using C = pkv::SimtCfg<To, D, kSimtWarps, kSimtStages, kSimtTile, pkv::fp8e4m3>;
-    auto k = pkv::paged_attn_simt_kernel<To, D, kSimtWarps, kSimtStages, kSimtTile, false, pkv::fp8e4m3>;
+static cudaError_t launch_head_fp8(const pkv::AttnParams& p, dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv,
+                                   cudaStream_t st) {
+    using C = pkv::Fp8Cfg<D, kMmaWarps, kFp8Stages>;
+    auto k = pkv::paged_attn_fp8_head_kernel<D, kMmaWarps, kFp8Stages, To>;
     static cudaError_t attr = set_smem(k, C::kSmemBytes);
     if (attr != cudaSuccess) return attr;
-    CUtensorMap none;
-    std::memset(&none, 0, sizeof none);
-    k<<<grid, kSimtWarps * 32, C::kSmemBytes, st>>>(p, none, none);
+    k<<<grid, kMmaWarps * 32, C::kSmemBytes, st>>>(p, mk, mv);
     g_launches++;
     return cudaGetLastError();
 }
@@ -305,8 +300,8 @@ static cudaError_t dispatch_attention_fp8(const pkv::AttnParams& p, int D, int n
         dim3 grid((p.Hkv + kMmaWarps - 1) / kMmaWarps, nparts, p.S);
         e = D == 64 ? launch_mma_fp8<To, 64>(p, grid, *mk, *mv, st) : launch_mma_fp8<To, 128>(p, grid, *mk, *mv, st);
     } else {
-        dim3 grid((p.Hq + kSimtWarps - 1) / kSimtWarps, nparts, p.S);
-        e = D == 64 ? launch_simt_fp8<To, 64>(p, grid, st) : launch_simt_fp8<To, 128>(p, grid, st);
+        dim3 grid((p.Hq + kMmaWarps - 1) / kMmaWarps, nparts, p.S);
+        e = D == 64 ? launch_head_fp8<To, 64>(p, grid, *mk, *mv, st) : launch_head_fp8<To, 128>(p, grid, *mk, *mv, st);
     }
     if (e != cudaSuccess || p.maxP <= 1) return e;
     pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
@@ -433,12 +428,12 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
     p.max_group_size = grp.max_size;
     p.max_shared = grp.max_shared;
 
-    const bool use_mma = dtype != PKV_F32 && p.G >= (kv.fp8 ? kFp8MmaMinGroup : 2) && p.G <= 16;
+    const bool use_mma = dtype != PKV_F32 && p.G >= 2 && p.G <= 16;
     CUtensorMap mk, mv;
-    if (kv.fp8) {
+    if (kv.fp8) {  // both FP8 kernels read 16-token boxes of codes
         const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
-        if (use_mma && (!make_pool_map(&mk, k_pool, rows, head_dim, PKV_FP8_E4M3, head_dim == 128) ||
-                        !make_pool_map(&mv, v_pool, rows, head_dim, PKV_FP8_E4M3, head_dim == 128))) {
+        if (!make_pool_map(&mk, k_pool, rows, head_dim, PKV_FP8_E4M3, head_dim == 128) ||
+            !make_pool_map(&mv, v_pool, rows, head_dim, PKV_FP8_E4M3, head_dim == 128)) {
             g_msg = "pkv_paged_attention_decode_fp8: cuTensorMapEncodeTiled failed";
             return PKV_ERR_CUDA;
         }

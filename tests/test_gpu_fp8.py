@@ -53,7 +53,7 @@ def test_kv_append_fp8_bit_exact(src, scales):
 
 
 @pytest.mark.parametrize("qdt", ["bf16", "f16"])
-@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 2), (8, 1), (32, 2)])
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 2), (8, 1), (32, 2), (40, 2)])
 @pytest.mark.parametrize("bs,D", [(16, 128), (64, 128), (32, 64)])
 @pytest.mark.parametrize("P", [0, 32, 512])
 def test_decode_fp8_matches_oracle(qdt, Hq, Hkv, bs, D, P):
@@ -68,6 +68,28 @@ def test_decode_fp8_matches_oracle(qdt, Hq, Hkv, bs, D, P):
     pkv.paged_attention_decode_fp8(out, b.q.cuda(), kc.cuda(), vc.cuda(), torch.from_numpy(b.block_tables).cuda(),
                                    torch.from_numpy(b.lens.astype(np.int32)).cuda(), ks, vs, partition_size=P)
     assert pkv.device_error() == 0
+    assert max_err(out, ref) <= TOL[out.dtype]
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 4)])
+def test_decode_fp8_empty_and_one_token_contexts(Hq, Hkv):
+    """Zero-length contexts give zeros; one-token contexts give that token's
+    value (dequantized), through both the per-head and the grouped kernel."""
+    import paged_kv_cache_405_b200 as pkv
+    sh = synth.shrink(synth.CONFIGS["llama7b"], S=7, Hq=Hq, Hkv=Hkv, len_uniform=(1, 40), seed=3)
+    b = synth.make_batch(sh)
+    lens = b.lens.copy()
+    lens[[0, 3]] = 0
+    lens[[1, 5]] = 1
+    ks, vs = 1 / 16, 1 / 4
+    kc, vc = fp8_pools(b, 2, ks, vs)
+    ref = oracle.paged_attention_kv(b.q, kc, vc, ks, vs, b.block_tables, lens, threads=oracle.max_threads())
+    out = torch.full_like(b.q, float("nan"), device="cuda")
+    pkv.paged_attention_decode_fp8(out, b.q.cuda(), kc.cuda(), vc.cuda(), torch.from_numpy(b.block_tables).cuda(),
+                                   torch.from_numpy(lens.astype(np.int32)).cuda(), ks, vs)
+    assert pkv.device_error() == 0
+    o = out.float().cpu()
+    assert torch.all(o[[0, 3]] == 0)
     assert max_err(out, ref) <= TOL[out.dtype]
 
 
