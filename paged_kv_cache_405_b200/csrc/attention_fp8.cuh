@@ -53,6 +53,20 @@ __device__ __forceinline__ int fp8_chunk(int r, int c) {
     else return r * D + (c << 4);
 }
 
+// V rows past the context (the end of a partial tile) may hold any code, NaN
+// included, and a zero weight times NaN would poison the sum: clear them in
+// the stage before reading it (whole rows, so the swizzle does not matter).
+template <int D>
+__device__ __forceinline__ void zero_tail_rows(uint8_t* vt, int valid, int lane) {
+    if (valid >= kTileTok) return;
+    for (int idx = lane; idx < (kTileTok - valid) * (D / 16); idx += 32) {
+        const int r = valid + idx / (D / 16);
+        *reinterpret_cast<uint4*>(vt + r * D + (idx % (D / 16)) * 16) = make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async();  // these generic writes precede the stage's next TMA refill
+    __syncwarp();
+}
+
 template <int D, int WARPS, int STAGES, typename To>
 __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_fp8_kernel(const AttnParams p,
                                                                        const __grid_constant__ CUtensorMap tmK,
@@ -151,6 +165,7 @@ __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_fp8_kernel(const Att
                 kw[nt][4 * c + 3] = w.w;
             }
         }
+        zero_tail_rows<D>(const_cast<uint8_t*>(vt), valid, lane);
         uint32_t vw[4][VW];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -164,12 +179,6 @@ __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_fp8_kernel(const Att
                 const uint2 w = *reinterpret_cast<const uint2*>(vt + vtok[t] * D + gid * 8);
                 vw[t][0] = w.x;
                 vw[t][1] = w.y;
-            }
-            // Rows past the context may hold any code (NaN included): a zero
-            // weight times NaN would poison the sum, so drop them here.
-            if (vtok[t] >= valid) {
-#pragma unroll
-                for (int w = 0; w < VW; ++w) vw[t][w] = 0u;
             }
         }
         __syncwarp();
@@ -359,6 +368,7 @@ __global__ void __launch_bounds__(WARPS * 32, 4) paged_attn_fp8_head_kernel(cons
                 kw[hh][4 * c + 3] = w.w;
             }
         }
+        zero_tail_rows<D>(const_cast<uint8_t*>(vt), valid, lane);
         uint32_t vw[4][VW];
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
@@ -372,10 +382,6 @@ __global__ void __launch_bounds__(WARPS * 32, 4) paged_attn_fp8_head_kernel(cons
                 const uint2 w = *reinterpret_cast<const uint2*>(vt + vtok[t] * D + gid * 8);
                 vw[t][0] = w.x;
                 vw[t][1] = w.y;
-            }
-            if (vtok[t] >= valid) {  // rows past the context may hold NaN codes
-#pragma unroll
-                for (int w = 0; w < VW; ++w) vw[t][w] = 0u;
             }
         }
         __syncwarp();

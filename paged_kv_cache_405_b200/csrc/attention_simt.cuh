@@ -30,16 +30,15 @@
 
 namespace pkv {
 
-// T: element type of q and out; KV: element type of the pools (T, or FP8
-// codes whose values are code x k_scale / v_scale).
-template <typename T, int D, int WARPS, int STAGES, int TILE = kTileTok, typename KV = T>
+// T: element type of q, out and the pools.
+template <typename T, int D, int WARPS, int STAGES, int TILE = kTileTok>
 struct SimtCfg {
     static constexpr int kTile = TILE;                 // tokens per pipeline stage
-    static constexpr int kRowBytes = D * (int)sizeof(KV);
+    static constexpr int kRowBytes = D * (int)sizeof(T);
     static constexpr int kTileBytes = TILE * kRowBytes;
     static constexpr int kLPT = kRowBytes / 16;        // lanes per token row
     static constexpr int kTPI = 32 / kLPT;             // tokens per pass
-    static constexpr int kEPL = 16 / (int)sizeof(KV);  // elements per lane
+    static constexpr int kEPL = 16 / (int)sizeof(T);  // elements per lane
     static constexpr int kPasses = TILE / kTPI;       // tokens of one lane group per tile
     static_assert(kPasses >= 1 && kPasses * 2 <= kLPT, "tile must give each lane group 1..LPT/2 tokens");
     static constexpr int kStageBytes = 2 * kTileBytes;
@@ -50,7 +49,7 @@ struct SimtCfg {
 
 // One tile of the CUDA-core kernel (see the kernel below).  FULL = every
 // token of the tile is inside the context, so no masking is needed.
-template <typename C, typename KV, bool FULL>
+template <typename C, typename T, bool FULL>
 __device__ __forceinline__ void simt_tile(const uint8_t* Ks, const uint8_t* Vs, int valid, int lane, int sub, int c,
                                           const float (&qf)[C::kEPL], float (&o)[C::kEPL], float& m, float& l) {
     constexpr int LPT = C::kLPT, TPI = C::kTPI, EPL = C::kEPL;
@@ -63,7 +62,7 @@ __device__ __forceinline__ void simt_tile(const uint8_t* Ks, const uint8_t* Vs, 
         const int r = ps * TPI + sub;
         const uint4 kv = *reinterpret_cast<const uint4*>(Ks + r * C::kRowBytes + c * 16);
         float kf[EPL];
-        Elt<KV>::widen(kv, kf);
+        Elt<T>::widen(kv, kf);
         float acc = 0.f;
 #pragma unroll
         for (int e = 0; e < EPL; ++e) acc = fmaf(qf[e], kf[e], acc);
@@ -106,17 +105,17 @@ __device__ __forceinline__ void simt_tile(const uint8_t* Ks, const uint8_t* Vs, 
         uint4 vv = *reinterpret_cast<const uint4*>(Vs + r * C::kRowBytes + c * 16);
         if (!FULL && r >= valid) vv = make_uint4(0u, 0u, 0u, 0u);  // rows past the context may hold NaN
         float vf[EPL];
-        Elt<KV>::widen(vv, vf);
+        Elt<T>::widen(vv, vf);
 #pragma unroll
         for (int e = 0; e < EPL; ++e) o[e] = fmaf(pw, vf[e], o[e]);
     }
 }
 
-template <typename T, int D, int WARPS, int STAGES, int TILE, bool TENSOR, typename KV = T>
+template <typename T, int D, int WARPS, int STAGES, int TILE, bool TENSOR>
 __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_simt_kernel(const AttnParams p,
                                                                        const __grid_constant__ CUtensorMap tmK,
                                                                        const __grid_constant__ CUtensorMap tmV) {
-    using C = SimtCfg<T, D, WARPS, STAGES, TILE, KV>;
+    using C = SimtCfg<T, D, WARPS, STAGES, TILE>;
     constexpr int LPT = C::kLPT, EPL = C::kEPL;
     extern __shared__ __align__(128) uint8_t smem[];
 
@@ -205,8 +204,8 @@ __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_simt_kernel(const At
         const int valid = min(TILE, t_end - (t_begin + i * TILE));
         const uint8_t* Ks = ring + st * C::kStageBytes;
         const uint8_t* Vs = Ks + C::kTileBytes;
-        if (valid == TILE) simt_tile<C, KV, true>(Ks, Vs, valid, lane, sub, c, qf, o, m, l);
-        else simt_tile<C, KV, false>(Ks, Vs, valid, lane, sub, c, qf, o, m, l);
+        if (valid == TILE) simt_tile<C, T, true>(Ks, Vs, valid, lane, sub, c, qf, o, m, l);
+        else simt_tile<C, T, false>(Ks, Vs, valid, lane, sub, c, qf, o, m, l);
         __syncwarp();
         if (i + STAGES < ntiles) issue(i + STAGES);
     }
@@ -223,7 +222,7 @@ __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_simt_kernel(const At
     }
     if (sub != 0) return;
     if (u.direct) {
-        const float inv = p.v_scale / l;
+        const float inv = 1.f / l;
         float r[EPL];
 #pragma unroll
         for (int e = 0; e < EPL; ++e) r[e] = o[e] * inv;
@@ -233,7 +232,7 @@ __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_simt_kernel(const At
         float4* dst = reinterpret_cast<float4*>(p.ws_o + idx * D + c * EPL);
 #pragma unroll
         for (int e = 0; e < EPL; e += 4)
-            dst[e / 4] = make_float4(o[e] * p.v_scale, o[e + 1] * p.v_scale, o[e + 2] * p.v_scale, o[e + 3] * p.v_scale);
+            dst[e / 4] = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
         if (c == 0) *reinterpret_cast<float2*>(p.ws_ml + idx * 2) = make_float2(m, l);
     }
 }

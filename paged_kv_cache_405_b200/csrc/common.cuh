@@ -198,11 +198,6 @@ struct Elt<__half> {
     }
 };
 
-// FP8 E4M3 storage element (a pool of codes; values = code value x scale).
-struct fp8e4m3 {
-    uint8_t bits;
-};
-
 // Two E4M3 codes (low byte first) -> two halves, exactly (every E4M3 value
 // is an FP16 value).
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t two) {
@@ -218,27 +213,6 @@ __device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
     return r;
 }
-
-template <>
-struct Elt<fp8e4m3> {
-    static constexpr int kPer16B = 16;
-    __device__ __forceinline__ static void widen4(uint32_t w, float* f) {
-        const uint32_t a = e4m3x2_to_f16x2((uint16_t)(w & 0xffffu));
-        const uint32_t b = e4m3x2_to_f16x2((uint16_t)(w >> 16));
-        const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&a));
-        const float2 y = __half22float2(*reinterpret_cast<const __half2*>(&b));
-        f[0] = x.x;
-        f[1] = x.y;
-        f[2] = y.x;
-        f[3] = y.y;
-    }
-    __device__ __forceinline__ static void widen(const uint4& v, float* f) {
-        widen4(v.x, f);
-        widen4(v.y, f + 4);
-        widen4(v.z, f + 8);
-        widen4(v.w, f + 12);
-    }
-};
 
 // EPL consecutive elements of T <-> floats, in 16-byte pieces.
 template <typename T, int EPL>
