@@ -166,13 +166,10 @@ class DecodeSession:
         return out
 
     def chunk_to_device(self, p: ChunkPlan) -> dict:
-        dev = self.device
-
-        def up(a):
-            return torch.from_numpy(np.ascontiguousarray(a)).to(dev)
-        return dict(slot_mapping=up(p.slot_mapping), n_cow=len(p.cow_pairs),
-                    cow_pairs=up(p.cow_pairs) if len(p.cow_pairs) else None, lens=up(p.lens),
-                    block_tables=up(p.block_tables), query_start=up(p.query_start), max_query_len=p.max_query_len)
+        """Copy a chunk plan to the device (one packed asynchronous copy)."""
+        sm, cow, lens, bt, qs = self._pack_h2d([p.slot_mapping, p.cow_pairs, p.lens, p.block_tables, p.query_start])
+        return dict(slot_mapping=sm, n_cow=len(p.cow_pairs), cow_pairs=cow if len(p.cow_pairs) else None, lens=lens,
+                    block_tables=bt, query_start=qs, max_query_len=p.max_query_len)
 
     def reserve_chunk_workspace(self, num_tokens: int):
         """Grow the workspace for chunk calls of up to num_tokens query rows."""
@@ -248,20 +245,41 @@ class DecodeSession:
         return out_host
 
     def upload(self, p: StepPlan) -> DevicePlan:
-        """Copy a plan to the device through pinned staging buffers (asynchronous)."""
-        d = DevicePlan(*(self._h2d(n, a) for n, a in (("slots", p.slot_mapping), ("cow", p.cow_pairs),
-                                                      ("lens", p.lens), ("bt", p.block_tables))),
-                       len(p.cow_pairs))
+        """Copy a plan to the device: its arrays packed into one pinned staging
+        buffer and sent with a single asynchronous copy."""
+        arrs = [p.slot_mapping, p.cow_pairs, p.lens, p.block_tables]
         if p.has_groups:
-            d.group_first = self._h2d("gfirst", p.group_first)
-            d.group_shared = self._h2d("gshared", p.group_shared)
+            arrs += [p.group_first, p.group_shared]
+        dv = self._pack_h2d(arrs)
+        d = DevicePlan(dv[0], dv[1], dv[2], dv[3], len(p.cow_pairs))
+        if p.has_groups:
+            d.group_first, d.group_shared = dv[4], dv[5]
             d.max_group_size, d.max_shared_len = p.max_group_size, p.max_shared_len
         return d
 
-    def _h2d(self, name, a: np.ndarray) -> torch.Tensor:
-        src = torch.from_numpy(np.ascontiguousarray(a))
-        if src.numel() == 0:
-            return torch.zeros(a.shape, dtype=src.dtype, device=self.device)
-        pin = self._pin(name, src)
-        pin.copy_(src)
-        return pin.to(self.device, non_blocking=True)
+    def _pack_h2d(self, arrays) -> list:
+        """One host->device copy for several host arrays (each at a 256-byte
+        aligned offset); returns device views of the original shapes/dtypes.
+        Two staging buffers alternate, and a buffer is refilled only after its
+        previous copy has completed, so calls need no synchronisation."""
+        arrays = [np.ascontiguousarray(a) for a in arrays]
+        offs, total = [], 0
+        for a in arrays:
+            offs.append(total)
+            total += (a.nbytes + 255) // 256 * 256
+        total = max(total, 256)
+        k = self._stage_next = getattr(self, "_stage_next", 0) ^ 1
+        stage, ev = self._pinned.get(("stage", k), (None, None))
+        if ev is not None:
+            ev.synchronize()
+        if stage is None or stage.numel() < total:
+            stage = torch.empty(max(total, 1 << 16), dtype=torch.uint8, pin_memory=True)
+        sv = stage.numpy()
+        for a, o in zip(arrays, offs):
+            sv[o:o + a.nbytes] = a.reshape(-1).view(np.uint8)
+        dev = stage[:total].to(self.device, non_blocking=True)
+        ev = torch.cuda.Event()
+        ev.record()
+        self._pinned[("stage", k)] = (stage, ev)
+        return [dev[o:o + a.nbytes].view(torch.from_numpy(a[:0].reshape(-1)).dtype).view(a.shape)
+                for a, o in zip(arrays, offs)]

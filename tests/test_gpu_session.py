@@ -1,0 +1,87 @@
+"""DecodeSession through its host-buffer path (``step`` and ``upload``):
+several decode steps with a fork (copy-on-write of the shared last block),
+against the oracle allocator, ``block_copy``, ``kv_append`` and attention."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from gpu_helpers import TOL, max_err
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 2)])
+def test_session_steps_from_host_buffers_match_oracle(Hq, Hkv):
+    import paged_kv_cache_405_b200 as m
+    sh = synth.shrink(synth.CONFIGS["llama7b"], S=5, Hq=Hq, Hkv=Hkv, len_uniform=(1, 300), seed=11,
+                      reserve_tokens=64)
+    b = synth.make_batch(sh)
+    dev = torch.device("cuda")
+    k, v = b.k_pool.to(dev), b.v_pool.to(dev)
+    ss = m.DecodeSession(k, v, sh.Hq, b.max_blocks, free_order=b.free_order, max_batch=2 * sh.S,
+                         partition_size=32)
+    orc = oracle.Allocator(b.num_blocks, sh.bs, b.free_order)
+    kc, vc = b.k_pool.clone(), b.v_pool.clone()
+    for s in range(sh.S):
+        ss.add(s, int(b.lens[s]))
+        orc.seq_add(s)
+        assert orc.seq_append_slots(s, int(b.lens[s]))[0] == 0
+    g = torch.Generator().manual_seed(5)
+    attend = list(range(sh.S))
+    # a sampled continuation of a sequence whose last block is partly filled
+    # at step 2 shares all its blocks, so its first write copies that block
+    parent = next(s for s in range(sh.S) if (int(b.lens[s]) + 2) % sh.bs != 0)
+    for step in range(5):
+        if step == 2:
+            ss.fork(parent, 100)
+            orc.seq_fork(parent, 100)
+            attend = attend + [100]
+        n = len(attend)
+        q = synth.randn((n, sh.Hq, sh.D), g, torch.bfloat16, "cpu").pin_memory()
+        kn = synth.randn((n, sh.Hkv, sh.D), g, torch.bfloat16, "cpu").pin_memory()
+        vn = synth.randn((n, sh.Hkv, sh.D), g, torch.bfloat16, "cpu").pin_memory()
+        out = ss.step(q, kn, vn, attend).clone()
+        slots, pairs = [], []
+        for sid in attend:
+            st, sl, pr = orc.seq_append_slots(sid, 1)
+            assert st == 0
+            slots += sl
+            pairs += pr
+        if step == 2:
+            assert pairs, "the fork must copy the shared partial block"
+        oracle.block_copy(kc, vc, pairs)
+        oracle.kv_append(kc, vc, kn, vn, slots)
+        bt = np.full((n, b.max_blocks), -1, np.int32)
+        lens = np.zeros(n, np.int64)
+        for i, sid in enumerate(attend):
+            _, t, L = orc.seq_block_table(sid)
+            bt[i, :len(t)] = t
+            lens[i] = L
+        ref = oracle.paged_attention(q, kc, vc, bt, lens)
+        assert m.device_error() == 0
+        assert max_err(out, ref) <= TOL[out.dtype], step
+    assert torch.equal(k.cpu(), kc) and torch.equal(v.cpu(), vc)
+
+
+def test_back_to_back_uploads_keep_their_plans():
+    """Plans uploaded one after another without waiting (the staging buffers
+    alternate and wait for their previous copy) arrive intact."""
+    import paged_kv_cache_405_b200 as m
+    sh = synth.shrink(synth.CONFIGS["llama7b"], S=6, Hq=4, Hkv=4, len_uniform=(1, 200), seed=12,
+                      reserve_tokens=64)
+    b = synth.make_batch(sh)
+    dev = torch.device("cuda")
+    ss = m.DecodeSession(b.k_pool.to(dev), b.v_pool.to(dev), sh.Hq, b.max_blocks, free_order=b.free_order,
+                         max_batch=sh.S)
+    for s in range(sh.S):
+        ss.add(s, int(b.lens[s]))
+    plans = [ss.plan(list(range(sh.S))) for _ in range(5)]
+    devs = [ss.upload(p) for p in plans]
+    torch.cuda.synchronize()
+    for p, d in zip(plans, devs):
+        assert np.array_equal(d.slot_mapping.cpu().numpy(), p.slot_mapping)
+        assert np.array_equal(d.lens.cpu().numpy(), p.lens)
+        assert np.array_equal(d.block_tables.cpu().numpy(), p.block_tables)
+        assert d.cow_pairs.shape == (0, 2) and d.n_cow == 0
