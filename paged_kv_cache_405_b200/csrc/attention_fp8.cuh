@@ -67,7 +67,8 @@ __device__ __forceinline__ void zero_tail_rows(uint8_t* vt, int valid, int lane)
     __syncwarp();
 }
 
-template <int D, int WARPS, int STAGES, typename To>
+// HI: more than 8 heads per group (rows 8..15 of the MMA are live).
+template <int D, int WARPS, int STAGES, typename To, bool HI>
 __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_fp8_kernel(const AttnParams p,
                                                                        const __grid_constant__ CUtensorMap tmK,
                                                                        const __grid_constant__ CUtensorMap tmV) {
@@ -196,7 +197,7 @@ __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_fp8_kernel(const Att
             }
         }
         uint32_t pa[4];
-        mma_softmax(acc, sacc, tig, valid, valid, p.scale_log2, pa);
+        mma_softmax<__half, D, HI>(acc, sacc, tig, valid, valid, p.scale_log2, p.scale_log2, pa);
 
         // O += P V
 #pragma unroll

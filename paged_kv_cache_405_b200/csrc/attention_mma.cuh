@@ -95,42 +95,51 @@ struct MmaAcc {
 // Online-softmax step for one 16 x 16 score tile (log2 domain).  sacc holds
 // the raw scores, element e of n-tile nt being token nt*8 + 2*tig + (e & 1) of
 // row gid (e < 2) or gid + 8 (e >= 2); row gid sees the first seen_lo tokens,
-// row gid + 8 the first seen_hi.  Updates the running max and sum, rescales
+// row gid + 8 the first seen_hi; scale_lo / scale_hi turn the raw scores of
+// the two rows into the log2 domain.  Updates the running max and sum, rescales
 // the output accumulators and returns the probabilities packed as the A
-// fragments of the P V product.
-template <typename T, int D>
+// fragments of the P V product.  HI = false: rows 8..15 are padding (at most
+// 8 live rows), so their state is left alone and their probabilities are 0.
+template <typename T, int D, bool HI = true>
 __device__ __forceinline__ void mma_softmax(MmaAcc<T, D>& acc, float (&sacc)[2][4], int tig, int seen_lo,
-                                            int seen_hi, float scale_log2, uint32_t (&pa)[4]) {
+                                            int seen_hi, float scale_lo, float scale_hi, uint32_t (&pa)[4]) {
     constexpr int NT_O = D / 8;
-    float mx_lo = -INFINITY, mx_hi = -INFINITY;
+    constexpr int NE = HI ? 4 : 2;  // accumulator elements of live rows
+    if (__all_sync(0xffffffffu, seen_lo >= kTileTok && (!HI || seen_hi >= kTileTok))) {
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+        for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int tok = nt * 8 + 2 * tig + (e & 1);
-            const float x = tok < (e < 2 ? seen_lo : seen_hi) ? sacc[nt][e] * scale_log2 : -INFINITY;
-            sacc[nt][e] = x;
-            if (e < 2) mx_lo = fmaxf(mx_lo, x);
-            else mx_hi = fmaxf(mx_hi, x);
+            for (int e = 0; e < NE; ++e) sacc[nt][e] *= e < 2 ? scale_lo : scale_hi;
+    } else {  // a partial tile or a causal limit inside it
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+            for (int e = 0; e < NE; ++e) {
+                const int tok = nt * 8 + 2 * tig + (e & 1);
+                sacc[nt][e] = tok < (e < 2 ? seen_lo : seen_hi) ? sacc[nt][e] * (e < 2 ? scale_lo : scale_hi)
+                                                                : -INFINITY;
+            }
         }
     }
+    float mx_lo = fmaxf(fmaxf(sacc[0][0], sacc[0][1]), fmaxf(sacc[1][0], sacc[1][1]));
+    float mx_hi = HI ? fmaxf(fmaxf(sacc[0][2], sacc[0][3]), fmaxf(sacc[1][2], sacc[1][3])) : 0.f;
 #pragma unroll
     for (int off = 1; off < 4; off <<= 1) {
         mx_lo = fmaxf(mx_lo, __shfl_xor_sync(0xffffffffu, mx_lo, off));
-        mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, off));
+        if (HI) mx_hi = fmaxf(mx_hi, __shfl_xor_sync(0xffffffffu, mx_hi, off));
     }
-    const float mn_lo = fmaxf(acc.m_lo, mx_lo), mn_hi = fmaxf(acc.m_hi, mx_hi);
+    const float mn_lo = fmaxf(acc.m_lo, mx_lo), mn_hi = HI ? fmaxf(acc.m_hi, mx_hi) : 0.f;
     // A row that has seen no token yet keeps m = -inf; exponentiate against 0
     // then, so that no -inf - -inf appears.
     const float b_lo = mn_lo == -INFINITY ? 0.f : mn_lo, b_hi = mn_hi == -INFINITY ? 0.f : mn_hi;
-    const float a_lo = ex2(acc.m_lo - b_lo), a_hi = ex2(acc.m_hi - b_hi);
+    const float a_lo = ex2(acc.m_lo - b_lo), a_hi = HI ? ex2(acc.m_hi - b_hi) : 1.f;
     acc.m_lo = mn_lo;
-    acc.m_hi = mn_hi;
+    if (HI) acc.m_hi = mn_hi;
     float ps_lo = 0.f, ps_hi = 0.f;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
+        for (int e = 0; e < NE; ++e) {
             const float pr = ex2(sacc[nt][e] - (e < 2 ? b_lo : b_hi));
             sacc[nt][e] = pr;
             if (e < 2) ps_lo += pr;
@@ -138,7 +147,7 @@ __device__ __forceinline__ void mma_softmax(MmaAcc<T, D>& acc, float (&sacc)[2][
         }
     }
     acc.l_lo = acc.l_lo * a_lo + ps_lo;
-    acc.l_hi = acc.l_hi * a_hi + ps_hi;
+    if (HI) acc.l_hi = acc.l_hi * a_hi + ps_hi;
     // Once the running maxima settle, every factor is exactly 1 and the
     // multiplications change nothing: skip them when that holds warp-wide.
     if (!__all_sync(0xffffffffu, a_lo == 1.f && a_hi == 1.f)) {
@@ -146,14 +155,16 @@ __device__ __forceinline__ void mma_softmax(MmaAcc<T, D>& acc, float (&sacc)[2][
         for (int j = 0; j < NT_O; ++j) {
             acc.o[j][0] *= a_lo;
             acc.o[j][1] *= a_lo;
-            acc.o[j][2] *= a_hi;
-            acc.o[j][3] *= a_hi;
+            if (HI) {
+                acc.o[j][2] *= a_hi;
+                acc.o[j][3] *= a_hi;
+            }
         }
     }
     pa[0] = Elt<T>::pack2(sacc[0][0], sacc[0][1]);
-    pa[1] = Elt<T>::pack2(sacc[0][2], sacc[0][3]);
+    pa[1] = HI ? Elt<T>::pack2(sacc[0][2], sacc[0][3]) : 0u;
     pa[2] = Elt<T>::pack2(sacc[1][0], sacc[1][1]);
-    pa[3] = Elt<T>::pack2(sacc[1][2], sacc[1][3]);
+    pa[3] = HI ? Elt<T>::pack2(sacc[1][2], sacc[1][3]) : 0u;
 }
 
 // Per-lane wait for stage st of tile i; on a timeout anywhere in the warp,
@@ -236,7 +247,7 @@ __device__ __forceinline__ bool mma_attend(const AttnParams& p, const CUtensorMa
             mma_16816<T>(sacc[1], acc.qa[kk], b2, b3);
         }
         uint32_t pa[4];
-        mma_softmax(acc, sacc, tig, seen_lo, seen_hi, p.scale_log2, pa);
+        mma_softmax(acc, sacc, tig, seen_lo, seen_hi, p.scale_log2, p.scale_log2, pa);
 
         // Rows past the context may hold anything (even NaN): zero them in V so
         // that 0-weights cannot turn into NaN inside the MMA.

@@ -70,8 +70,10 @@ class DevicePlan:
 class DecodeSession:
     def __init__(self, k_pool: torch.Tensor, v_pool: torch.Tensor, num_q_heads: int, max_blocks_per_seq: int,
                  free_order=None, partition_size: int = 0, max_batch: int = 0, share_prefixes: bool = True,
-                 min_group_size: int = 4, kv_scales=None):
-        """Pools of a 16-bit/fp32 type, or uint8 FP8 E4M3 codes with kv_scales = (k_scale, v_scale)."""
+                 min_group_size: int = 4, kv_scales=None, prefix_caching: bool = False):
+        """Pools of a 16-bit/fp32 type, or uint8 FP8 E4M3 codes with kv_scales = (k_scale, v_scale).
+        prefix_caching: full prompt blocks registered by ``add_prompt`` are
+        reused by later prompts with the same leading tokens."""
         self.k_pool, self.v_pool = k_pool, v_pool
         self.fp8 = k_pool.dtype == torch.uint8
         if self.fp8 and kv_scales is None:
@@ -81,7 +83,7 @@ class DecodeSession:
         self.num_q_heads = num_q_heads
         self.max_blocks = max_blocks_per_seq
         self.partition_size = partition_size
-        self.alloc = B.BlockAllocator(self.num_blocks, self.block_size, free_order)
+        self.alloc = B.BlockAllocator(self.num_blocks, self.block_size, free_order, prefix_caching=prefix_caching)
         self.device = k_pool.device
         # Runs of sequences sharing leading blocks go through the shared-prefix
         # pass (16-bit pools only: it runs on tensor cores).
@@ -109,6 +111,21 @@ class DecodeSession:
             assert not cow
             return slots
         return []
+
+    def add_prompt(self, sid: int, tokens: Sequence[int]):
+        """Register a sequence by its prompt token ids (automatic prefix
+        caching): the longest run of cached full blocks matching the prompt's
+        leading blocks is mapped into its table as is (their K/V are already in
+        the pools), the remaining tokens get fresh slots.  Returns
+        (n_cached, slots): the number of reused tokens and the int64 slots of
+        the others, where the caller's ``kv_append`` writes their K/V."""
+        st, n_cached, slots = self.alloc.seq_add_with_prompt(sid, tokens)
+        self._ok(st)
+        return n_cached, np.asarray(slots, dtype=np.int64)
+
+    def cache_stats(self) -> dict:
+        """Prefix-cache counters (lookups, hits, cached / evictable blocks, evictions)."""
+        return self.alloc.cache_stats()
 
     def fork(self, parent: int, child: int):
         self._ok(self.alloc.seq_fork(parent, child))

@@ -93,6 +93,29 @@ def test_decode_fp8_empty_and_one_token_contexts(Hq, Hkv):
     assert max_err(out, ref) <= TOL[out.dtype]
 
 
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 4)])
+def test_decode_fp8_query_magnitudes(Hq, Hkv):
+    """Query rows spanning many orders of magnitude (down into the FP16
+    subnormal range the query is rounded to), a zero head and an all-zero
+    sequence."""
+    import paged_kv_cache_405_b200 as pkv
+    sh = synth.shrink(synth.CONFIGS["llama7b"], S=6, Hq=Hq, Hkv=Hkv, len_uniform=(1, 400), seed=8)
+    b = synth.make_batch(sh)
+    q = b.q.float().clone()
+    for s, f in enumerate([1e-4, 3e-2, 1.0, 2.5, 6.0, 0.0]):
+        q[s] *= f
+    q[2, 0] = 0.0                       # one zero head inside an otherwise ordinary sequence
+    q = q.to(b.q.dtype)
+    ks, vs = 1 / 16, 1 / 4
+    kc, vc = fp8_pools(b, 4, ks, vs)
+    ref = oracle.paged_attention_kv(q, kc, vc, ks, vs, b.block_tables, b.lens, threads=oracle.max_threads())
+    out = torch.full_like(q, float("nan"), device="cuda")
+    pkv.paged_attention_decode_fp8(out, q.cuda(), kc.cuda(), vc.cuda(), torch.from_numpy(b.block_tables).cuda(),
+                                   torch.from_numpy(b.lens.astype(np.int32)).cuda(), ks, vs)
+    assert pkv.device_error() == 0
+    assert max_err(out, ref) <= TOL[out.dtype]
+
+
 def test_fp8_decode_step_end_to_end():
     """Quantized append of one new token per sequence, then attention over
     L+1 tokens, against the oracle's quantizer and attention."""
