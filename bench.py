@@ -82,7 +82,9 @@ def attention_bytes(bt: np.ndarray, lens: np.ndarray, Hq: int, Hkv: int, D: int,
     nparts = -(-sh // P) + -(-(lens - sh) // P)
     merged = (nparts > 1) | (sh > 0)
     ws = int((2 * nparts * Hq * (D + 2) * 4)[merged].sum())
-    return dict(kv=kv, logical_kv=logical, total=kv + qo + tables + ws, ws=ws)
+    # KV memory utilisation: tokens held / slots of the physical blocks in use
+    util = tok / max(1, int((best > 0).sum()) * bs)
+    return dict(kv=kv, logical_kv=logical, total=kv + qo + tables + ws, ws=ws, kv_util=util)
 
 
 def append_bytes(T, Hkv, D, elt):
@@ -256,6 +258,9 @@ def recorded_traffic(config):
         if len(f) >= 3 and not line.startswith("#") and f[0] == config and f[1] == src:
             return float(f[2])
     return None
+
+
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e nominal, for context beside the measured copy bandwidth
 
 
 def measured_hbm_peak():
@@ -480,9 +485,11 @@ def run_ours(args, world, rank, local):
                        if not shape.chunk and plans[W].group_shared is not None else 0},
             "pct_of_peak": round(100 * value / peak, 1),
             "seq_steps_per_s": round(seq_steps, 1),
+            "kv_utilisation": round(float(np.mean([a["kv_util"] for a in attn_bytes[W:]])), 4),
             "attention_us": round(a_s * 1e6, 2),
             "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
+                         "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
                          "kernel": "paged_attention_decode (attention + split-K reduce)",
                          "algorithmic_bytes": round(a_bytes)},
             "e2e": e2e,

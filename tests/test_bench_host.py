@@ -49,6 +49,8 @@ def test_attention_bytes_counts_shared_blocks_once():
     # blocks 5, 6 once (32 tokens) + block 1 (8 tokens) + block 2 (3 tokens)
     assert a["kv"] == 2 * 8 * 2 * (32 + 8 + 3)
     assert a["logical_kv"] == 2 * 8 * 2 * 75 and a["ws"] == 0
+    # KV memory utilisation: 43 tokens held in 4 physical blocks of 16 slots
+    assert a["kv_util"] == 43 / 64
 
 
 def _ranks(rank, world, port, q):
