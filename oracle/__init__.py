@@ -19,6 +19,7 @@ from __future__ import annotations
 
 import ctypes
 import math
+import os
 
 import numpy as np
 import torch
@@ -33,7 +34,9 @@ _lib = None
 def _load():
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(_build.build())
+        # ORACLE_LIBRARY may name another build of oracle.c (the tests build
+        # copies with planted mistakes to show that the pins catch them).
+        lib = ctypes.CDLL(os.environ.get("ORACLE_LIBRARY") or _build.build())
         lib.oracle_paged_attention.restype = ctypes.c_int
         lib.oracle_paged_attention.argtypes = [
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,

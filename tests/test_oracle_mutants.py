@@ -1,0 +1,98 @@
+"""The pins catch plausible mistakes: each case copies the oracle's C source,
+plants one mistake (a dropped term, a wrong sign or index, a swapped
+operand, a wrong widening), builds it and runs the pin tests against that
+build, which must fail; the allocator cases do the same to a copy of the
+oracle allocator and run the brute-force payload model on it.  (The
+mistakes live only in these temporary copies.)"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+ROOT = os.path.dirname(HERE)
+SRC = os.path.join(ROOT, "oracle", "oracle.c")
+
+# name: (text in oracle.c, replacement)
+MUTANTS = {
+    "softmax scale dropped": ("x[t] = scale * acc;", "x[t] = acc;"),
+    "kv head of a query head": ("        int g = h / G;\n        int64_t L = context_lens[s];\n        if (L <= 0) continue;\n"
+                                "        if (L > (int64_t)max_blocks * block_size) { status = -1; continue; }\n"
+                                "        const int32_t *bt = block_tables + (int64_t)s * max_blocks;\n        int bad = 0;",
+                                "        int g = h % Hkv;\n        int64_t L = context_lens[s];\n        if (L <= 0) continue;\n"
+                                "        if (L > (int64_t)max_blocks * block_size) { status = -1; continue; }\n"
+                                "        const int32_t *bt = block_tables + (int64_t)s * max_blocks;\n        int bad = 0;"),
+    "exponent sign": ("double w = exp(x[t] - mx);", "double w = exp(mx - x[t]);"),
+    "slot offset": ("return (int64_t)bt[t / block_size] * block_size + t % block_size;",
+                    "return (int64_t)bt[t / block_size] * block_size + (t + 1) % block_size;"),
+    "K read for V": ("o[d] += w * pool_value(v_pool, vbase + d, kv_dtype, v_scale);",
+                     "o[d] += w * pool_value(k_pool, vbase + d, kv_dtype, v_scale);"),
+    "query elements reversed": ("acc += widen(q, qbase + d, q_dtype) * pool_value(k_pool, kbase + d, kv_dtype, k_scale);",
+                                "acc += widen(q, qbase + (D - 1 - d), q_dtype) * pool_value(k_pool, kbase + d, kv_dtype, k_scale);"),
+    "no normalisation": ("        for (int d = 0; d < D; ++d) o[d] /= den;\n        free(x);\n    }\n    return status;\n}\n\n/*\n * Causal",
+                         "        free(x);\n    }\n    return status;\n}\n\n/*\n * Causal"),
+    "bf16 widening": ("uint32_t u = (uint32_t)h << 16;", "uint32_t u = (uint32_t)h << 15;"),
+    "f16 widening": ("else v = ldexp((double)(m | 1024), e - 25);", "else v = ldexp((double)(m | 1024), e - 24);"),
+    "e4m3 exponent bias": ("else v = ldexp((double)(8 + m), e - 10);", "else v = ldexp((double)(8 + m), e - 11);"),
+    "causal limit": ("int64_t upto = L - n + (t - query_start[s]) + 1;", "int64_t upto = L - n + (t - query_start[s]);"),
+}
+
+
+@pytest.mark.parametrize("name", list(MUTANTS))
+def test_pins_catch_planted_mistake(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, "the planted mistake must replace exactly one place"
+    mutant = tmp_path / "oracle_mutant.c"
+    mutant.write_text(src.replace(old, new))
+    lib = tmp_path / "liboracle_mutant.so"
+    subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-fopenmp", "-shared", "-fPIC", "-std=c11", "-o",
+                           str(lib), str(mutant), "-lm"])
+    env = dict(os.environ, ORACLE_LIBRARY=str(lib))
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(HERE, "test_oracle_pins.py"), "-x", "-q",
+                        "-p", "no:cacheprovider"], cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode != 0, "no pin caught: %s" % name
+    assert "failed" in r.stdout, r.stdout[-2000:]
+
+
+# Planted mistakes in the Python allocator (class Allocator, the first class
+# of oracle/allocator.py): (text, replacement, which occurrence).
+ALLOC_MUTANTS = {
+    "copy-on-write skipped": ("elif self.ref[bt[j]] > 1:", "elif False:", 0),
+    "fork leaves refcounts": ("            self.ref[b] += 1\n        self.seqs[child]", "            pass\n        self.seqs[child]", 0),
+    "freed blocks lost": ("self.free.append(b)", "pass", 0),
+    "fresh block unreferenced": ("                self.ref[b] = 1\n                bt.append(b)",
+                                 "                self.ref[b] = 0\n                bt.append(b)", 0),
+    "block index of a token": ("j = t // bs", "j = (t + 1) // bs", 0),
+}
+
+
+def _mutant_allocator(old, new, which):
+    import types
+    src = open(os.path.join(ROOT, "oracle", "allocator.py")).read()
+    at = -1
+    for _ in range(which + 1):
+        at = src.index(old, at + 1)
+    src = src[:at] + new + src[at + len(old):]
+    mod = types.ModuleType("oracle_allocator_mutant")
+    exec(compile(src, "oracle_allocator_mutant", "exec"), mod.__dict__)
+    return mod.Allocator
+
+
+@pytest.mark.parametrize("name", list(ALLOC_MUTANTS))
+def test_allocator_pins_catch_planted_mistake(name):
+    import numpy as np
+    import synth
+    from test_oracle_pins import run_ops
+    Broken = _mutant_allocator(*ALLOC_MUTANTS[name])
+    caught = False
+    for seed in range(3000):
+        nb = 4 + seed % 3
+        a = Broken(nb, 2, list(np.random.default_rng(seed).permutation(nb)))
+        try:
+            run_ops(a, synth.random_ops(seed, 8, max_seqs=4, max_append=4), 2)
+        except (AssertionError, IndexError, KeyError, ValueError):
+            caught = True
+            break
+    assert caught, "no pin caught: %s" % name
