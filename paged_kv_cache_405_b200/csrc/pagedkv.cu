@@ -274,7 +274,9 @@ template <typename T, int D>
 static cudaError_t launch_reduce(const pkv::ReduceParams& r, cudaStream_t st) {
     const unsigned rows = (unsigned)((r.query_start ? r.T : r.S) * r.Hq);
     if (r.maxP > 32) return launch_k(pkv::splitk_reduce_kernel<T, D, 8, 1>, dim3(rows), dim3(256), 0, st, r);
-    return launch_k(pkv::splitk_reduce_kernel<T, D, 1, 8>, dim3((rows + 7) / 8), dim3(256), 0, st, r);
+    const dim3 grid((rows + 7) / 8), block(256);
+    if (r.maxP <= 8) return launch_k(pkv::splitk_reduce_warp_kernel<T, D, 8, 8>, grid, block, 0, st, r);
+    return launch_k(pkv::splitk_reduce_warp_kernel<T, D, 8, 0>, grid, block, 0, st, r);
 }
 
 template <typename T>

@@ -26,23 +26,25 @@ struct ReduceParams {
 };
 
 // Partials to merge for one output row (0 = the attention kernel wrote it).
-__device__ __forceinline__ int reduce_count(const ReduceParams& p, int row) {
+// qs / gf: query_start / group_first, from global memory or a shared copy.
+__device__ __forceinline__ int reduce_count(const ReduceParams& p, int row, const int32_t* qs,
+                                            const int32_t* gf) {
     const int h_rows = p.Hq;
     if (p.query_start) {  // causal chunk: row = t * Hq + h
         const int t = row / h_rows;
-        if (t < p.query_start[0] || t >= p.query_start[p.S]) return 0;
+        if (t < qs[0] || t >= qs[p.S]) return 0;
         int lo = 0, hi = p.S;
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (p.query_start[mid] <= t) lo = mid;
+            if (qs[mid] <= t) lo = mid;
             else hi = mid;
         }
         int L = p.context_lens[lo];
         L = L < 0 ? 0 : (L > p.max_len ? p.max_len : L);
-        const int n = p.query_start[lo + 1] - p.query_start[lo];
+        const int n = qs[lo + 1] - qs[lo];
         if (n > L) return 0;  // reported by the attention kernel
         if ((L + p.P - 1) / p.P <= 1) return 0;
-        const int pos = L - n + (t - p.query_start[lo]);
+        const int pos = L - n + (t - qs[lo]);
         return pos / p.P + 1;
     }
     const int s = row / h_rows;
@@ -52,11 +54,11 @@ __device__ __forceinline__ int reduce_count(const ReduceParams& p, int row) {
     // A member of a valid shared-prefix group has ceil(shared/P) prefix
     // partials followed by its own ones (same rule as the attention kernels).
     int shared = 0;
-    if (p.num_groups > 0 && s >= p.group_first[0] && s < p.group_first[p.num_groups]) {
+    if (p.num_groups > 0 && s >= gf[0] && s < gf[p.num_groups]) {
         int lo = 0, hi = p.num_groups;
         while (hi - lo > 1) {
             const int mid = (lo + hi) >> 1;
-            if (p.group_first[mid] <= s) lo = mid;
+            if (gf[mid] <= s) lo = mid;
             else hi = mid;
         }
         const int sh = p.group_shared[lo];
@@ -95,7 +97,7 @@ __global__ void __launch_bounds__(W * ROWS * 32) splitk_reduce_kernel(const Redu
     float (&s_max)[W] = s_max_all[sub];
     const int nrows = p.query_start ? p.T * p.Hq : p.S * p.Hq;
     if (row >= nrows) return;  // whole rows return together (W warps of a row)
-    const int nP = reduce_count(p, row);
+    const int nP = reduce_count(p, row, p.query_start, p.group_first);
     if (nP == 0) return;
     const int64_t base = (int64_t)row * p.maxP;
     const float* ml = p.ws_ml + base * 2;
@@ -173,6 +175,106 @@ __global__ void __launch_bounds__(W * ROWS * 32) splitk_reduce_kernel(const Redu
         for (int w = 1; w < W; ++w) a += s_acc[w][lane * kPerLane + k];
         dst[k] = static_cast<T>(a * inv);
     }
+}
+
+// Few partitions (maxP <= 32): one warp per row, ROWS rows per CTA.  The
+// loads that do not depend on the row's partition count go out first -- the
+// (m, l) pair of every slot (lane i holds slot i) and, with SPEC >= maxP, the
+// partial outputs of every slot -- together with the context length, so a
+// row costs one round trip to memory (two without SPEC).  A chunk call's
+// query_start, or a shared-prefix call's group_first, is searched in a
+// shared-memory copy when it fits.  Slots past the row's count are never
+// used (selected out, so stale values cannot leak in); the outputs are
+// summed in slot order, so the result does not depend on timing.
+constexpr int kReduceIdxMax = 4096;
+
+template <typename T, int D, int ROWS, int SPEC>
+__global__ void __launch_bounds__(ROWS * 32) splitk_reduce_warp_kernel(const ReduceParams p) {
+    constexpr int KPL = D / 32;  // 2 or 4 floats per lane
+    __shared__ int32_t s_idx[kReduceIdxMax];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * ROWS + warp;
+    const int32_t* qs = p.query_start;
+    const int32_t* gf = p.group_first;
+    const int32_t* src = qs ? qs : (p.num_groups > 0 ? gf : nullptr);
+    const int n_idx = qs ? p.S + 1 : p.num_groups + 1;
+    if (src != nullptr && n_idx <= kReduceIdxMax) {  // uniform over the CTA
+        for (int i = threadIdx.x; i < n_idx; i += ROWS * 32) s_idx[i] = src[i];
+        __syncthreads();
+        if (qs) qs = s_idx;
+        else gf = s_idx;
+    }
+    const int nrows = p.query_start ? p.T * p.Hq : p.S * p.Hq;
+    if (row >= nrows) return;
+    const int64_t base = (int64_t)row * p.maxP;
+    const float* o = p.ws_o + base * D + lane * KPL;
+    const float2 mlv = lane < p.maxP ? *reinterpret_cast<const float2*>(p.ws_ml + (base + lane) * 2)
+                                     : make_float2(-INFINITY, 0.f);
+    float v[SPEC > 0 ? SPEC : 1][KPL];
+#pragma unroll
+    for (int i = 0; i < SPEC; ++i) {
+        if (i < p.maxP) {
+            if constexpr (KPL == 4) {
+                const float4 x = *reinterpret_cast<const float4*>(o + (int64_t)i * D);
+                v[i][0] = x.x; v[i][1] = x.y; v[i][2] = x.z; v[i][3] = x.w;
+            } else {
+                const float2 x = *reinterpret_cast<const float2*>(o + (int64_t)i * D);
+                v[i][0] = x.x; v[i][1] = x.y;
+            }
+        }
+    }
+    const int nP = reduce_count(p, row, qs, gf);
+    if (nP == 0) return;
+
+    float M = lane < nP ? mlv.x : -INFINITY;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float w_lane = lane < nP ? ex2(mlv.x - M) : 0.f;
+    float den = w_lane * (lane < nP ? mlv.y : 0.f);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+
+    float acc[KPL];
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) acc[k] = 0.f;
+    if constexpr (SPEC > 0) {
+#pragma unroll
+        for (int i = 0; i < SPEC; ++i) {
+            const float w = __shfl_sync(0xffffffffu, w_lane, i);
+            if (i < nP) {
+#pragma unroll
+                for (int k = 0; k < KPL; ++k) acc[k] += w * v[i][k];
+            }
+        }
+    } else {
+        constexpr int U = 4;  // partitions per batch of loads
+        for (int i0 = 0; i0 < nP; i0 += U) {
+            float x[U][KPL];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int i = i0 + u < nP ? i0 + u : i0;  // past the count: reload a valid slot, unused
+                if constexpr (KPL == 4) {
+                    const float4 y = *reinterpret_cast<const float4*>(o + (int64_t)i * D);
+                    x[u][0] = y.x; x[u][1] = y.y; x[u][2] = y.z; x[u][3] = y.w;
+                } else {
+                    const float2 y = *reinterpret_cast<const float2*>(o + (int64_t)i * D);
+                    x[u][0] = y.x; x[u][1] = y.y;
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const float w = __shfl_sync(0xffffffffu, w_lane, (i0 + u) & 31);
+                if (i0 + u < nP) {
+#pragma unroll
+                    for (int k = 0; k < KPL; ++k) acc[k] += w * x[u][k];
+                }
+            }
+        }
+    }
+    const float inv = 1.f / den;
+    T* dst = reinterpret_cast<T*>(p.out) + (int64_t)row * D + lane * KPL;
+#pragma unroll
+    for (int k = 0; k < KPL; ++k) dst[k] = static_cast<T>(acc[k] * inv);
 }
 
 }  // namespace pkv
