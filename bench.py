@@ -304,6 +304,17 @@ def oracle_sample(batch, budget_s, threads):
     return bytes_done / secs / 1e9, seqs / secs, desc, secs
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (for the CPU-baseline record)."""
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 # ------------------------------------------------------------------- runners
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -497,11 +508,14 @@ def run_ours(args, world, rank, local):
             "clocks": clk,
         }
         if world == 1 and not args.no_cpu_baseline:
-            v, sps, desc, secs = oracle_sample(host_batch(shape, shape.seed + rank), args.cpu_seconds,
-                                               threads=os.cpu_count())
+            hb = host_batch(shape, shape.seed + rank)
+            v, sps, desc, secs = oracle_sample(hb, args.cpu_seconds, threads=os.cpu_count())
+            v1, sps1, _, secs1 = oracle_sample(hb, max(1.0, args.cpu_seconds / 4), threads=1)
             line["cpu_baseline"] = {"value": round(v, 3), "unit": "GB/s", "cores": os.cpu_count(),
                                     "kind": "oracle", "sample": desc, "seq_steps_per_s": round(sps, 3),
-                                    "seconds": round(secs, 1)}
+                                    "seconds": round(secs, 1), "cpu_model": cpu_model(),
+                                    "single_thread": {"value": round(v1, 3), "seq_steps_per_s": round(sps1, 3),
+                                                      "seconds": round(secs1, 1)}}
     return line
 
 

@@ -74,3 +74,10 @@ def test_rank_reductions_gloo():
     for p in ps:
         p.join(timeout=60)
     assert res == [(0, 2.0, 3.0), (1, 2.0, 3.0)]
+
+
+def test_cpu_baseline_sample_runs_on_one_thread():
+    b = synth.make_batch(synth.CONFIGS["tiny"])
+    v, sps, desc, secs = bench.oracle_sample(b, 0.05, threads=1)
+    assert v > 0 and sps > 0 and secs >= 0.05 and "1 threads" in desc
+    assert isinstance(bench.cpu_model(), str) and bench.cpu_model()
