@@ -5,16 +5,19 @@
  * `block_size` tokens drawn from one shared physical pool; a per-sequence block
  * table maps logical block j (tokens j*block_size .. (j+1)*block_size-1) to a
  * physical block.  Sources (web pages, cited by site, title and section):
- *   [E]  openeuler.csdn.net, PagedAttention explainer: 4.1 fixed-size blocks,
- *        4.2 block table (logical -> physical), 4.3 on-demand growth,
- *        6.1 shared prefix, 6.2 copy-on-write.
+ *   [E]  openeuler.csdn.net, PagedAttention explainer: 2.1-2.2 decode and the
+ *        KV cache, 4.1 fixed-size blocks, 4.2 block table (logical ->
+ *        physical), 4.3 on-demand growth, 6.1 shared prefix, 6.2
+ *        copy-on-write.
  *   [B]  agent.csdn.net, PagedAttention blog: 2.1 blocks of 16 tokens, only the
  *        last block partly filled; 2.2 copy-on-write for parallel samples and
- *        beams; 3.1 block-manager sketch (allocate a free block on demand).
+ *        beams; 3.1 block-manager sketch (allocate a free block on demand);
+ *        4.2 bandwidth decides the fastest precision.
  *   [T]  aiknowledge.cn, "2.2 PagedAttention 与 KV Cache 分页管理": 2.2.2 free
  *        pool, blocks freed on finish or preemption; 2.2.3 worked example
  *        (35 tokens -> physical blocks 7, 3, 9) and prefix sharing; 2.2.4 a
- *        kernel fused over non-contiguous blocks; 2.2.13 pool monitoring.
+ *        kernel fused over non-contiguous blocks; 2.2.8 byte-identical
+ *        prefixes reused; 2.2.13 pool monitoring.
  *
  * Conventions for every call
  *   - Device pointers are caller-owned device memory, 16-byte aligned; the
@@ -36,7 +39,8 @@
  *     pool[num_blocks][num_kv_heads][block_size][head_dim], row-major,
  * so the `block_size x head_dim` tile of one (block, kv head) is contiguous.
  * Element types: PKV_F32, PKV_BF16, PKV_F16; q, new K/V, pools and the output
- * of one call share one type.
+ * of one call share one type, except in the _fp8 calls (FP8 E4M3 pools with
+ * 16-bit q and output).
  */
 #ifndef PAGEDKV_H
 #define PAGEDKV_H
