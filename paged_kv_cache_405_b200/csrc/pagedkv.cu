@@ -270,6 +270,38 @@ static cudaError_t launch_head_fp8(const pkv::AttnParams& p, dim3 grid, const CU
     return launch_k(k, grid, dim3(kMmaWarps * 32), C::kSmemBytes, st, p, mk, mv);
 }
 
+// Side stream for the shared-prefix pass, which runs concurrently with the
+// same call's decode kernel: both only read the pools and write disjoint
+// partial slots, and the reduce waits for both.  One stream and a fork / join
+// event pair per device, created on first use (no device memory); the mutex
+// keeps one call's fork ... join sequence from interleaving with another
+// thread's.  Without them the pass runs on the caller's stream first.
+struct SideStream {
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    bool tried = false, ok = false;
+};
+constexpr int kMaxSideDevices = 64;
+static SideStream g_side[kMaxSideDevices];
+static std::mutex g_side_mu;
+
+static SideStream* side_stream() {  // the caller holds g_side_mu
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxSideDevices) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    SideStream& s = g_side[dev];
+    if (!s.tried) {
+        s.tried = true;
+        s.ok = cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking) == cudaSuccess &&
+               cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) == cudaSuccess &&
+               cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) == cudaSuccess;
+        if (!s.ok) cudaGetLastError();  // fall back to the caller's stream
+    }
+    return s.ok ? &s : nullptr;
+}
+
 template <typename T, int D>
 static cudaError_t launch_reduce(const pkv::ReduceParams& r, cudaStream_t st) {
     const unsigned rows = (unsigned)((r.query_start ? r.T : r.S) * r.Hq);
@@ -279,6 +311,20 @@ static cudaError_t launch_reduce(const pkv::ReduceParams& r, cudaStream_t st) {
     return launch_k(pkv::splitk_reduce_warp_kernel<T, D, 8, 0>, grid, block, 0, st, r);
 }
 
+// The per-sequence decode kernel of a call (no prefix pass, no reduce).
+template <typename T>
+static cudaError_t decode_pass(const pkv::AttnParams& p, int D, int nparts, bool use_mma, const CUtensorMap* mk,
+                               const CUtensorMap* mv, cudaStream_t st) {
+    if constexpr (!std::is_same<T, float>::value) {
+        if (use_mma) {
+            dim3 grid((p.Hkv + kMmaWarps - 1) / kMmaWarps, nparts, p.S);
+            return D == 64 ? launch_mma<T, 64>(p, grid, *mk, *mv, st) : launch_mma<T, 128>(p, grid, *mk, *mv, st);
+        }
+    }
+    dim3 grid((p.Hq + kSimtWarps - 1) / kSimtWarps, nparts, p.S);
+    return D == 64 ? launch_simt<T, 64>(p, grid, st) : launch_simt<T, 128>(p, grid, st);
+}
+
 template <typename T>
 static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int nparts, int npre, bool use_mma,
                                       bool shared_mode, const CUtensorMap* mk, const CUtensorMap* mv,
@@ -286,21 +332,27 @@ static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int npart
     cudaError_t e = cudaSuccess;
     if constexpr (std::is_same<T, float>::value) {
         if (use_mma || shared_mode) return cudaErrorInvalidValue;
+        e = decode_pass<T>(p, D, nparts, use_mma, mk, mv, st);
     } else {
         if (shared_mode && p.num_groups > 0 && npre > 0) {
             const int tiles = (p.max_group_size * p.G + 15) / 16;
             dim3 grid(tiles, npre, p.num_groups * p.Hkv);
-            e = D == 64 ? launch_prefix<T, 64>(p, grid, *mk, *mv, st) : launch_prefix<T, 128>(p, grid, *mk, *mv, st);
-            if (e != cudaSuccess) return e;
+            std::unique_lock<std::mutex> lk(g_side_mu);
+            SideStream* ss = side_stream();
+            cudaStream_t ps = st;
+            if (ss != nullptr && cudaEventRecord(ss->fork, st) == cudaSuccess &&
+                cudaStreamWaitEvent(ss->stream, ss->fork, 0) == cudaSuccess)
+                ps = ss->stream;
+            e = D == 64 ? launch_prefix<T, 64>(p, grid, *mk, *mv, ps) : launch_prefix<T, 128>(p, grid, *mk, *mv, ps);
+            if (e == cudaSuccess) e = decode_pass<T>(p, D, nparts, use_mma, mk, mv, st);
+            if (ps != st) {  // join, whatever happened above
+                const cudaError_t j = cudaEventRecord(ss->join, ps);
+                const cudaError_t w = j == cudaSuccess ? cudaStreamWaitEvent(st, ss->join, 0) : j;
+                if (e == cudaSuccess) e = w;
+            }
+        } else {
+            e = decode_pass<T>(p, D, nparts, use_mma, mk, mv, st);
         }
-        if (use_mma) {
-            dim3 grid((p.Hkv + kMmaWarps - 1) / kMmaWarps, nparts, p.S);
-            e = D == 64 ? launch_mma<T, 64>(p, grid, *mk, *mv, st) : launch_mma<T, 128>(p, grid, *mk, *mv, st);
-        }
-    }
-    if (!use_mma) {
-        dim3 grid((p.Hq + kSimtWarps - 1) / kSimtWarps, nparts, p.S);
-        e = D == 64 ? launch_simt<T, 64>(p, grid, st) : launch_simt<T, 128>(p, grid, st);
     }
     if (e != cudaSuccess || p.maxP <= 1) return e;
     pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
