@@ -46,7 +46,7 @@ class PagedKVError(RuntimeError):
 
 def _load():
     if not os.path.exists(LIB_PATH):
-        raise ImportError("libpagedkv.so is not built; run `python -m paged_kv_cache_405_b200.build` "
+        raise ImportError("libpagedkv.so is not built; run `python paged_kv_cache_405_b200/build.py` "
                           "or __graft_entry__.build()")
     lib = ctypes.CDLL(LIB_PATH)
     c_int, c_i64, c_vp, c_sz = ctypes.c_int, ctypes.c_int64, ctypes.c_void_p, ctypes.c_size_t

@@ -96,3 +96,17 @@ def test_package_exposes_every_binding_call():
               if not n.startswith("_") and f.__module__ == binding.__name__]
     missing = [n for n in public if not hasattr(pkv, n)]
     assert not missing
+
+
+def test_build_runs_from_a_checkout_without_the_library(tmp_path):
+    """build() must not import the package (whose __init__ loads the library)
+    before it has compiled it: a fresh checkout has no libpagedkv.so."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import sys, __graft_entry__ as g\n"
+            "m = g._load_by_path('_b', g.os.path.join(g.ROOT, 'paged_kv_cache_405_b200', 'build.py'))\n"
+            "assert callable(m.build)\n"
+            "assert 'paged_kv_cache_405_b200' not in sys.modules\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
