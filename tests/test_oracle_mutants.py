@@ -2,8 +2,10 @@
 plants one mistake (a dropped term, a wrong sign or index, a swapped
 operand, a wrong widening), builds it and runs the pin tests against that
 build, which must fail; the allocator cases do the same to a copy of the
-oracle allocator and run the brute-force payload model on it.  (The
-mistakes live only in these temporary copies.)"""
+oracle allocator and run the brute-force payload model on it, the caching
+cases to a copy of the caching allocator under the prefix-cache pins, and
+the quantizer cases to a copy of the E4M3 quantizer under its pin against
+torch's cast.  (The mistakes live only in these temporary copies.)"""
 import os
 import subprocess
 import sys
@@ -68,7 +70,7 @@ ALLOC_MUTANTS = {
 }
 
 
-def _mutant_allocator(old, new, which):
+def _mutant_allocator_module(old, new, which):
     import types
     src = open(os.path.join(ROOT, "oracle", "allocator.py")).read()
     at = -1
@@ -77,7 +79,11 @@ def _mutant_allocator(old, new, which):
     src = src[:at] + new + src[at + len(old):]
     mod = types.ModuleType("oracle_allocator_mutant")
     exec(compile(src, "oracle_allocator_mutant", "exec"), mod.__dict__)
-    return mod.Allocator
+    return mod
+
+
+def _mutant_allocator(old, new, which):
+    return _mutant_allocator_module(old, new, which).Allocator
 
 
 @pytest.mark.parametrize("name", list(ALLOC_MUTANTS))
@@ -93,6 +99,76 @@ def test_allocator_pins_catch_planted_mistake(name):
         try:
             run_ops(a, synth.random_ops(seed, 8, max_seqs=4, max_append=4), 2)
         except (AssertionError, IndexError, KeyError, ValueError):
+            caught = True
+            break
+    assert caught, "no pin caught: %s" % name
+
+
+# Planted mistakes in the caching allocator (class CachingAllocator of
+# oracle/allocator.py), caught by the prefix-cache pins that do not involve
+# the product: the prefix payload model, the closed-form hit counts, the
+# eviction order and the all-or-nothing prompt registration.
+CACHE_MUTANTS = {
+    "evicts the newest released block": ("b = self.lru.pop(0)", "b = self.lru.pop()"),
+    "released cached block goes back to the free queue": ("if b in self.key_of:\n                self.lru.append(b)",
+                                                          "if False:\n                self.lru.append(b)"),
+    "block key without its parent": ("key = (parent, tuple(block_toks))", "key = (self.ROOT, tuple(block_toks))"),
+    "a hit takes no reference": ("            self.ref[b] += 1\n        n_cached", "            pass\n        n_cached"),
+    "lookup skips a missed block": ("            if b is None:\n                break",
+                                    "            if b is None:\n                continue"),
+    "partial blocks registered": ("if t % bs == bs - 1:", "if True:"),
+    "lookups counted in tokens": ("self.lookups += len(toks) // bs", "self.lookups += len(toks)"),
+    "chain restarts after the cached blocks": ("        self.chain[sid] = node\n        st, slots, _",
+                                               "        self.chain[sid] = self.ROOT\n        st, slots, _"),
+}
+CACHE_PINS = ["test_caching_oracle_payload_model", "test_hit_counts_closed_form",
+              "test_freed_cached_blocks_are_evicted_oldest_first", "test_prompt_that_does_not_fit_changes_nothing"]
+
+
+@pytest.mark.parametrize("name", list(CACHE_MUTANTS))
+def test_prefix_cache_pins_catch_planted_mistake(name, monkeypatch):
+    import test_prefix_cache as pins
+    old, new = CACHE_MUTANTS[name]
+    monkeypatch.setattr(pins, "CachingAllocator", _mutant_allocator_module(old, new, 0).CachingAllocator)
+    caught = []
+    for pin in CACHE_PINS:
+        try:
+            getattr(pins, pin)()
+        except (AssertionError, IndexError, KeyError, ValueError):
+            caught.append(pin)
+    assert caught, "no pin caught: %s" % name
+
+
+# Planted mistakes in the oracle's E4M3 quantizer, caught by the pin against
+# torch's float8_e4m3fn cast (exact ties included).
+QUANT_MUTANTS = {
+    "ties rounded away from zero": ("np.where(even_hi, hi, lo)", "hi"),
+    "ties rounded toward zero": ("np.where(even_hi, hi, lo)", "lo"),
+    "nearest taken the wrong way": ("dl < dh", "dl > dh"),
+    "scale multiplied instead of divided": ("inv = np.float32(1.0) / np.float32(scale)", "inv = np.float32(scale)"),
+    "sign dropped": ("code = np.where(np.signbit(y), code | 0x80, code).astype(np.uint8)",
+                     "code = code.astype(np.uint8)"),
+}
+
+
+@pytest.mark.parametrize("name", list(QUANT_MUTANTS))
+def test_quantizer_pins_catch_planted_mistake(name, monkeypatch):
+    import inspect
+    import textwrap
+
+    import oracle
+    import test_oracle_pins as pins
+    old, new = QUANT_MUTANTS[name]
+    src = textwrap.dedent(inspect.getsource(oracle.quantize_e4m3))
+    assert src.count(old) == 1, "the planted mistake must replace exactly one place"
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), "quantize_e4m3_mutant", "exec"), ns)
+    monkeypatch.setattr(oracle, "quantize_e4m3", ns["quantize_e4m3"])
+    caught = False
+    for scale in (1.0, 0.125, 0.37):
+        try:
+            pins.test_e4m3_quantize_matches_torch_cast_and_saturates(scale)
+        except AssertionError:
             caught = True
             break
     assert caught, "no pin caught: %s" % name

@@ -464,11 +464,23 @@ def test_e4m3_table_matches_torch_float8():
     assert np.array_equal(got[~np.isnan(got)], ref[~np.isnan(ref)])
 
 
+def e4m3_midpoints():
+    """Every point halfway between two adjacent non-negative E4M3 values (from
+    torch's decoding of the 256 codes), both signs: exact ties, which random
+    inputs essentially never hit, so that ties-to-even is pinned too."""
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    v = np.unique(ref[np.isfinite(ref) & (ref >= 0)])
+    mids = (v[:-1] + v[1:]) / 2
+    return torch.from_numpy(np.concatenate([mids, -mids])).float()
+
+
 @pytest.mark.parametrize("scale", [1.0, 0.125, 0.37])
 def test_e4m3_quantize_matches_torch_cast_and_saturates(scale):
     g = torch.Generator().manual_seed(3)
+    # times a power-of-two scale, each midpoint is still an exact tie after x * (1/scale)
     x = torch.cat([torch.randn(200000, generator=g) * 60, torch.tensor([0.0, -0.0, 1e-30, -1e-30, 447.9, 448.0,
-                                                                         449.0, 463.9, 1e6, -1e6])])
+                                                                         449.0, 463.9, 1e6, -1e6]),
+                   e4m3_midpoints() * scale])
     codes = oracle.quantize_e4m3(x, scale)
     y = (x.float() * (torch.tensor(1.0, dtype=torch.float32) / torch.tensor(scale, dtype=torch.float32)))
     inside = y.abs() < 448

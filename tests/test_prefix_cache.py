@@ -1,5 +1,7 @@
-"""Automatic prefix caching: the oracle's caching allocator pinned by a token
-payload model, and the product's allocator bit-exact against it."""
+"""Automatic prefix caching: the oracle's caching allocator pinned by a
+payload model in which every slot holds the whole prefix ending at its token
+(a cached block may only serve an identical prefix), and the product's
+allocator bit-exact against it."""
 import numpy as np
 import pytest
 
@@ -42,12 +44,15 @@ def apply(a, op):
 
 
 def check(a: CachingAllocator, model, data):
+    """data[slot] is the whole prefix ending at the token held there: a
+    token's K/V depends on every token before it, so a block may serve a
+    sequence only if it was written under the same prefix."""
     bs = a.block_size
     refs = [0] * a.num_blocks
     for sid, (bt, n) in a.seqs.items():
         assert len(bt) == -(-n // bs) and len(model[sid]) == n
-        for t in range(n):   # every sequence reads back its own tokens
-            assert data.get(bt[t // bs] * bs + t % bs) == model[sid][t]
+        for t in range(n):   # every sequence reads back its own tokens, each under its own prefix
+            assert data.get(bt[t // bs] * bs + t % bs) == tuple(model[sid][:t + 1])
         for b in bt:
             refs[b] += 1
     assert refs == a.ref
@@ -57,7 +62,7 @@ def check(a: CachingAllocator, model, data):
     assert not (set(a.free) & set(a.lru)) and not (set(a.free) & used)
     for key, b in a.cache.items():     # a cached block holds exactly its key's tokens
         assert a.key_of[b] == key
-        assert [data.get(b * bs + o) for o in range(bs)] == list(key[1])
+        assert [(data.get(b * bs + o) or (None,))[-1] for o in range(bs)] == list(key[1])
 
 
 def run(a, ops):
@@ -69,8 +74,8 @@ def run(a, ops):
             sid, toks = op[1], op[2]
             n_cached, slots = r[1], r[2]
             assert n_cached % a.block_size == 0 and len(slots) == len(toks) - n_cached
-            for sl, tok in zip(slots, toks[n_cached:]):
-                data[sl] = tok
+            for i, sl in enumerate(slots):
+                data[sl] = tuple(toks[:n_cached + i + 1])
             model[sid] = list(toks)
         elif k in ("tokens", "slots") and r[0] == OK:
             st, slots, pairs = r
@@ -79,9 +84,10 @@ def run(a, ops):
                     if src * a.block_size + o in data:
                         data[dst * a.block_size + o] = data[src * a.block_size + o]
             toks = op[2] if k == "tokens" else [None] * op[2]
-            for sl, tok in zip(slots, toks):
-                data[sl] = tok
-            model[op[1]] = model[op[1]] + list(toks)
+            before = model[op[1]]
+            for i, sl in enumerate(slots):
+                data[sl] = tuple(before + list(toks[:i + 1]))
+            model[op[1]] = before + list(toks)
         elif k == "fork" and r == OK:
             model[op[2]] = list(model[op[1]])
         elif k == "free" and r == OK:
