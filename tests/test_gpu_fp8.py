@@ -52,6 +52,32 @@ def test_kv_append_fp8_bit_exact(src, scales):
     assert np.array_equal(kd.cpu().numpy(), kc) and np.array_equal(vd.cpu().numpy(), vc)
 
 
+@pytest.mark.parametrize("src", [torch.bfloat16, torch.float16, torch.float32])
+@pytest.mark.parametrize("scale", [1.0, 1 / 64])
+def test_kv_append_fp8_rounds_ties_to_even(src, scale):
+    """Every midpoint between adjacent E4M3 values, as an exact tie after the
+    x * (1/scale) product (power-of-two scales), quantized bit-exactly like
+    the oracle (ties to the even code)."""
+    import paged_kv_cache_405_b200 as pkv
+    from test_oracle_pins import e4m3_midpoints
+    NB, Hkv, bs, D, T = 4, 2, 16, 128, 2
+    mids = e4m3_midpoints() * scale
+    flat = torch.zeros(T * Hkv * D)
+    flat[:len(mids)] = mids
+    kn = flat.view(T, Hkv, D).to(src)
+    assert torch.equal(kn.float(), flat.view(T, Hkv, D))      # the ties are exact in the input type
+    vn = kn.flip(0)
+    slots = np.array([5, 37], np.int64)
+    kc = np.zeros((NB, Hkv, bs, D), np.uint8)
+    vc = np.zeros((NB, Hkv, bs, D), np.uint8)
+    oracle.kv_append_fp8(kc, vc, kn, vn, scale, scale, slots)
+    kd = torch.zeros((NB, Hkv, bs, D), dtype=torch.uint8, device="cuda")
+    vd = torch.zeros_like(kd)
+    pkv.kv_append_fp8(kn.cuda(), vn.cuda(), kd, vd, torch.from_numpy(slots).cuda(), scale, scale)
+    assert pkv.device_error() == 0
+    assert np.array_equal(kd.cpu().numpy(), kc) and np.array_equal(vd.cpu().numpy(), vc)
+
+
 @pytest.mark.parametrize("qdt", ["bf16", "f16"])
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 2), (8, 1), (32, 2), (40, 2)])
 @pytest.mark.parametrize("bs,D", [(16, 128), (64, 128), (32, 64)])
