@@ -67,6 +67,9 @@ ALLOC_MUTANTS = {
     "fresh block unreferenced": ("                self.ref[b] = 1\n                bt.append(b)",
                                  "                self.ref[b] = 0\n                bt.append(b)", 0),
     "block index of a token": ("j = t // bs", "j = (t + 1) // bs", 0),
+    "freed blocks to the front": ("self.free.append(b)", "self.free.appendleft(b)", 0),
+    "freed in reverse table order": ("        bt, _ = self.seqs.pop(sid)\n        for b in bt:",
+                                     "        bt, _ = self.seqs.pop(sid)\n        for b in reversed(bt):", 0),
 }
 
 
@@ -101,6 +104,16 @@ def test_allocator_pins_catch_planted_mistake(name):
         except (AssertionError, IndexError, KeyError, ValueError):
             caught = True
             break
+    if not caught:              # the free-queue order is pinned by a closed-form case
+        import test_oracle_pins as pins
+        saved = pins.Allocator
+        pins.Allocator = Broken
+        try:
+            pins.test_free_queue_takes_from_the_front_and_frees_to_the_back_in_table_order()
+        except AssertionError:
+            caught = True
+        finally:
+            pins.Allocator = saved
     assert caught, "no pin caught: %s" % name
 
 

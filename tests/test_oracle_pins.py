@@ -5,7 +5,8 @@ Each test below would fail under a plausible mistake in the oracle:
 * attention (dropped scale, sign, transposed K/V, wrong head group, off-by-one
   length, wrong widening of bf16/f16) -> torch SDPA on the contiguous layout,
   closed forms, GQA via SDPA's own grouping, fp32/bf16/f16 agreement;
-* allocator -> worked example, brute-force payload model and invariants.
+* allocator -> worked example, brute-force payload model and invariants,
+  the free queue's order in closed form.
 """
 import math
 import os
@@ -378,6 +379,24 @@ def test_allocator_exhaustion_is_atomic():
     st, slots, pairs = a.seq_append_slots(1, 4)          # needs a 4th block
     assert st == NO_FREE_BLOCK and slots == [] and a.seqs[1][1] == 9
     assert a.stats() == dict(free_blocks=0, used_blocks=3, alloc_failures=1, cow_copies=0)
+
+
+def test_free_queue_takes_from_the_front_and_frees_to_the_back_in_table_order():
+    """The pages only say that a block is taken from the free pool when needed
+    and returns to it when its sequence ends (aiknowledge.cn 2.2.2,
+    openeuler.csdn.net explainer 8.2); the reading taken is a FIFO queue:
+    take from the front, and a freed sequence's blocks join the back in
+    block-table order, so a just-freed block is the last to be reused."""
+    a = Allocator(6, 2, [5, 4, 3, 2, 1, 0])
+    assert a.seq_add(0) == OK and a.seq_append_slots(0, 5)[0] == OK       # takes 5, 4, 3
+    assert a.seq_block_table(0)[1] == [5, 4, 3]
+    assert a.seq_add(1) == OK and a.seq_append_slots(1, 2)[0] == OK       # takes 2
+    assert a.seq_free(0) == OK                                          # 5, 4, 3 join the back
+    assert list(a.free) == [1, 0, 5, 4, 3]
+    assert a.seq_add(2) == OK and a.seq_append_slots(2, 8)[0] == OK       # 1, 0 first, then 5, 4
+    assert a.seq_block_table(2)[1] == [1, 0, 5, 4]
+    st, slots, _ = a.seq_append_slots(2, 1)                              # token 8 opens a 5th block: 3
+    assert st == OK and slots == [3 * 2 + 0]
 
 
 def test_fork_then_append_copies_partial_block_once_per_writer():
