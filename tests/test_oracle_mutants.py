@@ -38,6 +38,15 @@ MUTANTS = {
     "f16 widening": ("else v = ldexp((double)(m | 1024), e - 25);", "else v = ldexp((double)(m | 1024), e - 24);"),
     "e4m3 exponent bias": ("else v = ldexp((double)(8 + m), e - 10);", "else v = ldexp((double)(8 + m), e - 11);"),
     "causal limit": ("int64_t upto = L - n + (t - query_start[s]) + 1;", "int64_t upto = L - n + (t - query_start[s]);"),
+    "FP8 V scaled by the K scale": ("o[d] += w * pool_value(v_pool, vbase + d, kv_dtype, v_scale);",
+                                    "o[d] += w * pool_value(v_pool, vbase + d, kv_dtype, k_scale);"),
+    "FP8 K scale dropped": ("acc += widen(q, qbase + d, q_dtype) * pool_value(k_pool, kbase + d, kv_dtype, k_scale);",
+                            "acc += widen(q, qbase + d, q_dtype) * pool_value(k_pool, kbase + d, kv_dtype, 1.0);"),
+    "chunk kv head of a query head": ("        int g = h / G;\n        const int32_t *bt = block_tables + (int64_t)s * max_blocks;",
+                                      "        int g = h % Hkv;\n        const int32_t *bt = block_tables + (int64_t)s * max_blocks;"),
+    "f16 subnormal exponent": ("if (e == 0) v = ldexp((double)m, -24);", "if (e == 0) v = ldexp((double)m, -25);"),
+    "context length off by one": ("        int64_t L = context_lens[s];\n        if (L <= 0) continue;",
+                                  "        int64_t L = context_lens[s] - 1;\n        if (L <= 0) continue;"),
 }
 
 
