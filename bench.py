@@ -394,7 +394,19 @@ def run_ours(args, world, rank, local):
     out = torch.empty_like(inputs[0][0])
     stream = torch.cuda.current_stream()
 
+    if args.nvtx:
+        pkv.set_nvtx(True)      # one range per library call, inside one per step
+
     def run_step(i, ev=None):
+        if not args.nvtx:
+            return step_calls(i, ev)
+        torch.cuda.nvtx.range_push("decode_step")
+        try:
+            return step_calls(i, ev)
+        finally:
+            torch.cuda.nvtx.range_pop()
+
+    def step_calls(i, ev=None):
         d = plans[i]
         q, kn, vn = inputs[i]
         if shape.chunk:
@@ -492,6 +504,7 @@ def run_ours(args, world, rank, local):
                        "l2": "inputs larger than L2 (K/V pool %.2f GB per rank)" % (
                            2 * ss.k_pool.numel() * ss.k_pool.element_size() / 1e9),
                        "parallelism": "replica per GPU" if world > 1 else "1 GPU",
+                       **({"nvtx_ranges": True} if args.nvtx else {}),
                        "shared_prefix_groups": int((plans[W].group_shared > 0).sum().item())
                        if not shape.chunk and plans[W].group_shared is not None else 0},
             "pct_of_peak": round(100 * value / peak, 1),
@@ -729,6 +742,8 @@ def main(argv=None):
     ap.add_argument("--allocator-bench", action="store_true",
                     help="host-only prefix-caching allocator simulation (prints its own JSON line)")
     ap.add_argument("--requests", type=int, default=2000)
+    ap.add_argument("--nvtx", action="store_true",
+                    help="NVTX ranges around each step and each library call (e.g. for ncu --nvtx filters)")
     ap.add_argument("--clock-warm-s", type=float, default=0.5,
                     help="seconds of untimed repeats before the timed region, while clocks are sampled")
     args = ap.parse_args(argv)

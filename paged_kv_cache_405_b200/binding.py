@@ -10,6 +10,7 @@ this module fails; device calls demand CUDA tensors.
 from __future__ import annotations
 
 import ctypes
+import functools
 import os
 from typing import Optional
 
@@ -137,7 +138,35 @@ def _dt(t: torch.Tensor) -> int:
     return _DTYPE[t.dtype]
 
 
+# ------------------------------------------------------------------ NVTX ranges
+_NVTX = False
+
+
+def set_nvtx(on: bool) -> None:
+    """Mark every device call with an NVTX range named after its C entry point
+    (``pkv_kv_append``, ``pkv_paged_attention_decode`` ...), for ``ncu --nvtx``
+    filters and timeline tools.  Off by default."""
+    global _NVTX
+    _NVTX = bool(on)
+
+
+def _ranged(cname: str):
+    def wrap(fn):
+        @functools.wraps(fn)
+        def call(*args, **kwargs):
+            if not _NVTX:
+                return fn(*args, **kwargs)
+            torch.cuda.nvtx.range_push(cname)
+            try:
+                return fn(*args, **kwargs)
+            finally:
+                torch.cuda.nvtx.range_pop()
+        return call
+    return wrap
+
+
 # ------------------------------------------------------------------ device calls
+@_ranged("pkv_kv_append")
 def kv_append(k_new, v_new, k_pool, v_pool, slot_mapping, stream=None) -> None:
     """Write token i's K/V ``[T, Hkv, D]`` into pool slot ``slot_mapping[i]`` (int64; < 0 skips)."""
     NB, Hkv, bs, D = k_pool.shape
@@ -168,6 +197,7 @@ def workspace_for(q, block_tables, block_size, partition_size=0) -> torch.Tensor
     return torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
 
 
+@_ranged("pkv_paged_attention_decode")
 def paged_attention_decode(out, q, k_pool, v_pool, block_tables, context_lens, scale: float = 0.0,
                            partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
                            stream=None) -> torch.Tensor:
@@ -188,6 +218,7 @@ def paged_attention_decode(out, q, k_pool, v_pool, block_tables, context_lens, s
     return out
 
 
+@_ranged("pkv_paged_attention_decode_static")
 def paged_attention_decode_static(out, q, k_pool, v_pool, block_tables, context_lens, scale: float = 0.0,
                                   partition_size: int = 0, stream=None) -> torch.Tensor:
     """Decode attention that allocates nothing: the split-K scratch is a fixed
@@ -229,6 +260,7 @@ def find_shared_prefix_groups(block_tables: np.ndarray, context_lens: np.ndarray
     return first[:n + 1] if n else first[:0], shared[:n]
 
 
+@_ranged("pkv_paged_attention_decode_shared")
 def paged_attention_decode_shared(out, q, k_pool, v_pool, block_tables, context_lens, group_first, group_shared,
                                   max_group_size: int, max_shared_len: int, scale: float = 0.0,
                                   partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
@@ -260,6 +292,7 @@ def attention_chunk_workspace_bytes(num_tokens: int, num_q_heads: int, head_dim:
                                                        partition_size))
 
 
+@_ranged("pkv_paged_attention_chunk")
 def paged_attention_chunk(out, q, k_pool, v_pool, block_tables, context_lens, query_start, max_query_len: int,
                           scale: float = 0.0, partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
                           stream=None) -> torch.Tensor:
@@ -283,6 +316,7 @@ def paged_attention_chunk(out, q, k_pool, v_pool, block_tables, context_lens, qu
     return out
 
 
+@_ranged("pkv_kv_append_fp8")
 def kv_append_fp8(k_new, v_new, k_pool, v_pool, slot_mapping, k_scale: float, v_scale: float,
                   stream=None) -> None:
     """Quantize new K/V ([T, Hkv, D], f32/bf16/f16) into FP8 E4M3 pools (uint8 [NB, Hkv, bs, D])."""
@@ -296,6 +330,7 @@ def kv_append_fp8(k_new, v_new, k_pool, v_pool, slot_mapping, k_scale: float, v_
                                  Hkv, D, bs, _dt(k_new), float(k_scale), float(v_scale), _stream(stream)))
 
 
+@_ranged("pkv_paged_attention_decode_fp8")
 def paged_attention_decode_fp8(out, q, k_pool, v_pool, block_tables, context_lens, k_scale: float,
                                v_scale: float, scale: float = 0.0, partition_size: int = 0,
                                workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
@@ -317,6 +352,7 @@ def paged_attention_decode_fp8(out, q, k_pool, v_pool, block_tables, context_len
     return out
 
 
+@_ranged("pkv_block_copy")
 def block_copy(k_pool, v_pool, pairs, stream=None) -> None:
     """Copy whole blocks ``pairs[i] = (src, dst)`` (int32 ``[n, 2]`` on the device), K and V."""
     NB, Hkv, bs, D = k_pool.shape

@@ -110,3 +110,27 @@ def test_build_runs_from_a_checkout_without_the_library(tmp_path):
             "assert 'paged_kv_cache_405_b200' not in sys.modules\n")
     r = subprocess.run([sys.executable, "-c", code], cwd=root, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
+
+
+def test_nvtx_ranges_name_the_entry_point_and_always_close(monkeypatch):
+    """With NVTX on, each device call opens a range named after its C entry
+    point and closes it even when the call raises (here: CPU tensors)."""
+    import torch
+    events = []
+    monkeypatch.setattr(torch.cuda.nvtx, "range_push", lambda name: events.append(("push", name)))
+    monkeypatch.setattr(torch.cuda.nvtx, "range_pop", lambda: events.append(("pop",)))
+    k = torch.zeros(4, 2, 16, 64, dtype=torch.bfloat16)
+    new = torch.zeros(1, 2, 64, dtype=torch.bfloat16)
+    pkv.set_nvtx(True)
+    try:
+        with pytest.raises((ValueError, TypeError)):
+            pkv.kv_append(new, new, k, k, torch.zeros(1, dtype=torch.int64))
+        with pytest.raises((ValueError, TypeError)):
+            pkv.block_copy(k, k, torch.zeros(1, 2, dtype=torch.int32))
+    finally:
+        pkv.set_nvtx(False)
+    assert events == [("push", "pkv_kv_append"), ("pop",), ("push", "pkv_block_copy"), ("pop",)]
+    pkv.set_nvtx(False)
+    with pytest.raises((ValueError, TypeError)):   # off: no ranges
+        pkv.kv_append(new, new, k, k, torch.zeros(1, dtype=torch.int64))
+    assert len(events) == 4
