@@ -99,18 +99,32 @@ class DecodeSession:
 
     # ------------------------------------------------------------ host side
     def add(self, sid: int, num_tokens: int = 0, shared_prefix: Optional[Sequence[int]] = None,
-            prefix_tokens: int = 0) -> list:
+            prefix_tokens: int = 0, stream=None) -> list:
         """Register a sequence; map a shared prefix onto existing blocks, then
-        reserve slots for ``num_tokens`` more tokens.  Returns their slots."""
+        reserve slots for ``num_tokens`` more tokens.  Returns their slots.
+
+        A prefix that ends part-way through a block leaves that block shared
+        and partly filled: the first reserved slot then lies in a private copy
+        of it, which this call makes (``block_copy`` on ``stream``) before it
+        returns, so the caller's ``kv_append`` to the returned slots must follow
+        on the same stream.  If any step fails the sequence is not registered."""
         self._ok(self.alloc.seq_add(sid))
-        if shared_prefix is not None:
-            self._ok(self.alloc.seq_share_prefix(sid, shared_prefix, prefix_tokens))
-        if num_tokens:
+        try:
+            if shared_prefix is not None:
+                self._ok(self.alloc.seq_share_prefix(sid, shared_prefix, prefix_tokens))
+            if not num_tokens:
+                return []
             st, slots, cow = self.alloc.seq_append_slots(sid, num_tokens)
             self._ok(st)
-            assert not cow
-            return slots
-        return []
+        except Exception:
+            self.alloc.seq_free(sid)
+            raise
+        if cow:
+            s = torch.cuda.current_stream() if stream is None else stream
+            with torch.cuda.stream(s):
+                pairs = torch.tensor(cow, dtype=torch.int32).to(self.device)
+                B.block_copy(self.k_pool, self.v_pool, pairs, stream=s)
+        return slots
 
     def add_prompt(self, sid: int, tokens: Sequence[int]):
         """Register a sequence by its prompt token ids (automatic prefix

@@ -85,3 +85,59 @@ def test_back_to_back_uploads_keep_their_plans():
         assert np.array_equal(d.lens.cpu().numpy(), p.lens)
         assert np.array_equal(d.block_tables.cpu().numpy(), p.block_tables)
         assert d.cow_pairs.shape == (0, 2) and d.n_cow == 0
+
+
+@pytest.mark.parametrize("prefix_tokens", [20, 33])
+def test_add_with_a_prefix_ending_inside_a_block_copies_that_block(prefix_tokens):
+    """Sequences mapped onto a prompt that ends part-way through a block: each
+    one's first token lands in a private copy of that shared block (made by
+    ``add``), the prompt's owner keeps the original; pools and attention match
+    the oracle allocator + block_copy + kv_append + attention."""
+    import paged_kv_cache_405_b200 as m
+    NB, Hq, Hkv, bs, D, S, n_own = 24, 8, 2, 16, 64, 3, 5
+    g = torch.Generator().manual_seed(prefix_tokens)
+    k0 = synth.randn((NB, Hkv, bs, D), g, torch.bfloat16, "cpu")
+    v0 = synth.randn((NB, Hkv, bs, D), g, torch.bfloat16, "cpu")
+    order = list(np.random.default_rng(prefix_tokens).permutation(NB))
+    dev = torch.device("cuda")
+    k, v = k0.to(dev), v0.to(dev)
+    ss = m.DecodeSession(k, v, Hq, 8, free_order=order, max_batch=S, share_prefixes=False)
+    orc = oracle.Allocator(NB, bs, order)
+    kc, vc = k0.clone(), v0.clone()
+
+    def write(slots, kn, vn, pairs=()):
+        oracle.block_copy(kc, vc, list(pairs))
+        oracle.kv_append(kc, vc, kn, vn, slots)
+        m.kv_append(kn.to(dev), vn.to(dev), k, v, torch.tensor(slots, dtype=torch.int64, device=dev))
+
+    slots = ss.add(-1, prefix_tokens)                      # the prompt's owner
+    orc.seq_add(-1)
+    st, oslots, _ = orc.seq_append_slots(-1, prefix_tokens)
+    assert st == 0 and oslots == slots
+    write(slots, synth.randn((prefix_tokens, Hkv, D), g, torch.bfloat16, "cpu"),
+          synth.randn((prefix_tokens, Hkv, D), g, torch.bfloat16, "cpu"))
+    prompt, _ = ss.table(-1)
+    for s in range(S):
+        slots = ss.add(s, n_own, shared_prefix=prompt, prefix_tokens=prefix_tokens)
+        orc.seq_add(s)
+        assert orc.seq_share_prefix(s, prompt, prefix_tokens) == 0
+        st, oslots, pairs = orc.seq_append_slots(s, n_own)
+        assert st == 0 and oslots == slots and len(pairs) == 1      # the shared partial block is copied
+        write(slots, synth.randn((n_own, Hkv, D), g, torch.bfloat16, "cpu"),
+              synth.randn((n_own, Hkv, D), g, torch.bfloat16, "cpu"), pairs)
+    torch.cuda.synchronize()
+    assert torch.equal(k.cpu(), kc) and torch.equal(v.cpu(), vc)
+    ids = [-1] + list(range(S))
+    bt = np.full((len(ids), 8), -1, np.int32)
+    lens = np.zeros(len(ids), np.int32)
+    for i, sid in enumerate(ids):
+        t, L = ss.table(sid)
+        assert (t, L) == tuple(orc.seq_block_table(sid)[1:])
+        bt[i, :len(t)] = t
+        lens[i] = L
+    q = synth.randn((len(ids), Hq, D), g, torch.bfloat16, "cpu")
+    out = torch.empty(len(ids), Hq, D, dtype=torch.bfloat16, device=dev)
+    m.paged_attention_decode(out, q.to(dev), k, v, torch.from_numpy(bt).to(dev), torch.from_numpy(lens).to(dev))
+    ref = oracle.paged_attention(q, kc, vc, bt, lens)
+    assert m.device_error() == 0
+    assert max_err(out, ref) <= TOL[out.dtype]

@@ -1,0 +1,36 @@
+"""DecodeSession's host side on CPU tensors: a failed ``add`` leaves no
+sequence behind (the id can be registered again) and gives back every block
+it took or mapped."""
+import pytest
+import torch
+
+import paged_kv_cache_405_b200 as pkv
+
+
+def session(num_blocks=4, bs=16):
+    k = torch.zeros(num_blocks, 1, bs, 64, dtype=torch.bfloat16)
+    return pkv.DecodeSession(k, k.clone(), 1, 8, max_batch=2)
+
+
+def test_add_that_runs_out_of_blocks_registers_nothing():
+    ss = session()
+    with pytest.raises(pkv.PagedKVError):
+        ss.add(0, 5 * 16)                          # needs 5 of 4 blocks
+    assert ss.alloc.stats()["free_blocks"] == 4
+    assert ss.add(0, 16) == list(range(0, 16))    # the id is free again; block 0 first
+    assert ss.table(0) == ([0], 16)
+
+
+def test_add_with_a_bad_prefix_registers_nothing_and_keeps_refcounts():
+    ss = session()
+    ss.add(0, 20)                                  # blocks 0, 1
+    prompt, _ = ss.table(0)
+    with pytest.raises(pkv.PagedKVError):
+        ss.add(1, 3, shared_prefix=prompt, prefix_tokens=40)   # 40 tokens need 3 blocks, not 2
+    assert [ss.alloc.refcount(b) for b in prompt] == [1, 1]
+    with pytest.raises(pkv.PagedKVError):
+        ss.add(1, 3 * 16, shared_prefix=prompt, prefix_tokens=32)   # mapped, then out of blocks
+    assert [ss.alloc.refcount(b) for b in prompt] == [1, 1]
+    assert ss.alloc.stats()["free_blocks"] == 2
+    assert ss.add(1, 0, shared_prefix=prompt, prefix_tokens=32) == []
+    assert [ss.alloc.refcount(b) for b in prompt] == [2, 2]
