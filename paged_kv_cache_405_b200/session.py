@@ -161,6 +161,7 @@ class DecodeSession:
         """Reserve one new slot for every sequence in ``write`` (default: ``attend``),
         collect copy-on-write pairs, and snapshot the tables of ``attend``."""
         write = list(attend if write is None else write)
+        self._check_fits(attend, write)
         st, slots, pairs = self.alloc.seq_append_slots_batch(write)
         self._ok(st)
         st, bt, lens = self.alloc.seq_block_tables_batch(list(attend), self.max_blocks)
@@ -174,10 +175,28 @@ class DecodeSession:
                 plan.max_shared_len = int(gs.max())
         return plan
 
+    def _check_fits(self, attend: Sequence[int], write) -> None:
+        """Fail before any slot is reserved (the step's reservations cannot be
+        undone): every sequence of ``attend`` must exist and still fit in
+        max_blocks_per_seq blocks after this step's tokens."""
+        st, _, lens = self.alloc.seq_block_tables_batch(list(attend), self.max_blocks)
+        self._ok(st)
+        if not len(lens):
+            return
+        ids, counts = np.unique(np.asarray(write, dtype=np.int64), return_counts=True)
+        grow = dict(zip(ids.tolist(), counts.tolist()))
+        tokens = lens.astype(np.int64) + np.array([grow.get(int(sid), 0) for sid in attend], dtype=np.int64)
+        blocks = -(-tokens // self.block_size)
+        if blocks.max() > self.max_blocks:
+            i = int(blocks.argmax())
+            raise B.PagedKVError(B.INVALID, "sequence %d would need %d blocks, more than max_blocks_per_seq = %d"
+                                 % (int(attend[i]), int(blocks[i]), self.max_blocks))
+
     def plan_chunk(self, seq_ids: Sequence[int], n_new: Sequence[int]) -> ChunkPlan:
         """Reserve slots for n_new[i] new tokens of seq_ids[i] (a causal chunk:
         draft tokens to verify, or part of a prompt)."""
         ids = np.repeat(np.asarray(seq_ids, dtype=np.int64), np.asarray(n_new, dtype=np.int64))
+        self._check_fits(seq_ids, ids)
         st, slots, pairs = self.alloc.seq_append_slots_batch(ids)
         self._ok(st)
         st, bt, lens = self.alloc.seq_block_tables_batch(list(seq_ids), self.max_blocks)

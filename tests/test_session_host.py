@@ -34,3 +34,24 @@ def test_add_with_a_bad_prefix_registers_nothing_and_keeps_refcounts():
     assert ss.alloc.stats()["free_blocks"] == 2
     assert ss.add(1, 0, shared_prefix=prompt, prefix_tokens=32) == []
     assert [ss.alloc.refcount(b) for b in prompt] == [2, 2]
+
+
+def test_plan_fails_before_reserving_anything():
+    """A step that names an unknown sequence, or would grow a sequence past
+    max_blocks_per_seq, raises with every table and the free pool unchanged."""
+    k = torch.zeros(8, 1, 16, 64, dtype=torch.bfloat16)
+    ss = pkv.DecodeSession(k, k.clone(), 1, 2, max_batch=4)          # at most 2 blocks per sequence
+    ss.add(0, 10)
+    ss.add(1, 32)                                                    # full: 2 blocks
+    before = (ss.table(0), ss.table(1), ss.alloc.stats())
+    with pytest.raises(pkv.PagedKVError):
+        ss.plan([0, 7])                                              # unknown sequence 7
+    with pytest.raises(pkv.PagedKVError):
+        ss.plan([0, 1])                                              # token 32 of seq 1 needs a 3rd block
+    with pytest.raises(pkv.PagedKVError):
+        ss.plan_chunk([0], [23])                                     # 10 + 23 tokens need 3 blocks
+    assert (ss.table(0), ss.table(1), ss.alloc.stats()) == before
+    p = ss.plan([0], write=[0, 0])                                   # two tokens of seq 0 still fit
+    assert p.lens.tolist() == [12] and ss.table(0)[1] == 12
+    p = ss.plan_chunk([0], [20])                                     # exactly 32 tokens: fits
+    assert p.lens.tolist() == [32]
