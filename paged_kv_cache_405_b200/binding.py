@@ -138,6 +138,50 @@ def _dt(t: torch.Tensor) -> int:
     return _DTYPE[t.dtype]
 
 
+# The C calls see pointers and the sizes passed next to them, not the tensors:
+# these checks make the sizes read off one tensor hold for the others, so that
+# no call reads or writes past a caller's buffer.
+def _cuda(**tensors) -> None:
+    for name, t in tensors.items():
+        if not isinstance(t, torch.Tensor) or not t.is_cuda:
+            raise TypeError("%s must be a CUDA tensor" % name)
+
+
+def _check_pools(k_pool, v_pool) -> None:
+    if k_pool.dim() != 4:
+        raise ValueError("pools must be [num_blocks, num_kv_heads, block_size, head_dim]")
+    if v_pool.shape != k_pool.shape or v_pool.dtype != k_pool.dtype:
+        raise ValueError("k_pool and v_pool must have the same shape and element type")
+
+
+def _check_new(k_new, v_new, k_pool, slot_mapping, pool_type: bool) -> None:
+    """New K/V [T, num_kv_heads, head_dim] of the pools, one slot per token;
+    pool_type: in the pools' element type (the FP8 append converts)."""
+    if k_new.dim() != 3 or tuple(k_new.shape[1:]) != (k_pool.shape[1], k_pool.shape[3]):
+        raise ValueError("new K/V must be [T, num_kv_heads, head_dim] of the pools")
+    if v_new.shape != k_new.shape or v_new.dtype != k_new.dtype:
+        raise ValueError("k_new and v_new must have the same shape and element type")
+    if pool_type and k_new.dtype != k_pool.dtype:
+        raise TypeError("new K/V must have the pools' element type")
+    if slot_mapping.numel() < k_new.shape[0]:
+        raise ValueError("slot_mapping needs one entry per new token")
+
+
+def _check_attention(out, q, k_pool, block_tables, context_lens, rows: int, pool_type: bool) -> None:
+    """out like q [rows of q, num_q_heads, head_dim]; tables and lengths for
+    ``rows`` sequences; pool_type: q in the pools' element type (not FP8)."""
+    if q.dim() != 3 or out.shape != q.shape or out.dtype != q.dtype:
+        raise ValueError("out must have the shape and element type of q [rows, num_q_heads, head_dim]")
+    if q.shape[2] != k_pool.shape[3]:
+        raise ValueError("q's head_dim differs from the pools'")
+    if pool_type and q.dtype != k_pool.dtype:
+        raise TypeError("q, out and the pools must share one element type")
+    if block_tables.dim() != 2 or block_tables.shape[0] < rows:
+        raise ValueError("block_tables must be [num_seqs, max_blocks_per_seq]")
+    if context_lens.numel() < rows:
+        raise ValueError("context_lens needs one entry per sequence")
+
+
 # ------------------------------------------------------------------ NVTX ranges
 _NVTX = False
 
@@ -169,10 +213,13 @@ def _ranged(cname: str):
 @_ranged("pkv_kv_append")
 def kv_append(k_new, v_new, k_pool, v_pool, slot_mapping, stream=None) -> None:
     """Write token i's K/V ``[T, Hkv, D]`` into pool slot ``slot_mapping[i]`` (int64; < 0 skips)."""
+    _cuda(k_new=k_new, v_new=v_new, k_pool=k_pool, v_pool=v_pool, slot_mapping=slot_mapping)
+    _check_pools(k_pool, v_pool)
     NB, Hkv, bs, D = k_pool.shape
     T = k_new.shape[0]
     if slot_mapping.dtype != torch.int64:
         raise TypeError("slot_mapping must be int64")
+    _check_new(k_new, v_new, k_pool, slot_mapping, pool_type=True)
     _check(lib.pkv_kv_append(_dev(k_new, "k_new"), _dev(v_new, "v_new"), _dev(k_pool, "k_pool"),
                              _dev(v_pool, "v_pool"), _dev(slot_mapping, "slot_mapping"), T, NB, Hkv, D, bs,
                              _dt(k_pool), _stream(stream)))
@@ -202,10 +249,13 @@ def paged_attention_decode(out, q, k_pool, v_pool, block_tables, context_lens, s
                            partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
                            stream=None) -> torch.Tensor:
     """Decode attention: ``out[s, h] = softmax(scale q K^T) V`` over ``context_lens[s]`` cached tokens."""
+    _cuda(out=out, q=q, k_pool=k_pool, v_pool=v_pool, block_tables=block_tables, context_lens=context_lens)
+    _check_pools(k_pool, v_pool)
     S, Hq, D = q.shape
-    NB, Hkv, bs, D2 = k_pool.shape
+    NB, Hkv, bs, _ = k_pool.shape
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise TypeError("block_tables and context_lens must be int32")
+    _check_attention(out, q, k_pool, block_tables, context_lens, S, pool_type=True)
     maxB = block_tables.shape[1]
     if workspace is None:
         workspace = workspace_for(q, block_tables, bs, partition_size)
@@ -225,10 +275,13 @@ def paged_attention_decode_static(out, q, k_pool, v_pool, block_tables, context_
     64 MiB buffer inside the library (one per GPU), for callers that cannot
     allocate device memory.  Calls on one device share that buffer, so calls
     that overlap on the GPU must not be issued; oversized calls raise."""
+    _cuda(out=out, q=q, k_pool=k_pool, v_pool=v_pool, block_tables=block_tables, context_lens=context_lens)
+    _check_pools(k_pool, v_pool)
     S, Hq, D = q.shape
-    NB, Hkv, bs, D2 = k_pool.shape
+    NB, Hkv, bs, _ = k_pool.shape
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise TypeError("block_tables and context_lens must be int32")
+    _check_attention(out, q, k_pool, block_tables, context_lens, S, pool_type=True)
     _check(lib.pkv_paged_attention_decode_static(
         _dev(out, "out"), _dev(q, "q"), _dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
         _dev(block_tables, "block_tables"), block_tables.shape[1], _dev(context_lens, "context_lens"), S, Hq, Hkv,
@@ -267,11 +320,17 @@ def paged_attention_decode_shared(out, q, k_pool, v_pool, block_tables, context_
                                   stream=None) -> torch.Tensor:
     """Decode attention with shared-prefix groups (device int32 group_first [n+1], group_shared [n];
     host bounds max_group_size and max_shared_len)."""
+    _cuda(out=out, q=q, k_pool=k_pool, v_pool=v_pool, block_tables=block_tables, context_lens=context_lens,
+          group_first=group_first, group_shared=group_shared)
+    _check_pools(k_pool, v_pool)
     S, Hq, D = q.shape
-    NB, Hkv, bs, D2 = k_pool.shape
+    NB, Hkv, bs, _ = k_pool.shape
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise TypeError("block_tables and context_lens must be int32")
+    _check_attention(out, q, k_pool, block_tables, context_lens, S, pool_type=True)
     n = group_shared.numel()
+    if n and group_first.numel() < n + 1:
+        raise ValueError("group_first needs num_groups + 1 entries")
     maxB = block_tables.shape[1]
     if workspace is None:
         nb = attention_shared_workspace_bytes(S, Hq, D, maxB * bs, partition_size)
@@ -297,12 +356,18 @@ def paged_attention_chunk(out, q, k_pool, v_pool, block_tables, context_lens, qu
                           scale: float = 0.0, partition_size: int = 0, workspace: Optional[torch.Tensor] = None,
                           stream=None) -> torch.Tensor:
     """Causal attention of the last ``query_start[s+1]-query_start[s]`` tokens of each sequence."""
+    _cuda(out=out, q=q, k_pool=k_pool, v_pool=v_pool, block_tables=block_tables, context_lens=context_lens,
+          query_start=query_start)
+    _check_pools(k_pool, v_pool)
     T, Hq, D = q.shape
-    NB, Hkv, bs, D2 = k_pool.shape
+    NB, Hkv, bs, _ = k_pool.shape
     for t, nm in ((block_tables, "block_tables"), (context_lens, "context_lens"), (query_start, "query_start")):
         if t.dtype != torch.int32:
             raise TypeError("%s must be int32" % nm)
     S = context_lens.numel()
+    _check_attention(out, q, k_pool, block_tables, context_lens, S, pool_type=True)
+    if query_start.numel() < S + 1:
+        raise ValueError("query_start needs num_seqs + 1 entries")
     maxB = block_tables.shape[1]
     if workspace is None:
         nb = attention_chunk_workspace_bytes(T, Hq, D, maxB * bs, partition_size)
@@ -320,11 +385,14 @@ def paged_attention_chunk(out, q, k_pool, v_pool, block_tables, context_lens, qu
 def kv_append_fp8(k_new, v_new, k_pool, v_pool, slot_mapping, k_scale: float, v_scale: float,
                   stream=None) -> None:
     """Quantize new K/V ([T, Hkv, D], f32/bf16/f16) into FP8 E4M3 pools (uint8 [NB, Hkv, bs, D])."""
+    _cuda(k_new=k_new, v_new=v_new, k_pool=k_pool, v_pool=v_pool, slot_mapping=slot_mapping)
+    _check_pools(k_pool, v_pool)
     NB, Hkv, bs, D = k_pool.shape
     if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
         raise TypeError("FP8 pools are uint8 tensors of E4M3 codes")
     if slot_mapping.dtype != torch.int64:
         raise TypeError("slot_mapping must be int64")
+    _check_new(k_new, v_new, k_pool, slot_mapping, pool_type=False)
     _check(lib.pkv_kv_append_fp8(_dev(k_new, "k_new"), _dev(v_new, "v_new"), _dev(k_pool, "k_pool"),
                                  _dev(v_pool, "v_pool"), _dev(slot_mapping, "slot_mapping"), k_new.shape[0], NB,
                                  Hkv, D, bs, _dt(k_new), float(k_scale), float(v_scale), _stream(stream)))
@@ -335,12 +403,15 @@ def paged_attention_decode_fp8(out, q, k_pool, v_pool, block_tables, context_len
                                v_scale: float, scale: float = 0.0, partition_size: int = 0,
                                workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Decode attention over FP8 E4M3 pools (values = code x k_scale / x v_scale); q/out bf16 or f16."""
+    _cuda(out=out, q=q, k_pool=k_pool, v_pool=v_pool, block_tables=block_tables, context_lens=context_lens)
+    _check_pools(k_pool, v_pool)
     S, Hq, D = q.shape
-    NB, Hkv, bs, D2 = k_pool.shape
+    NB, Hkv, bs, _ = k_pool.shape
     if k_pool.dtype != torch.uint8 or v_pool.dtype != torch.uint8:
         raise TypeError("FP8 pools are uint8 tensors of E4M3 codes")
     if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
         raise TypeError("block_tables and context_lens must be int32")
+    _check_attention(out, q, k_pool, block_tables, context_lens, S, pool_type=False)
     maxB = block_tables.shape[1]
     if workspace is None:
         workspace = workspace_for(q, block_tables, bs, partition_size)
@@ -355,9 +426,13 @@ def paged_attention_decode_fp8(out, q, k_pool, v_pool, block_tables, context_len
 @_ranged("pkv_block_copy")
 def block_copy(k_pool, v_pool, pairs, stream=None) -> None:
     """Copy whole blocks ``pairs[i] = (src, dst)`` (int32 ``[n, 2]`` on the device), K and V."""
+    _cuda(k_pool=k_pool, v_pool=v_pool, pairs=pairs)
+    _check_pools(k_pool, v_pool)
     NB, Hkv, bs, D = k_pool.shape
     if pairs.dtype != torch.int32:
         raise TypeError("pairs must be int32")
+    if pairs.numel() and (pairs.dim() != 2 or pairs.shape[1] != 2):
+        raise ValueError("pairs must be [n, 2] (src, dst)")
     n = pairs.shape[0] if pairs.numel() else 0
     dt = FP8_E4M3 if k_pool.dtype == torch.uint8 else _dt(k_pool)
     _check(lib.pkv_block_copy(_dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),

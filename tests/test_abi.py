@@ -134,3 +134,43 @@ def test_nvtx_ranges_name_the_entry_point_and_always_close(monkeypatch):
     with pytest.raises((ValueError, TypeError)):   # off: no ranges
         pkv.kv_append(new, new, k, k, torch.zeros(1, dtype=torch.int64))
     assert len(events) == 4
+
+
+def test_binding_rejects_inconsistent_buffers():
+    """The C calls see pointers and sizes only: the binding rejects tensors
+    whose sizes or element types disagree with the sizes it passes, each of
+    which would make a kernel read or write past a buffer."""
+    import torch
+    bf, f32, u8 = torch.bfloat16, torch.float32, torch.uint8
+    k = torch.zeros(8, 2, 16, 64, dtype=bf)
+    q = torch.zeros(3, 4, 64, dtype=bf)
+    bt = torch.zeros(3, 5, dtype=torch.int32)
+    cl = torch.zeros(3, dtype=torch.int32)
+    new = torch.zeros(2, 2, 64, dtype=bf)
+    sm = torch.zeros(2, dtype=torch.int64)
+    # consistent arguments pass
+    binding._check_pools(k, k.clone())
+    binding._check_attention(q.clone(), q, k, bt, cl, 3, pool_type=True)
+    binding._check_attention(q.clone(), q, k.to(u8), bt, cl, 3, pool_type=False)   # FP8 pools
+    binding._check_new(new, new.clone(), k, sm, pool_type=True)
+    binding._check_new(new.float(), new.float(), k.to(u8), sm, pool_type=False)   # FP8 append converts
+    bad = [
+        lambda: binding._check_pools(k, k[:4].clone()),                                   # V pool smaller
+        lambda: binding._check_pools(k, k.float()),                                       # V pool wider type
+        lambda: binding._check_pools(k[0], k[0]),                                         # not 4-D
+        lambda: binding._check_attention(q.float(), q, k, bt, cl, 3, pool_type=True),     # out wider than q
+        lambda: binding._check_attention(q[:2].clone(), q, k, bt, cl, 3, pool_type=True),  # out smaller
+        lambda: binding._check_attention(q.float(), q.float(), k, bt, cl, 3, pool_type=True),   # q vs pools
+        lambda: binding._check_attention(q[..., :32].clone(), q[..., :32].clone(), k, bt, cl, 3, pool_type=True),
+        lambda: binding._check_attention(q.clone(), q, k, bt[:2], cl, 3, pool_type=True),  # table rows
+        lambda: binding._check_attention(q.clone(), q, k, bt, cl[:2], 3, pool_type=True),  # lengths
+        lambda: binding._check_new(new, new, k, sm[:1], pool_type=True),                  # one slot short
+        lambda: binding._check_new(new.float(), new.float(), k, sm, pool_type=True),      # wider than pool
+        lambda: binding._check_new(new, new.float(), k, sm, pool_type=True),              # K / V differ
+        lambda: binding._check_new(torch.zeros(2, 4, 64, dtype=bf), torch.zeros(2, 4, 64, dtype=bf), k, sm,
+                                   pool_type=True),                                       # kv heads
+    ]
+    for i, call in enumerate(bad):
+        with pytest.raises((ValueError, TypeError)):
+            call()
+            raise AssertionError("case %d passed" % i)
