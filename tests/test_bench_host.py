@@ -81,3 +81,33 @@ def test_cpu_baseline_sample_runs_on_one_thread():
     v, sps, desc, secs = bench.oracle_sample(b, 0.05, threads=1)
     assert v > 0 and sps > 0 and secs >= 0.05 and "1 threads" in desc
     assert isinstance(bench.cpu_model(), str) and bench.cpu_model()
+
+
+def test_reference_arm_prints_one_contract_line():
+    """``bench.py --impl reference`` (the CPU oracle on the host cores) prints
+    one JSON line with the contract's keys, its own cpu_baseline and an e2e
+    object without host<->device bytes."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--config", "tiny", "--steps", "2",
+                        "--warmup", "3", "--reference-step-seconds", "0.5"], cwd=root, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in d, key
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3 and d["n_gpus"] == 1
+    assert d["config"]["workload"] == "tiny" and d["value"] > 0 and d["higher_is_better"] is True
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_warmup_below_three_is_refused():
+    with pytest.raises(SystemExit):
+        bench.main(["--warmup", "2", "--impl", "reference", "--config", "tiny"])
