@@ -23,6 +23,10 @@
  *   - Device pointers are caller-owned device memory, 16-byte aligned; the
  *     library never allocates device memory (the split-K workspace is passed
  *     in; query its size first).
+ *   - Sizes are trusted: the library cannot see a buffer's extent, so every
+ *     buffer must hold at least what its size arguments describe (a table
+ *     row and a length per sequence, a slot per new token, q-shaped output);
+ *     a shorter one is read or written past its end.
  *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *     stream).  Device calls are asynchronous on that stream.
  *   - Host-side validation happens before any launch; a rejected call returns
