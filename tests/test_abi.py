@@ -74,6 +74,17 @@ def test_decode_validation(over, status):
     assert call_decode(**over) == status
 
 
+@pytest.mark.parametrize("over,why", [
+    (dict(S=65536), "at most 65535 sequences"),                       # one grid dimension
+    (dict(maxB=65536, P=16), "too many partitions"),                  # 65536 partitions of 16 tokens
+    (dict(maxB=(1 << 26) + 1), "max_blocks_per_seq*block_size too large"),   # over 2^30 tokens
+    (dict(NB=1 << 25, Hkv=4, Hq=4, bs=16), "2^31 or more rows"),     # 32-bit TMA row coordinates
+])
+def test_decode_size_limits_are_refused_before_any_launch(over, why):
+    assert call_decode(**over) == binding.INVALID
+    assert why in binding.lib.pkv_last_error().decode()
+
+
 def test_append_and_copy_validation():
     lib = binding.lib
     # head_dim*elem not a multiple of 16 bytes
