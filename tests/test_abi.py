@@ -48,7 +48,17 @@ def test_workspace_size_rules():
         pkv.attention_workspace_bytes(64, 32, 128, 2048, auto)
 
 
+def host_only():
+    """The validation tests below pass fake device pointers (address 16) and
+    rely on every case being refused before a launch; where a GPU is present
+    they are skipped, so that a case let through could never launch on them."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host-validation test with fake device pointers")
+
+
 def call_decode(**over):
+    host_only()
     a = dict(out=16, q=16, k=16, v=16, bt=16, maxB=4, cl=16, S=1, Hq=4, Hkv=4, D=64, bs=16, NB=8,
              scale=0.0, P=0, ws=None, wsb=0, dt=1, stream=None)
     a.update(over)
@@ -86,6 +96,7 @@ def test_decode_size_limits_are_refused_before_any_launch(over, why):
 
 
 def test_append_and_copy_validation():
+    host_only()
     lib = binding.lib
     # head_dim*elem not a multiple of 16 bytes
     assert lib.pkv_kv_append(16, 16, 16, 16, 16, 1, 4, 1, 6, 16, 1, None) == binding.INVALID
@@ -185,3 +196,51 @@ def test_binding_rejects_inconsistent_buffers():
         with pytest.raises((ValueError, TypeError)):
             call()
             raise AssertionError("case %d passed" % i)
+
+
+def call_chunk(**over):
+    host_only()
+    a = dict(out=16, q=16, k=16, v=16, bt=16, maxB=4, cl=16, qs=16, S=1, T=2, mq=2, Hq=4, Hkv=4, D=64, bs=16,
+             NB=8, scale=0.0, P=0, ws=None, wsb=0, dt=1, stream=None)
+    a.update(over)
+    return binding.lib.pkv_paged_attention_chunk(a["out"], a["q"], a["k"], a["v"], a["bt"], a["maxB"], a["cl"],
+                                                 a["qs"], a["S"], a["T"], a["mq"], a["Hq"], a["Hkv"], a["D"],
+                                                 a["bs"], a["NB"], a["scale"], a["P"], a["ws"], a["wsb"], a["dt"],
+                                                 a["stream"])
+
+
+@pytest.mark.parametrize("over,status,why", [
+    (dict(dt=0), binding.UNSUPPORTED, "16-bit element types only"),
+    (dict(Hq=64, Hkv=2), binding.INVALID, "1..16 times num_kv_heads"),
+    (dict(mq=0), binding.INVALID, "sizes must be positive"),
+    (dict(qs=None), binding.INVALID, "null pointer"),
+    (dict(maxB=4096, P=16, mq=512, Hq=8, Hkv=1), binding.INVALID, "row tiles x partitions"),
+    (dict(S=0, out=None), binding.OK, ""),
+])
+def test_chunk_validation(over, status, why):
+    assert call_chunk(**over) == status
+    assert why in binding.lib.pkv_last_error().decode()
+
+
+def test_fp8_calls_validation():
+    host_only()
+    lib = binding.lib
+
+    def append(**over):
+        a = dict(T=1, D=64, src=1, ks=1.0, vs=1.0)
+        a.update(over)
+        return lib.pkv_kv_append_fp8(16, 16, 16, 16, 16, a["T"], 4, 1, a["D"], 16, a["src"], a["ks"], a["vs"], None)
+
+    assert append(ks=0.0) == binding.INVALID and "positive and finite" in lib.pkv_last_error().decode()
+    assert append(vs=float("inf")) == binding.INVALID
+    assert append(D=72) == binding.INVALID and "multiple of 16" in lib.pkv_last_error().decode()
+    assert append(src=binding.FP8_E4M3) == binding.INVALID                  # new K/V are 16- or 32-bit
+
+    def decode(**over):
+        a = dict(dt=1, ks=1.0, vs=1.0)
+        a.update(over)
+        return lib.pkv_paged_attention_decode_fp8(16, 16, 16, 16, 16, 4, 16, 1, 4, 4, 64, 16, 8, 0.0, a["ks"],
+                                                  a["vs"], 0, None, 0, a["dt"], None)
+
+    assert decode(dt=0) == binding.UNSUPPORTED                              # fp32 q/out
+    assert decode(ks=-1.0) == binding.INVALID and "positive and finite" in lib.pkv_last_error().decode()
