@@ -55,3 +55,62 @@ def test_plan_fails_before_reserving_anything():
     assert p.lens.tolist() == [12] and ss.table(0)[1] == 12
     p = ss.plan_chunk([0], [20])                                     # exactly 32 tokens: fits
     assert p.lens.tolist() == [32]
+
+
+def test_session_plans_match_the_oracle_allocator_on_random_steps():
+    """Random mixes of add / fork / free / plan / plan_chunk: every plan's
+    slots, copy pairs, padded tables and lengths equal what the oracle
+    allocator gives for the same calls one token at a time; a step that
+    would outgrow max_blocks_per_seq is refused and changes nothing."""
+    import numpy as np
+
+    import oracle
+    bs, max_blocks, NB = 16, 4, 400
+    for seed in range(60):
+        rng = np.random.default_rng(seed)
+        order = rng.permutation(NB).tolist()
+        k = torch.zeros(NB, 1, bs, 64, dtype=torch.bfloat16)
+        ss = pkv.DecodeSession(k, k.clone(), 1, max_blocks, free_order=order, max_batch=16, share_prefixes=False)
+        orc = oracle.Allocator(NB, bs, order)
+        live, next_id = [], 0
+        for _ in range(40):
+            op = rng.choice(["add", "add", "fork", "free", "plan", "plan", "chunk"])
+            if op == "add" or not live:
+                n = int(rng.integers(0, max_blocks * bs + 1))
+                assert ss.add(next_id, n) == (orc.seq_add(next_id), orc.seq_append_slots(next_id, n))[1][1]
+                live.append(next_id)
+                next_id += 1
+            elif op == "fork":
+                p = live[int(rng.integers(len(live)))]
+                ss.fork(p, next_id)
+                orc.seq_fork(p, next_id)
+                live.append(next_id)
+                next_id += 1
+            elif op == "free":
+                sid = live.pop(int(rng.integers(len(live))))
+                ss.free(sid)
+                orc.seq_free(sid)
+            else:
+                ids = [live[i] for i in sorted(rng.choice(len(live), size=int(rng.integers(1, len(live) + 1)),
+                                                          replace=False))]
+                n_new = [1] * len(ids) if op == "plan" else rng.integers(1, 4, size=len(ids)).tolist()
+                lens = {s: orc.seq_block_table(s)[2] for s in ids}
+                too_long = any(-(-(lens[s] + n) // bs) > max_blocks for s, n in zip(ids, n_new))
+                before = [ss.table(s) for s in ids]
+                if too_long:
+                    with pytest.raises(pkv.PagedKVError):
+                        ss.plan(ids) if op == "plan" else ss.plan_chunk(ids, n_new)
+                    assert [ss.table(s) for s in ids] == before
+                    continue
+                p = ss.plan(ids) if op == "plan" else ss.plan_chunk(ids, n_new)
+                slots, pairs = [], []
+                for s, n in zip(ids, n_new):
+                    st, sl, pr = orc.seq_append_slots(s, n)
+                    assert st == 0
+                    slots += sl
+                    pairs += pr
+                assert p.slot_mapping.tolist() == slots, seed
+                assert [tuple(x) for x in p.cow_pairs.tolist()] == [tuple(x) for x in pairs], seed
+                for i, s in enumerate(ids):
+                    _, t, L = orc.seq_block_table(s)
+                    assert p.lens[i] == L and p.block_tables[i].tolist() == t + [-1] * (max_blocks - len(t))
