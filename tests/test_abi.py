@@ -244,3 +244,27 @@ def test_fp8_calls_validation():
 
     assert decode(dt=0) == binding.UNSUPPORTED                              # fp32 q/out
     assert decode(ks=-1.0) == binding.INVALID and "positive and finite" in lib.pkv_last_error().decode()
+
+
+def test_workspace_queries_cover_every_call_random():
+    """For random shapes, the size each workspace query reports holds the
+    partials the call writes under the partition size the library picks:
+    (rows) x (partitions, + 1 slot in shared-prefix mode) x (D + 2) floats
+    whenever a context spans more than one partition."""
+    import numpy as np
+    rng = np.random.default_rng(0)
+    for _ in range(2000):
+        S, Hq = int(rng.integers(1, 300)), int(rng.choice([1, 8, 32, 64]))
+        D = int(rng.choice([64, 128]))
+        max_len = int(rng.integers(1, 4096)) * int(rng.choice([16, 64, 256]))
+        P = int(rng.choice([0, 0, 16, 64, 256, 512, 1024]))
+        eff = pkv.attention_partition_size(S, Hq, 1, D, max_len, P)
+        assert eff > 0 and eff % 16 == 0 and (P == 0 or eff == P)
+        nparts = -(-max_len // eff)
+        per = Hq * (D + 2) * 4
+        ws = pkv.attention_workspace_bytes(S, Hq, D, max_len, P)
+        assert ws >= (S * nparts * per if nparts > 1 else 0)
+        assert pkv.attention_shared_workspace_bytes(S, Hq, D, max_len, P) >= S * (nparts + 1) * per
+        T = S * int(rng.integers(1, 5))
+        cw = pkv.attention_chunk_workspace_bytes(T, Hq, D, max_len, P)
+        assert cw >= (T * nparts * per if nparts > 1 else 0)
