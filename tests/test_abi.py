@@ -268,3 +268,19 @@ def test_workspace_queries_cover_every_call_random():
         T = S * int(rng.integers(1, 5))
         cw = pkv.attention_chunk_workspace_bytes(T, Hq, D, max_len, P)
         assert cw >= (T * nparts * per if nparts > 1 else 0)
+
+
+def test_plain_c_consumer_builds_and_runs(tmp_path):
+    """The header compiles as C99 with warnings as errors, a C program links
+    the library, and its host-only calls (allocator on the pages' worked
+    example, fork and copy-on-write, exhaustion, queries, an empty batch)
+    behave as documented."""
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    libdir = os.path.dirname(binding.LIB_PATH)
+    exe = str(tmp_path / "host_calls")
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(root, "include"),
+                           "-o", exe, os.path.join(root, "tests", "c_abi", "host_calls.c"), "-L", libdir,
+                           "-l:" + os.path.basename(binding.LIB_PATH), "-Wl,-rpath," + libdir])
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
