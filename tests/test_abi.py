@@ -284,3 +284,29 @@ def test_plain_c_consumer_builds_and_runs(tmp_path):
                            "-l:" + os.path.basename(binding.LIB_PATH), "-Wl,-rpath," + libdir])
     r = subprocess.run([exe], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
+
+
+def test_last_error_is_per_thread():
+    """pkv_last_error() describes the last failed call on the calling thread:
+    two threads failing different calls concurrently each read their own
+    message (ctypes releases the GIL inside the calls)."""
+    import threading
+    lib = binding.lib
+    results = {}
+
+    def worker(name, call, expect):
+        ok = True
+        for _ in range(2000):
+            call()
+            ok &= expect in lib.pkv_last_error().decode()
+        results[name] = ok
+
+    a = threading.Thread(target=worker, args=("append", lambda: lib.pkv_kv_append(
+        None, None, None, None, None, -1, 4, 1, 64, 16, 1, None), "pkv_kv_append"))
+    b = threading.Thread(target=worker, args=("alloc", lambda: lib.pkv_alloc_create(0, 16, None),
+                                               "pkv_alloc_create"))
+    a.start()
+    b.start()
+    a.join()
+    b.join()
+    assert results == {"append": True, "alloc": True}
