@@ -111,3 +111,49 @@ def test_reference_arm_prints_one_contract_line():
 def test_warmup_below_three_is_refused():
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "2", "--impl", "reference", "--config", "tiny"])
+
+
+def fake_smi(tmp_path, lines):
+    d = tmp_path / "bin"
+    d.mkdir(exist_ok=True)
+    exe = d / "nvidia-smi"
+    exe.write_text("#!/bin/sh\n" + "".join("echo '%s'\n" % ln for ln in lines) + "exec sleep 30\n")
+    exe.chmod(0o755)
+    return str(d)
+
+
+def test_clock_sampler_reports_median_max_and_active_reasons(tmp_path, monkeypatch):
+    """The clocks object of the bench line from nvidia-smi samples (index,
+    SM clock, max SM clock, power, reason mask, then hw_slowdown,
+    hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap): median SM clock,
+    max clock, every reason seen active, sample count; other lines ignored."""
+    import time
+    monkeypatch.setenv("PATH", fake_smi(tmp_path, [
+        "0, 1965, 1965, 700.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1950, 1965, 710.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1980, 1965, 690.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, [N/A], 1965, 690.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]) + os.pathsep + os.environ["PATH"])
+    c = bench.ClockSampler(0)
+    c.start()
+    time.sleep(0.5)
+    assert c.stop() == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
+
+    monkeypatch.setenv("PATH", fake_smi(tmp_path, [
+        "0, 1400, 1965, 990.0, 0x0000000000000008, Active, Not Active, Not Active, Not Active",
+        "0, 1500, 1965, 990.0, 0x0000000000000020, Not Active, Active, Not Active, Active",
+    ]) + os.pathsep + os.environ["PATH"])
+    c = bench.ClockSampler(0)
+    c.start()
+    time.sleep(0.5)
+    got = c.stop()
+    assert got["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_power_cap"] and got["sm_mhz"] == 1450.0
+
+
+def test_clock_sampler_without_nvidia_smi_reports_nothing(tmp_path, monkeypatch):
+    empty = tmp_path / "empty"
+    empty.mkdir()
+    monkeypatch.setenv("PATH", str(empty))
+    c = bench.ClockSampler(0)
+    c.start()
+    assert c.stop() is None
