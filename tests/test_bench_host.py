@@ -157,3 +157,26 @@ def test_clock_sampler_without_nvidia_smi_reports_nothing(tmp_path, monkeypatch)
     c = bench.ClockSampler(0)
     c.start()
     assert c.stop() is None
+
+
+def test_roofline_peak_and_traffic_lookups(tmp_path, monkeypatch):
+    """The peak comes from MEASURED_PEAKS.json (else the 6.65 TB/s fallback);
+    recorded DRAM traffic is reported only for entries taken on the current
+    kernel sources (their hash), else null."""
+    import json
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.measured_hbm_peak() == (6650.0, "fallback")
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps({"hbm_gbs": 6545.3, "bf16_tflops": 1590}))
+    assert bench.measured_hbm_peak() == (6545.3, "measured")
+
+    csrc = tmp_path / "paged_kv_cache_405_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text("__global__ void k() {}\n")
+    (tmp_path / "profiles").mkdir()
+    h = bench.kernel_source_hash()
+    (tmp_path / "profiles" / "dram_traffic.txt").write_text(
+        "# workload hash bytes note\nllama7b %s 1132961280 note\nllama7b 0000000000000000 1 stale\n" % h)
+    assert bench.recorded_traffic("llama7b") == 1132961280.0
+    assert bench.recorded_traffic("llama13b_prefix") is None
+    (csrc / "k.cu").write_text("__global__ void k() { }\n")      # the kernel changed: the entry is stale
+    assert bench.kernel_source_hash() != h and bench.recorded_traffic("llama7b") is None
