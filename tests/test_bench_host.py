@@ -180,3 +180,15 @@ def test_roofline_peak_and_traffic_lookups(tmp_path, monkeypatch):
     assert bench.recorded_traffic("llama13b_prefix") is None
     (csrc / "k.cu").write_text("__global__ void k() { }\n")      # the kernel changed: the entry is stale
     assert bench.kernel_source_hash() != h and bench.recorded_traffic("llama7b") is None
+
+
+def test_allocator_bench_line():
+    """--allocator-bench (host only): one JSON line with the prefix-cache
+    hit rate and host cost, and the product's counters equal the oracle's on
+    a sample of the same requests."""
+    import argparse
+    d = bench.run_allocator_bench(argparse.Namespace(requests=60))
+    assert d["mode"] == "allocator-bench" and d["requests"] == 60
+    assert 0.5 < d["hit_rate"] <= 1.0 and 0.5 < d["prefill_tokens_skipped_frac"] <= 1.0
+    assert d["host_us_per_call"] > 0 and d["calls"] > 0
+    assert d["oracle"]["same_counters_on_sample"] is True
