@@ -310,3 +310,18 @@ def test_last_error_is_per_thread():
     a.join()
     b.join()
     assert results == {"append": True, "alloc": True}
+
+
+def test_build_tracks_every_source_and_targets_sm100a():
+    """Every CUDA/C++ source and header of the library is a build dependency
+    (an edit rebuilds the library), and the build targets sm_100a only."""
+    import importlib.util
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    spec = importlib.util.spec_from_file_location("_b", os.path.join(root, "paged_kv_cache_405_b200", "build.py"))
+    b = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(b)
+    files = {f for f in os.listdir(b.CSRC) if f.endswith((".cu", ".cuh", ".cpp", ".h"))}
+    assert files <= set(b.DEPS), files - set(b.DEPS)
+    i = b.FLAGS.index("-gencode")
+    assert b.FLAGS[i + 1] == "arch=compute_100a,code=sm_100a" and b.FLAGS.count("-gencode") == 1
+    assert "-lineinfo" in b.FLAGS
