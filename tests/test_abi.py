@@ -325,3 +325,24 @@ def test_build_tracks_every_source_and_targets_sm100a():
     i = b.FLAGS.index("-gencode")
     assert b.FLAGS[i + 1] == "arch=compute_100a,code=sm_100a" and b.FLAGS.count("-gencode") == 1
     assert "-lineinfo" in b.FLAGS
+
+
+def test_product_and_oracle_import_nothing_of_each_other():
+    """The product package loads no part of the oracle and the oracle loads no
+    part of the product (fresh interpreters), and no product source names it."""
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import sys, {mod}\n"
+            "bad = [m for m in sys.modules if m == {other!r} or m.startswith({other!r} + '.')]\n"
+            "assert not bad, bad\n")
+    for mod, other in (("paged_kv_cache_405_b200", "oracle"), ("oracle", "paged_kv_cache_405_b200")):
+        r = subprocess.run([sys.executable, "-c", code.format(mod=mod, other=other)], cwd=root,
+                           capture_output=True, text=True, timeout=120)
+        assert r.returncode == 0, r.stderr[-2000:]
+    pkg = os.path.join(root, "paged_kv_cache_405_b200")
+    for dirpath, _, names in os.walk(pkg):
+        for n in names:
+            if n.endswith((".py", ".cu", ".cuh", ".cpp", ".h")):
+                text = open(os.path.join(dirpath, n), encoding="utf-8").read()
+                assert "import oracle" not in text and "from oracle" not in text and "oracle.c" not in text, n
