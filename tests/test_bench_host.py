@@ -114,12 +114,26 @@ def test_warmup_below_three_is_refused():
 
 
 def fake_smi(tmp_path, lines):
+    """A stand-in nvidia-smi: prints the given sample lines, leaves a marker
+    file once they are out, then waits to be stopped."""
     d = tmp_path / "bin"
     d.mkdir(exist_ok=True)
     exe = d / "nvidia-smi"
-    exe.write_text("#!/bin/sh\n" + "".join("echo '%s'\n" % ln for ln in lines) + "exec sleep 30\n")
+    marker = tmp_path / "printed"
+    if marker.exists():
+        marker.unlink()
+    exe.write_text("#!/bin/sh\n" + "".join("echo '%s'\n" % ln for ln in lines) +
+                   "touch '%s'\nexec sleep 30\n" % marker)
     exe.chmod(0o755)
     return str(d)
+
+
+def wait_printed(tmp_path):
+    import time
+    t0 = time.time()
+    while not (tmp_path / "printed").exists():
+        assert time.time() - t0 < 30, "the stand-in nvidia-smi never ran"
+        time.sleep(0.02)
 
 
 def test_clock_sampler_reports_median_max_and_active_reasons(tmp_path, monkeypatch):
@@ -127,7 +141,6 @@ def test_clock_sampler_reports_median_max_and_active_reasons(tmp_path, monkeypat
     SM clock, max SM clock, power, reason mask, then hw_slowdown,
     hw_thermal_slowdown, sw_thermal_slowdown, sw_power_cap): median SM clock,
     max clock, every reason seen active, sample count; other lines ignored."""
-    import time
     monkeypatch.setenv("PATH", fake_smi(tmp_path, [
         "0, 1965, 1965, 700.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
         "0, 1950, 1965, 710.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
@@ -136,7 +149,7 @@ def test_clock_sampler_reports_median_max_and_active_reasons(tmp_path, monkeypat
     ]) + os.pathsep + os.environ["PATH"])
     c = bench.ClockSampler(0)
     c.start()
-    time.sleep(0.5)
+    wait_printed(tmp_path)
     assert c.stop() == {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"], "samples": 3}
 
     monkeypatch.setenv("PATH", fake_smi(tmp_path, [
@@ -145,7 +158,7 @@ def test_clock_sampler_reports_median_max_and_active_reasons(tmp_path, monkeypat
     ]) + os.pathsep + os.environ["PATH"])
     c = bench.ClockSampler(0)
     c.start()
-    time.sleep(0.5)
+    wait_printed(tmp_path)
     got = c.stop()
     assert got["reasons"] == ["hw_slowdown", "hw_thermal_slowdown", "sw_power_cap"] and got["sm_mhz"] == 1450.0
 
