@@ -194,3 +194,55 @@ def test_quantizer_pins_catch_planted_mistake(name, monkeypatch):
             caught = True
             break
     assert caught, "no pin caught: %s" % name
+
+
+# Planted mistakes in the oracle's Python helpers (oracle/__init__.py):
+# (function, text, replacement, the pins expected to catch it).
+PY_MUTANTS = {
+    "append writes V into K": ("kv_append", "        k_pool[blk, :, off, :] = k_new[i]\n",
+                               "        k_pool[blk, :, off, :] = v_new[i]\n",
+                               ["test_worked_example_kv_append_lands_in_block_9"]),
+    "append writes at negative slots": ("kv_append", "        if sl < 0:\n            continue\n", "",
+                                        ["test_worked_example_kv_append_lands_in_block_9"]),
+    "copy moves only K": ("block_copy", "    v_pool[dst] = vs\n", "", ["test_block_copy_copies_only_that_block"]),
+    "FP8 append writes at negative slots": ("kv_append_fp8", "        if sl < 0:\n            continue\n", "",
+                                            ["test_fp8_append_places_torch_codes_at_the_slots"]),
+    "FP8 append puts V codes in the K pool": ("kv_append_fp8", "        k_codes[blk, :, off, :] = kq[i]\n",
+                                              "        k_codes[blk, :, off, :] = vq[i]\n",
+                                              ["test_fp8_append_places_torch_codes_at_the_slots"]),
+}
+
+
+@pytest.mark.parametrize("name", list(PY_MUTANTS))
+def test_python_helper_pins_catch_planted_mistake(name, monkeypatch):
+    import inspect
+    import textwrap
+
+    import oracle
+    import test_oracle_pins as pins
+    fn, old, new, pin_names = PY_MUTANTS[name]
+    src = textwrap.dedent(inspect.getsource(getattr(oracle, fn)))
+    assert src.count(old) == 1, "the planted mistake must replace exactly one place"
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), "oracle_helper_mutant", "exec"), ns)
+    monkeypatch.setattr(oracle, fn, ns[fn])
+    caught = False
+    for pin in pin_names:
+        try:
+            getattr(pins, pin)()
+        except (AssertionError, IndexError, ValueError):
+            caught = True
+    assert caught, "no pin caught: %s" % name
+
+
+def test_swapped_dtype_codes_are_caught(monkeypatch):
+    """The oracle tells its C code the element type by a code; swapping the
+    bf16 and f16 codes is caught by the exact-widening pin."""
+    import torch
+
+    import oracle
+    import test_oracle_pins as pins
+    monkeypatch.setitem(oracle._DT, torch.bfloat16, 2)
+    monkeypatch.setitem(oracle._DT, torch.float16, 1)
+    with pytest.raises(AssertionError):
+        pins.test_narrow_types_widen_exactly(torch.bfloat16)

@@ -511,6 +511,31 @@ def test_e4m3_quantize_matches_torch_cast_and_saturates(scale):
     assert np.array_equal(np.sign(table[codes[out]]), np.sign(y.numpy()[out]))
 
 
+def test_fp8_append_places_torch_codes_at_the_slots():
+    """Each new token's K and V, cast by torch's float8_e4m3fn after the
+    x * fp32(1/scale) product, land at their slots (block slot // bs, offset
+    slot % bs, every kv head); negative slots write nothing; every other code
+    is untouched."""
+    NB, Hkv, bs, D = 6, 2, 16, 32
+    g = torch.Generator().manual_seed(11)
+    kn = torch.randn(5, Hkv, D, generator=g) * 10
+    vn = torch.randn(5, Hkv, D, generator=g) * 3
+    slots = [3, -1, 40, 95, -7]
+    ks, vs = 0.25, 0.0625
+    kc = np.full((NB, Hkv, bs, D), 0x55, np.uint8)
+    vc = np.full((NB, Hkv, bs, D), 0x55, np.uint8)
+    oracle.kv_append_fp8(kc, vc, kn, vn, ks, vs, slots)
+    ek = np.full_like(kc, 0x55)
+    ev = np.full_like(vc, 0x55)
+    for i, sl in enumerate(slots):
+        if sl < 0:
+            continue
+        for codes, x, sc in ((ek, kn, ks), (ev, vn, vs)):
+            y = x[i].float() * (torch.tensor(1.0) / torch.tensor(sc, dtype=torch.float32))
+            codes[sl // bs, :, sl % bs, :] = y.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(kc, ek) and np.array_equal(vc, ev)
+
+
 def test_fp8_attention_equals_attention_on_dequantized_values():
     """Pools of codes with power-of-two scales == the same values held as fp32."""
     b = synth.make_batch(synth.shrink(synth.CONFIGS["llama3_gqa_bs16"], S=3, Hq=8, Hkv=2, D=64,
