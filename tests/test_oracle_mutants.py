@@ -210,6 +210,18 @@ PY_MUTANTS = {
     "FP8 append puts V codes in the K pool": ("kv_append_fp8", "        k_codes[blk, :, off, :] = kq[i]\n",
                                               "        k_codes[blk, :, off, :] = vq[i]\n",
                                               ["test_fp8_append_places_torch_codes_at_the_slots"]),
+    "FP8 K and V scales swapped": ("paged_attention_kv", "float(np.float32(k_scale)),\n        float(np.float32(v_scale))",
+                                   "float(np.float32(v_scale)),\n        float(np.float32(k_scale))",
+                                   ["test_fp8_attention_equals_attention_on_dequantized_values"]),
+    "default scale 1/D": ("paged_attention", "        scale = 1.0 / math.sqrt(D)\n", "        scale = 1.0 / D\n",
+                          ["test_two_token_closed_form_pins_scale_and_sign"]),
+    "chunk default scale 1/D": ("paged_attention_chunk", "        scale = 1.0 / math.sqrt(D)\n",
+                                "        scale = 1.0 / D\n", [("test_chunk_equals_sdpa_with_causal_mask",
+                                                                  ("float32", 4, 4, 64, 16))]),
+    "sampled items' row and head swapped": ("paged_attention",
+                                            "    its_s = np.ascontiguousarray(its[:, 0])\n    its_h = np.ascontiguousarray(its[:, 1])\n",
+                                            "    its_s = np.ascontiguousarray(its[:, 1])\n    its_h = np.ascontiguousarray(its[:, 0])\n",
+                                            [("test_contiguous_equals_sdpa", ("float32", 4, 4, 64, 16, 35))]),
 }
 
 
@@ -217,6 +229,8 @@ PY_MUTANTS = {
 def test_python_helper_pins_catch_planted_mistake(name, monkeypatch):
     import inspect
     import textwrap
+
+    import torch
 
     import oracle
     import test_oracle_pins as pins
@@ -228,8 +242,10 @@ def test_python_helper_pins_catch_planted_mistake(name, monkeypatch):
     monkeypatch.setattr(oracle, fn, ns[fn])
     caught = False
     for pin in pin_names:
+        pin, args = (pin, ()) if isinstance(pin, str) else pin
+        args = tuple(getattr(torch, a) if isinstance(a, str) else a for a in args)
         try:
-            getattr(pins, pin)()
+            getattr(pins, pin)(*args)
         except (AssertionError, IndexError, ValueError):
             caught = True
     assert caught, "no pin caught: %s" % name
