@@ -91,6 +91,29 @@ def test_worked_example_kv_append_lands_in_block_9():
     assert all(r == [9, 3] for r in changed)
 
 
+def test_tiny_decode_step_allocates_only_where_the_last_block_is_full():
+    """The tiny workload's decode step (lengths before the step 35, 16, 1, 50;
+    the step appends token L of each sequence): only sequence 1, whose single
+    block is full, takes a fresh block -- the front of the free pool -- while
+    the others write into their partly filled last block at offset L mod 16
+    (aiknowledge.cn 2.2.3: a new block only once the last one is full)."""
+    b = synth.make_batch(synth.CONFIGS["tiny"])
+    a = Allocator(b.num_blocks, 16, b.free_order)
+    for s in range(4):
+        assert a.seq_add(s) == OK and a.seq_append_slots(s, int(b.lens[s]))[0] == OK
+    tables = [a.seq_block_table(s)[1] for s in range(4)]
+    front, free_before = a.free[0], len(a.free)
+    got = [a.seq_append_slots(s, 1) for s in range(4)]
+    assert all(st == OK and pairs == [] for st, _, pairs in got)
+    slots = [sl[0] for _, sl, _ in got]
+    assert slots[0] == 9 * 16 + 3                                # block 9 of the worked example, offset 35 mod 16
+    assert slots[1] == front * 16 and a.seq_block_table(1)[1] == tables[1] + [front]
+    assert slots[2] == tables[2][0] * 16 + 1
+    assert slots[3] == tables[3][3] * 16 + 50 % 16
+    assert len(a.free) == free_before - 1
+    assert [a.seq_block_table(s)[2] for s in range(4)] == [36, 17, 2, 51]
+
+
 def test_block_copy_copies_only_that_block():
     b = synth.make_batch(synth.CONFIGS["tiny"])
     k, v = b.k_pool.clone(), b.v_pool.clone()
