@@ -727,21 +727,24 @@ def run_allocator_bench(args):
 
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", default="llama7b", choices=sorted(synth.CONFIGS))
-    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--partition-size", type=int, default=0)
+    ap.add_argument("--gpus", type=int, default=1, help="GPUs (one rank each under torchrun; replicas, weak scaling)")
+    ap.add_argument("--steps", type=int, default=20, help="timed decode steps")
+    ap.add_argument("--warmup", type=int, default=5, help="untimed warm-up steps (at least 3)")
+    ap.add_argument("--config", default="llama7b", choices=sorted(synth.CONFIGS), help="workload (see synth.CONFIGS)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"],
+                    help="ours: the CUDA library; reference: the CPU oracle on the host cores")
+    ap.add_argument("--partition-size", type=int, default=0,
+                    help="split-K partition in tokens (0: the workload's, else the library's choice)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (small cases for profiling)")
-    ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
-    ap.add_argument("--reference-step-seconds", type=float, default=3.0)
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg from host buffers")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle sample length (all cores)")
+    ap.add_argument("--reference-step-seconds", type=float, default=3.0,
+                    help="CPU-oracle work per step of --impl reference")
     ap.add_argument("--allocator-bench", action="store_true",
                     help="host-only prefix-caching allocator simulation (prints its own JSON line)")
-    ap.add_argument("--requests", type=int, default=2000)
+    ap.add_argument("--requests", type=int, default=2000, help="requests of --allocator-bench")
     ap.add_argument("--nvtx", action="store_true",
                     help="NVTX ranges around each step and each library call (e.g. for ncu --nvtx filters)")
     ap.add_argument("--clock-warm-s", type=float, default=0.5,
