@@ -142,9 +142,23 @@ CACHE_MUTANTS = {
     "lookups counted in tokens": ("self.lookups += len(toks) // bs", "self.lookups += len(toks)"),
     "chain restarts after the cached blocks": ("        self.chain[sid] = node\n        st, slots, _",
                                                "        self.chain[sid] = self.ROOT\n        st, slots, _"),
+    "revived block left in the LRU list": ("            if self.ref[b] == 0:\n                self.lru.remove(b)\n",
+                                           "            pass\n"),
+    "counters bumped by a refused prompt": (
+        "        if st != OK:\n            self._restore(snap)\n            return st, 0, []\n        self.lookups",
+        "        if st != OK:\n            self._restore(snap)\n            self.lookups += 1\n            return st, 0, []\n"
+        "        self.lookups"),
+    "evicted before the free queue is empty": ("        if self.free:\n            return self.free.popleft()\n",
+                                               "        if self.free and not self.lru:\n            return self.free.popleft()\n"),
+    "eviction keeps the key": ("            del self.cache[self.key_of.pop(b)]\n", "            self.key_of.pop(b)\n"),
+    "released blocks at the front of the LRU list": ("            if b in self.key_of:\n                self.lru.append(b)",
+                                                      "            if b in self.key_of:\n                self.lru.insert(0, b)"),
+    "fork drops the token ids": ("            self.tokens[child] = None if t is None else list(t)\n",
+                                 "            self.tokens[child] = None\n"),
 }
 CACHE_PINS = ["test_caching_oracle_payload_model", "test_hit_counts_closed_form",
-              "test_freed_cached_blocks_are_evicted_oldest_first", "test_prompt_that_does_not_fit_changes_nothing"]
+              "test_freed_cached_blocks_are_evicted_oldest_first", "test_prompt_that_does_not_fit_changes_nothing",
+              "test_forked_sequence_keeps_registering_its_blocks"]
 
 
 @pytest.mark.parametrize("name", list(CACHE_MUTANTS))

@@ -136,6 +136,20 @@ def test_freed_cached_blocks_are_evicted_oldest_first():
     assert st == NO_FREE_BLOCK or n_cached == 0
 
 
+def test_forked_sequence_keeps_registering_its_blocks():
+    """A fork inherits the parent's token ids, so a block the child fills with
+    known tokens is cached too: a later prompt equal to the child's tokens
+    finds both full blocks."""
+    a = CachingAllocator(16, 2)
+    st, n_cached, _ = a.seq_add_with_prompt(0, [1, 2, 3])     # [1, 2] cached, [3] partly filled
+    assert st == OK and n_cached == 0
+    assert a.seq_fork(0, 1) == OK
+    st, slots, pairs = a.seq_append_tokens(1, [4])             # the child's write copies the shared block
+    assert st == OK and len(pairs) == 1
+    st, n_cached, _ = a.seq_add_with_prompt(2, [1, 2, 3, 4, 5])
+    assert st == OK and n_cached == 4
+
+
 def test_prompt_that_does_not_fit_changes_nothing():
     a = CachingAllocator(3, 2)
     a.seq_add_with_prompt(0, [1, 2, 3, 4])
