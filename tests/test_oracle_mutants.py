@@ -79,7 +79,22 @@ ALLOC_MUTANTS = {
     "freed blocks to the front": ("self.free.append(b)", "self.free.appendleft(b)", 0),
     "freed in reverse table order": ("        bt, _ = self.seqs.pop(sid)\n        for b in bt:",
                                      "        bt, _ = self.seqs.pop(sid)\n        for b in reversed(bt):", 0),
+    "share without refcounts": ("        for b in blocks:\n            self.ref[b] += 1\n",
+                                "        for b in blocks:\n            pass\n", 0),
+    "copy pair reversed": ("pairs.append((bt[j], b))", "pairs.append((b, bt[j]))", 0),
+    "copy keeps the old block's count": ("                self.ref[bt[j]] -= 1\n", "", 0),
+    "fork child starts empty": ("        self.seqs[child] = [list(bt), n]", "        self.seqs[child] = [list(bt), 0]", 0),
+    "failed append not rolled back": ("                if not self.free:\n                    self._restore(snap)\n",
+                                      "                if not self.free:\n", 0),
+    "failure not counted": ("                    self.alloc_failures += 1\n", "", 0),
+    "copies not counted": ("                self.cow_copies += 1\n", "", 0),
+    "slot in the table's first block": ("            slots.append(bt[j] * bs + t % bs)",
+                                        "            slots.append(bt[0] * bs + t % bs)", 0),
 }
+# closed-form allocator pins tried when the brute-force model does not catch a mistake
+ALLOC_PINS = ["test_worked_example_allocator_growth", "test_allocator_exhaustion_is_atomic",
+              "test_fork_then_append_copies_partial_block_once_per_writer",
+              "test_free_queue_takes_from_the_front_and_frees_to_the_back_in_table_order"]
 
 
 def _mutant_allocator_module(old, new, which):
@@ -113,14 +128,16 @@ def test_allocator_pins_catch_planted_mistake(name):
         except (AssertionError, IndexError, KeyError, ValueError):
             caught = True
             break
-    if not caught:              # the free-queue order is pinned by a closed-form case
+    if not caught:              # counters and the free-queue order are pinned by closed-form cases
         import test_oracle_pins as pins
         saved = pins.Allocator
         pins.Allocator = Broken
         try:
-            pins.test_free_queue_takes_from_the_front_and_frees_to_the_back_in_table_order()
-        except AssertionError:
-            caught = True
+            for pin in ALLOC_PINS:
+                try:
+                    getattr(pins, pin)()
+                except (AssertionError, IndexError, KeyError, ValueError):
+                    caught = True
         finally:
             pins.Allocator = saved
     assert caught, "no pin caught: %s" % name

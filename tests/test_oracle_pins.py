@@ -441,6 +441,7 @@ def test_fork_then_append_copies_partial_block_once_per_writer():
     assert all(p[0][0] == last for p in copies[:3])
     assert a.refcount(last) == 1 and a.seqs[0][0][1] == last
     assert a.refcount(a.seqs[0][0][0]) == 4                # full blocks stay shared
+    assert a.stats()["cow_copies"] == 3                     # the monitoring counter counts each copy
 
 
 # ------------------------------------------------ chunks of new tokens (causal)
