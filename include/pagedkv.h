@@ -110,8 +110,8 @@ int pkv_attention_partition_size(int num_seqs, int num_q_heads, int num_kv_heads
 /*
  * pkv_paged_attention_decode -- one query token per sequence attends to its
  * cached tokens, read block by block through its block table
- * ([E] 4.2 "the kernel reads KV at block granularity via the block table";
- *  [T] 2.2.4 fused over non-contiguous blocks).  For sequence s, query head h:
+ * ([E] 4.2: the kernel reads the KV cache block by block through the block
+ *  table; [T] 2.2.4 fused over non-contiguous blocks).  For sequence s, query head h:
  *     g   = h / (num_q_heads / num_kv_heads)   (grouped-query attention)
  *     x_t = scale * q[s,h,:] . K[slot(s,t), g, :],  t < context_lens[s]
  *     out[s,h,:] = sum_t softmax(x)_t V[slot(s,t), g, :]
@@ -405,6 +405,9 @@ pkv_status pkv_seq_block_tables_batch(const pkv_alloc* a, const int64_t* seq_ids
  * free; a fresh block comes from the free queue first, then by evicting the
  * oldest evictable block.  Appending without token ids (pkv_seq_append_slots,
  * _batch) or sharing by block list stops a sequence from registering blocks.
+ * A cached block is never written in place: a sequence that holds one with
+ * fewer of its tokens (a prefix shared part-way into it) gets a copy-on-write
+ * pair for it, as when another sequence holds it.
  */
 pkv_status pkv_alloc_set_prefix_caching(pkv_alloc* a, int enable);
 

@@ -171,6 +171,9 @@ class CachingAllocator(Allocator):
       back of an LRU list) instead of returning to the free queue; a fresh
       block comes from the free queue first, then by evicting the front of
       the LRU list, which drops its key;
+    * a cached block is never written in place: a sequence that holds one
+      with fewer of its tokens (a prefix shared part-way into it) copies it
+      before writing, as a writer of a shared block does;
     * lookups/hits are counted in full blocks of the prompts looked up.
     """
 
@@ -285,7 +288,7 @@ class CachingAllocator(Allocator):
                     return NO_FREE_BLOCK, [], []
                 self.ref[b] = 1
                 bt.append(b)
-            elif self.ref[bt[j]] > 1:
+            elif self.ref[bt[j]] > 1 or bt[j] in self.key_of:   # shared, or cached: copy first
                 b = self._take()
                 if b is None:
                     self._restore(snap)

@@ -80,6 +80,12 @@ struct pkv_alloc {
 
     int64_t available() const { return (int64_t)free_q.size() + (int64_t)lru.size(); }
 
+    // A write into block b goes to a private copy when another sequence holds
+    // b, or when b is cached: a cached block's tokens are never overwritten
+    // (a sequence can hold a cached block with fewer of its tokens when it
+    // was given a prefix that ends part-way into it).
+    bool must_copy(int32_t b) const { return ref[b] > 1 || node_of[b] >= 0; }
+
     // A fresh block: the free queue's front, else the least recently released
     // cached block (its key is dropped).  Callers check available() first.
     int32_t take() {
@@ -234,7 +240,7 @@ static pkv_status append_impl(pkv_alloc* a, pkv_alloc::Seq& s, int ntok, const i
     const int64_t L = s.len;
     // Only the first new token can land in an existing block (the partly
     // filled last one); it needs a private copy if that block is shared.
-    bool cow = ntok > 0 && (L % bs) != 0 && a->ref[s.table[L / bs]] > 1;
+    bool cow = ntok > 0 && (L % bs) != 0 && a->must_copy(s.table[L / bs]);
     int64_t fresh = ceil_div(L + ntok, bs) - (int64_t)s.table.size();
     int64_t need = fresh + (cow ? 1 : 0);
     if (cow && (cow_cap < 1 || !cow_out)) {
@@ -253,7 +259,7 @@ static pkv_status append_impl(pkv_alloc* a, pkv_alloc::Seq& s, int ntok, const i
             int32_t b = a->take();
             a->ref[b] = 1;
             s.table.push_back(b);
-        } else if (a->ref[s.table[j]] > 1) {
+        } else if (a->must_copy(s.table[j])) {
             int32_t src = s.table[j];
             int32_t dst = a->take();
             cow_out[2 * ncow] = src;
@@ -400,7 +406,7 @@ pkv_status pkv_seq_append_slots_batch(pkv_alloc* a, const int64_t* seq_ids, int 
         } else if (k == 0) {
             const int32_t b = s.table[L / bs];
             int32_t& drop = ref_drop[b];
-            if (a->ref[b] - drop > 1) {  // still shared when this sequence writes
+            if (a->ref[b] - drop > 1 || a->node_of[b] >= 0) {  // still shared, or cached, when this sequence writes
                 need += 1;
                 ncow += 1;
                 drop += 1;

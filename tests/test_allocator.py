@@ -9,7 +9,7 @@ import pytest
 import oracle
 import synth
 from paged_kv_cache_405_b200 import BlockAllocator
-from oracle.allocator import OK, INVALID, NO_FREE_BLOCK
+from oracle.allocator import INVALID, NO_FREE_BLOCK, OK, CachingAllocator
 
 
 def compare(prod: BlockAllocator, orc: oracle.Allocator, sids):
@@ -215,3 +215,42 @@ def test_shared_prefix_layout_is_one_group():
     b = synth.make_batch(synth.shrink(synth.CONFIGS["llama13b_prefix"], D=64, Hq=1, Hkv=1))
     gf, gs = pkv.find_shared_prefix_groups(b.block_tables, b.lens, 16, 4)
     assert gf.tolist() == [0, 256] and gs.tolist() == [512]
+
+
+def test_batch_calls_equal_sequential_calls_with_cached_blocks():
+    """Caching mode: sequences given a prefix that ends part-way into a cached
+    block copy it before writing (a cached block is never written in place);
+    the batched step call equals one call per sequence, product and oracle."""
+    for seed in range(300):
+        rng = np.random.default_rng(seed)
+        bs = (2, 4)[seed % 2]
+        nb = 14 + seed % 5
+        prompt = [int(x) for x in rng.integers(0, 3, size=3 * bs)]
+        ntok = int(rng.integers(1, 3 * bs))                 # often ends inside a full, cached block
+        a1 = BlockAllocator(nb, bs, prefix_caching=True)
+        a2 = BlockAllocator(nb, bs, prefix_caching=True)
+        o = CachingAllocator(nb, bs)
+        for a in (a1, a2, o):
+            assert a.seq_add_with_prompt(0, prompt)[0] == OK
+            blocks = a.seq_block_table(0)[1][:-(-ntok // bs)]
+            for s in (1, 2, 3):
+                assert a.seq_add(s) == OK and a.seq_share_prefix(s, blocks, ntok) == OK
+            if seed % 3:
+                assert a.seq_free(0) == OK                  # the sharers (and the cache) hold the blocks
+        ids = [int(x) for x in rng.integers(1, 4, size=int(rng.integers(1, 7)))]
+        st, slots, pairs = a1.seq_append_slots_batch(ids)
+        seq = [a2.seq_append_slots(i, 1) for i in ids]
+        oseq = [o.seq_append_slots(i, 1) for i in ids]
+        assert seq == oseq, seed
+        if all(r[0] == OK for r in seq):
+            assert st == OK
+            assert slots.tolist() == [r[1][0] for r in seq]
+            assert [tuple(p) for p in pairs.tolist()] == [p for r in seq for p in r[2]]
+            written = {r[1][0] // bs for r in seq}
+            cached = set(o.key_of)
+            assert not (written & cached), seed               # no write lands in a cached block
+        else:
+            assert st == next(r[0] for r in seq if r[0] != OK) and slots.size == 0
+        for s in (1, 2, 3):
+            assert a1.seq_block_table(s) == a2.seq_block_table(s)
+        assert a1.cache_stats() == a2.cache_stats() == o.cache_stats()

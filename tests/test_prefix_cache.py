@@ -14,7 +14,7 @@ def caching_ops(seed, n_ops, max_seqs=5, vocab=3):
     stems = [list(rng.integers(0, vocab, size=int(rng.integers(0, 9)))) for _ in range(3)]
     ops = []
     for _ in range(n_ops):
-        k = rng.choice(["prompt", "prompt", "tokens", "tokens", "slots", "fork", "free", "free"])
+        k = rng.choice(["prompt", "prompt", "tokens", "tokens", "slots", "fork", "share", "free", "free"])
         a = int(rng.integers(0, max_seqs))
         if k == "prompt":
             toks = list(stems[int(rng.integers(0, 3))]) + list(rng.integers(0, vocab, size=int(rng.integers(0, 4))))
@@ -25,6 +25,8 @@ def caching_ops(seed, n_ops, max_seqs=5, vocab=3):
             ops.append(("slots", a, int(rng.integers(1, 3))))
         elif k == "fork":
             ops.append(("fork", a, int(rng.integers(0, max_seqs))))
+        elif k == "share":    # register a, then map it onto donor's first ntok tokens
+            ops.append(("share", a, int(rng.integers(0, max_seqs)), int(rng.integers(1, 6))))
         else:
             ops.append(("free", a))
     return ops
@@ -40,6 +42,18 @@ def apply(a, op):
         return a.seq_append_slots(op[1], op[2])
     if k == "fork":
         return a.seq_fork(op[1], op[2])
+    if k == "share":
+        sid, donor, ntok = op[1], op[2], op[3]
+        st, bt, n = a.seq_block_table(donor)
+        if st != OK or ntok > n:
+            return INVALID
+        st = a.seq_add(sid)
+        if st != OK:
+            return st
+        st = a.seq_share_prefix(sid, bt[:-(-ntok // a.block_size)], ntok)
+        if st != OK:
+            a.seq_free(sid)
+        return st
     return a.seq_free(op[1])
 
 
@@ -90,6 +104,8 @@ def run(a, ops):
             model[op[1]] = before + list(toks)
         elif k == "fork" and r == OK:
             model[op[2]] = list(model[op[1]])
+        elif k == "share" and r == OK:
+            model[op[1]] = list(model[op[2]][:op[3]])
         elif k == "free" and r == OK:
             del model[op[1]]
         check(a, model, data)
