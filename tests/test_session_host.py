@@ -114,3 +114,64 @@ def test_session_plans_match_the_oracle_allocator_on_random_steps():
                 for i, s in enumerate(ids):
                     _, t, L = orc.seq_block_table(s)
                     assert p.lens[i] == L and p.block_tables[i].tolist() == t + [-1] * (max_blocks - len(t))
+
+
+def test_caching_session_matches_the_oracle_on_random_steps():
+    """A DecodeSession with prefix caching: random prompts (a few shared
+    stems), decode steps, forks and frees give the caching oracle's cached
+    token counts, slots, copy pairs, tables and cache counters."""
+    import numpy as np
+
+    from oracle.allocator import CachingAllocator
+    bs, max_blocks, NB = 16, 8, 48
+    for seed in range(40):
+        rng = np.random.default_rng(seed)
+        stems = [rng.integers(0, 4, size=int(rng.integers(0, 3 * bs))).tolist() for _ in range(3)]
+        order = rng.permutation(NB).tolist()
+        k = torch.zeros(NB, 1, bs, 64, dtype=torch.bfloat16)
+        ss = pkv.DecodeSession(k, k.clone(), 1, max_blocks, free_order=order, max_batch=8, share_prefixes=False,
+                               prefix_caching=True)
+        orc = CachingAllocator(NB, bs, order)
+        live, next_id = [], 0
+        for _ in range(30):
+            op = rng.choice(["prompt", "prompt", "plan", "plan", "fork", "free"])
+            if op == "prompt" or not live:
+                toks = stems[int(rng.integers(3))] + rng.integers(0, 4, size=int(rng.integers(1, bs))).tolist()
+                st, n_cached, oslots = orc.seq_add_with_prompt(next_id, toks)
+                if st != 0:
+                    with pytest.raises(pkv.PagedKVError):
+                        ss.add_prompt(next_id, toks)
+                    continue
+                got_n, got_slots = ss.add_prompt(next_id, toks)
+                assert (got_n, got_slots.tolist()) == (n_cached, oslots), seed
+                live.append(next_id)
+                next_id += 1
+            elif op == "fork":
+                p = live[int(rng.integers(len(live)))]
+                ss.fork(p, next_id)
+                orc.seq_fork(p, next_id)
+                live.append(next_id)
+                next_id += 1
+            elif op == "free":
+                sid = live.pop(int(rng.integers(len(live))))
+                ss.free(sid)
+                orc.seq_free(sid)
+            else:
+                ids = [live[i] for i in sorted(rng.choice(len(live), size=int(rng.integers(1, len(live) + 1)),
+                                                          replace=False))]
+                lens = {s: orc.seq_block_table(s)[2] for s in ids}
+                need = sum(1 for s in ids if lens[s] % bs == 0) + len(ids)
+                if any(-(-(lens[s] + 1) // bs) > max_blocks for s in ids) or need > orc.stats()["free_blocks"]:
+                    continue                                  # keep to steps both sides can take
+                p = ss.plan(ids)
+                slots, pairs = [], []
+                for s in ids:
+                    st, sl, pr = orc.seq_append_slots(s, 1)
+                    assert st == 0
+                    slots += sl
+                    pairs += pr
+                assert p.slot_mapping.tolist() == slots and [tuple(x) for x in p.cow_pairs.tolist()] == pairs, seed
+                for i, s in enumerate(ids):
+                    _, t, L = orc.seq_block_table(s)
+                    assert p.lens[i] == L and p.block_tables[i].tolist() == t + [-1] * (max_blocks - len(t))
+            assert ss.cache_stats() == orc.cache_stats(), seed
