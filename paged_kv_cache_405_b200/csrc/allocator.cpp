@@ -242,12 +242,19 @@ static pkv_status append_impl(pkv_alloc* a, pkv_alloc::Seq& s, int ntok, const i
     // filled last one); it needs a private copy if that block is shared.
     bool cow = ntok > 0 && (L % bs) != 0 && a->must_copy(s.table[L / bs]);
     int64_t fresh = ceil_div(L + ntok, bs) - (int64_t)s.table.size();
-    int64_t need = fresh + (cow ? 1 : 0);
     if (cow && (cow_cap < 1 || !cow_out)) {
         set_error("pkv_seq_append_slots: a copy-on-write pair is due but cow_cap < 1");
         return PKV_ERR_INVALID;
     }
-    if (need > a->available()) {
+    // The copy is taken first; when this sequence was the last holder of the
+    // (cached) original, the original becomes evictable for the fresh blocks.
+    int64_t avail = a->available();
+    bool short_of_blocks = false;
+    if (cow) {
+        if (avail == 0) short_of_blocks = true;
+        else avail += (a->ref[s.table[L / bs]] == 1) ? 0 : -1;
+    }
+    if (short_of_blocks || fresh > avail) {
         a->alloc_failures += 1;
         set_error("pkv_seq_append_slots: free pool exhausted");
         return PKV_ERR_NO_FREE_BLOCK;
@@ -386,11 +393,14 @@ pkv_status pkv_seq_append_slots_batch(pkv_alloc* a, const int64_t* seq_ids, int 
         set_error("pkv_seq_append_slots_batch: bad arguments");
         return PKV_ERR_INVALID;
     }
-    // Dry run: count the blocks and copy pairs the whole batch needs.  A
-    // sequence listed twice sees its own first reservation (its length grows).
+    // Dry run, in call order: every block the batch takes must be available
+    // when it is taken.  A sequence listed twice sees its own first
+    // reservation (its length grows); a copy made by the last holder of a
+    // cached block leaves that block evictable, so later takes may use it.
     std::unordered_map<int64_t, int64_t> extra;      // tokens already reserved in this call
-    std::unordered_map<int32_t, int32_t> ref_drop;   // copies already made of a shared block
-    int64_t need = 0, ncow = 0;
+    std::unordered_map<int32_t, int32_t> ref_drop;   // references given up by copies made in this call
+    int64_t avail = a->available(), ncow = 0;
+    bool short_of_blocks = false;
     for (int i = 0; i < n; ++i) {
         auto it = a->seqs.find(seq_ids[i]);
         if (it == a->seqs.end()) {
@@ -401,15 +411,19 @@ pkv_status pkv_seq_append_slots_batch(pkv_alloc* a, const int64_t* seq_ids, int 
         const int64_t bs = a->block_size;
         int64_t& k = extra[seq_ids[i]];
         const int64_t L = s.len + k;
-        if (L % bs == 0) {
-            need += 1;
+        if (L % bs == 0) {  // a fresh block
+            if (avail == 0) short_of_blocks = true;
+            else avail -= 1;
         } else if (k == 0) {
             const int32_t b = s.table[L / bs];
             int32_t& drop = ref_drop[b];
-            if (a->ref[b] - drop > 1 || a->node_of[b] >= 0) {  // still shared, or cached, when this sequence writes
-                need += 1;
+            const int32_t holders = a->ref[b] - drop;
+            if (holders > 1 || a->node_of[b] >= 0) {  // still shared, or cached, when this sequence writes
+                if (avail == 0) short_of_blocks = true;
+                else avail -= 1;
                 ncow += 1;
                 drop += 1;
+                if (holders == 1) avail += 1;  // the cached original is released, evictable from now on
             }
         }
         k += 1;
@@ -418,7 +432,7 @@ pkv_status pkv_seq_append_slots_batch(pkv_alloc* a, const int64_t* seq_ids, int 
         set_error("pkv_seq_append_slots_batch: cow_cap too small");
         return PKV_ERR_INVALID;
     }
-    if (need > a->available()) {
+    if (short_of_blocks) {
         a->alloc_failures += 1;
         set_error("pkv_seq_append_slots_batch: free pool exhausted");
         return PKV_ERR_NO_FREE_BLOCK;

@@ -220,12 +220,15 @@ def test_shared_prefix_layout_is_one_group():
 def test_batch_calls_equal_sequential_calls_with_cached_blocks():
     """Caching mode: sequences given a prefix that ends part-way into a cached
     block copy it before writing (a cached block is never written in place);
-    the batched step call equals one call per sequence, product and oracle."""
-    for seed in range(300):
+    the batched step call equals one call per sequence, product and oracle,
+    and on a pool too small for all the copies it fails as a whole, changing
+    nothing but the failure count."""
+    n_fail = 0
+    for seed in range(400):
         rng = np.random.default_rng(seed)
         bs = (2, 4)[seed % 2]
-        nb = 14 + seed % 5
         prompt = [int(x) for x in rng.integers(0, 3, size=3 * bs)]
+        nb = 3 + int(rng.integers(0, 5))                   # the prompt's 3 blocks + a few free ones
         ntok = int(rng.integers(1, 3 * bs))                 # often ends inside a full, cached block
         a1 = BlockAllocator(nb, bs, prefix_caching=True)
         a2 = BlockAllocator(nb, bs, prefix_caching=True)
@@ -237,20 +240,28 @@ def test_batch_calls_equal_sequential_calls_with_cached_blocks():
                 assert a.seq_add(s) == OK and a.seq_share_prefix(s, blocks, ntok) == OK
             if seed % 3:
                 assert a.seq_free(0) == OK                  # the sharers (and the cache) hold the blocks
+        before = ([a1.seq_block_table(s) for s in (1, 2, 3)], a1.stats(), a1.cache_stats())
         ids = [int(x) for x in rng.integers(1, 4, size=int(rng.integers(1, 7)))]
         st, slots, pairs = a1.seq_append_slots_batch(ids)
-        seq = [a2.seq_append_slots(i, 1) for i in ids]
-        oseq = [o.seq_append_slots(i, 1) for i in ids]
+        seq, oseq = [], []
+        for i in ids:                                       # one call per sequence, stopping at a failure
+            seq.append(a2.seq_append_slots(i, 1))
+            oseq.append(o.seq_append_slots(i, 1))
+            if seq[-1][0] != OK:
+                break
         assert seq == oseq, seed
         if all(r[0] == OK for r in seq):
             assert st == OK
             assert slots.tolist() == [r[1][0] for r in seq]
             assert [tuple(p) for p in pairs.tolist()] == [p for r in seq for p in r[2]]
-            written = {r[1][0] // bs for r in seq}
-            cached = set(o.key_of)
-            assert not (written & cached), seed               # no write lands in a cached block
+            assert not ({r[1][0] // bs for r in seq} & set(o.key_of)), seed   # no write in a cached block
+            for s in (1, 2, 3):
+                assert a1.seq_block_table(s) == a2.seq_block_table(s)
+            assert a1.cache_stats() == a2.cache_stats() == o.cache_stats()
         else:
-            assert st == next(r[0] for r in seq if r[0] != OK) and slots.size == 0
-        for s in (1, 2, 3):
-            assert a1.seq_block_table(s) == a2.seq_block_table(s)
-        assert a1.cache_stats() == a2.cache_stats() == o.cache_stats()
+            n_fail += 1
+            assert st == NO_FREE_BLOCK and slots.size == 0 and pairs.size == 0
+            stats = dict(before[1], alloc_failures=before[1]["alloc_failures"] + 1)
+            assert ([a1.seq_block_table(s) for s in (1, 2, 3)], a1.stats(), a1.cache_stats()) == \
+                (before[0], stats, before[2]), seed
+    assert n_fail > 20     # the tight pools were exercised

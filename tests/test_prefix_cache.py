@@ -206,3 +206,35 @@ def test_caching_off_behaves_like_plain_allocator():
     assert a.stats() == o.stats() and a.cache_stats()["cached_blocks"] == 0
     st, n_cached, _ = a.seq_add_with_prompt(1, list(range(10)))
     assert n_cached == 0
+
+
+def test_copy_of_a_cached_block_by_its_last_holder_frees_the_original():
+    """A sequence holding a cached block with fewer of its tokens copies it
+    before writing; when it was the block's last holder the original turns
+    evictable at once, so the same call can take it back as a fresh block.
+    The product allocator (single and batched calls) agrees with the oracle
+    on every pool size, including the tightest."""
+    from paged_kv_cache_405_b200 import BlockAllocator
+    bs = 2
+    for nb in range(3, 8):
+        for n in range(1, 5):
+            out = []
+            for a in (BlockAllocator(nb, bs, prefix_caching=True), CachingAllocator(nb, bs)):
+                assert a.seq_add_with_prompt(0, [1, 2, 3, 4])[0] == OK      # two cached blocks
+                blocks = a.seq_block_table(0)[1]
+                assert a.seq_add(1) == OK and a.seq_share_prefix(1, blocks, 3) == OK
+                assert a.seq_free(0) == OK                                  # sequence 1 is the last holder
+                st, slots, pairs = a.seq_append_slots(1, n)
+                out.append((st, list(slots), [tuple(p) for p in pairs], a.seq_block_table(1), a.stats(),
+                            a.cache_stats()))
+            assert out[0] == out[1], (nb, n)
+            assert out[1][0] == OK or nb == 3                              # only the 3-block pool runs short
+            b = BlockAllocator(nb, bs, prefix_caching=True)                # batched: the same steps
+            b.seq_add_with_prompt(0, [1, 2, 3, 4])
+            b.seq_add(1)
+            b.seq_share_prefix(1, b.seq_block_table(0)[1], 3)
+            b.seq_free(0)
+            st, slots, pairs = b.seq_append_slots_batch([1] * n)
+            assert st == out[0][0]
+            if st == OK:
+                assert slots.tolist() == out[0][1] and [tuple(p) for p in pairs.tolist()] == out[0][2]
