@@ -50,21 +50,40 @@ MUTANTS = {
 }
 
 
-@pytest.mark.parametrize("name", list(MUTANTS))
-def test_pins_catch_planted_mistake(name, tmp_path):
+def _build_and_run(d, name):
     old, new = MUTANTS[name]
     src = open(SRC).read()
-    assert src.count(old) == 1, "the planted mistake must replace exactly one place"
-    mutant = tmp_path / "oracle_mutant.c"
-    mutant.write_text(src.replace(old, new))
-    lib = tmp_path / "liboracle_mutant.so"
+    if src.count(old) != 1:
+        return "the planted mistake must replace exactly one place"
+    tag = "m%d" % list(MUTANTS).index(name)
+    mutant, lib = os.path.join(d, tag + ".c"), os.path.join(d, "liboracle_%s.so" % tag)
+    open(mutant, "w").write(src.replace(old, new))
     subprocess.check_call(["gcc", "-O2", "-fno-fast-math", "-fopenmp", "-shared", "-fPIC", "-std=c11", "-o",
-                           str(lib), str(mutant), "-lm"])
-    env = dict(os.environ, ORACLE_LIBRARY=str(lib))
+                           lib, mutant, "-lm"])
     r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(HERE, "test_oracle_pins.py"), "-x", "-q",
-                        "-p", "no:cacheprovider"], cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
-    assert r.returncode != 0, "no pin caught: %s" % name
-    assert "failed" in r.stdout, r.stdout[-2000:]
+                        "-p", "no:cacheprovider"], cwd=ROOT, env=dict(os.environ, ORACLE_LIBRARY=lib),
+                       capture_output=True, text=True, timeout=600)
+    if r.returncode == 0:
+        return "no pin caught it"
+    if "failed" not in r.stdout:
+        return r.stdout[-2000:]
+    return None
+
+
+@pytest.fixture(scope="module")
+def c_outcomes(tmp_path_factory):
+    """Build each mutant oracle library and run the pins against it, the runs
+    side by side (independent processes)."""
+    from concurrent.futures import ThreadPoolExecutor
+    d = str(tmp_path_factory.mktemp("oracle_mutants"))
+    with ThreadPoolExecutor(max_workers=max(2, min(len(MUTANTS), os.cpu_count() or 2))) as ex:
+        futures = {name: ex.submit(_build_and_run, d, name) for name in MUTANTS}
+        return {name: f.result() for name, f in futures.items()}
+
+
+@pytest.mark.parametrize("name", list(MUTANTS))
+def test_pins_catch_planted_mistake(name, c_outcomes):
+    assert c_outcomes[name] is None, "%s: %s" % (name, c_outcomes[name])
 
 
 # Planted mistakes in the Python allocator (class Allocator, the first class
