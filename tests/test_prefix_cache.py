@@ -238,3 +238,50 @@ def test_copy_of_a_cached_block_by_its_last_holder_frees_the_original():
             assert st == out[0][0]
             if st == OK:
                 assert slots.tolist() == out[0][1] and [tuple(p) for p in pairs.tolist()] == out[0][2]
+
+
+def test_batched_appends_equal_single_calls_after_random_histories():
+    """Caching mode, random histories (prompts, token appends, forks, shared
+    prefixes, frees), then one batched step over random live sequences: it
+    equals one call per sequence in order (product and oracle) when those all
+    succeed, and otherwise fails as a whole, changing nothing but the
+    failure count."""
+    from paged_kv_cache_405_b200 import BlockAllocator
+    n_ok = n_fail = 0
+    for seed in range(600):
+        rng = np.random.default_rng(seed)
+        nb, bs = 6 + seed % 5, (2, 3)[seed % 2]
+        order = rng.permutation(nb)
+        prod1 = BlockAllocator(nb, bs, order, prefix_caching=True)
+        prod2 = BlockAllocator(nb, bs, order, prefix_caching=True)
+        orc = CachingAllocator(nb, bs, order)
+        for op in caching_ops(seed, 10):
+            r = [apply(a, op) for a in (prod1, prod2, orc)]
+            assert r[0] == r[1] == r[2], (seed, op)
+        live = [s for s in range(5) if s in orc.seqs]
+        if not live:
+            continue
+        ids = [live[int(i)] for i in rng.integers(0, len(live), size=int(rng.integers(1, 6)))]
+        before = ([prod1.seq_block_table(s) for s in range(5)], prod1.stats(), prod1.cache_stats())
+        st, slots, pairs = prod1.seq_append_slots_batch(ids)
+        seq, oseq = [], []
+        for i in ids:
+            seq.append(prod2.seq_append_slots(i, 1))
+            oseq.append(orc.seq_append_slots(i, 1))
+            if seq[-1][0] != OK:
+                break
+        assert seq == oseq, seed
+        if all(x[0] == OK for x in seq):
+            n_ok += 1
+            assert st == OK, seed
+            assert slots.tolist() == [x[1][0] for x in seq]
+            assert [tuple(p) for p in pairs.tolist()] == [p for x in seq for p in x[2]]
+            assert [prod1.seq_block_table(s) for s in range(5)] == [prod2.seq_block_table(s) for s in range(5)]
+            assert prod1.cache_stats() == prod2.cache_stats() == orc.cache_stats()
+        else:
+            n_fail += 1
+            assert st == NO_FREE_BLOCK and slots.size == 0, seed
+            after = ([prod1.seq_block_table(s) for s in range(5)], prod1.stats(), prod1.cache_stats())
+            fails = dict(before[1], alloc_failures=before[1]["alloc_failures"] + 1)
+            assert after == (before[0], fails, before[2]), seed
+    assert n_ok > 100 and n_fail > 10
