@@ -364,9 +364,10 @@ pkv_status pkv_seq_fork(pkv_alloc* a, int64_t parent, int64_t child);
  *              (pkv_block_copy) before writing the new tokens; at most one
  *              per call, so cow_cap >= 1 suffices.  *n_cow = pairs written.
  * A fresh block is taken when the last block is full; if the token lands in a
- * block whose reference count is above one, that block alone is copied to a
- * fresh block and replaced in this sequence's table ([E] 6.2).
- * PKV_ERR_NO_FREE_BLOCK if the pool runs out (counted in alloc_failures).
+ * block whose reference count is above one (or, with prefix caching, a cached
+ * block), that block alone is copied to a fresh block and replaced in this
+ * sequence's table ([E] 6.2).  PKV_ERR_NO_FREE_BLOCK if the pool runs out
+ * (counted in alloc_failures); the call then changes nothing else.
  */
 pkv_status pkv_seq_append_slots(pkv_alloc* a, int64_t seq_id, int ntok, int64_t* slots_out,
                                 int32_t* cow_out, int cow_cap, int* n_cow);
@@ -378,7 +379,9 @@ pkv_status pkv_seq_append_slots(pkv_alloc* a, int64_t seq_id, int ntok, int64_t*
  *   slots_out  int64 [n]
  *   cow_out    int32 [cow_cap][2]; *n_cow = pairs written (at most n).
  * All-or-nothing: if any sequence fails (unknown id, pool exhausted, cow_cap
- * too small), nothing changes and *n_cow = 0.
+ * too small), nothing changes and *n_cow = 0 (an exhausted pool still counts
+ * one allocation failure in pkv_alloc_stats).  Blocks are counted in call
+ * order, so a step that the n single calls complete is never refused.
  */
 pkv_status pkv_seq_append_slots_batch(pkv_alloc* a, const int64_t* seq_ids, int n, int64_t* slots_out,
                                       int32_t* cow_out, int cow_cap, int* n_cow);
