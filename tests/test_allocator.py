@@ -265,3 +265,43 @@ def test_batch_calls_equal_sequential_calls_with_cached_blocks():
             assert ([a1.seq_block_table(s) for s in (1, 2, 3)], a1.stats(), a1.cache_stats()) == \
                 (before[0], stats, before[2]), seed
     assert n_fail > 20     # the tight pools were exercised
+
+
+def test_batched_appends_equal_single_calls_after_random_histories():
+    """Random histories (append, fork, share, free), then one batched step
+    over random live sequences: equal to one call per sequence (product and
+    oracle) when those all succeed, else refused as a whole with nothing
+    changed but the failure count."""
+    n_ok = n_fail = 0
+    for seed in range(600):
+        rng = np.random.default_rng(seed)
+        nb, bs = 4 + seed % 5, (1, 2, 4)[seed % 3]
+        order = np.random.default_rng(seed).permutation(nb)
+        p1, p2, o = BlockAllocator(nb, bs, order), BlockAllocator(nb, bs, order), oracle.Allocator(nb, bs, order)
+        for op in synth.random_ops(seed, 10, max_seqs=4, max_append=6):
+            r = [apply(a, op, bs) for a in (p1, p2, o)]
+            assert r[0] == r[1] == r[2], (seed, op)
+        live = [s for s in range(4) if s in o.seqs]
+        if not live:
+            continue
+        ids = [live[int(i)] for i in rng.integers(0, len(live), size=int(rng.integers(1, 6)))]
+        before = ([p1.seq_block_table(s) for s in range(4)], p1.stats())
+        st, slots, pairs = p1.seq_append_slots_batch(ids)
+        seq, oseq = [], []
+        for i in ids:
+            seq.append(p2.seq_append_slots(i, 1))
+            oseq.append(o.seq_append_slots(i, 1))
+            if seq[-1][0] != OK:
+                break
+        assert seq == oseq, seed
+        if all(x[0] == OK for x in seq):
+            n_ok += 1
+            assert st == OK and slots.tolist() == [x[1][0] for x in seq], seed
+            assert [tuple(p) for p in pairs.tolist()] == [p for x in seq for p in x[2]]
+            assert [p1.seq_block_table(s) for s in range(4)] == [p2.seq_block_table(s) for s in range(4)]
+        else:
+            n_fail += 1
+            assert st == NO_FREE_BLOCK and slots.size == 0, seed
+            fails = dict(before[1], alloc_failures=before[1]["alloc_failures"] + 1)
+            assert ([p1.seq_block_table(s) for s in range(4)], p1.stats()) == (before[0], fails), seed
+    assert n_ok > 100 and n_fail > 10
