@@ -98,7 +98,8 @@ pkv_status pkv_kv_append(const void* k_new, const void* v_new, void* k_pool, voi
  *                    call uses max_blocks_per_seq*block_size as that bound.
  *   partition_size   as in the decode call (0 = library's choice; the size
  *                    returned then covers whatever the library picks).
- * Returns 0 when no workspace is needed (every context fits one partition).
+ * Returns 0 when no workspace is needed (every context fits one partition),
+ * and SIZE_MAX when the size does not fit in size_t (such a call cannot run).
  */
 size_t pkv_attention_workspace_bytes(int num_seqs, int num_q_heads, int head_dim,
                                      int max_context_len, int partition_size);
@@ -129,7 +130,8 @@ int pkv_attention_partition_size(int num_seqs, int num_q_heads, int num_kv_heads
  *   workspace       >= pkv_attention_workspace_bytes(...) bytes of device
  *                   memory, 256-byte aligned; contents need no initialisation.
  * Supported: head_dim 64 or 128; block_size 16, 32, 64, 128 or 256;
- * num_blocks*num_kv_heads*block_size < 2^31.  16-bit types with a query group
+ * num_blocks*num_kv_heads*block_size < 2^31; at most 65535 sequences, query
+ * heads and partitions per call.  16-bit types with a query group
  * of 2..16 heads run on tensor cores; other cases on CUDA cores.
  * Deterministic: the same inputs give bit-identical outputs.
  */
@@ -286,10 +288,14 @@ pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, const void* 
  *     (num_seqs * num_q_heads * ceil(max_blocks_per_seq*block_size /
  *     partition) * (head_dim + 2) * 4 bytes) is rejected with
  *     PKV_ERR_INVALID and a message; nothing is launched.
- *   - Set-up: the first call on each device looks up the buffer's device
- *     address (a CUDA runtime query made with that device current).  Make
- *     that first call before any stream capture.  Calls run on the device
- *     that is current when they are made.
+ *   - Set-up: every call that splits its contexts looks up the buffer's
+ *     device address on the device current at the call (a CUDA runtime
+ *     query that allocates nothing), so a new context on that device is
+ *     always served at the right address.  The first such call on a device
+ *     may also load the library's device code: make it before any stream
+ *     capture.  Calls run on the device that is current when they are made.
+ *   - The size limit is checked after every other argument, so an invalid
+ *     argument is reported as itself, not as a lack of scratch.
  *   - Sharing: every call on a device uses the same buffer, and it keeps
  *     whatever the last call left in it.  Nothing in it needs to start at
  *     zero.  Calls that overlap on the GPU (different streams, no ordering

@@ -69,18 +69,30 @@ static int choose_partition(int max_len, int requested) {
     return 512;
 }
 
+// Bytes of split-K partials for rows x slots x (D + 2) floats; SIZE_MAX when
+// the product does not fit in size_t (no buffer is that large, so every
+// size check against it fails).
+static size_t partials_bytes(int64_t rows, int64_t slots, int D) {
+    size_t a = 0, b = 0, c = 0;
+    if (rows < 0 || slots < 0 || D < 0) return SIZE_MAX;
+    if (__builtin_mul_overflow((size_t)rows, (size_t)slots, &a) ||
+        __builtin_mul_overflow(a, (size_t)D + 2, &b) || __builtin_mul_overflow(b, sizeof(float), &c))
+        return SIZE_MAX;
+    return c;
+}
+
 static size_t workspace_for(int S, int Hq, int D, int max_len, int P) {
-    const int64_t maxP = (max_len + P - 1) / P;
+    const int64_t maxP = ((int64_t)max_len + P - 1) / P;
     if (maxP <= 1) return 0;
-    return (size_t)S * Hq * maxP * (size_t)(D + 2) * sizeof(float);
+    return partials_bytes((int64_t)S * Hq, maxP, D);
 }
 
 // Shared-prefix mode: one more partial slot per (sequence, head) than
 // partitions, since a member's prefix and suffix partitions can each end
 // part-way through a partition.
 static size_t shared_workspace_for(int S, int Hq, int D, int max_len, int P) {
-    const int64_t slots = (max_len + P - 1) / P + 1;
-    return (size_t)S * Hq * slots * (size_t)(D + 2) * sizeof(float);
+    const int64_t slots = ((int64_t)max_len + P - 1) / P + 1;
+    return partials_bytes((int64_t)S * Hq, slots, D);
 }
 
 // Smallest partition the library's own choice can produce for max_len: the
@@ -377,6 +389,34 @@ static cudaError_t dispatch_attention_fp8(const pkv::AttnParams& p, int D, int n
     return D == 64 ? launch_reduce<To, 64>(r, st) : launch_reduce<To, 128>(r, st);
 }
 
+// Built-in split-K scratch, for callers that cannot allocate.
+//
+// Some callers have no way to hand us device memory for the split-K
+// workspace: code that runs where cudaMalloc is off limits (a host process
+// whose allocator owns all device memory and forbids side allocations, a
+// plug-in that may only use what it is given, code that must not reach a
+// synchronising allocation in the middle of a step).  For them
+// pkv_paged_attention_decode_static takes the partials from a fixed buffer
+// compiled into this library.
+//
+// The buffer is one file-scope device array of kStaticScratchBytes per GPU,
+// held by every GPU that loads this library until the process exits.  Its
+// device address is looked up on each call that needs it (cudaGetSymbolAddress
+// allocates nothing), with the calling device current, so a module reloaded
+// at another address (a new context on the device) is always found; the
+// host-side name of the array is not a device address and is never handed to
+// a kernel.
+constexpr size_t kStaticScratchBytes = size_t(64) << 20;  // 64 MiB per GPU
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+static cudaError_t static_scratch(void** ptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+    if (e != cudaSuccess) return e;
+    *ptr = p;
+    return cudaSuccess;
+}
+
 struct KvArgs {
     pkv_dtype dtype = PKV_BF16;  // pool element type (the call's type unless FP8)
     bool fp8 = false;
@@ -396,7 +436,8 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
                               const int32_t* block_tables, int max_blocks_per_seq, const int32_t* context_lens,
                               int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
                               int num_blocks, float scale, int partition_size, const GroupArgs& grp, void* workspace,
-                              size_t workspace_bytes, pkv_dtype dtype, void* stream, const KvArgs& kv = KvArgs()) {
+                              size_t workspace_bytes, pkv_dtype dtype, void* stream, const KvArgs& kv = KvArgs(),
+                              bool builtin_scratch = false) {
     if (!valid_dtype(dtype)) return invalid("pkv_paged_attention_decode: bad dtype");
     if (kv.fp8) {
         if (dtype == PKV_F32) {
@@ -412,6 +453,7 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
     }
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0)
         return invalid("pkv_paged_attention_decode: sizes must be positive");
+    if (num_q_heads > 65535) return invalid("pkv_paged_attention_decode: at most 65535 query heads");
     if (num_q_heads % num_kv_heads != 0)
         return invalid("pkv_paged_attention_decode: num_q_heads must be a multiple of num_kv_heads");
     if (!valid_block_size(block_size))
@@ -460,6 +502,18 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
     const int64_t slots = nparts + (grp.mode ? 1 : 0);
     const size_t need = grp.mode ? shared_workspace_for(num_seqs, num_q_heads, head_dim, max_len, P)
                                  : workspace_for(num_seqs, num_q_heads, head_dim, max_len, P);
+    if (need > 0 && builtin_scratch) {  // every other argument has passed by now
+        if (need > kStaticScratchBytes) {
+            g_msg = "pkv_paged_attention_decode_static: this call needs " + std::to_string(need) +
+                    " bytes of split-K scratch but the built-in buffer holds " + std::to_string(kStaticScratchBytes) +
+                    "; use a larger partition_size, fewer sequences, or pkv_paged_attention_decode with a "
+                    "caller-provided workspace";
+            return PKV_ERR_INVALID;
+        }
+        const cudaError_t e = static_scratch(&workspace);
+        if (e != cudaSuccess) return cuda_fail("pkv_paged_attention_decode_static: scratch address", e);
+        workspace_bytes = kStaticScratchBytes;
+    }
     if (need > 0) {
         if (!workspace || workspace_bytes < need) return invalid("pkv_paged_attention_decode: workspace too small");
         if (reinterpret_cast<uintptr_t>(workspace) & 255u)
@@ -758,9 +812,9 @@ extern "C" pkv_status pkv_paged_attention_decode_fp8(void* out, const void* q, c
 namespace pkv_host {
 
 static size_t chunk_workspace_for(int T, int Hq, int D, int max_len, int P) {
-    const int64_t nparts = (max_len + P - 1) / P;
+    const int64_t nparts = ((int64_t)max_len + P - 1) / P;
     if (nparts <= 1) return 0;
-    return (size_t)T * Hq * nparts * (size_t)(D + 2) * sizeof(float);
+    return partials_bytes((int64_t)T * Hq, nparts, D);
 }
 
 template <typename T>
@@ -804,6 +858,7 @@ extern "C" pkv_status pkv_paged_attention_chunk(void* out, const void* q, const 
     if (num_seqs < 0 || num_tokens < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 ||
         max_blocks_per_seq <= 0 || max_query_len < 1)
         return invalid("pkv_paged_attention_chunk: sizes must be positive");
+    if (num_q_heads > 65535) return invalid("pkv_paged_attention_chunk: at most 65535 query heads");
     if (num_q_heads % num_kv_heads != 0 || num_q_heads / num_kv_heads > 16)
         return invalid("pkv_paged_attention_chunk: num_q_heads must be 1..16 times num_kv_heads");
     if (!valid_block_size(block_size))
@@ -877,49 +932,6 @@ extern "C" pkv_status pkv_paged_attention_chunk(void* out, const void* q, const 
     return e == cudaSuccess ? PKV_OK : cuda_fail(fn, e);
 }
 
-// ---------------------------------------------------------------------------
-// Decode attention with built-in scratch, for callers that cannot allocate.
-//
-// Some callers have no way to hand us device memory for the split-K
-// workspace: code that runs where cudaMalloc is off limits (a host process
-// whose allocator owns all device memory and forbids side allocations, a
-// plug-in that may only use what it is given, code that must not reach a
-// synchronising allocation in the middle of a step).  For them this entry
-// point takes the partials from a fixed buffer compiled into this library.
-//
-// The buffer is one file-scope device array of kStaticScratchBytes per GPU,
-// held by every GPU that loads this library until the process exits.  Its
-// device address is looked up once per device (cudaGetSymbolAddress, with
-// that device current) on the first call made on that device; the host-side
-// name of the array is not a device address and is never handed to a kernel.
-// ---------------------------------------------------------------------------
-namespace pkv_host {
-
-constexpr size_t kStaticScratchBytes = size_t(64) << 20;  // 64 MiB per GPU
-static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
-
-constexpr int kMaxDevices = 64;
-static void* g_static_scratch_ptr[kMaxDevices];
-static std::mutex g_static_scratch_mu;
-
-static cudaError_t static_scratch(void** ptr) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_static_scratch_mu);
-    if (!g_static_scratch_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_static_scratch);
-        if (e != cudaSuccess) return e;
-        g_static_scratch_ptr[dev] = p;
-    }
-    *ptr = g_static_scratch_ptr[dev];
-    return cudaSuccess;
-}
-
-}  // namespace pkv_host
-
 extern "C" pkv_status pkv_paged_attention_decode_static(void* out, const void* q, const void* k_pool,
                                                         const void* v_pool, const int32_t* block_tables,
                                                         int max_blocks_per_seq, const int32_t* context_lens,
@@ -927,24 +939,7 @@ extern "C" pkv_status pkv_paged_attention_decode_static(void* out, const void* q
                                                         int block_size, int num_blocks, float scale,
                                                         int partition_size, pkv_dtype dtype, void* stream) {
     using namespace pkv_host;
-    if (max_blocks_per_seq > 0 && block_size > 0 && num_seqs > 0 && num_q_heads > 0 && head_dim > 0 &&
-        partition_size >= 0 && (int64_t)max_blocks_per_seq * block_size <= ((int64_t)1 << 30)) {
-        const int max_len = max_blocks_per_seq * block_size;
-        const int P = choose_partition(max_len, partition_size);
-        const size_t need = P > 0 ? workspace_for(num_seqs, num_q_heads, head_dim, max_len, P) : 0;
-        if (need > kStaticScratchBytes) {
-            g_msg = "pkv_paged_attention_decode_static: this call needs " + std::to_string(need) +
-                    " bytes of split-K scratch but the built-in buffer holds " +
-                    std::to_string(kStaticScratchBytes) +
-                    "; use a larger partition_size, fewer sequences, or pkv_paged_attention_decode with a "
-                    "caller-provided workspace";
-            return PKV_ERR_INVALID;
-        }
-    }
-    void* scratch = nullptr;
-    cudaError_t e = static_scratch(&scratch);
-    if (e != cudaSuccess) return cuda_fail("pkv_paged_attention_decode_static: scratch address", e);
-    return pkv_paged_attention_decode(out, q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens,
-                                      num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks, scale,
-                                      partition_size, scratch, kStaticScratchBytes, dtype, stream);
+    return decode_impl(out, q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads,
+                       num_kv_heads, head_dim, block_size, num_blocks, scale, partition_size, GroupArgs(), nullptr, 0,
+                       dtype, stream, KvArgs(), true);
 }

@@ -89,10 +89,53 @@ def test_decode_validation(over, status):
     (dict(maxB=65536, P=16), "too many partitions"),                  # 65536 partitions of 16 tokens
     (dict(maxB=(1 << 26) + 1), "max_blocks_per_seq*block_size too large"),   # over 2^30 tokens
     (dict(NB=1 << 25, Hkv=4, Hq=4, bs=16), "2^31 or more rows"),     # 32-bit TMA row coordinates
+    (dict(Hq=65536, Hkv=4), "at most 65535 query heads"),             # keeps workspace sizes in range
 ])
 def test_decode_size_limits_are_refused_before_any_launch(over, why):
     assert call_decode(**over) == binding.INVALID
     assert why in binding.lib.pkv_last_error().decode()
+
+
+def call_decode_static(**over):
+    host_only()
+    a = dict(out=16, q=16, k=16, v=16, bt=16, maxB=4, cl=16, S=1, Hq=4, Hkv=4, D=64, bs=16, NB=8,
+             scale=0.0, P=0, dt=1, stream=None)
+    a.update(over)
+    return binding.lib.pkv_paged_attention_decode_static(a["out"], a["q"], a["k"], a["v"], a["bt"], a["maxB"],
+                                                         a["cl"], a["S"], a["Hq"], a["Hkv"], a["D"], a["bs"],
+                                                         a["NB"], a["scale"], a["P"], a["dt"], a["stream"])
+
+
+@pytest.mark.parametrize("over,why", [
+    (dict(P=24), "partition_size must be 0 or a positive multiple of 16"),
+    (dict(maxB=65536 * 2, P=16), "too many partitions"),
+    (dict(bs=24), "block_size must be"),
+    (dict(q=8), "16-byte aligned"),
+])
+def test_static_decode_reports_the_real_cause_before_the_scratch_size(over, why):
+    """The built-in scratch is sized only once every other argument has
+    passed, so a bad argument is named as such (no scratch message)."""
+    assert call_decode_static(**over) == binding.INVALID
+    msg = binding.lib.pkv_last_error().decode()
+    assert why in msg and "scratch" not in msg
+
+
+def test_static_decode_refuses_calls_beyond_its_scratch_before_any_launch():
+    # 64 seqs x 32 heads x 128 partitions of 16 tokens x 130 floats > 64 MiB
+    assert call_decode_static(S=64, Hq=32, Hkv=32, D=128, maxB=128, P=16) == binding.INVALID
+    assert "split-K scratch" in binding.lib.pkv_last_error().decode()
+    # an empty batch needs nothing and is accepted
+    assert call_decode_static(S=0, out=None) == binding.OK
+
+
+def test_workspace_queries_saturate_instead_of_wrapping():
+    size_max = (1 << (8 * ctypes.sizeof(ctypes.c_size_t))) - 1
+    big = (1 << 31) - 1
+    assert pkv.attention_workspace_bytes(65535, big, 128, 1 << 30, 16) == size_max
+    assert pkv.attention_shared_workspace_bytes(big, big, 128, 1 << 30, 16) == size_max
+    assert pkv.attention_chunk_workspace_bytes(big, 65535, 128, 1 << 30, 16) == size_max
+    # in range: the plain product
+    assert pkv.attention_workspace_bytes(2, 3, 64, 64, 16) == 2 * 3 * 4 * 66 * 4
 
 
 def test_append_and_copy_validation():
