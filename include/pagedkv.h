@@ -72,7 +72,9 @@ typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_F16 = 2, PKV_FP8_E4M3 = 3 /* pools
 #define PKV_DEVERR_SLOT       2u  /* slot outside [0, num_blocks*block_size) */
 #define PKV_DEVERR_CONTEXT    4u  /* context length < 0 or > max_blocks_per_seq*block_size */
 #define PKV_DEVERR_TIMEOUT    8u  /* a bounded wait on an async copy gave up */
-#define PKV_DEVERR_GROUP     16u  /* a shared-prefix group has more members than max_group_size */
+#define PKV_DEVERR_GROUP     16u  /* a shared-prefix group description does not hold: more members than
+                                     max_group_size, a shared run over max_shared_len, or a member whose
+                                     leading blocks are not its group's */
 
 /* ------------------------------------------------------------------ device */
 
@@ -159,17 +161,25 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_po
  *                 handled as in pkv_paged_attention_decode.
  *   group_shared  device int32 [num_groups]: number of leading tokens the
  *                 members of group g share, a multiple of block_size, at most
- *                 every member's context length.  The first
- *                 group_shared[g]/block_size block-table entries of every
- *                 member must be those of the group's first sequence (the
- *                 prefix pass reads the first sequence's).  A value breaking
- *                 these rules is recorded (PKV_DEVERR_CONTEXT) and the group's
- *                 members are then handled as non-members.
- *   max_group_size  host bound on members per group (PKV_DEVERR_GROUP if a
- *                 group is larger; its extra members get no prefix result).
+ *                 every member's context length.  A value breaking these
+ *                 rules is recorded (PKV_DEVERR_CONTEXT) and the members it
+ *                 breaks them for are handled as non-members.
+ *                 The prefix pass reads the first group_shared[g]/block_size
+ *                 block-table entries of the group's first sequence; only
+ *                 members whose own first entries are the same take its
+ *                 result ([E] 6.1, [T] 2.2.8: only identical prefixes are
+ *                 shared).  Every kernel of the call compares them on the
+ *                 device; a member whose entries differ is recorded
+ *                 (PKV_DEVERR_GROUP) and handled as a non-member.
+ *   max_group_size  host bound on members per group (it sizes the prefix
+ *                 pass); members past it are recorded (PKV_DEVERR_GROUP)
+ *                 and handled as non-members.
  *   max_shared_len  host bound on every group_shared[g] (it sizes the prefix
- *                 pass; a larger group_shared is recorded as PKV_DEVERR_GROUP
- *                 and its tokens past the bound get no prefix result).
+ *                 pass); a larger group_shared is recorded as
+ *                 PKV_DEVERR_GROUP and its members handled as non-members.
+ * A non-member attends to its whole context through its own table, so the
+ * result equals pkv_paged_attention_decode's whatever the group description
+ * says; only the speed depends on it.
  *   workspace     >= pkv_attention_shared_workspace_bytes(...) bytes.
  * 16-bit element types only (PKV_ERR_UNSUPPORTED for fp32).
  */

@@ -77,6 +77,29 @@ __device__ __forceinline__ int group_shared_len(const AttnParams& p, int gi, int
 }
 
 
+// Whether the first `shared / bs` block-table entries of sequence s are those
+// of sequence `first` (the group's first sequence, whose table the prefix
+// pass reads): only sequences that really hold the same blocks may share the
+// prefix result (openeuler.csdn.net PagedAttention explainer 6.1;
+// aiknowledge.cn "2.2 PagedAttention 与 KV Cache 分页管理" 2.2.8).
+// Warp-collective: every lane calls it with the same s, first and shared
+// (shared <= max_blocks_per_seq * bs, so both rows are read in bounds).
+__device__ __forceinline__ bool same_leading_blocks(const int32_t* block_tables, int maxB, int bs, int s, int first,
+                                                    int shared, int lane) {
+    if (s == first) return true;
+    const int n = shared / bs;
+    const int32_t* a = block_tables + (int64_t)s * maxB;
+    const int32_t* b = block_tables + (int64_t)first * maxB;
+    bool same = true;
+    for (int j = lane; j < n; j += 32) same = same && a[j] == b[j];
+    return __all_sync(0xffffffffu, same);
+}
+
+// The group's first sequence as the prefix pass uses it (clamped into the batch).
+__device__ __forceinline__ int group_first_seq(const int32_t* group_first, int gi, int S) {
+    return max(0, min(group_first[gi], S));
+}
+
 // Context length of sequence s, clamped into [0, max_len]; an out-of-range
 // value is recorded once per sequence (by the unit that owns partition 0).
 __device__ __forceinline__ int load_context_len(const AttnParams& p, int s, bool report) {
@@ -88,7 +111,8 @@ __device__ __forceinline__ int load_context_len(const AttnParams& p, int s, bool
     return L;
 }
 
-__device__ __forceinline__ Unit resolve_unit(const AttnParams& p, int s, int part, bool report) {
+// Warp-collective (every lane of the warp, same s and part).
+__device__ __forceinline__ Unit resolve_unit(const AttnParams& p, int s, int part, bool report, int lane) {
     Unit u;
     u.L = load_context_len(p, s, report);
     u.shared = 0;
@@ -97,8 +121,17 @@ __device__ __forceinline__ Unit resolve_unit(const AttnParams& p, int s, int par
     if (gi >= 0) {
         const int sh = group_shared_len(p, gi, u.L, report);
         if (sh > 0) {
-            u.shared = sh;
-            u.member = true;
+            // A member past the prefix pass's grid (max_group_size), or whose
+            // leading blocks are not the group's, attends to its whole context
+            // through its own table, like a non-member.
+            const int first = group_first_seq(p.group_first, gi, p.S);
+            if (s - first < p.max_group_size &&
+                same_leading_blocks(p.block_tables, p.maxB, p.bs, s, first, sh, lane)) {
+                u.shared = sh;
+                u.member = true;
+            } else if (report) {
+                flag_error(16u /* PKV_DEVERR_GROUP */);
+            }
         }
     }
     u.npre = (u.shared + p.P - 1) / p.P;

@@ -368,7 +368,8 @@ static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int npart
     }
     if (e != cudaSuccess || p.maxP <= 1) return e;
     pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
-                        p.group_first, p.group_shared, p.num_groups, p.max_shared, nullptr, 0};
+                        p.group_first, p.group_shared, p.num_groups, p.max_shared, p.max_group_size,
+                        p.block_tables, p.maxB, nullptr, 0};
     return D == 64 ? launch_reduce<T, 64>(r, st) : launch_reduce<T, 128>(r, st);
 }
 
@@ -385,7 +386,7 @@ static cudaError_t dispatch_attention_fp8(const pkv::AttnParams& p, int D, int n
     }
     if (e != cudaSuccess || p.maxP <= 1) return e;
     pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
-                        nullptr, nullptr, 0, 0, nullptr, 0};
+                        nullptr, nullptr, 0, 0, 0, p.block_tables, p.maxB, nullptr, 0};
     return D == 64 ? launch_reduce<To, 64>(r, st) : launch_reduce<To, 128>(r, st);
 }
 
@@ -827,7 +828,7 @@ static cudaError_t dispatch_chunk(const pkv::AttnParams& p, const pkv::ChunkPara
         cudaError_t e = D == 64 ? launch_chunk<T, 64>(p, c, grid, mk, mv, st) : launch_chunk<T, 128>(p, c, grid, mk, mv, st);
         if (e != cudaSuccess || c.nparts <= 1) return e;
         pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
-                            nullptr, nullptr, 0, 0, c.query_start, c.T};
+                            nullptr, nullptr, 0, 0, 0, p.block_tables, p.maxB, c.query_start, c.T};
         return D == 64 ? launch_reduce<T, 64>(r, st) : launch_reduce<T, 128>(r, st);
     }
 }

@@ -8,7 +8,7 @@
 // One warp per (sequence, query head); partitions are merged in index order,
 // so the result is deterministic.
 #pragma once
-#include "common.cuh"
+#include "attention_common.cuh"
 
 namespace pkv {
 
@@ -20,15 +20,18 @@ struct ReduceParams {
     int S, Hq, D, P, maxP, max_len, bs;
     const int32_t* group_first;   // shared-prefix groups, as in AttnParams
     const int32_t* group_shared;
-    int num_groups, max_shared;
+    int num_groups, max_shared, max_group_size;
+    const int32_t* block_tables;  // [S][maxB] (members' leading blocks are compared)
+    int maxB;
     const int32_t* query_start;   // chunk mode (non-null): rows are (query row, head), [S + 1]
     int T;
 };
 
 // Partials to merge for one output row (0 = the attention kernel wrote it).
 // qs / gf: query_start / group_first, from global memory or a shared copy.
+// Warp-collective (every lane of the warp, same row).
 __device__ __forceinline__ int reduce_count(const ReduceParams& p, int row, const int32_t* qs,
-                                            const int32_t* gf) {
+                                            const int32_t* gf, int lane) {
     const int h_rows = p.Hq;
     if (p.query_start) {  // causal chunk: row = t * Hq + h
         const int t = row / h_rows;
@@ -62,7 +65,12 @@ __device__ __forceinline__ int reduce_count(const ReduceParams& p, int row, cons
             else hi = mid;
         }
         const int sh = p.group_shared[lo];
-        if (sh > 0 && sh % p.bs == 0 && sh <= L && sh <= p.max_shared) shared = sh;
+        if (sh > 0 && sh % p.bs == 0 && sh <= L && sh <= p.max_shared) {
+            const int first = max(0, min(gf[lo], p.S));
+            if (s - first < p.max_group_size &&
+                same_leading_blocks(p.block_tables, p.maxB, p.bs, s, first, sh, lane))
+                shared = sh;
+        }
     }
     const int nsuf = (L - shared + p.P - 1) / p.P;
     const int nP = (shared + p.P - 1) / p.P + nsuf;
@@ -97,7 +105,7 @@ __global__ void __launch_bounds__(W * ROWS * 32) splitk_reduce_kernel(const Redu
     float (&s_max)[W] = s_max_all[sub];
     const int nrows = p.query_start ? p.T * p.Hq : p.S * p.Hq;
     if (row >= nrows) return;  // whole rows return together (W warps of a row)
-    const int nP = reduce_count(p, row, p.query_start, p.group_first);
+    const int nP = reduce_count(p, row, p.query_start, p.group_first, lane);
     if (nP == 0) return;
     const int64_t base = (int64_t)row * p.maxP;
     const float* ml = p.ws_ml + base * 2;
@@ -223,7 +231,7 @@ __global__ void __launch_bounds__(ROWS * 32) splitk_reduce_warp_kernel(const Red
             }
         }
     }
-    const int nP = reduce_count(p, row, qs, gf);
+    const int nP = reduce_count(p, row, qs, gf, lane);
     if (nP == 0) return;
 
     float M = lane < nP ? mlv.x : -INFINITY;

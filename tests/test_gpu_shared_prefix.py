@@ -108,10 +108,53 @@ def test_malformed_group_is_reported_and_falls_back():
     assert max_err(out, oracle_attention(b)) <= TOL[out.dtype]
 
 
-def test_group_larger_than_declared_is_reported():
+@pytest.mark.parametrize("P", [0, 64])
+def test_group_larger_than_declared_is_reported(P):
     b = mixed_batch(seed=6)
-    run_shared(b, [0, 6, 9, 16], [256, 0, 128], 0, max_group=4)
+    out = run_shared(b, [0, 6, 9, 16], [256, 0, 128], P, max_group=4)
     assert pkv().device_error() & 16
+    # members past the bound are attended wholly through their own tables
+    assert max_err(out, oracle_attention(b)) <= TOL[out.dtype]
+
+
+@pytest.mark.parametrize("seq,entry", [(3, 7), (5, 15), (0, 2), (12, 0)])
+@pytest.mark.parametrize("P", [0, 32, 128])
+def test_member_whose_leading_blocks_differ_is_reported_and_uses_its_own_table(seq, entry, P):
+    """Only sequences that really hold the same blocks may share the prefix
+    result (openeuler.csdn.net PagedAttention explainer 6.1; aiknowledge.cn
+    "2.2 PagedAttention 与 KV Cache 分页管理" 2.2.8).  One shared table entry of
+    one member points at another block (holding other values): the call
+    records PKV_DEVERR_GROUP and that member attends to its whole context
+    through its own table, so every output still equals the oracle's.  Seq 0
+    is a group's first sequence: then no other member matches it."""
+    b = mixed_batch(seed=9)
+    gf, gs = pkv().find_shared_prefix_groups(b.block_tables, b.lens, 16, 3)
+    assert gf.tolist() == [0, 6, 9, 16] and gs.tolist() == [256, 0, 128]
+    used = set(b.block_tables[b.block_tables >= 0].tolist())
+    spare = next(int(x) for x in b.free_order[::-1] if int(x) not in used)
+    b.block_tables[seq, entry] = spare                 # the description above no longer holds for seq
+    out = run_shared(b, gf, gs, P)
+    assert pkv().device_error() & pkv().binding.DEVERR_GROUP
+    assert max_err(out, oracle_attention(b)) <= TOL[out.dtype]
+
+
+def test_mha_tile_of_sixteen_members_with_one_stranger():
+    """Multi-head attention: a prefix-pass tile holds 16 different sequences;
+    the one whose leading blocks differ gets no prefix partial."""
+    sh = synth.shrink(synth.CONFIGS["llama13b_prefix"], S=24, Hq=4, Hkv=4, prefix=256)
+    b = synth.make_batch(sh, fill_unused=float("nan"))
+    gf, gs = pkv().find_shared_prefix_groups(b.block_tables, b.lens, sh.bs, 4)
+    assert gs.tolist() == [256]
+    used = set(b.block_tables[b.block_tables >= 0].tolist())
+    spare = next(int(x) for x in b.free_order[::-1] if int(x) not in used)
+    g = torch.Generator().manual_seed(11)                # covered now: real values, not the NaN fill
+    b.k_pool[spare] = synth.randn(tuple(b.k_pool[spare].shape), g, b.k_pool.dtype, "cpu")
+    b.v_pool[spare] = synth.randn(tuple(b.v_pool[spare].shape), g, b.v_pool.dtype, "cpu")
+    b.block_tables[10, 3] = spare
+    for P in (0, 128):
+        out = run_shared(b, gf, gs, P)
+        assert pkv().device_error() & pkv().binding.DEVERR_GROUP
+        assert max_err(out, oracle_attention(b)) <= TOL[out.dtype]
 
 
 def test_session_uses_groups_for_the_prefix_workload():
