@@ -15,10 +15,19 @@ value  -- algorithmic bytes of the step (unique K/V bytes the attention must
 e2e    -- the same metric through DecodeSession.step: allocator on the host,
           step inputs copied in from pinned host memory, output copied back.
 
+The headline workload (``--config``, default ``llama3_gqa_bs16``: 128
+sequences x 8192 tokens, 32 query / 8 kv heads, the largest one-GPU decode
+workload) gives the line's value, roofline, e2e and CPU baseline; the
+``targets`` object carries the same device and end-to-end numbers for the
+workloads timed after it in the same run (by default the shared-system-prompt
+and 100k-token-context workloads, which carry the >= 70 % of HBM peak target,
+and the Llama-2-7B-shaped MHA layer).
+
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
-       [--impl ours|reference].  Under torchrun each rank runs its own
-replica (own pool, own sequences; no collective on the data path): weak
-scaling.  ``--impl reference`` times the CPU oracle instead (rank 0 only).
+       [--targets A,B|none] [--impl ours|reference].  Under torchrun each
+rank runs its own replica (own pool, own sequences; no collective on the data
+path): weak scaling.  ``--impl reference`` times the CPU oracle instead (rank
+0 only) and names the same workload in its ``config``.
 """
 import argparse
 import hashlib
@@ -38,6 +47,9 @@ import torch  # noqa: E402
 import synth  # noqa: E402
 
 METRIC = "paged decode attention HBM GB/s (% of B200 peak) and seq-steps/s per layer"
+# Headline workload: the largest one-GPU decode configuration (Llama-3-8B-shaped
+# grouped-query decode, 128 sequences x 8192 tokens, 4.29 GB of K/V per call).
+DEFAULT_CONFIG = "llama3_gqa_bs16"
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -354,8 +366,8 @@ def barrier(world):
         torch.distributed.barrier()
 
 
-def workload_shape(args):
-    shape = synth.CONFIGS[args.config]
+def workload_shape(args, name=None):
+    shape = synth.CONFIGS[args.config if name is None else name]
     if args.batch:
         shape = synth.shrink(shape, S=args.batch)
     # room in every table and in the pool for the tokens the run appends
@@ -365,14 +377,35 @@ def workload_shape(args):
     return shape
 
 
-def run_ours(args, world, rank, local):
+def workload_config(name, shape, batch, args, world) -> dict:
+    """The ``config`` object of a bench line: the workload, its shape and how
+    L2 is handled.  Both arms build it from the same seeded batch, so the
+    reference arm's line names exactly the workload this arm times."""
+    pool_gb = 2 * batch.k_pool.numel() * batch.k_pool.element_size() / 1e9
+    return {"workload": name + ("" if not args.batch else "@batch%d" % args.batch),
+            "description": shape.description, "batch": shape.S,
+            "q_heads": shape.Hq, "kv_heads": shape.Hkv, "head_dim": shape.D, "block_size": shape.bs,
+            "kv_dtype": "e4m3" if shape.kv_fp8 else shape.dtype,
+            "partition_size": args.partition_size or shape.partition_size,
+            "mean_context": round(float(np.mean(batch.lens)), 1),
+            "new_tokens_per_seq": max(1, shape.chunk),
+            "l2": "inputs larger than L2 (K/V pool %.2f GB per rank)" % pool_gb,
+            "parallelism": "replica per GPU" if world > 1 else "1 GPU"}
+
+
+def measure_workload(name, args, world, rank, local, e2e=True):
+    """Time K decode steps of workload ``name`` after W warm-up steps, inputs
+    resident in HBM (CUDA events on the launching stream, max over ranks),
+    then the same steps end to end from host buffers.  Returns the numbers
+    of one bench line (without the CPU baseline)."""
     import paged_kv_cache_405_b200 as pkv
-    shape = workload_shape(args)
+    shape = workload_shape(args, name)
     dev = torch.device("cuda", local)
     wl = Workload(shape, shape.seed + rank, dev, args.partition_size)
     ss = wl.session
     K, W = args.steps, args.warmup
     dt = synth.DTYPES[shape.dtype]
+    config = workload_config(name, shape, wl.batch, args, world)
 
     # ---- plan every step on the host first (device-resident inputs)
     plans, step_bytes, attn_bytes = [], [], []
@@ -435,7 +468,7 @@ def run_ours(args, world, rank, local):
         run_step(i)
     torch.cuda.synchronize()
     if pkv.device_error() != 0:
-        raise RuntimeError("device-side check failed during warm-up")
+        raise RuntimeError("device-side check failed during warm-up (%s)" % name)
     attn_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
@@ -463,7 +496,7 @@ def run_ours(args, world, rank, local):
     clk = clocks.stop()
     barrier(world)
     if pkv.device_error() != 0:
-        raise RuntimeError("device-side check failed during the timed steps")
+        raise RuntimeError("device-side check failed during the timed steps (%s)" % name)
     ms = t0.elapsed_time(t1)
     attn_ms = [a.elapsed_time(b) for a, b in attn_ev]
     ms_max = max_over_ranks(ms, world)
@@ -475,72 +508,88 @@ def run_ours(args, world, rank, local):
     # ---- roofline of the decode-attention call (attention kernel + its split-K reduce)
     peak, peak_kind = measured_hbm_peak()
     a_bytes = float(np.mean([a["total"] for a in attn_bytes[W:]]))
-    a_s = float(np.mean(attn_ms)) * 1e-3
+    a_s = max_over_ranks(float(np.mean(attn_ms)), world) * 1e-3
     achieved = a_bytes / a_s / 1e9
-    traffic = recorded_traffic(args.config)
-
-    # ---- end to end through DecodeSession.step (host buffers)
-    e2e = None
-    if not args.no_e2e:
+    traffic = recorded_traffic(name)
+    launch = {"effective_partition_size": wl.eff_P,
+              "shared_prefix_groups": int((plans[W].group_shared > 0).sum().item())
+              if not shape.chunk and plans[W].group_shared is not None else 0,
+              **({"nvtx_ranges": True} if args.nvtx else {})}
+    res = {
+        "value": round(value, 1), "ms_per_step": round(ms_max / K, 4), "config": config, "launch": launch,
+        "dtype": shape.dtype + ("+e4m3-kv" if shape.kv_fp8 else ""),
+        "pct_of_peak": round(100 * value / peak, 1),
+        "seq_steps_per_s": round(seq_steps, 1),
+        "kv_utilisation": round(float(np.mean([a["kv_util"] for a in attn_bytes[W:]])), 4),
+        "attention_us": round(a_s * 1e6, 2),
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
+                     "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+                     "kernel": "paged_attention_decode (attention + split-K reduce)",
+                     "algorithmic_bytes": round(a_bytes)},
+        "gpu_launches": int(launches),
+        "clocks": clk,
+    }
+    res["e2e"] = None
+    if e2e and not args.no_e2e:
         wl2 = Workload(shape, shape.seed + rank, dev, args.partition_size)
-        del wl
+        del wl, ss, plans, inputs, out
         torch.cuda.empty_cache()
-        e2e = run_e2e(args, wl2, world, rank, dev)
+        res["e2e"] = run_e2e(args, wl2, world, rank, dev)
+        del wl2
+    torch.cuda.empty_cache()
+    return res
 
-    line = None
-    if rank == 0:
-        line = {
-            "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K,
-            "warmup": W, "ms_per_step": round(ms_max / K, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": shape.dtype + ("+e4m3-kv" if shape.kv_fp8 else ""),
-            "data": "synthetic (seeded N(0,1) K/V/q; pages' workload shapes)",
-            "config": {"workload": args.config + ("" if not args.batch else "@batch%d" % args.batch),
-                       "description": shape.description, "batch": shape.S,
-                       "q_heads": shape.Hq, "kv_heads": shape.Hkv, "head_dim": shape.D, "block_size": shape.bs,
-                       "partition_size": wl_P(shape, args), "effective_partition_size": eff_P_of(shape, args, plans),
-                       "mean_context": round(float((plans[W]["lens"] if shape.chunk else plans[W].lens)
-                                                   .float().mean().item()), 1),
-                       "new_tokens_per_seq": max(1, shape.chunk),
-                       "l2": "inputs larger than L2 (K/V pool %.2f GB per rank)" % (
-                           2 * ss.k_pool.numel() * ss.k_pool.element_size() / 1e9),
-                       "parallelism": "replica per GPU" if world > 1 else "1 GPU",
-                       **({"nvtx_ranges": True} if args.nvtx else {}),
-                       "shared_prefix_groups": int((plans[W].group_shared > 0).sum().item())
-                       if not shape.chunk and plans[W].group_shared is not None else 0},
-            "pct_of_peak": round(100 * value / peak, 1),
-            "seq_steps_per_s": round(seq_steps, 1),
-            "kv_utilisation": round(float(np.mean([a["kv_util"] for a in attn_bytes[W:]])), 4),
-            "attention_us": round(a_s * 1e6, 2),
-            "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                         "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
-                         "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
-                         "kernel": "paged_attention_decode (attention + split-K reduce)",
-                         "algorithmic_bytes": round(a_bytes)},
-            "e2e": e2e,
-            "gpu_launches": int(launches),
-            "clocks": clk,
-        }
-        if world == 1 and not args.no_cpu_baseline:
-            hb = host_batch(shape, shape.seed + rank)
-            v, sps, desc, secs = oracle_sample(hb, args.cpu_seconds, threads=os.cpu_count())
-            v1, sps1, _, secs1 = oracle_sample(hb, max(1.0, args.cpu_seconds / 4), threads=1)
-            line["cpu_baseline"] = {"value": round(v, 3), "unit": "GB/s", "cores": os.cpu_count(),
-                                    "kind": "oracle", "sample": desc, "seq_steps_per_s": round(sps, 3),
-                                    "seconds": round(secs, 1), "cpu_model": cpu_model(),
-                                    "single_thread": {"value": round(v1, 3), "seq_steps_per_s": round(sps1, 3),
-                                                      "seconds": round(secs1, 1)}}
+
+# Configurations timed beside the headline in the default run: the two that
+# carry the >= 70 % target (shared system prompt, 100k-token contexts) and
+# the Llama-2-7B-shaped MHA layer.
+DEFAULT_TARGETS = ("llama13b_prefix", "longctx_beam", "llama7b")
+
+
+def target_names(args):
+    if args.targets == "none":
+        return []
+    if args.targets:
+        return [t for t in args.targets.split(",") if t]
+    if args.batch or args.config != DEFAULT_CONFIG:
+        return []
+    return list(DEFAULT_TARGETS)
+
+
+def run_ours(args, world, rank, local):
+    head = measure_workload(args.config, args, world, rank, local)
+    targets = {}
+    for name in target_names(args):
+        r = measure_workload(name, args, world, rank, local)
+        targets[name] = {k: r[k] for k in ("value", "ms_per_step", "attention_us", "seq_steps_per_s",
+                                           "pct_of_peak", "roofline", "e2e", "clocks", "config", "dtype")}
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": head["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": head["dtype"],
+        "data": "synthetic (seeded N(0,1) K/V/q; pages' workload shapes)",
+        "config": head["config"], "launch": head["launch"],
+        "pct_of_peak": head["pct_of_peak"], "seq_steps_per_s": head["seq_steps_per_s"],
+        "kv_utilisation": head["kv_utilisation"], "attention_us": head["attention_us"],
+        "roofline": head["roofline"], "e2e": head["e2e"], "gpu_launches": head["gpu_launches"],
+        "clocks": head["clocks"],
+    }
+    if targets:
+        line["targets"] = targets
+    if world == 1 and not args.no_cpu_baseline:
+        shape = workload_shape(args)
+        hb = host_batch(shape, shape.seed + rank)
+        v, sps, desc, secs = oracle_sample(hb, args.cpu_seconds, threads=os.cpu_count())
+        v1, sps1, _, secs1 = oracle_sample(hb, max(1.0, args.cpu_seconds / 4), threads=1)
+        line["cpu_baseline"] = {"value": round(v, 3), "unit": "GB/s", "cores": os.cpu_count(),
+                                "kind": "oracle", "sample": desc, "seq_steps_per_s": round(sps, 3),
+                                "seconds": round(secs, 1), "cpu_model": cpu_model(),
+                                "single_thread": {"value": round(v1, 3), "seq_steps_per_s": round(sps1, 3),
+                                                  "seconds": round(secs1, 1)}}
     return line
-
-
-def wl_P(shape, args):
-    return args.partition_size or shape.partition_size
-
-
-def eff_P_of(shape, args, plans):
-    import paged_kv_cache_405_b200 as pkv
-    bt = plans[0]["block_tables"] if shape.chunk else plans[0].block_tables
-    return pkv.attention_partition_size(shape.S, shape.Hq, shape.Hkv, shape.D, bt.shape[1] * shape.bs,
-                                        wl_P(shape, args))
 
 
 def host_batch(shape, seed):
@@ -648,7 +697,7 @@ def run_reference(args, world, rank):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * float(np.mean(secs)), 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (same seeded workload, host copy)",
-        "config": {"workload": args.config, "description": shape.description},
+        "config": workload_config(args.config, shape, batch, args, world),
         "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": os.cpu_count(), "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -730,7 +779,12 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1, help="GPUs (one rank each under torchrun; replicas, weak scaling)")
     ap.add_argument("--steps", type=int, default=20, help="timed decode steps")
     ap.add_argument("--warmup", type=int, default=5, help="untimed warm-up steps (at least 3)")
-    ap.add_argument("--config", default="llama7b", choices=sorted(synth.CONFIGS), help="workload (see synth.CONFIGS)")
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=sorted(synth.CONFIGS),
+                    help="headline workload (see synth.CONFIGS); default: the largest one-GPU decode workload")
+    ap.add_argument("--targets", default="",
+                    help="comma-separated workloads timed in the same run and reported under 'targets' "
+                         "(default: %s when the headline is the default one; 'none' for none)"
+                         % ",".join(DEFAULT_TARGETS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"],
                     help="ours: the CUDA library; reference: the CPU oracle on the host cores")
     ap.add_argument("--partition-size", type=int, default=0,

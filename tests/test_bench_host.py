@@ -103,9 +103,42 @@ def test_reference_arm_prints_one_contract_line():
         assert key in d, key
     assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3 and d["n_gpus"] == 1
     assert d["config"]["workload"] == "tiny" and d["value"] > 0 and d["higher_is_better"] is True
+    import argparse
+    sh = bench.workload_shape(argparse.Namespace(config="tiny", batch=0, warmup=3, steps=2))
+    assert d["config"]["batch"] == sh.S and d["config"]["head_dim"] == sh.D and d["config"]["block_size"] == sh.bs
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["value"] == d["value"] and cb["cores"] >= 1 and cb["sample"]
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_both_arms_name_the_same_config():
+    """The reference arm's ``config`` is built by the same function from the
+    same seeded batch as this arm's, so the two lines name one workload
+    (shape keys included)."""
+    import argparse
+    args = argparse.Namespace(config="llama7b", batch=0, partition_size=0, warmup=5, steps=20)
+    sh = bench.workload_shape(args)
+    a = bench.workload_config("llama7b", sh, synth.make_batch(sh, device="cpu"), args, 1)
+    b = bench.workload_config("llama7b", sh, synth.make_batch(sh, device="cpu", seed=sh.seed), args, 1)
+    assert a == b
+    for key in ("workload", "batch", "q_heads", "kv_heads", "head_dim", "block_size", "partition_size",
+                "mean_context", "l2", "parallelism"):
+        assert key in a, key
+    assert a["batch"] == 64 and a["q_heads"] == 32 and a["head_dim"] == 128 and a["block_size"] == 16
+
+
+def test_default_run_times_the_largest_config_and_the_targets():
+    import argparse
+    assert bench.DEFAULT_CONFIG == "llama3_gqa_bs16"
+    big = max((s.S * s.Hkv * (s.len_fixed or 0), n) for n, s in synth.CONFIGS.items() if not s.kv_fp8)
+    assert big[1].startswith("llama3_gqa")
+    ns = argparse.Namespace(targets="", batch=0, config=bench.DEFAULT_CONFIG)
+    assert bench.target_names(ns) == ["llama13b_prefix", "longctx_beam", "llama7b"]
+    assert bench.target_names(argparse.Namespace(targets="", batch=64, config=bench.DEFAULT_CONFIG)) == []
+    assert bench.target_names(argparse.Namespace(targets="", batch=0, config="llama7b")) == []
+    assert bench.target_names(argparse.Namespace(targets="none", batch=0, config=bench.DEFAULT_CONFIG)) == []
+    assert bench.target_names(argparse.Namespace(targets="tiny,llama7b", batch=8, config="tiny")) == \
+        ["tiny", "llama7b"]
 
 
 def test_warmup_below_three_is_refused():

@@ -1,8 +1,14 @@
 """Full-size parity: one step of every benchmark workload at its full size, in
 the launch configuration the benchmark times (the benchmark's own workload
 object: DecodeSession, the workload's partition size, shared-prefix groups,
-copy-on-write forks, chunks, FP8 pools), checked on sampled outputs the
-oracle computes one by one, and on sampled appended rows byte for byte."""
+copy-on-write forks, chunks, FP8 pools).
+
+Every output row (every sequence or chunk row, every query head) is compared
+with the oracle, which computes them all on the host cores; and both whole K/V
+pools after the step are compared byte for byte with the oracle's
+``block_copy`` and ``kv_append`` applied to the pools as they were before it
+(the copy-on-write destinations of the beam workload, every appended row, and
+no write anywhere else)."""
 import numpy as np
 import pytest
 import torch
@@ -17,8 +23,12 @@ WORKLOADS = ["llama7b", "llama13b_prefix", "llama3_gqa_bs16", "llama3_gqa_bs32",
              "llama7b_fp8", "llama3_gqa_fp8"]
 
 
+def _bits(t: torch.Tensor) -> torch.Tensor:
+    return t.view(torch.uint8) if t.dtype == torch.uint8 else t.view(torch.int16)
+
+
 @pytest.mark.parametrize("cfg", WORKLOADS)
-def test_full_size_step_on_sampled_outputs(cfg):
+def test_full_size_step_every_output_and_whole_pools(cfg):
     import bench
     import paged_kv_cache_405_b200 as m
     shape = synth.CONFIGS[cfg]
@@ -33,41 +43,38 @@ def test_full_size_step_on_sampled_outputs(cfg):
     q = synth.randn((Tq, shape.Hq, shape.D), g, dt, "cpu")
     kn = synth.randn((T, shape.Hkv, shape.D), g, dt, "cpu")
     vn = synth.randn((T, shape.Hkv, shape.D), g, dt, "cpu")
+    torch.cuda.synchronize()
+    k0, v0 = wl.session.k_pool.cpu(), wl.session.v_pool.cpu()      # the pools before the step
     out = torch.full((Tq, shape.Hq, shape.D), float("nan"), dtype=dt, device=dev)
     wl.launch(d, q.to(dev), kn.to(dev), vn.to(dev), out)
     torch.cuda.synchronize()
     assert m.device_error() == 0
     kc, vc = wl.session.k_pool.cpu(), wl.session.v_pool.cpu()
+    got = out.cpu()
+    del out, d, wl
+    torch.cuda.empty_cache()
 
-    rng = np.random.default_rng(99)
-    bs = shape.bs
-    # appended rows, byte for byte (the quantized codes for FP8 pools)
-    for i in rng.choice(T, size=min(T, 24), replace=False).tolist():
-        sl = int(p.slot_mapping[i])
-        blk, off = sl // bs, sl % bs
-        if shape.kv_fp8:
-            assert np.array_equal(kc[blk, :, off].numpy(), oracle.quantize_e4m3(kn[i], shape.kv_scale))
-            assert np.array_equal(vc[blk, :, off].numpy(), oracle.quantize_e4m3(vn[i], shape.kv_scale))
-        else:
-            assert torch.equal(kc[blk, :, off].view(torch.int16), kn[i].view(torch.int16))
-            assert torch.equal(vc[blk, :, off].view(torch.int16), vn[i].view(torch.int16))
-
-    # sampled outputs: the longest context, the first and last rows, and random ones
-    lens = np.asarray(p.lens)
-    if shape.chunk:
-        qs = np.asarray(p.query_start)
-        seqs = [int(np.argmax(lens)), 0, len(lens) - 1] + rng.choice(len(lens), size=9).tolist()
-        rows = [int(qs[s] + rng.integers(0, qs[s + 1] - qs[s])) for s in seqs] + [int(qs[-1]) - 1]
+    # the pools: the oracle's copies, then its appends, on the pre-step pools
+    if shape.beams:
+        assert len(p.cow_pairs) == shape.S * (shape.beams - 1)     # 3 copies per parent (4 beams)
+    oracle.block_copy(k0, v0, p.cow_pairs)
+    if shape.kv_fp8:
+        oracle.kv_append_fp8(k0.numpy(), v0.numpy(), kn, vn, shape.kv_scale, shape.kv_scale, p.slot_mapping)
     else:
-        rows = [int(np.argmax(lens)), 0, Tq - 1] + rng.choice(Tq, size=9).tolist()
-    items = [(r, int(rng.integers(0, shape.Hq))) for r in rows]
+        oracle.kv_append(k0, v0, kn, vn, p.slot_mapping)
+    assert torch.equal(_bits(kc), _bits(k0)), "K pool differs from the oracle's copies + appends"
+    assert torch.equal(_bits(vc), _bits(v0)), "V pool differs from the oracle's copies + appends"
+    del k0, v0
+
+    # every output row
+    lens = np.asarray(p.lens)
     th = oracle.max_threads()
     if shape.chunk:
-        ref = oracle.paged_attention_chunk(q, kc, vc, p.block_tables, lens, p.query_start, items=items, threads=th)
+        ref = oracle.paged_attention_chunk(q, kc, vc, p.block_tables, lens, p.query_start, threads=th)
     elif shape.kv_fp8:
         ref = oracle.paged_attention_kv(q, kc.numpy(), vc.numpy(), shape.kv_scale, shape.kv_scale, p.block_tables,
-                                        lens, items=items, threads=th)
+                                        lens, threads=th)
     else:
-        ref = oracle.paged_attention(q, kc, vc, p.block_tables, lens, items=items, threads=th)
-    got = torch.stack([out[r, h] for r, h in items]).cpu()
+        ref = oracle.paged_attention(q, kc, vc, p.block_tables, lens, threads=th)
+    assert ref.shape == tuple(got.shape)
     assert max_err(got, ref) <= TOL[dt]

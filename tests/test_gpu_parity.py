@@ -87,6 +87,27 @@ def test_attention_matches_oracle(cfg, partition_size):
     assert max_err(out, ref) <= TOL[out.dtype]
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 2)])
+@pytest.mark.parametrize("partition_size", [0, 128])
+def test_values_scaled_by_inverse_sqrt_head_dim(dtype, Hq, Hkv, partition_size):
+    """The other reading of the Llama-2-7B-shaped workload's "q/K/V ~N(0,1)
+    scaled 1/sqrt(128)": the values themselves scaled, so the logits are
+    ~N(0, 1/128^2) and the softmax is almost uniform over up to 2048 tokens
+    (long sums of nearly equal weights instead of a peaked softmax).  The
+    outputs are then ~0.09/sqrt(L), below the absolute tolerance, so they are
+    also held to 2e-2 of their own largest magnitude (an all-zero output
+    fails that)."""
+    import math
+    sh = synth.shrink(synth.CONFIGS["llama7b"], S=10, Hq=Hq, Hkv=Hkv, dtype=dtype, seed=21)
+    b = synth.make_batch(sh, value_scale=1 / math.sqrt(128), fill_unused=float("nan"))
+    ref = oracle_attention(b)
+    out = gpu_attention(b, partition_size=partition_size)
+    err = max_err(out, ref)
+    assert err <= TOL[out.dtype]
+    assert err <= 2e-2 * float(np.abs(ref).max())
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f16", "f32"])
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (8, 4), (16, 2), (32, 2), (8, 1)])
 @pytest.mark.parametrize("bs", [16, 32, 64])
