@@ -168,9 +168,10 @@ pkv_status pkv_paged_attention_decode(void* out, const void* q, const void* k_po
  *                 block-table entries of the group's first sequence; only
  *                 members whose own first entries are the same take its
  *                 result ([E] 6.1, [T] 2.2.8: only identical prefixes are
- *                 shared).  Every kernel of the call compares them on the
- *                 device; a member whose entries differ is recorded
- *                 (PKV_DEVERR_GROUP) and handled as a non-member.
+ *                 shared).  The call compares them on the device, once
+ *                 per sequence, before its attention kernels run; a member
+ *                 whose entries differ is recorded (PKV_DEVERR_GROUP) and
+ *                 handled as a non-member.
  *   max_group_size  host bound on members per group (it sizes the prefix
  *                 pass); members past it are recorded (PKV_DEVERR_GROUP)
  *                 and handled as non-members.
@@ -193,7 +194,10 @@ pkv_status pkv_paged_attention_decode_shared(void* out, const void* q, const voi
                                              pkv_dtype dtype, void* stream);
 
 /* Workspace bytes for pkv_paged_attention_decode_shared (arguments as in
- * pkv_attention_workspace_bytes; never 0 for num_seqs > 0). */
+ * pkv_attention_workspace_bytes; never 0 for num_seqs > 0): the split-K
+ * partials with one extra slot per row, then 8 bytes per sequence in which
+ * the call records, once, whether the sequence takes its group's prefix
+ * result. */
 size_t pkv_attention_shared_workspace_bytes(int num_seqs, int num_q_heads, int head_dim, int max_context_len,
                                             int partition_size);
 

@@ -27,6 +27,10 @@ struct AttnParams {
     int num_groups;
     int max_group_size;           // prefix-pass grid covers groups up to this many sequences
     int max_shared;               // ... and shared runs up to this many tokens
+    // Membership decided once per call by group_members_kernel (nullptr: no
+    // groups): member[s] = (group index + 1, shared tokens) when sequence s
+    // takes its group's prefix result, (0, 0) otherwise.
+    const int2* member;
 };
 
 // A chunk of new tokens per sequence (causal): sequence s owns query rows
@@ -111,27 +115,16 @@ __device__ __forceinline__ int load_context_len(const AttnParams& p, int s, bool
     return L;
 }
 
-// Warp-collective (every lane of the warp, same s and part).
-__device__ __forceinline__ Unit resolve_unit(const AttnParams& p, int s, int part, bool report, int lane) {
+__device__ __forceinline__ Unit resolve_unit(const AttnParams& p, int s, int part, bool report) {
     Unit u;
     u.L = load_context_len(p, s, report);
     u.shared = 0;
     u.member = false;
-    const int gi = find_group(p, s);
-    if (gi >= 0) {
-        const int sh = group_shared_len(p, gi, u.L, report);
-        if (sh > 0) {
-            // A member past the prefix pass's grid (max_group_size), or whose
-            // leading blocks are not the group's, attends to its whole context
-            // through its own table, like a non-member.
-            const int first = group_first_seq(p.group_first, gi, p.S);
-            if (s - first < p.max_group_size &&
-                same_leading_blocks(p.block_tables, p.maxB, p.bs, s, first, sh, lane)) {
-                u.shared = sh;
-                u.member = true;
-            } else if (report) {
-                flag_error(16u /* PKV_DEVERR_GROUP */);
-            }
+    if (p.member != nullptr) {
+        const int2 m = p.member[s];
+        if (m.x > 0 && m.y > 0 && m.y <= u.L) {
+            u.shared = m.y;
+            u.member = true;
         }
     }
     u.npre = (u.shared + p.P - 1) / p.P;
@@ -141,6 +134,37 @@ __device__ __forceinline__ Unit resolve_unit(const AttnParams& p, int s, int par
     u.slot = u.npre + part;
     u.direct = !u.member && u.nsuf == 1;
     return u;
+}
+
+// Shared-prefix membership of every sequence of a call, decided once before
+// the attention kernels run (one warp per sequence, 8 per CTA), so that the
+// decode kernels, the prefix pass and the reduce all read the same answer
+// from member[s] (see AttnParams::member).  A sequence of group gi takes the
+// prefix result when the group's shared length is usable for it (a multiple
+// of block_size within its context and within max_shared_len), it lies
+// within max_group_size of the group's first sequence (the prefix pass's
+// grid), and its first shared/block_size table entries are the first
+// sequence's -- the blocks the prefix pass reads.  Failures are recorded once
+// per sequence; such a sequence attends to its whole context through its own
+// table.
+__global__ void __launch_bounds__(256) group_members_kernel(const AttnParams p, int2* member) {
+    const int lane = threadIdx.x & 31;
+    const int s = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (s >= p.S) return;
+    int2 m = make_int2(0, 0);
+    const int L = load_context_len(p, s, false);  // a bad length is reported by the decode kernels
+    const int gi = find_group(p, s);
+    if (gi >= 0) {
+        const int sh = group_shared_len(p, gi, L, lane == 0);
+        if (sh > 0) {
+            const int first = group_first_seq(p.group_first, gi, p.S);
+            const bool within = s - first < p.max_group_size;
+            const bool same = same_leading_blocks(p.block_tables, p.maxB, p.bs, s, first, sh, lane);
+            if (within && same) m = make_int2(gi + 1, sh);
+            else if (lane == 0) flag_error(16u /* PKV_DEVERR_GROUP */);
+        }
+    }
+    if (lane == 0) member[s] = m;
 }
 
 // Block-table window held in registers: lane l holds entry (first + base + l)

@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_fp8_kernel(const Att
     const int G = p.G;
     const int h0 = g * G;
 
-    const Unit u = resolve_unit(p, s, part, part == 0 && g == 0 && lane == 0, lane);
+    const Unit u = resolve_unit(p, s, part, part == 0 && g == 0 && lane == 0);
     if (u.t_begin >= u.L) {
         if (part == 0 && u.L == 0) {  // empty context: zeros for the group's heads
             To* o = reinterpret_cast<To*>(p.out) + ((int64_t)s * p.Hq + h0) * D;
@@ -298,7 +298,7 @@ __global__ void __launch_bounds__(WARPS * 32, 4) paged_attn_fp8_head_kernel(cons
     const int gid = lane >> 2, tig = lane & 3;
     const int g = h / p.G;
 
-    const Unit u = resolve_unit(p, s, part, part == 0 && h == 0 && lane == 0, lane);
+    const Unit u = resolve_unit(p, s, part, part == 0 && h == 0 && lane == 0);
     if (u.t_begin >= u.L) {
         if (part == 0 && u.L == 0) {  // empty context: zeros
             To* o = reinterpret_cast<To*>(p.out) + ((int64_t)s * p.Hq + h) * D;

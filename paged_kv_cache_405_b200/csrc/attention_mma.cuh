@@ -347,7 +347,7 @@ __global__ void __launch_bounds__(WARPS * 32) paged_attn_mma_kernel(const AttnPa
     const int G = p.G;
     const int h0 = g * G;
 
-    const Unit u = resolve_unit(p, s, part, part == 0 && g == 0 && lane == 0, lane);
+    const Unit u = resolve_unit(p, s, part, part == 0 && g == 0 && lane == 0);
     if (u.t_begin >= u.L) {
         if (part == 0 && u.L == 0) {  // empty context: zeros for the group's heads
             T* o = reinterpret_cast<T*>(p.out) + ((int64_t)s * p.Hq + h0) * D;
@@ -420,33 +420,15 @@ __global__ void __launch_bounds__(WARPS * 32) prefix_attn_mma_kernel(const AttnP
     const int per = ((t1 - t0 + WARPS * kTileTok - 1) / (WARPS * kTileTok)) * kTileTok;
     const int w0 = min(t1, t0 + warp * per), w1 = min(t1, w0 + per);
 
-    // Rows of this tile that take the prefix result (bit k: row tile*16 + k):
-    // those whose sequence's context covers the shared run and whose leading
-    // blocks are the group's -- the decode kernels and the reduce apply the
-    // same tests (and report the failures), so a sequence failing them is
-    // attended wholly by its own partitions and gets no prefix partial.
-    unsigned live = 0;
-    {
-        int prev = -1;
-        bool prev_ok = false;
-        for (int k = 0; k < 16 && tile * 16 + k < rows; ++k) {
-            const int sq = first + (tile * 16 + k) / G;  // warp-uniform
-            if (sq != prev) {
-                const int L = min(max(p.context_lens[sq], 0), p.max_len);  // same clamp as the decode kernels
-                const bool same = same_leading_blocks(p.block_tables, p.maxB, p.bs, sq, first, shared, lane);
-                prev_ok = L >= shared && same;
-                prev = sq;
-            }
-            if (prev_ok) live |= 1u << k;
-        }
-    }
-    // Query rows of this lane (gid, gid+8).
+    // Query rows of this lane (gid, gid+8).  Only rows whose sequence takes
+    // this group's prefix result (decided once per call, see
+    // group_members_kernel) are attended and written.
     int rs[2], rh[2];
     bool use[2];
 #pragma unroll
     for (int hi = 0; hi < 2; ++hi) {
         const int r = tile * 16 + gid + 8 * hi;
-        use[hi] = ((live >> (gid + 8 * hi)) & 1u) != 0;
+        use[hi] = r < rows && p.member[first + r / G].x == gi + 1;
         rs[hi] = first + (use[hi] ? r / G : 0);
         rh[hi] = g * G + (use[hi] ? r % G : 0);
     }
@@ -488,9 +470,10 @@ __global__ void __launch_bounds__(WARPS * 32) prefix_attn_mma_kernel(const AttnP
     static_assert(kCols % 4 == 0, "float4 columns");
     const int r = threadIdx.x / kPerRow;
     const int c0 = (threadIdx.x % kPerRow) * kCols;
-    if (((live >> r) & 1u) == 0) return;  // also every row past the group
     const int rr = tile * 16 + r;
+    if (rr >= rows) return;
     const int s_r = first + rr / G, h_r = g * G + rr % G;
+    if (p.member[s_r].x != gi + 1) return;
     float M = -INFINITY;
 #pragma unroll
     for (int w = 0; w < WARPS; ++w) M = fmaxf(M, sm[w * 16 + r]);

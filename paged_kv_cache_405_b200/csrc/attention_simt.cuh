@@ -126,7 +126,7 @@ __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_simt_kernel(const At
     const int s = blockIdx.z;
     if (h >= p.Hq) return;
 
-    const Unit u = resolve_unit(p, s, part, part == 0 && h == 0 && lane == 0, lane);
+    const Unit u = resolve_unit(p, s, part, part == 0 && h == 0 && lane == 0);
     const int sub = lane / LPT;  // which token of a pass
     const int c = lane % LPT;    // which 16-byte slice of the row
     if (u.t_begin >= u.L) {

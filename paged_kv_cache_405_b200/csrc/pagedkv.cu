@@ -89,10 +89,13 @@ static size_t workspace_for(int S, int Hq, int D, int max_len, int P) {
 
 // Shared-prefix mode: one more partial slot per (sequence, head) than
 // partitions, since a member's prefix and suffix partitions can each end
-// part-way through a partition.
+// part-way through a partition; then the per-sequence membership (8 bytes
+// per sequence, see group_members_kernel).
 static size_t shared_workspace_for(int S, int Hq, int D, int max_len, int P) {
     const int64_t slots = ((int64_t)max_len + P - 1) / P + 1;
-    return partials_bytes((int64_t)S * Hq, slots, D);
+    const size_t parts = partials_bytes((int64_t)S * Hq, slots, D);
+    const size_t members = ((size_t)S * sizeof(int2) + 255) / 256 * 256;
+    return parts > SIZE_MAX - members ? SIZE_MAX : parts + members;
 }
 
 // Smallest partition the library's own choice can produce for max_len: the
@@ -346,6 +349,11 @@ static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int npart
         if (use_mma || shared_mode) return cudaErrorInvalidValue;
         e = decode_pass<T>(p, D, nparts, use_mma, mk, mv, st);
     } else {
+        if (shared_mode && p.num_groups > 0) {  // membership first: every later kernel reads it
+            e = launch_k(pkv::group_members_kernel, dim3((unsigned)((p.S + 7) / 8)), dim3(256), 0, st, p,
+                         const_cast<int2*>(p.member));
+            if (e != cudaSuccess) return e;
+        }
         if (shared_mode && p.num_groups > 0 && npre > 0) {
             const int tiles = (p.max_group_size * p.G + 15) / 16;
             dim3 grid(tiles, npre, p.num_groups * p.Hkv);
@@ -368,8 +376,7 @@ static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int npart
     }
     if (e != cudaSuccess || p.maxP <= 1) return e;
     pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
-                        p.group_first, p.group_shared, p.num_groups, p.max_shared, p.max_group_size,
-                        p.block_tables, p.maxB, nullptr, 0};
+                        p.member, nullptr, 0};
     return D == 64 ? launch_reduce<T, 64>(r, st) : launch_reduce<T, 128>(r, st);
 }
 
@@ -386,7 +393,7 @@ static cudaError_t dispatch_attention_fp8(const pkv::AttnParams& p, int D, int n
     }
     if (e != cudaSuccess || p.maxP <= 1) return e;
     pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
-                        nullptr, nullptr, 0, 0, 0, p.block_tables, p.maxB, nullptr, 0};
+                        nullptr, nullptr, 0};
     return D == 64 ? launch_reduce<To, 64>(r, st) : launch_reduce<To, 128>(r, st);
 }
 
@@ -550,6 +557,8 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
     p.num_groups = grp.num;
     p.max_group_size = grp.max_size;
     p.max_shared = grp.max_shared;
+    // Shared-prefix membership after the partials (8-byte aligned: (D+2)*4 is).
+    p.member = grp.mode && grp.num > 0 ? reinterpret_cast<const int2*>(p.ws_ml + n_part * 2) : nullptr;
 
     const bool use_mma = dtype != PKV_F32 && p.G >= 2 && p.G <= 16;
     CUtensorMap mk, mv;
@@ -828,7 +837,7 @@ static cudaError_t dispatch_chunk(const pkv::AttnParams& p, const pkv::ChunkPara
         cudaError_t e = D == 64 ? launch_chunk<T, 64>(p, c, grid, mk, mv, st) : launch_chunk<T, 128>(p, c, grid, mk, mv, st);
         if (e != cudaSuccess || c.nparts <= 1) return e;
         pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
-                            nullptr, nullptr, 0, 0, 0, p.block_tables, p.maxB, c.query_start, c.T};
+                            nullptr, c.query_start, c.T};
         return D == 64 ? launch_reduce<T, 64>(r, st) : launch_reduce<T, 128>(r, st);
     }
 }

@@ -18,20 +18,14 @@ struct ReduceParams {
     const float* ws_ml;         // [S][Hq][maxP][2]
     const int32_t* context_lens;
     int S, Hq, D, P, maxP, max_len, bs;
-    const int32_t* group_first;   // shared-prefix groups, as in AttnParams
-    const int32_t* group_shared;
-    int num_groups, max_shared, max_group_size;
-    const int32_t* block_tables;  // [S][maxB] (members' leading blocks are compared)
-    int maxB;
+    const int2* member;           // shared-prefix membership, as in AttnParams (nullptr: none)
     const int32_t* query_start;   // chunk mode (non-null): rows are (query row, head), [S + 1]
     int T;
 };
 
 // Partials to merge for one output row (0 = the attention kernel wrote it).
-// qs / gf: query_start / group_first, from global memory or a shared copy.
-// Warp-collective (every lane of the warp, same row).
-__device__ __forceinline__ int reduce_count(const ReduceParams& p, int row, const int32_t* qs,
-                                            const int32_t* gf, int lane) {
+// qs: query_start, from global memory or a shared copy.
+__device__ __forceinline__ int reduce_count(const ReduceParams& p, int row, const int32_t* qs) {
     const int h_rows = p.Hq;
     if (p.query_start) {  // causal chunk: row = t * Hq + h
         const int t = row / h_rows;
@@ -54,23 +48,12 @@ __device__ __forceinline__ int reduce_count(const ReduceParams& p, int row, cons
     int L = p.context_lens[s];
     if (L < 0) L = 0;
     if (L > p.max_len) L = p.max_len;
-    // A member of a valid shared-prefix group has ceil(shared/P) prefix
-    // partials followed by its own ones (same rule as the attention kernels).
+    // A member of a shared-prefix group has ceil(shared/P) prefix partials
+    // followed by its own ones (same rule as the attention kernels).
     int shared = 0;
-    if (p.num_groups > 0 && s >= gf[0] && s < gf[p.num_groups]) {
-        int lo = 0, hi = p.num_groups;
-        while (hi - lo > 1) {
-            const int mid = (lo + hi) >> 1;
-            if (gf[mid] <= s) lo = mid;
-            else hi = mid;
-        }
-        const int sh = p.group_shared[lo];
-        if (sh > 0 && sh % p.bs == 0 && sh <= L && sh <= p.max_shared) {
-            const int first = max(0, min(gf[lo], p.S));
-            if (s - first < p.max_group_size &&
-                same_leading_blocks(p.block_tables, p.maxB, p.bs, s, first, sh, lane))
-                shared = sh;
-        }
+    if (p.member != nullptr) {
+        const int2 m = p.member[s];
+        if (m.x > 0 && m.y > 0 && m.y <= L) shared = m.y;
     }
     const int nsuf = (L - shared + p.P - 1) / p.P;
     const int nP = (shared + p.P - 1) / p.P + nsuf;
@@ -105,7 +88,7 @@ __global__ void __launch_bounds__(W * ROWS * 32) splitk_reduce_kernel(const Redu
     float (&s_max)[W] = s_max_all[sub];
     const int nrows = p.query_start ? p.T * p.Hq : p.S * p.Hq;
     if (row >= nrows) return;  // whole rows return together (W warps of a row)
-    const int nP = reduce_count(p, row, p.query_start, p.group_first, lane);
+    const int nP = reduce_count(p, row, p.query_start);
     if (nP == 0) return;
     const int64_t base = (int64_t)row * p.maxP;
     const float* ml = p.ws_ml + base * 2;
@@ -190,10 +173,10 @@ __global__ void __launch_bounds__(W * ROWS * 32) splitk_reduce_kernel(const Redu
 // (m, l) pair of every slot (lane i holds slot i) and, with SPEC >= maxP, the
 // partial outputs of every slot -- together with the context length, so a
 // row costs one round trip to memory (two without SPEC).  A chunk call's
-// query_start, or a shared-prefix call's group_first, is searched in a
-// shared-memory copy when it fits.  Slots past the row's count are never
-// used (selected out, so stale values cannot leak in); the outputs are
-// summed in slot order, so the result does not depend on timing.
+// query_start is searched in a shared-memory copy when it fits.  Slots past
+// the row's count are never used (selected out, so stale values cannot leak
+// in); the outputs are summed in slot order, so the result does not depend
+// on timing.
 constexpr int kReduceIdxMax = 4096;
 
 template <typename T, int D, int ROWS, int SPEC>
@@ -203,14 +186,11 @@ __global__ void __launch_bounds__(ROWS * 32) splitk_reduce_warp_kernel(const Red
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = blockIdx.x * ROWS + warp;
     const int32_t* qs = p.query_start;
-    const int32_t* gf = p.group_first;
-    const int32_t* src = qs ? qs : (p.num_groups > 0 ? gf : nullptr);
-    const int n_idx = qs ? p.S + 1 : p.num_groups + 1;
-    if (src != nullptr && n_idx <= kReduceIdxMax) {  // uniform over the CTA
-        for (int i = threadIdx.x; i < n_idx; i += ROWS * 32) s_idx[i] = src[i];
+    const int n_idx = p.S + 1;
+    if (qs != nullptr && n_idx <= kReduceIdxMax) {  // uniform over the CTA
+        for (int i = threadIdx.x; i < n_idx; i += ROWS * 32) s_idx[i] = qs[i];
         __syncthreads();
-        if (qs) qs = s_idx;
-        else gf = s_idx;
+        qs = s_idx;
     }
     const int nrows = p.query_start ? p.T * p.Hq : p.S * p.Hq;
     if (row >= nrows) return;
@@ -231,7 +211,7 @@ __global__ void __launch_bounds__(ROWS * 32) splitk_reduce_warp_kernel(const Red
             }
         }
     }
-    const int nP = reduce_count(p, row, qs, gf, lane);
+    const int nP = reduce_count(p, row, qs);
     if (nP == 0) return;
 
     float M = lane < nP ? mlv.x : -INFINITY;

@@ -293,7 +293,8 @@ def test_workspace_queries_cover_every_call_random():
     """For random shapes, the size each workspace query reports holds the
     partials the call writes under the partition size the library picks:
     (rows) x (partitions, + 1 slot in shared-prefix mode) x (D + 2) floats
-    whenever a context spans more than one partition."""
+    whenever a context spans more than one partition, and in shared-prefix
+    mode 8 bytes per sequence of membership after them."""
     import numpy as np
     rng = np.random.default_rng(0)
     for _ in range(2000):
@@ -307,7 +308,7 @@ def test_workspace_queries_cover_every_call_random():
         per = Hq * (D + 2) * 4
         ws = pkv.attention_workspace_bytes(S, Hq, D, max_len, P)
         assert ws >= (S * nparts * per if nparts > 1 else 0)
-        assert pkv.attention_shared_workspace_bytes(S, Hq, D, max_len, P) >= S * (nparts + 1) * per
+        assert pkv.attention_shared_workspace_bytes(S, Hq, D, max_len, P) >= S * (nparts + 1) * per + 8 * S
         T = S * int(rng.integers(1, 5))
         cw = pkv.attention_chunk_workspace_bytes(T, Hq, D, max_len, P)
         assert cw >= (T * nparts * per if nparts > 1 else 0)

@@ -49,8 +49,9 @@ def test_static_scratch_rejects_oversized_calls():
     b = synth.make_batch(synth.shrink(synth.CONFIGS["llama7b"], S=4, Hq=8, Hkv=8, len_uniform=(1, 64)))
     d = to_dev(b)
     out = torch.zeros_like(d["q"])
-    # 4 seqs x 8 heads x (2^20 / 16) partitions x 130 floats is far beyond the buffer
-    bt = torch.zeros((4, (1 << 20) // 16), dtype=torch.int32, device="cuda")
+    # 4 seqs x 8 heads x 8192 partitions of 16 tokens x 130 floats = 136 MB: a
+    # valid call otherwise, but beyond the 64 MiB buffer
+    bt = torch.zeros((4, 8192), dtype=torch.int32, device="cuda")
     with pytest.raises(pkv.PagedKVError) as e:
         pkv.paged_attention_decode_static(out, d["q"], d["k"], d["v"], bt, d["cl"], partition_size=16)
     assert "scratch" in str(e.value)
