@@ -599,13 +599,15 @@ def host_batch(shape, seed):
 
 def run_e2e(args, wl, world, rank, dev):
     """The same steps through the public API from host buffers: every step's
-    q / new K / new V go in from pinned host memory (one packed copy), its
-    plan goes in (one packed copy), the attention output comes back and the
-    host waits for it before the next step's inputs are sent.  The next
-    step's host planning (allocator calls) runs while the device works, as a
-    serving loop that schedules ahead would."""
+    q / new K / new V arrive in pinned host memory, DecodeSession.launch_step
+    sends them and the step's plan to the device, runs block_copy, kv_append
+    and attention and copies the output back, and the host waits for that
+    output before the next step's inputs go.  The next step's host planning
+    (allocator calls) runs while the device works, as a serving loop that
+    schedules ahead would."""
     import paged_kv_cache_405_b200 as pkv
     shape = wl.shape
+    ss = wl.session
     K, W = args.steps, args.warmup
     dt = synth.DTYPES[shape.dtype]
     T = shape.S * max(1, shape.beams, shape.chunk)
@@ -616,38 +618,32 @@ def run_e2e(args, wl, world, rank, dev):
     for sh_ in shapes:
         offs.append(total)
         total += (int(np.prod(sh_)) * esz + 255) // 256 * 256
-    host_inputs = []
+    host_inputs = []        # per step: q, new K, new V in one pinned host buffer
     for i in range(W + K):
         g = torch.Generator().manual_seed(104729 * (i + 1) + rank)
         buf = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+        views = []
         for sh_, o in zip(shapes, offs):
             t = synth.randn(sh_, g, dt, "cpu")
             buf[o:o + t.numel() * esz].copy_(t.reshape(-1).view(torch.uint8))
-        host_inputs.append(buf)
+            views.append(buf[o:o + t.numel() * esz].view(dt).view(sh_))
+        host_inputs.append((buf, views))
     out_host = torch.empty(shapes[0], dtype=dt, pin_memory=True)
     stream = torch.cuda.current_stream()
     plans = []
-
-    def issue(i, p):
-        d = wl.upload(p)
-        dbuf = host_inputs[i].to(dev, non_blocking=True)
-        q, kd, vd = (dbuf[o:o + int(np.prod(sh_)) * esz].view(dt).view(sh_) for sh_, o in zip(shapes, offs))
-        out = torch.empty_like(q)
-        wl.launch(d, q, kd, vd, out)
-        out_host.copy_(out, non_blocking=True)
 
     def run(first, n):
         p = wl.plan()
         plans.append(p)
         for i in range(first, first + n):
-            issue(i, p)
+            ss.launch_step(p, *host_inputs[i][1], out_host=out_host, stream=stream)
             if i + 1 < first + n:
                 p = wl.plan()       # host work of the next step, overlapping this step's kernels
                 plans.append(p)
             stream.synchronize()    # this step's output is on the host
 
     def plan_bytes(p):
-        arrs = [p.slot_mapping, p.cow_pairs, p.lens, p.block_tables]
+        arrs = [p.slot_mapping, p.lens, p.block_tables] + ([p.cow_pairs] if len(p.cow_pairs) else [])
         if shape.chunk:
             arrs.append(p.query_start)
         elif p.has_groups:
@@ -668,12 +664,13 @@ def run_e2e(args, wl, world, rank, dev):
     tot = sum_over_ranks(float(sum(nbytes)), world)
     if pkv.device_error() != 0:
         raise RuntimeError("device-side check failed during the end-to-end steps")
-    h2d = total + plan_bytes(timed[-1])
+    h2d = sum(int(np.prod(sh_)) * esz for sh_ in shapes) + plan_bytes(timed[-1])
     d2h = out_host.numel() * out_host.element_size()
     return {"value": round(tot / (ms * 1e-3) / 1e9, 1), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms / K, 4),
-            "api": "DecodeSession plan (next step planned during this one) + packed pinned H2D of inputs and plan "
-                   "+ block_copy/kv_append/attention + D2H of the output, host waits for it every step"}
+            "api": "DecodeSession.plan (next step planned during this one) + DecodeSession.launch_step (H2D of "
+                   "the inputs from pinned host memory and of the plan, block_copy/kv_append/attention, D2H of "
+                   "the output), host waits for the output every step"}
 
 
 def run_reference(args, world, rank):

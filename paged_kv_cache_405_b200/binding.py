@@ -209,6 +209,23 @@ def _ranged(cname: str):
     return wrap
 
 
+def raw_call(cname: str, *args) -> None:
+    """Call the C entry point ``cname`` with arguments already marshalled
+    (device pointers as ints, sizes, a stream handle) and raise on a non-OK
+    status.  For callers that checked their buffers against the sizes once,
+    up front (``DecodeSession``'s host-buffer steps reuse buffers it made
+    itself); the C call still does its own argument checks."""
+    f = getattr(lib, cname)
+    if not _NVTX:
+        _check(f(*args))
+        return
+    torch.cuda.nvtx.range_push(cname)
+    try:
+        _check(f(*args))
+    finally:
+        torch.cuda.nvtx.range_pop()
+
+
 # ------------------------------------------------------------------ device calls
 @_ranged("pkv_kv_append")
 def kv_append(k_new, v_new, k_pool, v_pool, slot_mapping, stream=None) -> None:

@@ -96,6 +96,8 @@ class DecodeSession:
             ws = max(ws, B.attention_shared_workspace_bytes(n, num_q_heads, self.head_dim, max_len, partition_size))
         self.workspace = torch.empty(max(256, ws), dtype=torch.uint8, device=self.device)
         self._pinned = {}
+        self._layouts = {}      # host-buffer steps: staging per layout of the step's arrays
+        self._io = {}           # host-buffer steps: device q / new K / new V / out per shape
 
     # ------------------------------------------------------------ host side
     def add(self, sid: int, num_tokens: int = 0, shared_prefix: Optional[Sequence[int]] = None,
@@ -278,21 +280,163 @@ class DecodeSession:
 
     def step(self, q_host: torch.Tensor, k_new_host: torch.Tensor, v_new_host: torch.Tensor,
              attend: Sequence[int], out_host: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-        """A full step from host buffers: plan, copy inputs in, run, copy the output back."""
+        """A full step from host buffers: plan, copy inputs in, run, copy the output back, wait."""
         p = self.plan(attend)
         s = torch.cuda.current_stream() if stream is None else stream
-        with torch.cuda.stream(s):
-            d = self.upload(p)
-            q = q_host.to(self.device, non_blocking=True)
-            kn = k_new_host.to(self.device, non_blocking=True)
-            vn = v_new_host.to(self.device, non_blocking=True)
-            out = torch.empty_like(q)
-            self.launch(d, q, kn, vn, out, stream=s)
-            if out_host is None:
-                out_host = self._pin("out", out)
-            out_host.copy_(out, non_blocking=True)
+        out_host = self.launch_step(p, q_host, k_new_host, v_new_host, out_host, stream=s)
         s.synchronize()
         return out_host
+
+    # ------------------------------------------------- host-buffer steps
+    # A serving loop hands each step's inputs over in host memory and wants
+    # the output back in host memory.  launch_step does that for a planned
+    # step with as little host work as it can: the plan's arrays are packed
+    # into a pinned staging buffer and sent with one copy into a device buffer
+    # made for that layout of arrays; q / new K / new V go into device buffers
+    # kept per shape; the three C calls are made directly with pointers that
+    # were checked against the sizes when those buffers were made; the output
+    # comes back with one copy.  Nothing is allocated once a layout has been
+    # seen, so the host cost is a few copies and three C calls.
+    #
+    # Reuse rules: the device buffers of a layout are reused by later steps of
+    # the same layout, so all host-buffer steps of a session go on one stream
+    # (stream order then keeps a step's kernels ahead of the next step's
+    # copies into the same buffers).  Two staging buffers alternate per
+    # layout, and one is refilled only after its previous copy has completed.
+
+    _MAX_LAYOUTS = 32
+
+    def _staged(self, arrays, stream) -> list:
+        """Device views of ``arrays`` (host numpy), sent with one copy on ``stream``."""
+        key = tuple((a.dtype.str, a.shape) for a in arrays)
+        lay = self._layouts.get(key)
+        if lay is None:
+            if len(self._layouts) >= self._MAX_LAYOUTS:
+                self._layouts.pop(next(iter(self._layouts)))
+            offs, total = [], 0
+            for a in arrays:
+                offs.append(total)
+                total += (a.nbytes + 255) // 256 * 256
+            total = max(total, 256)
+            sets = []
+            for _ in range(2):
+                host = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+                dev = torch.empty(total, dtype=torch.uint8, device=self.device)
+                hv = host.numpy()
+                hviews = [hv[o:o + a.nbytes].view(a.dtype).reshape(a.shape) for a, o in zip(arrays, offs)]
+                dviews = [dev[o:o + a.nbytes].view(torch.from_numpy(a[:0].reshape(-1)).dtype).view(a.shape)
+                          for a, o in zip(arrays, offs)]
+                sets.append({"host": host, "dev": dev, "hviews": hviews, "dviews": dviews,
+                             "ptrs": [t.data_ptr() for t in dviews], "event": None})
+            lay = self._layouts[key] = [0, sets]
+        lay[0] ^= 1
+        st = lay[1][lay[0]]
+        if st["event"] is not None:
+            st["event"].synchronize()           # the previous copy out of this staging buffer is done
+        for hv, a in zip(st["hviews"], arrays):
+            np.copyto(hv, a, casting="no")
+        st["dev"].copy_(st["host"], non_blocking=True)
+        if st["event"] is None:
+            st["event"] = torch.cuda.Event()
+        st["event"].record(stream)
+        return st
+
+    def _io_buffers(self, q_host, k_new_host, v_new_host):
+        """Device q / new K / new V / out for these host shapes (made once per shape)."""
+        key = (tuple(q_host.shape), tuple(k_new_host.shape), q_host.dtype, k_new_host.dtype)
+        io = self._io.get(key)
+        if io is None:
+            if q_host.dim() != 3 or tuple(q_host.shape[1:]) != (self.num_q_heads, self.head_dim):
+                raise ValueError("q must be [rows, num_q_heads, head_dim]")
+            if k_new_host.dim() != 3 or tuple(k_new_host.shape[1:]) != (self.num_kv_heads, self.head_dim):
+                raise ValueError("new K/V must be [T, num_kv_heads, head_dim]")
+            if self.fp8:
+                if q_host.dtype not in (torch.bfloat16, torch.float16):
+                    raise TypeError("q must be bf16 or f16 with FP8 pools")
+            elif q_host.dtype != self.k_pool.dtype or k_new_host.dtype != self.k_pool.dtype:
+                raise TypeError("q and new K/V must have the pools' element type")
+            if len(self._io) >= self._MAX_LAYOUTS:
+                self._io.pop(next(iter(self._io)))
+            q = torch.empty(q_host.shape, dtype=q_host.dtype, device=self.device)
+            kn = torch.empty(k_new_host.shape, dtype=k_new_host.dtype, device=self.device)
+            vn = torch.empty(k_new_host.shape, dtype=k_new_host.dtype, device=self.device)
+            out = torch.empty_like(q)
+            io = self._io[key] = (q, kn, vn, out)
+        if v_new_host.shape != k_new_host.shape or v_new_host.dtype != k_new_host.dtype:
+            raise ValueError("k_new and v_new must have the same shape and element type")
+        return io
+
+    def launch_step(self, p, q_host: torch.Tensor, k_new_host: torch.Tensor, v_new_host: torch.Tensor,
+                    out_host: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        """Issue one planned step (a StepPlan, or a ChunkPlan) from host
+        buffers without waiting: the plan and the inputs go to the device,
+        block_copy -> kv_append -> attention run, and the output is copied into
+        ``out_host`` (pinned; made if None) -- complete once ``stream`` reaches
+        this point.  q_host [rows, num_q_heads, head_dim]; k/v_new_host
+        [tokens written, num_kv_heads, head_dim]; pinned host memory lets the
+        copies run asynchronously."""
+        s = torch.cuda.current_stream() if stream is None else stream
+        chunk = isinstance(p, ChunkPlan)
+        T = len(p.slot_mapping)
+        rows = T if chunk else len(p.seq_ids)
+        if q_host.shape[0] != rows or k_new_host.shape[0] != T:
+            raise ValueError("q needs one row per %s and new K/V one per written token"
+                             % ("new token" if chunk else "attending sequence"))
+        q, kn, vn, out = self._io_buffers(q_host, k_new_host, v_new_host)
+        if out_host is None:
+            out_host = self._pin("out", out)
+        elif out_host.shape != out.shape or out_host.dtype != out.dtype:
+            raise ValueError("out_host must have the shape and element type of q")
+        n_cow = len(p.cow_pairs)
+        arrays = [p.slot_mapping, p.lens, p.block_tables] + ([p.cow_pairs] if n_cow else [])
+        if chunk:
+            arrays.append(p.query_start)
+        elif p.has_groups:
+            arrays += [p.group_first, p.group_shared]
+        with torch.cuda.stream(s):
+            st = self._staged(arrays, s)
+            q.copy_(q_host, non_blocking=True)
+            kn.copy_(k_new_host, non_blocking=True)
+            vn.copy_(v_new_host, non_blocking=True)
+            self._calls(p, st["ptrs"], n_cow, q, kn, vn, out, s.cuda_stream)
+            out_host.copy_(out, non_blocking=True)
+        return out_host
+
+    def _calls(self, p, ptrs, n_cow, q, kn, vn, out, sh) -> None:
+        """block_copy -> kv_append -> attention through the C ABI, on the
+        staged plan (pointers in the order launch_step packed the arrays)."""
+        NB, Hkv, bs, D = self.num_blocks, self.num_kv_heads, self.block_size, self.head_dim
+        kp, vp = self.k_pool.data_ptr(), self.v_pool.data_ptr()
+        sm, cl, bt = ptrs[0], ptrs[1], ptrs[2]
+        maxB = p.block_tables.shape[1]
+        T = len(p.slot_mapping)
+        if n_cow:
+            B.raw_call("pkv_block_copy", kp, vp, ptrs[3], n_cow, NB, Hkv, D, bs,
+                       B.FP8_E4M3 if self.fp8 else B._dt(self.k_pool), sh)
+        qdt = B._dt(q)
+        if self.fp8:
+            B.raw_call("pkv_kv_append_fp8", kn.data_ptr(), vn.data_ptr(), kp, vp, sm, T, NB, Hkv, D, bs,
+                       B._dt(kn), float(self.kv_scales[0]), float(self.kv_scales[1]), sh)
+        else:
+            B.raw_call("pkv_kv_append", kn.data_ptr(), vn.data_ptr(), kp, vp, sm, T, NB, Hkv, D, bs, qdt, sh)
+        ws, wsb = self.workspace.data_ptr(), self.workspace.numel()
+        P = self.partition_size
+        rest = ptrs[3 + (1 if n_cow else 0):]
+        if isinstance(p, ChunkPlan):
+            B.raw_call("pkv_paged_attention_chunk", out.data_ptr(), q.data_ptr(), kp, vp, bt, maxB, cl, rest[0],
+                       len(p.lens), T, int(p.max_query_len), self.num_q_heads, Hkv, D, bs, NB, 0.0, P, ws, wsb,
+                       qdt, sh)
+        elif self.fp8:
+            B.raw_call("pkv_paged_attention_decode_fp8", out.data_ptr(), q.data_ptr(), kp, vp, bt, maxB, cl,
+                       len(p.lens), self.num_q_heads, Hkv, D, bs, NB, 0.0, float(self.kv_scales[0]),
+                       float(self.kv_scales[1]), P, ws, wsb, qdt, sh)
+        elif p.has_groups:
+            B.raw_call("pkv_paged_attention_decode_shared", out.data_ptr(), q.data_ptr(), kp, vp, bt, maxB, cl,
+                       len(p.lens), self.num_q_heads, Hkv, D, bs, NB, 0.0, P, rest[0], rest[1],
+                       len(p.group_shared), int(p.max_group_size), int(p.max_shared_len), ws, wsb, qdt, sh)
+        else:
+            B.raw_call("pkv_paged_attention_decode", out.data_ptr(), q.data_ptr(), kp, vp, bt, maxB, cl,
+                       len(p.lens), self.num_q_heads, Hkv, D, bs, NB, 0.0, P, ws, wsb, qdt, sh)
 
     def upload(self, p: StepPlan) -> DevicePlan:
         """Copy a plan to the device: its arrays packed into one pinned staging

@@ -141,3 +141,61 @@ def test_add_with_a_prefix_ending_inside_a_block_copies_that_block(prefix_tokens
     ref = oracle.paged_attention(q, kc, vc, bt, lens)
     assert m.device_error() == 0
     assert max_err(out, ref) <= TOL[out.dtype]
+
+
+@pytest.mark.parametrize("cfg,over", [
+    ("llama13b_prefix", dict(S=12, Hq=4, Hkv=4)),                              # shared-prefix groups
+    ("longctx_beam", dict(S=2, Hq=16, Hkv=2, len_fixed=2000)),                 # forks: copy-on-write pairs
+    ("spec_verify", dict(S=5, Hq=8, Hkv=2, len_uniform=(20, 700))),            # causal chunks
+    ("llama7b_fp8", dict(S=6, Hq=4, Hkv=4, len_uniform=(1, 600))),             # FP8 pools
+    ("llama3_gqa_bs32", dict(S=4, len_fixed=None, len_uniform=(1, 900))),      # grouped-query heads
+])
+def test_launch_step_planned_ahead_matches_oracle(cfg, over):
+    """DecodeSession.launch_step from pinned host buffers, the next step
+    planned while the device works (as bench.py's end-to-end leg does),
+    on every kind of plan: after each step the output equals the oracle's
+    attention and, at the end, both pools equal the oracle's copies and
+    appends.  Layouts repeat from step to step, so staging and device buffers
+    are reused."""
+    import bench
+    import paged_kv_cache_405_b200 as m
+    sh = synth.shrink(synth.CONFIGS[cfg], reserve_tokens=64, **over)
+    dev = torch.device("cuda")
+    wl = bench.Workload(sh, sh.seed, dev, 0)
+    ss = wl.session
+    kc, vc = ss.k_pool.cpu(), ss.v_pool.cpu()
+    dt = synth.DTYPES[sh.dtype]
+    g = torch.Generator().manual_seed(31)
+    out_host = None
+    p = wl.plan()
+    for step in range(4):
+        T = len(p.slot_mapping)
+        rows = T if sh.chunk else len(p.seq_ids)
+        q = synth.randn((rows, sh.Hq, sh.D), g, dt, "cpu").pin_memory()
+        kn = synth.randn((T, sh.Hkv, sh.D), g, dt, "cpu").pin_memory()
+        vn = synth.randn((T, sh.Hkv, sh.D), g, dt, "cpu").pin_memory()
+        out_host = ss.launch_step(p, q, kn, vn, out_host)
+        nxt = wl.plan()                          # planned while this step runs
+        torch.cuda.current_stream().synchronize()
+        oracle.block_copy(kc, vc, p.cow_pairs)
+        if sh.kv_fp8:
+            oracle.kv_append_fp8(kc.numpy(), vc.numpy(), kn, vn, sh.kv_scale, sh.kv_scale, p.slot_mapping)
+            ref = oracle.paged_attention_kv(q, kc.numpy(), vc.numpy(), sh.kv_scale, sh.kv_scale, p.block_tables,
+                                            p.lens, threads=oracle.max_threads())
+        else:
+            oracle.kv_append(kc, vc, kn, vn, p.slot_mapping)
+            if sh.chunk:
+                ref = oracle.paged_attention_chunk(q, kc, vc, p.block_tables, p.lens, p.query_start,
+                                                   threads=oracle.max_threads())
+            else:
+                ref = oracle.paged_attention(q, kc, vc, p.block_tables, p.lens, threads=oracle.max_threads())
+        assert m.device_error() == 0
+        assert max_err(out_host, ref) <= TOL[dt], step
+        if cfg == "llama13b_prefix":
+            assert p.has_groups
+        if cfg == "longctx_beam":
+            assert len(p.cow_pairs) == sh.S * (sh.beams - 1)
+        p = nxt
+    bits = (lambda t: t.view(torch.uint8)) if sh.kv_fp8 else (lambda t: t.view(torch.int16))
+    assert torch.equal(bits(ss.k_pool.cpu()), bits(kc)) and torch.equal(bits(ss.v_pool.cpu()), bits(vc))
+    assert len(ss._layouts) <= 2          # one layout per kind of step (the first may differ)
