@@ -344,6 +344,91 @@ pkv_status pkv_device_error(void* stream, uint32_t* code);
 /* Number of kernels this library has launched in this process. */
 uint64_t pkv_launch_count(void);
 
+/*
+ * pkv_step_from_host -- a whole step of the path in one call, for a serving
+ * loop that holds each step's inputs and wants its output in host memory.
+ * One decode step, as the pages describe it: the step's new K/V are written
+ * into the slots the allocator gave them ([E] 2.2, [T] 2.2.3), after the
+ * copy-on-write copies of shared blocks being written ([E] 6.2, [B] 2.2), and
+ * every query attends to its cache through its block table ([E] 4.2).  On
+ * `stream`, in this order:
+ *   1. the n_in copies in[i] (typically host -> device: q, the new K/V and the
+ *      plan arrays the allocator produced),
+ *   2. pkv_block_copy of num_pairs pairs (skipped when num_pairs = 0),
+ *   3. pkv_kv_append (PKV_STEP_DECODE_FP8: pkv_kv_append_fp8) of num_tokens
+ *      new tokens (skipped when num_tokens = 0),
+ *   4. the attention call of `kind` (skipped when num_seqs = 0),
+ *   5. the n_out copies out[i] (typically device -> host: the output).
+ * Each copy is one cudaMemcpyAsync (cudaMemcpyDefault: the direction follows
+ * from the pointers); from pinned host memory it does not wait for the
+ * stream.  The device pointers in the struct (pools, pairs, k_new, v_new,
+ * slot_mapping, out, q, tables, lengths, groups, query_start, workspace) are
+ * the arguments of the separate calls above, with their meaning, layout and
+ * checks, and may be the destinations of the copies of step 1.  Sizes are
+ * trusted as everywhere else.  Ownership: every buffer is the caller's.
+ * Errors: each call checks its own arguments before it launches; the first
+ * non-OK status is returned and nothing after it is issued, but what was
+ * issued before it (copies, calls) stays issued, so a refused step leaves the
+ * pools in an intermediate state -- check a step's arguments once, then reuse
+ * them.  struct_size must be sizeof(pkv_step) (PKV_ERR_INVALID otherwise),
+ * so a caller built against another version of this header is refused.
+ */
+typedef struct {
+    void* dst;
+    const void* src;
+    size_t bytes;
+} pkv_copy;
+
+typedef enum {
+    PKV_STEP_DECODE = 0,         /* pkv_paged_attention_decode */
+    PKV_STEP_DECODE_SHARED = 1,  /* pkv_paged_attention_decode_shared */
+    PKV_STEP_DECODE_FP8 = 2,     /* pkv_kv_append_fp8 + pkv_paged_attention_decode_fp8 */
+    PKV_STEP_CHUNK = 3           /* pkv_paged_attention_chunk (rows = num_tokens) */
+} pkv_step_kind;
+
+typedef struct {
+    size_t struct_size;          /* sizeof(pkv_step) */
+    int kind;                    /* pkv_step_kind */
+    const pkv_copy* in;          /* [n_in], made first */
+    int n_in;
+    const pkv_copy* out;         /* [n_out], made last */
+    int n_out;
+    /* pools: [num_blocks][num_kv_heads][block_size][head_dim] */
+    void* k_pool;
+    void* v_pool;
+    int num_blocks, num_kv_heads, head_dim, block_size;
+    int dtype;                   /* pkv_dtype of q, out and the new K/V (the pools' type unless FP8) */
+    float k_scale, v_scale;      /* FP8 pools only */
+    /* copy-on-write pairs, int32 [num_pairs][2] */
+    const int32_t* pairs;
+    int num_pairs;
+    /* new tokens: [num_tokens][num_kv_heads][head_dim], int64 slots */
+    const void* k_new;
+    const void* v_new;
+    const int64_t* slot_mapping;
+    int num_tokens;
+    /* attention */
+    void* attn_out;
+    const void* q;
+    const int32_t* block_tables;
+    int max_blocks_per_seq;
+    const int32_t* context_lens;
+    int num_seqs, num_q_heads;
+    float scale;
+    int partition_size;
+    void* workspace;
+    size_t workspace_bytes;
+    /* PKV_STEP_DECODE_SHARED */
+    const int32_t* group_first;
+    const int32_t* group_shared;
+    int num_groups, max_group_size, max_shared_len;
+    /* PKV_STEP_CHUNK */
+    const int32_t* query_start;
+    int max_query_len;
+} pkv_step;
+
+pkv_status pkv_step_from_host(const pkv_step* step, void* stream);
+
 /* --------------------------------------------------------- host allocator */
 
 /*

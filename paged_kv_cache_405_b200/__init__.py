@@ -9,5 +9,5 @@ from .binding import (BlockAllocator, PagedKVError, attention_partition_size,  #
                       attention_chunk_workspace_bytes, attention_shared_workspace_bytes, attention_workspace_bytes, block_copy, device_error,
                       find_shared_prefix_groups, kv_append, kv_append_fp8, launch_count, paged_attention_chunk, paged_attention_decode,
                       paged_attention_decode_fp8, paged_attention_decode_shared, paged_attention_decode_static,
-                      set_nvtx, workspace_for)
+                      PkvCopy, PkvStep, raw_call, set_nvtx, step_from_host, workspace_for)
 from .session import ChunkPlan, DecodeSession, DevicePlan, StepPlan  # noqa: F401,E402

@@ -35,8 +35,39 @@ EXPORTS = [
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_add", "pkv_seq_share_prefix", "pkv_seq_fork",
     "pkv_alloc_set_prefix_caching", "pkv_seq_add_with_prompt", "pkv_seq_append_tokens", "pkv_prefix_cache_stats",
     "pkv_seq_append_slots", "pkv_seq_append_slots_batch", "pkv_seq_block_tables_batch", "pkv_seq_free", "pkv_seq_block_table", "pkv_alloc_stats",
-    "pkv_block_refcount", "pkv_status_str", "pkv_last_error",
+    "pkv_block_refcount", "pkv_status_str", "pkv_last_error", "pkv_step_from_host",
 ]
+
+# pkv_step_kind
+STEP_DECODE, STEP_DECODE_SHARED, STEP_DECODE_FP8, STEP_CHUNK = range(4)
+
+
+class PkvCopy(ctypes.Structure):
+    """pkv_copy: one asynchronous copy of pkv_step_from_host."""
+    _fields_ = [("dst", ctypes.c_void_p), ("src", ctypes.c_void_p), ("bytes", ctypes.c_size_t)]
+
+
+class PkvStep(ctypes.Structure):
+    """pkv_step, field for field (``in_`` is the header's ``in``)."""
+    _fields_ = [
+        ("struct_size", ctypes.c_size_t), ("kind", ctypes.c_int),
+        ("in_", ctypes.POINTER(PkvCopy)), ("n_in", ctypes.c_int),
+        ("out", ctypes.POINTER(PkvCopy)), ("n_out", ctypes.c_int),
+        ("k_pool", ctypes.c_void_p), ("v_pool", ctypes.c_void_p),
+        ("num_blocks", ctypes.c_int), ("num_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int),
+        ("block_size", ctypes.c_int), ("dtype", ctypes.c_int), ("k_scale", ctypes.c_float),
+        ("v_scale", ctypes.c_float),
+        ("pairs", ctypes.c_void_p), ("num_pairs", ctypes.c_int),
+        ("k_new", ctypes.c_void_p), ("v_new", ctypes.c_void_p), ("slot_mapping", ctypes.c_void_p),
+        ("num_tokens", ctypes.c_int),
+        ("attn_out", ctypes.c_void_p), ("q", ctypes.c_void_p), ("block_tables", ctypes.c_void_p),
+        ("max_blocks_per_seq", ctypes.c_int), ("context_lens", ctypes.c_void_p),
+        ("num_seqs", ctypes.c_int), ("num_q_heads", ctypes.c_int), ("scale", ctypes.c_float),
+        ("partition_size", ctypes.c_int), ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+        ("group_first", ctypes.c_void_p), ("group_shared", ctypes.c_void_p), ("num_groups", ctypes.c_int),
+        ("max_group_size", ctypes.c_int), ("max_shared_len", ctypes.c_int),
+        ("query_start", ctypes.c_void_p), ("max_query_len", ctypes.c_int),
+    ]
 
 
 class PagedKVError(RuntimeError):
@@ -99,6 +130,7 @@ def _load():
                                     ctypes.POINTER(c_i64), ctypes.POINTER(c_i64)]),
         "pkv_block_refcount": (c_int, [c_vp, c_int]),
         "pkv_status_str": (ctypes.c_char_p, [c_int]),
+        "pkv_step_from_host": (c_int, [ctypes.POINTER(PkvStep), c_vp]),
         "pkv_last_error": (ctypes.c_char_p, []),
     }
     for name, (res, args) in sig.items():
@@ -454,6 +486,12 @@ def block_copy(k_pool, v_pool, pairs, stream=None) -> None:
     dt = FP8_E4M3 if k_pool.dtype == torch.uint8 else _dt(k_pool)
     _check(lib.pkv_block_copy(_dev(k_pool, "k_pool"), _dev(v_pool, "v_pool"),
                               _dev(pairs, "pairs") if n else None, n, NB, Hkv, D, bs, dt, _stream(stream)))
+
+
+def step_from_host(step: PkvStep, stream=None) -> None:
+    """One whole step in one C call (see pkv_step_from_host): ``step`` is a
+    filled-in ``PkvStep``; DecodeSession.launch_step builds and fills one."""
+    raw_call("pkv_step_from_host", ctypes.byref(step), _stream(stream))
 
 
 def device_error(stream=None) -> int:

@@ -270,24 +270,45 @@ __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_fp8_kernel(const Att
 //    above); B column 0 = q, held by the lanes with gid = 0, other columns 0.
 //    The score of token gid (gid + 8) lands in the lane (gid, tig = 0).
 //  * O^T += V^T p^T.  A = V^T: m-tile mt, row r is head-dim element
-//    gid*D/8 + 2mt (r = gid) or gid*D/8 + 2mt + 1 (r = gid + 8), contraction
-//    over the tokens in S-column order (2tig, 2tig+1, 8+2tig, 9+2tig); the
-//    lane reads D/8 consecutive codes of each of its four tokens, as in the
-//    grouped kernel.  B column 0 = p, gathered into the gid = 0 lanes with
-//    four shuffles.  The lane (gid, tig = 0) ends with output elements
-//    gid*D/8 .. gid*D/8 + D/8 - 1.
-// Half the MMAs of the grouped layout (8 + 8 per tile at D = 128) and a
+//    gid*D/8 + 2mt (r = gid) or gid*D/8 + 2mt + 1 (r = gid + 8); B column 0 =
+//    p, held by the gid = 0 lanes.  A dot product may take its terms in any
+//    order, so the contraction pairs up tokens j and j + 8, whose scores both
+//    sit in lane (j, 0): that lane packs their two probabilities once, and
+//    lane (0, tig) gathers the packs of lanes (2tig, 0) and (2tig+1, 0) with
+//    two shuffles as its contraction indices (2tig, 2tig+1) and (2tig+8,
+//    2tig+9).  The A operand follows: lane tig reads D/8 consecutive codes of
+//    tokens 2tig, 2tig+8, 2tig+1, 2tig+9 and pairs the codes of two tokens
+//    with one byte permute per four columns.  The lane (gid, tig = 0) ends
+//    with output elements gid*D/8 .. gid*D/8 + D/8 - 1.
+// Half the MMAs of the grouped layout (8 + 8 per 16 tokens at D = 128) and a
 // quarter of the CUDA-core instructions of widening every code to fp32.
-template <int D, int WARPS, int STAGES, typename To>
-__global__ void __launch_bounds__(WARPS * 32, 4) paged_attn_fp8_head_kernel(const AttnParams p,
-                                                                            const __grid_constant__ CUtensorMap tmK,
-                                                                            const __grid_constant__ CUtensorMap tmV) {
-    using C = Fp8Cfg<D, WARPS, STAGES>;
+//
+// TT tokens per pipeline stage (16 or 32): a 32-token stage is two 16-token
+// tiles (each found through the block table on its own, so any block_size
+// works) under one barrier, one softmax step and one loop iteration, which
+// halves the fixed cost per token of everything but the widening and the
+// MMAs.
+template <int D, int TT>
+struct Fp8HeadCfg {
+    static constexpr int kHalves = TT / kTileTok;
+    static constexpr int kTileBytes = kTileTok * D;           // one 16-token K (or V) tile of codes
+    static constexpr int kStageBytes = 2 * kHalves * kTileBytes;  // K tiles, then V tiles
+    static_assert(TT == 16 || TT == 32, "16 or 32 tokens per stage");
+};
+
+template <int D, int WARPS, int STAGES, typename To, int TT = kTileTok, int MINB = 4>
+__global__ void __launch_bounds__(WARPS * 32, MINB) paged_attn_fp8_head_kernel(const AttnParams p,
+                                                                               const __grid_constant__ CUtensorMap tmK,
+                                                                               const __grid_constant__ CUtensorMap tmV) {
+    using C = Fp8HeadCfg<D, TT>;
     using H = MmaAcc<__half, D>;
+    constexpr int HV = C::kHalves;
     constexpr int KSTEPS = D / 16;  // S^T k-steps; also 32-bit words of K codes per lane and row
     constexpr int NMT = D / 16;     // O^T m-tiles
     constexpr int VW = D / 32;      // 32-bit words of V codes per lane and token (D/8 codes)
     constexpr int SPAN = D / 8;     // output elements per lane with tig = 0
+    constexpr int kWarpBytes = STAGES * C::kStageBytes;
+    constexpr int kDataBytes = WARPS * kWarpBytes;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -307,7 +328,7 @@ __global__ void __launch_bounds__(WARPS * 32, 4) paged_attn_fp8_head_kernel(cons
         return;
     }
     uint32_t bar0;
-    uint8_t* ring = ring_setup<C::kWarpBytes, C::kDataBytes, STAGES>(smem_raw, warp, lane, bar0, &tmK, &tmV);
+    uint8_t* ring = ring_setup<kWarpBytes, kDataBytes, STAGES>(smem_raw, warp, lane, bar0, &tmK, &tmV);
     const uint32_t ring_s = smem_u32(ring);
 
     // q as column 0 of the B operand of S^T (lanes gid = 0).
@@ -326,119 +347,155 @@ __global__ void __launch_bounds__(WARPS * 32, 4) paged_attn_fp8_head_kernel(cons
     float m = -INFINITY, l = 0.f;  // m warp-uniform; l a per-lane share
 
     const int t_begin = u.t_begin, t_end = u.t_end;
-    const int ntiles = (t_end - t_begin + kTileTok - 1) / kTileTok;
+    const int ntiles = (t_end - t_begin + TT - 1) / TT;
     const int jb0 = t_begin / p.bs;
     BlockWindow win;
     win.init(p.block_tables + (int64_t)s * p.maxB, jb0, (t_end - 1) / p.bs - jb0 + 1, lane);
 
     auto issue = [&](int i) {
-        const int t0 = t_begin + i * kTileTok;
-        const int blk = win.get(t0 / p.bs - jb0, lane, p.NB);
+        const int t0 = t_begin + i * TT;
+        int rows[HV];
+        int nh = 0;  // 16-token tiles of the stage that hold tokens of the unit
+#pragma unroll
+        for (int hh = 0; hh < HV; ++hh) {
+            const int th = t0 + hh * kTileTok;
+            if (th < t_end) {  // warp-uniform
+                const int blk = win.get(th / p.bs - jb0, lane, p.NB);
+                rows[hh] = (blk * p.Hkv + g) * p.bs + (th % p.bs);
+                nh = hh + 1;
+            }
+        }
         if (lane == 0) {
-            const int row = (blk * p.Hkv + g) * p.bs + (t0 % p.bs);
             const int st = i % STAGES;
             const uint32_t bar = bar0 + 8 * st;
             const uint32_t dst = ring_s + st * C::kStageBytes;
             fence_proxy_async();
-            mbar_arrive_expect_tx(bar, C::kStageBytes);
-            tma_load_2d(dst, &tmK, 0, row, bar);
-            tma_load_2d(dst + C::kTileBytes, &tmV, 0, row, bar);
+            mbar_arrive_expect_tx(bar, 2 * nh * C::kTileBytes);
+#pragma unroll
+            for (int hh = 0; hh < HV; ++hh) {
+                if (hh < nh) {
+                    tma_load_2d(dst + hh * C::kTileBytes, &tmK, 0, rows[hh], bar);
+                    tma_load_2d(dst + (HV + hh) * C::kTileBytes, &tmV, 0, rows[hh], bar);
+                }
+            }
         }
     };
     const int npre = ntiles < STAGES ? ntiles : STAGES;
     for (int i = 0; i < npre; ++i) issue(i);
 
-    const int vtok[4] = {2 * tig, 2 * tig + 1, 8 + 2 * tig, 9 + 2 * tig};
+    // This lane's tokens for the P V contraction (see above).
+    const int vtok[4] = {2 * tig, 2 * tig + 8, 2 * tig + 1, 2 * tig + 9};
 
     for (int i = 0; i < ntiles; ++i) {
         const int st = i % STAGES;
         if (!ring_wait<STAGES>(bar0, i, ntiles)) return;
-        const int valid = min(kTileTok, t_end - (t_begin + i * kTileTok));
-        const uint8_t* kt = ring + st * C::kStageBytes;
-        const uint8_t* vt = kt + C::kTileBytes;
+        const int valid = min(TT, t_end - (t_begin + i * TT));
+        const uint8_t* stage = ring + st * C::kStageBytes;
 
-        uint32_t kw[2][KSTEPS];  // codes of rows gid and gid + 8
+        // Codes of this lane's fragments, then the stage goes back to TMA.
+        uint32_t kw[HV][2][KSTEPS];  // codes of rows gid and gid + 8 of each tile
+        uint32_t vw[HV][4][VW];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
+        for (int hh = 0; hh < HV; ++hh) {
+            const int vh = valid - hh * kTileTok;  // tokens of this tile (warp-uniform)
+            if (vh <= 0) continue;
+            const uint8_t* kt = stage + hh * C::kTileBytes;
+            const uint8_t* vt = stage + (HV + hh) * C::kTileBytes;
 #pragma unroll
-            for (int c = 0; c < KSTEPS / 4; ++c) {
-                const uint4 w = *reinterpret_cast<const uint4*>(kt + fp8_chunk<D>(hh * 8 + gid, tig * (KSTEPS / 4) + c));
-                kw[hh][4 * c] = w.x;
-                kw[hh][4 * c + 1] = w.y;
-                kw[hh][4 * c + 2] = w.z;
-                kw[hh][4 * c + 3] = w.w;
+            for (int r = 0; r < 2; ++r) {
+#pragma unroll
+                for (int c = 0; c < KSTEPS / 4; ++c) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(kt + fp8_chunk<D>(r * 8 + gid, tig * (KSTEPS / 4) + c));
+                    kw[hh][r][4 * c] = w.x;
+                    kw[hh][r][4 * c + 1] = w.y;
+                    kw[hh][r][4 * c + 2] = w.z;
+                    kw[hh][r][4 * c + 3] = w.w;
+                }
             }
-        }
-        zero_tail_rows<D>(const_cast<uint8_t*>(vt), valid, lane);
-        uint32_t vw[4][VW];
+            zero_tail_rows<D>(const_cast<uint8_t*>(vt), vh, lane);
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            if constexpr (VW == 4) {
-                const uint4 w = *reinterpret_cast<const uint4*>(vt + fp8_chunk<D>(vtok[t], gid));
-                vw[t][0] = w.x;
-                vw[t][1] = w.y;
-                vw[t][2] = w.z;
-                vw[t][3] = w.w;
-            } else {
-                const uint2 w = *reinterpret_cast<const uint2*>(vt + vtok[t] * D + gid * 8);
-                vw[t][0] = w.x;
-                vw[t][1] = w.y;
+            for (int t = 0; t < 4; ++t) {
+                if constexpr (VW == 4) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(vt + fp8_chunk<D>(vtok[t], gid));
+                    vw[hh][t][0] = w.x;
+                    vw[hh][t][1] = w.y;
+                    vw[hh][t][2] = w.z;
+                    vw[hh][t][3] = w.w;
+                } else {
+                    const uint2 w = *reinterpret_cast<const uint2*>(vt + vtok[t] * D + gid * 8);
+                    vw[hh][t][0] = w.x;
+                    vw[hh][t][1] = w.y;
+                }
             }
         }
         __syncwarp();
         if (i + STAGES < ntiles) issue(i + STAGES);
 
-        // S^T: two accumulator chains (even / odd k-steps) halve the MMA
-        // dependency depth.
-        float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int kk = 0; kk < KSTEPS; ++kk) {
-            const uint32_t a[4] = {e4m3x2_to_f16x2((uint16_t)(kw[0][kk] & 0xffffu)),
-                                   e4m3x2_to_f16x2((uint16_t)(kw[1][kk] & 0xffffu)),
-                                   e4m3x2_to_f16x2((uint16_t)(kw[0][kk] >> 16)),
-                                   e4m3x2_to_f16x2((uint16_t)(kw[1][kk] >> 16))};
-            mma_16816<__half>(sa[kk & 1], a, qb[kk][0], qb[kk][1]);
-        }
+        // S^T of each tile: two accumulator chains (even / odd k-steps) halve
+        // the MMA dependency depth.
+        float x[HV][2];  // scores of tokens gid and gid + 8 of each tile (lanes tig = 0)
         const bool live = tig == 0;
-        const float x_lo = live && gid < valid ? (sa[0][0] + sa[1][0]) * p.scale_log2 : -INFINITY;
-        const float x_hi = live && gid + 8 < valid ? (sa[0][2] + sa[1][2]) * p.scale_log2 : -INFINITY;
-        float mt = fmaxf(x_lo, x_hi);
+#pragma unroll
+        for (int hh = 0; hh < HV; ++hh) {
+            const int vh = valid - hh * kTileTok;
+            x[hh][0] = x[hh][1] = -INFINITY;
+            if (vh <= 0) continue;
+            float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+            for (int kk = 0; kk < KSTEPS; ++kk) {
+                const uint32_t a[4] = {e4m3x2_to_f16x2((uint16_t)(kw[hh][0][kk] & 0xffffu)),
+                                       e4m3x2_to_f16x2((uint16_t)(kw[hh][1][kk] & 0xffffu)),
+                                       e4m3x2_to_f16x2((uint16_t)(kw[hh][0][kk] >> 16)),
+                                       e4m3x2_to_f16x2((uint16_t)(kw[hh][1][kk] >> 16))};
+                mma_16816<__half>(sa[kk & 1], a, qb[kk][0], qb[kk][1]);
+            }
+            if (live && gid < vh) x[hh][0] = (sa[0][0] + sa[1][0]) * p.scale_log2;
+            if (live && gid + 8 < vh) x[hh][1] = (sa[0][2] + sa[1][2]) * p.scale_log2;
+        }
+        float mt = fmaxf(x[0][0], x[0][1]);
+#pragma unroll
+        for (int hh = 1; hh < HV; ++hh) mt = fmaxf(mt, fmaxf(x[hh][0], x[hh][1]));
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, off));
         const float mn = fmaxf(m, mt);
         const float b = mn == -INFINITY ? 0.f : mn;  // no -inf - -inf
         const float alpha = ex2(m - b);
-        const float p_lo = ex2(x_lo - b), p_hi = ex2(x_hi - b);
-        l = l * alpha + p_lo + p_hi;
         m = mn;
         if (alpha != 1.f) {  // warp-uniform; exactly 1 once the maximum settles
+            l *= alpha;
 #pragma unroll
             for (int j = 0; j < NMT; ++j) {
                 o[j][0] *= alpha;
                 o[j][2] *= alpha;
             }
         }
-        // p^T column 0: tokens 2tig, 2tig+1 (b0) and 8+2tig, 9+2tig (b1).
-        const float p0 = __shfl_sync(0xffffffffu, p_lo, 8 * tig);
-        const float p1 = __shfl_sync(0xffffffffu, p_lo, 8 * tig + 4);
-        const float p2 = __shfl_sync(0xffffffffu, p_hi, 8 * tig);
-        const float p3 = __shfl_sync(0xffffffffu, p_hi, 8 * tig + 4);
-        const uint32_t pb0 = gid == 0 ? Elt<__half>::pack2(p0, p1) : 0u;
-        const uint32_t pb1 = gid == 0 ? Elt<__half>::pack2(p2, p3) : 0u;
-
-        // O^T += V^T p^T
 #pragma unroll
-        for (int w = 0; w < VW; ++w) {
-            const uint32_t lo0 = __byte_perm(vw[0][w], vw[1][w], 0x5140);
-            const uint32_t hi0 = __byte_perm(vw[0][w], vw[1][w], 0x7362);
-            const uint32_t lo1 = __byte_perm(vw[2][w], vw[3][w], 0x5140);
-            const uint32_t hi1 = __byte_perm(vw[2][w], vw[3][w], 0x7362);
-            const uint32_t a0[4] = {e4m3x2_to_f16x2((uint16_t)(lo0 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(lo0 >> 16)),
-                                    e4m3x2_to_f16x2((uint16_t)(lo1 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(lo1 >> 16))};
-            mma_16816<__half>(o[2 * w], a0, pb0, pb1);
-            const uint32_t a1[4] = {e4m3x2_to_f16x2((uint16_t)(hi0 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(hi0 >> 16)),
-                                    e4m3x2_to_f16x2((uint16_t)(hi1 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(hi1 >> 16))};
-            mma_16816<__half>(o[2 * w + 1], a1, pb0, pb1);
+        for (int hh = 0; hh < HV; ++hh) {
+            if (valid - hh * kTileTok <= 0) continue;  // warp-uniform
+            const float p_lo = ex2(x[hh][0] - b), p_hi = ex2(x[hh][1] - b);
+            l += p_lo + p_hi;
+            // Lane (j, 0) holds the pair (token j, token j + 8) = contraction
+            // indices (2j, 2j+1); lane (0, tig) gathers pairs 2tig and 2tig+1.
+            const uint32_t pair = Elt<__half>::pack2(p_lo, p_hi);
+            const uint32_t g0 = __shfl_sync(0xffffffffu, pair, 8 * tig);
+            const uint32_t g1 = __shfl_sync(0xffffffffu, pair, 8 * tig + 4);
+            const uint32_t pb0 = gid == 0 ? g0 : 0u;
+            const uint32_t pb1 = gid == 0 ? g1 : 0u;
+
+            // O^T += V^T p^T
+#pragma unroll
+            for (int w = 0; w < VW; ++w) {
+                const uint32_t lo0 = __byte_perm(vw[hh][0][w], vw[hh][1][w], 0x5140);
+                const uint32_t hi0 = __byte_perm(vw[hh][0][w], vw[hh][1][w], 0x7362);
+                const uint32_t lo1 = __byte_perm(vw[hh][2][w], vw[hh][3][w], 0x5140);
+                const uint32_t hi1 = __byte_perm(vw[hh][2][w], vw[hh][3][w], 0x7362);
+                const uint32_t a0[4] = {e4m3x2_to_f16x2((uint16_t)(lo0 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(lo0 >> 16)),
+                                        e4m3x2_to_f16x2((uint16_t)(lo1 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(lo1 >> 16))};
+                mma_16816<__half>(o[2 * w], a0, pb0, pb1);
+                const uint32_t a1[4] = {e4m3x2_to_f16x2((uint16_t)(hi0 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(hi0 >> 16)),
+                                        e4m3x2_to_f16x2((uint16_t)(hi1 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(hi1 >> 16))};
+                mma_16816<__half>(o[2 * w + 1], a1, pb0, pb1);
+            }
         }
     }
 #pragma unroll

@@ -275,14 +275,25 @@ static cudaError_t launch_mma_fp8(const pkv::AttnParams& p, dim3 grid, const CUt
                    : launch_mma_fp8_rows<To, D, false>(p, grid, mk, mv, st);
 }
 
+// Per-head FP8 kernel: tokens per pipeline stage (16 or 32) and CTAs per SM
+// it is compiled for; build-time tunables.
+#ifndef PKV_FP8_HEAD_TT
+#define PKV_FP8_HEAD_TT 16
+#endif
+#ifndef PKV_FP8_HEAD_MINB
+#define PKV_FP8_HEAD_MINB 4
+#endif
+
 template <typename To, int D>
 static cudaError_t launch_head_fp8(const pkv::AttnParams& p, dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv,
                                    cudaStream_t st) {
-    using C = pkv::Fp8Cfg<D, kMmaWarps, kFp8Stages>;
-    auto k = pkv::paged_attn_fp8_head_kernel<D, kMmaWarps, kFp8Stages, To>;
-    static cudaError_t attr = set_smem(k, C::kSmemBytes);
+    constexpr int TT = PKV_FP8_HEAD_TT;
+    using C = pkv::Fp8HeadCfg<D, TT>;
+    constexpr int kSmem = 1024 + kMmaWarps * kFp8Stages * (C::kStageBytes + 8);
+    auto k = pkv::paged_attn_fp8_head_kernel<D, kMmaWarps, kFp8Stages, To, TT, PKV_FP8_HEAD_MINB>;
+    static cudaError_t attr = set_smem(k, kSmem);
     if (attr != cudaSuccess) return attr;
-    return launch_k(k, grid, dim3(kMmaWarps * 32), C::kSmemBytes, st, p, mk, mv);
+    return launch_k(k, grid, dim3(kMmaWarps * 32), kSmem, st, p, mk, mv);
 }
 
 // Side stream for the shared-prefix pass, which runs concurrently with the
@@ -952,4 +963,89 @@ extern "C" pkv_status pkv_paged_attention_decode_static(void* out, const void* q
     return decode_impl(out, q, k_pool, v_pool, block_tables, max_blocks_per_seq, context_lens, num_seqs, num_q_heads,
                        num_kv_heads, head_dim, block_size, num_blocks, scale, partition_size, GroupArgs(), nullptr, 0,
                        dtype, stream, KvArgs(), true);
+}
+
+// ---------------------------------------------------------------------------
+// A whole step from host buffers in one call: copies in, block_copy,
+// kv_append, attention, copies out -- each part the same code as its own
+// entry point, on one stream.
+// ---------------------------------------------------------------------------
+namespace pkv_host {
+
+static pkv_status copies(const pkv_copy* c, int n, cudaStream_t st, const char* what) {
+    for (int i = 0; i < n; ++i) {
+        if (c[i].bytes == 0) continue;
+        if (!c[i].dst || !c[i].src) {
+            g_msg = std::string("pkv_step_from_host: null pointer in the ") + what + " copies";
+            return PKV_ERR_INVALID;
+        }
+        const cudaError_t e = cudaMemcpyAsync(c[i].dst, c[i].src, c[i].bytes, cudaMemcpyDefault, st);
+        if (e != cudaSuccess) return cuda_fail("pkv_step_from_host: copy", e);
+    }
+    return PKV_OK;
+}
+
+}  // namespace pkv_host
+
+extern "C" pkv_status pkv_step_from_host(const pkv_step* s, void* stream) {
+    using namespace pkv_host;
+    if (!s) return invalid("pkv_step_from_host: null step");
+    if (s->struct_size != sizeof(pkv_step))
+        return invalid("pkv_step_from_host: struct_size is not sizeof(pkv_step) (header version mismatch)");
+    if (s->kind < PKV_STEP_DECODE || s->kind > PKV_STEP_CHUNK) return invalid("pkv_step_from_host: bad kind");
+    if (s->n_in < 0 || s->n_out < 0 || (s->n_in > 0 && !s->in) || (s->n_out > 0 && !s->out))
+        return invalid("pkv_step_from_host: bad copy lists");
+    if (s->num_pairs < 0 || s->num_tokens < 0 || s->num_seqs < 0)
+        return invalid("pkv_step_from_host: counts must be >= 0");
+    cudaStream_t st = (cudaStream_t)stream;
+    const pkv_dtype dt = (pkv_dtype)s->dtype;
+    const bool fp8 = s->kind == PKV_STEP_DECODE_FP8;
+    pkv_status r = copies(s->in, s->n_in, st, "input");
+    if (r != PKV_OK) return r;
+    if (s->num_pairs > 0) {
+        r = pkv_block_copy(s->k_pool, s->v_pool, s->pairs, s->num_pairs, s->num_blocks, s->num_kv_heads,
+                           s->head_dim, s->block_size, fp8 ? PKV_FP8_E4M3 : dt, stream);
+        if (r != PKV_OK) return r;
+    }
+    if (s->num_tokens > 0) {
+        r = fp8 ? pkv_kv_append_fp8(s->k_new, s->v_new, s->k_pool, s->v_pool, s->slot_mapping, s->num_tokens,
+                                    s->num_blocks, s->num_kv_heads, s->head_dim, s->block_size, dt, s->k_scale,
+                                    s->v_scale, stream)
+                : pkv_kv_append(s->k_new, s->v_new, s->k_pool, s->v_pool, s->slot_mapping, s->num_tokens,
+                                s->num_blocks, s->num_kv_heads, s->head_dim, s->block_size, dt, stream);
+        if (r != PKV_OK) return r;
+    }
+    if (s->num_seqs > 0) {
+        switch (s->kind) {
+            case PKV_STEP_DECODE:
+                r = pkv_paged_attention_decode(s->attn_out, s->q, s->k_pool, s->v_pool, s->block_tables,
+                                               s->max_blocks_per_seq, s->context_lens, s->num_seqs, s->num_q_heads,
+                                               s->num_kv_heads, s->head_dim, s->block_size, s->num_blocks, s->scale,
+                                               s->partition_size, s->workspace, s->workspace_bytes, dt, stream);
+                break;
+            case PKV_STEP_DECODE_SHARED:
+                r = pkv_paged_attention_decode_shared(
+                    s->attn_out, s->q, s->k_pool, s->v_pool, s->block_tables, s->max_blocks_per_seq, s->context_lens,
+                    s->num_seqs, s->num_q_heads, s->num_kv_heads, s->head_dim, s->block_size, s->num_blocks,
+                    s->scale, s->partition_size, s->group_first, s->group_shared, s->num_groups, s->max_group_size,
+                    s->max_shared_len, s->workspace, s->workspace_bytes, dt, stream);
+                break;
+            case PKV_STEP_DECODE_FP8:
+                r = pkv_paged_attention_decode_fp8(s->attn_out, s->q, s->k_pool, s->v_pool, s->block_tables,
+                                                   s->max_blocks_per_seq, s->context_lens, s->num_seqs,
+                                                   s->num_q_heads, s->num_kv_heads, s->head_dim, s->block_size,
+                                                   s->num_blocks, s->scale, s->k_scale, s->v_scale,
+                                                   s->partition_size, s->workspace, s->workspace_bytes, dt, stream);
+                break;
+            default:
+                r = pkv_paged_attention_chunk(s->attn_out, s->q, s->k_pool, s->v_pool, s->block_tables,
+                                              s->max_blocks_per_seq, s->context_lens, s->query_start, s->num_seqs,
+                                              s->num_tokens, s->max_query_len, s->num_q_heads, s->num_kv_heads,
+                                              s->head_dim, s->block_size, s->num_blocks, s->scale, s->partition_size,
+                                              s->workspace, s->workspace_bytes, dt, stream);
+                break;
+        }
+        if (r != PKV_OK) return r;
+    }
+    return copies(s->out, s->n_out, st, "output");
 }

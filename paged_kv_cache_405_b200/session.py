@@ -17,6 +17,7 @@ serving loop makes every step (inputs in, attention output out).
 """
 from __future__ import annotations
 
+import ctypes
 from dataclasses import dataclass
 from typing import Optional, Sequence
 
@@ -290,24 +291,25 @@ class DecodeSession:
     # ------------------------------------------------- host-buffer steps
     # A serving loop hands each step's inputs over in host memory and wants
     # the output back in host memory.  launch_step does that for a planned
-    # step with as little host work as it can: the plan's arrays are packed
-    # into a pinned staging buffer and sent with one copy into a device buffer
-    # made for that layout of arrays; q / new K / new V go into device buffers
-    # kept per shape; the three C calls are made directly with pointers that
-    # were checked against the sizes when those buffers were made; the output
-    # comes back with one copy.  Nothing is allocated once a layout has been
-    # seen, so the host cost is a few copies and three C calls.
+    # step with one C call (pkv_step_from_host): the plan's arrays, packed into
+    # a pinned staging buffer, and q / new K / new V go to device buffers in
+    # four copies, then block_copy -> kv_append -> attention run and the output
+    # comes back in one copy.  The device buffers are made once per layout of
+    # the plan's arrays (and per input shape) and the step description is
+    # built and checked against their sizes then; a step only refills the
+    # staging buffer, sets the host pointers and makes the call.
     #
     # Reuse rules: the device buffers of a layout are reused by later steps of
     # the same layout, so all host-buffer steps of a session go on one stream
     # (stream order then keeps a step's kernels ahead of the next step's
     # copies into the same buffers).  Two staging buffers alternate per
-    # layout, and one is refilled only after its previous copy has completed.
+    # layout, and one is refilled only after the step that last used it has
+    # completed.
 
     _MAX_LAYOUTS = 32
 
-    def _staged(self, arrays, stream) -> list:
-        """Device views of ``arrays`` (host numpy), sent with one copy on ``stream``."""
+    def _layout(self, arrays) -> dict:
+        """The next staging set for this layout of plan arrays (made once)."""
         key = tuple((a.dtype.str, a.shape) for a in arrays)
         lay = self._layouts.get(key)
         if lay is None:
@@ -323,23 +325,13 @@ class DecodeSession:
                 host = torch.empty(total, dtype=torch.uint8, pin_memory=True)
                 dev = torch.empty(total, dtype=torch.uint8, device=self.device)
                 hv = host.numpy()
-                hviews = [hv[o:o + a.nbytes].view(a.dtype).reshape(a.shape) for a, o in zip(arrays, offs)]
-                dviews = [dev[o:o + a.nbytes].view(torch.from_numpy(a[:0].reshape(-1)).dtype).view(a.shape)
-                          for a, o in zip(arrays, offs)]
-                sets.append({"host": host, "dev": dev, "hviews": hviews, "dviews": dviews,
-                             "ptrs": [t.data_ptr() for t in dviews], "event": None})
+                sets.append({"host": host, "dev": dev, "bytes": total,
+                             "hviews": [hv[o:o + a.nbytes].view(a.dtype).reshape(a.shape)
+                                        for a, o in zip(arrays, offs)],
+                             "ptrs": [dev.data_ptr() + o for o in offs], "event": None, "steps": {}})
             lay = self._layouts[key] = [0, sets]
         lay[0] ^= 1
-        st = lay[1][lay[0]]
-        if st["event"] is not None:
-            st["event"].synchronize()           # the previous copy out of this staging buffer is done
-        for hv, a in zip(st["hviews"], arrays):
-            np.copyto(hv, a, casting="no")
-        st["dev"].copy_(st["host"], non_blocking=True)
-        if st["event"] is None:
-            st["event"] = torch.cuda.Event()
-        st["event"].record(stream)
-        return st
+        return lay[1][lay[0]]
 
     def _io_buffers(self, q_host, k_new_host, v_new_host):
         """Device q / new K / new V / out for these host shapes (made once per shape)."""
@@ -351,8 +343,8 @@ class DecodeSession:
             if k_new_host.dim() != 3 or tuple(k_new_host.shape[1:]) != (self.num_kv_heads, self.head_dim):
                 raise ValueError("new K/V must be [T, num_kv_heads, head_dim]")
             if self.fp8:
-                if q_host.dtype not in (torch.bfloat16, torch.float16):
-                    raise TypeError("q must be bf16 or f16 with FP8 pools")
+                if q_host.dtype not in (torch.bfloat16, torch.float16) or k_new_host.dtype != q_host.dtype:
+                    raise TypeError("with FP8 pools q and new K/V must be bf16 or f16, of one type")
             elif q_host.dtype != self.k_pool.dtype or k_new_host.dtype != self.k_pool.dtype:
                 raise TypeError("q and new K/V must have the pools' element type")
             if len(self._io) >= self._MAX_LAYOUTS:
@@ -361,10 +353,50 @@ class DecodeSession:
             kn = torch.empty(k_new_host.shape, dtype=k_new_host.dtype, device=self.device)
             vn = torch.empty(k_new_host.shape, dtype=k_new_host.dtype, device=self.device)
             out = torch.empty_like(q)
-            io = self._io[key] = (q, kn, vn, out)
+            io = self._io[key] = (key, q, kn, vn, out)
         if v_new_host.shape != k_new_host.shape or v_new_host.dtype != k_new_host.dtype:
             raise ValueError("k_new and v_new must have the same shape and element type")
+        if not (q_host.is_contiguous() and k_new_host.is_contiguous() and v_new_host.is_contiguous()):
+            raise ValueError("host inputs must be contiguous")
+        if q_host.is_cuda or k_new_host.is_cuda or v_new_host.is_cuda:
+            raise TypeError("launch_step takes host tensors")
         return io
+
+    def _step_struct(self, st: dict, p, io, n_cow: int) -> B.PkvStep:
+        """The pkv_step of one staging set and one input shape (host pointers
+        left to fill per step)."""
+        _, q, kn, vn, out = io
+        chunk = isinstance(p, ChunkPlan)
+        ins = (B.PkvCopy * 4)()
+        ins[0] = B.PkvCopy(st["dev"].data_ptr(), st["host"].data_ptr(), st["bytes"])
+        for c, t in zip(ins[1:], (q, kn, vn)):
+            c.dst, c.bytes = t.data_ptr(), t.numel() * t.element_size()
+        outs = (B.PkvCopy * 1)()
+        outs[0].src, outs[0].bytes = out.data_ptr(), out.numel() * out.element_size()
+        ptrs = st["ptrs"]
+        rest = ptrs[3 + (1 if n_cow else 0):]
+        kind = B.STEP_CHUNK if chunk else B.STEP_DECODE_FP8 if self.fp8 else \
+            B.STEP_DECODE_SHARED if p.has_groups else B.STEP_DECODE
+        k_scale, v_scale = self.kv_scales if self.fp8 else (1.0, 1.0)
+        step = B.PkvStep(
+            struct_size=ctypes.sizeof(B.PkvStep), kind=kind, in_=ins, n_in=4, out=outs, n_out=1,
+            k_pool=self.k_pool.data_ptr(), v_pool=self.v_pool.data_ptr(), num_blocks=self.num_blocks,
+            num_kv_heads=self.num_kv_heads, head_dim=self.head_dim, block_size=self.block_size,
+            dtype=B._dt(q), k_scale=float(k_scale), v_scale=float(v_scale),
+            pairs=ptrs[3] if n_cow else None, num_pairs=n_cow,
+            k_new=kn.data_ptr(), v_new=vn.data_ptr(), slot_mapping=ptrs[0], num_tokens=len(p.slot_mapping),
+            attn_out=out.data_ptr(), q=q.data_ptr(), block_tables=ptrs[2],
+            max_blocks_per_seq=p.block_tables.shape[1], context_lens=ptrs[1], num_seqs=len(p.lens),
+            num_q_heads=self.num_q_heads, scale=0.0, partition_size=self.partition_size,
+            workspace=self.workspace.data_ptr(), workspace_bytes=self.workspace.numel(),
+            group_first=rest[0] if (not chunk and p.has_groups) else None,
+            group_shared=rest[1] if (not chunk and p.has_groups) else None,
+            num_groups=len(p.group_shared) if (not chunk and p.has_groups) else 0,
+            max_group_size=int(p.max_group_size) if not chunk else 0,
+            max_shared_len=int(p.max_shared_len) if not chunk else 0,
+            query_start=rest[0] if chunk else None, max_query_len=int(p.max_query_len) if chunk else 0)
+        step._copies = (ins, outs)          # the arrays the struct points to stay alive with it
+        return step
 
     def launch_step(self, p, q_host: torch.Tensor, k_new_host: torch.Tensor, v_new_host: torch.Tensor,
                     out_host: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
@@ -382,61 +414,40 @@ class DecodeSession:
         if q_host.shape[0] != rows or k_new_host.shape[0] != T:
             raise ValueError("q needs one row per %s and new K/V one per written token"
                              % ("new token" if chunk else "attending sequence"))
-        q, kn, vn, out = self._io_buffers(q_host, k_new_host, v_new_host)
+        io = self._io_buffers(q_host, k_new_host, v_new_host)
+        out = io[4]
         if out_host is None:
             out_host = self._pin("out", out)
-        elif out_host.shape != out.shape or out_host.dtype != out.dtype:
-            raise ValueError("out_host must have the shape and element type of q")
+        elif out_host.shape != out.shape or out_host.dtype != out.dtype or out_host.is_cuda or \
+                not out_host.is_contiguous():
+            raise ValueError("out_host must be a contiguous host tensor of q's shape and element type")
         n_cow = len(p.cow_pairs)
         arrays = [p.slot_mapping, p.lens, p.block_tables] + ([p.cow_pairs] if n_cow else [])
         if chunk:
             arrays.append(p.query_start)
         elif p.has_groups:
             arrays += [p.group_first, p.group_shared]
-        with torch.cuda.stream(s):
-            st = self._staged(arrays, s)
-            q.copy_(q_host, non_blocking=True)
-            kn.copy_(k_new_host, non_blocking=True)
-            vn.copy_(v_new_host, non_blocking=True)
-            self._calls(p, st["ptrs"], n_cow, q, kn, vn, out, s.cuda_stream)
-            out_host.copy_(out, non_blocking=True)
+        st = self._layout(arrays)
+        if st["event"] is not None:
+            st["event"].synchronize()           # the step that last used this staging buffer is done
+        for hv, a in zip(st["hviews"], arrays):
+            np.copyto(hv, a, casting="no")
+        step = st["steps"].get(io[0])
+        if step is None:
+            step = st["steps"][io[0]] = self._step_struct(st, p, io, n_cow)
+        ins, outs = step._copies
+        ins[1].src, ins[2].src, ins[3].src = q_host.data_ptr(), k_new_host.data_ptr(), v_new_host.data_ptr()
+        outs[0].dst = out_host.data_ptr()
+        if chunk:                                # the plan's values that its layout does not fix
+            step.max_query_len = int(p.max_query_len)
+        elif p.has_groups:
+            step.max_group_size, step.max_shared_len = int(p.max_group_size), int(p.max_shared_len)
+        B.raw_call("pkv_step_from_host", ctypes.byref(step), s.cuda_stream)
+        if st["event"] is None:
+            st["event"] = torch.cuda.Event()
+        st["event"].record(s)
         return out_host
 
-    def _calls(self, p, ptrs, n_cow, q, kn, vn, out, sh) -> None:
-        """block_copy -> kv_append -> attention through the C ABI, on the
-        staged plan (pointers in the order launch_step packed the arrays)."""
-        NB, Hkv, bs, D = self.num_blocks, self.num_kv_heads, self.block_size, self.head_dim
-        kp, vp = self.k_pool.data_ptr(), self.v_pool.data_ptr()
-        sm, cl, bt = ptrs[0], ptrs[1], ptrs[2]
-        maxB = p.block_tables.shape[1]
-        T = len(p.slot_mapping)
-        if n_cow:
-            B.raw_call("pkv_block_copy", kp, vp, ptrs[3], n_cow, NB, Hkv, D, bs,
-                       B.FP8_E4M3 if self.fp8 else B._dt(self.k_pool), sh)
-        qdt = B._dt(q)
-        if self.fp8:
-            B.raw_call("pkv_kv_append_fp8", kn.data_ptr(), vn.data_ptr(), kp, vp, sm, T, NB, Hkv, D, bs,
-                       B._dt(kn), float(self.kv_scales[0]), float(self.kv_scales[1]), sh)
-        else:
-            B.raw_call("pkv_kv_append", kn.data_ptr(), vn.data_ptr(), kp, vp, sm, T, NB, Hkv, D, bs, qdt, sh)
-        ws, wsb = self.workspace.data_ptr(), self.workspace.numel()
-        P = self.partition_size
-        rest = ptrs[3 + (1 if n_cow else 0):]
-        if isinstance(p, ChunkPlan):
-            B.raw_call("pkv_paged_attention_chunk", out.data_ptr(), q.data_ptr(), kp, vp, bt, maxB, cl, rest[0],
-                       len(p.lens), T, int(p.max_query_len), self.num_q_heads, Hkv, D, bs, NB, 0.0, P, ws, wsb,
-                       qdt, sh)
-        elif self.fp8:
-            B.raw_call("pkv_paged_attention_decode_fp8", out.data_ptr(), q.data_ptr(), kp, vp, bt, maxB, cl,
-                       len(p.lens), self.num_q_heads, Hkv, D, bs, NB, 0.0, float(self.kv_scales[0]),
-                       float(self.kv_scales[1]), P, ws, wsb, qdt, sh)
-        elif p.has_groups:
-            B.raw_call("pkv_paged_attention_decode_shared", out.data_ptr(), q.data_ptr(), kp, vp, bt, maxB, cl,
-                       len(p.lens), self.num_q_heads, Hkv, D, bs, NB, 0.0, P, rest[0], rest[1],
-                       len(p.group_shared), int(p.max_group_size), int(p.max_shared_len), ws, wsb, qdt, sh)
-        else:
-            B.raw_call("pkv_paged_attention_decode", out.data_ptr(), q.data_ptr(), kp, vp, bt, maxB, cl,
-                       len(p.lens), self.num_q_heads, Hkv, D, bs, NB, 0.0, P, ws, wsb, qdt, sh)
 
     def upload(self, p: StepPlan) -> DevicePlan:
         """Copy a plan to the device: its arrays packed into one pinned staging

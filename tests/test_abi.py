@@ -330,6 +330,62 @@ def test_plain_c_consumer_builds_and_runs(tmp_path):
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stderr
 
 
+def test_step_struct_layout_matches_the_header(tmp_path):
+    """The binding's ctypes pkv_step / pkv_copy have the header's size and
+    field offsets (a C program compiled against the header prints them)."""
+    import subprocess
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    fields = [f for f, _ in binding.PkvStep._fields_]
+    cnames = ["in" if f == "in_" else f for f in fields]
+    src = ["#include <stddef.h>", "#include <stdio.h>", '#include "pagedkv.h"', "int main(void) {",
+           '  printf("%zu %zu\\n", sizeof(pkv_step), sizeof(pkv_copy));',
+           '  printf("%zu %zu %zu\\n", offsetof(pkv_copy, dst), offsetof(pkv_copy, src), offsetof(pkv_copy, bytes));']
+    src += ['  printf("%%zu\\n", offsetof(pkv_step, %s));' % c for c in cnames]
+    src += ["  return 0;", "}"]
+    c = tmp_path / "layout.c"
+    c.write_text("\n".join(src) + "\n")
+    exe = str(tmp_path / "layout")
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(root, "include"), "-o", exe,
+                           str(c)])
+    out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()
+    assert int(out[0]) == ctypes.sizeof(binding.PkvStep) and int(out[1]) == ctypes.sizeof(binding.PkvCopy)
+    assert [int(x) for x in out[2:5]] == [binding.PkvCopy.dst.offset, binding.PkvCopy.src.offset,
+                                          binding.PkvCopy.bytes.offset]
+    assert [int(x) for x in out[5:]] == [getattr(binding.PkvStep, f).offset for f in fields]
+
+
+def step_struct(**over):
+    st = binding.PkvStep(struct_size=ctypes.sizeof(binding.PkvStep), kind=binding.STEP_DECODE, num_blocks=8,
+                         num_kv_heads=4, head_dim=64, block_size=16, dtype=1, k_scale=1.0, v_scale=1.0,
+                         max_blocks_per_seq=4, num_q_heads=4)
+    for k, v in over.items():
+        setattr(st, k, v)
+    return st
+
+
+@pytest.mark.parametrize("over,why", [
+    (dict(struct_size=8), "struct_size"),
+    (dict(kind=7), "bad kind"),
+    (dict(n_in=-1), "bad copy lists"),
+    (dict(n_out=2), "bad copy lists"),                      # no list given
+    (dict(num_tokens=-3), "counts must be >= 0"),
+    (dict(num_pairs=1, pairs=16, k_pool=16, v_pool=8), "16-byte aligned"),        # pkv_block_copy's own check
+    (dict(num_tokens=2, k_new=16, v_new=16, k_pool=16, v_pool=16, slot_mapping=16, head_dim=6), "multiple of 16"),
+    (dict(num_seqs=1, q=16, attn_out=16, k_pool=16, v_pool=16, block_tables=16, context_lens=16, num_q_heads=6),
+     "multiple of num_kv_heads"),                             # the attention call's own check
+])
+def test_step_from_host_refuses_bad_steps(over, why):
+    host_only()
+    assert binding.lib.pkv_step_from_host(ctypes.byref(step_struct(**over)), None) == binding.INVALID
+    assert why in binding.lib.pkv_last_error().decode()
+
+
+def test_step_from_host_empty_step_and_null():
+    host_only()
+    assert binding.lib.pkv_step_from_host(ctypes.byref(step_struct()), None) == binding.OK   # nothing to do
+    assert binding.lib.pkv_step_from_host(None, None) == binding.INVALID
+
+
 def test_last_error_is_per_thread():
     """pkv_last_error() describes the last failed call on the calling thread:
     two threads failing different calls concurrently each read their own
