@@ -292,8 +292,9 @@ class DecodeSession:
     # A serving loop hands each step's inputs over in host memory and wants
     # the output back in host memory.  launch_step does that for a planned
     # step with one C call (pkv_step_from_host): the plan's arrays, packed into
-    # a pinned staging buffer, and q / new K / new V go to device buffers in
-    # four copies, then block_copy -> kv_append -> attention run and the output
+    # a pinned staging buffer, go in one copy and q / new K / new V in one more
+    # (three when they are not laid out in one host buffer like the device
+    # block), then block_copy -> kv_append -> attention run and the output
     # comes back in one copy.  The device buffers are made once per layout of
     # the plan's arrays (and per input shape) and the step description is
     # built and checked against their sizes then; a step only refills the
@@ -349,11 +350,18 @@ class DecodeSession:
                 raise TypeError("q and new K/V must have the pools' element type")
             if len(self._io) >= self._MAX_LAYOUTS:
                 self._io.pop(next(iter(self._io)))
-            q = torch.empty(q_host.shape, dtype=q_host.dtype, device=self.device)
-            kn = torch.empty(k_new_host.shape, dtype=k_new_host.dtype, device=self.device)
-            vn = torch.empty(k_new_host.shape, dtype=k_new_host.dtype, device=self.device)
+            # q, new K, new V in one device block, each at a 256-byte aligned
+            # offset: host inputs laid out the same way go in one copy.
+            qb = q_host.numel() * q_host.element_size()
+            kb = k_new_host.numel() * k_new_host.element_size()
+            ok = (qb + 255) // 256 * 256
+            ov = ok + (kb + 255) // 256 * 256
+            block = torch.empty(ov + kb, dtype=torch.uint8, device=self.device)
+            q = block[:qb].view(q_host.dtype).view(q_host.shape)
+            kn = block[ok:ok + kb].view(k_new_host.dtype).view(k_new_host.shape)
+            vn = block[ov:ov + kb].view(k_new_host.dtype).view(k_new_host.shape)
             out = torch.empty_like(q)
-            io = self._io[key] = (key, q, kn, vn, out)
+            io = self._io[key] = (key, q, kn, vn, out, (block, ok, ov))
         if v_new_host.shape != k_new_host.shape or v_new_host.dtype != k_new_host.dtype:
             raise ValueError("k_new and v_new must have the same shape and element type")
         if not (q_host.is_contiguous() and k_new_host.is_contiguous() and v_new_host.is_contiguous()):
@@ -365,7 +373,7 @@ class DecodeSession:
     def _step_struct(self, st: dict, p, io, n_cow: int) -> B.PkvStep:
         """The pkv_step of one staging set and one input shape (host pointers
         left to fill per step)."""
-        _, q, kn, vn, out = io
+        _, q, kn, vn, out, _ = io
         chunk = isinstance(p, ChunkPlan)
         ins = (B.PkvCopy * 4)()
         ins[0] = B.PkvCopy(st["dev"].data_ptr(), st["host"].data_ptr(), st["bytes"])
@@ -406,7 +414,9 @@ class DecodeSession:
         ``out_host`` (pinned; made if None) -- complete once ``stream`` reaches
         this point.  q_host [rows, num_q_heads, head_dim]; k/v_new_host
         [tokens written, num_kv_heads, head_dim]; pinned host memory lets the
-        copies run asynchronously."""
+        copies run asynchronously.  Inputs that sit in one host buffer -- q,
+        then new K at the next 256-byte boundary after q, then new V at the
+        next after new K -- are sent with a single copy."""
         s = torch.cuda.current_stream() if stream is None else stream
         chunk = isinstance(p, ChunkPlan)
         T = len(p.slot_mapping)
@@ -436,7 +446,15 @@ class DecodeSession:
         if step is None:
             step = st["steps"][io[0]] = self._step_struct(st, p, io, n_cow)
         ins, outs = step._copies
-        ins[1].src, ins[2].src, ins[3].src = q_host.data_ptr(), k_new_host.data_ptr(), v_new_host.data_ptr()
+        block, ok, ov = io[5]
+        qp, kp, vp = q_host.data_ptr(), k_new_host.data_ptr(), v_new_host.data_ptr()
+        if kp - qp == ok and vp - qp == ov:      # inputs packed like the device block: one copy
+            ins[1].src, ins[1].bytes = qp, block.numel()
+            step.n_in = 2
+        else:
+            ins[1].src, ins[1].bytes = qp, q_host.numel() * q_host.element_size()
+            ins[2].src, ins[3].src = kp, vp
+            step.n_in = 4
         outs[0].dst = out_host.data_ptr()
         if chunk:                                # the plan's values that its layout does not fix
             step.max_query_len = int(p.max_query_len)

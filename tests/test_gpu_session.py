@@ -143,6 +143,25 @@ def test_add_with_a_prefix_ending_inside_a_block_copies_that_block(prefix_tokens
     assert max_err(out, ref) <= TOL[out.dtype]
 
 
+def packed_inputs(rows, T, sh, dt, g):
+    """q, new K, new V in one pinned buffer at 256-byte aligned offsets (the
+    layout launch_step sends with one copy)."""
+    shapes = [(rows, sh.Hq, sh.D), (T, sh.Hkv, sh.D), (T, sh.Hkv, sh.D)]
+    esz = torch.empty((), dtype=dt).element_size()
+    offs, total = [], 0
+    for shp in shapes:
+        offs.append(total)
+        total += (int(np.prod(shp)) * esz + 255) // 256 * 256
+    buf = torch.empty(total, dtype=torch.uint8).pin_memory()
+    views = []
+    for shp, o in zip(shapes, offs):
+        v = buf[o:o + int(np.prod(shp)) * esz].view(dt).view(shp)
+        v.copy_(synth.randn(shp, g, dt, "cpu"))
+        views.append(v)
+    return views
+
+
+@pytest.mark.parametrize("packed", [False, True])
 @pytest.mark.parametrize("cfg,over", [
     ("llama13b_prefix", dict(S=12, Hq=4, Hkv=4)),                              # shared-prefix groups
     ("longctx_beam", dict(S=2, Hq=16, Hkv=2, len_fixed=2000)),                 # forks: copy-on-write pairs
@@ -150,7 +169,7 @@ def test_add_with_a_prefix_ending_inside_a_block_copies_that_block(prefix_tokens
     ("llama7b_fp8", dict(S=6, Hq=4, Hkv=4, len_uniform=(1, 600))),             # FP8 pools
     ("llama3_gqa_bs32", dict(S=4, len_fixed=None, len_uniform=(1, 900))),      # grouped-query heads
 ])
-def test_launch_step_planned_ahead_matches_oracle(cfg, over):
+def test_launch_step_planned_ahead_matches_oracle(cfg, over, packed):
     """DecodeSession.launch_step from pinned host buffers, the next step
     planned while the device works (as bench.py's end-to-end leg does),
     on every kind of plan: after each step the output equals the oracle's
@@ -171,9 +190,12 @@ def test_launch_step_planned_ahead_matches_oracle(cfg, over):
     for step in range(4):
         T = len(p.slot_mapping)
         rows = T if sh.chunk else len(p.seq_ids)
-        q = synth.randn((rows, sh.Hq, sh.D), g, dt, "cpu").pin_memory()
-        kn = synth.randn((T, sh.Hkv, sh.D), g, dt, "cpu").pin_memory()
-        vn = synth.randn((T, sh.Hkv, sh.D), g, dt, "cpu").pin_memory()
+        if packed:           # one host buffer: one copy
+            q, kn, vn = packed_inputs(rows, T, sh, dt, g)
+        else:
+            q = synth.randn((rows, sh.Hq, sh.D), g, dt, "cpu").pin_memory()
+            kn = synth.randn((T, sh.Hkv, sh.D), g, dt, "cpu").pin_memory()
+            vn = synth.randn((T, sh.Hkv, sh.D), g, dt, "cpu").pin_memory()
         out_host = ss.launch_step(p, q, kn, vn, out_host)
         nxt = wl.plan()                          # planned while this step runs
         torch.cuda.current_stream().synchronize()
