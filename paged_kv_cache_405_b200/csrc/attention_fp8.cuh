@@ -296,7 +296,10 @@ struct Fp8HeadCfg {
     static_assert(TT == 16 || TT == 32, "16 or 32 tokens per stage");
 };
 
-template <int D, int WARPS, int STAGES, typename To, int TT = kTileTok, int MINB = 4>
+// LATE_V: the V codes are read from the stage after the softmax (the stage
+// goes back to TMA then) instead of with the K codes, so the K and V codes
+// are never held in registers at the same time.
+template <int D, int WARPS, int STAGES, typename To, int TT = kTileTok, int MINB = 4, bool LATE_V = false>
 __global__ void __launch_bounds__(WARPS * 32, MINB) paged_attn_fp8_head_kernel(const AttnParams p,
                                                                                const __grid_constant__ CUtensorMap tmK,
                                                                                const __grid_constant__ CUtensorMap tmV) {
@@ -392,15 +395,40 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) paged_attn_fp8_head_kernel(c
         const int valid = min(TT, t_end - (t_begin + i * TT));
         const uint8_t* stage = ring + st * C::kStageBytes;
 
-        // Codes of this lane's fragments, then the stage goes back to TMA.
+        // Codes of this lane's fragments; the stage goes back to TMA once
+        // both the K and the V codes are in registers.
         uint32_t kw[HV][2][KSTEPS];  // codes of rows gid and gid + 8 of each tile
         uint32_t vw[HV][4][VW];
+        auto load_v = [&]() {
+#pragma unroll
+            for (int hh = 0; hh < HV; ++hh) {
+                const int vh = valid - hh * kTileTok;  // tokens of this tile (warp-uniform)
+                if (vh <= 0) continue;
+                const uint8_t* vt = stage + (HV + hh) * C::kTileBytes;
+                zero_tail_rows<D>(const_cast<uint8_t*>(vt), vh, lane);
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    if constexpr (VW == 4) {
+                        const uint4 w = *reinterpret_cast<const uint4*>(vt + fp8_chunk<D>(vtok[t], gid));
+                        vw[hh][t][0] = w.x;
+                        vw[hh][t][1] = w.y;
+                        vw[hh][t][2] = w.z;
+                        vw[hh][t][3] = w.w;
+                    } else {
+                        const uint2 w = *reinterpret_cast<const uint2*>(vt + vtok[t] * D + gid * 8);
+                        vw[hh][t][0] = w.x;
+                        vw[hh][t][1] = w.y;
+                    }
+                }
+            }
+            __syncwarp();
+            if (i + STAGES < ntiles) issue(i + STAGES);
+        };
 #pragma unroll
         for (int hh = 0; hh < HV; ++hh) {
             const int vh = valid - hh * kTileTok;  // tokens of this tile (warp-uniform)
             if (vh <= 0) continue;
             const uint8_t* kt = stage + hh * C::kTileBytes;
-            const uint8_t* vt = stage + (HV + hh) * C::kTileBytes;
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
 #pragma unroll
@@ -412,24 +440,8 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) paged_attn_fp8_head_kernel(c
                     kw[hh][r][4 * c + 3] = w.w;
                 }
             }
-            zero_tail_rows<D>(const_cast<uint8_t*>(vt), vh, lane);
-#pragma unroll
-            for (int t = 0; t < 4; ++t) {
-                if constexpr (VW == 4) {
-                    const uint4 w = *reinterpret_cast<const uint4*>(vt + fp8_chunk<D>(vtok[t], gid));
-                    vw[hh][t][0] = w.x;
-                    vw[hh][t][1] = w.y;
-                    vw[hh][t][2] = w.z;
-                    vw[hh][t][3] = w.w;
-                } else {
-                    const uint2 w = *reinterpret_cast<const uint2*>(vt + vtok[t] * D + gid * 8);
-                    vw[hh][t][0] = w.x;
-                    vw[hh][t][1] = w.y;
-                }
-            }
         }
-        __syncwarp();
-        if (i + STAGES < ntiles) issue(i + STAGES);
+        if constexpr (!LATE_V) load_v();
 
         // S^T of each tile: two accumulator chains (even / odd k-steps) halve
         // the MMA dependency depth.
@@ -469,6 +481,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) paged_attn_fp8_head_kernel(c
                 o[j][2] *= alpha;
             }
         }
+        if constexpr (LATE_V) load_v();
 #pragma unroll
         for (int hh = 0; hh < HV; ++hh) {
             if (valid - hh * kTileTok <= 0) continue;  // warp-uniform

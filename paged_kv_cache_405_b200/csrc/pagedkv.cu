@@ -283,6 +283,9 @@ static cudaError_t launch_mma_fp8(const pkv::AttnParams& p, dim3 grid, const CUt
 #ifndef PKV_FP8_HEAD_MINB
 #define PKV_FP8_HEAD_MINB 4
 #endif
+#ifndef PKV_FP8_HEAD_LATE_V
+#define PKV_FP8_HEAD_LATE_V 0
+#endif
 
 template <typename To, int D>
 static cudaError_t launch_head_fp8(const pkv::AttnParams& p, dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv,
@@ -290,7 +293,8 @@ static cudaError_t launch_head_fp8(const pkv::AttnParams& p, dim3 grid, const CU
     constexpr int TT = PKV_FP8_HEAD_TT;
     using C = pkv::Fp8HeadCfg<D, TT>;
     constexpr int kSmem = 1024 + kMmaWarps * kFp8Stages * (C::kStageBytes + 8);
-    auto k = pkv::paged_attn_fp8_head_kernel<D, kMmaWarps, kFp8Stages, To, TT, PKV_FP8_HEAD_MINB>;
+    auto k = pkv::paged_attn_fp8_head_kernel<D, kMmaWarps, kFp8Stages, To, TT, PKV_FP8_HEAD_MINB,
+                                             PKV_FP8_HEAD_LATE_V != 0>;
     static cudaError_t attr = set_smem(k, kSmem);
     if (attr != cudaSuccess) return attr;
     return launch_k(k, grid, dim3(kMmaWarps * 32), kSmem, st, p, mk, mv);
