@@ -371,7 +371,7 @@ def workload_shape(args, name=None):
     if args.batch:
         shape = synth.shrink(shape, S=args.batch)
     # room in every table and in the pool for the tokens the run appends
-    grow = (args.warmup + args.steps + 8) * max(1, shape.chunk)
+    grow = (max(args.warmup, 10) + args.steps + 8) * max(1, shape.chunk)
     if grow > shape.reserve_tokens:
         shape = synth.shrink(shape, reserve_tokens=grow)
     return shape
@@ -608,7 +608,7 @@ def run_e2e(args, wl, world, rank, dev):
     import paged_kv_cache_405_b200 as pkv
     shape = wl.shape
     ss = wl.session
-    K, W = args.steps, args.warmup
+    K, W = args.steps, max(args.warmup, 10)      # untimed steps: at least 10 (staging for every layout made)
     dt = synth.DTYPES[shape.dtype]
     T = shape.S * max(1, shape.beams, shape.chunk)
     Tq = shape.S * max(1, shape.chunk)
@@ -632,10 +632,15 @@ def run_e2e(args, wl, world, rank, dev):
     stream = torch.cuda.current_stream()
     plans = []
 
-    def run(first, n):
+    step_ev = []
+
+    def run(first, n, events=False):
         p = wl.plan()
         plans.append(p)
         for i in range(first, first + n):
+            if events:
+                step_ev.append(torch.cuda.Event(enable_timing=True))
+                step_ev[-1].record(stream)
             ss.launch_step(p, *host_inputs[i][1], out_host=out_host, stream=stream)
             if i + 1 < first + n:
                 p = wl.plan()       # host work of the next step, overlapping this step's kernels
@@ -655,10 +660,11 @@ def run_e2e(args, wl, world, rank, dev):
     torch.cuda.synchronize()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     t0.record(stream)
-    run(W, K)
+    run(W, K, events=True)
     t1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(t0.elapsed_time(t1), world)
+    per_step = [a.elapsed_time(b) for a, b in zip(step_ev, step_ev[1:] + [t1])]
     timed = plans[W:]
     nbytes = [wl.step_bytes(p)[0] for p in timed]
     tot = sum_over_ranks(float(sum(nbytes)), world)
@@ -668,6 +674,7 @@ def run_e2e(args, wl, world, rank, dev):
     d2h = out_host.numel() * out_host.element_size()
     return {"value": round(tot / (ms * 1e-3) / 1e9, 1), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms / K, 4),
+            "ms_per_step_median": round(float(np.median(per_step)), 4),
             "api": "DecodeSession.plan (next step planned during this one) + DecodeSession.launch_step (H2D of "
                    "the inputs from pinned host memory and of the plan, block_copy/kv_append/attention, D2H of "
                    "the output), host waits for the output every step"}

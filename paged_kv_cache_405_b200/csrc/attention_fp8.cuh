@@ -191,8 +191,8 @@ __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_fp8_kernel(const Att
         for (int kk = 0; kk < KSTEPS; ++kk) {
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
-                const uint32_t b0 = e4m3x2_to_f16x2((uint16_t)(kw[nt][kk] & 0xffffu));
-                const uint32_t b1 = e4m3x2_to_f16x2((uint16_t)(kw[nt][kk] >> 16));
+                uint32_t b0, b1;
+                e4m3x4_to_f16x2x2(kw[nt][kk], b0, b1);
                 mma_16816<__half>(sacc[nt], acc.qa[kk], b0, b1);
             }
         }
@@ -207,14 +207,15 @@ __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_fp8_kernel(const Att
             const uint32_t hi0 = __byte_perm(vw[0][w], vw[1][w], 0x7362);
             const uint32_t lo1 = __byte_perm(vw[2][w], vw[3][w], 0x5140);
             const uint32_t hi1 = __byte_perm(vw[2][w], vw[3][w], 0x7362);
-            mma_16816<__half>(acc.o[4 * w], pa, e4m3x2_to_f16x2((uint16_t)(lo0 & 0xffffu)),
-                              e4m3x2_to_f16x2((uint16_t)(lo1 & 0xffffu)));
-            mma_16816<__half>(acc.o[4 * w + 1], pa, e4m3x2_to_f16x2((uint16_t)(lo0 >> 16)),
-                              e4m3x2_to_f16x2((uint16_t)(lo1 >> 16)));
-            mma_16816<__half>(acc.o[4 * w + 2], pa, e4m3x2_to_f16x2((uint16_t)(hi0 & 0xffffu)),
-                              e4m3x2_to_f16x2((uint16_t)(hi1 & 0xffffu)));
-            mma_16816<__half>(acc.o[4 * w + 3], pa, e4m3x2_to_f16x2((uint16_t)(hi0 >> 16)),
-                              e4m3x2_to_f16x2((uint16_t)(hi1 >> 16)));
+            uint32_t l0a, l0b, l1a, l1b, h0a, h0b, h1a, h1b;
+            e4m3x4_to_f16x2x2(lo0, l0a, l0b);
+            e4m3x4_to_f16x2x2(lo1, l1a, l1b);
+            e4m3x4_to_f16x2x2(hi0, h0a, h0b);
+            e4m3x4_to_f16x2x2(hi1, h1a, h1b);
+            mma_16816<__half>(acc.o[4 * w], pa, l0a, l1a);
+            mma_16816<__half>(acc.o[4 * w + 1], pa, l0b, l1b);
+            mma_16816<__half>(acc.o[4 * w + 2], pa, h0a, h1a);
+            mma_16816<__half>(acc.o[4 * w + 3], pa, h0b, h1b);
         }
     }
 #pragma unroll
@@ -455,10 +456,9 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) paged_attn_fp8_head_kernel(c
             float sa[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
             for (int kk = 0; kk < KSTEPS; ++kk) {
-                const uint32_t a[4] = {e4m3x2_to_f16x2((uint16_t)(kw[hh][0][kk] & 0xffffu)),
-                                       e4m3x2_to_f16x2((uint16_t)(kw[hh][1][kk] & 0xffffu)),
-                                       e4m3x2_to_f16x2((uint16_t)(kw[hh][0][kk] >> 16)),
-                                       e4m3x2_to_f16x2((uint16_t)(kw[hh][1][kk] >> 16))};
+                uint32_t a[4];
+                e4m3x4_to_f16x2x2(kw[hh][0][kk], a[0], a[2]);
+                e4m3x4_to_f16x2x2(kw[hh][1][kk], a[1], a[3]);
                 mma_16816<__half>(sa[kk & 1], a, qb[kk][0], qb[kk][1]);
             }
             if (live && gid < vh) x[hh][0] = (sa[0][0] + sa[1][0]) * p.scale_log2;
@@ -502,11 +502,12 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) paged_attn_fp8_head_kernel(c
                 const uint32_t hi0 = __byte_perm(vw[hh][0][w], vw[hh][1][w], 0x7362);
                 const uint32_t lo1 = __byte_perm(vw[hh][2][w], vw[hh][3][w], 0x5140);
                 const uint32_t hi1 = __byte_perm(vw[hh][2][w], vw[hh][3][w], 0x7362);
-                const uint32_t a0[4] = {e4m3x2_to_f16x2((uint16_t)(lo0 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(lo0 >> 16)),
-                                        e4m3x2_to_f16x2((uint16_t)(lo1 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(lo1 >> 16))};
+                uint32_t a0[4], a1[4];
+                e4m3x4_to_f16x2x2(lo0, a0[0], a0[1]);
+                e4m3x4_to_f16x2x2(lo1, a0[2], a0[3]);
                 mma_16816<__half>(o[2 * w], a0, pb0, pb1);
-                const uint32_t a1[4] = {e4m3x2_to_f16x2((uint16_t)(hi0 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(hi0 >> 16)),
-                                        e4m3x2_to_f16x2((uint16_t)(hi1 & 0xffffu)), e4m3x2_to_f16x2((uint16_t)(hi1 >> 16))};
+                e4m3x4_to_f16x2x2(hi0, a1[0], a1[1]);
+                e4m3x4_to_f16x2x2(hi1, a1[2], a1[3]);
                 mma_16816<__half>(o[2 * w + 1], a1, pb0, pb1);
             }
         }

@@ -206,6 +206,18 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t two) {
     return h;
 }
 
+// Four E4M3 codes (one 32-bit word, byte 0 first) -> two half pairs, exactly:
+// lo = codes 0, 1; hi = codes 2, 3.  The word is split into its two 16-bit
+// halves inside the asm, so no shift or mask is spent on it.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 l, h;\n\t"
+        "mov.b32 {l, h}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, l;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, h;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
+}
+
 // Two floats -> two E4M3 codes (lo in the low byte), round to nearest even,
 // saturating to +-448.
 __device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
