@@ -15,6 +15,7 @@
 
 #include "../../include/pagedkv.h"
 #include "attention_fp8.cuh"
+#include "attention_fp8_tc.cuh"
 #include "attention_mma.cuh"
 #include "attention_simt.cuh"
 #include "block_copy.cuh"
@@ -395,6 +396,24 @@ static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int npart
     return D == 64 ? launch_reduce<T, 64>(r, st) : launch_reduce<T, 128>(r, st);
 }
 
+// Per-head FP8 decode at head_dim 128 on tcgen05 (build-time switch).
+#ifndef PKV_FP8_TC
+#define PKV_FP8_TC 0
+#endif
+#ifndef PKV_FP8_TC_STAGES
+#define PKV_FP8_TC_STAGES 2
+#endif
+
+template <typename To>
+static cudaError_t launch_head_fp8_tc(const pkv::AttnParams& p, int nparts, const CUtensorMap& mk, const CUtensorMap& mv,
+                                      cudaStream_t st) {
+    using C = pkv::Fp8TcCfg<PKV_FP8_TC_STAGES>;
+    auto k = pkv::paged_attn_fp8_tc_kernel<PKV_FP8_TC_STAGES, To>;
+    static cudaError_t attr = set_smem(k, C::kSmemBytes);
+    if (attr != cudaSuccess) return attr;
+    return launch_k(k, dim3(p.Hq, nparts, p.S), dim3(128), C::kSmemBytes, st, p, mk, mv);
+}
+
 template <typename To>
 static cudaError_t dispatch_attention_fp8(const pkv::AttnParams& p, int D, int nparts, bool use_mma,
                                           const CUtensorMap* mk, const CUtensorMap* mv, cudaStream_t st) {
@@ -402,6 +421,8 @@ static cudaError_t dispatch_attention_fp8(const pkv::AttnParams& p, int D, int n
     if (use_mma) {
         dim3 grid((p.Hkv + kMmaWarps - 1) / kMmaWarps, nparts, p.S);
         e = D == 64 ? launch_mma_fp8<To, 64>(p, grid, *mk, *mv, st) : launch_mma_fp8<To, 128>(p, grid, *mk, *mv, st);
+    } else if (PKV_FP8_TC && D == 128) {
+        e = launch_head_fp8_tc<To>(p, nparts, *mk, *mv, st);
     } else {
         dim3 grid((p.Hq + kMmaWarps - 1) / kMmaWarps, nparts, p.S);
         e = D == 64 ? launch_head_fp8<To, 64>(p, grid, *mk, *mv, st) : launch_head_fp8<To, 128>(p, grid, *mk, *mv, st);
