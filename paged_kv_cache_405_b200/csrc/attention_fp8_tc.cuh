@@ -17,24 +17,30 @@
 //                  q_hi + q_lo up to 2^-8 relative), other rows zero.  Thread t
 //                  reads columns 0, 1 of lane t: token t's score is
 //                  (c0 + c1) / s_q (times the softmax scale and k_scale).
-//   softmax        each thread owns one token; the tile maximum and, at the
-//                  end, the sum go through shared memory across the 4 warps.
-//   O^T = V^T P^T  M = 128 head-dim elements, N = 16, K = tokens (32 per MMA).
-//                  A = the V tile read MN-major (a token row of 128 codes is
-//                  128 consecutive M elements); B = P: row 0 = p_hi, row 1 =
-//                  p_lo, 448 p split into two E4M3 terms like q.  The tile's
-//                  O^T is written fresh into TMEM; thread t reads columns 0,
-//                  1 of lane t and accumulates o[t] = o[t] * alpha + c0 + c1
-//                  in a register (head-dim element t).
+//   softmax        per warp: warp w owns tokens 32w .. 32w+31 of every tile
+//                  and keeps its own running maximum m_w and sum l_w (a
+//                  split of the context into four interleaved parts, merged
+//                  at the end as split-K partials are), so a tile needs no
+//                  exchange between warps.
+//   O^T = V^T P^T  M = 128 head-dim elements, N = 16, K = tokens (32 per MMA,
+//                  one warp's tokens).  A = the V tile read MN-major (a token
+//                  row of 128 codes is 128 consecutive M elements); B = P:
+//                  rows 2w, 2w+1 = p_hi, p_lo of warp w's tokens (448 p split
+//                  into two E4M3 terms like q) and zero elsewhere, so output
+//                  columns 2w, 2w+1 collect warp w's tokens only.  Thread t
+//                  reads columns 0-7 of lane t and keeps, per warp w,
+//                  o_w[t] = o_w[t] * alpha_w + c_2w + c_2w+1 (head-dim element t).
 // The splits keep ~8 significant bits of q and of every softmax weight, as
 // much as a bf16 operand; K and V codes are used exactly.
 //
-// Synchronisation: one thread issues the TMA copies and the MMAs; MMA
-// completion arrives on an mbarrier (tcgen05.commit); every wait is bounded
-// in time, and on a give-up the CTA records PKV_DEVERR_TIMEOUT, waits
-// (bounded) for its copies and MMAs in flight, frees its tensor memory and
-// returns.  Tensor memory: 32 columns per CTA (S^T in columns 0-15, O^T in
-// 16-31), at most 3 CTAs per SM (shared memory), so an allocation never waits.
+// Pipeline: one thread issues the TMA copies and the MMAs, and issues the
+// next tile's S^T right behind this tile's O^T, so that the two overlap; MMA
+// completion arrives on mbarriers (tcgen05.commit); one CTA barrier per tile
+// (P written -> O^T issued).  Every wait is bounded in time, and on a give-up
+// the CTA records PKV_DEVERR_TIMEOUT, waits (bounded) for its copies and
+// MMAs in flight, frees its tensor memory and returns.  Tensor memory: 32
+// columns per CTA (S^T in columns 0-15, O^T in 16-31), few enough CTAs per SM
+// (shared memory bounds them) that an allocation never waits.
 #pragma once
 #include "attention_common.cuh"
 
@@ -121,16 +127,20 @@ struct Fp8TcCfg {
     static constexpr int kStageBytes = 2 * kTcTileBytes;  // K tile, then V tile
     static constexpr int kQOff = STAGES * kStageBytes;    // Q operand: 16 rows x 128 codes
     static constexpr int kPOff = kQOff + 2048;            // P operand: 16 rows x 128 codes
-    static constexpr int kBarOff = kPOff + 2048;          // STAGES TMA barriers, then the MMA barrier
-    static constexpr int kRedOff = kBarOff + 8 * (STAGES + 1);  // 4 floats of block reductions
-    static constexpr int kTmemOff = kRedOff + 16;         // tensor-memory address
+    static constexpr int kBarOff = kPOff + 2048;          // STAGES TMA barriers, S^T and O^T barriers
+    static constexpr int kRedOff = kBarOff + 8 * (STAGES + 2);  // 16 floats: alphas (2 x 4), m (4), l (4)
+    static constexpr int kTmemOff = kRedOff + 64;         // tensor-memory address
     static constexpr int kSmemBytes = 1024 + kTmemOff + 16;  // + alignment slack
 };
 
+#ifndef PKV_FP8_TC_MINB
+#define PKV_FP8_TC_MINB 3
+#endif
+
 template <int STAGES, typename To>
-__global__ void __launch_bounds__(128, 3) paged_attn_fp8_tc_kernel(const AttnParams p,
-                                                                   const __grid_constant__ CUtensorMap tmK,
-                                                                   const __grid_constant__ CUtensorMap tmV) {
+__global__ void __launch_bounds__(128, PKV_FP8_TC_MINB) paged_attn_fp8_tc_kernel(const AttnParams p,
+                                                                                 const __grid_constant__ CUtensorMap tmK,
+                                                                                 const __grid_constant__ CUtensorMap tmV) {
     using C = Fp8TcCfg<STAGES>;
     constexpr int D = 128;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -149,8 +159,9 @@ __global__ void __launch_bounds__(128, 3) paged_attn_fp8_tc_kernel(const AttnPar
     uint8_t* qmat = smem + C::kQOff;
     uint8_t* pmat = smem + C::kPOff;
     const uint32_t bar0 = sbase + C::kBarOff;          // TMA stage barriers
-    const uint32_t mbar = bar0 + 8 * STAGES;           // MMA completion barrier
-    float* red = reinterpret_cast<float*>(smem + C::kRedOff);
+    const uint32_t sbar = bar0 + 8 * STAGES;           // S^T completion
+    const uint32_t obar = sbar + 8;                    // O^T completion
+    float* red = reinterpret_cast<float*>(smem + C::kRedOff);  // [0, 8): alphas by tile parity; [8, 12): m; [12, 16): l
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kTmemOff);
 
     // ---- set-up: tensor memory, barriers, the Q and P operands
@@ -162,14 +173,12 @@ __global__ void __launch_bounds__(128, 3) paged_attn_fp8_tc_kernel(const AttnPar
     if (tid == 0) {
         prefetch_tensor_map(&tmK);
         prefetch_tensor_map(&tmV);
-        for (int i = 0; i <= STAGES; ++i) mbar_init(bar0 + 8 * i, 1);
+        for (int i = 0; i < STAGES + 2; ++i) mbar_init(bar0 + 8 * i, 1);
         fence_barrier_init();
     }
-    // rows 2..15 of Q and P stay zero; rows 0, 1 are written below / per tile
-    for (int i = tid; i < 2 * 2048 / 16; i += 128) {
-        const int off = i < 128 ? i * 16 : 2048 + (i - 128) * 16;
-        *reinterpret_cast<uint4*>(qmat + off) = make_uint4(0u, 0u, 0u, 0u);
-    }
+    // every row of Q and P starts at zero; Q rows 0, 1 are written below,
+    // P rows 2w, 2w+1 by warp w in its own 32 columns each tile
+    for (int i = tid; i < 2 * 2048 / 16; i += 128) *reinterpret_cast<uint4*>(qmat + i * 16) = make_uint4(0u, 0u, 0u, 0u);
     float qv;
     {
         const To* qr = reinterpret_cast<const To*>(p.q) + ((int64_t)s * p.Hq + h) * D;
@@ -189,7 +198,7 @@ __global__ void __launch_bounds__(128, 3) paged_attn_fp8_tc_kernel(const AttnPar
         qmat[tc::sw128(0, tid)] = (uint8_t)hi;
         qmat[tc::sw128(1, tid)] = (uint8_t)lo;
     }
-    fence_proxy_async();  // generic writes of Q / P zeros before the MMAs read them
+    fence_proxy_async();  // generic writes of Q / P before the MMAs read them
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -202,7 +211,9 @@ __global__ void __launch_bounds__(128, 3) paged_attn_fp8_tc_kernel(const AttnPar
     BlockWindow win;  // used by warp 0 only
     if (warp == 0) win.init(p.block_tables + (int64_t)s * p.maxB, jb0, (t_end - 1) / p.bs - jb0 + 1, lane);
 
-    auto issue = [&](int i) {  // warp 0
+    int issued = 0;  // tiles whose copies were issued (warp 0)
+    auto issue_tma = [&](int i) {  // warp 0
+        issued = i + 1;
         const int t0 = t_begin + i * kTcTile;
         const int st = i % STAGES;
         const uint32_t bar = bar0 + 8 * st;
@@ -222,97 +233,110 @@ __global__ void __launch_bounds__(128, 3) paged_attn_fp8_tc_kernel(const AttnPar
             }
         }
     };
-    if (warp == 0) {
-        const int npre = ntiles < STAGES ? ntiles : STAGES;
-        for (int i = 0; i < npre; ++i) issue(i);
-    }
-
     constexpr uint32_t kIdS = tc::idesc_e4m3_m128_n16(false);
     constexpr uint32_t kIdO = tc::idesc_e4m3_m128_n16(true);
     const uint32_t qaddr = sbase + C::kQOff, paddr = sbase + C::kPOff;
-    float m = -INFINITY, lpart = 0.f, o = 0.f;
-    uint32_t mphase = 0;
+    // tid 0: wait for tile i's copies, then S^T(i); false if the wait gave up
+    auto issue_s = [&](int i) -> bool {
+        const int st = i % STAGES;
+        if (!mbar_wait(bar0 + 8 * st, (i / STAGES) & 1)) return false;
+        tc::fence_after_sync();
+        const uint32_t kaddr = sbase + st * C::kStageBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 32; ++kk)
+            tc::mma_f8f6f4(tmem + kTcColsS, tc::smem_desc_sw128(kaddr + kk * 32, 16, 1024),
+                           tc::smem_desc_sw128(qaddr + kk * 32, 16, 1024), kIdS, kk > 0);
+        tc::commit(sbar);
+        return true;
+    };
+
+    if (warp == 0) {
+        const int npre = ntiles < STAGES ? ntiles : STAGES;
+        for (int i = 0; i < npre; ++i) issue_tma(i);
+    }
     bool ok = true;
+    if (tid == 0) ok = issue_s(0);
+
+    float m = -INFINITY, lsum = 0.f;        // this warp's running max; this lane's share of its sum
+    float o[4] = {0.f, 0.f, 0.f, 0.f};      // head-dim element tid, one partial per warp
+    uint32_t sph = 0, oph = 0;
     int i = 0;
     for (; i < ntiles; ++i) {
         const int st = i % STAGES;
-        const uint32_t kaddr = sbase + st * C::kStageBytes, vaddr = kaddr + kTcTileBytes;
+        const uint32_t vaddr = sbase + st * C::kStageBytes + kTcTileBytes;
         const int valid = min(kTcTile, t_end - (t_begin + i * kTcTile));
-        ok = mbar_wait(bar0 + 8 * st, (i / STAGES) & 1);
-        if (!__syncthreads_and(ok ? 1 : 0)) break;
-        // V rows past the context inside the last 32-token group may hold any
-        // code (NaN included) and would meet a zero weight: clear them.
         const int vrows = (valid + 31) & ~31;
-        if (valid < vrows) {
-            uint8_t* vt = smem + st * C::kStageBytes + kTcTileBytes;
-            for (int idx = tid; idx < (vrows - valid) * 8; idx += 128)
-                *reinterpret_cast<uint4*>(vt + (valid + idx / 8) * 128 + (idx % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
-            fence_proxy_async();
-        }
-        __syncthreads();
-        // S^T = K Q^T
-        if (tid == 0) {
-            tc::fence_after_sync();
-#pragma unroll
-            for (int kk = 0; kk < D / 32; ++kk)
-                tc::mma_f8f6f4(tmem + kTcColsS, tc::smem_desc_sw128(kaddr + kk * 32, 16, 1024),
-                               tc::smem_desc_sw128(qaddr + kk * 32, 16, 1024), kIdS, kk > 0);
-            tc::commit(mbar);
-        }
-        ok = mbar_wait(mbar, mphase);
-        mphase ^= 1;
+        ok = ok && mbar_wait(sbar, sph);  // (tid 0 whose copies gave up does not wait)
+        sph ^= 1;
         if (!__syncthreads_and(ok ? 1 : 0)) break;
         tc::fence_after_sync();
         float c0, c1;
         tc::ld_x2(tmem + t_lane + kTcColsS, c0, c1);
         const float x = tid < valid ? (c0 + c1) * (p.scale_log2 / sq) : -INFINITY;
-        float tmax = x;
+        float wmax = x;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, off));
-        if (lane == 0) red[warp] = tmax;
-        __syncthreads();
-        tmax = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
-        const float mn = fmaxf(m, tmax);
+        for (int off = 16; off > 0; off >>= 1) wmax = fmaxf(wmax, __shfl_xor_sync(0xffffffffu, wmax, off));
+        const float mn = fmaxf(m, wmax);
         const float b = mn == -INFINITY ? 0.f : mn;
         const float alpha = ex2(m - b);
         const float pt = ex2(x - b);
-        lpart = lpart * alpha + pt;
+        lsum = lsum * alpha + pt;
         m = mn;
         {
             const float a = pt * 448.f;
             const uint32_t hi = tc::e4m3_code(a);
             const uint32_t lo = tc::e4m3_code(a - tc::e4m3_value(hi));
-            pmat[tc::sw128(0, tid)] = (uint8_t)hi;
-            pmat[tc::sw128(1, tid)] = (uint8_t)lo;
+            pmat[tc::sw128(2 * warp, tid)] = (uint8_t)hi;
+            pmat[tc::sw128(2 * warp + 1, tid)] = (uint8_t)lo;
+        }
+        if (lane == 0) red[(i & 1) * 4 + warp] = alpha;
+        // V rows past the context inside the last 32-token group may hold any
+        // code (NaN included) and would meet a zero weight: the warp owning
+        // those tokens clears them (the tile's copies are complete: S^T(i)
+        // was issued after them).
+        if (valid < vrows && warp == (valid >> 5)) {
+            uint8_t* vt = smem + st * C::kStageBytes + kTcTileBytes;
+            for (int idx = lane; idx < (vrows - valid) * 8; idx += 32)
+                *reinterpret_cast<uint4*>(vt + (valid + idx / 8) * 128 + (idx % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
         fence_proxy_async();
         tc::fence_before_sync();
         __syncthreads();
-        // O^T = V^T P^T over the tile's 32-token groups that hold tokens
+        // O^T(i), then S^T(i+1) behind it
         if (tid == 0) {
             tc::fence_after_sync();
             for (int kk = 0; kk < vrows / 32; ++kk)
                 tc::mma_f8f6f4(tmem + kTcColsO, tc::smem_desc_sw128(vaddr + kk * 4096, 16, 1024),
                                tc::smem_desc_sw128(paddr + kk * 32, 16, 1024), kIdO, kk > 0);
-            tc::commit(mbar);
+            tc::commit(obar);
+            if (STAGES > 1 && i + 1 < ntiles) ok = issue_s(i + 1);
         }
-        ok = mbar_wait(mbar, mphase);
-        mphase ^= 1;
-        if (!__syncthreads_and(ok ? 1 : 0)) break;
+        const bool ook = mbar_wait(obar, oph);
+        oph ^= 1;
+        if (!__syncthreads_and(ook ? 1 : 0)) { ok = false; break; }
         tc::fence_after_sync();
-        float d0, d1;
-        tc::ld_x2(tmem + t_lane + kTcColsO, d0, d1);
-        o = o * alpha + (d0 + d1);
+        {
+            uint32_t c[8];
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                         : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3]), "=r"(c[4]), "=r"(c[5]), "=r"(c[6]),
+                           "=r"(c[7])
+                         : "r"(tmem + t_lane + kTcColsO));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+            for (int w = 0; w < 4; ++w)
+                o[w] = o[w] * red[(i & 1) * 4 + w] + (__uint_as_float(c[2 * w]) + __uint_as_float(c[2 * w + 1]));
+        }
         tc::fence_before_sync();
-        __syncthreads();  // the stage, S, O and P are free for the next tile
-        if (warp == 0 && i + STAGES < ntiles) issue(i + STAGES);
+        // the stage of tile i is free (O^T(i) has completed): refill it
+        if (warp == 0 && i + STAGES < ntiles) issue_tma(i + STAGES);
+        if (STAGES == 1 && tid == 0 && i + 1 < ntiles) ok = issue_s(i + 1);
     }
 
     if (i < ntiles) {  // gave up: let the copies and MMAs in flight finish (bounded), then leave
         if (tid == 0) {
-            tc::commit(mbar);
-            mbar_wait(mbar, mphase);
-            for (int k = i; k < ntiles && k < i + STAGES; ++k) mbar_wait(bar0 + 8 * (k % STAGES), (k / STAGES) & 1);
+            tc::commit(obar);
+            mbar_wait(obar, oph);
+            for (int k = i; k < issued; ++k) mbar_wait(bar0 + 8 * (k % STAGES), (k / STAGES) & 1);
         }
         tc::fence_before_sync();
         __syncthreads();
@@ -320,22 +344,32 @@ __global__ void __launch_bounds__(128, 3) paged_attn_fp8_tc_kernel(const AttnPar
         return;
     }
 
-    // ---- sum of the weights, output
+    // ---- merge the four warps' parts (as split-K partials), output
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) lpart += __shfl_xor_sync(0xffffffffu, lpart, off);
-    if (lane == 0) red[warp] = lpart;
+    for (int off = 16; off > 0; off >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, off);
+    if (lane == 0) {
+        red[8 + warp] = m;
+        red[12 + warp] = lsum;
+    }
     tc::fence_before_sync();
     __syncthreads();
-    const float l = (red[0] + red[1]) + (red[2] + red[3]);
     if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)kTcCols));
-    const float ov = o * (p.v_scale / 448.f);
+    const float M = fmaxf(fmaxf(red[8], red[9]), fmaxf(red[10], red[11]));
+    float ov = 0.f, l = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const float f = ex2(red[8 + w] - M);  // 0 for a warp that saw no token
+        ov += f * o[w];
+        l += f * red[12 + w];
+    }
+    ov *= p.v_scale / 448.f;
     const int64_t row = (int64_t)s * p.Hq + h;
     if (u.direct) {
         reinterpret_cast<To*>(p.out)[row * D + tid] = static_cast<To>(ov / l);
     } else {
         const int64_t idx = row * p.maxP + u.slot;
         p.ws_o[idx * D + tid] = ov;
-        if (tid == 0) *reinterpret_cast<float2*>(p.ws_ml + idx * 2) = make_float2(m, l);
+        if (tid == 0) *reinterpret_cast<float2*>(p.ws_ml + idx * 2) = make_float2(M, l);
     }
 }
 
