@@ -30,15 +30,19 @@ def _stale() -> bool:
     return any(os.path.getmtime(f) > t for f in srcs)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
+def build(force: bool = False, verbose: bool = False, defines=(), out: str = None) -> str:
+    """Build the library (when stale, or always with force).  ``defines``
+    (e.g. ["PKV_FP8_TC=1"]) select build-time options; ``out`` puts such a
+    variant at another path, leaving the default library alone."""
+    lib = out or LIB
+    if not force and out is None and not defines and not _stale():
         return LIB
-    tmp = LIB + ".tmp%d" % os.getpid()
-    cmd = [NVCC] + FLAGS + (["-Xptxas", "-v"] if verbose else []) + \
+    tmp = lib + ".tmp%d" % os.getpid()
+    cmd = [NVCC] + FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-D" + d for d in defines] + \
         [os.path.join(CSRC, f) for f in SOURCES] + ["-o", tmp]
     subprocess.check_call(cmd)
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
