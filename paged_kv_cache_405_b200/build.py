@@ -46,4 +46,11 @@ def build(force: bool = False, verbose: bool = False, defines=(), out: str = Non
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    # python build.py [--force] [-v] [-D NAME=VALUE ...] [-o PATH]
+    args, defines, out = sys.argv[1:], [], None
+    for i, a in enumerate(args):
+        if a == "-D":
+            defines.append(args[i + 1])
+        elif a == "-o":
+            out = args[i + 1]
+    print(build(force="--force" in args, verbose="-v" in args, defines=defines, out=out))
