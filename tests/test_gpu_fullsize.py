@@ -19,12 +19,12 @@ from gpu_helpers import TOL, max_err
 
 pytestmark = pytest.mark.gpu
 
-WORKLOADS = ["llama7b", "llama13b_prefix", "llama3_gqa_bs16", "llama3_gqa_bs32", "longctx_beam", "spec_verify",
+WORKLOADS = ["tiny", "llama7b", "llama13b_prefix", "llama3_gqa_bs16", "llama3_gqa_bs32", "longctx_beam", "spec_verify",
              "llama7b_fp8", "llama3_gqa_fp8"]
 
 
 def _bits(t: torch.Tensor) -> torch.Tensor:
-    return t.view(torch.uint8) if t.dtype == torch.uint8 else t.view(torch.int16)
+    return t.view({1: torch.uint8, 2: torch.int16, 4: torch.int32}[t.element_size()])
 
 
 @pytest.mark.parametrize("cfg", WORKLOADS)
