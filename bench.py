@@ -370,6 +370,8 @@ def workload_shape(args, name=None):
     shape = synth.CONFIGS[args.config if name is None else name]
     if args.batch:
         shape = synth.shrink(shape, S=args.batch)
+    if getattr(args, "prefix", 0) and shape.prefix and name is None:
+        shape = synth.shrink(shape, prefix=args.prefix)
     # room in every table and in the pool for the tokens the run appends
     grow = (max(args.warmup, 10) + args.steps + 8) * max(1, shape.chunk)
     if grow > shape.reserve_tokens:
@@ -382,7 +384,9 @@ def workload_config(name, shape, batch, args, world) -> dict:
     L2 is handled.  Both arms build it from the same seeded batch, so the
     reference arm's line names exactly the workload this arm times."""
     pool_gb = 2 * batch.k_pool.numel() * batch.k_pool.element_size() / 1e9
-    return {"workload": name + ("" if not args.batch else "@batch%d" % args.batch),
+    tag = ("" if not args.batch else "@batch%d" % args.batch) + \
+        ("" if not (getattr(args, "prefix", 0) and shape.prefix) else "@prefix%d" % shape.prefix)
+    return {"workload": name + tag,
             "description": shape.description, "batch": shape.S,
             "q_heads": shape.Hq, "kv_heads": shape.Hkv, "head_dim": shape.D, "block_size": shape.bs,
             "kv_dtype": "e4m3" if shape.kv_fp8 else shape.dtype,
@@ -795,6 +799,8 @@ def main(argv=None):
                     help="split-K partition in tokens (0: the workload's, else the library's choice)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch size (small cases for profiling)")
+    ap.add_argument("--prefix", type=int, default=0,
+                    help="shared-prompt length of a shared-prefix workload (0: the workload's own)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg from host buffers")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle sample length (all cores)")

@@ -15,7 +15,7 @@ INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 
 SOURCES = ["pagedkv.cu", "allocator.cpp"]
-DEPS = SOURCES + ["common.cuh", "attention_common.cuh", "attention_simt.cuh", "attention_mma.cuh", "attention_fp8.cuh", "attention_fp8_tc.cuh",
+DEPS = SOURCES + ["common.cuh", "attention_common.cuh", "attention_simt.cuh", "attention_mma.cuh", "attention_fp8.cuh", "attention_fp8_tc.cuh", "prefix_tc.cuh",
                   "kv_append.cuh", "block_copy.cuh", "reduce.cuh"]
 
 FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-Werror", "all-warnings",

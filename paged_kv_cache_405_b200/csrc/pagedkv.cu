@@ -16,6 +16,7 @@
 #include "../../include/pagedkv.h"
 #include "attention_fp8.cuh"
 #include "attention_fp8_tc.cuh"
+#include "prefix_tc.cuh"
 #include "attention_mma.cuh"
 #include "attention_simt.cuh"
 #include "block_copy.cuh"
@@ -229,6 +230,22 @@ static cudaError_t launch_mma(const pkv::AttnParams& p, dim3 grid, const CUtenso
     return launch_k(k, grid, dim3(kMmaWarps * 32), C::kSmemBytes, st, p, mk, mv);
 }
 
+// Shared-prefix pass at head_dim 128 on tcgen05 (build-time switch).
+#ifndef PKV_PREFIX_TC
+#define PKV_PREFIX_TC 0
+#endif
+
+template <typename T>
+static cudaError_t launch_prefix_tc(const pkv::AttnParams& p, int npre, const CUtensorMap& mk, const CUtensorMap& mv,
+                                    cudaStream_t st) {
+    using C = pkv::PrefixTcCfg;
+    auto k = pkv::prefix_attn_tc_kernel<T>;
+    static cudaError_t attr = set_smem(k, C::kSmemBytes);
+    if (attr != cudaSuccess) return attr;
+    const dim3 grid((p.max_group_size * p.G + 127) / 128, npre, p.num_groups * p.Hkv);
+    return launch_k(k, grid, dim3(128), C::kSmemBytes, st, p, mk, mv);
+}
+
 template <typename T, int D>
 static cudaError_t launch_prefix(const pkv::AttnParams& p, dim3 grid, const CUtensorMap& mk, const CUtensorMap& mv,
                                  cudaStream_t st) {
@@ -379,7 +396,9 @@ static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int npart
             if (ss != nullptr && cudaEventRecord(ss->fork, st) == cudaSuccess &&
                 cudaStreamWaitEvent(ss->stream, ss->fork, 0) == cudaSuccess)
                 ps = ss->stream;
-            e = D == 64 ? launch_prefix<T, 64>(p, grid, *mk, *mv, ps) : launch_prefix<T, 128>(p, grid, *mk, *mv, ps);
+            e = D == 64            ? launch_prefix<T, 64>(p, grid, *mk, *mv, ps)
+                : PKV_PREFIX_TC != 0 ? launch_prefix_tc<T>(p, npre, *mk, *mv, ps)
+                                     : launch_prefix<T, 128>(p, grid, *mk, *mv, ps);
             if (e == cudaSuccess) e = decode_pass<T>(p, D, nparts, use_mma, mk, mv, st);
             if (ps != st) {  // join, whatever happened above
                 const cudaError_t j = cudaEventRecord(ss->join, ps);

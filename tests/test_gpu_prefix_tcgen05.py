@@ -1,0 +1,28 @@
+"""The shared-prefix pass built for the 5th-generation tensor cores
+(tcgen05.mma kind::f16, 128 queries x 128 shared tokens per product,
+accumulators in tensor memory; build option PKV_PREFIX_TC=1) against the
+oracle: the library is built with the option into a temporary file and the
+shared-prefix parity tests run through it in a child process (the library
+is chosen when the binding is imported)."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def test_tcgen05_prefix_pass_matches_oracle(tmp_path):
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("_pkv_build", os.path.join(ROOT, "paged_kv_cache_405_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    lib = mod.build(defines=["PKV_PREFIX_TC=1"], out=str(tmp_path / "libpagedkv_prefix_tcgen05.so"))
+    env = dict(os.environ, PKV_LIBRARY=lib)
+    r = subprocess.run([sys.executable, "-m", "pytest", "tests/test_gpu_shared_prefix.py", "tests/test_gpu_prefix_cache.py",
+                        "-q", "-p", "no:cacheprovider"], cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
+    assert " passed" in r.stdout and "failed" not in r.stdout
