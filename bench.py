@@ -370,7 +370,8 @@ def workload_shape(args, name=None):
     shape = synth.CONFIGS[args.config if name is None else name]
     if args.batch:
         shape = synth.shrink(shape, S=args.batch)
-    if getattr(args, "prefix", 0) and shape.prefix and name is None:
+    # --prefix overrides the shared-prompt length of the headline workload only
+    if getattr(args, "prefix", 0) and shape.prefix and (name is None or name == args.config):
         shape = synth.shrink(shape, prefix=args.prefix)
     # room in every table and in the pool for the tokens the run appends
     grow = (max(args.warmup, 10) + args.steps + 8) * max(1, shape.chunk)

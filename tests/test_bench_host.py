@@ -238,3 +238,13 @@ def test_allocator_bench_line():
     assert 0.5 < d["hit_rate"] <= 1.0 and 0.5 < d["prefill_tokens_skipped_frac"] <= 1.0
     assert d["host_us_per_call"] > 0 and d["calls"] > 0
     assert d["oracle"]["same_counters_on_sample"] is True
+
+
+def test_prefix_override_reaches_the_headline_workload_only():
+    import argparse
+    ns = argparse.Namespace(config="llama13b_prefix", batch=0, prefix=4096, warmup=3, steps=5, targets="")
+    assert bench.workload_shape(ns).prefix == 4096
+    assert bench.workload_shape(ns, "llama13b_prefix").prefix == 4096      # the headline, named as measured
+    ns2 = argparse.Namespace(config="llama3_gqa_bs16", batch=0, prefix=4096, warmup=3, steps=5, targets="")
+    assert bench.workload_shape(ns2, "llama13b_prefix").prefix == synth.CONFIGS["llama13b_prefix"].prefix
+    assert bench.workload_shape(ns2).prefix == 0                            # no shared prompt to override
