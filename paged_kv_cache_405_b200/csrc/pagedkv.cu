@@ -235,15 +235,24 @@ static cudaError_t launch_mma(const pkv::AttnParams& p, dim3 grid, const CUtenso
 #define PKV_PREFIX_TC 0
 #endif
 
+template <typename T, int QT, int KS, int VS>
+static cudaError_t launch_prefix_tc_q(const pkv::AttnParams& p, int npre, const CUtensorMap& mk, const CUtensorMap& mv,
+                                      cudaStream_t st) {
+    using C = pkv::PrefixTcCfg<QT, KS, VS>;
+    auto k = pkv::prefix_attn_tc_kernel<T, QT, KS, VS>;
+    static cudaError_t attr = set_smem(k, C::kSmemBytes);
+    if (attr != cudaSuccess) return attr;
+    const int rows = p.max_group_size * p.G;
+    const dim3 grid((rows + 128 * QT - 1) / (128 * QT), npre, p.num_groups * p.Hkv);
+    return launch_k(k, grid, dim3(C::kThreads), C::kSmemBytes, st, p, mk, mv);
+}
+
+// Groups of more than 128 rows: two Q tiles per CTA share every K/V tile.
 template <typename T>
 static cudaError_t launch_prefix_tc(const pkv::AttnParams& p, int npre, const CUtensorMap& mk, const CUtensorMap& mv,
                                     cudaStream_t st) {
-    using C = pkv::PrefixTcCfg;
-    auto k = pkv::prefix_attn_tc_kernel<T>;
-    static cudaError_t attr = set_smem(k, C::kSmemBytes);
-    if (attr != cudaSuccess) return attr;
-    const dim3 grid((p.max_group_size * p.G + 127) / 128, npre, p.num_groups * p.Hkv);
-    return launch_k(k, grid, dim3(128), C::kSmemBytes, st, p, mk, mv);
+    return p.max_group_size * p.G > 128 ? launch_prefix_tc_q<T, 2, 4, 4>(p, npre, mk, mv, st)
+                                        : launch_prefix_tc_q<T, 1, 2, 2>(p, npre, mk, mv, st);
 }
 
 template <typename T, int D>

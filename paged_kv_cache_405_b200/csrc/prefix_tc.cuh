@@ -6,36 +6,46 @@
 // system prompt stored once: openeuler.csdn.net PagedAttention explainer 6.1;
 // aiknowledge.cn "2.2 PagedAttention 与 KV Cache 分页管理" 2.2.3) attend to
 // those shared tokens, one split-K partial (o, m, l) per partition of them,
-// merged with each sequence's own partitions by the reduce kernel.  Here a
-// CTA of four warps takes 128 query rows of one (group, kv head, partition)
-// -- a real dense contraction: every shared K/V tile meets 128 queries.
+// merged with each sequence's own partitions by the reduce kernel.  Here one
+// CTA takes QT tiles of 128 query rows of one (group, kv head, partition) --
+// a real dense contraction: every shared K/V tile meets 128 * QT queries.
 //
-// Per 128-token tile of the shared run (thread t owns query row t = TMEM lane t):
-//   S = Q K^T   M = 128 rows, N = 128 tokens, K = 128 head-dim elements (8
+// Per 64-token tile j of the partition and Q tile q (thread t of softmax
+// warpgroup q owns query row t = TMEM lane t):
+//   S = Q K^T   M = 128 rows, N = 64 tokens, K = 128 head-dim elements (8
 //               MMAs of 16).  A = Q (built in shared memory from the rows'
 //               query vectors, K-major, 128-byte swizzle, two 64-element
-//               column blocks); B = the K tile as loaded by TMA (K-major, the
-//               same two blocks).  Two tiles at a time (TMEM columns 0-255).
-//   softmax     each thread reads its row of S from TMEM twice: for the
-//               maximum over the two tiles, then to write exp2(s - m) as P
-//               (the pool's element type) into shared memory (K-major, the
-//               A operand of the next product).
+//               column blocks); B = the K tile as TMA loads it (K-major, the
+//               same two blocks).  S goes to one of two TMEM buffers, so the
+//               next tile's S is computed while this one's softmax runs.
+//   softmax     the thread reads its 64 scores and writes P = exp2(s - m) in
+//               the pool's element type back over them in tensor memory (two
+//               values per 32-bit column).  m is a reference maximum: it
+//               moves (and O and l are rescaled by exp2(m_old - m_new)) only
+//               when a tile's maximum exceeds it by more than 8, so P stays
+//               below 2^8 and O is rarely touched; o, l and m stay one
+//               consistent partial, whose value is the softmax's exactly.
 //   O += P V    M = 128 rows, N = 128 head-dim elements, K = tokens (16 per
-//               MMA).  B = the V tile read MN-major (a token row of 64
-//               elements per 128-byte block, the two blocks 16 KB apart).  O
-//               stays in TMEM (columns 256-383) across tiles; when a pair
-//               of tiles raises a row's maximum, the row is rescaled in TMEM
-//               before the pair's products are added.
+//               MMA).  A = P read from tensor memory; B = the V tile read
+//               MN-major (a token row of 64 elements per 128-byte row, the
+//               two head-dim blocks kHalf bytes apart).  O stays in TMEM.
 // Rows are (sequence first + r / G, query head g*G + r % G), as in the mma.sync
 // pass; rows whose sequence does not take the group's prefix result (see
 // group_members_kernel) get zero queries and no output.
 //
-// One thread issues the TMA copies and the MMAs; completions arrive on
-// mbarriers; every wait is bounded in time, and on a give-up the CTA records
-// PKV_DEVERR_TIMEOUT, waits (bounded) for its copies and MMAs in flight,
-// frees its tensor memory and returns.  Shared memory (about 225 KB) allows
-// one CTA per SM, and a CTA takes 512 TMEM columns, so an allocation never
-// waits on another CTA of this kernel.
+// Warp roles: warps 0 .. 4*QT-1 are the softmax warpgroups (warp w reads TMEM
+// lanes 32*(w % 4) ..), then one warp issues the K copies, one the V copies
+// (each into its own ring of KS / VS tiles, refilled as the MMAs release
+// slots), and lane 0 of the last warp issues every MMA.  MMAs and copies
+// complete on mbarriers.  Every wait is bounded in time; a give-up records
+// PKV_DEVERR_TIMEOUT and raises a CTA-wide abort flag that every other wait
+// also polls; then each role waits (bounded) for what it has in flight
+// (MMAs, copies), tensor memory is freed and the CTA returns.
+//
+// Sizes: QT = 2 (256 rows): 192 KB of shared memory, 512 TMEM columns, one
+// CTA per SM.  QT = 1: 96 KB, 256 columns, two CTAs per SM.  Either way the
+// CTAs an SM can hold never ask for more than its 512 columns, so an
+// allocation never waits on another CTA of this kernel.
 #pragma once
 #include "attention_fp8_tc.cuh"
 
@@ -43,19 +53,20 @@ namespace pkv {
 
 namespace tc {
 
-// Instruction descriptor of kind::f16: T x T -> F32, M = 128, N = 128;
+// Instruction descriptor of kind::f16: T x T -> F32, M = 128, N = n;
 // b_mn: B read MN-major.  T = bf16 (format 1) or f16 (format 0).
 template <typename T>
-__host__ __device__ constexpr uint32_t idesc_f16_m128_n128(bool b_mn) {
-    constexpr uint32_t fmt = std::is_same<T, __half>::value ? 0u : 1u;
-    return (1u << 4)                   // D format F32
-           | (fmt << 7) | (fmt << 10)  // A, B format
-           | (0u << 15)                // A K-major
-           | ((b_mn ? 1u : 0u) << 16)  // B major
-           | ((128u >> 3) << 17)       // N / 8
-           | ((128u >> 4) << 24);      // M / 16
+__host__ __device__ constexpr uint32_t idesc_f16_m128(uint32_t n, bool b_mn) {
+    return (1u << 4)                                             // D format F32
+           | ((std::is_same<T, __half>::value ? 0u : 1u) << 7)   // A format
+           | ((std::is_same<T, __half>::value ? 0u : 1u) << 10)  // B format
+           | (0u << 15)                                          // A K-major
+           | ((b_mn ? 1u : 0u) << 16)                            // B major
+           | ((n >> 3) << 17)                                    // N / 8
+           | ((128u >> 4) << 24);                                // M / 16
 }
 
+// D (+)= A B, A and B from shared memory.
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                         bool accumulate) {
     asm volatile(
@@ -67,64 +78,121 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64
         : "memory");
 }
 
-// 32 consecutive columns of this warp's 32 lanes (thread i: lane base + i).
-__device__ __forceinline__ void ld_x32(uint32_t taddr, float (&v)[32]) {
-    uint32_t r[32];
+// D (+)= A B, A from tensor memory (lane = row, two 16-bit elements per
+// 32-bit column), B from shared memory.
+__device__ __forceinline__ void mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                               bool accumulate) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void st_x32(uint32_t taddr, const float (&v)[32]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
-        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
-        ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-        "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])),
-        "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-        "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-        "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
-        "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
-        "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
-        "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
-        "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
-        "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        :
+        : "r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u)
         : "memory");
 }
+
+#define PKV_TO8(b)                                                                                            \
+    "=r"(r[b]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3]), "=r"(r[b + 4]), "=r"(r[b + 5]), "=r"(r[b + 6]), \
+        "=r"(r[b + 7])
+#define PKV_TI8(b) \
+    "r"(v[b]), "r"(v[b + 1]), "r"(v[b + 2]), "r"(v[b + 3]), "r"(v[b + 4]), "r"(v[b + 5]), "r"(v[b + 6]), "r"(v[b + 7])
+
+// Columns c .. c+31 (c+63) of this warp's 32 lanes (thread i of the warp: lane
+// base + i); the values are complete when the call returns (the wait is in
+// the same asm statement).
+__device__ __forceinline__ void ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "{\n\ttcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n\t}"
+        : PKV_TO8(0), PKV_TO8(8), PKV_TO8(16), PKV_TO8(24)
+        : "r"(taddr)
+        : "memory");
+}
+
+__device__ __forceinline__ void ld_x64(uint32_t taddr, uint32_t (&r)[64]) {
+    asm volatile(
+        "{\n\ttcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, "
+        "%35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, "
+        "%56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;\n\t}"
+        : PKV_TO8(0), PKV_TO8(8), PKV_TO8(16), PKV_TO8(24), PKV_TO8(32), PKV_TO8(40), PKV_TO8(48), PKV_TO8(56)
+        : "r"(taddr)
+        : "memory");
+}
+
+// Store 32 columns of this warp's lanes; written when the call returns.
+__device__ __forceinline__ void st_x32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "{\n\ttcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};\n\t"
+        "tcgen05.wait::st.sync.aligned;\n\t}"
+        :
+        : "r"(taddr), PKV_TI8(0), PKV_TI8(8), PKV_TI8(16), PKV_TI8(24)
+        : "memory");
+}
+#undef PKV_TO8
+#undef PKV_TI8
 
 }  // namespace tc
 
 // Shared memory of the pass (offsets from a 1024-byte aligned base).
+template <int QT, int KS, int VS>
 struct PrefixTcCfg {
-    static constexpr int kBlk = 128 * 128;           // one [128 rows x 128 bytes] swizzled block
-    static constexpr int kQOff = 0;                  // Q: 2 blocks (head-dim 0-63, 64-127)
-    static constexpr int kKOff = kQOff + 2 * kBlk;   // K ring: 2 tiles x 2 blocks
-    static constexpr int kVOff = kKOff + 4 * kBlk;   // V ring: 2 tiles x 2 blocks
-    static constexpr int kPOff = kVOff + 4 * kBlk;   // P: 2 tiles x 2 blocks (tokens 0-63, 64-127)
-    static constexpr int kBarOff = kPOff + 4 * kBlk; // K full x2, V full x2, S done, O done
-    static constexpr int kTmemOff = kBarOff + 8 * 6;
-    static constexpr int kSmemBytes = 1024 + kTmemOff + 16;
-    static constexpr int kCols = 512;                // S pair: 0-255, O: 256-383
-    static constexpr int kColS = 0, kColO = 256;
+    static constexpr int kTok = 64;            // tokens per K / V tile
+    static constexpr int kQBlk = 128 * 128;    // 128 query rows x 64 head-dim elements (16 KB)
+    static constexpr int kHalf = kTok * 128;   // 64 token rows x 64 head-dim elements (8 KB)
+    static constexpr int kTile = 2 * kHalf;    // one K or V tile, both head-dim halves
+    static constexpr int kQOff = 0;            // Q tile q: blocks 2q, 2q+1
+    static constexpr int kKOff = kQOff + QT * 2 * kQBlk;
+    static constexpr int kVOff = kKOff + KS * kTile;
+    static constexpr int kBarOff = kVOff + VS * kTile;
+    // kfull[KS], kempty[KS], vfull[VS], vempty[VS]; per Q tile sfull[2],
+    // pfull[2], obar, ofin; drain
+    static constexpr int kBars = 2 * KS + 2 * VS + 6 * QT + 1;
+    static constexpr int kTmemOff = kBarOff + 8 * kBars;
+    static constexpr int kAbortOff = kTmemOff + 4;
+    static constexpr int kSmemBytes = 1024 + kAbortOff + 4;
+    static constexpr int kCols = 256 * QT;     // per Q tile: S / P buffers at 0 and 64, O at 128-255
+    static constexpr int kWarps = 4 * QT + 3;  // softmax warpgroups, K copies, V copies, MMA
+    static constexpr int kThreads = 32 * kWarps;
+    static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+    static_assert(QT == 2 || 2 * (kSmemBytes + 1024) <= 228 * 1024, "two CTAs per SM at QT = 1");
+    static_assert(3 * (kSmemBytes + 1024) > 228 * 1024, "at most two CTAs per SM (tensor-memory columns)");
+    static_assert(QT == 1 || 2 * (kSmemBytes + 1024) > 228 * 1024, "one CTA per SM at QT = 2");
 };
 
-template <typename T>
-__global__ void __launch_bounds__(128, 1) prefix_attn_tc_kernel(const AttnParams p,
-                                                                const __grid_constant__ CUtensorMap tmK,
-                                                                const __grid_constant__ CUtensorMap tmV) {
-    using C = PrefixTcCfg;
-    constexpr int D = 128, TILE = 128;
+// A reference maximum moves only when a tile's maximum (log2 units) exceeds it
+// by more than this, so softmax weights stay below 2^8.
+constexpr float kPrefixRescaleLog2 = 8.f;
+
+// Bounded wait that also gives up once another role of the CTA has raised
+// the abort flag.
+__device__ __forceinline__ bool mbar_wait_or_abort(uint32_t bar, uint32_t parity, volatile int* abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = global_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (*abort_flag) return false;
+        if (global_ns() - t0 > kWaitLimitNs) {
+            flag_error(8u /* PKV_DEVERR_TIMEOUT */);
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+template <typename T, int QT, int KS, int VS>
+__global__ void __launch_bounds__(PrefixTcCfg<QT, KS, VS>::kThreads, QT == 1 ? 2 : 1)
+    prefix_attn_tc_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV) {
+    using C = PrefixTcCfg<QT, KS, VS>;
+    constexpr int D = 128, TOK = C::kTok;
+    constexpr int kWarpK = 4 * QT, kWarpV = 4 * QT + 1, kWarpM = 4 * QT + 2;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int tile_r = blockIdx.x;  // 128-row tile of the group
+    const int tile_r = blockIdx.x;  // 128*QT-row tile of the group
     const int pp = blockIdx.y;      // partition of the shared tokens
     const int gi = blockIdx.z / p.Hkv;
     const int g = blockIdx.z - gi * p.Hkv;
@@ -138,44 +206,72 @@ __global__ void __launch_bounds__(128, 1) prefix_attn_tc_kernel(const AttnParams
         last = first + p.max_group_size;
     }
     const int rows = (last - first) * G;
-    if (tile_r * TILE >= rows) return;  // CTA-uniform
+    const int row0 = tile_r * 128 * QT;
+    if (row0 >= rows) return;  // CTA-uniform
+    const int nq = min(QT, (rows - row0 + 127) / 128);  // Q tiles holding rows
     const int shared = p.group_shared[gi];
     if (shared <= 0 || shared % p.bs != 0 || shared > p.max_len || shared > p.max_shared) return;
     const int t0 = pp * p.P;
     if (t0 >= shared) return;
-    const int t1 = min(shared, t0 + p.P);
-    const int ntiles = (t1 - t0 + TILE - 1) / TILE;
+    const int t1 = min(shared, t0 + p.P);  // t1 - t0: a multiple of 16, as block sizes are
+    const int n = (t1 - t0 + TOK - 1) / TOK;
 
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t kfull = sbase + C::kBarOff, vfull = kfull + 16, sbar = kfull + 32, obar = kfull + 40;
+    const uint32_t b_kfull = sbase + C::kBarOff, b_kempty = b_kfull + 8 * KS;
+    const uint32_t b_vfull = b_kempty + 8 * KS, b_vempty = b_vfull + 8 * VS;
+    const uint32_t b_q = b_vempty + 8 * VS;  // Q tile q at +48q: sfull[2], pfull[2], obar, ofin
+    const uint32_t b_drain = b_q + 48 * QT;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kTmemOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kAbortOff);
 
-    // this thread's query row
-    const int r = tile_r * TILE + tid;
-    const int s_r = first + (r < rows ? r / G : 0);
-    const bool live = r < rows && p.member[s_r].x == gi + 1;
-    const int h_r = g * G + (r < rows ? r % G : 0);
+    // softmax threads: this thread's query row
+    const bool is_soft = warp < 4 * QT;
+    const int q = warp >> 2;  // Q tile of a softmax thread
+    const int t = tid & 127;  // its row in the tile = its TMEM lane
+    const int r = row0 + q * 128 + t;
+    const bool inrow = is_soft && r < rows;
+    const int s_r = first + (inrow ? r / G : 0);
+    const int h_r = g * G + (inrow ? r % G : 0);
+    const bool live = inrow && p.member[s_r].x == gi + 1;
 
     // ---- set-up: tensor memory, barriers, Q
-    if (warp == 0) {
+    if (warp == kWarpM) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
                      "r"((uint32_t)C::kCols));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::);
     }
-    if (tid == 0) {
+    if (tid == kWarpK * 32) {
         prefetch_tensor_map(&tmK);
         prefetch_tensor_map(&tmV);
-        for (int i = 0; i < 6; ++i) mbar_init(kfull + 8 * i, 1);
+        for (int i = 0; i < KS; ++i) {
+            mbar_init(b_kfull + 8 * i, 1);
+            mbar_init(b_kempty + 8 * i, 1);
+        }
+        for (int i = 0; i < VS; ++i) {
+            mbar_init(b_vfull + 8 * i, 1);
+            mbar_init(b_vempty + 8 * i, 1);
+        }
+        for (int i = 0; i < QT; ++i) {
+            mbar_init(b_q + 48 * i, 1);
+            mbar_init(b_q + 48 * i + 8, 1);
+            mbar_init(b_q + 48 * i + 16, 128);  // every softmax thread of the Q tile
+            mbar_init(b_q + 48 * i + 24, 128);
+            mbar_init(b_q + 48 * i + 32, 1);
+            mbar_init(b_q + 48 * i + 40, 1);
+        }
+        mbar_init(b_drain, 1);
+        *abort_flag = 0;
         fence_barrier_init();
     }
-    {
+    if (is_soft && q < nq) {
         const uint4* qsrc = reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.q) +
                                                              ((int64_t)s_r * p.Hq + h_r) * D);
+        uint8_t* qrow = smem + C::kQOff + q * 2 * C::kQBlk + t * 128;
 #pragma unroll
         for (int c = 0; c < 16; ++c) {  // 16-byte chunk c: block c / 8, chunk c % 8 of the row
             const uint4 v = live ? qsrc[c] : make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(smem + C::kQOff + (c >> 3) * C::kBlk + tid * 128 + (((c & 7) ^ (tid & 7)) << 4)) = v;
+            *reinterpret_cast<uint4*>(qrow + (c >> 3) * C::kQBlk + (((c & 7) ^ (t & 7)) << 4)) = v;
         }
     }
     fence_proxy_async();
@@ -183,201 +279,187 @@ __global__ void __launch_bounds__(128, 1) prefix_attn_tc_kernel(const AttnParams
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_lane = (uint32_t)(warp * 32) << 16;
 
-    // ---- copies: tile i of K (V) into ring slot i % 2 of 2 blocks each; K and
-    // V walk the same block-table entries, each with its own window (warp 0)
-    const int jb0 = t0 / p.bs;
-    BlockWindow kwin, vwin;
-    if (warp == 0) {
-        kwin.init(p.block_tables + (int64_t)first * p.maxB, jb0, (t1 - 1) / p.bs - jb0 + 1, lane);
-        vwin = kwin;
-    }
-    int kiss = 0, viss = 0;  // tiles whose K / V copies were issued (warp 0), in order
-    auto issue = [&](int i, bool is_v, BlockWindow& win) {  // warp 0
-        const int tt0 = t0 + i * TILE;
-        const int nbox = min(TILE, t1 - tt0) / kTileTok;  // shared runs are whole 16-token boxes
-        const uint32_t bar = (is_v ? vfull : kfull) + 8 * (i & 1);
-        const uint32_t dst = sbase + (is_v ? C::kVOff : C::kKOff) + (i & 1) * 2 * C::kBlk;
+    int issued = 0;  // tiles whose copies this producer warp issued
+    if (warp == kWarpK || warp == kWarpV) {
+        // ---- copies: tile j into ring slot j % S, refilled once the MMAs
+        // that read the slot's previous tile have completed
+        const bool isv = warp == kWarpV;
+        const int S = isv ? VS : KS;
+        const uint32_t full = isv ? b_vfull : b_kfull, empty = isv ? b_vempty : b_kempty;
+        const uint32_t ring = sbase + (isv ? C::kVOff : C::kKOff);
+        const CUtensorMap* map = isv ? &tmV : &tmK;
+        const int jb0 = t0 / p.bs;
+        BlockWindow win;
+        win.init(p.block_tables + (int64_t)first * p.maxB, jb0, (t1 - 1) / p.bs - jb0 + 1, lane);
+        for (int j = 0; j < n; ++j) {
+            const int slot = j % S;
+            if (j >= S) {
+                bool w = true;
+                if (lane == 0) w = mbar_wait_or_abort(empty + 8 * slot, ((j / S) - 1) & 1, abort_flag);
+                if (!__shfl_sync(0xffffffffu, w ? 1 : 0, 0)) break;
+            }
+            const int tt0 = t0 + j * TOK;
+            const int nbox = min(TOK, t1 - tt0) / kTileTok;
+            const uint32_t dst = ring + slot * C::kTile, bar = full + 8 * slot;
+            if (lane == 0) mbar_arrive_expect_tx(bar, (uint32_t)(nbox * kTileTok * D * 2));
+            for (int b = 0; b < nbox; ++b) {
+                const int th = tt0 + b * kTileTok;
+                const int blk = win.get(th / p.bs - jb0, lane, p.NB);
+                if (lane == 0) {
+                    const int row = (blk * p.Hkv + g) * p.bs + (th % p.bs);
+                    tma_load_2d(dst + b * kTileTok * 128, map, 0, row, bar);
+                    tma_load_2d(dst + C::kHalf + b * kTileTok * 128, map, 64, row, bar);
+                }
+            }
+            issued = j + 1;
+        }
+    } else if (warp == kWarpM) {
+        // ---- MMAs (lane 0): S of tile j+1 goes in before O += P V of tile j
         if (lane == 0) {
-            fence_proxy_async();
-            mbar_arrive_expect_tx(bar, (uint32_t)(nbox * kTileTok * D * 2));
-        }
-        for (int j = 0; j < nbox; ++j) {
-            const int th = tt0 + j * kTileTok;
-            const int blk = win.get(th / p.bs - jb0, lane, p.NB);
-            if (lane == 0) {
-                const int row = (blk * p.Hkv + g) * p.bs + (th % p.bs);
-                const CUtensorMap* map = is_v ? &tmV : &tmK;
-                tma_load_2d(dst + j * kTileTok * 128, map, 0, row, bar);
-                tma_load_2d(dst + C::kBlk + j * kTileTok * 128, map, 64, row, bar);
-            }
-        }
-        if (is_v) viss = i + 1;
-        else kiss = i + 1;
-    };
-    if (warp == 0) {
-        for (int i = 0; i < ntiles && i < 2; ++i) issue(i, false, kwin);
-        for (int i = 0; i < ntiles && i < 2; ++i) issue(i, true, vwin);
-    }
-
-    constexpr uint32_t kIdS = tc::idesc_f16_m128_n128<T>(false);
-    constexpr uint32_t kIdO = tc::idesc_f16_m128_n128<T>(true);
-    const float sl2 = p.scale_log2;
-    float m = -INFINITY, l = 0.f;
-    uint32_t sph = 0, oph = 0;
-    bool ok = true, o_started = false;
-    int pair = 0;
-    for (int a = 0; a < ntiles; a += 2, ++pair) {
-        const int nt = min(2, ntiles - a);  // tiles of this pair
-        // S = Q K^T for the pair's tiles
-        if (tid == 0) {
-            for (int u = 0; u < nt && ok; ++u) {
-                const int i = a + u;
-                ok = mbar_wait(kfull + 8 * (i & 1), (i >> 1) & 1);
-                if (!ok) break;
+            constexpr uint32_t kIdS = tc::idesc_f16_m128<T>(64, false);
+            constexpr uint32_t kIdO = tc::idesc_f16_m128<T>(128, true);
+            auto issue_s = [&](int j) -> bool {
+                const int slot = j % KS;
+                if (!mbar_wait_or_abort(b_kfull + 8 * slot, (j / KS) & 1, abort_flag)) return false;
                 tc::fence_after_sync();
-                const uint32_t kb = sbase + C::kKOff + (i & 1) * 2 * C::kBlk;
+                const uint32_t kb = sbase + C::kKOff + slot * C::kTile;
+                for (int qq = 0; qq < nq; ++qq) {
+                    const uint32_t qb = sbase + C::kQOff + qq * 2 * C::kQBlk;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk)
-                    tc::mma_f16(tmem + C::kColS + u * TILE,
-                                tc::smem_desc_sw128(sbase + C::kQOff + (kk >> 2) * C::kBlk + (kk & 3) * 32, 16, 1024),
-                                tc::smem_desc_sw128(kb + (kk >> 2) * C::kBlk + (kk & 3) * 32, 16, 1024), kIdS, kk > 0);
+                    for (int kk = 0; kk < D / 16; ++kk)
+                        tc::mma_f16(tmem + qq * 256 + (j & 1) * 64,
+                                    tc::smem_desc_sw128(qb + (kk >> 2) * C::kQBlk + (kk & 3) * 32, 16, 1024),
+                                    tc::smem_desc_sw128(kb + (kk >> 2) * C::kHalf + (kk & 3) * 32, 16, 1024), kIdS,
+                                    kk > 0);
+                    tc::commit(b_q + 48 * qq + 8 * (j & 1));  // S of tile j ready
+                }
+                tc::commit(b_kempty + 8 * slot);  // K slot free
+                return true;
+            };
+            bool ok = issue_s(0);
+            for (int j = 0; ok && j < n; ++j) {
+                if (j + 1 < n && !(ok = issue_s(j + 1))) break;
+                const int slot = j % VS;
+                if (!(ok = mbar_wait_or_abort(b_vfull + 8 * slot, (j / VS) & 1, abort_flag))) break;
+                const int valid = min(TOK, t1 - (t0 + j * TOK));
+                const uint32_t vb = sbase + C::kVOff + slot * C::kTile;
+                for (int qq = 0; qq < nq; ++qq) {
+                    if (!(ok = mbar_wait_or_abort(b_q + 48 * qq + 16 + 8 * (j & 1), (j >> 1) & 1, abort_flag))) break;
+                    tc::fence_after_sync();
+                    for (int kk = 0; kk < valid / 16; ++kk)
+                        tc::mma_f16_tmem_a(tmem + qq * 256 + 128, tmem + qq * 256 + (j & 1) * 64 + kk * 8,
+                                           tc::smem_desc_sw128(vb + kk * 16 * 128, C::kHalf, 1024), kIdO,
+                                           j > 0 || kk > 0);
+                    tc::commit(b_q + 48 * qq + 32);  // O products of tile j done
+                }
+                if (!ok) break;
+                tc::commit(b_vempty + 8 * slot);  // V slot free
             }
-            if (ok) tc::commit(sbar);
+            if (ok)
+                for (int qq = 0; qq < nq; ++qq) tc::commit(b_q + 48 * qq + 40);  // O final
+            // every MMA issued, and so every arrival it owes, has completed
+            // before the CTA can leave (bounded)
+            tc::commit(b_drain);
+            mbar_wait(b_drain, 0);
         }
-        ok = ok && mbar_wait(sbar, sph);
-        sph ^= 1;
-        if (!__syncthreads_and(ok ? 1 : 0)) break;
-        tc::fence_after_sync();
-        // the pair's K slots are free: copy the next pair's K
-        if (warp == 0)
-            for (int u = 0; u < 2; ++u)
-                if (a + 2 + u < ntiles) issue(a + 2 + u, false, kwin);
-        // row maximum over the pair's valid tokens
-        float pm = -INFINITY;
-        for (int u = 0; u < nt; ++u) {
-            const int valid = min(TILE, t1 - (t0 + (a + u) * TILE));
-            for (int c = 0; c < TILE / 32; ++c) {
-                float v[32];
-                tc::ld_x32(tmem + t_lane + C::kColS + u * TILE + c * 32, v);
-#pragma unroll
-                for (int k = 0; k < 32; ++k)
-                    if (c * 32 + k < valid) pm = fmaxf(pm, v[k] * sl2);
+        __syncwarp();
+    } else if (q < nq) {
+        // ---- softmax of Q tile q: thread t owns row t (TMEM lane t)
+        const uint32_t tq = tmem + ((uint32_t)((warp & 3) * 32) << 16) + q * 256;
+        const uint32_t sfull = b_q + 48 * q, pfull = sfull + 16, obar = sfull + 32, ofin = sfull + 40;
+        const float sl2 = p.scale_log2;
+        float m = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n; ++j) {
+            const bool w = mbar_wait_or_abort(sfull + 8 * (j & 1), (j >> 1) & 1, abort_flag);
+            if (!__all_sync(0xffffffffu, w)) {
+                ok = false;
+                break;
             }
-        }
-        const float mn = fmaxf(m, pm);
-        const float alpha = ex2(m - mn);  // 0 on the first pair (m = -inf)
-        // the previous pair's O products read P and V: wait for them, then
-        // rescale the rows whose maximum rose, and refill the V slots
-        if (o_started) {
-            const bool ook = mbar_wait(obar, oph);
-            oph ^= 1;
-            if (!__syncthreads_and(ook ? 1 : 0)) { ok = false; break; }
             tc::fence_after_sync();
-            if (__any_sync(0xffffffffu, alpha != 1.f)) {
+            uint32_t sr[64];
+            tc::ld_x64(tq + (j & 1) * 64, sr);
+            const int valid = min(TOK, t1 - (t0 + j * TOK));
+            float x[64];
+            float mt = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < 64; ++k) {
+                x[k] = __uint_as_float(sr[k]) * sl2;
+                if (k < valid) mt = fmaxf(mt, x[k]);
+            }
+            const bool need = mt > m + kPrefixRescaleLog2;  // always on the first tile
+            const float mn = need ? mt : m;
+            const float alpha = ex2(m - mn);  // 1 when m stays; 0 on the first tile (m = -inf)
+            uint32_t pw[32];
+            float ls = 0.f;
+#pragma unroll
+            for (int k = 0; k < 64; k += 2) {
+                const float p0 = k < valid ? ex2(x[k] - mn) : 0.f;
+                const float p1 = k + 1 < valid ? ex2(x[k + 1] - mn) : 0.f;
+                ls += p0 + p1;
+                pw[k / 2] = Elt<T>::pack2(p0, p1);
+            }
+            if (j > 0 && __any_sync(0xffffffffu, need)) {
+                // the previous tile's O products must have landed before O is rescaled
+                const bool w2 = mbar_wait_or_abort(obar, (j - 1) & 1, abort_flag);
+                if (!__all_sync(0xffffffffu, w2)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+#pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
-                    float v[32];
-                    tc::ld_x32(tmem + t_lane + C::kColO + c * 32, v);
+                    uint32_t o[32];
+                    tc::ld_x32(tq + 128 + c * 32, o);
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) v[k] *= alpha;
-                    tc::st_x32(tmem + t_lane + C::kColO + c * 32, v);
-                }
-                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-            }
-            if (warp == 0)
-                for (int u = 0; u < nt; ++u) issue(a + u, true, vwin);
-        }
-        l *= alpha;
-        m = mn;
-        // P = exp2(s - m) in the pool's type, as the A operand of O += P V
-        for (int u = 0; u < nt; ++u) {
-            const int valid = min(TILE, t1 - (t0 + (a + u) * TILE));
-            uint8_t* pb = smem + C::kPOff + u * 2 * C::kBlk;
-            for (int c = 0; c < TILE / 32; ++c) {
-                float v[32];
-                tc::ld_x32(tmem + t_lane + C::kColS + u * TILE + c * 32, v);
-                uint32_t w[16];
-#pragma unroll
-                for (int k = 0; k < 32; k += 2) {
-                    const float p0 = c * 32 + k < valid ? ex2(v[k] * sl2 - mn) : 0.f;
-                    const float p1 = c * 32 + k + 1 < valid ? ex2(v[k + 1] * sl2 - mn) : 0.f;
-                    l += p0 + p1;
-                    w[k / 2] = Elt<T>::pack2(p0, p1);
-                }
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {  // tokens c*32 + q4*8 .. +7: block, chunk of the row
-                    const int tok = c * 32 + q4 * 8;
-                    *reinterpret_cast<uint4*>(pb + (tok >> 6) * C::kBlk + tid * 128 + ((((tok & 63) >> 3) ^ (tid & 7)) << 4)) =
-                        make_uint4(w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+                    for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+                    tc::st_x32(tq + 128 + c * 32, o);
                 }
             }
+            l = l * alpha + ls;
+            m = mn;
+            tc::st_x32(tq + (j & 1) * 64, pw);  // P over the scores it came from
+            tc::fence_before_sync();
+            mbar_arrive(pfull + 8 * (j & 1));
         }
-        fence_proxy_async();
-        tc::fence_before_sync();
-        __syncthreads();
-        // O += P V over the pair's valid tokens (16 per MMA)
-        if (tid == 0) {
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait_or_abort(ofin, 0, abort_flag));
+        if (ok) {
+            // ---- the row's partial: o (unnormalised, at reference maximum m), m, l
             tc::fence_after_sync();
-            for (int u = 0; u < nt && ok; ++u) {
-                const int i = a + u;
-                const int valid = min(TILE, t1 - (t0 + i * TILE));
-                ok = mbar_wait(vfull + 8 * (i & 1), (i >> 1) & 1);
-                if (!ok) break;
-                tc::fence_after_sync();
-                const uint32_t vb = sbase + C::kVOff + (i & 1) * 2 * C::kBlk;
-                const uint32_t pbase = sbase + C::kPOff + u * 2 * C::kBlk;
-                for (int kk = 0; kk < valid / 16; ++kk) {
-                    tc::mma_f16(tmem + C::kColO,
-                                tc::smem_desc_sw128(pbase + (kk >> 2) * C::kBlk + (kk & 3) * 32, 16, 1024),
-                                tc::smem_desc_sw128(vb + kk * 16 * 128, C::kBlk, 1024), kIdO, o_started || kk > 0);
+            const int64_t idx = ((int64_t)s_r * p.Hq + h_r) * p.maxP + pp;
+            float* dst = p.ws_o + idx * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t o[32];
+                tc::ld_x32(tq + 128 + c * 32, o);
+                if (live) {
+#pragma unroll
+                    for (int k = 0; k < 32; k += 4)
+                        *reinterpret_cast<float4*>(dst + c * 32 + k) =
+                            make_float4(__uint_as_float(o[k]), __uint_as_float(o[k + 1]), __uint_as_float(o[k + 2]),
+                                        __uint_as_float(o[k + 3]));
                 }
-                o_started = true;
             }
-            if (ok) tc::commit(obar);
+            if (live) *reinterpret_cast<float2*>(p.ws_ml + idx * 2) = make_float2(m, l);
         }
-        o_started = true;  // every thread: the pair's products were issued (tid 0) or the CTA gives up below
-        ok = __syncthreads_and(ok ? 1 : 0) != 0;
-        if (!ok) break;
     }
 
-    bool done = ok;
-    if (done) {
-        done = mbar_wait(obar, oph);
-        done = __syncthreads_and(done ? 1 : 0) != 0;
+    // ---- teardown: after a give-up, the copies still in flight land first
+    // (bounded); the MMA warp has drained its MMAs above
+    __syncthreads();
+    if (*abort_flag && (warp == kWarpK || warp == kWarpV) && lane == 0) {
+        const int S = warp == kWarpV ? VS : KS;
+        const uint32_t full = warp == kWarpV ? b_vfull : b_kfull;
+        for (int j = max(0, issued - S); j < issued; ++j)  // the last tile issued into each slot
+            mbar_wait(full + 8 * (j % S), (j / S) & 1);
     }
-    if (!done) {  // gave up: let the copies and MMAs in flight finish (bounded), then leave
-        if (tid == 0) {
-            tc::commit(obar);
-            mbar_wait(obar, oph ^ 1);
-            mbar_wait(obar, oph);
-        }
-        if (warp == 0 && lane == 0) {
-            for (int i = 0; i < kiss; ++i) mbar_wait(kfull + 8 * (i & 1), (i >> 1) & 1);
-            for (int i = 0; i < viss; ++i) mbar_wait(vfull + 8 * (i & 1), (i >> 1) & 1);
-        }
-        tc::fence_before_sync();
-        __syncthreads();
-        if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::kCols));
-        return;
-    }
-    tc::fence_after_sync();
-    // ---- the row's partial: o (unnormalised, at maximum m), m, l
-    const int64_t idx = ((int64_t)s_r * p.Hq + h_r) * p.maxP + pp;
-    float* dst = p.ws_o + idx * D;
-    for (int c = 0; c < D / 32; ++c) {
-        float v[32];
-        tc::ld_x32(tmem + t_lane + C::kColO + c * 32, v);
-        if (live) {
-#pragma unroll
-            for (int k = 0; k < 32; k += 4)
-                *reinterpret_cast<float4*>(dst + c * 32 + k) = make_float4(v[k], v[k + 1], v[k + 2], v[k + 3]);
-        }
-    }
-    if (live) *reinterpret_cast<float2*>(p.ws_ml + idx * 2) = make_float2(m, l);
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::kCols));
+    if (warp == kWarpM) {
+        tc::fence_after_sync();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"((uint32_t)C::kCols));
+    }
 }
 
 }  // namespace pkv

@@ -1,9 +1,12 @@
 """The shared-prefix pass built for the 5th-generation tensor cores
-(tcgen05.mma kind::f16, 128 queries x 128 shared tokens per product,
-accumulators in tensor memory; build option PKV_PREFIX_TC=1) against the
-oracle: the library is built with the option into a temporary file and the
-shared-prefix parity tests run through it in a child process (the library
-is chosen when the binding is imported)."""
+(tcgen05.mma kind::f16, 128 queries x 64 shared tokens per product, P
+written back to tensor memory as the A operand of the V product; build option
+PKV_PREFIX_TC=1) against the oracle: the library is built with the option
+into a temporary file and the shared-prefix parity tests -- small groups
+(one 128-row query tile per CTA), groups of more than 128 rows (two tiles
+sharing every K/V tile), and the full-size shared-prompt decode step, 256
+rows per group -- run through it in a child process (the library is chosen
+when the binding is imported)."""
 import os
 import subprocess
 import sys
@@ -22,7 +25,8 @@ def test_tcgen05_prefix_pass_matches_oracle(tmp_path):
     spec.loader.exec_module(mod)
     lib = mod.build(defines=["PKV_PREFIX_TC=1"], out=str(tmp_path / "libpagedkv_prefix_tcgen05.so"))
     env = dict(os.environ, PKV_LIBRARY=lib)
-    r = subprocess.run([sys.executable, "-m", "pytest", "tests/test_gpu_shared_prefix.py", "tests/test_gpu_prefix_cache.py",
-                        "-q", "-p", "no:cacheprovider"], cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
+    files = ["tests/test_gpu_shared_prefix.py", "tests/test_gpu_prefix_cache.py", "tests/test_gpu_fullsize.py"]
+    r = subprocess.run([sys.executable, "-m", "pytest", *files, "-k", "not fullsize or llama13b_prefix", "-q",
+                        "-p", "no:cacheprovider"], cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-2000:]
     assert " passed" in r.stdout and "failed" not in r.stdout
