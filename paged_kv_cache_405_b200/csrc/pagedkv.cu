@@ -230,16 +230,17 @@ static cudaError_t launch_mma(const pkv::AttnParams& p, dim3 grid, const CUtenso
     return launch_k(k, grid, dim3(kMmaWarps * 32), C::kSmemBytes, st, p, mk, mv);
 }
 
-// Shared-prefix pass at head_dim 128 on tcgen05 (build-time switch).
+// Shared-prefix pass at head_dim 128: on tcgen05 (default), or with
+// PKV_PREFIX_TC=0 the mma.sync pass that head_dim 64 always uses.
 #ifndef PKV_PREFIX_TC
-#define PKV_PREFIX_TC 0
+#define PKV_PREFIX_TC 1
 #endif
 
-template <typename T, int QT, int KS, int VS>
+template <typename T, int QT>
 static cudaError_t launch_prefix_tc_q(const pkv::AttnParams& p, int npre, const CUtensorMap& mk, const CUtensorMap& mv,
                                       cudaStream_t st) {
-    using C = pkv::PrefixTcCfg<QT, KS, VS>;
-    auto k = pkv::prefix_attn_tc_kernel<T, QT, KS, VS>;
+    using C = pkv::PrefixTcCfg<QT>;
+    auto k = pkv::prefix_attn_tc_kernel<T, QT>;
     static cudaError_t attr = set_smem(k, C::kSmemBytes);
     if (attr != cudaSuccess) return attr;
     const int rows = p.max_group_size * p.G;
@@ -251,8 +252,8 @@ static cudaError_t launch_prefix_tc_q(const pkv::AttnParams& p, int npre, const 
 template <typename T>
 static cudaError_t launch_prefix_tc(const pkv::AttnParams& p, int npre, const CUtensorMap& mk, const CUtensorMap& mv,
                                     cudaStream_t st) {
-    return p.max_group_size * p.G > 128 ? launch_prefix_tc_q<T, 2, 4, 4>(p, npre, mk, mv, st)
-                                        : launch_prefix_tc_q<T, 1, 2, 2>(p, npre, mk, mv, st);
+    return p.max_group_size * p.G > 128 ? launch_prefix_tc_q<T, 2>(p, npre, mk, mv, st)
+                                        : launch_prefix_tc_q<T, 1>(p, npre, mk, mv, st);
 }
 
 template <typename T, int D>
