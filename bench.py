@@ -12,8 +12,11 @@ value  -- algorithmic bytes of the step (unique K/V bytes the attention must
           read, shared blocks counted once, plus q, out, tables, split-K
           workspace, appended and copied bytes) / device time, inputs already
           resident in HBM (the step's plan is made on the host beforehand).
-e2e    -- the same metric through DecodeSession.step: allocator on the host,
-          step inputs copied in from pinned host memory, output copied back.
+e2e    -- the same metric through DecodeSession.launch_step: allocator on the
+          host, every step's inputs copied in from pinned host memory and its
+          output copied back to pinned host memory and waited for, two steps
+          in flight (--e2e-in-flight; the line also carries the figure with
+          the host waiting for each output before the next step goes).
 
 The headline workload (``--config``, default ``llama3_gqa_bs16``: 128
 sequences x 8192 tokens, 32 query / 8 kv heads, the largest one-GPU decode
@@ -537,11 +540,18 @@ def measure_workload(name, args, world, rank, local, e2e=True):
     }
     res["e2e"] = None
     if e2e and not args.no_e2e:
-        wl2 = Workload(shape, shape.seed + rank, dev, args.partition_size)
         del wl, ss, plans, inputs, out
         torch.cuda.empty_cache()
-        res["e2e"] = run_e2e(args, wl2, world, rank, dev)
+        depth = max(1, args.e2e_in_flight)
+        wl2 = Workload(shape, shape.seed + rank, dev, args.partition_size)
+        res["e2e"] = run_e2e(args, wl2, world, rank, dev, depth)
         del wl2
+        torch.cuda.empty_cache()
+        if depth > 1:           # the same steps with the host waiting before each issue, for comparison
+            wl3 = Workload(shape, shape.seed + rank, dev, args.partition_size)
+            one = run_e2e(args, wl3, world, rank, dev, 1)
+            res["e2e"]["one_in_flight"] = {k: one[k] for k in ("value", "unit", "ms_per_step", "ms_per_step_median")}
+            del wl3
     torch.cuda.empty_cache()
     return res
 
@@ -602,14 +612,19 @@ def host_batch(shape, seed):
     return synth.make_batch(shape, device="cpu", seed=seed)
 
 
-def run_e2e(args, wl, world, rank, dev):
+def run_e2e(args, wl, world, rank, dev, depth=1):
     """The same steps through the public API from host buffers: every step's
     q / new K / new V arrive in pinned host memory, DecodeSession.launch_step
     sends them and the step's plan to the device, runs block_copy, kv_append
-    and attention and copies the output back, and the host waits for that
-    output before the next step's inputs go.  The next step's host planning
-    (allocator calls) runs while the device works, as a serving loop that
-    schedules ahead would."""
+    and attention and copies the output back to pinned host memory, and the
+    host waits for every step's output.  ``depth`` steps are in flight: the
+    host issues step i, plans step i+1, and then waits for the output of step
+    i - depth + 1 (depth 1: the host waits for each step's output before it
+    issues the next; depth 2: while it reads one step's output, the next
+    step's copies and kernels are already queued, as a serving loop with two
+    batches -- or two layers -- in flight would).  All copies and kernels go
+    to one stream, so each step's H2D, kernels and D2H still run in order on
+    the device."""
     import paged_kv_cache_405_b200 as pkv
     shape = wl.shape
     ss = wl.session
@@ -633,7 +648,8 @@ def run_e2e(args, wl, world, rank, dev):
             buf[o:o + t.numel() * esz].copy_(t.reshape(-1).view(torch.uint8))
             views.append(buf[o:o + t.numel() * esz].view(dt).view(sh_))
         host_inputs.append((buf, views))
-    out_host = torch.empty(shapes[0], dtype=dt, pin_memory=True)
+    outs = [torch.empty(shapes[0], dtype=dt, pin_memory=True) for _ in range(depth)]
+    out_host = outs[0]
     stream = torch.cuda.current_stream()
     plans = []
 
@@ -642,15 +658,22 @@ def run_e2e(args, wl, world, rank, dev):
     def run(first, n, events=False):
         p = wl.plan()
         plans.append(p)
+        pending = []            # steps whose output the host has not waited for, oldest first
         for i in range(first, first + n):
             if events:
                 step_ev.append(torch.cuda.Event(enable_timing=True))
                 step_ev[-1].record(stream)
-            ss.launch_step(p, *host_inputs[i][1], out_host=out_host, stream=stream)
+            ss.launch_step(p, *host_inputs[i][1], out_host=outs[i % depth], stream=stream)
+            done = torch.cuda.Event()
+            done.record(stream)
+            pending.append(done)
             if i + 1 < first + n:
                 p = wl.plan()       # host work of the next step, overlapping this step's kernels
                 plans.append(p)
-            stream.synchronize()    # this step's output is on the host
+            while len(pending) >= depth:
+                pending.pop(0).synchronize()   # that step's output is on the host
+        for e in pending:
+            e.synchronize()
 
     def plan_bytes(p):
         arrs = [p.slot_mapping, p.lens, p.block_tables] + ([p.cow_pairs] if len(p.cow_pairs) else [])
@@ -679,10 +702,12 @@ def run_e2e(args, wl, world, rank, dev):
     d2h = out_host.numel() * out_host.element_size()
     return {"value": round(tot / (ms * 1e-3) / 1e9, 1), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms / K, 4),
-            "ms_per_step_median": round(float(np.median(per_step)), 4),
+            "ms_per_step_median": round(float(np.median(per_step)), 4), "steps_in_flight": depth,
             "api": "DecodeSession.plan (next step planned during this one) + DecodeSession.launch_step (H2D of "
                    "the inputs from pinned host memory and of the plan, block_copy/kv_append/attention, D2H of "
-                   "the output), host waits for the output every step"}
+                   "the output), one stream; the host waits for every step's output, %s" %
+                   ("before it issues the next step" if depth == 1 else
+                    "with %d steps in flight" % depth)}
 
 
 def run_reference(args, world, rank):
@@ -803,6 +828,9 @@ def main(argv=None):
     ap.add_argument("--prefix", type=int, default=0,
                     help="shared-prompt length of a shared-prefix workload (0: the workload's own)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg from host buffers")
+    ap.add_argument("--e2e-in-flight", type=int, default=2,
+                    help="steps in flight in the end-to-end leg (1: the host waits for each step's output "
+                         "before it issues the next); the line also carries the 1-in-flight figure")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle sample length (all cores)")
     ap.add_argument("--reference-step-seconds", type=float, default=3.0,

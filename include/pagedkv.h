@@ -372,6 +372,21 @@ uint64_t pkv_launch_count(void);
  * pools in an intermediate state -- check a step's arguments once, then reuse
  * them.  struct_size must be sizeof(pkv_step) (PKV_ERR_INVALID otherwise),
  * so a caller built against another version of this header is refused.
+ *
+ * Overlapped input copies (copy_stream, inputs_free, inputs_ready: all three
+ * set, or all three null -- PKV_ERR_INVALID otherwise).  Then step 1's copies
+ * go on copy_stream instead of `stream`: copy_stream first waits for
+ * inputs_free, the copies follow, inputs_ready is recorded on copy_stream and
+ * `stream` waits for it before step 2; inputs_free is recorded on `stream`
+ * right after step 4 (after the last of steps 2-4 issued), the point after
+ * which no call of this step reads the copies' destinations.  So a step's
+ * input copies can run while earlier work on `stream` (a previous step's
+ * kernels) still runs, as long as they write other buffers: a caller that
+ * alternates sets of destination buffers gives each set its own
+ * inputs_free event (so a copy into a set waits only for the last step that
+ * read that set) and may share one inputs_ready.  The events are the
+ * caller's cudaEvent_t (made with cudaEventDisableTiming or not), the stream
+ * its cudaStream_t; the output copies (step 5) stay on `stream`.
  */
 typedef struct {
     void* dst;
@@ -425,6 +440,10 @@ typedef struct {
     /* PKV_STEP_CHUNK */
     const int32_t* query_start;
     int max_query_len;
+    /* overlapped input copies (see above): cudaStream_t, cudaEvent_t, cudaEvent_t, or all null */
+    void* copy_stream;
+    void* inputs_free;
+    void* inputs_ready;
 } pkv_step;
 
 pkv_status pkv_step_from_host(const pkv_step* step, void* stream);

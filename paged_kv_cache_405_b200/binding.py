@@ -67,6 +67,7 @@ class PkvStep(ctypes.Structure):
         ("group_first", ctypes.c_void_p), ("group_shared", ctypes.c_void_p), ("num_groups", ctypes.c_int),
         ("max_group_size", ctypes.c_int), ("max_shared_len", ctypes.c_int),
         ("query_start", ctypes.c_void_p), ("max_query_len", ctypes.c_int),
+        ("copy_stream", ctypes.c_void_p), ("inputs_free", ctypes.c_void_p), ("inputs_ready", ctypes.c_void_p),
     ]
 
 

@@ -1051,11 +1051,26 @@ extern "C" pkv_status pkv_step_from_host(const pkv_step* s, void* stream) {
         return invalid("pkv_step_from_host: bad copy lists");
     if (s->num_pairs < 0 || s->num_tokens < 0 || s->num_seqs < 0)
         return invalid("pkv_step_from_host: counts must be >= 0");
+    const bool split = s->copy_stream != nullptr;
+    if (split != (s->inputs_free != nullptr) || split != (s->inputs_ready != nullptr))
+        return invalid("pkv_step_from_host: copy_stream, inputs_free and inputs_ready go together");
     cudaStream_t st = (cudaStream_t)stream;
     const pkv_dtype dt = (pkv_dtype)s->dtype;
     const bool fp8 = s->kind == PKV_STEP_DECODE_FP8;
-    pkv_status r = copies(s->in, s->n_in, st, "input");
-    if (r != PKV_OK) return r;
+    pkv_status r;
+    if (split) {  // the input copies on copy_stream, after the last reader of their destinations
+        cudaStream_t cs = (cudaStream_t)s->copy_stream;
+        cudaError_t e = cudaStreamWaitEvent(cs, (cudaEvent_t)s->inputs_free, 0);
+        if (e != cudaSuccess) return cuda_fail("pkv_step_from_host: wait for inputs_free", e);
+        r = copies(s->in, s->n_in, cs, "input");
+        if (r != PKV_OK) return r;
+        e = cudaEventRecord((cudaEvent_t)s->inputs_ready, cs);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(st, (cudaEvent_t)s->inputs_ready, 0);
+        if (e != cudaSuccess) return cuda_fail("pkv_step_from_host: inputs_ready", e);
+    } else {
+        r = copies(s->in, s->n_in, st, "input");
+        if (r != PKV_OK) return r;
+    }
     if (s->num_pairs > 0) {
         r = pkv_block_copy(s->k_pool, s->v_pool, s->pairs, s->num_pairs, s->num_blocks, s->num_kv_heads,
                            s->head_dim, s->block_size, fp8 ? PKV_FP8_E4M3 : dt, stream);
@@ -1100,6 +1115,10 @@ extern "C" pkv_status pkv_step_from_host(const pkv_step* s, void* stream) {
                 break;
         }
         if (r != PKV_OK) return r;
+    }
+    if (split) {  // nothing of this step reads the input copies' destinations after this point
+        const cudaError_t e = cudaEventRecord((cudaEvent_t)s->inputs_free, st);
+        if (e != cudaSuccess) return cuda_fail("pkv_step_from_host: inputs_free", e);
     }
     return copies(s->out, s->n_out, st, "output");
 }

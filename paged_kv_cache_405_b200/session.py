@@ -71,10 +71,15 @@ class DevicePlan:
 class DecodeSession:
     def __init__(self, k_pool: torch.Tensor, v_pool: torch.Tensor, num_q_heads: int, max_blocks_per_seq: int,
                  free_order=None, partition_size: int = 0, max_batch: int = 0, share_prefixes: bool = True,
-                 min_group_size: int = 4, kv_scales=None, prefix_caching: bool = False):
+                 min_group_size: int = 4, kv_scales=None, prefix_caching: bool = False,
+                 overlap_input_copies: bool = True):
         """Pools of a 16-bit/fp32 type, or uint8 FP8 E4M3 codes with kv_scales = (k_scale, v_scale).
         prefix_caching: full prompt blocks registered by ``add_prompt`` are
-        reused by later prompts with the same leading tokens."""
+        reused by later prompts with the same leading tokens.
+        overlap_input_copies: ``launch_step`` sends a step's inputs on a copy
+        stream of the session's own, so that they cross while the previous
+        step's kernels still run (the kernels wait for them); off, they go on
+        the caller's stream ahead of the kernels."""
         self.k_pool, self.v_pool = k_pool, v_pool
         self.fp8 = k_pool.dtype == torch.uint8
         if self.fp8 and kv_scales is None:
@@ -98,7 +103,8 @@ class DecodeSession:
         self.workspace = torch.empty(max(256, ws), dtype=torch.uint8, device=self.device)
         self._pinned = {}
         self._layouts = {}      # host-buffer steps: staging per layout of the step's arrays
-        self._io = {}           # host-buffer steps: device q / new K / new V / out per shape
+        self.overlap_input_copies = overlap_input_copies
+        self._copy_stream = None
 
     # ------------------------------------------------------------ host side
     def add(self, sid: int, num_tokens: int = 0, shared_prefix: Optional[Sequence[int]] = None,
@@ -321,23 +327,35 @@ class DecodeSession:
                 offs.append(total)
                 total += (a.nbytes + 255) // 256 * 256
             total = max(total, 256)
+            if self.overlap_input_copies and self._copy_stream is None:
+                self._copy_stream = torch.cuda.Stream(device=self.device)
             sets = []
             for _ in range(2):
                 host = torch.empty(total, dtype=torch.uint8, pin_memory=True)
                 dev = torch.empty(total, dtype=torch.uint8, device=self.device)
                 hv = host.numpy()
-                sets.append({"host": host, "dev": dev, "bytes": total,
-                             "hviews": [hv[o:o + a.nbytes].view(a.dtype).reshape(a.shape)
-                                        for a, o in zip(arrays, offs)],
-                             "ptrs": [dev.data_ptr() + o for o in offs], "event": None, "steps": {}})
+                st = {"host": host, "dev": dev, "bytes": total,
+                      "hviews": [hv[o:o + a.nbytes].view(a.dtype).reshape(a.shape) for a, o in zip(arrays, offs)],
+                      "ptrs": [dev.data_ptr() + o for o in offs], "event": None, "steps": {}, "io": {}}
+                if self._copy_stream is not None:
+                    # events of the overlapped input copies (recorded once so
+                    # that they exist): the set's device buffers are free /
+                    # filled
+                    st["free"], st["ready"] = torch.cuda.Event(), torch.cuda.Event()
+                    st["free"].record(self._copy_stream)
+                    st["ready"].record(self._copy_stream)
+                sets.append(st)
             lay = self._layouts[key] = [0, sets]
         lay[0] ^= 1
         return lay[1][lay[0]]
 
-    def _io_buffers(self, q_host, k_new_host, v_new_host):
-        """Device q / new K / new V / out for these host shapes (made once per shape)."""
+    def _io_buffers(self, st: dict, q_host, k_new_host, v_new_host):
+        """Device q / new K / new V / out of a staging set for these host
+        shapes (made once per set and shape: the two sets of a layout never
+        share them, so one set's input copies can land while the other set's
+        step still reads its own)."""
         key = (tuple(q_host.shape), tuple(k_new_host.shape), q_host.dtype, k_new_host.dtype)
-        io = self._io.get(key)
+        io = st["io"].get(key)
         if io is None:
             if q_host.dim() != 3 or tuple(q_host.shape[1:]) != (self.num_q_heads, self.head_dim):
                 raise ValueError("q must be [rows, num_q_heads, head_dim]")
@@ -348,8 +366,8 @@ class DecodeSession:
                     raise TypeError("with FP8 pools q and new K/V must be bf16 or f16, of one type")
             elif q_host.dtype != self.k_pool.dtype or k_new_host.dtype != self.k_pool.dtype:
                 raise TypeError("q and new K/V must have the pools' element type")
-            if len(self._io) >= self._MAX_LAYOUTS:
-                self._io.pop(next(iter(self._io)))
+            if len(st["io"]) >= self._MAX_LAYOUTS:
+                st["io"].pop(next(iter(st["io"])))
             # q, new K, new V in one device block, each at a 256-byte aligned
             # offset: host inputs laid out the same way go in one copy.
             qb = q_host.numel() * q_host.element_size()
@@ -361,7 +379,7 @@ class DecodeSession:
             kn = block[ok:ok + kb].view(k_new_host.dtype).view(k_new_host.shape)
             vn = block[ov:ov + kb].view(k_new_host.dtype).view(k_new_host.shape)
             out = torch.empty_like(q)
-            io = self._io[key] = (key, q, kn, vn, out, (block, ok, ov))
+            io = st["io"][key] = (key, q, kn, vn, out, (block, ok, ov))
         if v_new_host.shape != k_new_host.shape or v_new_host.dtype != k_new_host.dtype:
             raise ValueError("k_new and v_new must have the same shape and element type")
         if not (q_host.is_contiguous() and k_new_host.is_contiguous() and v_new_host.is_contiguous()):
@@ -403,6 +421,9 @@ class DecodeSession:
             max_group_size=int(p.max_group_size) if not chunk else 0,
             max_shared_len=int(p.max_shared_len) if not chunk else 0,
             query_start=rest[0] if chunk else None, max_query_len=int(p.max_query_len) if chunk else 0)
+        if self._copy_stream is not None:   # input copies on the session's copy stream
+            step.copy_stream = self._copy_stream.cuda_stream
+            step.inputs_free, step.inputs_ready = st["free"].cuda_event, st["ready"].cuda_event
         step._copies = (ins, outs)          # the arrays the struct points to stay alive with it
         return step
 
@@ -411,12 +432,17 @@ class DecodeSession:
         """Issue one planned step (a StepPlan, or a ChunkPlan) from host
         buffers without waiting: the plan and the inputs go to the device,
         block_copy -> kv_append -> attention run, and the output is copied into
-        ``out_host`` (pinned; made if None) -- complete once ``stream`` reaches
-        this point.  q_host [rows, num_q_heads, head_dim]; k/v_new_host
-        [tokens written, num_kv_heads, head_dim]; pinned host memory lets the
-        copies run asynchronously.  Inputs that sit in one host buffer -- q,
-        then new K at the next 256-byte boundary after q, then new V at the
-        next after new K -- are sent with a single copy."""
+        ``out_host`` (pinned; if None, the session's own buffer, which the next
+        call without one reuses: with several steps in flight, pass one buffer
+        per step) -- complete once ``stream`` reaches this point.  q_host
+        [rows, num_q_heads, head_dim]; k/v_new_host [tokens written,
+        num_kv_heads, head_dim]; pinned host memory lets the copies run
+        asynchronously.  Inputs that sit in one host buffer -- q, then new K
+        at the next 256-byte boundary after q, then new V at the next after new
+        K -- are sent with a single copy.  With ``overlap_input_copies`` the
+        input copies run on the session's copy stream, and ``stream``'s
+        kernels wait for them; the host buffers must stay untouched until
+        ``stream`` reaches the end of the step either way."""
         s = torch.cuda.current_stream() if stream is None else stream
         chunk = isinstance(p, ChunkPlan)
         T = len(p.slot_mapping)
@@ -424,13 +450,6 @@ class DecodeSession:
         if q_host.shape[0] != rows or k_new_host.shape[0] != T:
             raise ValueError("q needs one row per %s and new K/V one per written token"
                              % ("new token" if chunk else "attending sequence"))
-        io = self._io_buffers(q_host, k_new_host, v_new_host)
-        out = io[4]
-        if out_host is None:
-            out_host = self._pin("out", out)
-        elif out_host.shape != out.shape or out_host.dtype != out.dtype or out_host.is_cuda or \
-                not out_host.is_contiguous():
-            raise ValueError("out_host must be a contiguous host tensor of q's shape and element type")
         n_cow = len(p.cow_pairs)
         arrays = [p.slot_mapping, p.lens, p.block_tables] + ([p.cow_pairs] if n_cow else [])
         if chunk:
@@ -438,8 +457,15 @@ class DecodeSession:
         elif p.has_groups:
             arrays += [p.group_first, p.group_shared]
         st = self._layout(arrays)
+        io = self._io_buffers(st, q_host, k_new_host, v_new_host)
+        out = io[4]
+        if out_host is None:
+            out_host = self._pin("out", out)
+        elif out_host.shape != out.shape or out_host.dtype != out.dtype or out_host.is_cuda or \
+                not out_host.is_contiguous():
+            raise ValueError("out_host must be a contiguous host tensor of q's shape and element type")
         if st["event"] is not None:
-            st["event"].synchronize()           # the step that last used this staging buffer is done
+            st["event"].synchronize()           # the step that last used this staging set is done
         for hv, a in zip(st["hviews"], arrays):
             np.copyto(hv, a, casting="no")
         step = st["steps"].get(io[0])

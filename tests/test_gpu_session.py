@@ -221,3 +221,65 @@ def test_launch_step_planned_ahead_matches_oracle(cfg, over, packed):
     bits = (lambda t: t.view(torch.uint8)) if sh.kv_fp8 else (lambda t: t.view(torch.int16))
     assert torch.equal(bits(ss.k_pool.cpu()), bits(kc)) and torch.equal(bits(ss.v_pool.cpu()), bits(vc))
     assert len(ss._layouts) <= 2          # one layout per kind of step (the first may differ)
+
+
+@pytest.mark.parametrize("cfg,over", [
+    ("llama13b_prefix", dict(S=12, Hq=4, Hkv=4)),                              # shared-prefix groups
+    ("longctx_beam", dict(S=2, Hq=16, Hkv=2, len_fixed=2000)),                 # forks: copy-on-write pairs
+    ("spec_verify", dict(S=5, Hq=8, Hkv=2, len_uniform=(20, 700))),            # causal chunks
+    ("llama7b_fp8", dict(S=6, Hq=4, Hkv=4, len_uniform=(1, 600))),             # FP8 pools
+])
+def test_launch_step_two_in_flight_matches_oracle(cfg, over):
+    """Two steps in flight, as bench.py's end-to-end leg runs them: step i+1
+    is planned and issued before the host waits for step i's output, each
+    step writing its own pinned output buffer (two alternate) and reading its
+    own pinned inputs.  Every step's output equals the oracle's attention on
+    the pools after that step, and at the end both pools equal the oracle's
+    copies and appends."""
+    import bench
+    import paged_kv_cache_405_b200 as m
+    sh = synth.shrink(synth.CONFIGS[cfg], reserve_tokens=64, **over)
+    dev = torch.device("cuda")
+    wl = bench.Workload(sh, sh.seed, dev, 0)
+    ss = wl.session
+    kc, vc = ss.k_pool.cpu(), ss.v_pool.cpu()
+    dt = synth.DTYPES[sh.dtype]
+    g = torch.Generator().manual_seed(47)
+    rows0 = sh.S * max(1, sh.chunk)
+    outs = [torch.empty((rows0, sh.Hq, sh.D), dtype=dt).pin_memory() for _ in range(2)]
+    pending = []                                 # (event, plan, q, new K, new V, out) not yet checked
+    stream = torch.cuda.current_stream()
+
+    def check(ev, p, q, kn, vn, out):
+        ev.synchronize()                         # this step's output is on the host
+        oracle.block_copy(kc, vc, p.cow_pairs)
+        if sh.kv_fp8:
+            oracle.kv_append_fp8(kc.numpy(), vc.numpy(), kn, vn, sh.kv_scale, sh.kv_scale, p.slot_mapping)
+            ref = oracle.paged_attention_kv(q, kc.numpy(), vc.numpy(), sh.kv_scale, sh.kv_scale, p.block_tables,
+                                            p.lens, threads=oracle.max_threads())
+        else:
+            oracle.kv_append(kc, vc, kn, vn, p.slot_mapping)
+            if sh.chunk:
+                ref = oracle.paged_attention_chunk(q, kc, vc, p.block_tables, p.lens, p.query_start,
+                                                   threads=oracle.max_threads())
+            else:
+                ref = oracle.paged_attention(q, kc, vc, p.block_tables, p.lens, threads=oracle.max_threads())
+        assert max_err(out, ref) <= TOL[dt]
+
+    p = wl.plan()
+    for step in range(5):
+        T = len(p.slot_mapping)
+        rows = T if sh.chunk else len(p.seq_ids)
+        q, kn, vn = packed_inputs(rows, T, sh, dt, g)
+        outs[step % 2] = ss.launch_step(p, q, kn, vn, outs[step % 2], stream=stream)
+        ev = torch.cuda.Event()
+        ev.record(stream)
+        pending.append((ev, p, q, kn, vn, outs[step % 2]))
+        p = wl.plan()                            # the step after, planned while two are in flight
+        if len(pending) == 2:
+            check(*pending.pop(0))
+    for item in pending:
+        check(*item)
+    assert m.device_error() == 0
+    bits = (lambda t: t.view(torch.uint8)) if sh.kv_fp8 else (lambda t: t.view(torch.int16))
+    assert torch.equal(bits(ss.k_pool.cpu()), bits(kc)) and torch.equal(bits(ss.v_pool.cpu()), bits(vc))
