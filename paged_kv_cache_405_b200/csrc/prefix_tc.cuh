@@ -105,27 +105,15 @@ __device__ __forceinline__ void mma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem,
 #define PKV_TI8(b) \
     "r"(v[b]), "r"(v[b + 1]), "r"(v[b + 2]), "r"(v[b + 3]), "r"(v[b + 4]), "r"(v[b + 5]), "r"(v[b + 6]), "r"(v[b + 7])
 
-// Columns c .. c+31 (c+63) of this warp's 32 lanes (thread i of the warp: lane
-// base + i); the values are complete when the call returns (the wait is in
-// the same asm statement).
+// Columns c .. c+31 (c+127) of this warp's 32 lanes (thread i of the warp:
+// lane base + i); the values are complete when the call returns (the wait is
+// in the same asm statement).
 __device__ __forceinline__ void ld_x32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
         "{\n\ttcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
         "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
         "tcgen05.wait::ld.sync.aligned;\n\t}"
         : PKV_TO8(0), PKV_TO8(8), PKV_TO8(16), PKV_TO8(24)
-        : "r"(taddr)
-        : "memory");
-}
-
-__device__ __forceinline__ void ld_x64(uint32_t taddr, uint32_t (&r)[64]) {
-    asm volatile(
-        "{\n\ttcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, "
-        "%35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, "
-        "%56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
-        "tcgen05.wait::ld.sync.aligned;\n\t}"
-        : PKV_TO8(0), PKV_TO8(8), PKV_TO8(16), PKV_TO8(24), PKV_TO8(32), PKV_TO8(40), PKV_TO8(48), PKV_TO8(56)
         : "r"(taddr)
         : "memory");
 }
@@ -143,19 +131,6 @@ __device__ __forceinline__ void ld_x128(uint32_t taddr, uint32_t (&r)[128]) {
         : PKV_TO8(0), PKV_TO8(8), PKV_TO8(16), PKV_TO8(24), PKV_TO8(32), PKV_TO8(40), PKV_TO8(48), PKV_TO8(56),
           PKV_TO8(64), PKV_TO8(72), PKV_TO8(80), PKV_TO8(88), PKV_TO8(96), PKV_TO8(104), PKV_TO8(112), PKV_TO8(120)
         : "r"(taddr)
-        : "memory");
-}
-
-__device__ __forceinline__ void st_x64(uint32_t taddr, const uint32_t (&v)[64]) {
-    asm volatile(
-        "{\n\ttcgen05.st.sync.aligned.32x32b.x64.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
-        "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, "
-        "%35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, "
-        "%56, %57, %58, %59, %60, %61, %62, %63, %64};\n\t"
-        "tcgen05.wait::st.sync.aligned;\n\t}"
-        :
-        : "r"(taddr), PKV_TI8(0), PKV_TI8(8), PKV_TI8(16), PKV_TI8(24), PKV_TI8(32), PKV_TI8(40), PKV_TI8(48),
-          PKV_TI8(56)
         : "memory");
 }
 

@@ -48,6 +48,24 @@ def run_plain(batch, P=0):
 ])
 @pytest.mark.parametrize("P", [0, 64, 512])
 def test_single_group_matches_oracle(over, P):
+    _single_group(over, P)
+
+
+# The tcgen05 pass's own shapes: 128-row query tiles, one or two per CTA
+# (groups of more than 128 rows), 128-token K/V tiles.
+@pytest.mark.parametrize("over", [
+    dict(S=130, Hq=2, Hkv=2, prefix=384),                 # 130 rows: a second query tile of 2 rows
+    dict(S=40, Hq=8, Hkv=2, prefix=640),                  # GQA, 160 rows (4 heads x 40 sequences)
+    dict(S=300, Hq=1, Hkv=1, prefix=2048),                # 300 rows: two CTAs per head, the second half full
+    dict(S=140, Hq=4, Hkv=4, prefix=768, bs=256),         # a block spans two 128-token tiles
+    dict(S=100, Hq=2, Hkv=2, prefix=112),                 # shared run shorter than one tile
+])
+@pytest.mark.parametrize("P", [0, 48, 1024])
+def test_single_group_large_tiles_match_oracle(over, P):
+    _single_group(over, P)
+
+
+def _single_group(over, P):
     sh = synth.shrink(synth.CONFIGS["llama13b_prefix"], **over)
     b = synth.make_batch(sh, fill_unused=float("nan"))
     gf, gs = pkv().find_shared_prefix_groups(b.block_tables, b.lens, sh.bs, 4)
