@@ -75,6 +75,9 @@ typedef enum { PKV_F32 = 0, PKV_BF16 = 1, PKV_F16 = 2, PKV_FP8_E4M3 = 3 /* pools
 #define PKV_DEVERR_GROUP     16u  /* a shared-prefix group description does not hold: more members than
                                      max_group_size, a shared run over max_shared_len, or a member whose
                                      leading blocks are not its group's */
+#define PKV_DEVERR_SPLIT     32u  /* a split-K counter word changed under a call in a way its own
+                                     partitions cannot explain (the workspace was in use by another
+                                     call at the same time); that row's output is not written */
 
 /* ------------------------------------------------------------------ device */
 
@@ -102,6 +105,13 @@ pkv_status pkv_kv_append(const void* k_new, const void* v_new, void* k_pool, voi
  *                    returned then covers whatever the library picks).
  * Returns 0 when no workspace is needed (every context fits one partition),
  * and SIZE_MAX when the size does not fit in size_t (such a call cannot run).
+ * Layout, for R = num_seqs*num_q_heads rows and N partitions: R*N*head_dim
+ * floats of partial outputs, R*N*2 floats of (max, sum) pairs, then, from the
+ * next 256-byte boundary, R 8-byte split counters, with which a decode
+ * kernel merges a row's partials itself once the row's last partition has
+ * finished (no reduce kernel).  A counter word holds a 48-bit stamp of the
+ * call that wrote it, so stale contents are ignored and the workspace needs
+ * no initialisation; one call at a time per workspace.
  */
 size_t pkv_attention_workspace_bytes(int num_seqs, int num_q_heads, int head_dim,
                                      int max_context_len, int partition_size);
@@ -128,7 +138,12 @@ int pkv_attention_partition_size(int num_seqs, int num_q_heads, int num_kv_heads
  *   scale           0 -> 1/sqrt(head_dim)
  *   partition_size  0 -> library's choice; > 0 (multiple of 16) splits every
  *                   context into partitions of that many tokens that run in
- *                   parallel, then a reduce kernel merges them.
+ *                   parallel, then a reduce kernel merges them (the FP8
+ *                   per-head kernel merges its own, up to 32 partitions).
+ *                   Without shared-prefix groups and for at most 256
+ *                   sequences, partitions are started longest first: every
+ *                   sequence's full partitions, then its short last ones by
+ *                   decreasing length.
  *   workspace       >= pkv_attention_workspace_bytes(...) bytes of device
  *                   memory, 256-byte aligned; contents need no initialisation.
  * Supported: head_dim 64 or 128; block_size 16, 32, 64, 128 or 256;

@@ -22,7 +22,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.environ.get("PKV_LIBRARY") or os.path.join(_HERE, "libpagedkv.so")
 
 OK, INVALID, NO_FREE_BLOCK, CUDA_ERROR, UNSUPPORTED, DEVICE_CHECK = range(6)
-DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_CONTEXT, DEVERR_TIMEOUT, DEVERR_GROUP = 1, 2, 4, 8, 16
+DEVERR_BLOCK_ID, DEVERR_SLOT, DEVERR_CONTEXT, DEVERR_TIMEOUT, DEVERR_GROUP, DEVERR_SPLIT = 1, 2, 4, 8, 16, 32
 _DTYPE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 FP8_E4M3 = 3  # pool element type of the _fp8 calls (uint8 tensors of E4M3 codes)
 

@@ -317,8 +317,14 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) paged_attn_fp8_head_kernel(c
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int h = blockIdx.x * WARPS + warp;  // query head
-    const int part = blockIdx.y;
-    const int s = blockIdx.z;
+    int part = blockIdx.y;
+    int s = blockIdx.z;
+    if (p.lpt) {
+        const int2 unit = lpt_unit_cta(p, blockIdx.z * gridDim.y + blockIdx.y);
+        if (unit.x < 0) return;
+        s = unit.x;
+        part = unit.y;
+    }
     if (h >= p.Hq) return;
     const int gid = lane >> 2, tig = lane & 3;
     const int g = h / p.G;
@@ -514,11 +520,11 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) paged_attn_fp8_head_kernel(c
     }
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) l += __shfl_xor_sync(0xffffffffu, l, off);
-    if (tig != 0) return;
 
     // Lane (gid, 0): elements gid*SPAN + 2mt (o[mt][0]) and + 2mt + 1 (o[mt][2]).
     const int64_t row = (int64_t)s * p.Hq + h;
     if (u.direct) {
+        if (tig != 0) return;
         const float inv = p.v_scale / l;
         uint32_t hw[NMT];
 #pragma unroll
@@ -526,7 +532,10 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) paged_attn_fp8_head_kernel(c
         uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<To*>(p.out) + row * D + gid * SPAN);
 #pragma unroll
         for (int v = 0; v < NMT / 4; ++v) dst[v] = make_uint4(hw[4 * v], hw[4 * v + 1], hw[4 * v + 2], hw[4 * v + 3]);
-    } else {
+        return;
+    }
+    const unsigned long long seen = p.split_count != nullptr && lane == 0 ? split_peek(p.split_count + row) : 0ull;
+    if (tig == 0) {
         const int64_t idx = row * p.maxP + u.slot;
         float4* dst = reinterpret_cast<float4*>(p.ws_o + idx * D + gid * SPAN);
 #pragma unroll
@@ -535,6 +544,7 @@ __global__ void __launch_bounds__(WARPS * 32, MINB) paged_attn_fp8_head_kernel(c
                                  o[2 * v + 1][2] * p.v_scale);
         if (gid == 0) *reinterpret_cast<float2*>(p.ws_ml + idx * 2) = make_float2(m, l);
     }
+    if (p.split_count != nullptr) merge_if_last<To, D>(p, row, u.nsuf, lane, seen);
 }
 
 }  // namespace pkv

@@ -122,8 +122,14 @@ __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_simt_kernel(const At
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int h = blockIdx.x * WARPS + warp;  // query head
-    const int part = blockIdx.y;
-    const int s = blockIdx.z;
+    int part = blockIdx.y;
+    int s = blockIdx.z;
+    if (p.lpt) {  // block-collective, before any warp leaves
+        const int2 unit = lpt_unit_cta(p, blockIdx.z * gridDim.y + blockIdx.y);
+        if (unit.x < 0) return;
+        s = unit.x;
+        part = unit.y;
+    }
     if (h >= p.Hq) return;
 
     const Unit u = resolve_unit(p, s, part, part == 0 && h == 0 && lane == 0);

@@ -8,6 +8,8 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <random>
+#include <chrono>
 #include <string>
 #include <utility>
 
@@ -83,10 +85,30 @@ static size_t partials_bytes(int64_t rows, int64_t slots, int D) {
     return c;
 }
 
+// Split-K workspace of a call without shared-prefix groups: the partials
+// (rows x partitions x D floats of o, then 2 floats of (m, l) each), then,
+// from the next 256-byte boundary, one 8-byte split counter per row
+// (pkv::split_arrive) for kernels that merge their own partials.
+static size_t split_counters_offset(size_t partials) { return (partials + 255) / 256 * 256; }
+
 static size_t workspace_for(int S, int Hq, int D, int max_len, int P) {
     const int64_t maxP = ((int64_t)max_len + P - 1) / P;
     if (maxP <= 1) return 0;
-    return partials_bytes((int64_t)S * Hq, maxP, D);
+    const size_t parts = partials_bytes((int64_t)S * Hq, maxP, D);
+    const size_t counters = (size_t)S * (size_t)Hq * sizeof(unsigned long long);
+    if (parts > SIZE_MAX - 256 || split_counters_offset(parts) > SIZE_MAX - counters) return SIZE_MAX;
+    return split_counters_offset(parts) + counters;
+}
+
+// A 48-bit stamp per decode call (pkv::split_arrive), starting from a random
+// value in each process.
+static unsigned long long next_call_stamp() {
+    static std::atomic<unsigned long long> next{[] {
+        std::random_device rd;
+        return ((unsigned long long)rd() << 32) ^ (unsigned long long)rd() ^
+               (unsigned long long)std::chrono::steady_clock::now().time_since_epoch().count();
+    }()};
+    return next.fetch_add(1) & ((1ull << 48) - 1);
 }
 
 // Shared-prefix mode: one more partial slot per (sequence, head) than
@@ -369,6 +391,26 @@ static cudaError_t launch_reduce(const pkv::ReduceParams& r, cudaStream_t st) {
     return launch_k(pkv::splitk_reduce_warp_kernel<T, D, 8, 0>, grid, block, 0, st, r);
 }
 
+// Split-K partials merged inside the decode kernel that supports it
+// (pkv::merge_if_last) instead of by the reduce kernel; PKV_SPLIT_MERGE=0
+// builds always run the reduce.
+#ifndef PKV_SPLIT_MERGE
+#define PKV_SPLIT_MERGE 1
+#endif
+
+// Longest-first unit order (pkv::lpt_unit): without shared-prefix groups, and
+// for at most 32 * kLptPerLane sequences; the value is the sequences per lane
+// (1, 2, 4 or 8), 0 for grid order.  PKV_LPT=0 builds keep grid order.
+#ifndef PKV_LPT
+#define PKV_LPT 1
+#endif
+static int lpt_order(const pkv::AttnParams& p) {
+    if (!PKV_LPT || p.member != nullptr || p.num_groups != 0 || p.S > 32 * pkv::kLptPerLane) return 0;
+    int per = 1;
+    while (32 * per < p.S) per *= 2;
+    return per;
+}
+
 // The per-sequence decode kernel of a call (no prefix pass, no reduce).
 template <typename T>
 static cudaError_t decode_pass(const pkv::AttnParams& p, int D, int nparts, bool use_mma, const CUtensorMap* mk,
@@ -380,7 +422,9 @@ static cudaError_t decode_pass(const pkv::AttnParams& p, int D, int nparts, bool
         }
     }
     dim3 grid((p.Hq + kSimtWarps - 1) / kSimtWarps, nparts, p.S);
-    return D == 64 ? launch_simt<T, 64>(p, grid, st) : launch_simt<T, 128>(p, grid, st);
+    pkv::AttnParams q = p;
+    q.lpt = lpt_order(p);
+    return D == 64 ? launch_simt<T, 64>(q, grid, st) : launch_simt<T, 128>(q, grid, st);
 }
 
 template <typename T>
@@ -447,16 +491,21 @@ template <typename To>
 static cudaError_t dispatch_attention_fp8(const pkv::AttnParams& p, int D, int nparts, bool use_mma,
                                           const CUtensorMap* mk, const CUtensorMap* mv, cudaStream_t st) {
     cudaError_t e;
+    pkv::AttnParams q = p;  // the per-head kernel merges its own partials; the others leave them to the reduce
     if (use_mma) {
+        q.split_count = nullptr;
         dim3 grid((p.Hkv + kMmaWarps - 1) / kMmaWarps, nparts, p.S);
-        e = D == 64 ? launch_mma_fp8<To, 64>(p, grid, *mk, *mv, st) : launch_mma_fp8<To, 128>(p, grid, *mk, *mv, st);
+        e = D == 64 ? launch_mma_fp8<To, 64>(q, grid, *mk, *mv, st) : launch_mma_fp8<To, 128>(q, grid, *mk, *mv, st);
     } else if (PKV_FP8_TC && D == 128) {
-        e = launch_head_fp8_tc<To>(p, nparts, *mk, *mv, st);
+        q.split_count = nullptr;
+        e = launch_head_fp8_tc<To>(q, nparts, *mk, *mv, st);
     } else {
         dim3 grid((p.Hq + kMmaWarps - 1) / kMmaWarps, nparts, p.S);
-        e = D == 64 ? launch_head_fp8<To, 64>(p, grid, *mk, *mv, st) : launch_head_fp8<To, 128>(p, grid, *mk, *mv, st);
+        q.lpt = lpt_order(p);
+        if (!PKV_SPLIT_MERGE) q.split_count = nullptr;
+        e = D == 64 ? launch_head_fp8<To, 64>(q, grid, *mk, *mv, st) : launch_head_fp8<To, 128>(q, grid, *mk, *mv, st);
     }
-    if (e != cudaSuccess || p.maxP <= 1) return e;
+    if (e != cudaSuccess || p.maxP <= 1 || q.split_count != nullptr) return e;
     pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
                         nullptr, nullptr, 0};
     return D == 64 ? launch_reduce<To, 64>(r, st) : launch_reduce<To, 128>(r, st);
@@ -624,6 +673,14 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
     p.max_shared = grp.max_shared;
     // Shared-prefix membership after the partials (8-byte aligned: (D+2)*4 is).
     p.member = grp.mode && grp.num > 0 ? reinterpret_cast<const int2*>(p.ws_ml + n_part * 2) : nullptr;
+    // Split counters (their own region of the workspace without groups); a
+    // kernel that cannot merge its own partials gets nullptr and the reduce runs.
+    if (need > 0 && !grp.mode && slots <= 32) {
+        p.split_count = reinterpret_cast<unsigned long long*>(
+            static_cast<char*>(workspace) + split_counters_offset(partials_bytes((int64_t)num_seqs * num_q_heads,
+                                                                                 slots, head_dim)));
+        p.stamp = next_call_stamp();
+    }
 
     const bool use_mma = dtype != PKV_F32 && p.G >= 2 && p.G <= 16;
     CUtensorMap mk, mv;

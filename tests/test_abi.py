@@ -40,8 +40,10 @@ def test_status_strings():
 def test_workspace_size_rules():
     # fits one partition: no workspace
     assert pkv.attention_workspace_bytes(4, 4, 64, 512, 0) == 0
-    # forced 512-token partitions of a 100k context (8 seqs x 64 heads x 196 parts x (128+2) floats)
-    assert pkv.attention_workspace_bytes(8, 64, 128, 100_160, 512) == 8 * 64 * 196 * 130 * 4
+    # forced 512-token partitions of a 100k context
+    # (8 seqs x 64 heads x 196 parts x (128+2) floats, then 8-byte split counters per row from a 256-byte boundary)
+    parts = 8 * 64 * 196 * 130 * 4
+    assert pkv.attention_workspace_bytes(8, 64, 128, 100_160, 512) == -(-parts // 256) * 256 + 8 * 64 * 8
     # the library's own choice is covered by the size it reports
     auto = pkv.attention_partition_size(64, 32, 32, 128, 2048, 0)
     assert pkv.attention_workspace_bytes(64, 32, 128, 2048, 0) >= \
@@ -134,8 +136,8 @@ def test_workspace_queries_saturate_instead_of_wrapping():
     assert pkv.attention_workspace_bytes(65535, big, 128, 1 << 30, 16) == size_max
     assert pkv.attention_shared_workspace_bytes(big, big, 128, 1 << 30, 16) == size_max
     assert pkv.attention_chunk_workspace_bytes(big, 65535, 128, 1 << 30, 16) == size_max
-    # in range: the plain product
-    assert pkv.attention_workspace_bytes(2, 3, 64, 64, 16) == 2 * 3 * 4 * 66 * 4
+    # in range: the partials (2 x 3 rows x 4 parts x 66 floats), rounded up to 256 bytes, and a counter per row
+    assert pkv.attention_workspace_bytes(2, 3, 64, 64, 16) == -(-(2 * 3 * 4 * 66 * 4) // 256) * 256 + 2 * 3 * 8
 
 
 def test_append_and_copy_validation():

@@ -119,6 +119,30 @@ def test_decode_fp8_empty_and_one_token_contexts(Hq, Hkv):
     assert max_err(out, ref) <= TOL[out.dtype]
 
 
+@pytest.mark.parametrize("S,P", [(9, 32), (200, 48), (256, 32), (300, 32)])
+def test_decode_fp8_unit_order_edge_lengths(S, P):
+    """Contexts at and around multiples of the partition (0, 1, P-1, P, P+1,
+    2P, ...) over batches whose longest-first unit order the per-head kernel
+    derives with one to eight sequences per lane (S up to 256), and past
+    that bound (grid order): every unit is attended exactly once."""
+    import paged_kv_cache_405_b200 as pkv
+    rng = np.random.default_rng(S + P)
+    edge = [0, 1, P - 1, P, P + 1, 2 * P, 2 * P + 15, 3 * P - 1, 5 * P]
+    lens = [edge[i] if i < len(edge) else int(rng.integers(0, 5 * P + 1)) for i in range(S)]
+    rng.shuffle(lens)
+    sh = synth.shrink(synth.CONFIGS["llama7b"], S=S, Hq=2, Hkv=2, lens=lens, len_uniform=None, seed=S)
+    b = synth.make_batch(sh)
+    ks, vs = 1 / 32, 1 / 8
+    kc, vc = fp8_pools(b, 6, ks, vs)
+    ref = oracle.paged_attention_kv(b.q, kc, vc, ks, vs, b.block_tables, b.lens, threads=oracle.max_threads())
+    out = torch.full_like(b.q, float("nan"), device="cuda")
+    pkv.paged_attention_decode_fp8(out, b.q.cuda(), kc.cuda(), vc.cuda(), torch.from_numpy(b.block_tables).cuda(),
+                                   torch.from_numpy(b.lens.astype(np.int32)).cuda(), ks, vs, partition_size=P)
+    assert pkv.device_error() == 0
+    assert torch.all(out.float().cpu()[torch.from_numpy(b.lens == 0)] == 0)
+    assert max_err(out, ref) <= TOL[out.dtype]
+
+
 @pytest.mark.parametrize("Hq,Hkv", [(8, 8), (16, 4)])
 def test_decode_fp8_query_magnitudes(Hq, Hkv):
     """Query rows spanning many orders of magnitude (down into the FP16
@@ -186,4 +210,99 @@ def test_session_fp8_step_matches_oracle():
                                     threads=oracle.max_threads())
     assert m.device_error() == 0
     assert np.array_equal(k.cpu().numpy(), kc) and np.array_equal(v.cpu().numpy(), vc)
+    assert max_err(out, ref) <= TOL[out.dtype]
+
+
+def _fp8_split_case(S, Hq, lens_range, seed):
+    sh = synth.shrink(synth.CONFIGS["llama7b"], S=S, Hq=Hq, Hkv=Hq, len_uniform=lens_range, seed=seed,
+                      reserve_tokens=64)
+    b = synth.make_batch(sh)
+    ks, vs = 1 / 32, 1 / 8
+    kc, vc = fp8_pools(b, seed, ks, vs)
+    return b, kc, vc, ks, vs
+
+
+def test_decode_fp8_in_kernel_merge_over_stale_workspace_and_repeated_calls():
+    """The per-head kernel merges a row's split-K partials itself (up to 32
+    partitions), counting arrivals in workspace words stamped per call: a
+    workspace of random bytes, then of 0xff bytes, then back-to-back calls on
+    the same workspace all match the oracle."""
+    import paged_kv_cache_405_b200 as pkv
+    P = 32
+    b, kc, vc, ks, vs = _fp8_split_case(9, 4, (1, 700), 21)
+    maxB = b.block_tables.shape[1]
+    assert 1 < -(-maxB * 16 // P) <= 32
+    ref = oracle.paged_attention_kv(b.q, kc, vc, ks, vs, b.block_tables, b.lens, threads=oracle.max_threads())
+    n = pkv.attention_workspace_bytes(b.shape.S, b.shape.Hq, 128, maxB * 16, P)
+    g = torch.Generator().manual_seed(3)
+    ws = torch.randint(0, 256, (n,), dtype=torch.uint8, generator=g).cuda()
+    args = (b.q.cuda(), kc.cuda(), vc.cuda(), torch.from_numpy(b.block_tables).cuda(),
+            torch.from_numpy(b.lens.astype(np.int32)).cuda(), ks, vs)
+    for fill in ("random", "ones", "previous", "previous"):
+        if fill == "ones":
+            ws.fill_(0xFF)
+        out = torch.full_like(b.q, float("nan"), device="cuda")
+        pkv.paged_attention_decode_fp8(out, *args, partition_size=P, workspace=ws)
+        assert pkv.device_error() == 0
+        assert max_err(out, ref) <= TOL[out.dtype], fill
+
+
+def test_decode_fp8_in_kernel_merge_replayed_from_a_cuda_graph():
+    """CUDA-graph replays reuse one call stamp: every replay starts its
+    arrival counts from zero (the completing arrival resets them), also when
+    the lengths, and with them the partitions per row, change between
+    replays."""
+    import paged_kv_cache_405_b200 as pkv
+    P = 32
+    b, kc, vc, ks, vs = _fp8_split_case(6, 8, (200, 700), 22)
+    S, Hq, D = b.shape.S, b.shape.Hq, 128
+    maxB = b.block_tables.shape[1]
+    n = pkv.attention_workspace_bytes(S, Hq, D, maxB * 16, P)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    q = torch.empty(S, Hq, D, dtype=b.q.dtype, device="cuda")
+    lens = torch.empty(S, dtype=torch.int32, device="cuda")
+    out = torch.empty(S, Hq, D, dtype=b.q.dtype, device="cuda")
+    kd, vd, bt = kc.cuda(), vc.cuda(), torch.from_numpy(b.block_tables).cuda()
+    rng = np.random.default_rng(5)
+
+    def case(step):
+        g = torch.Generator().manual_seed(50 + step)
+        ln = np.minimum(b.lens, rng.integers(1, 701, size=S)).astype(np.int32)   # within each table
+        ln[step % S] = 0 if step == 2 else ln[step % S]                           # an empty row once
+        return synth.randn((S, Hq, D), g, b.q.dtype, "cpu"), ln
+
+    def run():
+        pkv.paged_attention_decode_fp8(out, q, kd, vd, bt, lens, ks, vs, partition_size=P, workspace=ws)
+
+    qh, ln = case(0)
+    q.copy_(qh)
+    lens.copy_(torch.from_numpy(ln))
+    run()                            # eager first call
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        run()
+    for step in range(1, 5):
+        qh, ln = case(step)
+        q.copy_(qh)
+        lens.copy_(torch.from_numpy(ln))
+        graph.replay()
+        torch.cuda.synchronize()
+        ref = oracle.paged_attention_kv(qh, kc, vc, ks, vs, b.block_tables, ln, threads=oracle.max_threads())
+        assert pkv.device_error() == 0
+        assert max_err(out, ref) <= TOL[out.dtype], step
+
+
+def test_decode_fp8_more_than_32_partitions_uses_the_reduce():
+    """Past 32 partitions per row the per-head kernel leaves the merge to the
+    reduce kernel; the result is the same."""
+    import paged_kv_cache_405_b200 as pkv
+    P = 16
+    b, kc, vc, ks, vs = _fp8_split_case(5, 4, (500, 900), 23)
+    assert -(-b.block_tables.shape[1] * 16 // P) > 32
+    ref = oracle.paged_attention_kv(b.q, kc, vc, ks, vs, b.block_tables, b.lens, threads=oracle.max_threads())
+    out = torch.full_like(b.q, float("nan"), device="cuda")
+    pkv.paged_attention_decode_fp8(out, b.q.cuda(), kc.cuda(), vc.cuda(), torch.from_numpy(b.block_tables).cuda(),
+                                   torch.from_numpy(b.lens.astype(np.int32)).cuda(), ks, vs, partition_size=P)
+    assert pkv.device_error() == 0
     assert max_err(out, ref) <= TOL[out.dtype]
