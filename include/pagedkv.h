@@ -140,10 +140,11 @@ int pkv_attention_partition_size(int num_seqs, int num_q_heads, int num_kv_heads
  *                   context into partitions of that many tokens that run in
  *                   parallel, then a reduce kernel merges them (the FP8
  *                   per-head kernel merges its own, up to 32 partitions).
- *                   Without shared-prefix groups and for at most 256
- *                   sequences, partitions are started longest first: every
- *                   sequence's full partitions, then its short last ones by
- *                   decreasing length.
+ *                   For at most 256 sequences and 1024 sequences x
+ *                   partitions per call, the MHA kernels start partitions
+ *                   longest first: every sequence's full partitions, then
+ *                   its short last ones by decreasing length (the same
+ *                   partitions, in another order).
  *   workspace       >= pkv_attention_workspace_bytes(...) bytes of device
  *                   memory, 256-byte aligned; contents need no initialisation.
  * Supported: head_dim 64 or 128; block_size 16, 32, 64, 128 or 256;

@@ -150,21 +150,23 @@ __device__ __forceinline__ Unit resolve_unit(const AttnParams& p, int s, int par
 // The hardware starts a grid's CTAs roughly in grid order, and a call's units
 // run from 1 to P tokens (each sequence's last partition is the short one):
 // a long unit started among the last CTAs sets the end of the kernel.  A
-// decode kernel without shared-prefix groups may instead take the unit of
+// decode kernel may instead take the unit of
 // rank r, its place in the (y, z) plane of the grid (r = z * gridDim.y + y;
-// every rank has gridDim.x CTAs, one per head group, started together):
-//   ranks 0 .. F-1      the full partitions (P tokens), in sequence order;
-//   ranks F .. F+R-1    the last partition of each sequence whose length is
-//                       not a multiple of P, and partition 0 of each empty
+// every rank has gridDim.x CTAs, one per head group, started together).  A
+// sequence's own tokens are its context less the prefix a shared-prefix
+// group member takes from the prefix pass (AttnParams::member):
+//   ranks 0 .. F-1      the full partitions (P own tokens), in sequence order;
+//   ranks F .. F+R-1    the last partition of each sequence whose own length
+//                       is not a multiple of P, and partition 0 of each empty
 //                       sequence, longest first (lengths in kLptBins bins of
 //                       about P/kLptBins tokens; ties in sequence order);
 //   higher ranks        no unit (the grid has nparts * S ranks).
-// These are exactly the units that partition order has (part < ceil(L/P),
+// These are exactly the units that partition order has (part < ceil(own/P),
 // or part 0 of an empty sequence), so resolve_unit and the split-K reduce
 // see the same (s, part) pairs.  One warp derives the order from
-// context_lens (clamped like load_context_len) with shuffles and a radix
-// select over the bins (lpt_unit, warp-collective); lpt_unit_cta hands the
-// answer to the CTA's other warps.  The host sets p.lpt = PER, the sequences
+// context_lens (clamped like load_context_len) and the membership with
+// shuffles and a radix select over the bins (lpt_unit, warp-collective);
+// lpt_unit_cta hands the answer to the CTA's other warps.  The host sets p.lpt = PER, the sequences
 // per lane (1, 2, 4 or 8: S <= 32 * PER), or 0 for grid order.
 constexpr int kLptBins = 256;  // 8-bit bin index
 constexpr int kLptPerLane = 8;  // largest PER
@@ -178,28 +180,35 @@ __device__ __forceinline__ int lpt_div(int L, int P, float inv_p) {
     return q;
 }
 
-// The unit (s, part) of rank r over context_lens[0 .. S-1], or (-1, -1);
-// S <= 32 * PER.
+// The unit (s, part) of rank r over context_lens[0 .. S-1] (and member, if
+// not null, as resolve_unit reads it), or (-1, -1); S <= 32 * PER.
 template <int PER>
-__device__ __noinline__ int2 lpt_unit(const int32_t* context_lens, int S, int P, int max_len, int r) {
+__device__ __noinline__ int2 lpt_unit(const int32_t* context_lens, const int2* member, int S, int P, int max_len,
+                                      int r) {
     const int lane = threadIdx.x & 31;
     const int s0 = min(S, lane * PER), s1 = min(S, s0 + PER);  // this lane's sequences
     const bool small = max_len < (1 << 24);
     const float inv_p = __frcp_rn((float)P);
-    int len[PER], f[PER];  // clamped lengths; full partitions
+    int len[PER], own_len[PER], f[PER];  // clamped lengths (-1: no sequence); own tokens; full partitions
     int fsum = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
         len[i] = -1;
+        own_len[i] = 0;
         f[i] = 0;
         if (s0 + i < s1) {
             const int L = context_lens[s0 + i];
             len[i] = L < 0 ? 0 : (L > max_len ? max_len : L);
+            own_len[i] = len[i];
+            if (member != nullptr) {
+                const int2 m = member[s0 + i];
+                if (m.x > 0 && m.y > 0 && m.y <= len[i]) own_len[i] -= m.y;
+            }
         }
     }
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
-        if (len[i] > 0) f[i] = small ? lpt_div(len[i], P, inv_p) : len[i] / P;
+        if (own_len[i] > 0) f[i] = small ? lpt_div(own_len[i], P, inv_p) : own_len[i] / P;
         fsum += f[i];
     }
     int x = fsum;  // inclusive prefix over lanes = over sequences
@@ -231,7 +240,7 @@ __device__ __noinline__ int2 lpt_unit(const int32_t* context_lens, int S, int P,
     int psum = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
-        const int rem = len[i] - f[i] * P;
+        const int rem = own_len[i] - f[i] * P;
         bin[i] = len[i] < 0 || (rem == 0 && len[i] != 0) ? -1
                  : rem == 0                                ? 0
                                                            : min(kLptBins - 1, 1 + __float2int_rz(__int2float_rn(rem - 1) * inv_p *
@@ -287,10 +296,10 @@ __device__ __forceinline__ int2 lpt_unit_cta(const AttnParams& p, int r) {
     if (threadIdx.x < 32) {
         int2 u;
         switch (p.lpt) {
-            case 1: u = lpt_unit<1>(p.context_lens, p.S, p.P, p.max_len, r); break;
-            case 2: u = lpt_unit<2>(p.context_lens, p.S, p.P, p.max_len, r); break;
-            case 4: u = lpt_unit<4>(p.context_lens, p.S, p.P, p.max_len, r); break;
-            default: u = lpt_unit<kLptPerLane>(p.context_lens, p.S, p.P, p.max_len, r); break;
+            case 1: u = lpt_unit<1>(p.context_lens, p.member, p.S, p.P, p.max_len, r); break;
+            case 2: u = lpt_unit<2>(p.context_lens, p.member, p.S, p.P, p.max_len, r); break;
+            case 4: u = lpt_unit<4>(p.context_lens, p.member, p.S, p.P, p.max_len, r); break;
+            default: u = lpt_unit<kLptPerLane>(p.context_lens, p.member, p.S, p.P, p.max_len, r); break;
         }
         if (threadIdx.x == 0) pick = u;
     }

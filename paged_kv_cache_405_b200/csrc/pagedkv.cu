@@ -398,14 +398,20 @@ static cudaError_t launch_reduce(const pkv::ReduceParams& r, cudaStream_t st) {
 #define PKV_SPLIT_MERGE 1
 #endif
 
-// Longest-first unit order (pkv::lpt_unit): without shared-prefix groups, and
-// for at most 32 * kLptPerLane sequences; the value is the sequences per lane
-// (1, 2, 4 or 8), 0 for grid order.  PKV_LPT=0 builds keep grid order.
+// Longest-first unit order (pkv::lpt_unit) for at most 32 * kLptPerLane
+// sequences and kLptMaxRanks ranks (sequences x partitions); the value is the
+// sequences per lane (1, 2, 4 or 8), 0 for grid order.  Ranks without a unit
+// come last in that order, each CTA of them deriving the order before it
+// leaves: with many more ranks than units (a long max_context_len over short
+// contexts) that tail costs more than the order saves, where grid order
+// spreads the empty CTAs among the working ones.  PKV_LPT=0 builds keep grid
+// order.
 #ifndef PKV_LPT
 #define PKV_LPT 1
 #endif
-static int lpt_order(const pkv::AttnParams& p) {
-    if (!PKV_LPT || p.member != nullptr || p.num_groups != 0 || p.S > 32 * pkv::kLptPerLane) return 0;
+constexpr int64_t kLptMaxRanks = 1024;
+static int lpt_order(const pkv::AttnParams& p, int nparts) {
+    if (!PKV_LPT || p.S > 32 * pkv::kLptPerLane || (int64_t)p.S * nparts > kLptMaxRanks) return 0;
     int per = 1;
     while (32 * per < p.S) per *= 2;
     return per;
@@ -423,7 +429,7 @@ static cudaError_t decode_pass(const pkv::AttnParams& p, int D, int nparts, bool
     }
     dim3 grid((p.Hq + kSimtWarps - 1) / kSimtWarps, nparts, p.S);
     pkv::AttnParams q = p;
-    q.lpt = lpt_order(p);
+    q.lpt = lpt_order(p, nparts);
     return D == 64 ? launch_simt<T, 64>(q, grid, st) : launch_simt<T, 128>(q, grid, st);
 }
 
@@ -501,7 +507,7 @@ static cudaError_t dispatch_attention_fp8(const pkv::AttnParams& p, int D, int n
         e = launch_head_fp8_tc<To>(q, nparts, *mk, *mv, st);
     } else {
         dim3 grid((p.Hq + kMmaWarps - 1) / kMmaWarps, nparts, p.S);
-        q.lpt = lpt_order(p);
+        q.lpt = lpt_order(p, nparts);
         if (!PKV_SPLIT_MERGE) q.split_count = nullptr;
         e = D == 64 ? launch_head_fp8<To, 64>(q, grid, *mk, *mv, st) : launch_head_fp8<To, 128>(q, grid, *mk, *mv, st);
     }

@@ -119,12 +119,13 @@ def test_decode_fp8_empty_and_one_token_contexts(Hq, Hkv):
     assert max_err(out, ref) <= TOL[out.dtype]
 
 
-@pytest.mark.parametrize("S,P", [(9, 32), (200, 48), (256, 32), (300, 32)])
+@pytest.mark.parametrize("S,P", [(9, 32), (100, 64), (144, 128), (256, 32), (300, 32)])
 def test_decode_fp8_unit_order_edge_lengths(S, P):
     """Contexts at and around multiples of the partition (0, 1, P-1, P, P+1,
     2P, ...) over batches whose longest-first unit order the per-head kernel
-    derives with one to eight sequences per lane (S up to 256), and past
-    that bound (grid order): every unit is attended exactly once."""
+    derives with one, four and eight sequences per lane (S up to 256 and at
+    most 1024 sequences x partitions), and past those bounds (grid order):
+    every unit is attended exactly once."""
     import paged_kv_cache_405_b200 as pkv
     rng = np.random.default_rng(S + P)
     edge = [0, 1, P - 1, P, P + 1, 2 * P, 2 * P + 15, 3 * P - 1, 5 * P]

@@ -117,6 +117,22 @@ def test_mixed_groups_and_gaps(P):
     assert max_err(out, oracle_attention(b)) <= TOL[out.dtype]
 
 
+@pytest.mark.parametrize("P", [0, 32, 128])
+def test_mha_mixed_groups_in_longest_first_order(P):
+    """MHA, where the per-sequence kernel starts its units longest first,
+    counting only a member's own tokens: members with no own token and with
+    one, own lengths across several partitions, non-members and an empty
+    sequence."""
+    b = mixed_batch(Hq=4, Hkv=4)
+    b.lens[7] = 0
+    gf, gs = pkv().find_shared_prefix_groups(b.block_tables, b.lens, 16, 3)
+    assert gs.tolist()[0] == 256 and gs.tolist()[-1] == 128
+    out = run_shared(b, gf, gs, P)
+    assert pkv().device_error() == 0
+    assert torch.all(out[7].float() == 0)
+    assert max_err(out, oracle_attention(b)) <= TOL[out.dtype]
+
+
 def test_malformed_group_is_reported_and_falls_back():
     b = mixed_batch(seed=5)
     # 200 is not a multiple of the block size: reported, the members are then
