@@ -16,7 +16,10 @@ e2e    -- the same metric through DecodeSession.launch_step: allocator on the
           host, every step's inputs copied in from pinned host memory and its
           output copied back to pinned host memory and waited for, two steps
           in flight (--e2e-in-flight; the line also carries the figure with
-          the host waiting for each output before the next step goes).
+          the host waiting for each output before the next step goes); input
+          and output copies on streams of the session's own, overlapping
+          the neighbouring steps' kernels (--e2e-serial-output keeps the
+          output copy on the kernels' stream).
 
 The headline workload (``--config``, default ``llama3_gqa_bs16``: 128
 sequences x 8192 tokens, 32 query / 8 kv heads, the largest one-GPU decode
@@ -114,7 +117,7 @@ def copy_bytes(n_pairs, Hkv, bs, D, elt):
 class Workload:
     """A batch laid out in the pool plus the session that drives its steps."""
 
-    def __init__(self, shape, seed, device, partition_size):
+    def __init__(self, shape, seed, device, partition_size, overlap_output_copies=True):
         import paged_kv_cache_405_b200 as pkv
         self.shape = shape
         self.batch = synth.make_batch(shape, device=device, seed=seed)
@@ -122,6 +125,7 @@ class Workload:
         self.P = partition_size or shape.partition_size
         self.session = pkv.DecodeSession(b.k_pool, b.v_pool, shape.Hq, b.max_blocks, free_order=b.free_order,
                                          partition_size=self.P, max_batch=shape.S,
+                                         overlap_output_copies=overlap_output_copies,
                                          kv_scales=(shape.kv_scale, shape.kv_scale) if shape.kv_fp8 else None)
         ss = self.session
         if shape.prefix:
@@ -543,12 +547,12 @@ def measure_workload(name, args, world, rank, local, e2e=True):
         del wl, ss, plans, inputs, out
         torch.cuda.empty_cache()
         depth = max(1, args.e2e_in_flight)
-        wl2 = Workload(shape, shape.seed + rank, dev, args.partition_size)
+        wl2 = Workload(shape, shape.seed + rank, dev, args.partition_size, not args.e2e_serial_output)
         res["e2e"] = run_e2e(args, wl2, world, rank, dev, depth)
         del wl2
         torch.cuda.empty_cache()
         if depth > 1:           # the same steps with the host waiting before each issue, for comparison
-            wl3 = Workload(shape, shape.seed + rank, dev, args.partition_size)
+            wl3 = Workload(shape, shape.seed + rank, dev, args.partition_size, not args.e2e_serial_output)
             one = run_e2e(args, wl3, world, rank, dev, 1)
             res["e2e"]["one_in_flight"] = {k: one[k] for k in ("value", "unit", "ms_per_step", "ms_per_step_median")}
             del wl3
@@ -622,9 +626,12 @@ def run_e2e(args, wl, world, rank, dev, depth=1):
     i - depth + 1 (depth 1: the host waits for each step's output before it
     issues the next; depth 2: while it reads one step's output, the next
     step's copies and kernels are already queued, as a serving loop with two
-    batches -- or two layers -- in flight would).  All copies and kernels go
-    to one stream, so each step's H2D, kernels and D2H still run in order on
-    the device."""
+    batches -- or two layers -- in flight would).  The input copies go on the
+    session's copy stream, the kernels on the current stream and the output
+    copies on the session's output stream (overlap_output_copies), so one
+    step's output can cross to the host while the next step's kernels run;
+    the host waits for each output through the event launch_step records
+    once that copy is complete."""
     import paged_kv_cache_405_b200 as pkv
     shape = wl.shape
     ss = wl.session
@@ -663,9 +670,8 @@ def run_e2e(args, wl, world, rank, dev, depth=1):
             if events:
                 step_ev.append(torch.cuda.Event(enable_timing=True))
                 step_ev[-1].record(stream)
-            ss.launch_step(p, *host_inputs[i][1], out_host=outs[i % depth], stream=stream)
             done = torch.cuda.Event()
-            done.record(stream)
+            ss.launch_step(p, *host_inputs[i][1], out_host=outs[i % depth], stream=stream, out_ready=done)
             pending.append(done)
             if i + 1 < first + n:
                 p = wl.plan()       # host work of the next step, overlapping this step's kernels
@@ -704,8 +710,8 @@ def run_e2e(args, wl, world, rank, dev, depth=1):
             "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms / K, 4),
             "ms_per_step_median": round(float(np.median(per_step)), 4), "steps_in_flight": depth,
             "api": "DecodeSession.plan (next step planned during this one) + DecodeSession.launch_step (H2D of "
-                   "the inputs from pinned host memory and of the plan, block_copy/kv_append/attention, D2H of "
-                   "the output), one stream; the host waits for every step's output, %s" %
+                   "the inputs from pinned host memory and of the plan on a copy stream, block_copy/kv_append/"
+                   "attention, D2H of the output on an output stream); the host waits for every step's output, %s" %
                    ("before it issues the next step" if depth == 1 else
                     "with %d steps in flight" % depth)}
 
@@ -831,6 +837,9 @@ def main(argv=None):
     ap.add_argument("--e2e-in-flight", type=int, default=2,
                     help="steps in flight in the end-to-end leg (1: the host waits for each step's output "
                          "before it issues the next); the line also carries the 1-in-flight figure")
+    ap.add_argument("--e2e-serial-output", action="store_true",
+                    help="end-to-end leg: copy each step's output back on the kernels' stream (no output-copy "
+                         "overlap), for comparison")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="CPU-oracle sample length (all cores)")
     ap.add_argument("--reference-step-seconds", type=float, default=3.0,

@@ -402,7 +402,22 @@ uint64_t pkv_launch_count(void);
  * inputs_free event (so a copy into a set waits only for the last step that
  * read that set) and may share one inputs_ready.  The events are the
  * caller's cudaEvent_t (made with cudaEventDisableTiming or not), the stream
- * its cudaStream_t; the output copies (step 5) stay on `stream`.
+ * its cudaStream_t.
+ *
+ * Overlapped output copies (out_stream, outputs_done: both set, or both
+ * null; they need the input-copy fields set too -- PKV_ERR_INVALID
+ * otherwise).  Then step 5's copies go on out_stream instead of `stream`:
+ * out_stream waits for inputs_free (recorded after step 4), the copies
+ * follow, and outputs_done is recorded on out_stream; before step 4 `stream`
+ * waits for outputs_done as last recorded (the previous step whose output
+ * copies read the same attention output buffer).  So the next step's kernels
+ * on `stream` need not wait for this step's output to cross to the host: a
+ * caller that alternates output buffers gives each its own outputs_done.
+ * With them the output is in its destination once outputs_done has been
+ * reached -- not when `stream` reaches the end of the call -- and
+ * out_stream should be another stream than copy_stream (output copies
+ * queued there would hold back the next step's input copies).  Without
+ * them the output copies stay on `stream`.
  */
 typedef struct {
     void* dst;
@@ -460,6 +475,9 @@ typedef struct {
     void* copy_stream;
     void* inputs_free;
     void* inputs_ready;
+    /* overlapped output copies (see above): cudaStream_t, cudaEvent_t, or both null */
+    void* out_stream;
+    void* outputs_done;
 } pkv_step;
 
 pkv_status pkv_step_from_host(const pkv_step* step, void* stream);

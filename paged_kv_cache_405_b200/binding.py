@@ -68,6 +68,7 @@ class PkvStep(ctypes.Structure):
         ("max_group_size", ctypes.c_int), ("max_shared_len", ctypes.c_int),
         ("query_start", ctypes.c_void_p), ("max_query_len", ctypes.c_int),
         ("copy_stream", ctypes.c_void_p), ("inputs_free", ctypes.c_void_p), ("inputs_ready", ctypes.c_void_p),
+        ("out_stream", ctypes.c_void_p), ("outputs_done", ctypes.c_void_p),
     ]
 
 

@@ -1117,6 +1117,11 @@ extern "C" pkv_status pkv_step_from_host(const pkv_step* s, void* stream) {
     const bool split = s->copy_stream != nullptr;
     if (split != (s->inputs_free != nullptr) || split != (s->inputs_ready != nullptr))
         return invalid("pkv_step_from_host: copy_stream, inputs_free and inputs_ready go together");
+    const bool split_out = s->out_stream != nullptr;
+    if (split_out != (s->outputs_done != nullptr))
+        return invalid("pkv_step_from_host: out_stream and outputs_done go together");
+    if (split_out && !split)
+        return invalid("pkv_step_from_host: out_stream needs copy_stream, inputs_free and inputs_ready");
     cudaStream_t st = (cudaStream_t)stream;
     const pkv_dtype dt = (pkv_dtype)s->dtype;
     const bool fp8 = s->kind == PKV_STEP_DECODE_FP8;
@@ -1146,6 +1151,10 @@ extern "C" pkv_status pkv_step_from_host(const pkv_step* s, void* stream) {
                 : pkv_kv_append(s->k_new, s->v_new, s->k_pool, s->v_pool, s->slot_mapping, s->num_tokens,
                                 s->num_blocks, s->num_kv_heads, s->head_dim, s->block_size, dt, stream);
         if (r != PKV_OK) return r;
+    }
+    if (split_out) {  // the previous output copies out of attn_out have finished
+        const cudaError_t e = cudaStreamWaitEvent(st, (cudaEvent_t)s->outputs_done, 0);
+        if (e != cudaSuccess) return cuda_fail("pkv_step_from_host: wait for outputs_done", e);
     }
     if (s->num_seqs > 0) {
         switch (s->kind) {
@@ -1183,5 +1192,12 @@ extern "C" pkv_status pkv_step_from_host(const pkv_step* s, void* stream) {
         const cudaError_t e = cudaEventRecord((cudaEvent_t)s->inputs_free, st);
         if (e != cudaSuccess) return cuda_fail("pkv_step_from_host: inputs_free", e);
     }
-    return copies(s->out, s->n_out, st, "output");
+    if (!split_out) return copies(s->out, s->n_out, st, "output");
+    cudaStream_t os = (cudaStream_t)s->out_stream;  // the output copies after the kernels, off `stream`
+    cudaError_t e = cudaStreamWaitEvent(os, (cudaEvent_t)s->inputs_free, 0);
+    if (e != cudaSuccess) return cuda_fail("pkv_step_from_host: out_stream wait", e);
+    r = copies(s->out, s->n_out, os, "output");
+    if (r != PKV_OK) return r;
+    e = cudaEventRecord((cudaEvent_t)s->outputs_done, os);
+    return e == cudaSuccess ? PKV_OK : cuda_fail("pkv_step_from_host: outputs_done", e);
 }

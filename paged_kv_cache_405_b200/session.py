@@ -72,14 +72,20 @@ class DecodeSession:
     def __init__(self, k_pool: torch.Tensor, v_pool: torch.Tensor, num_q_heads: int, max_blocks_per_seq: int,
                  free_order=None, partition_size: int = 0, max_batch: int = 0, share_prefixes: bool = True,
                  min_group_size: int = 4, kv_scales=None, prefix_caching: bool = False,
-                 overlap_input_copies: bool = True):
+                 overlap_input_copies: bool = True, overlap_output_copies: bool = False):
         """Pools of a 16-bit/fp32 type, or uint8 FP8 E4M3 codes with kv_scales = (k_scale, v_scale).
         prefix_caching: full prompt blocks registered by ``add_prompt`` are
         reused by later prompts with the same leading tokens.
         overlap_input_copies: ``launch_step`` sends a step's inputs on a copy
         stream of the session's own, so that they cross while the previous
         step's kernels still run (the kernels wait for them); off, they go on
-        the caller's stream ahead of the kernels."""
+        the caller's stream ahead of the kernels.
+        overlap_output_copies (needs overlap_input_copies): ``launch_step``
+        copies a step's output back on a second stream of the session's own
+        after the kernels, so that the next step's kernels need not wait for
+        it; the caller then learns that the output has arrived only from the
+        ``out_ready`` event it passes to ``launch_step``, not from its
+        stream."""
         self.k_pool, self.v_pool = k_pool, v_pool
         self.fp8 = k_pool.dtype == torch.uint8
         if self.fp8 and kv_scales is None:
@@ -103,8 +109,12 @@ class DecodeSession:
         self.workspace = torch.empty(max(256, ws), dtype=torch.uint8, device=self.device)
         self._pinned = {}
         self._layouts = {}      # host-buffer steps: staging per layout of the step's arrays
+        if overlap_output_copies and not overlap_input_copies:
+            raise ValueError("overlap_output_copies needs overlap_input_copies")
         self.overlap_input_copies = overlap_input_copies
+        self.overlap_output_copies = overlap_output_copies
         self._copy_stream = None
+        self._out_stream = None
 
     # ------------------------------------------------------------ host side
     def add(self, sid: int, num_tokens: int = 0, shared_prefix: Optional[Sequence[int]] = None,
@@ -290,8 +300,9 @@ class DecodeSession:
         """A full step from host buffers: plan, copy inputs in, run, copy the output back, wait."""
         p = self.plan(attend)
         s = torch.cuda.current_stream() if stream is None else stream
-        out_host = self.launch_step(p, q_host, k_new_host, v_new_host, out_host, stream=s)
-        s.synchronize()
+        done = torch.cuda.Event()
+        out_host = self.launch_step(p, q_host, k_new_host, v_new_host, out_host, stream=s, out_ready=done)
+        done.synchronize()
         return out_host
 
     # ------------------------------------------------- host-buffer steps
@@ -329,6 +340,8 @@ class DecodeSession:
             total = max(total, 256)
             if self.overlap_input_copies and self._copy_stream is None:
                 self._copy_stream = torch.cuda.Stream(device=self.device)
+            if self.overlap_output_copies and self._out_stream is None:
+                self._out_stream = torch.cuda.Stream(device=self.device)
             sets = []
             for _ in range(2):
                 host = torch.empty(total, dtype=torch.uint8, pin_memory=True)
@@ -344,6 +357,11 @@ class DecodeSession:
                     st["free"], st["ready"] = torch.cuda.Event(), torch.cuda.Event()
                     st["free"].record(self._copy_stream)
                     st["ready"].record(self._copy_stream)
+                if self._out_stream is not None:
+                    # the set's output copies are done (its device output
+                    # buffers may be written again)
+                    st["odone"] = torch.cuda.Event()
+                    st["odone"].record(self._out_stream)
                 sets.append(st)
             lay = self._layouts[key] = [0, sets]
         lay[0] ^= 1
@@ -424,11 +442,13 @@ class DecodeSession:
         if self._copy_stream is not None:   # input copies on the session's copy stream
             step.copy_stream = self._copy_stream.cuda_stream
             step.inputs_free, step.inputs_ready = st["free"].cuda_event, st["ready"].cuda_event
+        if self._out_stream is not None:    # output copies on the session's output stream
+            step.out_stream, step.outputs_done = self._out_stream.cuda_stream, st["odone"].cuda_event
         step._copies = (ins, outs)          # the arrays the struct points to stay alive with it
         return step
 
     def launch_step(self, p, q_host: torch.Tensor, k_new_host: torch.Tensor, v_new_host: torch.Tensor,
-                    out_host: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+                    out_host: Optional[torch.Tensor] = None, stream=None, out_ready=None) -> torch.Tensor:
         """Issue one planned step (a StepPlan, or a ChunkPlan) from host
         buffers without waiting: the plan and the inputs go to the device,
         block_copy -> kv_append -> attention run, and the output is copied into
@@ -442,7 +462,12 @@ class DecodeSession:
         K -- are sent with a single copy.  With ``overlap_input_copies`` the
         input copies run on the session's copy stream, and ``stream``'s
         kernels wait for them; the host buffers must stay untouched until
-        ``stream`` reaches the end of the step either way."""
+        ``stream`` reaches the end of the step either way.  ``out_ready`` (a
+        torch.cuda.Event, optional) is recorded where the output copy is
+        complete: on ``stream``, or with ``overlap_output_copies`` on the
+        session's output stream -- then ``stream`` reaching the end of the
+        step does not mean the output has arrived, and out_ready is how to
+        wait for it."""
         s = torch.cuda.current_stream() if stream is None else stream
         chunk = isinstance(p, ChunkPlan)
         T = len(p.slot_mapping)
@@ -490,6 +515,8 @@ class DecodeSession:
         if st["event"] is None:
             st["event"] = torch.cuda.Event()
         st["event"].record(s)
+        if out_ready is not None:
+            out_ready.record(self._out_stream if self._out_stream is not None else s)
         return out_host
 
 

@@ -373,6 +373,8 @@ def step_struct(**over):
     (dict(num_tokens=-3), "counts must be >= 0"),
     (dict(copy_stream=16), "go together"),                  # overlapped copies: stream without its events
     (dict(inputs_free=16, inputs_ready=32), "go together"),  # events without the stream
+    (dict(out_stream=16), "go together"),                   # overlapped output copies: stream without its event
+    (dict(out_stream=16, outputs_done=32), "needs copy_stream"),  # ... without the overlapped input copies
     (dict(num_pairs=1, pairs=16, k_pool=16, v_pool=8), "16-byte aligned"),        # pkv_block_copy's own check
     (dict(num_tokens=2, k_new=16, v_new=16, k_pool=16, v_pool=16, slot_mapping=16, head_dim=6), "multiple of 16"),
     (dict(num_seqs=1, q=16, attn_out=16, k_pool=16, v_pool=16, block_tables=16, context_lens=16, num_q_heads=6),

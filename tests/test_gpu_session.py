@@ -196,9 +196,10 @@ def test_launch_step_planned_ahead_matches_oracle(cfg, over, packed):
             q = synth.randn((rows, sh.Hq, sh.D), g, dt, "cpu").pin_memory()
             kn = synth.randn((T, sh.Hkv, sh.D), g, dt, "cpu").pin_memory()
             vn = synth.randn((T, sh.Hkv, sh.D), g, dt, "cpu").pin_memory()
-        out_host = ss.launch_step(p, q, kn, vn, out_host)
+        done = torch.cuda.Event()
+        out_host = ss.launch_step(p, q, kn, vn, out_host, out_ready=done)
         nxt = wl.plan()                          # planned while this step runs
-        torch.cuda.current_stream().synchronize()
+        done.synchronize()                       # the output is on the host
         oracle.block_copy(kc, vc, p.cow_pairs)
         if sh.kv_fp8:
             oracle.kv_append_fp8(kc.numpy(), vc.numpy(), kn, vn, sh.kv_scale, sh.kv_scale, p.slot_mapping)
@@ -229,18 +230,21 @@ def test_launch_step_planned_ahead_matches_oracle(cfg, over, packed):
     ("spec_verify", dict(S=5, Hq=8, Hkv=2, len_uniform=(20, 700))),            # causal chunks
     ("llama7b_fp8", dict(S=6, Hq=4, Hkv=4, len_uniform=(1, 600))),             # FP8 pools
 ])
-def test_launch_step_two_in_flight_matches_oracle(cfg, over):
+@pytest.mark.parametrize("overlap_out", [True, False])
+def test_launch_step_two_in_flight_matches_oracle(cfg, over, overlap_out):
     """Two steps in flight, as bench.py's end-to-end leg runs them: step i+1
     is planned and issued before the host waits for step i's output, each
     step writing its own pinned output buffer (two alternate) and reading its
-    own pinned inputs.  Every step's output equals the oracle's attention on
-    the pools after that step, and at the end both pools equal the oracle's
-    copies and appends."""
+    own pinned inputs; the output copies on the session's output stream
+    (waited for through launch_step's out_ready event) or on the caller's
+    stream.  Every step's output equals the oracle's attention on the pools
+    after that step, and at the end both pools equal the oracle's copies and
+    appends."""
     import bench
     import paged_kv_cache_405_b200 as m
     sh = synth.shrink(synth.CONFIGS[cfg], reserve_tokens=64, **over)
     dev = torch.device("cuda")
-    wl = bench.Workload(sh, sh.seed, dev, 0)
+    wl = bench.Workload(sh, sh.seed, dev, 0, overlap_output_copies=overlap_out)
     ss = wl.session
     kc, vc = ss.k_pool.cpu(), ss.v_pool.cpu()
     dt = synth.DTYPES[sh.dtype]
@@ -271,9 +275,8 @@ def test_launch_step_two_in_flight_matches_oracle(cfg, over):
         T = len(p.slot_mapping)
         rows = T if sh.chunk else len(p.seq_ids)
         q, kn, vn = packed_inputs(rows, T, sh, dt, g)
-        outs[step % 2] = ss.launch_step(p, q, kn, vn, outs[step % 2], stream=stream)
         ev = torch.cuda.Event()
-        ev.record(stream)
+        outs[step % 2] = ss.launch_step(p, q, kn, vn, outs[step % 2], stream=stream, out_ready=ev)
         pending.append((ev, p, q, kn, vn, outs[step % 2]))
         p = wl.plan()                            # the step after, planned while two are in flight
         if len(pending) == 2:
