@@ -44,7 +44,15 @@ def test_workspace_size_rules():
     # (8 seqs x 64 heads x 196 parts x (128+2) floats, then 8-byte split counters per row from a 256-byte boundary)
     parts = 8 * 64 * 196 * 130 * 4
     assert pkv.attention_workspace_bytes(8, 64, 128, 100_160, 512) == -(-parts // 256) * 256 + 8 * 64 * 8
+    # the library's own partition: the whole context up to 512 tokens, else 512, for MHA and grouped queries
+    assert pkv.attention_partition_size(8, 32, 32, 128, 500, 0) == 512
+    assert pkv.attention_partition_size(8, 32, 32, 128, 8192, 0) == 512
+    assert pkv.attention_partition_size(8, 32, 8, 128, 8192, 0) == 512
+    assert pkv.attention_partition_size(8, 32, 8, 128, 8192, 1024) == 1024  # explicit sizes as given
     # the library's own choice is covered by the size it reports
+    for hkv in (32, 8):
+        auto = pkv.attention_partition_size(64, 32, hkv, 128, 8192, 0)
+        assert pkv.attention_workspace_bytes(64, 32, 128, 8192, 0) >= pkv.attention_workspace_bytes(64, 32, 128, 8192, auto)
     auto = pkv.attention_partition_size(64, 32, 32, 128, 2048, 0)
     assert pkv.attention_workspace_bytes(64, 32, 128, 2048, 0) >= \
         pkv.attention_workspace_bytes(64, 32, 128, 2048, auto)
