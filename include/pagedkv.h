@@ -138,8 +138,9 @@ int pkv_attention_partition_size(int num_seqs, int num_q_heads, int num_kv_heads
  *   scale           0 -> 1/sqrt(head_dim)
  *   partition_size  0 -> library's choice; > 0 (multiple of 16) splits every
  *                   context into partitions of that many tokens that run in
- *                   parallel, then a reduce kernel merges them (the FP8
- *                   per-head kernel merges its own, up to 32 partitions).
+ *                   parallel, then a reduce kernel merges them (the MHA
+ *                   kernels merge their own when there are at most 32
+ *                   partitions of at least 512 tokens, without groups).
  *                   For at most 256 sequences and 1024 sequences x
  *                   partitions per call, the MHA kernels start partitions
  *                   longest first: every sequence's full partitions, then

@@ -226,21 +226,26 @@ __global__ void __launch_bounds__(WARPS * 32, 3) paged_attn_simt_kernel(const At
 #pragma unroll
         for (int e = 0; e < EPL; ++e) o[e] += __shfl_xor_sync(0xffffffffu, o[e], off);
     }
-    if (sub != 0) return;
+    const int64_t row = (int64_t)s * p.Hq + h;
     if (u.direct) {
+        if (sub != 0) return;
         const float inv = 1.f / l;
         float r[EPL];
 #pragma unroll
         for (int e = 0; e < EPL; ++e) r[e] = o[e] * inv;
-        store_slice<T, EPL>(reinterpret_cast<T*>(p.out) + ((int64_t)s * p.Hq + h) * D + c * EPL, r);
-    } else {
-        const int64_t idx = ((int64_t)s * p.Hq + h) * p.maxP + u.slot;
+        store_slice<T, EPL>(reinterpret_cast<T*>(p.out) + row * D + c * EPL, r);
+        return;
+    }
+    const unsigned long long seen = p.split_count != nullptr && lane == 0 ? split_peek(p.split_count + row) : 0ull;
+    if (sub == 0) {
+        const int64_t idx = row * p.maxP + u.slot;
         float4* dst = reinterpret_cast<float4*>(p.ws_o + idx * D + c * EPL);
 #pragma unroll
         for (int e = 0; e < EPL; e += 4)
             dst[e / 4] = make_float4(o[e], o[e + 1], o[e + 2], o[e + 3]);
         if (c == 0) *reinterpret_cast<float2*>(p.ws_ml + idx * 2) = make_float2(m, l);
     }
+    if (p.split_count != nullptr) merge_if_last<T, D>(p, row, u.nsuf, lane, seen);
 }
 
 }  // namespace pkv

@@ -391,6 +391,8 @@ static cudaError_t launch_reduce(const pkv::ReduceParams& r, cudaStream_t st) {
     return launch_k(pkv::splitk_reduce_warp_kernel<T, D, 8, 0>, grid, block, 0, st, r);
 }
 
+constexpr int kMinMergePartition = 512;
+
 // Split-K partials merged inside the decode kernel that supports it
 // (pkv::merge_if_last) instead of by the reduce kernel; PKV_SPLIT_MERGE=0
 // builds always run the reduce.
@@ -418,9 +420,12 @@ static int lpt_order(const pkv::AttnParams& p, int nparts) {
 }
 
 // The per-sequence decode kernel of a call (no prefix pass, no reduce).
+// *merged: the kernel merges the call's split-K partials itself (the MHA
+// kernel with split counters), so no reduce kernel is to run.
 template <typename T>
 static cudaError_t decode_pass(const pkv::AttnParams& p, int D, int nparts, bool use_mma, const CUtensorMap* mk,
-                               const CUtensorMap* mv, cudaStream_t st) {
+                               const CUtensorMap* mv, cudaStream_t st, bool* merged) {
+    *merged = false;
     if constexpr (!std::is_same<T, float>::value) {
         if (use_mma) {
             dim3 grid((p.Hkv + kMmaWarps - 1) / kMmaWarps, nparts, p.S);
@@ -430,6 +435,8 @@ static cudaError_t decode_pass(const pkv::AttnParams& p, int D, int nparts, bool
     dim3 grid((p.Hq + kSimtWarps - 1) / kSimtWarps, nparts, p.S);
     pkv::AttnParams q = p;
     q.lpt = lpt_order(p, nparts);
+    if (!PKV_SPLIT_MERGE) q.split_count = nullptr;
+    *merged = q.split_count != nullptr;
     return D == 64 ? launch_simt<T, 64>(q, grid, st) : launch_simt<T, 128>(q, grid, st);
 }
 
@@ -438,9 +445,10 @@ static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int npart
                                       bool shared_mode, const CUtensorMap* mk, const CUtensorMap* mv,
                                       cudaStream_t st) {
     cudaError_t e = cudaSuccess;
+    bool merged = false;  // the decode kernel merged the partials itself
     if constexpr (std::is_same<T, float>::value) {
         if (use_mma || shared_mode) return cudaErrorInvalidValue;
-        e = decode_pass<T>(p, D, nparts, use_mma, mk, mv, st);
+        e = decode_pass<T>(p, D, nparts, use_mma, mk, mv, st, &merged);
     } else {
         if (shared_mode && p.num_groups > 0) {  // membership first: every later kernel reads it
             e = launch_k(pkv::group_members_kernel, dim3((unsigned)((p.S + 7) / 8)), dim3(256), 0, st, p,
@@ -459,17 +467,17 @@ static cudaError_t dispatch_attention(const pkv::AttnParams& p, int D, int npart
             e = D == 64            ? launch_prefix<T, 64>(p, grid, *mk, *mv, ps)
                 : PKV_PREFIX_TC != 0 ? launch_prefix_tc<T>(p, npre, *mk, *mv, ps)
                                      : launch_prefix<T, 128>(p, grid, *mk, *mv, ps);
-            if (e == cudaSuccess) e = decode_pass<T>(p, D, nparts, use_mma, mk, mv, st);
+            if (e == cudaSuccess) e = decode_pass<T>(p, D, nparts, use_mma, mk, mv, st, &merged);
             if (ps != st) {  // join, whatever happened above
                 const cudaError_t j = cudaEventRecord(ss->join, ps);
                 const cudaError_t w = j == cudaSuccess ? cudaStreamWaitEvent(st, ss->join, 0) : j;
                 if (e == cudaSuccess) e = w;
             }
         } else {
-            e = decode_pass<T>(p, D, nparts, use_mma, mk, mv, st);
+            e = decode_pass<T>(p, D, nparts, use_mma, mk, mv, st, &merged);
         }
     }
-    if (e != cudaSuccess || p.maxP <= 1) return e;
+    if (e != cudaSuccess || p.maxP <= 1 || merged) return e;
     pkv::ReduceParams r{p.out, p.ws_o, p.ws_ml, p.context_lens, p.S, p.Hq, D, p.P, p.maxP, p.max_len, p.bs,
                         p.member, nullptr, 0};
     return D == 64 ? launch_reduce<T, 64>(r, st) : launch_reduce<T, 128>(r, st);
@@ -680,8 +688,11 @@ static pkv_status decode_impl(void* out, const void* q, const void* k_pool, cons
     // Shared-prefix membership after the partials (8-byte aligned: (D+2)*4 is).
     p.member = grp.mode && grp.num > 0 ? reinterpret_cast<const int2*>(p.ws_ml + n_part * 2) : nullptr;
     // Split counters (their own region of the workspace without groups); a
-    // kernel that cannot merge its own partials gets nullptr and the reduce runs.
-    if (need > 0 && !grp.mode && slots <= 32) {
+    // kernel that cannot merge its own partials gets nullptr and the reduce
+    // runs.  The merge costs each CTA a fence and an exchange at its end,
+    // repaid only by long units: from 512-token partitions on (shorter ones
+    // measured 2-4 % slower than the reduce kernel).
+    if (need > 0 && !grp.mode && slots <= 32 && P >= kMinMergePartition) {
         p.split_count = reinterpret_cast<unsigned long long*>(
             static_cast<char*>(workspace) + split_counters_offset(partials_bytes((int64_t)num_seqs * num_q_heads,
                                                                                  slots, head_dim)));

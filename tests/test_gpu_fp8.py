@@ -224,13 +224,13 @@ def _fp8_split_case(S, Hq, lens_range, seed):
 
 
 def test_decode_fp8_in_kernel_merge_over_stale_workspace_and_repeated_calls():
-    """The per-head kernel merges a row's split-K partials itself (up to 32
-    partitions), counting arrivals in workspace words stamped per call: a
-    workspace of random bytes, then of 0xff bytes, then back-to-back calls on
-    the same workspace all match the oracle."""
+    """The per-head kernel merges a row's split-K partials itself (2 to 32
+    partitions of at least 512 tokens), counting arrivals in workspace words
+    stamped per call: a workspace of random bytes, then of 0xff bytes, then
+    back-to-back calls on the same workspace all match the oracle."""
     import paged_kv_cache_405_b200 as pkv
-    P = 32
-    b, kc, vc, ks, vs = _fp8_split_case(9, 4, (1, 700), 21)
+    P = 512
+    b, kc, vc, ks, vs = _fp8_split_case(9, 4, (1, 3000), 21)
     maxB = b.block_tables.shape[1]
     assert 1 < -(-maxB * 16 // P) <= 32
     ref = oracle.paged_attention_kv(b.q, kc, vc, ks, vs, b.block_tables, b.lens, threads=oracle.max_threads())
@@ -254,8 +254,8 @@ def test_decode_fp8_in_kernel_merge_replayed_from_a_cuda_graph():
     the lengths, and with them the partitions per row, change between
     replays."""
     import paged_kv_cache_405_b200 as pkv
-    P = 32
-    b, kc, vc, ks, vs = _fp8_split_case(6, 8, (200, 700), 22)
+    P = 512
+    b, kc, vc, ks, vs = _fp8_split_case(6, 8, (600, 3000), 22)
     S, Hq, D = b.shape.S, b.shape.Hq, 128
     maxB = b.block_tables.shape[1]
     n = pkv.attention_workspace_bytes(S, Hq, D, maxB * 16, P)
@@ -268,7 +268,7 @@ def test_decode_fp8_in_kernel_merge_replayed_from_a_cuda_graph():
 
     def case(step):
         g = torch.Generator().manual_seed(50 + step)
-        ln = np.minimum(b.lens, rng.integers(1, 701, size=S)).astype(np.int32)   # within each table
+        ln = np.minimum(b.lens, rng.integers(1, 3001, size=S)).astype(np.int32)  # within each table
         ln[step % S] = 0 if step == 2 else ln[step % S]                           # an empty row once
         return synth.randn((S, Hq, D), g, b.q.dtype, "cpu"), ln
 
@@ -294,13 +294,14 @@ def test_decode_fp8_in_kernel_merge_replayed_from_a_cuda_graph():
         assert max_err(out, ref) <= TOL[out.dtype], step
 
 
-def test_decode_fp8_more_than_32_partitions_uses_the_reduce():
-    """Past 32 partitions per row the per-head kernel leaves the merge to the
-    reduce kernel; the result is the same."""
+@pytest.mark.parametrize("P,lens", [(512, (16500, 17000)), (256, (500, 3000))])
+def test_decode_fp8_long_or_short_partitions_use_the_reduce(P, lens):
+    """Past 32 partitions per row, or with partitions under 512 tokens, the
+    per-head kernel leaves the merge to the reduce kernel; the result is the
+    same."""
     import paged_kv_cache_405_b200 as pkv
-    P = 16
-    b, kc, vc, ks, vs = _fp8_split_case(5, 4, (500, 900), 23)
-    assert -(-b.block_tables.shape[1] * 16 // P) > 32
+    b, kc, vc, ks, vs = _fp8_split_case(3, 2, lens, 23)
+    assert -(-b.block_tables.shape[1] * 16 // P) > (32 if P >= 512 else 1)
     ref = oracle.paged_attention_kv(b.q, kc, vc, ks, vs, b.block_tables, b.lens, threads=oracle.max_threads())
     out = torch.full_like(b.q, float("nan"), device="cuda")
     pkv.paged_attention_decode_fp8(out, b.q.cuda(), kc.cuda(), vc.cuda(), torch.from_numpy(b.block_tables).cuda(),
