@@ -175,3 +175,16 @@ def test_caching_session_matches_the_oracle_on_random_steps():
                     _, t, L = orc.seq_block_table(s)
                     assert p.lens[i] == L and p.block_tables[i].tolist() == t + [-1] * (max_blocks - len(t))
             assert ss.cache_stats() == orc.cache_stats(), seed
+
+
+def test_output_copy_overlap_needs_input_copy_overlap():
+    """The output copies may leave the caller's stream only when the input
+    copies do (the step's C call keys the output stream's wait on the input
+    side's event); both modes construct, one without the other is refused."""
+    k = torch.zeros(4, 1, 16, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="needs overlap_input_copies"):
+        pkv.DecodeSession(k, k.clone(), 1, 8, max_batch=2, overlap_input_copies=False, overlap_output_copies=True)
+    for ins, outs in ((True, True), (True, False), (False, False)):
+        ss = pkv.DecodeSession(k, k.clone(), 1, 8, max_batch=2, overlap_input_copies=ins,
+                               overlap_output_copies=outs)
+        assert (ss.overlap_input_copies, ss.overlap_output_copies) == (ins, outs)
