@@ -165,10 +165,13 @@ class Workload:
                     self.next_child += 1
         # children write first (each copies the shared last block); the parent
         # is then the block's only user and writes in place.
-        write = []
-        for i, p in enumerate(self.parents):
-            write += children[i * (sh.beams - 1):(i + 1) * (sh.beams - 1)] if sh.beams else []
-            write.append(p)
+        if sh.beams:
+            write = []
+            for i, p in enumerate(self.parents):
+                write += children[i * (sh.beams - 1):(i + 1) * (sh.beams - 1)]
+                write.append(p)
+        else:
+            write = self.parents
         plan = ss.plan(self.parents, write)
         for c in children:
             ss.free(c)

@@ -555,6 +555,14 @@ pkv_status pkv_seq_block_tables_batch(const pkv_alloc* a, const int64_t* seq_ids
                                       int max_blocks, int32_t* lens_out);
 
 /*
+ * Lengths in tokens of many sequences, without their tables: lens_out[i]
+ * (int64 [n]) = seq_ids[i]'s length.  PKV_ERR_INVALID (nothing written) if a
+ * sequence is unknown.  A host-side check before a step (will every sequence
+ * still fit its table?) needs only these.
+ */
+pkv_status pkv_seq_lens_batch(const pkv_alloc* a, const int64_t* seq_ids, int n, int64_t* lens_out);
+
+/*
  * Automatic prefix caching ([E] 7.4: a prompt prefix computed once is reused
  * by later requests, which skip that part of the prefill; [T] 2.2.3 shared
  * blocks, 2.2.8 only byte-identical prefixes may share, 2.2.13 hit rate).

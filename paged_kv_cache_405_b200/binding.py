@@ -34,7 +34,7 @@ EXPORTS = [
     "pkv_attention_chunk_workspace_bytes", "pkv_kv_append_fp8", "pkv_paged_attention_decode_fp8", "pkv_block_copy", "pkv_device_error", "pkv_launch_count",
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_add", "pkv_seq_share_prefix", "pkv_seq_fork",
     "pkv_alloc_set_prefix_caching", "pkv_seq_add_with_prompt", "pkv_seq_append_tokens", "pkv_prefix_cache_stats",
-    "pkv_seq_append_slots", "pkv_seq_append_slots_batch", "pkv_seq_block_tables_batch", "pkv_seq_free", "pkv_seq_block_table", "pkv_alloc_stats",
+    "pkv_seq_append_slots", "pkv_seq_append_slots_batch", "pkv_seq_block_tables_batch", "pkv_seq_lens_batch", "pkv_seq_free", "pkv_seq_block_table", "pkv_alloc_stats",
     "pkv_block_refcount", "pkv_status_str", "pkv_last_error", "pkv_step_from_host",
 ]
 
@@ -120,6 +120,7 @@ def _load():
         "pkv_seq_append_slots": (c_int, [c_vp, c_i64, c_int, c_vp, c_vp, c_int, ctypes.POINTER(c_int)]),
         "pkv_seq_append_slots_batch": (c_int, [c_vp, c_vp, c_int, c_vp, c_vp, c_int, ctypes.POINTER(c_int)]),
         "pkv_seq_block_tables_batch": (c_int, [c_vp, c_vp, c_int, c_vp, c_int, c_vp]),
+        "pkv_seq_lens_batch": (c_int, [c_vp, c_vp, c_int, c_vp]),
         "pkv_seq_free": (c_int, [c_vp, c_i64]),
         "pkv_alloc_set_prefix_caching": (c_int, [c_vp, c_int]),
         "pkv_seq_add_with_prompt": (c_int, [c_vp, c_i64, c_vp, c_int, c_vp, ctypes.POINTER(c_int)]),
@@ -581,6 +582,13 @@ class BlockAllocator:
         st = lib.pkv_seq_block_tables_batch(self._h, ids.ctypes.data, n, out.ctypes.data, max_blocks,
                                             lens_out.ctypes.data)
         return st, out, lens_out
+
+    def seq_lens_batch(self, sids):
+        """Lengths in tokens (int64 [n]) of many sequences.  Returns (status, lengths)."""
+        ids = np.ascontiguousarray(np.asarray(sids, dtype=np.int64))
+        lens = np.empty(len(ids), dtype=np.int64)
+        st = lib.pkv_seq_lens_batch(self._h, ids.ctypes.data, len(ids), lens.ctypes.data)
+        return st, lens
 
     def seq_add_with_prompt(self, sid: int, tokens):
         """Returns (status, cached tokens, slots of the remaining tokens)."""

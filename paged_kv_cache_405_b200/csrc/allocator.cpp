@@ -474,6 +474,21 @@ pkv_status pkv_seq_block_tables_batch(const pkv_alloc* a, const int64_t* seq_ids
     return PKV_OK;
 }
 
+pkv_status pkv_seq_lens_batch(const pkv_alloc* a, const int64_t* seq_ids, int n, int64_t* lens_out) {
+    if (!a || n < 0 || (n > 0 && (!seq_ids || !lens_out))) {
+        set_error("pkv_seq_lens_batch: bad arguments");
+        return PKV_ERR_INVALID;
+    }
+    for (int i = 0; i < n; ++i) {
+        if (a->seqs.find(seq_ids[i]) == a->seqs.end()) {
+            set_error("pkv_seq_lens_batch: unknown sequence");
+            return PKV_ERR_INVALID;
+        }
+    }
+    for (int i = 0; i < n; ++i) lens_out[i] = a->seqs.find(seq_ids[i])->second.len;
+    return PKV_OK;
+}
+
 pkv_status pkv_seq_free(pkv_alloc* a, int64_t seq_id) {
     if (!a) return PKV_ERR_INVALID;
     auto it = a->seqs.find(seq_id);

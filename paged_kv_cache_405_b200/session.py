@@ -198,13 +198,17 @@ class DecodeSession:
         """Fail before any slot is reserved (the step's reservations cannot be
         undone): every sequence of ``attend`` must exist and still fit in
         max_blocks_per_seq blocks after this step's tokens."""
-        st, _, lens = self.alloc.seq_block_tables_batch(list(attend), self.max_blocks)
+        a = np.asarray(attend, dtype=np.int64)
+        st, lens = self.alloc.seq_lens_batch(a)
         self._ok(st)
         if not len(lens):
             return
         ids, counts = np.unique(np.asarray(write, dtype=np.int64), return_counts=True)
-        grow = dict(zip(ids.tolist(), counts.tolist()))
-        tokens = lens.astype(np.int64) + np.array([grow.get(int(sid), 0) for sid in attend], dtype=np.int64)
+        grow = np.zeros(len(a), dtype=np.int64)     # new tokens of each attending sequence
+        if len(ids):
+            pos = np.minimum(np.searchsorted(ids, a), len(ids) - 1)
+            grow = np.where(ids[pos] == a, counts[pos], 0)
+        tokens = lens + grow
         blocks = -(-tokens // self.block_size)
         if blocks.max() > self.max_blocks:
             i = int(blocks.argmax())

@@ -305,3 +305,25 @@ def test_batched_appends_equal_single_calls_after_random_histories():
             fails = dict(before[1], alloc_failures=before[1]["alloc_failures"] + 1)
             assert ([p1.seq_block_table(s) for s in range(4)], p1.stats()) == (before[0], fails), seed
     assert n_ok > 100 and n_fail > 10
+
+
+def test_lengths_query_matches_the_tables_query():
+    """seq_lens_batch gives each sequence's length (what the session's
+    pre-step check reads) exactly as seq_block_tables_batch does, for
+    sequences that share a prefix, were forked and grew; an unknown id is
+    refused with nothing written."""
+    a = BlockAllocator(64, 16)
+    for sid, n in ((0, 35), (1, 0), (2, 16), (3, 100)):
+        assert a.seq_add(sid) == OK
+        if n:
+            a.seq_append_slots(sid, n)
+    assert a.seq_fork(0, 7) == OK
+    a.seq_append_slots(7, 3)
+    ids = [3, 0, 7, 1, 2, 0]
+    st, lens = a.seq_lens_batch(ids)
+    assert st == OK and lens.dtype == np.int64
+    st2, _, lens2 = a.seq_block_tables_batch(ids, 16)
+    assert st2 == OK and lens.tolist() == lens2.tolist() == [100, 35, 38, 0, 16, 35]
+    st, lens = a.seq_lens_batch([0, 99])
+    assert st == INVALID
+    assert a.seq_lens_batch([])[0] == OK
