@@ -520,7 +520,7 @@ def measure_workload(name, args, world, rank, local, e2e=True):
     value = total_bytes / (ms_max * 1e-3) / 1e9
     seq_steps = sum_over_ranks(float(shape.S * K), world) / (ms_max * 1e-3)
 
-    # ---- roofline of the decode-attention call (attention kernel + its split-K reduce)
+    # ---- roofline of the decode-attention call (attention kernel + its split-K merge or reduce)
     peak, peak_kind = measured_hbm_peak()
     a_bytes = float(np.mean([a["total"] for a in attn_bytes[W:]]))
     a_s = max_over_ranks(float(np.mean(attn_ms)), world) * 1e-3
@@ -540,7 +540,8 @@ def measure_workload(name, args, world, rank, local, e2e=True):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "traffic": traffic, "peak_source": peak_kind,
                      "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
-                     "kernel": "paged_attention_decode (attention + split-K reduce)",
+                     "kernel": "paged_attention_decode (the call's kernels: attention, and the split-K reduce where the "
+                               "attention kernel does not merge its own partials)",
                      "algorithmic_bytes": round(a_bytes)},
         "gpu_launches": int(launches),
         "clocks": clk,
